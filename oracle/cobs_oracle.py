@@ -1,0 +1,321 @@
+"""Plain fp64 CPU oracle for COBS block-sparse attention decode.
+
+TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the tests, the smoke check of
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import this
+module.  It shares no code with the CUDA library (no kernels, headers, helpers,
+tables or constants) and never imports it; the only thing both sides see is the
+seeded input generator in ``workloads/``.
+
+Everything here is written for a reader who wants to check it against the
+sources by eye: numpy fp64 throughout, library primitives (matmul, eigh, sort)
+as single steps, no blocking, fusion or reordering beyond what the method
+itself states.  Inputs arrive as the exact bf16 values widened to fp64.
+
+Sources (the pages the method is described on):
+
+* "COBS: Cumulant Order Block Sparse Attention" (AI-generated explainer,
+  gist.science paper 2607.09052), technical summary:
+    - §2.1 selection oracle: a block's attention mass m_b is the sum of
+      exp(q.k) over its keys; ranking blocks by m_b is the optimal criterion
+      and "oracle sparse attention" (OSA) ranks by the exact mass.
+    - §2.2 cumulant expansion: ln m_b = ln L + q.kappa1 + 1/2 q^T kappa2 q + ...
+      with kappa1 the block's mean key and kappa2 its key covariance.
+    - §2.3 COBS: score_b ~ q.mean_b + 1/2 q^T Sigma_b q; the covariance is kept
+      as its top-r eigenvectors and eigenvalues; block means are stored in bf16.
+* "LLMアテンション機構" (jisaku.com glossary), section on the computing
+  principle of self-attention: softmax(q K^T / sqrt(d_k)) V; GQA shares one
+  K/V head between several query heads; the KV cache keeps K and V per token.
+* "スライディングウィンドウアテンション" (jisaku.com glossary), overview and
+  extensions: a local window of the last w tokens; attention-sink tokens at the
+  start of the sequence are always kept.
+
+Readings taken where the pages are silent or garbled (each also listed in the
+design notes of the repository):
+
+* The score uses the attention logit scale: a = q / sqrt(d), so
+  score_b = ln n_b + a.mu_b + 1/2 a^T Sigma_b a
+          = ln n_b + (q.mu_b)/sqrt(d) + 1/2 ||U_b^T q||^2 / d.
+  The pages' formula for the score omits both 1/sqrt(d) and ln L; ln n_b is
+  kept (it is constant over the complete blocks that compete in top-k).
+* Sigma_b is the population covariance (1/n) sum (k - mu)(k - mu)^T: the
+  second cumulant of the block's empirical key distribution.
+* U_b = V_r Lambda_r^{1/2} (top-r eigenpairs, descending eigenvalue), each
+  column's sign fixed so that its largest-magnitude component is positive
+  (the score does not depend on the sign; this only makes dumps
+  deterministic).  The stored record is [mu; U columns as rows] rounded to bf16.
+* One selection per (batch, kv-head): the group score is the log of the
+  group's total estimated mass, S_b = ln sum_h exp(s_{h,b}).
+* Forced blocks: the first ``sink_blocks`` blocks (attention sink) and every
+  block that intersects the last ``local_tokens`` tokens, plus the partial
+  tail block (which has no statistics).  Top-k runs over the remaining
+  complete blocks; ties go to the lower block index.  Output ascending.
+* Attention over the selected blocks is one exact softmax over the union of
+  their valid tokens, with the 1/sqrt(d) logit scale.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "round_to_bf16",
+    "block_moments",
+    "covariance_factor",
+    "block_record",
+    "build_block_records",
+    "head_block_scores",
+    "group_block_scores",
+    "block_partition",
+    "select_blocks",
+    "select_from_records",
+    "tokens_of_blocks",
+    "softmax_attention",
+    "sparse_attention",
+    "dense_attention",
+    "osa_head_masses",
+    "osa_group_masses",
+    "decode_step",
+]
+
+
+# ---------------------------------------------------------------------------
+# bf16 storage (COBS explainer §2.3: block means are stored in BF16; the same
+# record format holds the covariance factor in this build)
+# ---------------------------------------------------------------------------
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), as fp64.
+
+    bf16 keeps 8 significant bits (7 stored), so on the fp64 bit pattern the
+    low 52 - 7 = 45 mantissa bits are rounded away in one step (no fp32
+    intermediate, hence no double rounding).  Valid for finite values inside
+    the bf16 normal range, which is all this oracle stores.
+    """
+    x64 = np.ascontiguousarray(x, dtype=np.float64)
+    u = x64.view(np.uint64)
+    drop = np.uint64(45)
+    lsb = (u >> drop) & np.uint64(1)
+    half = np.uint64((1 << 44) - 1)
+    mask = ~np.uint64((1 << 45) - 1)
+    r = ((u + half + lsb) & mask).view(np.float64)
+    return np.where(x64 == 0.0, x64, r)
+
+
+# ---------------------------------------------------------------------------
+# Block statistics (COBS explainer §2.2 cumulants, §2.3 low-rank factor)
+# ---------------------------------------------------------------------------
+
+def block_moments(keys: np.ndarray):
+    """First and second cumulants of one block's keys.
+
+    kappa1 = mean key; kappa2 = population covariance (1/n) sum (k-mu)(k-mu)^T,
+    computed two-pass (mean first, then centred products).
+    """
+    keys = np.asarray(keys, dtype=np.float64)
+    n = keys.shape[0]
+    mu = keys.sum(axis=0) / n
+    centred = keys - mu
+    sigma = centred.T @ centred / n
+    return mu, sigma
+
+
+def covariance_factor(sigma: np.ndarray, rank: int):
+    """Top-``rank`` eigenpairs of a covariance as a factor U with U U^T = Sigma_r.
+
+    COBS explainer §2.3 (low-rank factorisation): keep the top r eigenvectors
+    and eigenvalues.  Returns (U [d, r], eigenvalues [r], descending).
+    """
+    d = sigma.shape[0]
+    if rank == 0:
+        return np.zeros((d, 0)), np.zeros(0)
+    lam, vecs = np.linalg.eigh(sigma)
+    order = np.argsort(-lam, kind="stable")[:rank]
+    lam_r = np.clip(lam[order], 0.0, None)
+    v_r = vecs[:, order]
+    for j in range(v_r.shape[1]):
+        i = int(np.argmax(np.abs(v_r[:, j])))
+        if v_r[i, j] < 0:
+            v_r[:, j] = -v_r[:, j]
+    return v_r * np.sqrt(lam_r)[None, :], lam_r
+
+
+def block_record(keys: np.ndarray, rank: int, to_bf16: bool = True) -> np.ndarray:
+    """The stored statistics record of one complete block: [mu; U^T], (1+r, d).
+
+    With ``to_bf16`` (the storage format) every value is rounded to bf16.
+    """
+    mu, sigma = block_moments(keys)
+    u, _ = covariance_factor(sigma, rank)
+    rec = np.concatenate([mu[None, :], u.T], axis=0)
+    return round_to_bf16(rec) if to_bf16 else rec
+
+
+def build_block_records(keys_seq: np.ndarray, block: int, rank: int,
+                        block_begin: int, block_end: int,
+                        to_bf16: bool = True) -> np.ndarray:
+    """Records for complete blocks [block_begin, block_end) of one (b, kv-head)."""
+    recs = [block_record(keys_seq[j * block:(j + 1) * block], rank, to_bf16)
+            for j in range(block_begin, block_end)]
+    d = keys_seq.shape[1]
+    if not recs:
+        return np.zeros((0, 1 + rank, d))
+    return np.stack(recs, axis=0)
+
+
+# ---------------------------------------------------------------------------
+# Scores (COBS explainer §2.2 expansion, §2.3 second-order score)
+# ---------------------------------------------------------------------------
+
+def head_block_scores(q: np.ndarray, records: np.ndarray,
+                      n_tokens: np.ndarray) -> np.ndarray:
+    """s_b = ln n_b + (q.mu_b)/sqrt(d) + 1/2 sum_j (u_j.q)^2 / d for every block.
+
+    ``records``: [nb, 1+r, d]; row 0 is mu, rows 1..r are the columns of U.
+    With r = 0 this is the first-order (mean-only) score.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    linear = records[:, 0, :] @ q / math.sqrt(d)
+    proj = records[:, 1:, :] @ q                       # [nb, r]
+    quadratic = 0.5 * np.sum(proj * proj, axis=1) / d
+    return np.log(np.asarray(n_tokens, dtype=np.float64)) + linear + quadratic
+
+
+def _logsumexp(x: np.ndarray, axis: int) -> np.ndarray:
+    m = np.max(x, axis=axis, keepdims=True)
+    return (m + np.log(np.sum(np.exp(x - m), axis=axis, keepdims=True))).squeeze(axis)
+
+
+def group_block_scores(q_group: np.ndarray, records: np.ndarray,
+                       n_tokens: np.ndarray) -> np.ndarray:
+    """S_b = ln sum_h exp(s_{h,b}) over the G query heads of one kv-head."""
+    per_head = np.stack([head_block_scores(q, records, n_tokens)
+                         for q in np.asarray(q_group, dtype=np.float64)], axis=0)
+    return _logsumexp(per_head, axis=0)
+
+
+# ---------------------------------------------------------------------------
+# Selection: top-k + sink + local window
+# ---------------------------------------------------------------------------
+
+def block_partition(seq_len: int, block: int, sink_blocks: int,
+                    local_tokens: int):
+    """Split the blocks of a sequence into forced blocks and top-k candidates.
+
+    Returns (forced_sorted, candidate_begin, candidate_end): candidates are the
+    complete blocks in [candidate_begin, candidate_end).
+    """
+    n_blocks = -(-seq_len // block)
+    n_full = seq_len // block
+    first_local = min(n_full, max(0, seq_len - local_tokens) // block)
+    sink_end = min(sink_blocks, first_local)
+    forced = list(range(sink_end)) + list(range(first_local, n_blocks))
+    return forced, sink_end, first_local
+
+
+def select_blocks(scores: np.ndarray, seq_len: int, block: int, top_k: int,
+                  sink_blocks: int, local_tokens: int) -> np.ndarray:
+    """Top-k candidates by score (ties -> lower index), union forced, ascending.
+
+    ``scores`` is indexed by block number; only candidate entries are read.
+    """
+    forced, c0, c1 = block_partition(seq_len, block, sink_blocks, local_tokens)
+    cand = np.arange(c0, c1)
+    s = np.asarray(scores, dtype=np.float64)[c0:c1]
+    order = np.lexsort((cand, -s))            # primary: score desc; then index asc
+    chosen = cand[order[:top_k]]
+    return np.sort(np.concatenate([np.asarray(forced, dtype=np.int64),
+                                   chosen.astype(np.int64)]))
+
+
+def select_from_records(q_group, records, seq_len, block, top_k, sink_blocks,
+                        local_tokens):
+    """Score every complete block from its stored record, then select.
+
+    Returns (selected indices, group scores over complete blocks).
+    """
+    n_full = seq_len // block
+    recs = records[:n_full]
+    scores = group_block_scores(q_group, recs, np.full(n_full, block))
+    return select_blocks(scores, seq_len, block, top_k, sink_blocks,
+                         local_tokens), scores
+
+
+# ---------------------------------------------------------------------------
+# Attention (glossary "LLMアテンション機構": scaled dot-product attention)
+# ---------------------------------------------------------------------------
+
+def tokens_of_blocks(blocks, seq_len: int, block: int) -> np.ndarray:
+    """Valid token positions of the given blocks, in block order."""
+    parts = [np.arange(j * block, min((j + 1) * block, seq_len)) for j in blocks]
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+
+
+def softmax_attention(q_group: np.ndarray, keys: np.ndarray, values: np.ndarray,
+                      scale: float):
+    """softmax(q K^T * scale) V for each head; also ln sum exp(logits)."""
+    q_group = np.asarray(q_group, dtype=np.float64)
+    logits = q_group @ keys.T * scale                  # [G, n]
+    m = logits.max(axis=1, keepdims=True)
+    w = np.exp(logits - m)
+    l = w.sum(axis=1, keepdims=True)
+    out = (w @ values) / l
+    lse = (m + np.log(l))[:, 0]
+    return out, lse
+
+
+def sparse_attention(q_group, keys_seq, values_seq, blocks, seq_len, block,
+                     scale):
+    """Exact attention restricted to the valid tokens of the selected blocks."""
+    t = tokens_of_blocks(blocks, seq_len, block)
+    return softmax_attention(q_group, keys_seq[t], values_seq[t], scale)
+
+
+def dense_attention(q_group, keys_seq, values_seq, seq_len, scale):
+    """Exact attention over all ``seq_len`` cached tokens."""
+    return softmax_attention(q_group, keys_seq[:seq_len], values_seq[:seq_len],
+                             scale)
+
+
+# ---------------------------------------------------------------------------
+# Oracle sparse attention (COBS explainer §2.1): exact block masses
+# ---------------------------------------------------------------------------
+
+def osa_head_masses(q_group, keys_seq, seq_len, block, scale) -> np.ndarray:
+    """ln m_b per head and block: ln sum_{t in b} exp(q_h.k_t * scale), [G, nb]."""
+    q_group = np.asarray(q_group, dtype=np.float64)
+    n_blocks = -(-seq_len // block)
+    logits = q_group @ keys_seq[:seq_len].T * scale
+    out = np.empty((q_group.shape[0], n_blocks))
+    for j in range(n_blocks):
+        out[:, j] = _logsumexp(logits[:, j * block:min((j + 1) * block, seq_len)],
+                               axis=1)
+    return out
+
+
+def osa_group_masses(q_group, keys_seq, seq_len, block, scale) -> np.ndarray:
+    """ln of the group's total exact mass per block: ln sum_h m_b^(h)."""
+    return _logsumexp(osa_head_masses(q_group, keys_seq, seq_len, block, scale),
+                      axis=0)
+
+
+# ---------------------------------------------------------------------------
+# One decode step for one (batch, kv-head) pair
+# ---------------------------------------------------------------------------
+
+def decode_step(q_group, keys_seq, values_seq, records, seq_len, block, top_k,
+                sink_blocks, local_tokens, scale=None):
+    """Select from stored records, then attend exactly over the selection.
+
+    Returns (selected blocks, group scores, out [G, d], lse [G]).
+    """
+    d = keys_seq.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    sel, scores = select_from_records(q_group, records, seq_len, block, top_k,
+                                      sink_blocks, local_tokens)
+    out, lse = sparse_attention(q_group, keys_seq, values_seq, sel, seq_len,
+                                block, scale)
+    return sel, scores, out, lse
