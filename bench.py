@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Decode-step throughput of the COBS block-sparse attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cobs|reference]
+
+One step is one pass of the whole hot path over a batch of synthetic
+queries: the statistics of the block that just became complete (one block per
+(batch, kv-head)), the second-order block selection (scores + top-k + sink +
+local window) and the split-K sparse flash-decode with its log-sum-exp merge —
+three C-ABI calls, three kernel launches.  The KV cache and the statistics of
+all earlier blocks are resident in HBM before timing starts; L2 is flushed
+(256 MiB write) between timed steps and each step is timed with CUDA events
+on the stream its kernels run on.
+
+Workload (default): batch 32, 32 query / 8 KV heads, head_dim 128, 32768
+cached tokens, block 64, rank 8, top-k 16 + sink block + 512-token window,
+keys from tight/spread per-block Gaussians with 4 planted needles per
+(batch, kv-head) — seeded synthetic data (``workloads``).
+
+Multi-GPU: one process per GPU (torchrun); every rank decodes its own batch
+(weak scaling, no collective on the data path); the step time is the max over
+ranks and ``value`` counts the queries of all ranks.
+
+``--impl reference`` times the CPU oracle (``oracle/``) on the same workload,
+a bounded sample of (batch, kv-head) pairs per step, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode queries/s and achieved HBM GB/s (% of peak) at 32k context"
+UNIT = "queries/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["cobs", "reference"], default="cobs")
+    p.add_argument("--workload", default="batched_needles_32k")
+    p.add_argument("--gen-workers", type=int, default=0,
+                   help="processes drawing the synthetic cache (0 = auto)")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="time budget of the CPU-oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# byte model: what the method has to move per launch
+# ---------------------------------------------------------------------------
+
+def partition(T, B, sink, local):
+    n_blocks = -(-T // B)
+    n_full = T // B
+    first_local = min(n_full, max(0, T - local) // B)
+    sink_end = min(sink, first_local)
+    return n_blocks, n_full, sink_end, first_local
+
+
+def byte_model(w, n_sel):
+    """Algorithmic bytes per launch of each kernel for one step."""
+    B, d, r = w.block, w.head_dim, w.rank
+    pairs = w.batch * w.kv_heads
+    nbs, nfull, c0, c1 = partition(w.seq_len, B, w.sink_blocks, w.local_tokens)
+    q_bytes = w.batch * w.q_heads * d * 2
+    rec = (1 + r) * d * 2
+    stats_build = pairs * (B * d * 2 + rec)                 # one block in, one record out
+    select = pairs * (c1 - c0) * rec + q_bytes + pairs * (c1 - c0) * 4 + pairs * 4 * (1 + n_sel)
+    # valid tokens of the selected blocks (all complete here except a ragged tail)
+    kv = 0
+    tail = w.seq_len - (nbs - 1) * B
+    for_tail = 1 if tail < B else 0
+    toks = n_sel * B - (B - tail) * for_tail
+    kv = pairs * toks * d * 2 * 2
+    decode = kv + q_bytes + pairs * 4 * (1 + n_sel) + w.batch * w.q_heads * (d + 1) * 4
+    return {"stats": stats_build, "select": select, "decode": decode}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, r[5:9]):
+                if flag.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# kernel traffic recorded by ncu (profiles/traffic.json), tied to the source
+# ---------------------------------------------------------------------------
+
+def source_hash(name):
+    path = os.path.join(ROOT, "block_sparse_long_cobs_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file, workload):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(f"{kernel_file}:{workload}")
+    if not rec or rec.get("source_sha") != source_hash(kernel_file):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (baseline and --impl reference)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """Oracle decode steps for a few (batch, kv-head) pairs of the workload."""
+
+    def __init__(self, w, q_bits, k_bits, v_bits, pairs):
+        import oracle.cobs_oracle as O
+        from workloads import bits_to_f64
+        self.O, self.w = O, w
+        self.items = []
+        nfull = w.seq_len // w.block
+        for (b, h) in pairs:
+            keys = bits_to_f64(k_bits[b, h])
+            vals = bits_to_f64(v_bits[b, h])
+            qg = bits_to_f64(q_bits[b, h * w.group:(h + 1) * w.group])
+            recs = O.build_block_records(keys, w.block, w.rank, 0, nfull - 1)
+            self.items.append((qg, keys, vals, recs))
+
+    def step(self, i):
+        """Stats of the just-completed block + selection + attention, one pair."""
+        O, w = self.O, self.w
+        qg, keys, vals, recs = self.items[i % len(self.items)]
+        nfull = w.seq_len // w.block
+        last = O.build_block_records(keys, w.block, w.rank, nfull - 1, nfull)
+        allrec = np.concatenate([recs, last])
+        O.decode_step(qg, keys, vals, allrec, w.seq_len, w.block, w.top_k,
+                      w.sink_blocks, w.local_tokens)
+        return w.group                               # queries served
+
+
+def oracle_pairs(w, n):
+    pairs = [(b, h) for b in range(w.batch) for h in range(w.kv_heads)]
+    step = max(1, len(pairs) // n)
+    return pairs[::step][:n]
+
+
+def oracle_slices(w, pairs):
+    """Only the K/V slices the oracle sample needs (drawn per slice)."""
+    from workloads import make_kv_slice, make_queries
+    q = make_queries(w)
+    K = {}
+    V = {}
+    for (b, h) in pairs:
+        K[(b, h)], V[(b, h)] = make_kv_slice(w, b, h, q if w.needles else None)
+
+    class View:
+        def __init__(self, d):
+            self.d = d
+
+        def __getitem__(self, key):
+            return self.d[key]
+    return q, View(K), View(V)
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    from threadpoolctl import threadpool_limits
+    pairs = oracle_pairs(w, 4)
+    q, K, V = oracle_slices(w, pairs)
+    with threadpool_limits(1):
+        sample = OracleSample(w, q, K, V, pairs)
+        for i in range(args.warmup):
+            sample.step(i)
+        t0 = time.perf_counter()
+        served = 0
+        for i in range(args.steps):
+            served += sample.step(i)
+        dt = time.perf_counter() - t0
+    value = served / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+                   "kv_heads": w.kv_heads, "head_dim": w.head_dim, "seq_len": w.seq_len,
+                   "block": w.block, "rank": w.rank, "top_k": w.top_k,
+                   "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"per step one (batch, kv-head) pair of {pairs}: stats of "
+                                   "the completed block + selection + attention, fp64 numpy, "
+                                   "1 thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, q_bits, k_bits, v_bits, seconds):
+    from threadpoolctl import threadpool_limits
+    pairs = oracle_pairs(w, 4)
+    with threadpool_limits(1):
+        sample = OracleSample(w, q_bits, k_bits, v_bits, pairs)
+        sample.step(0)
+        t0 = time.perf_counter()
+        served, i = 0, 0
+        while time.perf_counter() - t0 < seconds:
+            served += sample.step(i)
+            i += 1
+        dt = time.perf_counter() - t0
+    return {"value": served / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{i} oracle decode steps cycling over (batch, kv-head) pairs {pairs} of "
+                      f"{w.name} (stats of the completed block + selection + attention per "
+                      f"pair, fp64 numpy, 1 thread), {dt:.1f} s, scaled to queries/s"}
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_cobs(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_long_cobs_b200 as cb
+    from workloads import make_kv, make_queries
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    workers = args.gen_workers or max(1, min(16, (os.cpu_count() or 2) // max(1, world) - 1))
+    q_bits = make_queries(w)
+    k_bits, v_bits = make_kv(w, q_bits if w.needles else None, workers=workers)
+
+    def up(x):
+        return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev)
+
+    dims = dict(batch=w.batch, num_q_heads=w.q_heads, num_kv_heads=w.kv_heads,
+                head_dim=w.head_dim, block_size=w.block, rank=w.rank,
+                capacity_tokens=w.cap)
+    q, k, v = up(q_bits), up(k_bits), up(v_bits)
+    nb_cap = w.cap // w.block
+    nfull = w.seq_len // w.block
+    stats = torch.zeros((w.batch, w.kv_heads, nb_cap, 1 + w.rank, w.head_dim),
+                        dtype=torch.int16, device=dev)
+    nsm = cb.cobs_selected_capacity(dims, w.top_k, w.sink_blocks, w.local_tokens)
+    idx = torch.zeros((w.batch, w.kv_heads, nsm), dtype=torch.int32, device=dev)
+    n_sel = torch.zeros((w.batch, w.kv_heads), dtype=torch.int32, device=dev)
+    out = torch.zeros((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.zeros((w.batch, w.q_heads), dtype=torch.float32, device=dev)
+    ws_bytes = cb.cobs_workspace_bytes(dims, w.top_k, w.sink_blocks, w.local_tokens)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cb.cobs_workspace_init(ws, ws_bytes, stream)
+    scale = 1.0 / math.sqrt(w.head_dim)
+
+    # statistics of every earlier complete block (setup, timed for information)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cb.cobs_build_block_stats(dims, k, 0, nfull - 1, stats, ws, ws_bytes, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    build_ms = e0.elapsed_time(e1)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
+                              w.local_tokens, idx, n_sel, None, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
+                              ws, ws_bytes, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    status = cb.cobs_read_device_status(ws, ws_bytes, stream)
+    if status != 0:
+        raise RuntimeError(f"device status {cb.cobs_status_string(status)} after warm-up")
+    sel_counts = n_sel.cpu().numpy()
+    n_sel_mean = float(sel_counts.mean())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clock_info = clocks.stop()
+    t_stats = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    t_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+    status = cb.cobs_read_device_status(ws, ws_bytes, stream)
+    if status != 0:
+        raise RuntimeError(f"device status {cb.cobs_status_string(status)} after timing")
+
+    # end to end through the public API with host buffers: queries and the
+    # appended token's K/V go host -> device, outputs come back
+    e2e = None
+    if not args.no_e2e:
+        q_host = torch.from_numpy(q_bits.view(np.int16)).pin_memory()
+        kn_host = torch.from_numpy(k_bits[:, :, w.seq_len - 1].view(np.int16)).pin_memory()
+        vn_host = torch.from_numpy(v_bits[:, :, w.seq_len - 1].view(np.int16)).pin_memory()
+        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        kn_dev = torch.empty_like(kn_host, device=dev)
+        vn_dev = torch.empty_like(vn_host, device=dev)
+        h2d = q_host.numel() * 2 + kn_host.numel() * 2 + vn_host.numel() * 2
+        d2h = out_host.numel() * 4 + lse_host.numel() * 4
+        n_e2e = max(1, args.steps // 4)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_e2e)]
+
+        def e2e_step(pair):
+            pair[0].record(stream)
+            q.copy_(q_host, non_blocking=True)
+            kn_dev.copy_(kn_host, non_blocking=True)
+            vn_dev.copy_(vn_host, non_blocking=True)
+            k[:, :, w.seq_len - 1].copy_(kn_dev)
+            v[:, :, w.seq_len - 1].copy_(vn_dev)
+            step()
+            out_host.copy_(out, non_blocking=True)
+            lse_host.copy_(lse, non_blocking=True)
+            pair[1].record(stream)
+
+        for _ in range(3):
+            flush.zero_()
+            e2e_step(ev[0])
+        torch.cuda.synchronize(dev)
+        for i in range(n_e2e):
+            flush.zero_()
+            e2e_step(ev[i])
+        torch.cuda.synchronize(dev)
+        t_e2e = sum(a.elapsed_time(b) for a, b in ev) / n_e2e
+        if world > 1:
+            tt = torch.tensor([t_e2e], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t_e2e = float(tt.item())
+        e2e = {"value": world * w.batch * w.q_heads / (t_e2e * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": t_e2e}
+
+    if world > 1:
+        tt = torch.tensor([t_step, t_stats, t_sel, t_dec], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step, t_stats, t_sel, t_dec = (float(x) for x in tt.tolist())
+    if rank != 0:
+        return
+
+    hbm, peak_kind = peaks()
+    bm = byte_model(w, round(n_sel_mean))
+    per_kernel = {"stats": (t_stats, bm["stats"], "stats.cu"),
+                  "select": (t_sel, bm["select"], "select.cu"),
+                  "decode": (t_dec, bm["decode"], "decode.cu")}
+    kernels = {name: {"ms": t, "bytes": b, "gbs": b / (t * 1e-3) / 1e9,
+                      "frac_of_hbm": b / (t * 1e-3) / 1e9 / hbm}
+               for name, (t, b, _) in per_kernel.items()}
+    dom = max(per_kernel, key=lambda n: per_kernel[n][0])
+    t_dom, b_dom, file_dom = per_kernel[dom]
+    achieved = b_dom / (t_dom * 1e-3) / 1e9
+    step_bytes = bm["select"] + bm["decode"] + bm["stats"]
+    value = world * w.batch * w.q_heads / (t_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_heads": w.q_heads,
+                   "kv_heads": w.kv_heads, "head_dim": w.head_dim, "seq_len": w.seq_len,
+                   "block": w.block, "rank": w.rank, "top_k": w.top_k,
+                   "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
+                   "selected_blocks_mean": n_sel_mean, "l2": "flushed (256 MiB) between steps",
+                   "parallelism": f"replicas x{world}",
+                   "step": "stats of the completed block + select + sparse decode"},
+        "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
+        "hbm_frac_step": step_bytes / (t_step * 1e-3) / 1e9 / hbm,
+        "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "traffic": recorded_traffic(file_dom, w.name)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clock_info,
+        "setup_stats_build_ms": build_ms,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q_bits, k_bits, v_bits, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_cobs(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

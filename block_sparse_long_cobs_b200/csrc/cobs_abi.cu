@@ -1,0 +1,342 @@
+// C ABI of the COBS decode library: argument checks, workspace layout, launch
+// configuration.  Everything that can be checked on the host is checked here,
+// before any CUDA call; kernels never see an invalid shape.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "cobs_internal.h"
+
+namespace cobs {
+namespace {
+
+thread_local std::string g_last_error;
+
+cobs_status fail(cobs_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+cobs_status ok() {
+  g_last_error.clear();
+  return COBS_OK;
+}
+
+cobs_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(COBS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+cobs_status check_dims(const cobs_dims* d) {
+  if (!d) return fail(COBS_ERR_INVALID_ARG, "dims is NULL");
+  if (d->batch < 1 || d->num_q_heads < 1 || d->num_kv_heads < 1)
+    return fail(COBS_ERR_INVALID_ARG, "batch and head counts must be >= 1");
+  if (d->num_q_heads % d->num_kv_heads != 0)
+    return fail(COBS_ERR_INVALID_ARG, "num_q_heads (%d) is not a multiple of num_kv_heads (%d)",
+                d->num_q_heads, d->num_kv_heads);
+  const int g = d->num_q_heads / d->num_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8)
+    return fail(COBS_ERR_UNSUPPORTED, "query heads per kv-head must be 1, 2, 4 or 8 (got %d)", g);
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return fail(COBS_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", d->head_dim);
+  if (d->block_size != kBlock)
+    return fail(COBS_ERR_UNSUPPORTED, "block_size must be 64 (got %d)", d->block_size);
+  if (d->rank < 0 || d->rank > kMaxRank)
+    return fail(COBS_ERR_UNSUPPORTED, "rank must be in [0, 16] (got %d)", d->rank);
+  if (d->capacity_tokens < kBlock || d->capacity_tokens % kBlock != 0)
+    return fail(COBS_ERR_INVALID_ARG, "capacity_tokens must be a positive multiple of 64");
+  const int64_t rows = int64_t(d->batch) * d->num_kv_heads * d->capacity_tokens;
+  if (rows >= (int64_t(1) << 31))
+    return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * capacity_tokens must be < 2^31");
+  return COBS_OK;
+}
+
+cobs_status check_select_params(int32_t top_k, int32_t sink_blocks, int32_t local_tokens) {
+  if (top_k < 0 || sink_blocks < 0 || local_tokens < 0)
+    return fail(COBS_ERR_INVALID_ARG, "top_k, sink_blocks and local_tokens must be >= 0");
+  return COBS_OK;
+}
+
+int32_t selected_capacity(const cobs_dims* d, int32_t top_k, int32_t sink, int32_t local) {
+  const int64_t nb = d->capacity_tokens / kBlock;
+  const int64_t want = int64_t(top_k) + sink + ceil_div(local, kBlock) + 1;
+  return int32_t(want < nb ? want : nb);
+}
+
+WorkspaceLayout layout(const cobs_dims* d, int32_t n_sel_max) {
+  WorkspaceLayout L{};
+  const size_t pairs = size_t(d->batch) * d->num_kv_heads;
+  L.nb_cap = d->capacity_tokens / kBlock;
+  L.n_sel_max = n_sel_max;
+  size_t off = 0;
+  L.status = off;
+  off = align256(off + 256);
+  L.sel_tickets = off;
+  off = align256(off + pairs * 4);
+  L.dec_tickets = off;
+  off = align256(off + pairs * 4);
+  L.scores = off;
+  off = align256(off + pairs * size_t(L.nb_cap) * 4);
+  L.partials = off;
+  off = align256(off + size_t(d->batch) * d->num_q_heads * size_t(n_sel_max) *
+                           (size_t(d->head_dim) + 2) * 4);
+  L.total = off;
+  return L;
+}
+
+// Smallest layout that still holds the status word (build_block_stats).
+constexpr size_t kStatusBytes = 256;
+
+cobs_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return fail(COBS_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned16(ws)) return fail(COBS_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (have < need)
+    return fail(COBS_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", have,
+                need);
+  return COBS_OK;
+}
+
+}  // namespace
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace cobs
+
+using namespace cobs;
+
+extern "C" {
+
+int32_t cobs_abi_version(void) { return COBS_ABI_VERSION; }
+
+const char* cobs_last_error(void) { return g_last_error.c_str(); }
+
+const char* cobs_status_string(cobs_status s) {
+  switch (s) {
+    case COBS_OK: return "COBS_OK";
+    case COBS_ERR_INVALID_ARG: return "COBS_ERR_INVALID_ARG";
+    case COBS_ERR_UNSUPPORTED: return "COBS_ERR_UNSUPPORTED";
+    case COBS_ERR_WORKSPACE: return "COBS_ERR_WORKSPACE";
+    case COBS_ERR_CUDA: return "COBS_ERR_CUDA";
+    case COBS_ERR_TIMEOUT: return "COBS_ERR_TIMEOUT";
+    case COBS_ERR_DEVICE: return "COBS_ERR_DEVICE";
+  }
+  return "COBS_ERR_UNKNOWN";
+}
+
+int32_t cobs_selected_capacity(const cobs_dims* dims, int32_t top_k, int32_t sink_blocks,
+                               int32_t local_tokens) {
+  if (check_dims(dims) != COBS_OK) return -1;
+  if (check_select_params(top_k, sink_blocks, local_tokens) != COBS_OK) return -1;
+  ok();
+  return selected_capacity(dims, top_k, sink_blocks, local_tokens);
+}
+
+size_t cobs_workspace_bytes(const cobs_dims* dims, int32_t top_k, int32_t sink_blocks,
+                            int32_t local_tokens) {
+  if (check_dims(dims) != COBS_OK) return 0;
+  if (check_select_params(top_k, sink_blocks, local_tokens) != COBS_OK) return 0;
+  ok();
+  return layout(dims, selected_capacity(dims, top_k, sink_blocks, local_tokens)).total;
+}
+
+cobs_status cobs_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return fail(COBS_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned16(ws)) return fail(COBS_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (ws_bytes < kStatusBytes) return fail(COBS_ERR_WORKSPACE, "workspace too small");
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  return ok();
+}
+
+cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k, int64_t block_begin,
+                                   int64_t block_end, void* stats, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  cobs_status st = check_dims(dims);
+  if (st != COBS_OK) return st;
+  if (!k || !stats) return fail(COBS_ERR_INVALID_ARG, "k and stats must not be NULL");
+  if (!aligned16(k) || !aligned16(stats))
+    return fail(COBS_ERR_INVALID_ARG, "k and stats must be 16-byte aligned");
+  const int64_t nb_cap = dims->capacity_tokens / kBlock;
+  if (block_begin < 0 || block_end < block_begin || block_end > nb_cap)
+    return fail(COBS_ERR_INVALID_ARG, "block range [%lld, %lld) outside [0, %lld]",
+                (long long)block_begin, (long long)block_end, (long long)nb_cap);
+  if ((st = check_ws(ws, ws_bytes, kStatusBytes)) != COBS_OK) return st;
+  if (block_end == block_begin) return ok();
+  StatsArgs a{};
+  a.k = static_cast<const uint16_t*>(k);
+  a.stats = static_cast<uint16_t*>(stats);
+  a.status = reinterpret_cast<int32_t*>(static_cast<char*>(ws));
+  a.cap = dims->capacity_tokens;
+  a.nb_cap = nb_cap;
+  a.block_begin = block_begin;
+  a.block_end = block_end;
+  a.batch = dims->batch;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.rank = dims->rank;
+  cudaError_t e = launch_stats(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block statistics launch");
+  return ok();
+}
+
+cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void* stats,
+                               int64_t seq_len, int32_t top_k, int32_t sink_blocks,
+                               int32_t local_tokens, int32_t* idx, int32_t* n_sel,
+                               float* scores_opt, void* ws, size_t ws_bytes, void* stream) {
+  cobs_status st = check_dims(dims);
+  if (st != COBS_OK) return st;
+  if ((st = check_select_params(top_k, sink_blocks, local_tokens)) != COBS_OK) return st;
+  if (!q || !stats || !idx || !n_sel)
+    return fail(COBS_ERR_INVALID_ARG, "q, stats, idx and n_sel must not be NULL");
+  if (!aligned16(q) || !aligned16(stats) || !aligned16(idx) || !aligned16(n_sel) ||
+      (scores_opt && !aligned16(scores_opt)))
+    return fail(COBS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (seq_len < 1 || seq_len > dims->capacity_tokens)
+    return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
+                (long long)seq_len);
+  const int32_t nsm = selected_capacity(dims, top_k, sink_blocks, local_tokens);
+  const WorkspaceLayout L = layout(dims, nsm);
+  if ((st = check_ws(ws, ws_bytes, L.partials)) != COBS_OK) return st;
+
+  // block partition: forced sink [0, sink_end), forced local [first_local, nbs)
+  const int64_t nbs = ceil_div(seq_len, kBlock);
+  const int64_t n_full = seq_len / kBlock;
+  int64_t first_local = (seq_len - local_tokens > 0 ? seq_len - local_tokens : 0) / kBlock;
+  if (first_local > n_full) first_local = n_full;
+  const int64_t sink_end = sink_blocks < first_local ? sink_blocks : first_local;
+
+  SelectArgs a{};
+  char* w = static_cast<char*>(ws);
+  a.q = static_cast<const uint16_t*>(q);
+  a.stats = static_cast<const uint16_t*>(stats);
+  a.idx = idx;
+  a.n_sel = n_sel;
+  a.scores_opt = scores_opt;
+  a.scores_ws = reinterpret_cast<float*>(w + L.scores);
+  a.tickets = reinterpret_cast<uint32_t*>(w + L.sel_tickets);
+  a.status = reinterpret_cast<int32_t*>(w + L.status);
+  a.nb_cap = L.nb_cap;
+  a.batch = dims->batch;
+  a.hq = dims->num_q_heads;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.rank = dims->rank;
+  a.idx_stride = nsm;
+  a.seq_len_blocks = int32_t(nbs);
+  a.cand_begin = int32_t(sink_end);
+  a.cand_end = int32_t(first_local);
+  a.sink_end = int32_t(sink_end);
+  a.first_local = int32_t(first_local);
+  a.top_k = top_k;
+
+  // chunking: about 4 CTAs per SM over all (batch, kv-head) pairs
+  const int per_pass = 256 / (dims->head_dim / 8);
+  const int64_t n_cand = first_local - sink_end;
+  const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
+  int sms = device_sm_count();
+  if (sms <= 0) sms = 148;
+  int64_t chunks = ceil_div(int64_t(4) * sms, pairs);
+  const int64_t max_chunks = n_cand > 0 ? ceil_div(n_cand, per_pass) : 1;
+  if (chunks > max_chunks) chunks = max_chunks;
+  if (chunks < 1) chunks = 1;
+  int64_t chunk_blocks = n_cand > 0 ? ceil_div(n_cand, chunks) : per_pass;
+  chunk_blocks = ceil_div(chunk_blocks, per_pass) * per_pass;
+  a.chunk_blocks = int32_t(chunk_blocks);
+  a.n_chunks = int32_t(n_cand > 0 ? ceil_div(n_cand, chunk_blocks) : 1);
+
+  cudaError_t e = launch_select(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block selection launch");
+  return ok();
+}
+
+cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void* k,
+                               const void* v, const int32_t* idx, const int32_t* n_sel,
+                               int32_t idx_stride, int64_t seq_len, float softmax_scale,
+                               float* out, float* lse, void* ws, size_t ws_bytes,
+                               void* stream) {
+  cobs_status st = check_dims(dims);
+  if (st != COBS_OK) return st;
+  if (!q || !k || !v || !idx || !n_sel || !out || !lse)
+    return fail(COBS_ERR_INVALID_ARG, "q, k, v, idx, n_sel, out and lse must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(n_sel) ||
+      !aligned16(out) || !aligned16(lse))
+    return fail(COBS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (seq_len < 1 || seq_len > dims->capacity_tokens)
+    return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
+                (long long)seq_len);
+  if (idx_stride < 1) return fail(COBS_ERR_INVALID_ARG, "idx_stride must be >= 1");
+  if (!(std::isfinite(softmax_scale)) || softmax_scale <= 0.f)
+    return fail(COBS_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  const WorkspaceLayout L = layout(dims, idx_stride);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != COBS_OK) return st;
+
+  DecodeArgs a{};
+  char* w = static_cast<char*>(ws);
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.idx = idx;
+  a.n_sel = n_sel;
+  a.out = out;
+  a.lse = lse;
+  a.partials = reinterpret_cast<float*>(w + L.partials);
+  a.tickets = reinterpret_cast<uint32_t*>(w + L.dec_tickets);
+  a.status = reinterpret_cast<int32_t*>(w + L.status);
+  a.cap = dims->capacity_tokens;
+  a.seq_len = seq_len;
+  a.batch = dims->batch;
+  a.hq = dims->num_q_heads;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.idx_stride = idx_stride;
+  a.part_stride = idx_stride;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+  // splits: about 4 CTAs per SM over all (batch, kv-head) pairs
+  const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
+  int sms = device_sm_count();
+  if (sms <= 0) sms = 148;
+  int64_t splits = ceil_div(int64_t(4) * sms, pairs);
+  if (splits > idx_stride) splits = idx_stride;
+  if (splits < 1) splits = 1;
+  const int64_t bps = ceil_div(idx_stride, splits);
+  a.blocks_per_split = int32_t(bps);
+  a.n_splits = int32_t(ceil_div(idx_stride, bps));
+
+  cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
+  return ok();
+}
+
+cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_status,
+                                    void* stream) {
+  if (!device_status) return fail(COBS_ERR_INVALID_ARG, "device_status is NULL");
+  cobs_status st = check_ws(ws, ws_bytes, kStatusBytes);
+  if (st != COBS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(v), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  *device_status = v;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/cobs.h"
+
+namespace cobs {
+
+constexpr int kBlock = 64;     // tokens per KV block
+constexpr int kMaxRank = 16;   // columns of the covariance factor
+constexpr int kMaxGroup = 8;   // query heads per kv-head
+
+// Byte layout of the caller's workspace.  Every region starts 256-aligned.
+struct WorkspaceLayout {
+  size_t status;       // int32 status word (+ padding)
+  size_t sel_tickets;  // uint32 [batch * Hkv], selection arrival counters
+  size_t dec_tickets;  // uint32 [batch * Hkv], decode arrival counters
+  size_t scores;       // float  [batch * Hkv * nb_cap], group scores
+  size_t partials;     // float  [batch * Hq * n_sel_max * (d + 2)]
+  size_t total;
+  int64_t nb_cap;      // capacity / B
+  int32_t n_sel_max;   // row length of idx the workspace is sized for
+};
+
+// Arguments of the scoring + top-k kernel.
+struct SelectArgs {
+  const uint16_t* q;      // [b][Hq][d]
+  const uint16_t* stats;  // [b][Hkv][nb_cap][1+r][d]
+  int32_t* idx;           // [b][Hkv][idx_stride]
+  int32_t* n_sel;         // [b][Hkv]
+  float* scores_opt;      // [b][Hkv][nb_cap] or null
+  float* scores_ws;       // [b][Hkv][nb_cap]
+  uint32_t* tickets;      // [b][Hkv]
+  int32_t* status;
+  int64_t nb_cap;
+  int32_t batch, hq, hkv, d, rank;
+  int32_t idx_stride;
+  int32_t seq_len_blocks;   // ceil(seq_len / B)
+  int32_t cand_begin, cand_end;  // candidate blocks [begin, end)
+  int32_t sink_end;         // forced blocks [0, sink_end)
+  int32_t first_local;      // forced blocks [first_local, seq_len_blocks)
+  int32_t top_k;
+  int32_t chunk_blocks;     // candidates per CTA
+  int32_t n_chunks;         // CTAs per (b, kv-head)
+};
+
+// Arguments of the split-K decode kernel.
+struct DecodeArgs {
+  const uint16_t* q;      // [b][Hq][d]
+  const uint16_t* k;      // [b][Hkv][cap][d]
+  const uint16_t* v;
+  const int32_t* idx;     // [b][Hkv][idx_stride]
+  const int32_t* n_sel;   // [b][Hkv]
+  float* out;             // [b][Hq][d]
+  float* lse;             // [b][Hq]
+  float* partials;        // [b][Hq][n_sel_max][d+2]
+  uint32_t* tickets;      // [b][Hkv]
+  int32_t* status;
+  int64_t cap;
+  int64_t seq_len;
+  int32_t batch, hq, hkv, d;
+  int32_t idx_stride;
+  int32_t part_stride;    // n_sel_max of the workspace (splits dimension)
+  int32_t n_splits;       // CTAs per (b, kv-head)
+  int32_t blocks_per_split;
+  float scale_log2;       // softmax_scale * log2(e)
+};
+
+// Arguments of the block-statistics kernel.
+struct StatsArgs {
+  const uint16_t* k;      // [b][Hkv][cap][d]
+  uint16_t* stats;        // [b][Hkv][nb_cap][1+r][d]
+  int32_t* status;
+  int64_t cap;
+  int64_t nb_cap;
+  int64_t block_begin, block_end;
+  int32_t batch, hkv, d, rank;
+};
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace cobs

@@ -1,0 +1,382 @@
+// Split-K flash-decode over the selected KV blocks, with a log-sum-exp merge.
+//
+// Exact attention (glossary "LLMアテンション機構": softmax(q K^T / sqrt d) V,
+// grouped-query heads sharing one K/V head) restricted to the tokens of the
+// blocks chosen by the COBS selector (COBS explainer, gist.science paper
+// 2607.09052, §1: block-sparse attention reads whole contiguous blocks; §2.1:
+// attention is reconstructed from the selected blocks only).
+//
+// Grid: (split, kv-head, batch).  A CTA walks its share of the block list of
+// one (batch, kv-head) and keeps, for each of the G query heads of the group,
+// an online-softmax triple (running max m, running sum l, accumulator o).
+// The last CTA of a (batch, kv-head) to finish (atomic ticket, no spinning)
+// merges the split triples:  M = max m_i,  out = sum e^(m_i-M) o_i /
+// sum e^(m_i-M) l_i,  lse = M + ln sum e^(m_i-M) l_i.
+//
+// Data movement: each selected block's K rows and V rows are contiguous in
+// the cache (B x d bf16 = 16 KB for d = 128), so each is staged with one bulk
+// async copy (TMA engine) into a 2-stage shared-memory ring guarded by
+// mbarriers.  Only the block's valid rows (< seq_len) are copied; nothing past
+// the sequence is ever read.
+//
+// Compute: q.K — a warp covers 16 tokens; the 16 lanes of a token (8 lanes for
+// d = 64) each own an 8-element d-slice and keep that slice of all G queries
+// in registers (pre-scaled by softmax_scale*log2 e), so each K element is read
+// from shared memory exactly once.  A reduce-scatter over those lanes leaves
+// one head's logit per lane.  P.V — lanes own 4 consecutive output dims,
+// warps own token ranges; partial accumulators are summed across warps once
+// per split.  Arithmetic is fp32 (packed fp32x2 FMA), logits in log2 units.
+#include <cfloat>
+
+#include "device_common.cuh"
+
+namespace cobs {
+namespace {
+
+constexpr int kDecThreads = 128;
+constexpr int kStages = 2;
+
+template <int D, int G>
+struct DecodeShape {
+  static constexpr int kSlices = D / 8;                 // lanes per token (q.K)
+  static constexpr int kTokPerRound = 32 / kSlices;     // tokens per warp round
+  static constexpr int kRounds = 16 / kTokPerRound;     // rounds per warp (16 tok)
+  static constexpr int kDimGroups = D / 4;              // P.V lanes (4 dims each)
+  static constexpr int kTokGroups = kDecThreads / kDimGroups;
+  static constexpr int kTokPerGroup = kBlock / kTokGroups;
+  static constexpr int kGP = G < 4 ? 4 : G;             // padded row of P
+  static constexpr int kTileElems = kBlock * D;         // bf16 per K or V tile
+  // shared memory carve-up (bytes)
+  static constexpr size_t kK = 0;
+  static constexpr size_t kV = kK + size_t(kStages) * kTileElems * 2;
+  static constexpr size_t kS = kV + size_t(kStages) * kTileElems * 2;   // [G][64]
+  static constexpr size_t kP = kS + size_t(G) * kBlock * 4;            // [64][GP]
+  static constexpr size_t kAlpha = kP + size_t(kBlock) * kGP * 4;      // [8]
+  static constexpr size_t kBar = kAlpha + 8 * 4;                        // [S] u64
+  static constexpr size_t kMisc = kBar + kStages * 8;                   // ints
+  static constexpr size_t kBytes = kMisc + 16 * 4;
+  static_assert(size_t(kTokGroups) * G * D * 4 <= size_t(kStages) * kTileElems * 2,
+                "reduction buffer must fit in the K stages");
+};
+
+// Reduce-scatter of G per-lane partial sums over the kSlices lanes of a token.
+// On return v[0] holds the full sum for head `head` (duplicated on the
+// kSlices/G lanes that share it when G < kSlices).
+template <int G, int kSlices>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane, int& head) {
+  int live = G;
+  head = 0;
+#pragma unroll
+  for (int m = kSlices / 2; m >= 1; m >>= 1) {
+    if (live > 1) {
+      const int half = live / 2;
+      const bool upper = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < G / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      if (upper) head += half;
+      live = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
+  return v[0];
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kDecThreads)
+sparse_decode_kernel(const DecodeArgs a) {
+  using S = DecodeShape<D, G>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint16_t* ks = reinterpret_cast<uint16_t*>(smem + S::kK);
+  uint16_t* vs = reinterpret_cast<uint16_t*>(smem + S::kV);
+  float* s_s = reinterpret_cast<float*>(smem + S::kS);
+  float* p_s = reinterpret_cast<float*>(smem + S::kP);
+  float* alpha_s = reinterpret_cast<float*>(smem + S::kAlpha);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  int* misc = reinterpret_cast<int*>(smem + S::kMisc);
+  int* nvalid_s = misc;          // [kStages]
+  int* abort_s = misc + 4;
+  int* last_s = misc + 5;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int split = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int bh = b * a.hkv + kvh;
+
+  // ---- this split's slice of the block list --------------------------------
+  int nsel = a.n_sel[bh];
+  if (nsel < 1 || nsel > a.idx_stride) {
+    if (split == 0 && tid == 0) report(a.status, COBS_ERR_DEVICE);
+    nsel = nsel < 0 ? 0 : (nsel > a.idx_stride ? a.idx_stride : nsel);
+  }
+  const int p0 = split * a.blocks_per_split;
+  const int p1 = min(p0 + a.blocks_per_split, nsel);
+  const int nblk = max(0, p1 - p0);
+  const int32_t* idx_row = a.idx + int64_t(bh) * a.idx_stride + p0;
+  const int64_t seq_blocks = (a.seq_len + kBlock - 1) / kBlock;
+  const uint16_t* kbase = a.k + int64_t(bh) * a.cap * D;
+  const uint16_t* vbase = a.v + int64_t(bh) * a.cap * D;
+
+  // ---- queries: this lane's 8-element d-slice of every head, pre-scaled ----
+  const int slice = lane % S::kSlices;
+  uint64_t qreg[G][4];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint4 w = *reinterpret_cast<const uint4*>(
+        a.q + (int64_t(b) * a.hq + kvh * G + h) * D + slice * 8);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float2 f = bf16x2_to_float2(ww[c]);
+      f.x *= a.scale_log2;
+      f.y *= a.scale_log2;
+      qreg[h][c] = pack2(f);
+    }
+  }
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    fence_barrier_init();
+    *abort_s = 0;
+  }
+  __syncthreads();
+
+  auto issue = [&](int i, int st) {  // called by thread 0 only
+    const int j = idx_row[i];
+    int nv = 0;
+    if (j >= 0 && int64_t(j) < seq_blocks) {
+      const int64_t rem = a.seq_len - int64_t(j) * kBlock;
+      nv = int(rem < kBlock ? rem : kBlock);
+    } else {
+      report(a.status, COBS_ERR_DEVICE);
+    }
+    nvalid_s[st] = nv;
+    const uint32_t bytes = uint32_t(nv) * D * 2;
+    mbar_arrive_expect_tx(&full[st], 2 * bytes);
+    if (nv > 0) {
+      bulk_g2s(ks + st * S::kTileElems, kbase + int64_t(j) * kBlock * D, bytes, &full[st]);
+      bulk_g2s(vs + st * S::kTileElems, vbase + int64_t(j) * kBlock * D, bytes, &full[st]);
+    }
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages && i < nblk; ++i) issue(i, i);
+  }
+
+  // online-softmax state: warp w owns heads w and w + 4
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  // P.V accumulators: 4 consecutive dims x G heads
+  const int dg = tid % S::kDimGroups;
+  const int tg = tid / S::kDimGroups;
+  float acc[G][4];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[h][c] = 0.f;
+
+  for (int i = 0; i < nblk; ++i) {
+    const int st = i % kStages;
+    const uint32_t parity = (i / kStages) & 1;
+    if (tid == 0) {
+      if (!mbar_wait_bounded(&full[st], parity, a.status)) {
+        *abort_s = 1;
+        // drain the copies still in flight for later stages (bounded)
+        for (int k2 = i + 1; k2 < nblk && k2 < i + kStages; ++k2)
+          mbar_wait_bounded(&full[k2 % kStages], (k2 / kStages) & 1, a.status);
+      }
+    }
+    __syncthreads();
+    if (*abort_s) break;
+    if (tid != 0) (void)mbar_try_wait(&full[st], parity);  // acquire the TMA writes
+    const int nv = nvalid_s[st];
+    const uint16_t* kt = ks + st * S::kTileElems;
+    const uint16_t* vt = vs + st * S::kTileElems;
+
+    // ---- logits: s_s[h][t] = q_h . k_t * scale * log2(e) -------------------
+#pragma unroll
+    for (int r = 0; r < S::kRounds; ++r) {
+      const int t = warp * 16 + r * S::kTokPerRound + lane / S::kSlices;
+      float part[G];
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (t < nv) w = *reinterpret_cast<const uint4*>(kt + t * D + slice * 8);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        uint64_t acc2 = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ffma2(acc2, pack2(bf16x2_to_float2(ww[c])), qreg[h][c]);
+        const float2 f = unpack2(acc2);
+        part[h] = f.x + f.y;
+      }
+      int head;
+      const float s = reduce_scatter<G, S::kSlices>(part, lane, head);
+      s_s[head * kBlock + t] = (t < nv) ? s : -INFINITY;
+    }
+    __syncthreads();
+
+    // ---- online softmax per head -------------------------------------------
+#pragma unroll
+    for (int k2 = 0; k2 < 2; ++k2) {
+      const int h = warp + 4 * k2;
+      if (h < G) {
+        const float s0 = s_s[h * kBlock + lane];
+        const float s1 = s_s[h * kBlock + lane + 32];
+        const float mx = warp_max(fmaxf(s0, s1));
+        const float m_new = fmaxf(m_run[k2], mx);
+        float alpha, p0, p1;
+        if (m_new == -INFINITY) {
+          alpha = 1.f;
+          p0 = p1 = 0.f;
+        } else {
+          alpha = hw_exp2(m_run[k2] - m_new);
+          p0 = hw_exp2(s0 - m_new);
+          p1 = hw_exp2(s1 - m_new);
+        }
+        l_run[k2] = l_run[k2] * alpha + warp_sum(p0 + p1);
+        m_run[k2] = m_new;
+        p_s[lane * S::kGP + h] = p0;
+        p_s[(lane + 32) * S::kGP + h] = p1;
+        if (lane == 0) alpha_s[h] = alpha;
+      }
+    }
+    __syncthreads();
+
+    // ---- accumulate P.V ------------------------------------------------------
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float al = alpha_s[h];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[h][c] *= al;
+    }
+    const int t0 = tg * S::kTokPerGroup;
+    const int t1 = min(t0 + S::kTokPerGroup, nv);
+    for (int t = t0; t < t1; ++t) {
+      const uint2 w = *reinterpret_cast<const uint2*>(vt + t * D + dg * 4);
+      const float2 v01 = bf16x2_to_float2(w.x);
+      const float2 v23 = bf16x2_to_float2(w.y);
+      const uint64_t pv01 = pack2(v01), pv23 = pack2(v23);
+#pragma unroll
+      for (int h4 = 0; h4 < S::kGP; h4 += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(p_s + t * S::kGP + h4);
+        const float pp[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          const int h = h4 + hh;
+          if (h < G) {
+            const uint64_t p2 = pack2(make_float2(pp[hh], pp[hh]));
+            uint64_t a01 = pack2(make_float2(acc[h][0], acc[h][1]));
+            uint64_t a23 = pack2(make_float2(acc[h][2], acc[h][3]));
+            ffma2(a01, pv01, p2);
+            ffma2(a23, pv23, p2);
+            const float2 r01 = unpack2(a01), r23 = unpack2(a23);
+            acc[h][0] = r01.x; acc[h][1] = r01.y; acc[h][2] = r23.x; acc[h][3] = r23.y;
+          }
+        }
+      }
+    }
+    __syncthreads();  // stage `st` is free again
+    if (tid == 0 && i + kStages < nblk) issue(i + kStages, st);
+  }
+
+  // ---- split epilogue: write (o, m, l) per head ------------------------------
+  float* red = reinterpret_cast<float*>(smem + S::kK);  // [tokgroups][G][D]
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    *reinterpret_cast<float4*>(red + (tg * G + h) * D + dg * 4) =
+        make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+  __syncthreads();
+  const int64_t part_row = int64_t(a.part_stride) * (D + 2);
+  for (int e = tid; e < G * D; e += kDecThreads) {
+    const int h = e / D, dd = e % D;
+    float sum = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < S::kTokGroups; ++g2) sum += red[(g2 * G + h) * D + dd];
+    float* prow = a.partials + (int64_t(b) * a.hq + kvh * G + h) * part_row +
+                  int64_t(split) * (D + 2);
+    prow[dd] = sum;
+  }
+#pragma unroll
+  for (int k2 = 0; k2 < 2; ++k2) {
+    const int h = warp + 4 * k2;
+    if (h < G && lane == 0) {
+      float* prow = a.partials + (int64_t(b) * a.hq + kvh * G + h) * part_row +
+                    int64_t(split) * (D + 2);
+      prow[D] = m_run[k2];
+      prow[D + 1] = l_run[k2];
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t prev = atomicAdd(&a.tickets[bh], 1u);
+    *last_s = (prev == uint32_t(a.n_splits - 1));
+  }
+  __syncthreads();
+  if (!*last_s) return;
+  __threadfence();
+
+  // ---- last CTA of this (batch, kv-head): log-sum-exp merge ------------------
+  constexpr float kLn2 = 0.69314718055994530942f;
+  for (int e = tid; e < G * D; e += kDecThreads) {
+    const int h = e / D, dd = e % D;
+    const int64_t hq = int64_t(b) * a.hq + kvh * G + h;
+    const float* base = a.partials + hq * part_row;
+    float M = -INFINITY;
+    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, __ldcg(base + int64_t(s) * (D + 2) + D));
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < a.n_splits; ++s) {
+        const float* prow = base + int64_t(s) * (D + 2);
+        const float ms = __ldcg(prow + D);
+        if (ms == -INFINITY) continue;
+        const float w = hw_exp2(ms - M);
+        L += w * __ldcg(prow + D + 1);
+        O += w * __ldcg(prow + dd);
+      }
+    }
+    a.out[hq * D + dd] = (L > 0.f) ? O / L : 0.f;
+    if (dd == 0) a.lse[hq] = (L > 0.f) ? (M + hw_log2(L)) * kLn2 : -INFINITY;
+  }
+  if (tid == 0) a.tickets[bh] = 0u;
+}
+
+template <int D, int G>
+cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
+  using S = DecodeShape<D, G>;
+  auto kern = sparse_decode_kernel<D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(S::kBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.n_splits, a.hkv, a.batch);
+  kern<<<grid, kDecThreads, S::kBytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_group(const DecodeArgs& a, cudaStream_t s) {
+  switch (a.hq / a.hkv) {
+    case 1: return launch_decode_t<D, 1>(a, s);
+    case 2: return launch_decode_t<D, 2>(a, s);
+    case 4: return launch_decode_t<D, 4>(a, s);
+    case 8: return launch_decode_t<D, 8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);
+}
+
+}  // namespace cobs

@@ -1,0 +1,191 @@
+/*
+ * cobs.h — C ABI of the COBS block-sparse attention decode library (sm_100a).
+ *
+ * The method (COBS: Cumulant Order Block Sparse Attention; AI-generated
+ * explainer on gist.science, paper 2607.09052):
+ *   - the KV cache is cut into contiguous blocks of B tokens (technical
+ *     summary §1 problem statement: block-sparse attention reads whole
+ *     contiguous blocks);
+ *   - every complete block keeps its mean key mu and a rank-r factor U of its
+ *     key covariance, Sigma ~ U U^T (§2.2 cumulants kappa1/kappa2; §2.3 "keep
+ *     only the top r eigenvectors and eigenvalues"; means stored in BF16);
+ *   - a query scores every block by the second-order cumulant estimate of its
+ *     log attention mass (§2.2 expansion, §2.3 score), with the attention
+ *     logit scale a = q / sqrt(d):
+ *         s_b = ln n_b + (q . mu_b) / sqrt(d) + 1/2 ||U_b^T q||^2 / d
+ *     (r = 0 gives the first-order, mean-only score);
+ *   - per (batch, kv-head) the top-k blocks by group score
+ *     S_b = ln sum_{h in group} exp(s_{h,b}) are kept, together with the
+ *     attention-sink block(s) at the start and every block touching the last
+ *     local_tokens tokens (glossary "スライディングウィンドウアテンション":
+ *     sliding window + attention sink);
+ *   - exact softmax attention (glossary "LLMアテンション機構": softmax(q K^T /
+ *     sqrt(d)) V, GQA) runs over the valid tokens of the selected blocks only.
+ *
+ * Conventions for every call:
+ *   - The caller owns all memory.  The library never allocates device or
+ *     pinned memory and keeps no global state except a thread-local copy of
+ *     the last error message.
+ *   - Device pointers must be 16-byte aligned.  Host-side argument checks
+ *     happen before anything is launched; a failed check returns an error
+ *     code and launches nothing.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and may be captured into a CUDA graph.
+ *   - bf16 tensors are raw IEEE bfloat16 (uint16 bit patterns); all layouts
+ *     are row-major with the innermost index last.
+ *   - Device-side faults the kernels detect themselves (an out-of-range block
+ *     index, a bounded wait that ran out) are recorded in a status word inside
+ *     the workspace; read it with cobs_read_device_status() after the work has
+ *     run.  Kernels never trap.
+ *
+ * Shapes (G = num_q_heads / num_kv_heads, d = head_dim, B = block_size):
+ *   K, V cache   [batch][num_kv_heads][capacity_tokens][d]        bf16
+ *   q            [batch][num_q_heads][d]                          bf16
+ *                (query head hq belongs to kv-head hq / G)
+ *   stats        [batch][num_kv_heads][capacity_tokens / B][1 + r][d] bf16
+ *                (row 0 = mu, rows 1..r = columns of U, eigenvalues descending)
+ *   idx          [batch][num_kv_heads][idx_stride]                int32
+ *   n_sel        [batch][num_kv_heads]                            int32
+ *   out          [batch][num_q_heads][d]                          fp32
+ *   lse          [batch][num_q_heads]  ln sum exp(logits)         fp32
+ *
+ * Supported: d in {64, 128}; B = 64; 0 <= r <= 16; G in {1, 2, 4, 8};
+ * capacity_tokens a positive multiple of B; one sequence length for the whole
+ * batch.
+ */
+#ifndef COBS_H_
+#define COBS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define COBS_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define COBS_API __attribute__((visibility("default")))
+#else
+#define COBS_API
+#endif
+
+typedef enum cobs_status {
+  COBS_OK = 0,
+  COBS_ERR_INVALID_ARG = 1,  /* a pointer, size or shape is wrong          */
+  COBS_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels cover  */
+  COBS_ERR_WORKSPACE = 3,    /* workspace missing or too small             */
+  COBS_ERR_CUDA = 4,         /* a CUDA runtime call failed                 */
+  COBS_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out             */
+  COBS_ERR_DEVICE = 6        /* device: a kernel rejected its input        */
+} cobs_status;
+
+typedef struct cobs_dims {
+  int32_t batch;             /* sequences in the batch                      */
+  int32_t num_q_heads;       /* query heads Hq                              */
+  int32_t num_kv_heads;      /* key/value heads Hkv (Hq % Hkv == 0)         */
+  int32_t head_dim;          /* d                                           */
+  int32_t block_size;        /* B (64)                                      */
+  int32_t rank;              /* r, columns of the covariance factor U       */
+  int64_t capacity_tokens;   /* cache length per (batch, kv-head)           */
+} cobs_dims;
+
+/* Version of this ABI (COBS_ABI_VERSION). */
+COBS_API int32_t cobs_abi_version(void);
+
+/* Length of one row of `idx`: the largest number of blocks a selection can
+ * return, min(ceil(capacity/B), top_k + sink_blocks + ceil(local_tokens/B) + 1).
+ * Returns -1 (and sets the last error) for invalid arguments. */
+COBS_API int32_t cobs_selected_capacity(const cobs_dims* dims, int32_t top_k,
+                               int32_t sink_blocks, int32_t local_tokens);
+
+/* Bytes of device workspace that cobs_build_block_stats, cobs_select_blocks
+ * and cobs_sparse_decode need for these settings (one workspace serves all
+ * three; it does not depend on the device).  Returns 0 for invalid arguments.
+ * The workspace holds a status word, per-(batch, kv-head) counters, block
+ * scores and split-K partial results. */
+COBS_API size_t cobs_workspace_bytes(const cobs_dims* dims, int32_t top_k,
+                            int32_t sink_blocks, int32_t local_tokens);
+
+/* Zero-fill a workspace.  Required once before its first use; afterwards the
+ * kernels leave their counters at zero themselves. */
+COBS_API cobs_status cobs_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Block statistics for the complete blocks [block_begin, block_end) of every
+ * (batch, kv-head): mu = mean key; Sigma = (1/B) sum (k - mu)(k - mu)^T;
+ * U = top-r eigenvectors of Sigma scaled by sqrt(eigenvalue), each column's
+ * largest-magnitude component made positive.  Written to `stats` in bf16.
+ * COBS explainer §2.2 (kappa1, kappa2) and §2.3 (low-rank factorisation).
+ * Call it when blocks become complete (e.g. after appending a chunk).
+ *   k      device, K cache (see shapes); only the named blocks are read.
+ *   stats  device, written for the named blocks only.
+ *   ws     device workspace (status word only is used here).
+ * Errors: INVALID_ARG (null/misaligned pointer, block range outside
+ * [0, capacity/B]), UNSUPPORTED, WORKSPACE, CUDA. */
+COBS_API cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k,
+                                   int64_t block_begin, int64_t block_end,
+                                   void* stats, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Score every complete block for the group of each (batch, kv-head) and keep
+ * the top_k of them by S_b (ties: lower block index first), plus blocks
+ * [0, sink_blocks) and every block that intersects the last `local_tokens`
+ * tokens or is the partial tail block.  Only complete blocks outside those
+ * forced sets compete; if there are at most top_k of them, all are kept.
+ * COBS explainer §2.1 (rank blocks by attention mass), §2.2–2.3 (score).
+ *   q           device [batch][Hq][d] bf16, this decode step's queries.
+ *   stats       device, records of every complete block below seq_len.
+ *   seq_len     tokens in the cache, 1 <= seq_len <= capacity_tokens.
+ *   idx         device [batch][Hkv][cobs_selected_capacity(...)] int32,
+ *               selected block indices ascending; entries past n_sel are
+ *               left untouched.
+ *   n_sel       device [batch][Hkv] int32, number of selected blocks.
+ *   scores_opt  device [batch][Hkv][capacity/B] fp32 or NULL: S_b of the
+ *               scored candidates (other entries untouched).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+COBS_API cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q,
+                               const void* stats, int64_t seq_len,
+                               int32_t top_k, int32_t sink_blocks,
+                               int32_t local_tokens, int32_t* idx,
+                               int32_t* n_sel, float* scores_opt, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Exact attention of every query head over the valid tokens (< seq_len) of
+ * the blocks listed for its kv-head: out = softmax(q K^T * softmax_scale) V,
+ * lse = ln sum exp(q K^T * softmax_scale), computed as a split-K flash-decode
+ * whose partial (max, sum, accumulator) triples are merged by log-sum-exp.
+ *   idx, n_sel  device, as written by cobs_select_blocks (any ascending or
+ *               unordered list of distinct in-range blocks is accepted);
+ *               idx_stride is the row length of idx.
+ *   softmax_scale  usually 1/sqrt(d).
+ *   out, lse    device fp32 outputs.
+ * A block index outside [0, ceil(seq_len/B)) or an n_sel outside
+ * [1, idx_stride] is skipped/clamped on the device and reported as
+ * COBS_ERR_DEVICE through the status word.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE (idx_stride larger than the
+ * workspace was sized for), CUDA. */
+COBS_API cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q,
+                               const void* k, const void* v,
+                               const int32_t* idx, const int32_t* n_sel,
+                               int32_t idx_stride, int64_t seq_len,
+                               float softmax_scale, float* out, float* lse,
+                               void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, copy the workspace status word to *device_status
+ * (COBS_OK or the first device-side error code since the last read) and
+ * clear it.  Returns CUDA on a failed copy, INVALID_ARG on bad pointers. */
+COBS_API cobs_status cobs_read_device_status(void* ws, size_t ws_bytes,
+                                    int32_t* device_status, void* stream);
+
+/* Message for the last error returned on this thread ("" if none). */
+COBS_API const char* cobs_last_error(void);
+
+/* Static name of a status code. */
+COBS_API const char* cobs_status_string(cobs_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COBS_H_ */

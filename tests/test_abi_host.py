@@ -1,0 +1,155 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, sizes its workspace as documented, and rejects bad arguments before
+touching the GPU (no compute call is made here, so these run without one)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_long_cobs_b200 as cb
+from workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cobs.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"COBS_API\s+[\w\s\*]+?\b(cobs_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) == 10, names
+    raw = ctypes.CDLL(cb.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    for n in names:
+        assert callable(getattr(cb, n)), n
+
+
+def test_version_and_status_strings():
+    assert cb.cobs_abi_version() == 1
+    assert cb.cobs_status_string(0) == "COBS_OK"
+    assert cb.cobs_status_string(5) == "COBS_ERR_TIMEOUT"
+    assert cb.cobs_status_string(99) == "COBS_ERR_UNKNOWN"
+
+
+def dims_of(w, **kw):
+    d = dict(batch=w.batch, num_q_heads=w.q_heads, num_kv_heads=w.kv_heads,
+             head_dim=w.head_dim, block_size=w.block, rank=w.rank,
+             capacity_tokens=w.cap)
+    d.update(kw)
+    return d
+
+
+def ceil_div(a, b):
+    return -(-a // b)
+
+
+def align(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_selected_capacity_and_workspace_size(name):
+    w = WORKLOADS[name]
+    d = dims_of(w)
+    nsm = cb.cobs_selected_capacity(d, w.top_k, w.sink_blocks, w.local_tokens)
+    assert nsm == min(w.cap // 64, w.top_k + w.sink_blocks + ceil_div(w.local_tokens, 64) + 1)
+    ws = cb.cobs_workspace_bytes(d, w.top_k, w.sink_blocks, w.local_tokens)
+    pairs = w.batch * w.kv_heads
+    want = 256 + 2 * align(pairs * 4) + align(pairs * (w.cap // 64) * 4) + \
+        align(w.batch * w.q_heads * nsm * (w.head_dim + 2) * 4)
+    assert ws == want
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_q_heads=12, num_kv_heads=4), cb.COBS_ERR_UNSUPPORTED),   # G = 3
+    (dict(num_q_heads=10, num_kv_heads=4), cb.COBS_ERR_INVALID_ARG),
+    (dict(head_dim=96), cb.COBS_ERR_UNSUPPORTED),
+    (dict(block_size=32), cb.COBS_ERR_UNSUPPORTED),
+    (dict(rank=17), cb.COBS_ERR_UNSUPPORTED),
+    (dict(rank=-1), cb.COBS_ERR_UNSUPPORTED),
+    (dict(capacity_tokens=1000), cb.COBS_ERR_INVALID_ARG),
+    (dict(batch=0), cb.COBS_ERR_INVALID_ARG),
+])
+def test_bad_dims_rejected_everywhere(kw, code):
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w, **kw)
+    fake = 1 << 20                     # never dereferenced: rejected first
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_build_block_stats(d, fake, 0, 1, fake, fake, 1 << 20)
+    assert e.value.status == code
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_select_blocks(d, fake, fake, 100, 8, 1, 64, fake, fake, None, fake, 1 << 20)
+    assert e.value.status == code
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_sparse_decode(d, fake, fake, fake, fake, fake, 10, 100, 0.1, fake, fake,
+                              fake, 1 << 20)
+    assert e.value.status == code
+    assert cb.cobs_selected_capacity is not None
+    assert cb.lib.cobs_workspace_bytes(ctypes.byref(cb.cobs_dims(**d)), 8, 1, 64) == 0
+    assert len(cb.cobs_last_error()) > 0
+
+
+def test_pointer_and_range_checks():
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w)
+    A = 1 << 20
+    ws_need = cb.cobs_workspace_bytes(d, w.top_k, 1, w.local_tokens)
+    nsm = cb.cobs_selected_capacity(d, w.top_k, 1, w.local_tokens)
+    cases = [
+        # build: null, misaligned, block range, workspace
+        (lambda: cb.cobs_build_block_stats(d, None, 0, 1, A, A, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_build_block_stats(d, A + 8, 0, 1, A, A, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_build_block_stats(d, A, 0, w.cap // 64 + 1, A, A, 4096),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_build_block_stats(d, A, 5, 4, A, A, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_build_block_stats(d, A, -1, 4, A, A, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_build_block_stats(d, A, 0, 4, A, None, 4096), cb.COBS_ERR_WORKSPACE),
+        (lambda: cb.cobs_build_block_stats(d, A, 0, 4, A, A, 16), cb.COBS_ERR_WORKSPACE),
+        # select
+        (lambda: cb.cobs_select_blocks(d, A, A, 0, 8, 1, 64, A, A, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, w.cap + 1, 8, 1, 64, A, A, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, -1, 1, 64, A, A, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, None, A, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, A + 4, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, A, A + 2, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 16, 1, 512, A, A, None, A, 1024),
+         cb.COBS_ERR_WORKSPACE),
+        # decode
+        (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, 0, 100, 0.1, A, A, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, nsm, 100, 0.0, A, A, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, nsm, 100, float("nan"), A, A, A,
+                                       ws_need), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, nsm + 1, 100, 0.1, A, A, A, ws_need),
+         cb.COBS_ERR_WORKSPACE),
+        (lambda: cb.cobs_sparse_decode(d, A, A, None, A, A, nsm, 100, 0.1, A, A, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, nsm, 100, 0.1, A, A + 12, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),
+        # workspace helpers
+        (lambda: cb.cobs_workspace_init(None, 4096), cb.COBS_ERR_WORKSPACE),
+        (lambda: cb.cobs_workspace_init(A + 1, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: cb.cobs_read_device_status(None, 4096), cb.COBS_ERR_WORKSPACE),
+    ]
+    for fn, code in cases:
+        with pytest.raises(cb.CobsError) as e:
+            fn()
+        assert e.value.status == code, (e.value, code)
+
+
+def test_status_read_rejects_null_output():
+    st = cb.lib.cobs_read_device_status(ctypes.c_void_p(1 << 20), 4096, None, None)
+    assert st == cb.COBS_ERR_INVALID_ARG
