@@ -334,7 +334,7 @@ def run_cobs(args, w, rank, world, local_rank):
         if ev is not None:
             ev[1].record(stream)
         cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
-                              w.local_tokens, idx, n_sel, None, ws, ws_bytes, stream)
+                              w.local_tokens, idx, nsm, n_sel, None, ws, ws_bytes, stream)
         if ev is not None:
             ev[2].record(stream)
         cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,

@@ -71,7 +71,7 @@ def _load() -> ctypes.CDLL:
         "cobs_workspace_bytes": (SZ, [D, I32, I32, I32]),
         "cobs_workspace_init": (I32, [P, SZ, P]),
         "cobs_build_block_stats": (I32, [D, P, I64, I64, P, P, SZ, P]),
-        "cobs_select_blocks": (I32, [D, P, P, I64, I32, I32, I32, P, P, P, P, SZ, P]),
+        "cobs_select_blocks": (I32, [D, P, P, I64, I32, I32, I32, P, I32, P, P, P, SZ, P]),
         "cobs_sparse_decode": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_last_error": (ctypes.c_char_p, []),
@@ -161,11 +161,12 @@ def cobs_build_block_stats(dims, k, block_begin, block_end, stats, ws, ws_bytes,
 
 
 def cobs_select_blocks(dims, q, stats, seq_len, top_k, sink_blocks, local_tokens,
-                       idx, n_sel, scores_opt, ws, ws_bytes, stream=None,
+                       idx, idx_stride, n_sel, scores_opt, ws, ws_bytes, stream=None,
                        check=True) -> int:
     st = lib.cobs_select_blocks(ctypes.byref(_dims(dims)), _ptr(q), _ptr(stats), seq_len,
-                                top_k, sink_blocks, local_tokens, _ptr(idx), _ptr(n_sel),
-                                _ptr(scores_opt), _ptr(ws), ws_bytes, _stream(stream))
+                                top_k, sink_blocks, local_tokens, _ptr(idx), idx_stride,
+                                _ptr(n_sel), _ptr(scores_opt), _ptr(ws), ws_bytes,
+                                _stream(stream))
     return _check("cobs_select_blocks", st, check)
 
 

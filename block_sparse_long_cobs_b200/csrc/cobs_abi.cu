@@ -196,8 +196,9 @@ cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k, int64_t
 
 cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void* stats,
                                int64_t seq_len, int32_t top_k, int32_t sink_blocks,
-                               int32_t local_tokens, int32_t* idx, int32_t* n_sel,
-                               float* scores_opt, void* ws, size_t ws_bytes, void* stream) {
+                               int32_t local_tokens, int32_t* idx, int32_t idx_stride,
+                               int32_t* n_sel, float* scores_opt, void* ws, size_t ws_bytes,
+                               void* stream) {
   cobs_status st = check_dims(dims);
   if (st != COBS_OK) return st;
   if ((st = check_select_params(top_k, sink_blocks, local_tokens)) != COBS_OK) return st;
@@ -210,6 +211,9 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
     return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
                 (long long)seq_len);
   const int32_t nsm = selected_capacity(dims, top_k, sink_blocks, local_tokens);
+  if (idx_stride < nsm)
+    return fail(COBS_ERR_INVALID_ARG, "idx_stride %d is below the %d blocks a selection can return",
+                idx_stride, nsm);
   const WorkspaceLayout L = layout(dims, nsm);
   if ((st = check_ws(ws, ws_bytes, L.partials)) != COBS_OK) return st;
 
@@ -236,7 +240,7 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.rank = dims->rank;
-  a.idx_stride = nsm;
+  a.idx_stride = idx_stride;
   a.seq_len_blocks = int32_t(nbs);
   a.cand_begin = int32_t(sink_end);
   a.cand_end = int32_t(first_local);

@@ -137,9 +137,10 @@ COBS_API cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k
  *   q           device [batch][Hq][d] bf16, this decode step's queries.
  *   stats       device, records of every complete block below seq_len.
  *   seq_len     tokens in the cache, 1 <= seq_len <= capacity_tokens.
- *   idx         device [batch][Hkv][cobs_selected_capacity(...)] int32,
- *               selected block indices ascending; entries past n_sel are
- *               left untouched.
+ *   idx         device [batch][Hkv][idx_stride] int32, selected block
+ *               indices ascending; entries past n_sel are left untouched.
+ *   idx_stride  row length of idx; at least cobs_selected_capacity() for
+ *               these top_k / sink_blocks / local_tokens (INVALID_ARG if not).
  *   n_sel       device [batch][Hkv] int32, number of selected blocks.
  *   scores_opt  device [batch][Hkv][capacity/B] fp32 or NULL: S_b of the
  *               scored candidates (other entries untouched).
@@ -148,8 +149,9 @@ COBS_API cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q,
                                const void* stats, int64_t seq_len,
                                int32_t top_k, int32_t sink_blocks,
                                int32_t local_tokens, int32_t* idx,
-                               int32_t* n_sel, float* scores_opt, void* ws,
-                               size_t ws_bytes, void* stream);
+                               int32_t idx_stride, int32_t* n_sel,
+                               float* scores_opt, void* ws, size_t ws_bytes,
+                               void* stream);
 
 /* Exact attention of every query head over the valid tokens (< seq_len) of
  * the blocks listed for its kv-head: out = softmax(q K^T * softmax_scale) V,

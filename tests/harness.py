@@ -92,7 +92,8 @@ class Problem:
                               w.top_k if top_k is None else top_k,
                               w.sink_blocks if sink is None else sink,
                               w.local_tokens if local is None else local,
-                              self.idx, self.n_sel, self.scores if scores else None,
+                              self.idx, self.idx.shape[-1], self.n_sel,
+                              self.scores if scores else None,
                               self.ws, self.ws_bytes)
 
     def decode(self, seq_len=None, idx=None, n_sel=None, stride=None):

@@ -84,7 +84,7 @@ def test_bad_dims_rejected_everywhere(kw, code):
         cb.cobs_build_block_stats(d, fake, 0, 1, fake, fake, 1 << 20)
     assert e.value.status == code
     with pytest.raises(cb.CobsError) as e:
-        cb.cobs_select_blocks(d, fake, fake, 100, 8, 1, 64, fake, fake, None, fake, 1 << 20)
+        cb.cobs_select_blocks(d, fake, fake, 100, 8, 1, 64, fake, 64, fake, None, fake, 1 << 20)
     assert e.value.status == code
     with pytest.raises(cb.CobsError) as e:
         cb.cobs_sparse_decode(d, fake, fake, fake, fake, fake, 10, 100, 0.1, fake, fake,
@@ -112,20 +112,22 @@ def test_pointer_and_range_checks():
         (lambda: cb.cobs_build_block_stats(d, A, 0, 4, A, None, 4096), cb.COBS_ERR_WORKSPACE),
         (lambda: cb.cobs_build_block_stats(d, A, 0, 4, A, A, 16), cb.COBS_ERR_WORKSPACE),
         # select
-        (lambda: cb.cobs_select_blocks(d, A, A, 0, 8, 1, 64, A, A, None, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, 0, 8, 1, 64, A, 64, A, None, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, w.cap + 1, 8, 1, 64, A, A, None, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, w.cap + 1, 8, 1, 64, A, 64, A, None, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, 100, -1, 1, 64, A, A, None, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, -1, 1, 64, A, 64, A, None, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, None, A, None, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, None, 64, A, None, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, A + 4, None, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, 64, A + 4, None, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, A, A + 2, A, ws_need),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 8, 1, 64, A, 64, A, A + 2, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),
-        (lambda: cb.cobs_select_blocks(d, A, A, 100, 16, 1, 512, A, A, None, A, 1024),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 16, 1, 512, A, 64, A, None, A, 1024),
          cb.COBS_ERR_WORKSPACE),
+        (lambda: cb.cobs_select_blocks(d, A, A, 100, 16, 1, 512, A, 25, A, None, A, ws_need),
+         cb.COBS_ERR_INVALID_ARG),                       # idx row too short for 26 blocks
         # decode
         (lambda: cb.cobs_sparse_decode(d, A, A, A, A, A, 0, 100, 0.1, A, A, A, ws_need),
          cb.COBS_ERR_INVALID_ARG),

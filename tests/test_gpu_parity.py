@@ -213,8 +213,8 @@ def test_repeat_and_graph_replay_are_stable(prob):
         with torch.cuda.graph(g, stream=s):
             import block_sparse_long_cobs_b200 as cb
             cb.cobs_select_blocks(p.dims, p.q, p.stats, w.seq_len, w.top_k, w.sink_blocks,
-                                  w.local_tokens, p.idx, p.n_sel, None, p.ws, p.ws_bytes,
-                                  stream=s)
+                                  w.local_tokens, p.idx, p.nsm, p.n_sel, None, p.ws,
+                                  p.ws_bytes, stream=s)
             cb.cobs_sparse_decode(p.dims, p.q, p.k, p.v, p.idx, p.n_sel, p.nsm, w.seq_len,
                                   1 / math.sqrt(w.head_dim), p.out, p.lse, p.ws,
                                   p.ws_bytes, stream=s)
@@ -223,7 +223,12 @@ def test_repeat_and_graph_replay_are_stable(prob):
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
-    assert torch.equal(ref[0], p.idx) and torch.equal(ref[2], p.out)
+    n = p.n_sel.cpu().numpy()
+    a_idx, b_idx = ref[0].cpu().numpy(), p.idx.cpu().numpy()
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            assert list(a_idx[b, h, :n[b, h]]) == list(b_idx[b, h, :n[b, h]])
+    assert torch.equal(ref[2], p.out) and torch.equal(ref[1], p.n_sel)
     del g
     assert p.device_status() == 0
 
@@ -265,7 +270,9 @@ def edge():
 def test_select_edge_cases(edge, seq_len, top_k, sink, local):
     p, recs = edge
     w = EDGE.scaled(seq_len=seq_len, top_k=top_k, sink_blocks=sink, local_tokens=local)
-    p.idx.fill_(-9)
+    import block_sparse_long_cobs_b200 as cb
+    nsm = cb.cobs_selected_capacity(p.dims, top_k, sink, local)
+    p.idx = torch.full((w.batch, w.kv_heads, nsm), -9, dtype=torch.int32, device="cuda")
     p.select(seq_len=seq_len, top_k=top_k, sink=sink, local=local)
     idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
     for (b, h), r in recs.items():
