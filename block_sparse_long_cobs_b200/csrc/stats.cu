@@ -17,14 +17,21 @@
 //      128-byte swizzle = the UMMA K-major canonical layout).
 //   2. Centring in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
 //      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T.
-//   3. Eigenpairs of Gc by one-sided (Hestenes) Jacobi on its columns, two
-//      warps per block (rows split in halves, dot products exchanged through
-//      shared memory), round-robin pairing, fp32.  On convergence column k is
-//      lambda_k w_k with w_k a unit eigenvector of Gc and lambda_k = n times
-//      the covariance eigenvalue.
-//   4. U[:, k] = Kc^T w_k / sqrt(n) for the r largest lambda_k (its squared
-//      norm is the covariance eigenvalue lambda_k / n), sign fixed so that the
-//      largest-magnitude component is positive; written with mu as bf16.
+//   3. Lanczos tridiagonalisation of Gc (64 steps, every new vector
+//      re-orthogonalised twice against all earlier ones by classical
+//      Gram-Schmidt, so the basis Q stays orthogonal to fp32 accuracy and
+//      T = Q^T Gc Q is similar to Gc); a fresh pseudo-random start vector
+//      whenever the Krylov space closes.  128 threads per block, each holding
+//      32 entries of Gc in registers; named barriers between the phases.
+//   4. Top-r eigenvalues of the tridiagonal T by multisection bisection on
+//      Sturm counts (8 threads per eigenvalue, 10 rounds of 9-way splits),
+//      their eigenvectors z_k by inverse iteration (LDL^T of T - lambda I),
+//      re-orthogonalised inside clusters of close eigenvalues; Ritz vectors
+//      w_k = Q z_k are unit eigenvectors of Gc with eigenvalue lambda_k
+//      (= n times the covariance eigenvalue).
+//   5. U[:, k] = Kc^T w_k / sqrt(n) (squared norm lambda_k / n), sign fixed
+//      so that the largest-magnitude component is positive; written with mu
+//      as bf16.
 #include <cfloat>
 #include <cuda.h>
 
@@ -33,27 +40,69 @@
 namespace cobs {
 namespace {
 
-constexpr int kStatThreads = 128;   // 2 blocks x 64 threads
-constexpr int kMaxSweeps = 12;
-constexpr float kJacobiTol = 1e-6f;
-constexpr int kGcStride = 65;       // padded row of the centred Gram
+constexpr int kStatThreads = 256;   // 2 blocks x 128 threads
+constexpr int kQStride = 72;        // floats per Lanczos vector: halves of 36
+constexpr int kGcStride = 65;       // padded row of the centred Gram (staging)
+constexpr int kBisectRounds = 10;
+constexpr int kInverseIters = 3;
 
 template <int D>
 struct StatsShape {
   static constexpr int kRegions = D / 64;           // 128-byte-wide column slabs
   static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B
-  static constexpr size_t kK = 0;                   // [regions][128 rows][128 B]
-  static constexpr size_t kGc = kK + size_t(kRegions) * kRegionBytes;   // [2][64][65] f32
-  static constexpr size_t kU = kGc + 2 * 64 * kGcStride * 4;            // [2][64][16] f32
-  static constexpr size_t kMu = kU + 2 * 64 * kMaxRank * 4;             // [2][D] f32
-  static constexpr size_t kR = kMu + 2 * D * 4;                         // [2][64] f32
-  static constexpr size_t kLam = kR + 2 * 64 * 4;                       // [2][64] f32
-  static constexpr size_t kX = kLam + 2 * 64 * 4;                       // [2][2][2][32] f4
-  static constexpr size_t kFlip = kX + 2 * 2 * 2 * 32 * 16;             // [2][2][16] u32x2
-  static constexpr size_t kBar = kFlip + 2 * 2 * kMaxRank * 8;
+  // per-block regions (x2)
+  static constexpr size_t kQBytes = 64 * kQStride * 4;        // Q, also Gc staging
+  static constexpr size_t kZBytes = kMaxRank * 64 * 4;        // eigenvectors of T
+  static constexpr size_t kWBytes = 64 * kMaxRank * 4;        // Ritz vectors [t][k]
+  static constexpr size_t kScrBytes = kMaxRank * 2 * 64 * 4;  // inverse iteration
+  static constexpr size_t kVecBytes = 2048;                   // small vectors
+  static constexpr size_t kK = 0;                             // [regions][128][128 B]
+  static constexpr size_t kQ = kK + size_t(kRegions) * kRegionBytes;
+  static constexpr size_t kZ = kQ + 2 * kQBytes;
+  static constexpr size_t kW = kZ + 2 * kZBytes;
+  static constexpr size_t kScr = kW + 2 * kWBytes;
+  static constexpr size_t kVec = kScr + 2 * kScrBytes;
+  static constexpr size_t kMu = kVec + 2 * kVecBytes;          // [2][D]
+  static constexpr size_t kRow = kMu + 2 * D * 4;              // [128] row means
+  static constexpr size_t kFlip = kRow + 128 * 4;              // [2][4][16] uint2
+  static constexpr size_t kBar = kFlip + 2 * 4 * kMaxRank * 8;
   static constexpr size_t kMisc = kBar + 16;
   static constexpr size_t kBytes = kMisc + 16 + 1024;  // + alignment slack
+  static_assert(64 * kGcStride * 4 <= kQBytes, "Gc staging must fit in Q");
 };
+
+// Offsets inside the per-block small-vector area (floats).
+constexpr int kVW = 0;        // w, split layout [2][36]
+constexpr int kVH = 72;       // CGS coefficients h [64]
+constexpr int kVRed = 136;    // reduction partials [8]
+constexpr int kVAlpha = 144;  // T diagonal [64]
+constexpr int kVBeta2 = 208;  // T off-diagonal squared [64]
+constexpr int kVBeta = 272;   // T off-diagonal [64]
+constexpr int kVLam = 336;    // eigenvalues (descending) [16]
+constexpr int kVTrace = 352;  // trace of Gc [1]
+
+__device__ __forceinline__ float hash_sign(uint32_t a, uint32_t b) {
+  uint32_t h = a * 0x9E3779B1u ^ (b + 0x7F4A7C15u) * 0x85EBCA77u;
+  h ^= h >> 15;
+  h *= 0x2C1B3C6Du;
+  h ^= h >> 12;
+  return (h & 1u) ? 1.f : -1.f;
+}
+
+// Number of eigenvalues of the tridiagonal T (diag alpha, off-diag^2 beta2)
+// below x: count of negative pivots of the LDL^T factorisation of T - x I.
+__device__ __forceinline__ int sturm_count(const float* alpha, const float* beta2, float x) {
+  int cnt = 0;
+  float d = alpha[0] - x;
+  cnt += d < 0.f;
+#pragma unroll 8
+  for (int i = 1; i < 64; ++i) {
+    const float dd = fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
+    d = alpha[i] - x - beta2[i - 1] / dd;
+    cnt += d < 0.f;
+  }
+  return cnt;
+}
 
 // ---- tcgen05 / TMA wrappers ---------------------------------------------------
 
@@ -161,12 +210,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ktile = smem + S::kK;
-  float* gc = reinterpret_cast<float*>(smem + S::kGc);
-  float* us = reinterpret_cast<float*>(smem + S::kU);
-  float* mus = reinterpret_cast<float*>(smem + S::kMu);
-  float* rs = reinterpret_cast<float*>(smem + S::kR);
-  float* lam_s = reinterpret_cast<float*>(smem + S::kLam);
-  float4* xch = reinterpret_cast<float4*>(smem + S::kX);
+  float* row_mean = reinterpret_cast<float*>(smem + S::kRow);
   uint2* flip_s = reinterpret_cast<uint2*>(smem + S::kFlip);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kMisc);
@@ -178,10 +222,19 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   const int64_t bh = int64_t(b) * a.hkv + kvh;
   const int64_t j0 = a.block_begin + 2 * int64_t(blockIdx.x);
   const bool has1 = j0 + 1 < a.block_end;
-  const int blk = tid >> 6;            // which of the two blocks this thread serves
-  const int i = tid & 63;              // row of that block's Gram
+  const int blk = tid >> 7;            // block of the pair this thread serves
+  const int bt = tid & 127;            // thread index inside that block's team
+  const int bwarp = bt >> 5;           // warp index inside the team
   const bool my_valid = blk == 0 || has1;
   const int r = a.rank;
+  const int bar_id = 1 + blk;
+
+  float* Qs = reinterpret_cast<float*>(smem + S::kQ + blk * S::kQBytes);
+  float* Zs = reinterpret_cast<float*>(smem + S::kZ + blk * S::kZBytes);
+  float* Ws = reinterpret_cast<float*>(smem + S::kW + blk * S::kWBytes);
+  float* Scr = reinterpret_cast<float*>(smem + S::kScr + blk * S::kScrBytes);
+  float* V = reinterpret_cast<float*>(smem + S::kVec + blk * S::kVecBytes);
+  float* mus = reinterpret_cast<float*>(smem + S::kMu) + blk * D;
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);  // TMA
@@ -226,11 +279,13 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   if (!aborted && tid != 0) (void)mbar_try_wait(&bars[1], 0);
   tc_fence_after();
 
-  // ---- 2. read this thread's Gram row back and centre it ---------------------
+  // ---- 2. Gram rows back from tensor memory (warps 0-3), centring -----------
+  // Thread t < 128 reads TMEM lane t = row (t & 63) of block (t >> 6).
   float g[64];
-  if (!aborted) {
+  const int rb = tid >> 6, ri = tid & 63;
+  if (!aborted && warp < 4) {
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t col0 = uint32_t(blk * 64);
+    const uint32_t col0 = uint32_t(rb * 64);
     float t32[32];
     tmem_ld32(tmem + lane_base + col0, t32);
 #pragma unroll
@@ -238,210 +293,297 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     tmem_ld32(tmem + lane_base + col0 + 32, t32);
 #pragma unroll
     for (int c = 0; c < 32; ++c) g[32 + c] = t32[c];
+    float rsum = 0.f;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) rsum += g[c];
+    row_mean[tid] = rsum * (1.f / 64.f);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 128);
   if (aborted) return;
-
-  float rsum = 0.f;
-#pragma unroll
-  for (int c = 0; c < 64; ++c) rsum += g[c];
-  rs[blk * 64 + i] = rsum * (1.f / 64.f);
-
-  // block mean (fp32 sum of 64 bf16 keys), DPT dims per thread
-  constexpr int DPT = D / 64;
-  {
-    float acc[DPT];
-#pragma unroll
-    for (int e = 0; e < DPT; ++e) acc[e] = 0.f;
-    for (int t = 0; t < kBlock; ++t) {
-      const int row = blk * 64 + t;
-      if constexpr (DPT == 2) {
-        const uint32_t w =
-            *reinterpret_cast<const uint32_t*>(ktile + k_offset<D>(row, 2 * i));
-        const float2 f = bf16x2_to_float2(w);
-        acc[0] += f.x;
-        acc[1] += f.y;
-      } else {
-        const uint16_t w = *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(row, i));
-        acc[0] += __uint_as_float(uint32_t(w) << 16);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < DPT; ++e) mus[blk * D + DPT * i + e] = acc[e] * (1.f / 64.f);
-  }
-  __syncthreads();
-  {
+  if (warp < 4) {
     float ssum = 0.f;
-    for (int c = 0; c < 64; ++c) ssum += rs[blk * 64 + c];
+    for (int c = 0; c < 64; ++c) ssum += row_mean[rb * 64 + c];
     const float smean = ssum * (1.f / 64.f);
-    const float ri = rs[blk * 64 + i];
+    const float rm = row_mean[tid];
+    float* stage = reinterpret_cast<float*>(smem + S::kQ + rb * S::kQBytes);
 #pragma unroll
     for (int c = 0; c < 64; ++c)
-      gc[(blk * 64 + i) * kGcStride + c] = g[c] - ri - rs[blk * 64 + c] + smean;
+      stage[ri * kGcStride + c] = g[c] - rm - row_mean[rb * 64 + c] + smean;
   }
-  __syncthreads();
 
-  // ---- 3. one-sided Jacobi on the columns of Gc (2 warps per block) ----------
-  const int hf = warp & 1;          // row half owned by this warp
-  const int bar_id = 1 + blk;
-  int top_id = lane, bot_id = 63 - lane;
-  float x[32], y[32];
-  if (r > 0 && my_valid) {
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      x[k] = gc[(blk * 64 + hf * 32 + k) * kGcStride + top_id];
-      y[k] = gc[(blk * 64 + hf * 32 + k) * kGcStride + bot_id];
-    }
-    int step = 0;
-    for (int sweep = 0; sweep < kMaxSweeps; ++sweep) {
-      bool rotated = false;
-      for (int round = 0; round < 63; ++round, ++step) {
-        float al = 0.f, be = 0.f, ga = 0.f;
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          al = fmaf(x[k], x[k], al);
-          be = fmaf(y[k], y[k], be);
-          ga = fmaf(x[k], y[k], ga);
-        }
-        float4* slot = xch + ((blk * 2 + (step & 1)) * 2) * 32;
-        slot[hf * 32 + lane] = make_float4(al, be, ga, 0.f);
-        named_bar(bar_id, 64);
-        const float4 o = slot[(1 - hf) * 32 + lane];
-        // identical sums in both warps: (half 0) + (half 1)
-        const float A = hf == 0 ? al + o.x : o.x + al;
-        const float Bv = hf == 0 ? be + o.y : o.y + be;
-        const float C = hf == 0 ? ga + o.z : o.z + ga;
-        if (fabsf(C) > kJacobiTol * sqrtf(A * Bv) && A * Bv > 0.f) {
-          const float zeta = (Bv - A) / (2.f * C);
-          const float t = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(1.f + zeta * zeta));
-          const float c = rsqrtf(1.f + t * t);
-          const float s = c * t;
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const float xv = x[k], yv = y[k];
-            x[k] = c * xv - s * yv;
-            y[k] = s * xv + c * yv;
-          }
-          rotated = true;
-        }
-        // round-robin: top slots shift right (lane 1 takes bottom of lane 0),
-        // bottom slots shift left (lane 31 takes top of lane 31); lane 0's top
-        // stays.
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float up = __shfl_up_sync(0xffffffffu, lane == 0 ? y[k] : x[k], 1);
-          const float dn = __shfl_down_sync(0xffffffffu, y[k], 1);
-          const float xo = x[k];
-          if (lane != 0) x[k] = up;
-          y[k] = (lane == 31) ? xo : dn;
-        }
-        {
-          const int up = __shfl_up_sync(0xffffffffu, lane == 0 ? bot_id : top_id, 1);
-          const int dn = __shfl_down_sync(0xffffffffu, bot_id, 1);
-          const int to = top_id;
-          if (lane != 0) top_id = up;
-          bot_id = (lane == 31) ? to : dn;
-        }
-      }
-      if (!__any_sync(0xffffffffu, rotated)) break;
-    }
-
-    // column norms (Gram eigenvalues) and ranking
-    float nx = 0.f, ny = 0.f;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      nx = fmaf(x[k], x[k], nx);
-      ny = fmaf(y[k], y[k], ny);
-    }
-    float4* slot = xch + ((blk * 2 + (step & 1)) * 2) * 32;
-    slot[hf * 32 + lane] = make_float4(nx, ny, 0.f, 0.f);
-    named_bar(bar_id, 64);
-    const float4 o = slot[(1 - hf) * 32 + lane];
-    const float lx = sqrtf(hf == 0 ? nx + o.x : o.x + nx);
-    const float ly = sqrtf(hf == 0 ? ny + o.y : o.y + ny);
-    if (hf == 0) {
-      lam_s[blk * 64 + top_id] = lx;
-      lam_s[blk * 64 + bot_id] = ly;
-    }
-    named_bar(bar_id, 64);
-    int rank_x = 0, rank_y = 0;
-    float lmax = 0.f;
-    for (int c = 0; c < 64; ++c) {
-      const float lc = lam_s[blk * 64 + c];
-      lmax = fmaxf(lmax, lc);
-      rank_x += (lc > lx || (lc == lx && c < top_id)) ? 1 : 0;
-      rank_y += (lc > ly || (lc == ly && c < bot_id)) ? 1 : 0;
-    }
-    const float floor_l = lmax * 1e-6f;
-    if (rank_x < r) {
-      const float inv = (lx > floor_l && lx > 0.f) ? 1.f / lx : 0.f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) us[(blk * 64 + hf * 32 + k) * kMaxRank + rank_x] = x[k] * inv;
-    }
-    if (rank_y < r) {
-      const float inv = (ly > floor_l && ly > 0.f) ? 1.f / ly : 0.f;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) us[(blk * 64 + hf * 32 + k) * kMaxRank + rank_y] = y[k] * inv;
-    }
-  }
-  __syncthreads();
-
-  // ---- 4. U = Kc^T w / sqrt(n), sign rule, bf16 record ------------------------
-  float uacc[DPT][kMaxRank];
-#pragma unroll
-  for (int e = 0; e < DPT; ++e)
-#pragma unroll
-    for (int k = 0; k < kMaxRank; ++k) uacc[e][k] = 0.f;
-  float mu_d[DPT];
-#pragma unroll
-  for (int e = 0; e < DPT; ++e) mu_d[e] = mus[blk * D + DPT * i + e];
-  if (r > 0 && my_valid) {
+  // block mean (fp32 sum of 64 bf16 keys): thread bt < D owns dim bt
+  if (bt < D) {
+    float acc = 0.f;
     for (int t = 0; t < kBlock; ++t) {
-      const int row = blk * 64 + t;
-      float kc[DPT];
-      if constexpr (DPT == 2) {
-        const float2 f = bf16x2_to_float2(
-            *reinterpret_cast<const uint32_t*>(ktile + k_offset<D>(row, 2 * i)));
-        kc[0] = f.x - mu_d[0];
-        kc[1] = f.y - mu_d[1];
-      } else {
-        const uint16_t w = *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(row, i));
-        kc[0] = __uint_as_float(uint32_t(w) << 16) - mu_d[0];
+      const uint16_t w =
+          *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(blk * 64 + t, bt));
+      acc += __uint_as_float(uint32_t(w) << 16);
+    }
+    mus[bt] = acc * (1.f / 64.f);
+  }
+  __syncthreads();
+
+  // ---- 3. Lanczos with full re-orthogonalisation -----------------------------
+  // Thread (i, hh) = (bt >> 1, bt & 1) owns Gram row i, columns 2k + hh.
+  const int li = bt >> 1, hh = bt & 1;
+  float gr[32];
+  {
+    const float* stage = Qs;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) gr[k] = stage[li * kGcStride + 2 * k + hh];
+  }
+  float trace_part = (hh == (li & 1)) ? gr[li >> 1] : 0.f;   // diagonal entry once
+  named_bar(bar_id, 128);                  // staging area becomes Q
+
+  const bool do_eig = r > 0 && my_valid;
+  auto block_sum = [&](float v) -> float {  // sum over the 128 threads of the team
+    v = warp_sum(v);
+    if (lane == 0) V[kVRed + bwarp] = v;
+    named_bar(bar_id, 128);
+    const float s = (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
+    return s;
+  };
+  // split layout: element e of a 64-vector sits at (e & 1) * 36 + (e >> 1)
+  auto qidx = [](int e) { return (e & 1) * 36 + (e >> 1); };
+
+  if (do_eig) {
+    const float trace = block_sum(trace_part);
+    const float tol = 1e-5f * trace;
+    named_bar(bar_id, 128);                 // everyone read the partials
+    if (hh == 0) Qs[qidx(li)] = hash_sign(7u, uint32_t(li)) * 0.125f;
+    named_bar(bar_id, 128);
+
+    // orthogonalise w (this thread's entry wi for row li) against Q[0..jmax]
+    auto cgs = [&](float& wi, int jmax, bool want_alpha, int jalpha) -> float {
+      float acoef = 0.f;
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        if (hh == 0) V[kVW + qidx(li)] = wi;
+        named_bar(bar_id, 128);
+        float hp = 0.f;
+        if (li <= jmax) {
+          const float4* qm = reinterpret_cast<const float4*>(Qs + li * kQStride + hh * 36);
+          const float4* ws = reinterpret_cast<const float4*>(V + kVW + hh * 36);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float4 x = qm[k], y = ws[k];
+            hp = fmaf(x.x, y.x, hp);
+            hp = fmaf(x.y, y.y, hp);
+            hp = fmaf(x.z, y.z, hp);
+            hp = fmaf(x.w, y.w, hp);
+          }
+        }
+        hp += __shfl_xor_sync(0xffffffffu, hp, 1);
+        if (hh == 0) V[kVH + li] = hp;
+        named_bar(bar_id, 128);
+        float corr = 0.f;
+        const int col = qidx(li);
+        for (int m = hh; m <= jmax; m += 2) corr = fmaf(Qs[m * kQStride + col], V[kVH + m], corr);
+        corr += __shfl_xor_sync(0xffffffffu, corr, 1);
+        wi -= corr;
+        if (want_alpha) acoef += V[kVH + jalpha];
       }
-      const float4* ut = reinterpret_cast<const float4*>(us + (blk * 64 + t) * kMaxRank);
+      return acoef;
+    };
+
+#pragma unroll 1
+    for (int j = 0; j < 64; ++j) {
+      // w = Gc q_j
+      const float4* qj = reinterpret_cast<const float4*>(Qs + j * kQStride + hh * 36);
+      float p = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 x = qj[k];
+        p = fmaf(gr[4 * k + 0], x.x, p);
+        p = fmaf(gr[4 * k + 1], x.y, p);
+        p = fmaf(gr[4 * k + 2], x.z, p);
+        p = fmaf(gr[4 * k + 3], x.w, p);
+      }
+      float wi = p + __shfl_xor_sync(0xffffffffu, p, 1);
+      const float aj = cgs(wi, j, true, j);
+      float beta = sqrtf(block_sum(hh == 0 ? wi * wi : 0.f));
+      if (bt == 0) V[kVAlpha + j] = aj;
+      if (j == 63) break;
+      if (!(beta > tol)) {
+        // the Krylov space closed: continue from a fresh vector
+        wi = hash_sign(uint32_t(j + 1), uint32_t(li));
+        named_bar(bar_id, 128);
+        cgs(wi, j, false, 0);
+        const float nrm = sqrtf(block_sum(hh == 0 ? wi * wi : 0.f));
+        wi = nrm > 0.f ? wi / nrm : 0.f;
+        beta = 0.f;
+      } else {
+        wi = wi / beta;
+      }
+      if (bt == 0) {
+        V[kVBeta + j] = beta;
+        V[kVBeta2 + j] = beta * beta;
+      }
+      if (hh == 0) Qs[(j + 1) * kQStride + qidx(li)] = wi;
+      named_bar(bar_id, 128);
+    }
+    named_bar(bar_id, 128);
+
+    // ---- 4. top-r eigenpairs of T -----------------------------------------
+    const float* alpha = V + kVAlpha;
+    const float* beta2 = V + kVBeta2;
+    const float* betav = V + kVBeta;
+    float lo = 0.f, hi = 0.f;
+    for (int i2 = 0; i2 < 64; ++i2) {
+      const float rad = (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < 63 ? fabsf(betav[i2]) : 0.f);
+      lo = fminf(lo, alpha[i2] - rad);
+      hi = fmaxf(hi, alpha[i2] + rad);
+    }
+    hi = hi * (1.f + 1e-6f) + 1e-30f;
+    lo = lo - 1e-6f * fabsf(hi) - 1e-30f;
+    const int grp = bt >> 3, sub = bt & 7;   // 8 threads per eigenvalue
+    const int kk = grp;                      // k-th largest
+    const int target = 63 - kk;              // count(x) <= target below it
+    float ea = lo, eb = hi;
+    for (int it = 0; it < kBisectRounds; ++it) {
+      const float step = (eb - ea) * (1.f / 9.f);
+      const float x = ea + step * float(sub + 1);
+      const bool above = sturm_count(alpha, beta2, x) > target;
+      const uint32_t bal = __ballot_sync(0xffffffffu, above);
+      const uint32_t mine = (bal >> ((lane >> 3) << 3)) & 0xffu;
+      const int first = mine ? __ffs(mine) - 1 : 8;   // first point above the eigenvalue
+      const float na = first == 0 ? ea : ea + step * float(first);
+      const float nb = first == 8 ? eb : ea + step * float(first + 1);
+      ea = na;
+      eb = nb;
+    }
+    const float lam = 0.5f * (ea + eb);
+    if (sub == 0 && kk < r) V[kVLam + kk] = lam;
+    named_bar(bar_id, 128);
+
+    // inverse iteration, one thread per eigenvalue: (T - lam I) z = y via LDL^T
+    if (sub == 0 && kk < r) {
+      float* zk = Zs + kk * 64;
+      float* dl = Scr + kk * 128;       // [0,64): l_i ; [64,128): d_i
+      float nrm2 = 0.f;
+      for (int i2 = 0; i2 < 64; ++i2) {
+        zk[i2] = 1.f + 0.25f * hash_sign(uint32_t(kk + 101), uint32_t(i2));
+      }
+      // factorisation (once)
+      {
+        float d = alpha[0] - lam;
+        d = fabsf(d) < 1e-30f ? 1e-30f : d;
+        dl[64] = d;
+        for (int i2 = 1; i2 < 64; ++i2) {
+          const float l = betav[i2 - 1] / d;
+          d = alpha[i2] - lam - l * betav[i2 - 1];
+          d = fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
+          dl[i2] = l;
+          dl[64 + i2] = d;
+        }
+      }
+      for (int it = 0; it < kInverseIters; ++it) {
+        for (int i2 = 1; i2 < 64; ++i2) zk[i2] -= dl[i2] * zk[i2 - 1];
+        for (int i2 = 0; i2 < 64; ++i2) zk[i2] /= dl[64 + i2];
+        for (int i2 = 62; i2 >= 0; --i2) zk[i2] -= dl[i2 + 1] * zk[i2 + 1];
+        float mx = 0.f;
+        for (int i2 = 0; i2 < 64; ++i2) mx = fmaxf(mx, fabsf(zk[i2]));
+        const float inv = mx > 0.f ? 1.f / mx : 1.f;
+        nrm2 = 0.f;
+        for (int i2 = 0; i2 < 64; ++i2) {
+          zk[i2] *= inv;
+          nrm2 += zk[i2] * zk[i2];
+        }
+      }
+      const float inv = rsqrtf(fmaxf(nrm2, 1e-30f));
+      for (int i2 = 0; i2 < 64; ++i2) zk[i2] *= inv;
+    }
+    named_bar(bar_id, 128);
+    // re-orthogonalise inside clusters of close eigenvalues (warp 0 of the team)
+    if (bwarp == 0) {
+      const float lam0 = V[kVLam + 0];
+      for (int k2 = 1; k2 < r; ++k2) {
+        const float lk = V[kVLam + k2];
+        float* zk = Zs + k2 * 64;
+        bool touched = false;
+        for (int l2 = 0; l2 < k2; ++l2) {
+          if (fabsf(V[kVLam + l2] - lk) > 1e-3f * fabsf(lam0)) continue;
+          const float* zl = Zs + l2 * 64;
+          const float c = warp_sum(zl[lane] * zk[lane] + zl[lane + 32] * zk[lane + 32]);
+          zk[lane] -= c * zl[lane];
+          zk[lane + 32] -= c * zl[lane + 32];
+          touched = true;
+          __syncwarp();
+        }
+        if (touched) {
+          const float n2 = warp_sum(zk[lane] * zk[lane] + zk[lane + 32] * zk[lane + 32]);
+          const float inv = rsqrtf(fmaxf(n2, 1e-30f));
+          zk[lane] *= inv;
+          zk[lane + 32] *= inv;
+        }
+        __syncwarp();
+      }
+    }
+    named_bar(bar_id, 128);
+    // Ritz vectors w_k = Q z_k, stored [t][k]; thread (t = li, hh) takes k = hh, hh+2, ...
+    {
+      const int col = qidx(li);
+      float acc[kMaxRank / 2];
+#pragma unroll
+      for (int k2 = 0; k2 < kMaxRank / 2; ++k2) acc[k2] = 0.f;
+      for (int m = 0; m < 64; ++m) {
+        const float qv = Qs[m * kQStride + col];
+#pragma unroll
+        for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
+          const int k = 2 * k2 + hh;
+          if (k < r) acc[k2] = fmaf(qv, Zs[k * 64 + m], acc[k2]);
+        }
+      }
+      const float lam0 = V[kVLam + 0];
+#pragma unroll
+      for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
+        const int k = 2 * k2 + hh;
+        if (k < r) {
+          const float lk = V[kVLam + k];
+          const bool keep = lk > 1e-6f * lam0 && lk > 0.f;
+          Ws[li * kMaxRank + k] = keep ? acc[k2] : 0.f;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- 5. U = Kc^T w / sqrt(n), sign rule, bf16 record ------------------------
+  // thread bt < D owns output dim d = bt
+  float uacc[kMaxRank];
+#pragma unroll
+  for (int k = 0; k < kMaxRank; ++k) uacc[k] = 0.f;
+  const float mu_d = bt < D ? mus[bt] : 0.f;
+  if (do_eig && bt < D) {
+    for (int t = 0; t < kBlock; ++t) {
+      const uint16_t w =
+          *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(blk * 64 + t, bt));
+      const float kc = __uint_as_float(uint32_t(w) << 16) - mu_d;
+      const float4* wt = reinterpret_cast<const float4*>(Ws + t * kMaxRank);
 #pragma unroll
       for (int k4 = 0; k4 < kMaxRank / 4; ++k4) {
         if (4 * k4 < r) {
-          const float4 u4 = ut[k4];
-#pragma unroll
-          for (int e = 0; e < DPT; ++e) {
-            uacc[e][4 * k4 + 0] = fmaf(kc[e], u4.x, uacc[e][4 * k4 + 0]);
-            uacc[e][4 * k4 + 1] = fmaf(kc[e], u4.y, uacc[e][4 * k4 + 1]);
-            uacc[e][4 * k4 + 2] = fmaf(kc[e], u4.z, uacc[e][4 * k4 + 2]);
-            uacc[e][4 * k4 + 3] = fmaf(kc[e], u4.w, uacc[e][4 * k4 + 3]);
-          }
+          const float4 u4 = wt[k4];
+          uacc[4 * k4 + 0] = fmaf(kc, u4.x, uacc[4 * k4 + 0]);
+          uacc[4 * k4 + 1] = fmaf(kc, u4.y, uacc[4 * k4 + 1]);
+          uacc[4 * k4 + 2] = fmaf(kc, u4.z, uacc[4 * k4 + 2]);
+          uacc[4 * k4 + 3] = fmaf(kc, u4.w, uacc[4 * k4 + 3]);
         }
       }
     }
   }
   // sign: the component of largest magnitude (lowest index on ties) is positive
-  uint32_t neg_mask = 0;
   if (r > 0) {
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
       if (k < r) {
-        float best = -1.f;
-        int bidx = 0x7fffffff;
-        uint32_t bneg = 0;
-#pragma unroll
-        for (int e = 0; e < DPT; ++e) {
-          const float v = uacc[e][k] * 0.125f;  // 1/sqrt(64)
-          uacc[e][k] = v;
-          const float av = fabsf(v);
-          if (av > best) { best = av; bidx = DPT * i + e; bneg = v < 0.f; }
-        }
+        const float v = uacc[k] * 0.125f;  // 1/sqrt(64)
+        uacc[k] = v;
+        float best = bt < D ? fabsf(v) : -1.f;
+        int bidx = bt;
+        uint32_t bneg = v < 0.f;
 #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) {
           const float ob = __shfl_xor_sync(0xffffffffu, best, m);
@@ -449,48 +591,37 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
           const uint32_t on = __shfl_xor_sync(0xffffffffu, bneg, m);
           if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; bneg = on; }
         }
-        if (lane == 0) flip_s[(blk * 2 + hf) * kMaxRank + k] =
-            make_uint2(__float_as_uint(best), (uint32_t(bidx) << 1) | bneg);
+        if (lane == 0)
+          flip_s[(blk * 4 + bwarp) * kMaxRank + k] =
+              make_uint2(__float_as_uint(best), (uint32_t(bidx) << 1) | bneg);
       }
     }
   }
   __syncthreads();
+  uint32_t neg_mask = 0;
   if (r > 0) {
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
       if (k < r) {
-        const uint2 h0 = flip_s[(blk * 2 + 0) * kMaxRank + k];
-        const uint2 h1 = flip_s[(blk * 2 + 1) * kMaxRank + k];
-        const float b0 = __uint_as_float(h0.x), b1 = __uint_as_float(h1.x);
-        const uint32_t pick = (b1 > b0 || (b1 == b0 && (h1.y >> 1) < (h0.y >> 1))) ? h1.y : h0.y;
-        neg_mask |= (pick & 1u) << k;
+        uint2 best = flip_s[(blk * 4 + 0) * kMaxRank + k];
+        for (int w2 = 1; w2 < 4; ++w2) {
+          const uint2 o = flip_s[(blk * 4 + w2) * kMaxRank + k];
+          const float bo = __uint_as_float(o.x), bb = __uint_as_float(best.x);
+          if (bo > bb || (bo == bb && (o.y >> 1) < (best.y >> 1))) best = o;
+        }
+        neg_mask |= (best.y & 1u) << k;
       }
     }
   }
-  if (my_valid) {
+  if (my_valid && bt < D) {
     const int64_t jb = j0 + blk;
     uint16_t* rec = a.stats + ((bh * a.nb_cap) + jb) * int64_t(1 + r) * D;
-    if constexpr (DPT == 2) {
-      const uint32_t w0 = uint32_t(float_to_bf16_bits(mu_d[0])) |
-                          (uint32_t(float_to_bf16_bits(mu_d[1])) << 16);
-      reinterpret_cast<uint32_t*>(rec)[i] = w0;
+    rec[bt] = float_to_bf16_bits(mu_d);
 #pragma unroll
-      for (int k = 0; k < kMaxRank; ++k) {
-        if (k < r) {
-          const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
-          const uint32_t w = uint32_t(float_to_bf16_bits(sg * uacc[0][k])) |
-                             (uint32_t(float_to_bf16_bits(sg * uacc[1][k])) << 16);
-          reinterpret_cast<uint32_t*>(rec + int64_t(1 + k) * D)[i] = w;
-        }
-      }
-    } else {
-      rec[i] = float_to_bf16_bits(mu_d[0]);
-#pragma unroll
-      for (int k = 0; k < kMaxRank; ++k) {
-        if (k < r) {
-          const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
-          rec[int64_t(1 + k) * D + i] = float_to_bf16_bits(sg * uacc[0][k]);
-        }
+    for (int k = 0; k < kMaxRank; ++k) {
+      if (k < r) {
+        const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
+        rec[int64_t(1 + k) * D + bt] = float_to_bf16_bits(sg * uacc[k]);
       }
     }
   }
