@@ -55,12 +55,17 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["cobs", "reference"], default="cobs")
     p.add_argument("--workload", default="batched_needles_32k")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch per GPU (smaller profiling cases)")
     p.add_argument("--gen-workers", type=int, default=0,
                    help="processes drawing the synthetic cache (0 = auto)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="time budget of the CPU-oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--stats-stream", choices=["side", "same"], default="side",
+                   help="run the completed block's stats build on a forked side stream "
+                        "(joined before the step ends) or in line before the selection")
     return p.parse_args()
 
 
@@ -327,10 +332,30 @@ def run_cobs(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     build_ms = e0.elapsed_time(e1)
 
+    side = torch.cuda.Stream(dev) if args.stats_stream == "side" else None
+    fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
+
     def step(ev=None):
+        # ev: [step start, selection start, decode start, step end, stats start, stats end]
         if ev is not None:
             ev[0].record(stream)
-        cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, stream)
+        if side is not None:
+            # the block completed at this step lies in the local window, so the
+            # selection below never reads the record being written
+            fork_ev.record(stream)
+            side.wait_event(fork_ev)
+            if ev is not None:
+                ev[4].record(side)
+            cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, side)
+            if ev is not None:
+                ev[5].record(side)
+            join_ev.record(side)
+        else:
+            if ev is not None:
+                ev[4].record(stream)
+            cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, stream)
+            if ev is not None:
+                ev[5].record(stream)
         if ev is not None:
             ev[1].record(stream)
         cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
@@ -339,6 +364,8 @@ def run_cobs(args, w, rank, world, local_rank):
             ev[2].record(stream)
         cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
                               ws, ws_bytes, stream)
+        if side is not None:
+            stream.wait_event(join_ev)
         if ev is not None:
             ev[3].record(stream)
 
@@ -352,7 +379,7 @@ def run_cobs(args, w, rank, world, local_rank):
     sel_counts = n_sel.cpu().numpy()
     n_sel_mean = float(sel_counts.mean())
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
@@ -365,7 +392,7 @@ def run_cobs(args, w, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     clock_info = clocks.stop()
-    t_stats = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    t_stats = sum(e[4].elapsed_time(e[5]) for e in evs) / args.steps
     t_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     t_dec = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
     t_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
@@ -434,7 +461,12 @@ def run_cobs(args, w, rank, world, local_rank):
     kernels = {name: {"ms": t, "bytes": b, "gbs": b / (t * 1e-3) / 1e9,
                       "frac_of_hbm": b / (t * 1e-3) / 1e9 / hbm}
                for name, (t, b, _) in per_kernel.items()}
-    dom = max(per_kernel, key=lambda n: per_kernel[n][0])
+    # the kernel with the largest share of the step's critical path; a stats
+    # build that overlaps on the side stream is off that path
+    on_path = dict(per_kernel)
+    if args.stats_stream == "side" and t_stats < t_sel + t_dec:
+        on_path.pop("stats")
+    dom = max(on_path, key=lambda n: on_path[n][0])
     t_dom, b_dom, file_dom = per_kernel[dom]
     achieved = b_dom / (t_dom * 1e-3) / 1e9
     step_bytes = bm["select"] + bm["decode"] + bm["stats"]
@@ -450,7 +482,8 @@ def run_cobs(args, w, rank, world, local_rank):
                    "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
                    "selected_blocks_mean": n_sel_mean, "l2": "flushed (256 MiB) between steps",
                    "parallelism": f"replicas x{world}",
-                   "step": "stats of the completed block + select + sparse decode"},
+                   "step": "stats of the completed block + select + sparse decode",
+                   "stats_stream": args.stats_stream},
         "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
         "hbm_frac_step": step_bytes / (t_step * 1e-3) / 1e9 / hbm,
         "kernels": kernels,
@@ -476,6 +509,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.batch:
+        w = w.scaled(batch=args.batch)
     if args.impl == "reference":
         run_reference(args, w, rank)
         return

@@ -248,13 +248,17 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   a.first_local = int32_t(first_local);
   a.top_k = top_k;
 
-  // chunking: about 4 CTAs per SM over all (batch, kv-head) pairs
+  // chunking: one wave of resident CTAs shared out over the (batch, kv-head)
+  // pairs; every chunk is a whole number of 16-record (32 for d = 64) stages
   const int per_pass = 256 / (dims->head_dim / 8);
   const int64_t n_cand = first_local - sink_end;
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
   int sms = device_sm_count();
   if (sms <= 0) sms = 148;
-  int64_t chunks = ceil_div(int64_t(4) * sms, pairs);
+  const int resident =
+      sms * select_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
+                               dims->rank);
+  int64_t chunks = resident / pairs;
   const int64_t max_chunks = n_cand > 0 ? ceil_div(n_cand, per_pass) : 1;
   if (chunks > max_chunks) chunks = max_chunks;
   if (chunks < 1) chunks = 1;
@@ -311,11 +315,13 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   a.part_stride = idx_stride;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
-  // splits: about 4 CTAs per SM over all (batch, kv-head) pairs
+  // splits: one wave of resident CTAs shared out over the (batch, kv-head) pairs
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
   int sms = device_sm_count();
   if (sms <= 0) sms = 148;
-  int64_t splits = ceil_div(int64_t(4) * sms, pairs);
+  const int resident =
+      sms * decode_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads);
+  int64_t splits = resident / pairs;
   if (splits > idx_stride) splits = idx_stride;
   if (splits < 1) splits = 1;
   const int64_t bps = ceil_div(idx_stride, splits);

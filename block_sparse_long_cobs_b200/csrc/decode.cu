@@ -19,13 +19,15 @@
 // mbarriers.  Only the block's valid rows (< seq_len) are copied; nothing past
 // the sequence is ever read.
 //
-// Compute: q.K — a warp covers 16 tokens; the 16 lanes of a token (8 lanes for
-// d = 64) each own an 8-element d-slice and keep that slice of all G queries
-// in registers (pre-scaled by softmax_scale*log2 e), so each K element is read
-// from shared memory exactly once.  A reduce-scatter over those lanes leaves
-// one head's logit per lane.  P.V — lanes own 4 consecutive output dims,
-// warps own token ranges; partial accumulators are summed across warps once
-// per split.  Arithmetic is fp32 (packed fp32x2 FMA), logits in log2 units.
+// Compute (256 threads): q.K — a warp covers 8 tokens; the 16 lanes of a token
+// (8 lanes for d = 64) each own an 8-element d-slice and keep that slice of
+// all G queries in registers (pre-scaled by softmax_scale*log2 e), so each K
+// element is read from shared memory exactly once.  A reduce-scatter over
+// those lanes leaves one head's logit per lane.  Softmax — warp h owns head h.
+// P.V — lanes own 4 consecutive output dims, warps own token ranges, the
+// accumulators stay packed for fp32x2 FMA; they are summed across warps once
+// per split.  Three barriers per block: the refill of a stage is issued right
+// after the barrier that shows every thread has finished with it.
 #include <cfloat>
 
 #include "device_common.cuh"
@@ -33,14 +35,16 @@
 namespace cobs {
 namespace {
 
-constexpr int kDecThreads = 128;
+constexpr int kDecThreads = 256;
 constexpr int kStages = 2;
 
 template <int D, int G>
 struct DecodeShape {
+  static constexpr int kWarps = kDecThreads / 32;
   static constexpr int kSlices = D / 8;                 // lanes per token (q.K)
   static constexpr int kTokPerRound = 32 / kSlices;     // tokens per warp round
-  static constexpr int kRounds = 16 / kTokPerRound;     // rounds per warp (16 tok)
+  static constexpr int kTokPerWarp = kBlock / kWarps;   // tokens per warp (q.K)
+  static constexpr int kRounds = kTokPerWarp / kTokPerRound;
   static constexpr int kDimGroups = D / 4;              // P.V lanes (4 dims each)
   static constexpr int kTokGroups = kDecThreads / kDimGroups;
   static constexpr int kTokPerGroup = kBlock / kTokGroups;
@@ -55,8 +59,8 @@ struct DecodeShape {
   static constexpr size_t kBar = kAlpha + 8 * 4;                        // [S] u64
   static constexpr size_t kMisc = kBar + kStages * 8;                   // ints
   static constexpr size_t kBytes = kMisc + 16 * 4;
-  static_assert(size_t(kTokGroups) * G * D * 4 <= size_t(kStages) * kTileElems * 2,
-                "reduction buffer must fit in the K stages");
+  static_assert(kRounds >= 1, "token tiling");
+  static_assert(size_t(kTokGroups) * G * D * 4 <= kS, "reduction buffer must fit in the stages");
 };
 
 // Reduce-scatter of G per-lane partial sums over the kSlices lanes of a token.
@@ -126,23 +130,6 @@ sparse_decode_kernel(const DecodeArgs a) {
   const uint16_t* kbase = a.k + int64_t(bh) * a.cap * D;
   const uint16_t* vbase = a.v + int64_t(bh) * a.cap * D;
 
-  // ---- queries: this lane's 8-element d-slice of every head, pre-scaled ----
-  const int slice = lane % S::kSlices;
-  uint64_t qreg[G][4];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint4 w = *reinterpret_cast<const uint4*>(
-        a.q + (int64_t(b) * a.hq + kvh * G + h) * D + slice * 8);
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float2 f = bf16x2_to_float2(ww[c]);
-      f.x *= a.scale_log2;
-      f.y *= a.scale_log2;
-      qreg[h][c] = pack2(f);
-    }
-  }
-
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
     fence_barrier_init();
@@ -172,17 +159,31 @@ sparse_decode_kernel(const DecodeArgs a) {
     for (int i = 0; i < kStages && i < nblk; ++i) issue(i, i);
   }
 
-  // online-softmax state: warp w owns heads w and w + 4
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.f, 0.f};
-  // P.V accumulators: 4 consecutive dims x G heads
+  // ---- queries: this lane's 8-element d-slice of every head, pre-scaled ----
+  const int slice = lane % S::kSlices;
+  uint64_t qreg[G][4];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const uint4 w = *reinterpret_cast<const uint4*>(
+        a.q + (int64_t(b) * a.hq + kvh * G + h) * D + slice * 8);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float2 f = bf16x2_to_float2(ww[c]);
+      f.x *= a.scale_log2;
+      f.y *= a.scale_log2;
+      qreg[h][c] = pack2(f);
+    }
+  }
+
+  // online-softmax state: warp w owns head w (w < G)
+  float m_run = -INFINITY, l_run = 0.f;
+  // P.V accumulators, packed pairs: dims (4 dg, 4 dg + 1) and (4 dg + 2, 4 dg + 3)
   const int dg = tid % S::kDimGroups;
   const int tg = tid / S::kDimGroups;
-  float acc[G][4];
+  uint64_t acc01[G], acc23[G];
 #pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[h][c] = 0.f;
+  for (int h = 0; h < G; ++h) acc01[h] = acc23[h] = 0;
 
   for (int i = 0; i < nblk; ++i) {
     const int st = i % kStages;
@@ -195,9 +196,11 @@ sparse_decode_kernel(const DecodeArgs a) {
           mbar_wait_bounded(&full[k2 % kStages], (k2 / kStages) & 1, a.status);
       }
     }
-    __syncthreads();
+    __syncthreads();  // (A) block i ready; everyone is done with block i - 1
     if (*abort_s) break;
     if (tid != 0) (void)mbar_try_wait(&full[st], parity);  // acquire the TMA writes
+    // the stage of block i - 1 is free: refill it with block i - 1 + kStages
+    if (tid == 0 && i >= 1 && i - 1 + kStages < nblk) issue(i - 1 + kStages, (i - 1) % kStages);
     const int nv = nvalid_s[st];
     const uint16_t* kt = ks + st * S::kTileElems;
     const uint16_t* vt = vs + st * S::kTileElems;
@@ -205,16 +208,19 @@ sparse_decode_kernel(const DecodeArgs a) {
     // ---- logits: s_s[h][t] = q_h . k_t * scale * log2(e) -------------------
 #pragma unroll
     for (int r = 0; r < S::kRounds; ++r) {
-      const int t = warp * 16 + r * S::kTokPerRound + lane / S::kSlices;
+      const int t = warp * S::kTokPerWarp + r * S::kTokPerRound + lane / S::kSlices;
       float part[G];
       uint4 w = make_uint4(0, 0, 0, 0);
       if (t < nv) w = *reinterpret_cast<const uint4*>(kt + t * D + slice * 8);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      const uint64_t k01 = pack2(bf16x2_to_float2(w.x)), k23 = pack2(bf16x2_to_float2(w.y));
+      const uint64_t k45 = pack2(bf16x2_to_float2(w.z)), k67 = pack2(bf16x2_to_float2(w.w));
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         uint64_t acc2 = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ffma2(acc2, pack2(bf16x2_to_float2(ww[c])), qreg[h][c]);
+        ffma2(acc2, k01, qreg[h][0]);
+        ffma2(acc2, k23, qreg[h][1]);
+        ffma2(acc2, k45, qreg[h][2]);
+        ffma2(acc2, k67, qreg[h][3]);
         const float2 f = unpack2(acc2);
         part[h] = f.x + f.y;
       }
@@ -222,49 +228,49 @@ sparse_decode_kernel(const DecodeArgs a) {
       const float s = reduce_scatter<G, S::kSlices>(part, lane, head);
       s_s[head * kBlock + t] = (t < nv) ? s : -INFINITY;
     }
-    __syncthreads();
+    __syncthreads();  // (B) logits ready
 
-    // ---- online softmax per head -------------------------------------------
-#pragma unroll
-    for (int k2 = 0; k2 < 2; ++k2) {
-      const int h = warp + 4 * k2;
-      if (h < G) {
-        const float s0 = s_s[h * kBlock + lane];
-        const float s1 = s_s[h * kBlock + lane + 32];
-        const float mx = warp_max(fmaxf(s0, s1));
-        const float m_new = fmaxf(m_run[k2], mx);
-        float alpha, p0, p1;
-        if (m_new == -INFINITY) {
-          alpha = 1.f;
-          p0 = p1 = 0.f;
-        } else {
-          alpha = hw_exp2(m_run[k2] - m_new);
-          p0 = hw_exp2(s0 - m_new);
-          p1 = hw_exp2(s1 - m_new);
-        }
-        l_run[k2] = l_run[k2] * alpha + warp_sum(p0 + p1);
-        m_run[k2] = m_new;
-        p_s[lane * S::kGP + h] = p0;
-        p_s[(lane + 32) * S::kGP + h] = p1;
-        if (lane == 0) alpha_s[h] = alpha;
+    // ---- online softmax: warp h handles head h ------------------------------
+    if (warp < G) {
+      const int h = warp;
+      const float s0 = s_s[h * kBlock + lane];
+      const float s1 = s_s[h * kBlock + lane + 32];
+      const float mx = warp_max(fmaxf(s0, s1));
+      const float m_new = fmaxf(m_run, mx);
+      float alpha, p0, p1;
+      if (m_new == -INFINITY) {
+        alpha = 1.f;
+        p0 = p1 = 0.f;
+      } else {
+        alpha = hw_exp2(m_run - m_new);
+        p0 = hw_exp2(s0 - m_new);
+        p1 = hw_exp2(s1 - m_new);
       }
+      l_run = l_run * alpha + warp_sum(p0 + p1);
+      m_run = m_new;
+      p_s[lane * S::kGP + h] = p0;
+      p_s[(lane + 32) * S::kGP + h] = p1;
+      if (lane == 0) alpha_s[h] = alpha;
     }
-    __syncthreads();
+    __syncthreads();  // (C) probabilities ready
 
     // ---- accumulate P.V ------------------------------------------------------
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float al = alpha_s[h];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[h][c] *= al;
+      const uint64_t al2 = pack2(make_float2(al, al));
+      uint64_t z01 = 0, z23 = 0;
+      ffma2(z01, acc01[h], al2);
+      ffma2(z23, acc23[h], al2);
+      acc01[h] = z01;
+      acc23[h] = z23;
     }
     const int t0 = tg * S::kTokPerGroup;
     const int t1 = min(t0 + S::kTokPerGroup, nv);
     for (int t = t0; t < t1; ++t) {
       const uint2 w = *reinterpret_cast<const uint2*>(vt + t * D + dg * 4);
-      const float2 v01 = bf16x2_to_float2(w.x);
-      const float2 v23 = bf16x2_to_float2(w.y);
-      const uint64_t pv01 = pack2(v01), pv23 = pack2(v23);
+      const uint64_t v01 = pack2(bf16x2_to_float2(w.x));
+      const uint64_t v23 = pack2(bf16x2_to_float2(w.y));
 #pragma unroll
       for (int h4 = 0; h4 < S::kGP; h4 += 4) {
         const float4 p4 = *reinterpret_cast<const float4*>(p_s + t * S::kGP + h4);
@@ -274,26 +280,23 @@ sparse_decode_kernel(const DecodeArgs a) {
           const int h = h4 + hh;
           if (h < G) {
             const uint64_t p2 = pack2(make_float2(pp[hh], pp[hh]));
-            uint64_t a01 = pack2(make_float2(acc[h][0], acc[h][1]));
-            uint64_t a23 = pack2(make_float2(acc[h][2], acc[h][3]));
-            ffma2(a01, pv01, p2);
-            ffma2(a23, pv23, p2);
-            const float2 r01 = unpack2(a01), r23 = unpack2(a23);
-            acc[h][0] = r01.x; acc[h][1] = r01.y; acc[h][2] = r23.x; acc[h][3] = r23.y;
+            ffma2(acc01[h], v01, p2);
+            ffma2(acc23[h], v23, p2);
           }
         }
       }
     }
-    __syncthreads();  // stage `st` is free again
-    if (tid == 0 && i + kStages < nblk) issue(i + kStages, st);
   }
+  __syncthreads();  // every thread is done with the stages
 
   // ---- split epilogue: write (o, m, l) per head ------------------------------
   float* red = reinterpret_cast<float*>(smem + S::kK);  // [tokgroups][G][D]
 #pragma unroll
-  for (int h = 0; h < G; ++h)
+  for (int h = 0; h < G; ++h) {
+    const float2 r01 = unpack2(acc01[h]), r23 = unpack2(acc23[h]);
     *reinterpret_cast<float4*>(red + (tg * G + h) * D + dg * 4) =
-        make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+        make_float4(r01.x, r01.y, r23.x, r23.y);
+  }
   __syncthreads();
   const int64_t part_row = int64_t(a.part_stride) * (D + 2);
   for (int e = tid; e < G * D; e += kDecThreads) {
@@ -305,15 +308,11 @@ sparse_decode_kernel(const DecodeArgs a) {
                   int64_t(split) * (D + 2);
     prow[dd] = sum;
   }
-#pragma unroll
-  for (int k2 = 0; k2 < 2; ++k2) {
-    const int h = warp + 4 * k2;
-    if (h < G && lane == 0) {
-      float* prow = a.partials + (int64_t(b) * a.hq + kvh * G + h) * part_row +
-                    int64_t(split) * (D + 2);
-      prow[D] = m_run[k2];
-      prow[D + 1] = l_run[k2];
-    }
+  if (warp < G && lane == 0) {
+    float* prow = a.partials + (int64_t(b) * a.hq + kvh * G + warp) * part_row +
+                  int64_t(split) * (D + 2);
+    prow[D] = m_run;
+    prow[D + 1] = l_run;
   }
   __threadfence();
   __syncthreads();
@@ -362,6 +361,30 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int D, int G>
+int occupancy_t() {
+  using S = DecodeShape<D, G>;
+  auto kern = sparse_decode_kernel<D, G>;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes)) !=
+      cudaSuccess)
+    return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecThreads, S::kBytes) !=
+      cudaSuccess)
+    return 1;
+  return n > 0 ? n : 1;
+}
+
+template <int D>
+int occupancy_group(int g) {
+  switch (g) {
+    case 1: return occupancy_t<D, 1>();
+    case 2: return occupancy_t<D, 2>();
+    case 4: return occupancy_t<D, 4>();
+    default: return occupancy_t<D, 8>();
+  }
+}
+
 template <int D>
 cudaError_t dispatch_group(const DecodeArgs& a, cudaStream_t s) {
   switch (a.hq / a.hkv) {
@@ -374,6 +397,10 @@ cudaError_t dispatch_group(const DecodeArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+int decode_ctas_per_sm(int d, int g) {
+  return d == 64 ? occupancy_group<64>(g) : occupancy_group<128>(g);
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);

@@ -11,12 +11,14 @@
 // the local/tail blocks, written in ascending order.
 //
 // Phase 1, grid (chunk, kv-head, batch): each CTA streams the packed stats
-// records of one chunk of candidate blocks with coalesced 128-bit loads.  The
-// d/8 lanes of a block each own an 8-element d-slice of every row and keep the
-// same slice of all G queries in registers (pre-scaled by 1/sqrt d); per row a
-// reduce-scatter leaves one head's dot product per lane, so the linear
-// (row 0) and quadratic (rows 1..r) terms accumulate without further
-// shuffles.  Scores go to the workspace (and to the optional output).
+// records of one chunk of candidate blocks (contiguous in HBM) through a
+// 2-stage shared-memory ring, one bulk async copy (TMA engine) per stage of
+// 256 / (d/8) records.  The d/8 lanes of a block each read a 128-bit slice of
+// every row from shared memory and keep the same slice of all G queries in
+// registers (pre-scaled by 1/sqrt d); per row a reduce-scatter leaves one
+// head's dot product per lane, so the linear (row 0) and quadratic (rows
+// 1..r) terms accumulate without further shuffles.  Scores go to the
+// workspace (and to the optional output).
 //
 // Phase 2, the last CTA of a (batch, kv-head) (atomic ticket, no spinning)
 // finds the k-th largest score with a 4 x 8-bit radix select over
@@ -65,14 +67,6 @@ __device__ __forceinline__ float reduce_scatter_sel(float (&v)[G], int lane, int
   return v[0];
 }
 
-__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
 // Exclusive prefix sum of one value per thread over the CTA (kSelThreads).
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,
                                                          uint32_t& total) {
@@ -114,10 +108,15 @@ select_blocks_kernel(const SelectArgs a) {
   __shared__ uint32_t warp_tot[kSelThreads / 32];
   __shared__ uint32_t sh_u32[4];
   __shared__ int last_s;
+  __shared__ int abort_s;
+  __shared__ __align__(8) uint64_t full[2];
+  extern __shared__ __align__(128) uint8_t stage_smem[];
 
   float* scores = a.scores_ws + int64_t(bh) * a.nb_cap;
 
   // ===================== phase 1: scores of this chunk =====================
+  // The chunk's records are contiguous; kPerPass of them at a time are staged
+  // in shared memory by one bulk async copy (2-stage ring, mbarrier-tracked).
   {
     const int slice = lane % kLanes;
     const float inv_sqrt_d = rsqrtf(float(D));
@@ -138,18 +137,49 @@ select_blocks_kernel(const SelectArgs a) {
     const float ln_n = logf(float(kBlock));
     const int c_lo = a.cand_begin + chunk * a.chunk_blocks;
     const int c_hi = min(a.cand_end, c_lo + a.chunk_blocks);
-    const int64_t rec_elems = int64_t(rows) * D;
-    for (int base = c_lo; base < c_hi; base += kPerPass) {
-      const int j = base + tid / kLanes;
+    const int rec_elems = rows * D;
+    const int stage_elems = kPerPass * rec_elems;
+    uint16_t* stage = reinterpret_cast<uint16_t*>(stage_smem);
+    const int npass = c_hi > c_lo ? (c_hi - c_lo + kPerPass - 1) / kPerPass : 0;
+    const uint16_t* src = a.stats + int64_t(bh) * a.nb_cap * rec_elems;
+
+    if (tid == 0) {
+      mbar_init(&full[0], 1);
+      mbar_init(&full[1], 1);
+      fence_barrier_init();
+      abort_s = 0;
+    }
+    __syncthreads();
+    auto issue = [&](int p) {  // thread 0 only
+      const int j0 = c_lo + p * kPerPass;
+      const int nb = min(kPerPass, c_hi - j0);
+      const uint32_t bytes = uint32_t(nb) * uint32_t(rec_elems) * 2u;
+      mbar_arrive_expect_tx(&full[p & 1], bytes);
+      bulk_g2s(stage + (p & 1) * stage_elems, src + int64_t(j0) * rec_elems, bytes, &full[p & 1]);
+    };
+    if (tid == 0) {
+      for (int p = 0; p < 2 && p < npass; ++p) issue(p);
+    }
+    for (int p = 0; p < npass; ++p) {
+      const uint32_t parity = (p >> 1) & 1;
+      if (tid == 0) {
+        if (!mbar_wait_bounded(&full[p & 1], parity, a.status)) {
+          abort_s = 1;
+          if (p + 1 < npass) mbar_wait_bounded(&full[(p + 1) & 1], ((p + 1) >> 1) & 1, a.status);
+        }
+      }
+      __syncthreads();
+      if (abort_s) break;
+      if (tid != 0) (void)mbar_try_wait(&full[p & 1], parity);  // acquire the copy
+      const int jj = tid / kLanes;
+      const int j = c_lo + p * kPerPass + jj;
       const bool valid = j < c_hi;
-      const uint16_t* rec = a.stats + (int64_t(bh) * a.nb_cap + (valid ? j : c_lo)) * rec_elems +
-                            slice * 8;
-      // issue every row load of this block up front
+      const uint16_t* rec = stage + (p & 1) * stage_elems + jj * rec_elems + slice * 8;
       uint4 w[RMAX + 1];
 #pragma unroll
       for (int r = 0; r <= RMAX; ++r) {
         w[r] = make_uint4(0, 0, 0, 0);
-        if (r < rows && valid) w[r] = ld_stream(rec + int64_t(r) * D);
+        if (r < rows && valid) w[r] = *reinterpret_cast<const uint4*>(rec + r * D);
       }
       float s = 0.f;
       int head = 0;
@@ -187,6 +217,8 @@ select_blocks_kernel(const SelectArgs a) {
         scores[j] = S;
         if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j] = S;
       }
+      __syncthreads();  // stage (p & 1) consumed
+      if (tid == 0 && p + 2 < npass) issue(p + 2);
     }
   }
 
@@ -301,9 +333,35 @@ select_blocks_kernel(const SelectArgs a) {
 
 template <int D, int G, int R>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
+  auto kern = select_blocks_kernel<D, G, R>;
+  const size_t smem = select_stage_bytes(a.d, a.rank);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.hkv, a.batch);
-  select_blocks_kernel<D, G, R><<<grid, kSelThreads, 0, s>>>(a);
+  kern<<<grid, kSelThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int G, int R>
+int occupancy_t(int rank) {
+  int n = 0;
+  auto kern = select_blocks_kernel<D, G, R>;
+  const size_t smem = select_stage_bytes(D, rank);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kSelThreads, smem) != cudaSuccess)
+    return 1;
+  return n > 0 ? n : 1;
+}
+
+template <int D, int G>
+int occupancy_rank(int rank) {
+  if (rank == 0) return occupancy_t<D, G, 0>(rank);
+  if (rank <= 4) return occupancy_t<D, G, 4>(rank);
+  if (rank <= 8) return occupancy_t<D, G, 8>(rank);
+  return occupancy_t<D, G, 16>(rank);
 }
 
 template <int D, int G>
@@ -325,7 +383,25 @@ cudaError_t dispatch_group(const SelectArgs& a, cudaStream_t s) {
   }
 }
 
+template <int D>
+int occupancy_group(int g, int rank) {
+  switch (g) {
+    case 1: return occupancy_rank<D, 1>(rank);
+    case 2: return occupancy_rank<D, 2>(rank);
+    case 4: return occupancy_rank<D, 4>(rank);
+    default: return occupancy_rank<D, 8>(rank);
+  }
+}
+
 }  // namespace
+
+size_t select_stage_bytes(int d, int rank) {
+  return size_t(2) * (kSelThreads / (d / 8)) * size_t(1 + rank) * d * 2;
+}
+
+int select_ctas_per_sm(int d, int g, int rank) {
+  return d == 64 ? occupancy_group<64>(g, rank) : occupancy_group<128>(g, rank);
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);

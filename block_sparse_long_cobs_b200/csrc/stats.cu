@@ -10,28 +10,30 @@
 // covariance, computed through the n x n Gram matrix because n = B = 64 < d):
 //   1. Raw Gram G = K K^T of the block's bf16 keys on the 5th-generation tensor
 //      cores: one tcgen05.mma chain (kind::f16, bf16 in, fp32 accumulate in
-//      tensor memory) computes the 128 x 128 Gram of two consecutive blocks
-//      stacked along M; the two diagonal 64 x 64 quadrants are the blocks'
-//      Grams.  Products of bf16 values are exact, so no precision is lost
+//      tensor memory) computes the 128 x 128 Gram of two blocks stacked along
+//      M (consecutive work items, possibly of different (batch, kv-head)
+//      pairs); the two diagonal 64 x 64 quadrants are the blocks' Grams.  Products of bf16 values are exact, so no precision is lost
 //      before the fp32 accumulation.  The keys arrive by TMA (2-d tensor map,
 //      128-byte swizzle = the UMMA K-major canonical layout).
 //   2. Centring in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
-//      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T.
-//   3. Lanczos tridiagonalisation of Gc (64 steps, every new vector
-//      re-orthogonalised twice against all earlier ones by classical
-//      Gram-Schmidt, so the basis Q stays orthogonal to fp32 accuracy and
-//      T = Q^T Gc Q is similar to Gc); a fresh pseudo-random start vector
+//      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T; then
+//      A = Gc^2 (same eigenvectors, squared eigenvalues: the top of the
+//      spectrum separates faster, so fewer Lanczos steps are needed).
+//   3. Lanczos tridiagonalisation of A, m = 28 / 36 / 52 steps for r <= 4 /
+//      <= 8 / <= 16 (at least 2 r + 20), every new
+//      vector re-orthogonalised twice against all earlier ones by classical
+//      Gram-Schmidt (basis kept row- and column-major in shared memory so both
+//      Gram-Schmidt phases are 128-bit loads), a fresh pseudo-random vector
 //      whenever the Krylov space closes.  128 threads per block, each holding
-//      32 entries of Gc in registers; named barriers between the phases.
-//   4. Top-r eigenvalues of the tridiagonal T by multisection bisection on
-//      Sturm counts (8 threads per eigenvalue, 10 rounds of 9-way splits),
-//      their eigenvectors z_k by inverse iteration (LDL^T of T - lambda I),
-//      re-orthogonalised inside clusters of close eigenvalues; Ritz vectors
-//      w_k = Q z_k are unit eigenvectors of Gc with eigenvalue lambda_k
-//      (= n times the covariance eigenvalue).
-//   5. U[:, k] = Kc^T w_k / sqrt(n) (squared norm lambda_k / n), sign fixed
-//      so that the largest-magnitude component is positive; written with mu
-//      as bf16.
+//      32 entries of A in registers; five named-barrier phases per step.
+//   4. Top-r eigenvalues of the m x m tridiagonal T by multisection bisection
+//      on Sturm counts (8 threads x 3 shifts per eigenvalue, 25-way splits),
+//      eigenvectors z_k by inverse iteration (LDL^T of T - theta I, vector in
+//      registers), re-orthogonalised inside clusters of close eigenvalues;
+//      Ritz vectors w_k = Q z_k are unit eigenvectors of Gc.
+//   5. U[:, k] = Kc^T w_k / sqrt(n) (its squared norm is the covariance
+//      eigenvalue), sign fixed so that the largest-magnitude component is
+//      positive; written with mu as bf16.
 #include <cfloat>
 #include <cuda.h>
 
@@ -41,24 +43,30 @@ namespace cobs {
 namespace {
 
 constexpr int kStatThreads = 256;   // 2 blocks x 128 threads
-constexpr int kQStride = 72;        // floats per Lanczos vector: halves of 36
-constexpr int kGcStride = 65;       // padded row of the centred Gram (staging)
-constexpr int kBisectRounds = 10;
-constexpr int kInverseIters = 3;
+constexpr int kQStride = 72;        // floats per basis row: halves of 36
+constexpr int kGStride = 68;        // 16-byte aligned row of the staged Grams
+constexpr int kBisectRounds = 5;   // 25-way splits: 25^5 ~ 1e7
+constexpr int kInverseIters = 2;
+
+// Lanczos length by rank bucket: m = 2 r + 20 for the largest r of the bucket
+__host__ __device__ constexpr int lanczos_steps(int rank) {
+  return rank <= 4 ? 28 : (rank <= 8 ? 36 : 52);
+}
 
 template <int D>
 struct StatsShape {
   static constexpr int kRegions = D / 64;           // 128-byte-wide column slabs
   static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B
   // per-block regions (x2)
-  static constexpr size_t kQBytes = 64 * kQStride * 4;        // Q, also Gc staging
+  static constexpr size_t kQBytes = 64 * kQStride * 4;        // Q rows; G^2 staging
   static constexpr size_t kZBytes = kMaxRank * 64 * 4;        // eigenvectors of T
   static constexpr size_t kWBytes = 64 * kMaxRank * 4;        // Ritz vectors [t][k]
   static constexpr size_t kScrBytes = kMaxRank * 2 * 64 * 4;  // inverse iteration
   static constexpr size_t kVecBytes = 2048;                   // small vectors
   static constexpr size_t kK = 0;                             // [regions][128][128 B]
   static constexpr size_t kQ = kK + size_t(kRegions) * kRegionBytes;
-  static constexpr size_t kZ = kQ + 2 * kQBytes;
+  static constexpr size_t kQT = kQ + 2 * kQBytes;             // Q^T rows; Gc staging
+  static constexpr size_t kZ = kQT + 2 * kQBytes;
   static constexpr size_t kW = kZ + 2 * kZBytes;
   static constexpr size_t kScr = kW + 2 * kWBytes;
   static constexpr size_t kVec = kScr + 2 * kScrBytes;
@@ -68,18 +76,17 @@ struct StatsShape {
   static constexpr size_t kBar = kFlip + 2 * 4 * kMaxRank * 8;
   static constexpr size_t kMisc = kBar + 16;
   static constexpr size_t kBytes = kMisc + 16 + 1024;  // + alignment slack
-  static_assert(64 * kGcStride * 4 <= kQBytes, "Gc staging must fit in Q");
+  static_assert(64 * kGStride * 4 <= kQBytes, "Gram staging must fit in a basis region");
 };
 
 // Offsets inside the per-block small-vector area (floats).
 constexpr int kVW = 0;        // w, split layout [2][36]
-constexpr int kVH = 72;       // CGS coefficients h [64]
-constexpr int kVRed = 136;    // reduction partials [8]
-constexpr int kVAlpha = 144;  // T diagonal [64]
-constexpr int kVBeta2 = 208;  // T off-diagonal squared [64]
-constexpr int kVBeta = 272;   // T off-diagonal [64]
-constexpr int kVLam = 336;    // eigenvalues (descending) [16]
-constexpr int kVTrace = 352;  // trace of Gc [1]
+constexpr int kVH = 72;       // Gram-Schmidt coefficients h, split layout [2][36]
+constexpr int kVRed = 144;    // reduction partials [4] + norm partials [4]
+constexpr int kVAlpha = 152;  // T diagonal [64]
+constexpr int kVBeta2 = 216;  // T off-diagonal squared [64]
+constexpr int kVBeta = 280;   // T off-diagonal [64]
+constexpr int kVLam = 344;    // eigenvalues of T (descending) [16]
 
 __device__ __forceinline__ float hash_sign(uint32_t a, uint32_t b) {
   uint32_t h = a * 0x9E3779B1u ^ (b + 0x7F4A7C15u) * 0x85EBCA77u;
@@ -89,19 +96,33 @@ __device__ __forceinline__ float hash_sign(uint32_t a, uint32_t b) {
   return (h & 1u) ? 1.f : -1.f;
 }
 
-// Number of eigenvalues of the tridiagonal T (diag alpha, off-diag^2 beta2)
-// below x: count of negative pivots of the LDL^T factorisation of T - x I.
-__device__ __forceinline__ int sturm_count(const float* alpha, const float* beta2, float x) {
-  int cnt = 0;
-  float d = alpha[0] - x;
-  cnt += d < 0.f;
-#pragma unroll 8
-  for (int i = 1; i < 64; ++i) {
-    const float dd = fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
-    d = alpha[i] - x - beta2[i - 1] / dd;
-    cnt += d < 0.f;
+// split layout: element e of a 64-vector sits at (e & 1) * 36 + (e >> 1)
+__device__ __forceinline__ int qidx(int e) { return (e & 1) * 36 + (e >> 1); }
+
+__device__ __forceinline__ float pivot_guard(float d) {
+  return fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
+}
+
+// Numbers of eigenvalues of the M x M tridiagonal T (diag al, off-diag^2 b2,
+// both in registers) below three shifts: negative pivots of LDL^T of T - x I,
+// the three recurrences interleaved so their latencies overlap.
+template <int M>
+__device__ __forceinline__ void sturm_count3(const float (&al)[M], const float (&b2)[M],
+                                             const float (&x)[3], int (&c)[3]) {
+  float d[3];
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    d[s] = al[0] - x[s];
+    c[s] = d[s] < 0.f;
   }
-  return cnt;
+#pragma unroll
+  for (int i = 1; i < M; ++i) {
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+      d[s] = al[i] - x[s] - __fdividef(b2[i - 1], pivot_guard(d[s]));
+      c[s] += d[s] < 0.f;
+    }
+  }
 }
 
 // ---- tcgen05 / TMA wrappers ---------------------------------------------------
@@ -201,7 +222,7 @@ __device__ __forceinline__ uint32_t k_offset(int row, int col) {
                   ((((c >> 3) ^ (row & 7))) << 4) + ((c & 7) << 1));
 }
 
-template <int D>
+template <int D, int M>
 __global__ void __launch_bounds__(kStatThreads)
 block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) {
   using S = StatsShape<D>;
@@ -218,18 +239,29 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   uint32_t* abort_s = misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kvh = blockIdx.y, b = blockIdx.z;
-  const int64_t bh = int64_t(b) * a.hkv + kvh;
-  const int64_t j0 = a.block_begin + 2 * int64_t(blockIdx.x);
-  const bool has1 = j0 + 1 < a.block_end;
+  // work items (bh, j) for every (batch, kv-head) pair and every block in
+  // [block_begin, block_end), two per CTA (they need not share a pair)
+  const int64_t nb_range = a.block_end - a.block_begin;
+  const int64_t n_items = int64_t(a.batch) * a.hkv * nb_range;
+  const int64_t item0 = 2 * int64_t(blockIdx.x);
+  const bool has1 = item0 + 1 < n_items;
+  int64_t item_bh[2], item_j[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int64_t it = (q == 0 || has1) ? item0 + q : item0;
+    item_bh[q] = it / nb_range;
+    item_j[q] = a.block_begin + it % nb_range;
+  }
   const int blk = tid >> 7;            // block of the pair this thread serves
   const int bt = tid & 127;            // thread index inside that block's team
   const int bwarp = bt >> 5;           // warp index inside the team
   const bool my_valid = blk == 0 || has1;
   const int r = a.rank;
   const int bar_id = 1 + blk;
+  constexpr int msteps = M;                 // Lanczos steps
 
   float* Qs = reinterpret_cast<float*>(smem + S::kQ + blk * S::kQBytes);
+  float* QTs = reinterpret_cast<float*>(smem + S::kQT + blk * S::kQBytes);
   float* Zs = reinterpret_cast<float*>(smem + S::kZ + blk * S::kZBytes);
   float* Ws = reinterpret_cast<float*>(smem + S::kW + blk * S::kWBytes);
   float* Scr = reinterpret_cast<float*>(smem + S::kScr + blk * S::kScrBytes);
@@ -253,7 +285,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     const int nblk = has1 ? 2 : 1;
     mbar_arrive_expect_tx(&bars[0], uint32_t(nblk) * kBlock * D * 2);
     for (int q = 0; q < nblk; ++q) {
-      const int y = int((bh * a.cap) + (j0 + q) * kBlock);
+      const int y = int(item_bh[q] * a.cap + item_j[q] * kBlock);
       for (int reg = 0; reg < S::kRegions; ++reg)
         tma_load_2d(ktile + reg * S::kRegionBytes + q * kBlock * 128, &kmap, reg * 64, y,
                     &bars[0]);
@@ -307,10 +339,12 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     for (int c = 0; c < 64; ++c) ssum += row_mean[rb * 64 + c];
     const float smean = ssum * (1.f / 64.f);
     const float rm = row_mean[tid];
-    float* stage = reinterpret_cast<float*>(smem + S::kQ + rb * S::kQBytes);
+    // Gc is symmetric: row ri is stored as column ri (consecutive lanes ->
+    // consecutive addresses)
+    float* stage = reinterpret_cast<float*>(smem + S::kQT + rb * S::kQBytes);
 #pragma unroll
     for (int c = 0; c < 64; ++c)
-      stage[ri * kGcStride + c] = g[c] - rm - row_mean[rb * 64 + c] + smean;
+      stage[c * kGStride + ri] = g[c] - rm - row_mean[rb * 64 + c] + smean;
   }
 
   // block mean (fp32 sum of 64 bf16 keys): thread bt < D owns dim bt
@@ -325,186 +359,279 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   }
   __syncthreads();
 
-  // ---- 3. Lanczos with full re-orthogonalisation -----------------------------
-  // Thread (i, hh) = (bt >> 1, bt & 1) owns Gram row i, columns 2k + hh.
-  const int li = bt >> 1, hh = bt & 1;
-  float gr[32];
-  {
-    const float* stage = Qs;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) gr[k] = stage[li * kGcStride + 2 * k + hh];
-  }
-  float trace_part = (hh == (li & 1)) ? gr[li >> 1] : 0.f;   // diagonal entry once
-  named_bar(bar_id, 128);                  // staging area becomes Q
-
   const bool do_eig = r > 0 && my_valid;
+  const int li = bt >> 1, hh = bt & 1;
   auto block_sum = [&](float v) -> float {  // sum over the 128 threads of the team
     v = warp_sum(v);
     if (lane == 0) V[kVRed + bwarp] = v;
     named_bar(bar_id, 128);
-    const float s = (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
-    return s;
+    return (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
   };
-  // split layout: element e of a 64-vector sits at (e & 1) * 36 + (e >> 1)
-  auto qidx = [](int e) { return (e & 1) * 36 + (e >> 1); };
 
   if (do_eig) {
+    // ---- 3a. A = Gc * Gc (4 x 8 register tile per thread) ----------------------
+    {
+      const float* gcs = QTs;           // Gc staging, stride kGStride
+      float* a2 = Qs;                   // A staging, stride kGStride
+      const int rg = bt >> 3, cg = bt & 7;
+      float acc[4][8];
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 8; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < 64; ++k) {
+        const float4 av = *reinterpret_cast<const float4*>(gcs + k * kGStride + 4 * rg);
+        const float4 b0 = *reinterpret_cast<const float4*>(gcs + k * kGStride + 8 * cg);
+        const float4 b1 = *reinterpret_cast<const float4*>(gcs + k * kGStride + 8 * cg + 4);
+        const float ar[4] = {av.x, av.y, av.z, av.w};
+        const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(ar[x], br[y], acc[x][y]);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        float* row = a2 + (4 * rg + x) * kGStride + 8 * cg;
+        *reinterpret_cast<float4*>(row) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
+        *reinterpret_cast<float4*>(row + 4) =
+            make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
+      }
+    }
+    named_bar(bar_id, 128);
+    // thread (li, hh) owns row li of A, columns 2k + hh
+    float gr[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) gr[k] = Qs[li * kGStride + 2 * k + hh];
+    const float trace_part = (hh == (li & 1)) ? gr[li >> 1] : 0.f;   // diagonal once
     const float trace = block_sum(trace_part);
     const float tol = 1e-5f * trace;
-    named_bar(bar_id, 128);                 // everyone read the partials
-    if (hh == 0) Qs[qidx(li)] = hash_sign(7u, uint32_t(li)) * 0.125f;
+    named_bar(bar_id, 128);                 // partials read, staging consumed
+    for (int e = bt; e < 64 * kQStride; e += 128) {
+      Qs[e] = 0.f;
+      QTs[e] = 0.f;
+    }
+    for (int e = bt; e < 144; e += 128) V[kVW + e] = 0.f;   // w and h
+    named_bar(bar_id, 128);
+    if (hh == 0) {
+      const float v0 = hash_sign(7u, uint32_t(li)) * 0.125f;
+      Qs[qidx(li)] = v0;
+      QTs[li * kQStride + qidx(0)] = v0;
+    }
     named_bar(bar_id, 128);
 
-    // orthogonalise w (this thread's entry wi for row li) against Q[0..jmax]
-    auto cgs = [&](float& wi, int jmax, bool want_alpha, int jalpha) -> float {
+    // Orthogonalise w (this thread's entry wi of row li) against Q[0..jmax],
+    // twice.  Returns the summed coefficient of q_jmax; sq receives |w|^2
+    // after the first pass minus |h|^2 of the second (= |w|^2 at the end).
+    auto cgs = [&](float& wi, int jmax, float& sq) -> float {
       float acoef = 0.f;
+      const int nc = ((jmax >> 1) >> 2) + 1;   // 4-wide chunks per parity
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
         if (hh == 0) V[kVW + qidx(li)] = wi;
+        if (pass == 1) {   // |w|^2 after the first pass: warp partials
+          const float ps = warp_sum(hh == 0 ? wi * wi : 0.f);
+          if (lane == 0) V[kVRed + 4 + bwarp] = ps;
+        }
         named_bar(bar_id, 128);
+        if (pass == 1)
+          sq = (V[kVRed + 4] + V[kVRed + 5]) + (V[kVRed + 6] + V[kVRed + 7]);
         float hp = 0.f;
         if (li <= jmax) {
           const float4* qm = reinterpret_cast<const float4*>(Qs + li * kQStride + hh * 36);
           const float4* ws = reinterpret_cast<const float4*>(V + kVW + hh * 36);
+          float h0 = 0.f, h1 = 0.f, h2 = 0.f, h3 = 0.f;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             const float4 x = qm[k], y = ws[k];
-            hp = fmaf(x.x, y.x, hp);
-            hp = fmaf(x.y, y.y, hp);
-            hp = fmaf(x.z, y.z, hp);
-            hp = fmaf(x.w, y.w, hp);
+            h0 = fmaf(x.x, y.x, h0);
+            h1 = fmaf(x.y, y.y, h1);
+            h2 = fmaf(x.z, y.z, h2);
+            h3 = fmaf(x.w, y.w, h3);
           }
+          hp = (h0 + h1) + (h2 + h3);
         }
         hp += __shfl_xor_sync(0xffffffffu, hp, 1);
-        if (hh == 0) V[kVH + li] = hp;
+        if (hh == 0) V[kVH + qidx(li)] = hp;       // zero for li > jmax
+        if (pass == 1) {   // |h|^2 of the second pass: warp partials
+          const float ph = warp_sum(hh == 0 ? hp * hp : 0.f);
+          if (lane == 0) V[kVRed + bwarp] = ph;
+        }
         named_bar(bar_id, 128);
-        float corr = 0.f;
-        const int col = qidx(li);
-        for (int m = hh; m <= jmax; m += 2) corr = fmaf(Qs[m * kQStride + col], V[kVH + m], corr);
+        // w_i -= sum_m Q[m][i] h_m over m of this thread's parity
+        const float4* qt = reinterpret_cast<const float4*>(QTs + li * kQStride + hh * 36);
+        const float4* hv = reinterpret_cast<const float4*>(V + kVH + hh * 36);
+        float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+        constexpr int kMaxChunks = ((M - 1) / 2) / 4 + 1;
+#pragma unroll
+        for (int c = 0; c < kMaxChunks; ++c) {
+          if (c < nc) {
+            const float4 x = qt[c], y = hv[c];
+            c0 = fmaf(x.x, y.x, c0);
+            c1 = fmaf(x.y, y.y, c1);
+            c2 = fmaf(x.z, y.z, c2);
+            c3 = fmaf(x.w, y.w, c3);
+          }
+        }
+        float corr = (c0 + c1) + (c2 + c3);
         corr += __shfl_xor_sync(0xffffffffu, corr, 1);
         wi -= corr;
-        if (want_alpha) acoef += V[kVH + jalpha];
+        acoef += V[kVH + qidx(jmax)];
+        if (pass == 1) {
+          const float s0 = (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
+          sq = fmaxf(sq - s0, 0.f);
+        }
       }
       return acoef;
     };
 
 #pragma unroll 1
-    for (int j = 0; j < 64; ++j) {
-      // w = Gc q_j
+    for (int j = 0; j < msteps; ++j) {
+      // w = A q_j
       const float4* qj = reinterpret_cast<const float4*>(Qs + j * kQStride + hh * 36);
-      float p = 0.f;
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 x = qj[k];
-        p = fmaf(gr[4 * k + 0], x.x, p);
-        p = fmaf(gr[4 * k + 1], x.y, p);
-        p = fmaf(gr[4 * k + 2], x.z, p);
-        p = fmaf(gr[4 * k + 3], x.w, p);
+        p0 = fmaf(gr[4 * k + 0], x.x, p0);
+        p1 = fmaf(gr[4 * k + 1], x.y, p1);
+        p2 = fmaf(gr[4 * k + 2], x.z, p2);
+        p3 = fmaf(gr[4 * k + 3], x.w, p3);
       }
+      const float p = (p0 + p1) + (p2 + p3);
       float wi = p + __shfl_xor_sync(0xffffffffu, p, 1);
-      const float aj = cgs(wi, j, true, j);
-      float beta = sqrtf(block_sum(hh == 0 ? wi * wi : 0.f));
+      float sq = 0.f;
+      const float aj = cgs(wi, j, sq);
+      float beta = sqrtf(sq);
       if (bt == 0) V[kVAlpha + j] = aj;
-      if (j == 63) break;
+      if (j == msteps - 1) break;
       if (!(beta > tol)) {
         // the Krylov space closed: continue from a fresh vector
         wi = hash_sign(uint32_t(j + 1), uint32_t(li));
         named_bar(bar_id, 128);
-        cgs(wi, j, false, 0);
-        const float nrm = sqrtf(block_sum(hh == 0 ? wi * wi : 0.f));
+        float sq2 = 0.f;
+        cgs(wi, j, sq2);
+        const float nrm = sqrtf(sq2);
         wi = nrm > 0.f ? wi / nrm : 0.f;
         beta = 0.f;
       } else {
-        wi = wi / beta;
+        wi = wi * (1.f / beta);
       }
       if (bt == 0) {
         V[kVBeta + j] = beta;
         V[kVBeta2 + j] = beta * beta;
       }
-      if (hh == 0) Qs[(j + 1) * kQStride + qidx(li)] = wi;
+      if (hh == 0) {
+        Qs[(j + 1) * kQStride + qidx(li)] = wi;
+        QTs[li * kQStride + qidx(j + 1)] = wi;
+      }
       named_bar(bar_id, 128);
     }
     named_bar(bar_id, 128);
 
-    // ---- 4. top-r eigenpairs of T -----------------------------------------
+    // ---- 4. top-r eigenpairs of T ---------------------------------------------
+    constexpr int m = msteps;
     const float* alpha = V + kVAlpha;
-    const float* beta2 = V + kVBeta2;
     const float* betav = V + kVBeta;
+    float al[m], b2[m];
+#pragma unroll
+    for (int i2 = 0; i2 < m; ++i2) {
+      al[i2] = alpha[i2];
+      b2[i2] = V[kVBeta2 + i2];
+    }
     float lo = 0.f, hi = 0.f;
-    for (int i2 = 0; i2 < 64; ++i2) {
-      const float rad = (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < 63 ? fabsf(betav[i2]) : 0.f);
-      lo = fminf(lo, alpha[i2] - rad);
-      hi = fmaxf(hi, alpha[i2] + rad);
+#pragma unroll
+    for (int i2 = 0; i2 < m; ++i2) {
+      const float rad =
+          (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < m - 1 ? fabsf(betav[i2]) : 0.f);
+      lo = fminf(lo, al[i2] - rad);
+      hi = fmaxf(hi, al[i2] + rad);
     }
     hi = hi * (1.f + 1e-6f) + 1e-30f;
     lo = lo - 1e-6f * fabsf(hi) - 1e-30f;
-    const int grp = bt >> 3, sub = bt & 7;   // 8 threads per eigenvalue
+    const int grp = bt >> 3, sub = bt & 7;   // 8 threads x 3 shifts per eigenvalue
     const int kk = grp;                      // k-th largest
-    const int target = 63 - kk;              // count(x) <= target below it
+    const int target = m - 1 - kk;           // count(x) <= target below it
     float ea = lo, eb = hi;
     for (int it = 0; it < kBisectRounds; ++it) {
-      const float step = (eb - ea) * (1.f / 9.f);
-      const float x = ea + step * float(sub + 1);
-      const bool above = sturm_count(alpha, beta2, x) > target;
-      const uint32_t bal = __ballot_sync(0xffffffffu, above);
-      const uint32_t mine = (bal >> ((lane >> 3) << 3)) & 0xffu;
-      const int first = mine ? __ffs(mine) - 1 : 8;   // first point above the eigenvalue
+      const float step = (eb - ea) * (1.f / 25.f);
+      float xs[3];
+      int cs[3];
+#pragma unroll
+      for (int s2 = 0; s2 < 3; ++s2) xs[s2] = ea + step * float(3 * sub + s2 + 1);
+      sturm_count3<m>(al, b2, xs, cs);
+      const int sh = (lane >> 3) << 3;
+      uint32_t mask24 = 0;
+#pragma unroll
+      for (int s2 = 0; s2 < 3; ++s2) {
+        const uint32_t bal = (__ballot_sync(0xffffffffu, cs[s2] > target) >> sh) & 0xffu;
+        // point 3u + s2 + 1 of lane u in the group -> bit 3u + s2
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mask24 |= ((bal >> u) & 1u) << (3 * u + s2);
+      }
+      const int first = mask24 ? __ffs(mask24) - 1 : 24;   // first point above
       const float na = first == 0 ? ea : ea + step * float(first);
-      const float nb = first == 8 ? eb : ea + step * float(first + 1);
+      const float nb = first == 24 ? eb : ea + step * float(first + 1);
       ea = na;
       eb = nb;
     }
-    const float lam = 0.5f * (ea + eb);
-    if (sub == 0 && kk < r) V[kVLam + kk] = lam;
+    const float theta = 0.5f * (ea + eb);
+    if (sub == 0 && kk < r) V[kVLam + kk] = theta;
     named_bar(bar_id, 128);
 
-    // inverse iteration, one thread per eigenvalue: (T - lam I) z = y via LDL^T
+    // inverse iteration, one thread per eigenvalue: (T - theta I) z = y, LDL^T
     if (sub == 0 && kk < r) {
-      float* zk = Zs + kk * 64;
-      float* dl = Scr + kk * 128;       // [0,64): l_i ; [64,128): d_i
-      float nrm2 = 0.f;
-      for (int i2 = 0; i2 < 64; ++i2) {
-        zk[i2] = 1.f + 0.25f * hash_sign(uint32_t(kk + 101), uint32_t(i2));
-      }
-      // factorisation (once)
+      float l[m], rd[m];
       {
-        float d = alpha[0] - lam;
-        d = fabsf(d) < 1e-30f ? 1e-30f : d;
-        dl[64] = d;
-        for (int i2 = 1; i2 < 64; ++i2) {
-          const float l = betav[i2 - 1] / d;
-          d = alpha[i2] - lam - l * betav[i2 - 1];
-          d = fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
-          dl[i2] = l;
-          dl[64 + i2] = d;
+        float d = pivot_guard(al[0] - theta);
+        rd[0] = 1.f / d;
+        l[0] = 0.f;
+#pragma unroll
+        for (int i2 = 1; i2 < m; ++i2) {
+          l[i2] = betav[i2 - 1] * rd[i2 - 1];
+          d = pivot_guard(al[i2] - theta - l[i2] * betav[i2 - 1]);
+          rd[i2] = 1.f / d;
         }
       }
+      float z[m];
+#pragma unroll
+      for (int i2 = 0; i2 < m; ++i2)
+        z[i2] = 1.f + 0.25f * hash_sign(uint32_t(kk + 101), uint32_t(i2));
+      float nrm2 = 1.f;
+#pragma unroll
       for (int it = 0; it < kInverseIters; ++it) {
-        for (int i2 = 1; i2 < 64; ++i2) zk[i2] -= dl[i2] * zk[i2 - 1];
-        for (int i2 = 0; i2 < 64; ++i2) zk[i2] /= dl[64 + i2];
-        for (int i2 = 62; i2 >= 0; --i2) zk[i2] -= dl[i2 + 1] * zk[i2 + 1];
+#pragma unroll
+        for (int i2 = 1; i2 < m; ++i2) z[i2] = fmaf(-l[i2], z[i2 - 1], z[i2]);
+#pragma unroll
+        for (int i2 = 0; i2 < m; ++i2) z[i2] *= rd[i2];
+#pragma unroll
+        for (int i2 = m - 2; i2 >= 0; --i2) z[i2] = fmaf(-l[i2 + 1], z[i2 + 1], z[i2]);
         float mx = 0.f;
-        for (int i2 = 0; i2 < 64; ++i2) mx = fmaxf(mx, fabsf(zk[i2]));
+#pragma unroll
+        for (int i2 = 0; i2 < m; ++i2) mx = fmaxf(mx, fabsf(z[i2]));
         const float inv = mx > 0.f ? 1.f / mx : 1.f;
         nrm2 = 0.f;
-        for (int i2 = 0; i2 < 64; ++i2) {
-          zk[i2] *= inv;
-          nrm2 += zk[i2] * zk[i2];
+#pragma unroll
+        for (int i2 = 0; i2 < m; ++i2) {
+          z[i2] *= inv;
+          nrm2 = fmaf(z[i2], z[i2], nrm2);
         }
       }
       const float inv = rsqrtf(fmaxf(nrm2, 1e-30f));
-      for (int i2 = 0; i2 < 64; ++i2) zk[i2] *= inv;
+#pragma unroll
+      for (int i2 = 0; i2 < 64; ++i2) Zs[kk * 64 + i2] = i2 < m ? z[i2] * inv : 0.f;
     }
     named_bar(bar_id, 128);
     // re-orthogonalise inside clusters of close eigenvalues (warp 0 of the team)
     if (bwarp == 0) {
-      const float lam0 = V[kVLam + 0];
+      const float th0 = V[kVLam + 0];
       for (int k2 = 1; k2 < r; ++k2) {
-        const float lk = V[kVLam + k2];
+        const float tk = V[kVLam + k2];
         float* zk = Zs + k2 * 64;
         bool touched = false;
         for (int l2 = 0; l2 < k2; ++l2) {
-          if (fabsf(V[kVLam + l2] - lk) > 1e-3f * fabsf(lam0)) continue;
+          if (fabsf(V[kVLam + l2] - tk) > 1e-3f * fabsf(th0)) continue;
           const float* zl = Zs + l2 * 64;
           const float c = warp_sum(zl[lane] * zk[lane] + zl[lane + 32] * zk[lane + 32]);
           zk[lane] -= c * zl[lane];
@@ -522,27 +649,28 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       }
     }
     named_bar(bar_id, 128);
-    // Ritz vectors w_k = Q z_k, stored [t][k]; thread (t = li, hh) takes k = hh, hh+2, ...
+    // Ritz vectors w_k = Q z_k stored [t][k]; thread (t = li, hh) takes
+    // k = hh, hh + 2, ...; eigenvalues below 1e-12 of the largest (of A = Gc^2)
+    // are treated as zero
     {
-      const int col = qidx(li);
       float acc[kMaxRank / 2];
 #pragma unroll
       for (int k2 = 0; k2 < kMaxRank / 2; ++k2) acc[k2] = 0.f;
-      for (int m = 0; m < 64; ++m) {
-        const float qv = Qs[m * kQStride + col];
+      for (int mm = 0; mm < m; ++mm) {
+        const float qv = QTs[li * kQStride + qidx(mm)];
 #pragma unroll
         for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
           const int k = 2 * k2 + hh;
-          if (k < r) acc[k2] = fmaf(qv, Zs[k * 64 + m], acc[k2]);
+          if (k < r) acc[k2] = fmaf(qv, Zs[k * 64 + mm], acc[k2]);
         }
       }
-      const float lam0 = V[kVLam + 0];
+      const float th0 = V[kVLam + 0];
 #pragma unroll
       for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
         const int k = 2 * k2 + hh;
         if (k < r) {
-          const float lk = V[kVLam + k];
-          const bool keep = lk > 1e-6f * lam0 && lk > 0.f;
+          const float tk = V[kVLam + k];
+          const bool keep = tk > 1e-12f * th0 && tk > 0.f;
           Ws[li * kMaxRank + k] = keep ? acc[k2] : 0.f;
         }
       }
@@ -585,10 +713,10 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
         int bidx = bt;
         uint32_t bneg = v < 0.f;
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) {
-          const float ob = __shfl_xor_sync(0xffffffffu, best, m);
-          const int oi = __shfl_xor_sync(0xffffffffu, bidx, m);
-          const uint32_t on = __shfl_xor_sync(0xffffffffu, bneg, m);
+        for (int mm = 16; mm >= 1; mm >>= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, mm);
+          const int oi = __shfl_xor_sync(0xffffffffu, bidx, mm);
+          const uint32_t on = __shfl_xor_sync(0xffffffffu, bneg, mm);
           if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; bneg = on; }
         }
         if (lane == 0)
@@ -614,8 +742,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     }
   }
   if (my_valid && bt < D) {
-    const int64_t jb = j0 + blk;
-    uint16_t* rec = a.stats + ((bh * a.nb_cap) + jb) * int64_t(1 + r) * D;
+    uint16_t* rec = a.stats + ((item_bh[blk] * a.nb_cap) + item_j[blk]) * int64_t(1 + r) * D;
     rec[bt] = float_to_bf16_bits(mu_d);
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
@@ -645,7 +772,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-template <int D>
+template <int D, int M>
 cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
   using S = StatsShape<D>;
   EncodeTiledFn enc = encode_fn();
@@ -659,12 +786,12 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = block_stats_kernel<D>;
+  auto kern = block_stats_kernel<D, M>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes));
   if (e != cudaSuccess) return e;
-  const int64_t nblocks = a.block_end - a.block_begin;
-  dim3 grid(unsigned((nblocks + 1) / 2), a.hkv, a.batch);
+  const int64_t n_items = int64_t(a.batch) * a.hkv * (a.block_end - a.block_begin);
+  dim3 grid(unsigned((n_items + 1) / 2), 1, 1);
   kern<<<grid, kStatThreads, S::kBytes, stream>>>(map, a);
   return cudaGetLastError();
 }
@@ -672,7 +799,15 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream) {
-  return a.d == 64 ? launch_stats_t<64>(a, stream) : launch_stats_t<128>(a, stream);
+  const int m = lanczos_steps(a.rank);
+  if (a.d == 64) {
+    if (m == 28) return launch_stats_t<64, 28>(a, stream);
+    if (m == 36) return launch_stats_t<64, 36>(a, stream);
+    return launch_stats_t<64, 52>(a, stream);
+  }
+  if (m == 28) return launch_stats_t<128, 28>(a, stream);
+  if (m == 36) return launch_stats_t<128, 36>(a, stream);
+  return launch_stats_t<128, 52>(a, stream);
 }
 
 }  // namespace cobs

@@ -1,0 +1,176 @@
+"""GPU parity at the full sizes of the five decode workloads, in the launch
+configuration bench.py uses (all blocks of all (batch, kv-head) pairs in one
+call), checked on sampled (batch, kv-head) pairs the oracle computes one by
+one.  Inputs and expected values come only from workloads/ and the oracle:
+for the selection and decode checks the oracle's own stats records and block
+lists are uploaded for the sampled pairs."""
+
+import gc
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.cobs_oracle as O
+from harness import (ENERGY_RTOL, LSE_ATOL, OUT_ATOL, PROJ_RTOL, Problem, from_dev_bits,
+                     selection_mismatch, stats_errors)
+from workloads import WORKLOADS, bits_to_f64, make_queries
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["tiny_4k", "single_32k", "batched_needles_32k", "long_128k", "build_256k"]
+WORKERS = max(1, min(16, (os.cpu_count() or 2) - 1))
+
+
+def sampled_pairs(w):
+    pairs = {(0, 0), (w.batch - 1, w.kv_heads - 1), (w.batch // 2, w.kv_heads // 2)}
+    return sorted(pairs)
+
+
+@pytest.fixture(scope="module", params=FULL)
+def full(request):
+    torch.cuda.empty_cache()
+    w = WORKLOADS[request.param]
+    p = Problem(w, workers=WORKERS)
+    p.build_stats()
+    torch.cuda.synchronize()
+    p.gpu_stats = p.stats.clone()
+    p.orc_recs = {bh: p.oracle_records(*bh) for bh in sampled_pairs(w)}
+    yield p
+    del p
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_full_stats(full):
+    p, w = full, full.w
+    st = from_dev_bits(p.gpu_stats)
+    rng = np.random.default_rng(1)
+    nfull = w.seq_len // w.block
+    for (b, h), orc in p.orc_recs.items():
+        keys = p.keys(b, h)
+        blocks = sorted(set([0, nfull - 1] + list(rng.choice(nfull, size=min(nfull, 48),
+                                                             replace=False))))
+        gpu = bits_to_f64(st[b, h])
+        for j in blocks:
+            mu_ok, rel, energy = stats_errors(gpu[j], orc[j], keys[j * 64:(j + 1) * 64], w.rank)
+            assert mu_ok, (b, h, j)
+            assert rel is None or rel <= PROJ_RTOL, (b, h, j, rel)
+            assert energy >= 1 - ENERGY_RTOL, (b, h, j, energy)
+    assert p.device_status() == 0
+
+
+def test_full_select_on_oracle_stats(full):
+    p, w = full, full.w
+    p.stats.copy_(p.gpu_stats)
+    for (b, h), recs in p.orc_recs.items():
+        p.upload_records(b, h, recs)
+    p.select()
+    idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+    for (b, h), recs in p.orc_recs.items():
+        sel, s = O.select_from_records(p.q_group(b, h), recs, w.seq_len, w.block, w.top_k,
+                                       w.sink_blocks, w.local_tokens)
+        got = idx[b, h, :n[b, h]]
+        assert np.all(np.diff(got) > 0)
+        assert len(got) == len(sel)
+        assert selection_mismatch(got, sel, s, w) == []
+    assert p.device_status() == 0
+
+
+def test_full_decode_on_oracle_selection(full):
+    p, w = full, full.w
+    scale = 1 / math.sqrt(w.head_dim)
+    idx = torch.zeros_like(p.idx)
+    n = torch.zeros_like(p.n_sel)
+    sels = {}
+    for (b, h), recs in p.orc_recs.items():
+        sel, _ = O.select_from_records(p.q_group(b, h), recs, w.seq_len, w.block, w.top_k,
+                                       w.sink_blocks, w.local_tokens)
+        sels[(b, h)] = sel
+    # every pair needs a valid list; unsampled pairs get the forced blocks only
+    forced, _, _ = O.block_partition(w.seq_len, w.block, w.sink_blocks, w.local_tokens)
+    idx[:, :, :len(forced)] = torch.tensor(forced, dtype=torch.int32, device="cuda")
+    n.fill_(len(forced))
+    for (b, h), sel in sels.items():
+        idx[b, h, :len(sel)] = torch.tensor(sel.astype(np.int32), device="cuda")
+        n[b, h] = len(sel)
+    p.decode(idx=idx, n_sel=n)
+    out, lse = p.out.cpu().numpy(), p.lse.cpu().numpy()
+    G = w.group
+    for (b, h), sel in sels.items():
+        o, l = O.sparse_attention(p.q_group(b, h), p.keys(b, h), p.values(b, h), sel,
+                                  w.seq_len, w.block, scale)
+        assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL
+        np.testing.assert_allclose(lse[b, h * G:(h + 1) * G], l, atol=LSE_ATOL)
+    assert p.device_status() == 0
+
+
+def test_full_end_to_end_flips_reported(full):
+    """GPU stats -> GPU selection, compared with the oracle end to end.  Flips
+    on near-degenerate spectra are reported, not failed (the eigen step is not
+    bit-reproducible); outputs must match wherever the selections agree."""
+    p, w = full, full.w
+    p.stats.copy_(p.gpu_stats)
+    p.select()
+    p.decode()
+    idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+    out = p.out.cpu().numpy()
+    G = w.group
+    flips = 0
+    for (b, h), recs in p.orc_recs.items():
+        sel, s = O.select_from_records(p.q_group(b, h), recs, w.seq_len, w.block, w.top_k,
+                                       w.sink_blocks, w.local_tokens)
+        got = idx[b, h, :n[b, h]]
+        if set(got.tolist()) != set(sel.tolist()):
+            flips += 1
+            continue
+        o, _ = O.sparse_attention(p.q_group(b, h), p.keys(b, h), p.values(b, h), sel,
+                                  w.seq_len, w.block, 1 / math.sqrt(w.head_dim))
+        assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL
+    print(f"{w.name}: end-to-end selection flips on {flips} of {len(p.orc_recs)} sampled pairs")
+    assert p.device_status() == 0
+
+
+def test_append_chunks_equal_one_shot_build(full):
+    p, w = full, full.w
+    if not w.append_chunk:
+        pytest.skip("workload is not built by appends")
+    p.stats.zero_()
+    per = w.append_chunk // w.block
+    nfull = w.seq_len // w.block
+    for c0 in range(0, nfull, per):
+        p.build_stats(c0, min(nfull, c0 + per))
+    torch.cuda.synchronize()
+    assert torch.equal(p.stats, p.gpu_stats)
+    assert p.device_status() == 0
+
+
+def test_decode_steps_with_fresh_queries(full):
+    p, w = full, full.w
+    if w.decode_steps <= 1:
+        pytest.skip("single decode step workload")
+    p.stats.copy_(p.gpu_stats)
+    scale = 1 / math.sqrt(w.head_dim)
+    G = w.group
+    for t in (0, w.decode_steps // 2, w.decode_steps - 1):
+        qb = make_queries(w, t)
+        p.q.copy_(torch.from_numpy(qb.view(np.int16)))
+        for (b, h), recs in p.orc_recs.items():
+            p.upload_records(b, h, recs)
+        p.select()
+        p.decode()
+        idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+        out = p.out.cpu().numpy()
+        for (b, h), recs in p.orc_recs.items():
+            qg = bits_to_f64(qb[b, h * G:(h + 1) * G])
+            sel, s = O.select_from_records(qg, recs, w.seq_len, w.block, w.top_k,
+                                           w.sink_blocks, w.local_tokens)
+            got = idx[b, h, :n[b, h]]
+            assert selection_mismatch(got, sel, s, w) == []
+            if set(got.tolist()) == set(sel.tolist()):
+                o, _ = O.sparse_attention(qg, p.keys(b, h), p.values(b, h), sel, w.seq_len,
+                                          w.block, scale)
+                assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL
+    assert p.device_status() == 0
