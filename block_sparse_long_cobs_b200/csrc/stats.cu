@@ -9,26 +9,29 @@
 // Method used on the GPU (same result as the eigen-decomposition of the d x d
 // covariance, computed through the n x n Gram matrix because n = B = 64 < d):
 //   1. Raw Gram G = K K^T of the block's bf16 keys on the 5th-generation tensor
-//      cores: one tcgen05.mma chain (kind::f16, bf16 in, fp32 accumulate in
-//      tensor memory) computes the 128 x 128 Gram of two blocks stacked along
-//      M (consecutive work items, possibly of different (batch, kv-head)
-//      pairs); the two diagonal 64 x 64 quadrants are the blocks' Grams.  Products of bf16 values are exact, so no precision is lost
-//      before the fp32 accumulation.  The keys arrive by TMA (2-d tensor map,
-//      128-byte swizzle = the UMMA K-major canonical layout).
+//      cores: one tcgen05.mma chain (kind::f16, M = 128, N = 64, bf16 in, fp32
+//      accumulate in tensor memory); rows 0-63 of the A tile hold the block,
+//      rows 64-127 are never read back.  Products of bf16 values are exact, so
+//      no precision is lost before the fp32 accumulation.  The keys arrive by
+//      TMA (2-d tensor map, 128-byte swizzle = the UMMA K-major canonical
+//      layout).  One block per CTA of 128 threads with a small shared-memory
+//      footprint (the key tile's space is reused for the Lanczos basis and U
+//      re-reads the keys through L2), so the kernel can share SMs with the
+//      selection and decode kernels when it runs on a side stream.
 //   2. Centring in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
 //      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T; then
 //      A = Gc^2 (same eigenvectors, squared eigenvalues: the top of the
 //      spectrum separates faster, so fewer Lanczos steps are needed).
 //   3. Lanczos tridiagonalisation of A, m = 28 / 36 / 52 steps for r <= 4 /
-//      <= 8 / <= 16 (at least 2 r + 20), every new
-//      vector re-orthogonalised twice against all earlier ones by classical
-//      Gram-Schmidt (basis kept row- and column-major in shared memory so both
-//      Gram-Schmidt phases are 128-bit loads), a fresh pseudo-random vector
-//      whenever the Krylov space closes.  128 threads per block, each holding
-//      32 entries of A in registers; five named-barrier phases per step.
+//      <= 8 / <= 16 (at least 2 r + 20), every new vector re-orthogonalised
+//      twice against all earlier ones by classical Gram-Schmidt (basis kept
+//      row- and column-major in shared memory so both Gram-Schmidt phases are
+//      128-bit loads), a fresh pseudo-random vector whenever the Krylov space
+//      closes.  Each thread holds 32 entries of A in registers; five barrier
+//      phases per step, norms reduced through those same barriers.
 //   4. Top-r eigenvalues of the m x m tridiagonal T by multisection bisection
 //      on Sturm counts (8 threads x 3 shifts per eigenvalue, 25-way splits),
-//      eigenvectors z_k by inverse iteration (LDL^T of T - theta I, vector in
+//      eigenvectors z_k by inverse iteration (LDL^T of T - theta I, all in
 //      registers), re-orthogonalised inside clusters of close eigenvalues;
 //      Ritz vectors w_k = Q z_k are unit eigenvectors of Gc.
 //   5. U[:, k] = Kc^T w_k / sqrt(n) (its squared norm is the covariance
@@ -42,10 +45,10 @@
 namespace cobs {
 namespace {
 
-constexpr int kStatThreads = 256;   // 2 blocks x 128 threads
+constexpr int kStatThreads = 128;   // one block per CTA
 constexpr int kQStride = 72;        // floats per basis row: halves of 36
 constexpr int kGStride = 68;        // 16-byte aligned row of the staged Grams
-constexpr int kBisectRounds = 5;   // 25-way splits: 25^5 ~ 1e7
+constexpr int kBisectRounds = 5;    // 25-way splits: 25^5 ~ 1e7
 constexpr int kInverseIters = 2;
 
 // Lanczos length by rank bucket: m = 2 r + 20 for the largest r of the bucket
@@ -56,30 +59,28 @@ __host__ __device__ constexpr int lanczos_steps(int rank) {
 template <int D>
 struct StatsShape {
   static constexpr int kRegions = D / 64;           // 128-byte-wide column slabs
-  static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B
-  // per-block regions (x2)
-  static constexpr size_t kQBytes = 64 * kQStride * 4;        // Q rows; G^2 staging
-  static constexpr size_t kZBytes = kMaxRank * 64 * 4;        // eigenvectors of T
-  static constexpr size_t kWBytes = 64 * kMaxRank * 4;        // Ritz vectors [t][k]
-  static constexpr size_t kScrBytes = kMaxRank * 2 * 64 * 4;  // inverse iteration
-  static constexpr size_t kVecBytes = 2048;                   // small vectors
-  static constexpr size_t kK = 0;                             // [regions][128][128 B]
-  static constexpr size_t kQ = kK + size_t(kRegions) * kRegionBytes;
-  static constexpr size_t kQT = kQ + 2 * kQBytes;             // Q^T rows; Gc staging
-  static constexpr size_t kZ = kQT + 2 * kQBytes;
-  static constexpr size_t kW = kZ + 2 * kZBytes;
-  static constexpr size_t kScr = kW + 2 * kWBytes;
-  static constexpr size_t kVec = kScr + 2 * kScrBytes;
-  static constexpr size_t kMu = kVec + 2 * kVecBytes;          // [2][D]
-  static constexpr size_t kRow = kMu + 2 * D * 4;              // [128] row means
-  static constexpr size_t kFlip = kRow + 128 * 4;              // [2][4][16] uint2
-  static constexpr size_t kBar = kFlip + 2 * 4 * kMaxRank * 8;
+  static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B (rows 64+ unused)
+  static constexpr size_t kQBytes = 64 * kQStride * 4;        // basis rows; Gram staging
+  // the key tile (needed until the Gram and the mean are done) and the two
+  // basis copies Q, Q^T share the first region
+  static constexpr size_t kKeyBytes = size_t(kRegions) * kRegionBytes;
+  static constexpr size_t kR1 = kKeyBytes > 2 * kQBytes ? kKeyBytes : 2 * kQBytes;
+  static constexpr size_t kK = 0;
+  static constexpr size_t kQ = 0;
+  static constexpr size_t kQT = kQBytes;
+  static constexpr size_t kZ = kR1;                                // eigenvectors of T
+  static constexpr size_t kW = kZ + kMaxRank * 64 * 4;             // Ritz vectors [t][k]
+  static constexpr size_t kVec = kW + 64 * kMaxRank * 4;           // small vectors
+  static constexpr size_t kMu = kVec + 2048;                       // [D]
+  static constexpr size_t kRow = kMu + D * 4;                      // [64] row means
+  static constexpr size_t kFlip = kRow + 64 * 4;                   // [4][16] uint2
+  static constexpr size_t kBar = kFlip + 4 * kMaxRank * 8;
   static constexpr size_t kMisc = kBar + 16;
   static constexpr size_t kBytes = kMisc + 16 + 1024;  // + alignment slack
   static_assert(64 * kGStride * 4 <= kQBytes, "Gram staging must fit in a basis region");
 };
 
-// Offsets inside the per-block small-vector area (floats).
+// Offsets inside the small-vector area (floats).
 constexpr int kVW = 0;        // w, split layout [2][36]
 constexpr int kVH = 72;       // Gram-Schmidt coefficients h, split layout [2][36]
 constexpr int kVRed = 144;    // reduction partials [4] + norm partials [4]
@@ -239,34 +240,23 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   uint32_t* abort_s = misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // work items (bh, j) for every (batch, kv-head) pair and every block in
-  // [block_begin, block_end), two per CTA (they need not share a pair)
+  // work item: block j of (batch, kv-head) pair bh
   const int64_t nb_range = a.block_end - a.block_begin;
-  const int64_t n_items = int64_t(a.batch) * a.hkv * nb_range;
-  const int64_t item0 = 2 * int64_t(blockIdx.x);
-  const bool has1 = item0 + 1 < n_items;
-  int64_t item_bh[2], item_j[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int64_t it = (q == 0 || has1) ? item0 + q : item0;
-    item_bh[q] = it / nb_range;
-    item_j[q] = a.block_begin + it % nb_range;
-  }
-  const int blk = tid >> 7;            // block of the pair this thread serves
-  const int bt = tid & 127;            // thread index inside that block's team
-  const int bwarp = bt >> 5;           // warp index inside the team
-  const bool my_valid = blk == 0 || has1;
+  const int64_t item_bh = int64_t(blockIdx.x) / nb_range;
+  const int64_t item_j = a.block_begin + int64_t(blockIdx.x) % nb_range;
+  const int bt = tid;                  // thread index (the whole CTA is one team)
+  const int bwarp = warp;
   const int r = a.rank;
-  const int bar_id = 1 + blk;
-  constexpr int msteps = M;                 // Lanczos steps
+  const int bar_id = 1;
+  constexpr int msteps = M;            // Lanczos steps
 
-  float* Qs = reinterpret_cast<float*>(smem + S::kQ + blk * S::kQBytes);
-  float* QTs = reinterpret_cast<float*>(smem + S::kQT + blk * S::kQBytes);
-  float* Zs = reinterpret_cast<float*>(smem + S::kZ + blk * S::kZBytes);
-  float* Ws = reinterpret_cast<float*>(smem + S::kW + blk * S::kWBytes);
-  float* Scr = reinterpret_cast<float*>(smem + S::kScr + blk * S::kScrBytes);
-  float* V = reinterpret_cast<float*>(smem + S::kVec + blk * S::kVecBytes);
-  float* mus = reinterpret_cast<float*>(smem + S::kMu) + blk * D;
+  float* Qs = reinterpret_cast<float*>(smem + S::kQ);
+  float* QTs = reinterpret_cast<float*>(smem + S::kQT);
+  float* Zs = reinterpret_cast<float*>(smem + S::kZ);
+  float* Ws = reinterpret_cast<float*>(smem + S::kW);
+  float* V = reinterpret_cast<float*>(smem + S::kVec);
+  float* mus = reinterpret_cast<float*>(smem + S::kMu);
+  const uint16_t* kglob = a.k + (item_bh * a.cap + item_j * kBlock) * D;
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);  // TMA
@@ -274,26 +264,22 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     fence_barrier_init();
     *abort_s = 0;
   }
-  if (warp == 0) tmem_alloc(tmem_slot, 128);
+  if (warp == 0) tmem_alloc(tmem_slot, 64);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // ---- 1. TMA load of the two blocks, then the Gram on the tensor cores ------
+  // ---- 1. TMA load of the block, then the Gram on the tensor cores -----------
   if (tid == 0) {
-    const int nblk = has1 ? 2 : 1;
-    mbar_arrive_expect_tx(&bars[0], uint32_t(nblk) * kBlock * D * 2);
-    for (int q = 0; q < nblk; ++q) {
-      const int y = int(item_bh[q] * a.cap + item_j[q] * kBlock);
-      for (int reg = 0; reg < S::kRegions; ++reg)
-        tma_load_2d(ktile + reg * S::kRegionBytes + q * kBlock * 128, &kmap, reg * 64, y,
-                    &bars[0]);
-    }
+    mbar_arrive_expect_tx(&bars[0], uint32_t(kBlock) * D * 2);
+    const int y = int(item_bh * a.cap + item_j * kBlock);
+    for (int reg = 0; reg < S::kRegions; ++reg)
+      tma_load_2d(ktile + reg * S::kRegionBytes, &kmap, reg * 64, y, &bars[0]);
     bool ok = mbar_wait_bounded(&bars[0], 0, a.status);
     if (ok) {
       tc_fence_after();
-      constexpr uint32_t idesc = umma_idesc_bf16(128, 128);
+      constexpr uint32_t idesc = umma_idesc_bf16(128, 64);
       const uint32_t kbase = smem_addr(ktile);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
@@ -311,57 +297,52 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   if (!aborted && tid != 0) (void)mbar_try_wait(&bars[1], 0);
   tc_fence_after();
 
-  // ---- 2. Gram rows back from tensor memory (warps 0-3), centring -----------
-  // Thread t < 128 reads TMEM lane t = row (t & 63) of block (t >> 6).
+  // ---- 2. Gram rows back from tensor memory (warps 0-1), mean, centring ------
   float g[64];
-  const int rb = tid >> 6, ri = tid & 63;
-  if (!aborted && warp < 4) {
+  const int ri = tid;                  // Gram row (threads 0-63)
+  if (!aborted && warp < 2) {
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t col0 = uint32_t(rb * 64);
     float t32[32];
-    tmem_ld32(tmem + lane_base + col0, t32);
+    tmem_ld32(tmem + lane_base, t32);
 #pragma unroll
     for (int c = 0; c < 32; ++c) g[c] = t32[c];
-    tmem_ld32(tmem + lane_base + col0 + 32, t32);
+    tmem_ld32(tmem + lane_base + 32, t32);
 #pragma unroll
     for (int c = 0; c < 32; ++c) g[32 + c] = t32[c];
     float rsum = 0.f;
 #pragma unroll
     for (int c = 0; c < 64; ++c) rsum += g[c];
-    row_mean[tid] = rsum * (1.f / 64.f);
+    row_mean[ri] = rsum * (1.f / 64.f);
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 128);
-  if (aborted) return;
-  if (warp < 4) {
-    float ssum = 0.f;
-    for (int c = 0; c < 64; ++c) ssum += row_mean[rb * 64 + c];
-    const float smean = ssum * (1.f / 64.f);
-    const float rm = row_mean[tid];
-    // Gc is symmetric: row ri is stored as column ri (consecutive lanes ->
-    // consecutive addresses)
-    float* stage = reinterpret_cast<float*>(smem + S::kQT + rb * S::kQBytes);
-#pragma unroll
-    for (int c = 0; c < 64; ++c)
-      stage[c * kGStride + ri] = g[c] - rm - row_mean[rb * 64 + c] + smean;
-  }
-
   // block mean (fp32 sum of 64 bf16 keys): thread bt < D owns dim bt
-  if (bt < D) {
+  if (!aborted && bt < D) {
     float acc = 0.f;
     for (int t = 0; t < kBlock; ++t) {
-      const uint16_t w =
-          *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(blk * 64 + t, bt));
+      const uint16_t w = *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(t, bt));
       acc += __uint_as_float(uint32_t(w) << 16);
     }
     mus[bt] = acc * (1.f / 64.f);
   }
+  tc_fence_before();
+  __syncthreads();                     // key tile and tensor memory no longer needed
+  if (warp == 0) tmem_dealloc(tmem, 64);
+  if (aborted) return;
+  if (warp < 2) {
+    float ssum = 0.f;
+    for (int c = 0; c < 64; ++c) ssum += row_mean[c];
+    const float smean = ssum * (1.f / 64.f);
+    const float rm = row_mean[ri];
+    // Gc is symmetric: row ri is stored as column ri (consecutive lanes ->
+    // consecutive addresses); the staging area overlays the key tile
+    float* stage = QTs;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) stage[c * kGStride + ri] = g[c] - rm - row_mean[c] + smean;
+  }
   __syncthreads();
 
-  const bool do_eig = r > 0 && my_valid;
+  const bool do_eig = r > 0;
   const int li = bt >> 1, hh = bt & 1;
-  auto block_sum = [&](float v) -> float {  // sum over the 128 threads of the team
+  auto block_sum = [&](float v) -> float {  // sum over the 128 threads
     v = warp_sum(v);
     if (lane == 0) V[kVRed + bwarp] = v;
     named_bar(bar_id, 128);
@@ -679,15 +660,15 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   __syncthreads();
 
   // ---- 5. U = Kc^T w / sqrt(n), sign rule, bf16 record ------------------------
-  // thread bt < D owns output dim d = bt
+  // thread bt < D owns output dim d = bt; keys re-read through L2 (coalesced rows)
   float uacc[kMaxRank];
 #pragma unroll
   for (int k = 0; k < kMaxRank; ++k) uacc[k] = 0.f;
   const float mu_d = bt < D ? mus[bt] : 0.f;
   if (do_eig && bt < D) {
+#pragma unroll 4
     for (int t = 0; t < kBlock; ++t) {
-      const uint16_t w =
-          *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(blk * 64 + t, bt));
+      const uint16_t w = kglob[int64_t(t) * D + bt];
       const float kc = __uint_as_float(uint32_t(w) << 16) - mu_d;
       const float4* wt = reinterpret_cast<const float4*>(Ws + t * kMaxRank);
 #pragma unroll
@@ -720,8 +701,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
           if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; bneg = on; }
         }
         if (lane == 0)
-          flip_s[(blk * 4 + bwarp) * kMaxRank + k] =
-              make_uint2(__float_as_uint(best), (uint32_t(bidx) << 1) | bneg);
+          flip_s[bwarp * kMaxRank + k] = make_uint2(__float_as_uint(best), (uint32_t(bidx) << 1) | bneg);
       }
     }
   }
@@ -731,9 +711,9 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
       if (k < r) {
-        uint2 best = flip_s[(blk * 4 + 0) * kMaxRank + k];
+        uint2 best = flip_s[k];
         for (int w2 = 1; w2 < 4; ++w2) {
-          const uint2 o = flip_s[(blk * 4 + w2) * kMaxRank + k];
+          const uint2 o = flip_s[w2 * kMaxRank + k];
           const float bo = __uint_as_float(o.x), bb = __uint_as_float(best.x);
           if (bo > bb || (bo == bb && (o.y >> 1) < (best.y >> 1))) best = o;
         }
@@ -741,8 +721,8 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       }
     }
   }
-  if (my_valid && bt < D) {
-    uint16_t* rec = a.stats + ((item_bh[blk] * a.nb_cap) + item_j[blk]) * int64_t(1 + r) * D;
+  if (bt < D) {
+    uint16_t* rec = a.stats + ((item_bh * a.nb_cap) + item_j) * int64_t(1 + r) * D;
     rec[bt] = float_to_bf16_bits(mu_d);
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
@@ -791,7 +771,7 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes));
   if (e != cudaSuccess) return e;
   const int64_t n_items = int64_t(a.batch) * a.hkv * (a.block_end - a.block_begin);
-  dim3 grid(unsigned((n_items + 1) / 2), 1, 1);
+  dim3 grid(unsigned(n_items), 1, 1);
   kern<<<grid, kStatThreads, S::kBytes, stream>>>(map, a);
   return cudaGetLastError();
 }
