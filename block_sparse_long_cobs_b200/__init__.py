@@ -1,188 +1,26 @@
-"""Thin Python binding of the COBS block-sparse decode C ABI (``include/cobs.h``).
+"""COBS block-sparse attention decode for B200 (sm_100a): Python binding.
 
-Argument marshalling only: every function here forwards to the function of
-the same name in ``libcobs_b200.so`` (built in-tree by
-``python -m block_sparse_long_cobs_b200.build``); all computation happens in
-the library's CUDA kernels.  Tensors may be given as torch tensors (their
-``data_ptr()`` is passed), integer addresses or ``None`` (NULL).  Streams may
-be a ``torch.cuda.Stream``, an integer handle or ``None`` (legacy default
-stream).  Importing this module fails if the library has not been built: there
-is no fallback path.
+The functions (``cobs_build_block_stats``, ``cobs_select_blocks``,
+``cobs_sparse_decode``, ...) forward to the C ABI of ``libcobs_b200.so``
+(declared in ``include/cobs.h``); see ``_binding.py``.  The library is loaded
+on first use, and that first use raises ImportError if it has not been built
+(``python -m block_sparse_long_cobs_b200.build``): there is no fallback path.
 """
 
-from __future__ import annotations
-
-import ctypes
-import os
+from importlib import import_module as _import_module
 
 __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
     "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
-    "cobs_sparse_decode", "cobs_read_device_status", "cobs_last_error",
-    "cobs_status_string",
+    "cobs_sparse_decode", "cobs_read_device_status",
+    "cobs_last_error", "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcobs_b200.so")
 
-COBS_OK = 0
-COBS_ERR_INVALID_ARG = 1
-COBS_ERR_UNSUPPORTED = 2
-COBS_ERR_WORKSPACE = 3
-COBS_ERR_CUDA = 4
-COBS_ERR_TIMEOUT = 5
-COBS_ERR_DEVICE = 6
-
-
-class CobsError(RuntimeError):
-    """A COBS call returned a non-OK status."""
-
-    def __init__(self, func: str, status: int, message: str):
-        super().__init__(f"{func}: {cobs_status_string(status)}: {message}")
-        self.status = status
-
-
-class cobs_dims(ctypes.Structure):
-    _fields_ = [
-        ("batch", ctypes.c_int32),
-        ("num_q_heads", ctypes.c_int32),
-        ("num_kv_heads", ctypes.c_int32),
-        ("head_dim", ctypes.c_int32),
-        ("block_size", ctypes.c_int32),
-        ("rank", ctypes.c_int32),
-        ("capacity_tokens", ctypes.c_int64),
-    ]
-
-
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"COBS CUDA library not found at {LIB_PATH}; build it with "
-            "`python -m block_sparse_long_cobs_b200.build` (needs nvcc)")
-    L = ctypes.CDLL(LIB_PATH)
-    P, I32, I64, SZ, F32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
-                            ctypes.c_size_t, ctypes.c_float)
-    D = ctypes.POINTER(cobs_dims)
-    sig = {
-        "cobs_abi_version": (I32, []),
-        "cobs_selected_capacity": (I32, [D, I32, I32, I32]),
-        "cobs_workspace_bytes": (SZ, [D, I32, I32, I32]),
-        "cobs_workspace_init": (I32, [P, SZ, P]),
-        "cobs_build_block_stats": (I32, [D, P, I64, I64, P, P, SZ, P]),
-        "cobs_select_blocks": (I32, [D, P, P, I64, I32, I32, I32, P, I32, P, P, P, SZ, P]),
-        "cobs_sparse_decode": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P, SZ, P]),
-        "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
-        "cobs_last_error": (ctypes.c_char_p, []),
-        "cobs_status_string": (ctypes.c_char_p, [I32]),
-    }
-    for name, (res, args) in sig.items():
-        f = getattr(L, name)
-        f.restype = res
-        f.argtypes = args
-    return L
-
-
-lib = _load()
-
-
-def _ptr(x):
-    if x is None:
-        return None
-    if isinstance(x, int):
-        return ctypes.c_void_p(x)
-    if hasattr(x, "data_ptr"):
-        return ctypes.c_void_p(x.data_ptr())
-    if hasattr(x, "ctypes"):
-        return ctypes.c_void_p(x.ctypes.data)
-    raise TypeError(f"cannot pass {type(x).__name__} as a pointer")
-
-
-def _stream(s):
-    if s is None:
-        return None
-    if isinstance(s, int):
-        return ctypes.c_void_p(s)
-    return ctypes.c_void_p(s.cuda_stream)
-
-
-def _check(func: str, status: int, check: bool) -> int:
-    if check and status != COBS_OK:
-        raise CobsError(func, status, cobs_last_error())
-    return status
-
-
-def _dims(d) -> cobs_dims:
-    if isinstance(d, cobs_dims):
-        return d
-    return cobs_dims(**d)
-
-
-def cobs_abi_version() -> int:
-    return lib.cobs_abi_version()
-
-
-def cobs_last_error() -> str:
-    return lib.cobs_last_error().decode()
-
-
-def cobs_status_string(status: int) -> str:
-    return lib.cobs_status_string(status).decode()
-
-
-def cobs_selected_capacity(dims, top_k, sink_blocks, local_tokens) -> int:
-    n = lib.cobs_selected_capacity(ctypes.byref(_dims(dims)), top_k, sink_blocks,
-                                   local_tokens)
-    if n < 0:
-        raise CobsError("cobs_selected_capacity", COBS_ERR_INVALID_ARG, cobs_last_error())
-    return n
-
-
-def cobs_workspace_bytes(dims, top_k, sink_blocks, local_tokens) -> int:
-    n = lib.cobs_workspace_bytes(ctypes.byref(_dims(dims)), top_k, sink_blocks,
-                                 local_tokens)
-    if n == 0:
-        raise CobsError("cobs_workspace_bytes", COBS_ERR_INVALID_ARG, cobs_last_error())
-    return n
-
-
-def cobs_workspace_init(ws, ws_bytes, stream=None, check=True) -> int:
-    return _check("cobs_workspace_init",
-                  lib.cobs_workspace_init(_ptr(ws), ws_bytes, _stream(stream)), check)
-
-
-def cobs_build_block_stats(dims, k, block_begin, block_end, stats, ws, ws_bytes,
-                           stream=None, check=True) -> int:
-    st = lib.cobs_build_block_stats(ctypes.byref(_dims(dims)), _ptr(k), block_begin,
-                                    block_end, _ptr(stats), _ptr(ws), ws_bytes,
-                                    _stream(stream))
-    return _check("cobs_build_block_stats", st, check)
-
-
-def cobs_select_blocks(dims, q, stats, seq_len, top_k, sink_blocks, local_tokens,
-                       idx, idx_stride, n_sel, scores_opt, ws, ws_bytes, stream=None,
-                       check=True) -> int:
-    st = lib.cobs_select_blocks(ctypes.byref(_dims(dims)), _ptr(q), _ptr(stats), seq_len,
-                                top_k, sink_blocks, local_tokens, _ptr(idx), idx_stride,
-                                _ptr(n_sel), _ptr(scores_opt), _ptr(ws), ws_bytes,
-                                _stream(stream))
-    return _check("cobs_select_blocks", st, check)
-
-
-def cobs_sparse_decode(dims, q, k, v, idx, n_sel, idx_stride, seq_len, softmax_scale,
-                       out, lse, ws, ws_bytes, stream=None, check=True) -> int:
-    st = lib.cobs_sparse_decode(ctypes.byref(_dims(dims)), _ptr(q), _ptr(k), _ptr(v),
-                                _ptr(idx), _ptr(n_sel), idx_stride, seq_len,
-                                ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
-                                _ptr(ws), ws_bytes, _stream(stream))
-    return _check("cobs_sparse_decode", st, check)
-
-
-def cobs_read_device_status(ws, ws_bytes, stream=None) -> int:
-    """Synchronise the stream and return (and clear) the device status word."""
-    out = ctypes.c_int32(0)
-    st = lib.cobs_read_device_status(_ptr(ws), ws_bytes, ctypes.byref(out),
-                                     _stream(stream))
-    _check("cobs_read_device_status", st, True)
-    return out.value
+def __getattr__(name):
+    if name in __all__:
+        return getattr(_import_module("._binding", __name__), name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

@@ -350,3 +350,4 @@ cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_s
 }
 
 }  // extern "C"
+
