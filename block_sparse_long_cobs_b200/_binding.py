@@ -19,7 +19,8 @@ __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
     "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
-    "cobs_sparse_decode", "cobs_read_device_status", "cobs_last_error",
+    "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_read_device_status",
+    "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",
@@ -73,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "cobs_build_block_stats": (I32, [D, P, I64, I64, P, P, SZ, P]),
         "cobs_select_blocks": (I32, [D, P, P, I64, I32, I32, I32, P, I32, P, P, P, SZ, P]),
         "cobs_sparse_decode": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P, SZ, P]),
+        "cobs_sparse_decode_no_alloc": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_last_error": (ctypes.c_char_p, []),
         "cobs_status_string": (ctypes.c_char_p, [I32]),
@@ -177,6 +179,17 @@ def cobs_sparse_decode(dims, q, k, v, idx, n_sel, idx_stride, seq_len, softmax_s
                                 ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
                                 _ptr(ws), ws_bytes, _stream(stream))
     return _check("cobs_sparse_decode", st, check)
+
+
+def cobs_sparse_decode_no_alloc(dims, q, k, v, idx, n_sel, idx_stride, seq_len,
+                                softmax_scale, out, lse, stream=None, check=True) -> int:
+    """cobs_sparse_decode without a workspace: for callers that cannot give the
+    library device memory; it uses the library's own fixed 16 MiB array."""
+    st = lib.cobs_sparse_decode_no_alloc(ctypes.byref(_dims(dims)), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(idx), _ptr(n_sel), idx_stride, seq_len,
+                                         ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
+                                         _stream(stream))
+    return _check("cobs_sparse_decode_no_alloc", st, check)
 
 
 def cobs_read_device_status(ws, ws_bytes, stream=None) -> int:

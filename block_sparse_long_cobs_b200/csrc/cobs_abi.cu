@@ -351,3 +351,122 @@ cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_s
 
 }  // extern "C"
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode: split-K scratch lives in a fixed device array that
+// belongs to the library instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace cobs {
+namespace {
+
+constexpr size_t kFixedScratchBytes = size_t(16) << 20;   // per device, held until exit
+__device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_fixed_scratch_addr[kMaxDevices];
+cudaError_t g_fixed_scratch_err[kMaxDevices];
+std::once_flag g_fixed_scratch_once[kMaxDevices];
+
+// Device address of g_fixed_scratch on the current device, looked up once per
+// device (the host-side name is only a stand-in, never a device address).
+cobs_status fixed_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(COBS_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices - 1);
+  std::call_once(g_fixed_scratch_once[dev], [dev]() {
+    void* p = nullptr;
+    g_fixed_scratch_err[dev] = cudaGetSymbolAddress(&p, g_fixed_scratch);
+    g_fixed_scratch_addr[dev] = p;
+  });
+  if (g_fixed_scratch_err[dev] != cudaSuccess)
+    return cuda_fail(g_fixed_scratch_err[dev], "cudaGetSymbolAddress(fixed scratch)");
+  *out = g_fixed_scratch_addr[dev];
+  return COBS_OK;
+}
+
+}  // namespace
+}  // namespace cobs
+
+extern "C" {
+
+cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, const void* k,
+                                        const void* v, const int32_t* idx,
+                                        const int32_t* n_sel, int32_t idx_stride,
+                                        int64_t seq_len, float softmax_scale, float* out,
+                                        float* lse, void* stream) {
+  cobs_status st = check_dims(dims);
+  if (st != COBS_OK) return st;
+  if (!q || !k || !v || !idx || !n_sel || !out || !lse)
+    return fail(COBS_ERR_INVALID_ARG, "q, k, v, idx, n_sel, out and lse must not be NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(idx) || !aligned16(n_sel) ||
+      !aligned16(out) || !aligned16(lse))
+    return fail(COBS_ERR_INVALID_ARG, "device pointers must be 16-byte aligned");
+  if (seq_len < 1 || seq_len > dims->capacity_tokens)
+    return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
+                (long long)seq_len);
+  if (idx_stride < 1) return fail(COBS_ERR_INVALID_ARG, "idx_stride must be >= 1");
+  if (!(std::isfinite(softmax_scale)) || softmax_scale <= 0.f)
+    return fail(COBS_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+
+  // split count exactly as in cobs_sparse_decode; the partials are packed with
+  // one row per split actually launched
+  const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
+  int sms = device_sm_count();
+  if (sms <= 0) sms = 148;
+  const int resident =
+      sms * decode_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads);
+  int64_t splits = resident / pairs;
+  if (splits > idx_stride) splits = idx_stride;
+  if (splits < 1) splits = 1;
+  const int64_t bps = ceil_div(idx_stride, splits);
+  const int64_t n_splits = ceil_div(idx_stride, bps);
+  const size_t tickets_bytes = align256(size_t(pairs) * 4);
+  const size_t need = tickets_bytes + size_t(dims->batch) * dims->num_q_heads *
+                                          size_t(n_splits) * (size_t(dims->head_dim) + 2) * 4;
+  if (need > kFixedScratchBytes)
+    return fail(COBS_ERR_WORKSPACE,
+                "this decode needs %zu bytes of scratch, above the library's fixed %zu; use "
+                "cobs_sparse_decode with a caller workspace",
+                need, kFixedScratchBytes);
+
+  void* scratch = nullptr;
+  if ((st = fixed_scratch_address(&scratch)) != COBS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // arrival counters must start at zero (the kernel leaves them at zero, but a
+  // previous call may have been cut short)
+  cudaError_t e = cudaMemsetAsync(scratch, 0, tickets_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed scratch counters");
+
+  DecodeArgs a{};
+  char* w = static_cast<char*>(scratch);
+  a.q = static_cast<const uint16_t*>(q);
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.idx = idx;
+  a.n_sel = n_sel;
+  a.out = out;
+  a.lse = lse;
+  a.tickets = reinterpret_cast<uint32_t*>(w);
+  a.partials = reinterpret_cast<float*>(w + tickets_bytes);
+  a.status = nullptr;   // no status word: out-of-range blocks are skipped silently
+  a.cap = dims->capacity_tokens;
+  a.seq_len = seq_len;
+  a.batch = dims->batch;
+  a.hq = dims->num_q_heads;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.idx_stride = idx_stride;
+  a.part_stride = int32_t(n_splits);
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.blocks_per_split = int32_t(bps);
+  a.n_splits = int32_t(n_splits);
+  e = launch_decode(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
+  return ok();
+}
+
+}  // extern "C"

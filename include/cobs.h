@@ -174,6 +174,35 @@ COBS_API cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q,
                                float softmax_scale, float* out, float* lse,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free form of cobs_sparse_decode (this library's own addition; the
+ * method's description has no counterpart).  Same arguments and results, but
+ * there is no workspace argument: the split-K partial results and arrival
+ * counters go to a fixed 16 MiB array that the library itself places in every
+ * GPU's memory when it is loaded and keeps until the process exits.  It is for
+ * callers that cannot hand the library device memory of its own: code whose
+ * host framework owns every device allocation, code running where allocation
+ * is forbidden or too slow (a real-time or latency-critical loop, an
+ * allocator callback), or bindings without a device allocator at all.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     the arrival counters are cleared at the start of every call.  Calls
+ *     that overlap on the GPU (for example on two streams at once) race on
+ *     it and give wrong results: serialise them.
+ *   - Nothing is allocated or freed (no cudaMalloc / cudaFree / library
+ *     allocator calls).  A problem whose scratch would exceed 16 MiB
+ *     (batch * num_q_heads * splits * (head_dim + 2) * 4 bytes plus the
+ *     counters) is rejected with COBS_ERR_WORKSPACE.
+ *   - There is no status word: an out-of-range block index is skipped
+ *     without being reported. */
+COBS_API cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q,
+                                                 const void* k, const void* v,
+                                                 const int32_t* idx, const int32_t* n_sel,
+                                                 int32_t idx_stride, int64_t seq_len,
+                                                 float softmax_scale, float* out,
+                                                 float* lse, void* stream);
+
 /* Synchronise `stream`, copy the workspace status word to *device_status
  * (COBS_OK or the first device-side error code since the last read) and
  * clear it.  Returns CUDA on a failed copy, INVALID_ARG on bad pointers. */
