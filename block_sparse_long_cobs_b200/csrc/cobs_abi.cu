@@ -249,8 +249,8 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   a.top_k = top_k;
 
   // chunking: one wave of resident CTAs shared out over the (batch, kv-head)
-  // pairs; every chunk is a whole number of 16-record (32 for d = 64) stages
-  const int per_pass = 256 / (dims->head_dim / 8);
+  // pairs; every chunk is a whole number of stages (128 record rows each)
+  const int per_pass = select_blocks_per_stage(dims->rank);
   const int64_t n_cand = first_local - sink_end;
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
   int sms = device_sm_count();

@@ -81,8 +81,8 @@ struct StatsArgs {
 };
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
-size_t select_stage_bytes(int d, int rank);      // dynamic shared memory of the selection
 int select_ctas_per_sm(int d, int g, int rank);  // resident selection CTAs per SM
+int select_blocks_per_stage(int rank);           // whole records per selection stage
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 int decode_ctas_per_sm(int d, int g);             // resident decode CTAs per SM
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);

@@ -10,15 +10,18 @@
 // forced sets, ties to the lower block index, united with the sink blocks and
 // the local/tail blocks, written in ascending order.
 //
-// Phase 1, grid (chunk, kv-head, batch): each CTA streams the packed stats
-// records of one chunk of candidate blocks (contiguous in HBM) through a
-// 2-stage shared-memory ring, one bulk async copy (TMA engine) per stage of
-// 256 / (d/8) records.  The d/8 lanes of a block each read a 128-bit slice of
-// every row from shared memory and keep the same slice of all G queries in
-// registers (pre-scaled by 1/sqrt d); per row a reduce-scatter leaves one
-// head's dot product per lane, so the linear (row 0) and quadratic (rows
-// 1..r) terms accumulate without further shuffles.  Scores go to the
-// workspace (and to the optional output).
+// Phase 1, grid (chunk, kv-head, batch), 128 threads: the dot products of
+// every record row with the G queries form a dense contraction
+// [rows x d] . [d x G], done on the 5th-generation tensor cores.  A chunk's
+// records are contiguous rows of the stats array seen as a 2-d [rows][d] bf16
+// tensor; a 3-stage ring of TMA tile loads (128-byte swizzle, 128 rows per
+// stage = the largest whole number of records that fit) feeds one
+// tcgen05.mma chain per stage (M = 128 rows, N = 16 = G queries padded with
+// zero rows, K = d, fp32 accumulate in tensor memory).  The epilogue reads
+// the 128 x G products back (tcgen05.ld), scales by 1/sqrt d, keeps row 0 of
+// a record (linear term) and squares-and-halves rows 1..r (quadratic term),
+// sums them per block and per head, adds ln 64 and takes the log-sum-exp over
+// the heads.  Scores go to the workspace (and to the optional output).
 //
 // Phase 2, the last CTA of a (batch, kv-head) (atomic ticket, no spinning)
 // finds the k-th largest score with a 4 x 8-bit radix select over
@@ -27,11 +30,15 @@
 #include <cfloat>
 
 #include "device_common.cuh"
+#include "tcgen05.cuh"
 
 namespace cobs {
 namespace {
 
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 128;
+constexpr int kSelStages = 3;
+constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
+constexpr int kRankMax = 1024;    // candidate sets ranked directly (n^2 compares)
 
 // Order-preserving map float -> uint32 (larger float -> larger key); NaN lowest.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -91,135 +98,168 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
   return base + x - v;
 }
 
-template <int D, int G, int RMAX>
+template <int D, int G>
 __global__ void __launch_bounds__(kSelThreads)
-select_blocks_kernel(const SelectArgs a) {
-  constexpr int kLanes = D / 8;                  // lanes per block record
-  constexpr int kPerPass = kSelThreads / kLanes; // blocks per CTA pass
+select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs a) {
+  constexpr int kRegions = D / 64;                  // 64-column slabs of a row
+  constexpr int kStageBytes = kRegions * 128 * 128; // 128 rows x 128 B per slab
+  constexpr int kQBytes = kRegions * 16 * 128;      // 16 query rows x 128 B per slab
   const int tid = threadIdx.x;
+  const int warp = tid >> 5;
   const int lane = tid & 31;
   const int chunk = blockIdx.x;
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
   const int bh = b * a.hkv + kvh;
   const int rows = 1 + a.rank;
+  const int per_stage = kStageRows / rows;          // whole records per stage
 
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_tot[kSelThreads / 32];
   __shared__ uint32_t sh_u32[4];
   __shared__ int last_s;
   __shared__ int abort_s;
-  __shared__ __align__(8) uint64_t full[2];
-  extern __shared__ __align__(128) uint8_t stage_smem[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ __align__(8) uint64_t full[kSelStages];
+  __shared__ __align__(8) uint64_t mma_done[kSelStages];
+  __shared__ __align__(16) float contrib[kStageRows * 8];   // [row][head]
+  extern __shared__ uint8_t dyn_smem[];
+  // 1024-byte alignment for the swizzled tiles
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t* qtile = base;                            // [kRegions][16][128 B]
+  uint8_t* stage = base + kQBytes;                  // [kSelStages][kRegions][128][128 B]
 
   float* scores = a.scores_ws + int64_t(bh) * a.nb_cap;
 
   // ===================== phase 1: scores of this chunk =====================
-  // The chunk's records are contiguous; kPerPass of them at a time are staged
-  // in shared memory by one bulk async copy (2-stage ring, mbarrier-tracked).
   {
-    const int slice = lane % kLanes;
-    const float inv_sqrt_d = rsqrtf(float(D));
-    uint64_t qreg[G][4];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint4 w = *reinterpret_cast<const uint4*>(
-          a.q + (int64_t(b) * a.hq + kvh * G + h) * D + slice * 8);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float2 f = bf16x2_to_float2(ww[c]);
-        f.x *= inv_sqrt_d;
-        f.y *= inv_sqrt_d;
-        qreg[h][c] = pack2(f);
-      }
-    }
-    const float ln_n = logf(float(kBlock));
     const int c_lo = a.cand_begin + chunk * a.chunk_blocks;
     const int c_hi = min(a.cand_end, c_lo + a.chunk_blocks);
-    const int rec_elems = rows * D;
-    const int stage_elems = kPerPass * rec_elems;
-    uint16_t* stage = reinterpret_cast<uint16_t*>(stage_smem);
-    const int npass = c_hi > c_lo ? (c_hi - c_lo + kPerPass - 1) / kPerPass : 0;
-    const uint16_t* src = a.stats + int64_t(bh) * a.nb_cap * rec_elems;
+    const int npass = c_hi > c_lo ? (c_hi - c_lo + per_stage - 1) / per_stage : 0;
+    const int64_t row0 = (int64_t(bh) * a.nb_cap) * rows;   // first row of this pair
 
     if (tid == 0) {
-      mbar_init(&full[0], 1);
-      mbar_init(&full[1], 1);
+      for (int s2 = 0; s2 < kSelStages; ++s2) {
+        mbar_init(&full[s2], 1);
+        mbar_init(&mma_done[s2], 1);
+      }
       fence_barrier_init();
       abort_s = 0;
     }
+    if (warp == 0) tmem_alloc(&tmem_slot, 32);
+    tc_fence_before();
     __syncthreads();
-    auto issue = [&](int p) {  // thread 0 only
-      const int j0 = c_lo + p * kPerPass;
-      const int nb = min(kPerPass, c_hi - j0);
-      const uint32_t bytes = uint32_t(nb) * uint32_t(rec_elems) * 2u;
-      mbar_arrive_expect_tx(&full[p & 1], bytes);
-      bulk_g2s(stage + (p & 1) * stage_elems, src + int64_t(j0) * rec_elems, bytes, &full[p & 1]);
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    auto issue = [&](int p) {  // thread 0 only: TMA tiles of pass p
+      const int j0 = c_lo + p * per_stage;
+      const int y = int(row0 + int64_t(j0) * rows);
+      uint8_t* dst = stage + (p % kSelStages) * kStageBytes;
+      // the box is always kStageRows rows; rows past the chunk are ignored
+      mbar_arrive_expect_tx(&full[p % kSelStages], uint32_t(kRegions) * kStageRows * 128);
+      for (int reg = 0; reg < kRegions; ++reg)
+        tma_load_2d(dst + reg * 128 * 128, &smap, reg * 64, y, &full[p % kSelStages]);
     };
+    // start the record stream first, build the query operand while it flies
     if (tid == 0) {
-      for (int p = 0; p < 2 && p < npass; ++p) issue(p);
+      for (int p = 0; p < kSelStages && p < npass; ++p) issue(p);
     }
+    // queries as the B operand: row n < G is query head kvh*G + n, rows G..15
+    // zero; 16-byte chunks written straight to their swizzled positions
+    for (int e = tid; e < kRegions * 16 * 8; e += kSelThreads) {
+      const int reg = e / (16 * 8), n = (e / 8) % 16, c = e % 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (n < G)
+        v = *reinterpret_cast<const uint4*>(a.q + (int64_t(b) * a.hq + kvh * G + n) * D +
+                                            reg * 64 + c * 8);
+      *reinterpret_cast<uint4*>(qtile + reg * 16 * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    const float inv_sqrt_d = rsqrtf(float(D));
+    const float ln_n = logf(float(kBlock));
+    constexpr uint32_t idesc = umma_idesc_bf16(128, 16);
+    // thread 0: wait for the tiles of pass p and issue its MMA into
+    // accumulator p & 1, completion signalled on mma_done[p % stages]
+    auto issue_mma = [&](int p) -> bool {
+      const int st = p % kSelStages;
+      if (!mbar_wait_bounded(&full[st], (p / kSelStages) & 1, a.status)) return false;
+      tc_fence_after();
+      const uint32_t abase = smem_addr(stage + st * kStageBytes);
+      const uint32_t bbase = smem_addr(qtile);
+      const uint32_t acc = tmem + uint32_t(16 * (p & 1));
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+        const uint64_t bd = umma_desc_sw128(bbase + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+        umma_bf16(acc, ad, bd, idesc, ks > 0 ? 1u : 0u);
+      }
+      umma_commit(&mma_done[st]);
+      return true;
+    };
+    if (tid == 0 && npass > 0 && !issue_mma(0)) abort_s = 1;
     for (int p = 0; p < npass; ++p) {
-      const uint32_t parity = (p >> 1) & 1;
-      if (tid == 0) {
-        if (!mbar_wait_bounded(&full[p & 1], parity, a.status)) {
-          abort_s = 1;
-          if (p + 1 < npass) mbar_wait_bounded(&full[(p + 1) & 1], ((p + 1) >> 1) & 1, a.status);
-        }
+      const int st = p % kSelStages;
+      const uint32_t parity = (p / kSelStages) & 1;
+      const uint32_t acc = tmem + uint32_t(16 * (p & 1));
+      if (tid == 0 && !abort_s) {
+        if (!mbar_wait_bounded(&mma_done[st], parity, a.status)) abort_s = 1;
       }
       __syncthreads();
       if (abort_s) break;
-      if (tid != 0) (void)mbar_try_wait(&full[p & 1], parity);  // acquire the copy
-      const int jj = tid / kLanes;
-      const int j = c_lo + p * kPerPass + jj;
-      const bool valid = j < c_hi;
-      const uint16_t* rec = stage + (p & 1) * stage_elems + jj * rec_elems + slice * 8;
-      uint4 w[RMAX + 1];
-#pragma unroll
-      for (int r = 0; r <= RMAX; ++r) {
-        w[r] = make_uint4(0, 0, 0, 0);
-        if (r < rows && valid) w[r] = *reinterpret_cast<const uint4*>(rec + r * D);
+      if (tid != 0) (void)mbar_try_wait(&mma_done[st], parity);
+      tc_fence_after();
+      if (tid == 0) {
+        // the stage of pass p has been read by its MMA: refill it, then start
+        // the next pass's MMA (other accumulator) so it runs under this epilogue
+        if (p + kSelStages < npass) issue(p + kSelStages);
+        if (p + 1 < npass && !issue_mma(p + 1)) abort_s = 1;
       }
-      float s = 0.f;
-      int head = 0;
+
+      // epilogue: row = warp * 32 + lane of this stage
+      const int j0 = c_lo + p * per_stage;
+      const int nb = min(per_stage, c_hi - j0);
+      float v[16];
+      tmem_ld16(acc + (uint32_t(warp * 32) << 16), v);
+      const int row = warp * 32 + lane;
+      const int rho = row % rows;
 #pragma unroll
-      for (int r = 0; r <= RMAX; ++r) {
-        if (r < rows) {
-          const uint32_t ww[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
-          uint64_t k2[4];
+      for (int h = 0; h < G; ++h) {
+        const float x = v[h] * inv_sqrt_d;
+        contrib[row * 8 + h] = (rho == 0) ? x : 0.5f * x * x;
+      }
+      tc_fence_before();
+      __syncthreads();
+      // per block and head: sum of the record's rows, then LSE over the heads
+      // (all threads take part in the shuffles; only valid ones write)
+      for (int t0 = 0; t0 < per_stage * G; t0 += kSelThreads) {
+        const int t = t0 + tid;
+        const int jj = t / G, h = t % G;
+        const bool valid = jj < nb;
+        float sacc = 0.f;
+        if (valid)
+          for (int k2 = 0; k2 < rows; ++k2) sacc += contrib[(jj * rows + k2) * 8 + h];
+        const float sh = sacc + ln_n;
+        float mx = sh;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) k2[c] = pack2(bf16x2_to_float2(ww[c]));
-          float part[G];
+        for (int m = G / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m, G));
+        float e = __expf(sh - mx);
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            uint64_t acc = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ffma2(acc, k2[c], qreg[h][c]);
-            const float2 f = unpack2(acc);
-            part[h] = f.x + f.y;
-          }
-          const float x = reduce_scatter_sel<G, kLanes>(part, lane, head);
-          s += (r == 0) ? x : 0.5f * x * x;
+        for (int m = G / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m, G);
+        if (valid && h == 0) {
+          const float S = mx + __logf(e);
+          scores[j0 + jj] = S;
+          if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
         }
       }
-      s += ln_n;
-      // group log-sum-exp over the G heads held by the kLanes lanes of a block
-      float mx = s;
-#pragma unroll
-      for (int m = kLanes / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-      constexpr int kDup = (kLanes / G) > 0 ? kLanes / G : 1;  // lanes sharing a head
-      float e = ((slice & (kDup - 1)) == 0) ? __expf(s - mx) : 0.f;
-#pragma unroll
-      for (int m = kLanes / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m);
-      const float S = mx + __logf(e);
-      if (valid && slice == 0) {
-        scores[j] = S;
-        if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j] = S;
-      }
-      __syncthreads();  // stage (p & 1) consumed
-      if (tid == 0 && p + 2 < npass) issue(p + 2);
+      __syncthreads();   // contrib buffer and accumulator reused next pass
     }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 32);
   }
 
   // ===================== arrival: last CTA of (b, kv-head) selects =========
@@ -238,15 +278,48 @@ select_blocks_kernel(const SelectArgs a) {
   const int nbs = a.seq_len_blocks;
   int k = a.top_k < n_cand ? a.top_k : n_cand;
 
+  // order keys of the candidates, staged in shared memory when they fit
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(stage);
+  const bool keys_in_smem = n_cand <= kSelStages * kStageBytes / 4;
+  if (keys_in_smem)
+    for (int j = tid; j < n_cand; j += kSelThreads) skeys[j] = order_key(__ldcg(scores + c0 + j));
+  __syncthreads();
+  auto key_of = [&](int j) -> uint32_t {   // j in [c0, c1)
+    return keys_in_smem ? skeys[j - c0] : order_key(__ldcg(scores + j));
+  };
+
+  // ---- small candidate sets: exact ranks in one pass ------------------------
+  // rank(j) = #{keys greater} + #{equal keys at a lower index}; the top k are
+  // the candidates with rank < k.  Marked in `chosen_s` (one byte per block).
+  const bool partial = (k > 0 && k < n_cand);
+  const bool by_rank = partial && keys_in_smem && n_cand <= kRankMax;
+  uint8_t* chosen_s = reinterpret_cast<uint8_t*>(stage) + kRankMax * 4;
+  if (by_rank) {
+    for (int jj = tid; jj < n_cand; jj += kSelThreads) {
+      const uint32_t kj = skeys[jj];
+      int rank = 0;
+      int i = 0;
+      for (; i + 4 <= n_cand; i += 4) {
+        const uint4 k4 = *reinterpret_cast<const uint4*>(skeys + i);
+        rank += (k4.x > kj) | ((k4.x == kj) & (i + 0 < jj));
+        rank += (k4.y > kj) | ((k4.y == kj) & (i + 1 < jj));
+        rank += (k4.z > kj) | ((k4.z == kj) & (i + 2 < jj));
+        rank += (k4.w > kj) | ((k4.w == kj) & (i + 3 < jj));
+      }
+      for (; i < n_cand; ++i) rank += (skeys[i] > kj) | ((skeys[i] == kj) & (i < jj));
+      chosen_s[jj] = rank < k ? 1 : 0;
+    }
+    __syncthreads();
+  }
+
   // ---- radix select of the k-th largest key among the candidates ----------
   uint32_t prefix = 0, mask = 0, krem = uint32_t(k);
-  const bool partial = (k > 0 && k < n_cand);
-  if (partial) {
+  if (partial && !by_rank) {
     for (int shift = 24; shift >= 0; shift -= 8) {
-      hist[tid] = 0;
+      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
       for (int j = c0 + tid; j < c1; j += kSelThreads) {
-        const uint32_t key = order_key(__ldcg(scores + j));
+        const uint32_t key = key_of(j);
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
@@ -292,9 +365,9 @@ select_blocks_kernel(const SelectArgs a) {
   const int j0 = min(nbs, tid * per), j1 = min(nbs, j0 + per);
   auto is_forced = [&](int j) { return j < a.sink_end || j >= a.first_local; };
   uint32_t n_eq = 0;
-  if (partial) {
+  if (partial && !by_rank) {
     for (int j = j0; j < j1; ++j)
-      if (j >= c0 && j < c1 && order_key(__ldcg(scores + j)) == prefix) ++n_eq;
+      if (j >= c0 && j < c1 && key_of(j) == prefix) ++n_eq;
   }
   uint32_t tot_unused;
   uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, tot_unused);
@@ -302,7 +375,8 @@ select_blocks_kernel(const SelectArgs a) {
     if (is_forced(j)) return true;
     if (j < c0 || j >= c1) return false;
     if (!partial) return k > 0;  // k == n_cand: everything; k == 0: nothing
-    const uint32_t key = order_key(__ldcg(scores + j));
+    if (by_rank) return chosen_s[j - c0] != 0;
+    const uint32_t key = key_of(j);
     if (key > prefix) return true;
     if (key == prefix) return (eq_seen++) < krem;
     return false;
@@ -331,23 +405,32 @@ select_blocks_kernel(const SelectArgs a) {
   }
 }
 
-template <int D, int G, int R>
+template <int D>
+constexpr size_t dyn_smem_bytes() {
+  return 1024 + size_t(D / 64) * 16 * 128 + size_t(kSelStages) * (D / 64) * 128 * 128;
+}
+
+template <int D, int G>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
-  auto kern = select_blocks_kernel<D, G, R>;
-  const size_t smem = select_stage_bytes(a.d, a.rank);
+  auto kern = select_blocks_kernel<D, G>;
+  constexpr size_t smem = dyn_smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
+  CUtensorMap map;
+  const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
+  e = make_bf16_tensor_map_sw128(&map, a.stats, D, total_rows, kStageRows);
+  if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.hkv, a.batch);
-  kern<<<grid, kSelThreads, smem, s>>>(a);
+  kern<<<grid, kSelThreads, smem, s>>>(map, a);
   return cudaGetLastError();
 }
 
-template <int D, int G, int R>
-int occupancy_t(int rank) {
+template <int D, int G>
+int occupancy_t() {
   int n = 0;
-  auto kern = select_blocks_kernel<D, G, R>;
-  const size_t smem = select_stage_bytes(D, rank);
+  auto kern = select_blocks_kernel<D, G>;
+  constexpr size_t smem = dyn_smem_bytes<D>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return 1;
@@ -356,52 +439,34 @@ int occupancy_t(int rank) {
   return n > 0 ? n : 1;
 }
 
-template <int D, int G>
-int occupancy_rank(int rank) {
-  if (rank == 0) return occupancy_t<D, G, 0>(rank);
-  if (rank <= 4) return occupancy_t<D, G, 4>(rank);
-  if (rank <= 8) return occupancy_t<D, G, 8>(rank);
-  return occupancy_t<D, G, 16>(rank);
-}
-
-template <int D, int G>
-cudaError_t dispatch_rank(const SelectArgs& a, cudaStream_t s) {
-  if (a.rank == 0) return launch_t<D, G, 0>(a, s);
-  if (a.rank <= 4) return launch_t<D, G, 4>(a, s);
-  if (a.rank <= 8) return launch_t<D, G, 8>(a, s);
-  return launch_t<D, G, 16>(a, s);
-}
-
 template <int D>
 cudaError_t dispatch_group(const SelectArgs& a, cudaStream_t s) {
   switch (a.hq / a.hkv) {
-    case 1: return dispatch_rank<D, 1>(a, s);
-    case 2: return dispatch_rank<D, 2>(a, s);
-    case 4: return dispatch_rank<D, 4>(a, s);
-    case 8: return dispatch_rank<D, 8>(a, s);
+    case 1: return launch_t<D, 1>(a, s);
+    case 2: return launch_t<D, 2>(a, s);
+    case 4: return launch_t<D, 4>(a, s);
+    case 8: return launch_t<D, 8>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int D>
-int occupancy_group(int g, int rank) {
+int occupancy_group(int g) {
   switch (g) {
-    case 1: return occupancy_rank<D, 1>(rank);
-    case 2: return occupancy_rank<D, 2>(rank);
-    case 4: return occupancy_rank<D, 4>(rank);
-    default: return occupancy_rank<D, 8>(rank);
+    case 1: return occupancy_t<D, 1>();
+    case 2: return occupancy_t<D, 2>();
+    case 4: return occupancy_t<D, 4>();
+    default: return occupancy_t<D, 8>();
   }
 }
 
 }  // namespace
 
-size_t select_stage_bytes(int d, int rank) {
-  return size_t(2) * (kSelThreads / (d / 8)) * size_t(1 + rank) * d * 2;
+int select_ctas_per_sm(int d, int g, int /*rank*/) {
+  return d == 64 ? occupancy_group<64>(g) : occupancy_group<128>(g);
 }
 
-int select_ctas_per_sm(int d, int g, int rank) {
-  return d == 64 ? occupancy_group<64>(g, rank) : occupancy_group<128>(g, rank);
-}
+int select_blocks_per_stage(int rank) { return kStageRows / (1 + rank); }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);
