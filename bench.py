@@ -51,7 +51,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--steps", type=int, default=5000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["cobs", "reference"], default="cobs")
     p.add_argument("--workload", default="batched_needles_32k")
@@ -125,7 +125,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -385,6 +385,15 @@ def run_cobs(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
+    # keep the GPU busy while nvidia-smi starts up (~0.2 s), so that its
+    # samples all fall under load
+    pre = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(2)]
+    t_pre = time.perf_counter()
+    while time.perf_counter() - t_pre < 0.3:
+        for _ in range(50):
+            flush.zero_()
+            step(pre[0])
+        torch.cuda.synchronize(dev)
     for i in range(args.steps):
         flush.zero_()
         step(evs[i])

@@ -115,6 +115,41 @@ int device_sm_count() {
   return n;
 }
 
+DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride) {
+  DecodePlan P{};
+  int sms = device_sm_count();
+  if (sms <= 0) sms = 148;
+  if (d == 128) {
+    // equal contiguous ranges of block-list slots, one wave of resident CTAs
+    const int64_t slots = pairs * idx_stride;
+    const int64_t resident = int64_t(sms) * decode_tc_ctas_per_sm(g);
+    int64_t R = ceil_div(slots, resident);
+    if (R > decode_tc_max_slots()) R = decode_tc_max_slots();
+    if (R < 1) R = 1;
+    P.slots_per_cta = int32_t(R);
+    P.n_ctas = int32_t(ceil_div(slots, R));
+    // a pair's idx_stride slots meet at most floor((S + R - 2) / R) + 1 ranges
+    int64_t rows = (int64_t(idx_stride) + R - 2) / R + 1;
+    if (rows > idx_stride) rows = idx_stride;
+    P.part_rows = int32_t(rows);
+  } else {
+    // one wave of resident CTAs shared out over the (batch, kv-head) pairs
+    const int64_t resident = int64_t(sms) * decode_d64_ctas_per_sm(g);
+    int64_t splits = resident / pairs;
+    if (splits > idx_stride) splits = idx_stride;
+    if (splits < 1) splits = 1;
+    const int64_t bps = ceil_div(idx_stride, splits);
+    P.blocks_per_split = int32_t(bps);
+    P.n_splits = int32_t(ceil_div(idx_stride, bps));
+    P.part_rows = P.n_splits;
+  }
+  return P;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+  return a.d == 128 ? launch_decode_tc(a, stream) : launch_decode_d64(a, stream);
+}
+
 }  // namespace cobs
 
 using namespace cobs;
@@ -288,6 +323,8 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
     return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
                 (long long)seq_len);
   if (idx_stride < 1) return fail(COBS_ERR_INVALID_ARG, "idx_stride must be >= 1");
+  if (int64_t(dims->batch) * dims->num_kv_heads * idx_stride >= (int64_t(1) << 31))
+    return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * idx_stride must be < 2^31");
   if (!(std::isfinite(softmax_scale)) || softmax_scale <= 0.f)
     return fail(COBS_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
   const WorkspaceLayout L = layout(dims, idx_stride);
@@ -312,21 +349,14 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.idx_stride = idx_stride;
-  a.part_stride = idx_stride;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-
-  // splits: one wave of resident CTAs shared out over the (batch, kv-head) pairs
-  const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
-  int sms = device_sm_count();
-  if (sms <= 0) sms = 148;
-  const int resident =
-      sms * decode_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads);
-  int64_t splits = resident / pairs;
-  if (splits > idx_stride) splits = idx_stride;
-  if (splits < 1) splits = 1;
-  const int64_t bps = ceil_div(idx_stride, splits);
-  a.blocks_per_split = int32_t(bps);
-  a.n_splits = int32_t(ceil_div(idx_stride, bps));
+  const DecodePlan P = plan_decode(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
+                                   int64_t(dims->batch) * dims->num_kv_heads, idx_stride);
+  a.part_stride = idx_stride;   // the workspace holds idx_stride >= P.part_rows rows
+  a.n_splits = P.n_splits;
+  a.blocks_per_split = P.blocks_per_split;
+  a.slots_per_cta = P.slots_per_cta;
+  a.n_ctas = P.n_ctas;
 
   cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
@@ -409,24 +439,19 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
     return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
                 (long long)seq_len);
   if (idx_stride < 1) return fail(COBS_ERR_INVALID_ARG, "idx_stride must be >= 1");
+  if (int64_t(dims->batch) * dims->num_kv_heads * idx_stride >= (int64_t(1) << 31))
+    return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * idx_stride must be < 2^31");
   if (!(std::isfinite(softmax_scale)) || softmax_scale <= 0.f)
     return fail(COBS_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
 
-  // split count exactly as in cobs_sparse_decode; the partials are packed with
-  // one row per split actually launched
+  // work split exactly as in cobs_sparse_decode; the partials are packed with
+  // as many rows per query head as that split produces
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
-  int sms = device_sm_count();
-  if (sms <= 0) sms = 148;
-  const int resident =
-      sms * decode_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads);
-  int64_t splits = resident / pairs;
-  if (splits > idx_stride) splits = idx_stride;
-  if (splits < 1) splits = 1;
-  const int64_t bps = ceil_div(idx_stride, splits);
-  const int64_t n_splits = ceil_div(idx_stride, bps);
+  const DecodePlan P = plan_decode(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
+                                   pairs, idx_stride);
   const size_t tickets_bytes = align256(size_t(pairs) * 4);
   const size_t need = tickets_bytes + size_t(dims->batch) * dims->num_q_heads *
-                                          size_t(n_splits) * (size_t(dims->head_dim) + 2) * 4;
+                                          size_t(P.part_rows) * (size_t(dims->head_dim) + 2) * 4;
   if (need > kFixedScratchBytes)
     return fail(COBS_ERR_WORKSPACE,
                 "this decode needs %zu bytes of scratch, above the library's fixed %zu; use "
@@ -460,10 +485,12 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.idx_stride = idx_stride;
-  a.part_stride = int32_t(n_splits);
+  a.part_stride = P.part_rows;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.blocks_per_split = int32_t(bps);
-  a.n_splits = int32_t(n_splits);
+  a.n_splits = P.n_splits;
+  a.blocks_per_split = P.blocks_per_split;
+  a.slots_per_cta = P.slots_per_cta;
+  a.n_ctas = P.n_ctas;
   e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
   return ok();

@@ -63,10 +63,19 @@ struct DecodeArgs {
   int64_t seq_len;
   int32_t batch, hq, hkv, d;
   int32_t idx_stride;
-  int32_t part_stride;    // n_sel_max of the workspace (splits dimension)
-  int32_t n_splits;       // CTAs per (b, kv-head)
+  int32_t part_stride;    // partial rows per query head (>= splits / segments of a pair)
+  int32_t n_splits;       // head_dim 64: CTAs per (b, kv-head)
   int32_t blocks_per_split;
+  int32_t slots_per_cta;  // head_dim 128: block-list slots per CTA (<= 30)
+  int32_t n_ctas;         // head_dim 128: grid size
   float scale_log2;       // softmax_scale * log2(e)
+};
+
+// Work split of one decode launch and the partial rows per query head it needs.
+struct DecodePlan {
+  int32_t n_splits, blocks_per_split;   // head_dim 64 kernel
+  int32_t slots_per_cta, n_ctas;        // head_dim 128 kernel
+  int32_t part_rows;
 };
 
 // Arguments of the block-statistics kernel.
@@ -83,8 +92,13 @@ struct StatsArgs {
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 int select_ctas_per_sm(int d, int g, int rank);  // resident selection CTAs per SM
 int select_blocks_per_stage(int rank);           // whole records per selection stage
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
-int decode_ctas_per_sm(int d, int g);             // resident decode CTAs per SM
+DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);  // either kernel
+cudaError_t launch_decode_d64(const DecodeArgs& a, cudaStream_t stream);
+int decode_d64_ctas_per_sm(int g);
+cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
+int decode_tc_ctas_per_sm(int g);
+int decode_tc_max_slots();
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);
 
 int device_sm_count();

@@ -1,4 +1,6 @@
-// Split-K flash-decode over the selected KV blocks, with a log-sum-exp merge.
+// Split-K flash-decode over the selected KV blocks, with a log-sum-exp merge:
+// the head_dim 64 kernel on the CUDA cores (head_dim 128 runs on the tensor
+// cores, decode_tc.cu).
 //
 // Exact attention (glossary "LLMアテンション機構": softmax(q K^T / sqrt d) V,
 // grouped-query heads sharing one K/V head) restricted to the tokens of the
@@ -375,35 +377,28 @@ int occupancy_t() {
   return n > 0 ? n : 1;
 }
 
-template <int D>
 int occupancy_group(int g) {
   switch (g) {
-    case 1: return occupancy_t<D, 1>();
-    case 2: return occupancy_t<D, 2>();
-    case 4: return occupancy_t<D, 4>();
-    default: return occupancy_t<D, 8>();
-  }
-}
-
-template <int D>
-cudaError_t dispatch_group(const DecodeArgs& a, cudaStream_t s) {
-  switch (a.hq / a.hkv) {
-    case 1: return launch_decode_t<D, 1>(a, s);
-    case 2: return launch_decode_t<D, 2>(a, s);
-    case 4: return launch_decode_t<D, 4>(a, s);
-    case 8: return launch_decode_t<D, 8>(a, s);
-    default: return cudaErrorInvalidValue;
+    case 1: return occupancy_t<64, 1>();
+    case 2: return occupancy_t<64, 2>();
+    case 4: return occupancy_t<64, 4>();
+    default: return occupancy_t<64, 8>();
   }
 }
 
 }  // namespace
 
-int decode_ctas_per_sm(int d, int g) {
-  return d == 64 ? occupancy_group<64>(g) : occupancy_group<128>(g);
-}
+int decode_d64_ctas_per_sm(int g) { return occupancy_group(g); }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);
+cudaError_t launch_decode_d64(const DecodeArgs& a, cudaStream_t stream) {
+  if (a.d != 64) return cudaErrorInvalidValue;
+  switch (a.hq / a.hkv) {
+    case 1: return launch_decode_t<64, 1>(a, stream);
+    case 2: return launch_decode_t<64, 2>(a, stream);
+    case 4: return launch_decode_t<64, 4>(a, stream);
+    case 8: return launch_decode_t<64, 8>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace cobs

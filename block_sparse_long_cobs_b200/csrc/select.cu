@@ -38,7 +38,6 @@ namespace {
 constexpr int kSelThreads = 128;
 constexpr int kSelStages = 3;
 constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
-constexpr int kRankMax = 1024;    // candidate sets ranked directly (n^2 compares)
 
 // Order-preserving map float -> uint32 (larger float -> larger key); NaN lowest.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -118,7 +117,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
   __shared__ uint32_t warp_tot[kSelThreads / 32];
   __shared__ uint32_t sh_u32[4];
   __shared__ int last_s;
-  __shared__ int abort_s;
   __shared__ uint32_t tmem_slot;
   __shared__ __align__(8) uint64_t full[kSelStages];
   __shared__ __align__(8) uint64_t mma_done[kSelStages];
@@ -145,7 +143,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
         mbar_init(&mma_done[s2], 1);
       }
       fence_barrier_init();
-      abort_s = 0;
     }
     if (warp == 0) tmem_alloc(&tmem_slot, 32);
     tc_fence_before();
@@ -153,7 +150,10 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
+    int n_issued = 0;          // thread 0: passes whose TMA copies were issued
+    int n_mma = 0;             // thread 0: passes whose MMA was issued
     auto issue = [&](int p) {  // thread 0 only: TMA tiles of pass p
+      n_issued = p + 1;
       const int j0 = c_lo + p * per_stage;
       const int y = int(row0 + int64_t(j0) * rows);
       uint8_t* dst = stage + (p % kSelStages) * kStageBytes;
@@ -198,25 +198,28 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
         umma_bf16(acc, ad, bd, idesc, ks > 0 ? 1u : 0u);
       }
       umma_commit(&mma_done[st]);
+      n_mma = p + 1;
       return true;
     };
-    if (tid == 0 && npass > 0 && !issue_mma(0)) abort_s = 1;
+    // thread 0 alone waits; the decision to stop is shared through the
+    // barrier's OR so that every thread leaves the loop at the same point
+    bool fail = false;
+    if (tid == 0 && npass > 0 && !issue_mma(0)) fail = true;
     for (int p = 0; p < npass; ++p) {
       const int st = p % kSelStages;
       const uint32_t parity = (p / kSelStages) & 1;
       const uint32_t acc = tmem + uint32_t(16 * (p & 1));
-      if (tid == 0 && !abort_s) {
-        if (!mbar_wait_bounded(&mma_done[st], parity, a.status)) abort_s = 1;
+      if (tid == 0 && !fail) {
+        if (!mbar_wait_bounded(&mma_done[st], parity, a.status)) fail = true;
       }
-      __syncthreads();
-      if (abort_s) break;
+      if (__syncthreads_or(fail)) break;
       if (tid != 0) (void)mbar_try_wait(&mma_done[st], parity);
       tc_fence_after();
       if (tid == 0) {
         // the stage of pass p has been read by its MMA: refill it, then start
         // the next pass's MMA (other accumulator) so it runs under this epilogue
         if (p + kSelStages < npass) issue(p + kSelStages);
-        if (p + 1 < npass && !issue_mma(p + 1)) abort_s = 1;
+        if (p + 1 < npass && !issue_mma(p + 1)) fail = true;
       }
 
       // epilogue: row = warp * 32 + lane of this stage
@@ -257,6 +260,15 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
       }
       __syncthreads();   // contrib buffer and accumulator reused next pass
     }
+    if (tid == 0 && fail) {
+      // let the copies and the MMA still in flight land before TMEM is freed
+      // and the CTA leaves (each wait bounded)
+      for (int p = n_issued > kSelStages ? n_issued - kSelStages : 0; p < n_issued; ++p)
+        (void)mbar_wait_bounded(&full[p % kSelStages], (p / kSelStages) & 1, a.status);
+      if (n_mma > 0)
+        (void)mbar_wait_bounded(&mma_done[(n_mma - 1) % kSelStages],
+                                ((n_mma - 1) / kSelStages) & 1, a.status);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 32);
@@ -288,33 +300,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
     return keys_in_smem ? skeys[j - c0] : order_key(__ldcg(scores + j));
   };
 
-  // ---- small candidate sets: exact ranks in one pass ------------------------
-  // rank(j) = #{keys greater} + #{equal keys at a lower index}; the top k are
-  // the candidates with rank < k.  Marked in `chosen_s` (one byte per block).
   const bool partial = (k > 0 && k < n_cand);
-  const bool by_rank = partial && keys_in_smem && n_cand <= kRankMax;
-  uint8_t* chosen_s = reinterpret_cast<uint8_t*>(stage) + kRankMax * 4;
-  if (by_rank) {
-    for (int jj = tid; jj < n_cand; jj += kSelThreads) {
-      const uint32_t kj = skeys[jj];
-      int rank = 0;
-      int i = 0;
-      for (; i + 4 <= n_cand; i += 4) {
-        const uint4 k4 = *reinterpret_cast<const uint4*>(skeys + i);
-        rank += (k4.x > kj) | ((k4.x == kj) & (i + 0 < jj));
-        rank += (k4.y > kj) | ((k4.y == kj) & (i + 1 < jj));
-        rank += (k4.z > kj) | ((k4.z == kj) & (i + 2 < jj));
-        rank += (k4.w > kj) | ((k4.w == kj) & (i + 3 < jj));
-      }
-      for (; i < n_cand; ++i) rank += (skeys[i] > kj) | ((skeys[i] == kj) & (i < jj));
-      chosen_s[jj] = rank < k ? 1 : 0;
-    }
-    __syncthreads();
-  }
 
   // ---- radix select of the k-th largest key among the candidates ----------
   uint32_t prefix = 0, mask = 0, krem = uint32_t(k);
-  if (partial && !by_rank) {
+  if (partial) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
@@ -365,7 +355,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
   const int j0 = min(nbs, tid * per), j1 = min(nbs, j0 + per);
   auto is_forced = [&](int j) { return j < a.sink_end || j >= a.first_local; };
   uint32_t n_eq = 0;
-  if (partial && !by_rank) {
+  if (partial) {
     for (int j = j0; j < j1; ++j)
       if (j >= c0 && j < c1 && key_of(j) == prefix) ++n_eq;
   }
@@ -375,7 +365,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
     if (is_forced(j)) return true;
     if (j < c0 || j >= c1) return false;
     if (!partial) return k > 0;  // k == n_cand: everything; k == 0: nothing
-    if (by_rank) return chosen_s[j - c0] != 0;
     const uint32_t key = key_of(j);
     if (key > prefix) return true;
     if (key == prefix) return (eq_seen++) < krem;

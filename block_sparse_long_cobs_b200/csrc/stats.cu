@@ -190,6 +190,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     for (int reg = 0; reg < S::kRegions; ++reg)
       tma_load_2d(ktile + reg * S::kRegionBytes, &kmap, reg * 64, y, &bars[0]);
     bool ok = mbar_wait_bounded(&bars[0], 0, a.status);
+    if (!ok) (void)mbar_wait_bounded(&bars[0], 0, a.status);  // copy still in flight
     if (ok) {
       tc_fence_after();
       constexpr uint32_t idesc = umma_idesc_bf16(128, 64);
@@ -202,6 +203,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       }
       umma_commit(&bars[1]);
       ok = mbar_wait_bounded(&bars[1], 0, a.status);
+      if (!ok) (void)mbar_wait_bounded(&bars[1], 0, a.status);  // MMA still running
     }
     *abort_s = ok ? 0u : 1u;
   }

@@ -40,4 +40,20 @@ cudaError_t make_bf16_tensor_map_sw128(CUtensorMap* map, const void* base, int c
   return cudaSuccess;
 }
 
+cudaError_t make_bf16_tensor_map_3d_sw128(CUtensorMap* map, const void* base, int cols,
+                                          uint64_t rows, uint64_t depth,
+                                          uint64_t depth_stride_bytes, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {cuuint64_t(cols), cuuint64_t(rows), cuuint64_t(depth)};
+  const cuuint64_t strides[2] = {cuuint64_t(cols) * 2, cuuint64_t(depth_stride_bytes)};
+  const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 }  // namespace cobs
