@@ -63,6 +63,8 @@ def parse_args():
                    help="time budget of the CPU-oracle baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="enqueue the timed steps call by call instead of replaying CUDA graphs")
     p.add_argument("--stats-stream", choices=["side", "same"], default="side",
                    help="run the completed block's stats build on a forked side stream "
                         "(joined before the step ends) or in line before the selection")
@@ -319,7 +321,16 @@ def run_cobs(args, w, rank, world, local_rank):
     lse = torch.zeros((w.batch, w.q_heads), dtype=torch.float32, device=dev)
     ws_bytes = cb.cobs_workspace_bytes(dims, w.top_k, w.sink_blocks, w.local_tokens)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def flush():
+        # write a buffer of 2x L2, then read another one: the dirty lines the
+        # write leaves are written back here, outside the timed step, and the
+        # step starts from a cold, clean L2
+        flush_w.zero_()
+        torch.amax(flush_r, dim=0, keepdim=True, out=flush_sink)
     stream = torch.cuda.current_stream(dev)
     cb.cobs_workspace_init(ws, ws_bytes, stream)
     scale = 1.0 / math.sqrt(w.head_dim)
@@ -335,14 +346,15 @@ def run_cobs(args, w, rank, world, local_rank):
     side = torch.cuda.Stream(dev) if args.stats_stream == "side" else None
     fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
 
-    def step(ev=None):
+    def step(ev=None, st=None):
         # ev: [step start, selection start, decode start, step end, stats start, stats end]
+        st = stream if st is None else st
         if ev is not None:
-            ev[0].record(stream)
+            ev[0].record(st)
         if side is not None:
             # the block completed at this step lies in the local window, so the
             # selection below never reads the record being written
-            fork_ev.record(stream)
+            fork_ev.record(st)
             side.wait_event(fork_ev)
             if ev is not None:
                 ev[4].record(side)
@@ -352,25 +364,25 @@ def run_cobs(args, w, rank, world, local_rank):
             join_ev.record(side)
         else:
             if ev is not None:
-                ev[4].record(stream)
-            cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, stream)
+                ev[4].record(st)
+            cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, st)
             if ev is not None:
-                ev[5].record(stream)
+                ev[5].record(st)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(st)
         cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
-                              w.local_tokens, idx, nsm, n_sel, None, ws, ws_bytes, stream)
+                              w.local_tokens, idx, nsm, n_sel, None, ws, ws_bytes, st)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(st)
         cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
-                              ws, ws_bytes, stream)
+                              ws, ws_bytes, st)
         if side is not None:
-            stream.wait_event(join_ev)
+            st.wait_event(join_ev)
         if ev is not None:
-            ev[3].record(stream)
+            ev[3].record(st)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize(dev)
     status = cb.cobs_read_device_status(ws, ws_bytes, stream)
@@ -379,7 +391,36 @@ def run_cobs(args, w, rank, world, local_rank):
     sel_counts = n_sel.cpu().numpy()
     n_sel_mean = float(sel_counts.mean())
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    # timed region: the steps are replayed from CUDA graphs of g_steps steps
+    # (L2 flush, stats, selection, decode and the per-step events captured),
+    # so that host launch overhead stays out of the device timing; without
+    # graphs the same steps are enqueued one call at a time
+    g_steps = max(d for d in range(1, min(50, args.steps) + 1) if args.steps % d == 0)
+    if args.no_graph:
+        g_steps = 1
+    # external: recorded inside a graph capture as event-record nodes
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+           for _ in range(g_steps)]
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cs = torch.cuda.current_stream(dev)
+            for i in range(g_steps):
+                flush()
+                step(evs[i], cs)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+    sums = [0.0, 0.0, 0.0, 0.0]   # stats, select, decode, step (ms)
+
+    def harvest():
+        for e in evs:
+            sums[0] += e[4].elapsed_time(e[5])
+            sums[1] += e[1].elapsed_time(e[2])
+            sums[2] += e[2].elapsed_time(e[3])
+            sums[3] += e[0].elapsed_time(e[3])
+
     clocks = ClockSampler(local_rank)
     if world > 1:
         dist.barrier()
@@ -387,24 +428,27 @@ def run_cobs(args, w, rank, world, local_rank):
     clocks.start()
     # keep the GPU busy while nvidia-smi starts up (~0.2 s), so that its
     # samples all fall under load
-    pre = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(2)]
     t_pre = time.perf_counter()
     while time.perf_counter() - t_pre < 0.3:
         for _ in range(50):
-            flush.zero_()
-            step(pre[0])
+            flush()
+            step()
         torch.cuda.synchronize(dev)
-    for i in range(args.steps):
-        flush.zero_()
-        step(evs[i])
+    t_host0 = time.perf_counter()
+    for i in range(args.steps // g_steps):
+        if graph is not None:
+            graph.replay()
+        else:
+            flush()
+            step(evs[0])
+        torch.cuda.synchronize(dev)
+        harvest()
+    t_host = (time.perf_counter() - t_host0) * 1e3 / args.steps   # wall time per step
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clock_info = clocks.stop()
-    t_stats = sum(e[4].elapsed_time(e[5]) for e in evs) / args.steps
-    t_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    t_dec = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    t_step = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+    t_stats, t_sel, t_dec, t_step = (x / args.steps for x in sums)
     status = cb.cobs_read_device_status(ws, ws_bytes, stream)
     if status != 0:
         raise RuntimeError(f"device status {cb.cobs_status_string(status)} after timing")
@@ -439,11 +483,11 @@ def run_cobs(args, w, rank, world, local_rank):
             pair[1].record(stream)
 
         for _ in range(3):
-            flush.zero_()
+            flush()
             e2e_step(ev[0])
         torch.cuda.synchronize(dev)
         for i in range(n_e2e):
-            flush.zero_()
+            flush()
             e2e_step(ev[i])
         torch.cuda.synchronize(dev)
         t_e2e = sum(a.elapsed_time(b) for a, b in ev) / n_e2e
@@ -466,7 +510,8 @@ def run_cobs(args, w, rank, world, local_rank):
     bm = byte_model(w, round(n_sel_mean))
     per_kernel = {"stats": (t_stats, bm["stats"], "stats.cu"),
                   "select": (t_sel, bm["select"], "select.cu"),
-                  "decode": (t_dec, bm["decode"], "decode.cu")}
+                  "decode": (t_dec, bm["decode"],
+                             "decode_tc.cu" if w.head_dim == 128 else "decode.cu")}
     kernels = {name: {"ms": t, "bytes": b, "gbs": b / (t * 1e-3) / 1e9,
                       "frac_of_hbm": b / (t * 1e-3) / 1e9 / hbm}
                for name, (t, b, _) in per_kernel.items()}
@@ -489,10 +534,12 @@ def run_cobs(args, w, rank, world, local_rank):
                    "kv_heads": w.kv_heads, "head_dim": w.head_dim, "seq_len": w.seq_len,
                    "block": w.block, "rank": w.rank, "top_k": w.top_k,
                    "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
-                   "selected_blocks_mean": n_sel_mean, "l2": "flushed (256 MiB) between steps",
+                   "selected_blocks_mean": n_sel_mean, "l2": "flushed between steps: 256 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{world}",
                    "step": "stats of the completed block + select + sparse decode",
-                   "stats_stream": args.stats_stream},
+                   "stats_stream": args.stats_stream,
+                   "launch": (f"CUDA graphs of {g_steps} steps" if graph is not None
+                              else "one call at a time")},
         "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
         "hbm_frac_step": step_bytes / (t_step * 1e-3) / 1e9 / hbm,
         "kernels": kernels,
@@ -503,6 +550,7 @@ def run_cobs(args, w, rank, world, local_rank):
         "gpu_launches": 3 * args.steps,
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,
+        "wall_ms_per_step": t_host,
     }
     if e2e is not None:
         line["e2e"] = e2e

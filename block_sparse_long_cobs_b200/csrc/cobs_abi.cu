@@ -1,6 +1,8 @@
 // C ABI of the COBS decode library: argument checks, workspace layout, launch
 // configuration.  Everything that can be checked on the host is checked here,
 // before any CUDA call; kernels never see an invalid shape.
+#include <mutex>
+#include <vector>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -112,6 +114,89 @@ int device_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+namespace {
+
+struct KernelState {
+  const void* kern;
+  int device;
+  int smem_bytes;
+  int threads;          // of the cached occupancy (0: not queried)
+  int occupancy;
+  cudaError_t prepared;
+};
+std::mutex g_kernel_mu;
+std::vector<KernelState> g_kernels;
+
+KernelState* find_kernel(const void* kern, int device) {
+  for (auto& k : g_kernels)
+    if (k.kern == kern && k.device == device) return &k;
+  return nullptr;
+}
+
+}  // namespace
+
+cudaError_t prepare_kernel(const void* kern, int smem_bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_kernel_mu);
+  KernelState* k = find_kernel(kern, dev);
+  if (k && k->smem_bytes == smem_bytes) return k->prepared;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             int(cudaSharedmemCarveoutMaxShared));
+  if (!k) {
+    g_kernels.push_back(KernelState{kern, dev, smem_bytes, 0, 0, e});
+  } else {
+    *k = KernelState{kern, dev, smem_bytes, 0, 0, e};
+  }
+  return e;
+}
+
+int kernel_occupancy(const void* kern, int threads, int smem_bytes) {
+  if (prepare_kernel(kern, smem_bytes) != cudaSuccess) return 1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> lock(g_kernel_mu);
+  KernelState* k = find_kernel(kern, dev);
+  if (k && k->threads == threads) return k->occupancy;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, size_t(smem_bytes)) !=
+      cudaSuccess)
+    n = 1;
+  // The runtime's answer can be lower than what the SM's resources allow for
+  // kernels that opt into more than 48 KB of shared memory; count the
+  // resources directly (shared memory incl. the per-block reservation,
+  // registers at warp granularity, threads) and keep the larger figure.
+  cudaFuncAttributes fa{};
+  int smem_sm = 0, reserved = 0, regs_sm = 0, threads_sm = 0;
+  if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) ==
+          cudaSuccess &&
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) ==
+          cudaSuccess &&
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) ==
+          cudaSuccess &&
+      cudaDeviceGetAttribute(&threads_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev) ==
+          cudaSuccess) {
+    const long per_block_smem = long(smem_bytes) + long(fa.sharedSizeBytes) + reserved;
+    const int warps = (threads + 31) / 32;
+    const long per_block_regs = long((fa.numRegs + 7) / 8 * 8) * 32 * warps;
+    long by = per_block_smem > 0 ? smem_sm / per_block_smem : 32;
+    if (per_block_regs > 0 && regs_sm / per_block_regs < by) by = regs_sm / per_block_regs;
+    if (threads_sm / threads < by) by = threads_sm / threads;
+    if (by > 32) by = 32;
+    if (by > n) n = int(by);
+  }
+  if (n < 1) n = 1;
+  if (k) {
+    k->threads = threads;
+    k->occupancy = n;
+  }
   return n;
 }
 
@@ -386,7 +471,6 @@ cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_s
 // belongs to the library instead of a caller-provided workspace.
 // ---------------------------------------------------------------------------
 
-#include <mutex>
 
 namespace cobs {
 namespace {

@@ -103,4 +103,17 @@ cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);
 
 int device_sm_count();
 
+// Opt a kernel into `bytes` of dynamic shared memory and ask for the largest
+// shared-memory carveout, so that occupancy queries and launches both see
+// the full 228 KB of an SM.  Done once per (kernel, device); later calls only
+// look the result up.
+cudaError_t prepare_kernel(const void* kern, int smem_bytes);
+// Resident CTAs per SM of a prepared kernel (>= 1), cached per (kernel, device).
+int kernel_occupancy(const void* kern, int threads, int smem_bytes);
+
+template <typename Kernel>
+cudaError_t set_smem_attrs(Kernel kern, int bytes) {
+  return prepare_kernel(reinterpret_cast<const void*>(kern), bytes);
+}
+
 }  // namespace cobs

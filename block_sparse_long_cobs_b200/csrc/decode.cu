@@ -355,8 +355,7 @@ template <int D, int G>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using S = DecodeShape<D, G>;
   auto kern = sparse_decode_kernel<D, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(S::kBytes));
+  cudaError_t e = set_smem_attrs(kern, int(S::kBytes));
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.hkv, a.batch);
   kern<<<grid, kDecThreads, S::kBytes, stream>>>(a);
@@ -366,15 +365,8 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
 template <int D, int G>
 int occupancy_t() {
   using S = DecodeShape<D, G>;
-  auto kern = sparse_decode_kernel<D, G>;
-  int n = 0;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes)) !=
-      cudaSuccess)
-    return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kDecThreads, S::kBytes) !=
-      cudaSuccess)
-    return 1;
-  return n > 0 ? n : 1;
+  return kernel_occupancy(reinterpret_cast<const void*>(sparse_decode_kernel<D, G>),
+                          kDecThreads, int(S::kBytes));
 }
 
 int occupancy_group(int g) {

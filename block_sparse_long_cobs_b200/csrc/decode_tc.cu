@@ -18,14 +18,14 @@
 //
 // One segment of nb blocks, T = ceil(nb / 2) tiles of two blocks (128 keys):
 //  * producer warp: TMA of the segment's K tiles, then its V tiles, through a
-//    2-stage ring; a tile is 128 keys x 128 dims bf16 as two 64-column slabs
+//    3-stage ring (two CTAs per SM keep six 32 KB tiles in flight); a tile is 128 keys x 128 dims bf16 as two 64-column slabs
 //    in the 128-byte swizzle.  The query group rides with the first K tile.
 //  * MMA warp: S_t = K_t q^T into TMEM columns [16t, 16t + 16) (M = 128 keys,
 //    N = 16; query rows past the group only fill columns nobody reads); then,
 //    per tile as its probabilities arrive, O^T += V_t^T P_t^T with the V tile
 //    read MN-major (M = 128 dims) and the result in TMEM columns [240, 256).
 //  * softmax warps, one TMEM lane (key) per thread: pass 1 takes the maximum
-//    of each head over the segment, pass 2 writes p = 2^(s - m) into a 4-slot
+//    of each head over the segment, pass 2 writes p = 2^(s - m) into a 2-slot
 //    ring as bf16 hi + lo parts (B rows h and 8 + h), so O_h = D[:, h] +
 //    D[:, 8 + h] keeps fp32-level accuracy, and sums l = sum p in fp32.  Then
 //    each thread reads back the output row of one dimension.
@@ -43,23 +43,31 @@ namespace {
 constexpr int kD = 128;
 constexpr int kThreads = 192;            // warps 0-3 softmax, 4 TMA, 5 MMA
 constexpr int kSoftThreads = 128;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kSlabBytes = 128 * 128;    // 128 keys x 64 dims bf16
 constexpr int kStageBytes = 2 * kSlabBytes;
 constexpr int kHalfBytes = 64 * 128;     // one block's 64 rows of a slab
 constexpr int kMaxTiles = 15;
 constexpr int kMaxSegBlocks = 2 * kMaxTiles;
-constexpr int kPSlots = 4;
+constexpr int kPSlots = 2;
 constexpr int kPSlotBytes = 4096;        // 2 halves x (hi atom, lo atom) of 1 KB
 constexpr uint32_t kOCol = 16 * kMaxTiles;
 constexpr uint32_t kTmemCols = 256;
 // dynamic shared memory, offsets from a 1024-aligned base
 constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;   // 2 buffers x 2 slabs x 1 KB
-constexpr int kOffP = kOffQ + 2 * 2048 + 1024;            // + the rows 8..15 the MMA reads
+// the MMA also reads rows 8..15 of the query operand 1 KB past each slab: for
+// the last slab those bytes are the P ring's first atom, harmless since the
+// columns they feed are never read
+constexpr int kOffP = kOffQ + 2 * 2048;
 constexpr int kDynSmem = kOffP + kPSlots * kPSlotBytes + 1024;
 
 static_assert(kOCol + 16 <= kTmemCols, "TMEM columns");
+// The query buffer of segment n is reloaded for segment n + 2 once ring item
+// (issue count - kStages) is free; every segment has >= 2 items (a K and a V
+// tile), so with kStages <= 4 that item is at or after segment n's last one,
+// whose release implies that segment n's S = K q^T products have completed.
+static_assert(kStages <= 4, "query double-buffering relies on kStages <= 4");
 
 // Bounded mbarrier wait that also gives up as soon as another role of the CTA
 // has given up.
@@ -145,6 +153,9 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   const int64_t seq_blocks = (a.seq_len + kBlock - 1) / kBlock;
 
   if (tid == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -451,17 +462,10 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
 template <int G>
 int occupancy_g() {
-  auto kern = sparse_decode_tc_kernel<G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem) !=
-      cudaSuccess)
-    return 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, kDynSmem) !=
-      cudaSuccess)
-    return 1;
-  const int by_tmem = 512 / int(kTmemCols);
-  n = n < by_tmem ? n : by_tmem;
-  return n > 0 ? n : 1;
+  const int n = kernel_occupancy(reinterpret_cast<const void*>(sparse_decode_tc_kernel<G>),
+                                 kThreads, kDynSmem);
+  const int by_tmem = 512 / int(kTmemCols);   // TMEM columns of an SM
+  return n < by_tmem ? n : by_tmem;
 }
 
 template <int G>
@@ -478,7 +482,7 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
     e = make_bf16_tensor_map_sw128(&qmap, a.q, kD, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;
   auto kern = sparse_decode_tc_kernel<G>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  e = set_smem_attrs(kern, kDynSmem);
   if (e != cudaSuccess) return e;
   kern<<<a.n_ctas, kThreads, kDynSmem, stream>>>(kmap, vmap, qmap, a);
   return cudaGetLastError();

@@ -403,8 +403,7 @@ template <int D, int G>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
   auto kern = select_blocks_kernel<D, G>;
   constexpr size_t smem = dyn_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = set_smem_attrs(kern, int(smem));
   if (e != cudaSuccess) return e;
   CUtensorMap map;
   const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
@@ -417,15 +416,8 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
 
 template <int D, int G>
 int occupancy_t() {
-  int n = 0;
-  auto kern = select_blocks_kernel<D, G>;
-  constexpr size_t smem = dyn_smem_bytes<D>();
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-      cudaSuccess)
-    return 1;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kSelThreads, smem) != cudaSuccess)
-    return 1;
-  return n > 0 ? n : 1;
+  return kernel_occupancy(reinterpret_cast<const void*>(select_blocks_kernel<D, G>),
+                          kSelThreads, int(dyn_smem_bytes<D>()));
 }
 
 template <int D>

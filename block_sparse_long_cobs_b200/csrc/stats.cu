@@ -657,7 +657,7 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
   if (e0 != cudaSuccess) return e0;
   auto kern = block_stats_kernel<D, M>;
   cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(S::kBytes));
+      set_smem_attrs(kern, int(S::kBytes));
   if (e != cudaSuccess) return e;
   const int64_t n_items = int64_t(a.batch) * a.hkv * (a.block_end - a.block_begin);
   dim3 grid(unsigned(n_items), 1, 1);
