@@ -86,7 +86,7 @@ WorkspaceLayout layout(const cobs_dims* d, int32_t n_sel_max) {
   L.sel_tickets = off;
   off = align256(off + pairs * 4);
   L.dec_tickets = off;
-  off = align256(off + pairs * 4);
+  off = align256(off + (pairs + 2) * 4);
   L.scores = off;
   off = align256(off + pairs * size_t(L.nb_cap) * 4);
   L.partials = off;
@@ -205,18 +205,23 @@ DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride) {
   int sms = device_sm_count();
   if (sms <= 0) sms = 148;
   if (d == 128) {
-    // equal contiguous ranges of block-list slots, one wave of resident CTAs
-    const int64_t slots = pairs * idx_stride;
+    // one wave of persistent CTAs pulling chunks off a counter.  A chunk is an
+    // even share of one pair's list, never two pairs.  A pair that is one
+    // chunk writes its output directly; splitting a pair costs partials, a
+    // ticket, a merge and a pipeline restart (measured: 26-slot pairs of the
+    // 32k workload took 45 us whole, 61 us as halves), so pairs are split
+    // only as far as it takes to give every resident CTA a chunk, with at
+    // least 8 slots per chunk.
     const int64_t resident = int64_t(sms) * decode_tc_ctas_per_sm(g);
-    int64_t R = ceil_div(slots, resident);
-    if (R > decode_tc_max_slots()) R = decode_tc_max_slots();
-    if (R < 1) R = 1;
-    P.slots_per_cta = int32_t(R);
-    P.n_ctas = int32_t(ceil_div(slots, R));
-    // a pair's idx_stride slots meet at most floor((S + R - 2) / R) + 1 ranges
-    int64_t rows = (int64_t(idx_stride) + R - 2) / R + 1;
-    if (rows > idx_stride) rows = idx_stride;
-    P.part_rows = int32_t(rows);
+    int64_t per_pair = pairs * 4 >= resident * 3 ? 1 : ceil_div(resident, pairs);
+    const int64_t max_per_pair = ceil_div(idx_stride, 8);
+    if (per_pair > max_per_pair) per_pair = max_per_pair;
+    if (per_pair < 1) per_pair = 1;
+    P.chunk_slots = int32_t(ceil_div(idx_stride, per_pair));
+    P.chunks_per_pair = int32_t(ceil_div(idx_stride, P.chunk_slots));
+    P.n_chunks = int32_t(pairs * P.chunks_per_pair);
+    P.n_ctas = int32_t(P.n_chunks < resident ? P.n_chunks : resident);
+    P.part_rows = P.chunks_per_pair;
   } else {
     // one wave of resident CTAs shared out over the (batch, kv-head) pairs
     const int64_t resident = int64_t(sms) * decode_d64_ctas_per_sm(g);
@@ -440,8 +445,11 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   a.part_stride = idx_stride;   // the workspace holds idx_stride >= P.part_rows rows
   a.n_splits = P.n_splits;
   a.blocks_per_split = P.blocks_per_split;
-  a.slots_per_cta = P.slots_per_cta;
+  a.chunk_slots = P.chunk_slots;
+  a.chunks_per_pair = P.chunks_per_pair;
+  a.n_chunks = P.n_chunks;
   a.n_ctas = P.n_ctas;
+  a.work = a.tickets + int64_t(dims->batch) * dims->num_kv_heads;
 
   cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
@@ -533,7 +541,7 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
   const DecodePlan P = plan_decode(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
                                    pairs, idx_stride);
-  const size_t tickets_bytes = align256(size_t(pairs) * 4);
+  const size_t tickets_bytes = align256((size_t(pairs) + 2) * 4);
   const size_t need = tickets_bytes + size_t(dims->batch) * dims->num_q_heads *
                                           size_t(P.part_rows) * (size_t(dims->head_dim) + 2) * 4;
   if (need > kFixedScratchBytes)
@@ -545,8 +553,8 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   void* scratch = nullptr;
   if ((st = fixed_scratch_address(&scratch)) != COBS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // arrival counters must start at zero (the kernel leaves them at zero, but a
-  // previous call may have been cut short)
+  // arrival and work counters must start at zero (the kernel leaves them at
+  // zero, but a previous call may have been cut short)
   cudaError_t e = cudaMemsetAsync(scratch, 0, tickets_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed scratch counters");
 
@@ -573,8 +581,11 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.n_splits = P.n_splits;
   a.blocks_per_split = P.blocks_per_split;
-  a.slots_per_cta = P.slots_per_cta;
+  a.chunk_slots = P.chunk_slots;
+  a.chunks_per_pair = P.chunks_per_pair;
+  a.n_chunks = P.n_chunks;
   a.n_ctas = P.n_ctas;
+  a.work = a.tickets + pairs;
   e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
   return ok();

@@ -17,7 +17,7 @@ constexpr int kMaxGroup = 8;   // query heads per kv-head
 struct WorkspaceLayout {
   size_t status;       // int32 status word (+ padding)
   size_t sel_tickets;  // uint32 [batch * Hkv], selection arrival counters
-  size_t dec_tickets;  // uint32 [batch * Hkv], decode arrival counters
+  size_t dec_tickets;  // uint32 [batch * Hkv + 2], decode arrival counters + work counters
   size_t scores;       // float  [batch * Hkv * nb_cap], group scores
   size_t partials;     // float  [batch * Hq * n_sel_max * (d + 2)]
   size_t total;
@@ -58,6 +58,7 @@ struct DecodeArgs {
   float* lse;             // [b][Hq]
   float* partials;        // [b][Hq][n_sel_max][d+2]
   uint32_t* tickets;      // [b][Hkv]
+  uint32_t* work;         // head_dim 128: [2] chunk counter, finished-CTA counter (start at 0)
   int32_t* status;
   int64_t cap;
   int64_t seq_len;
@@ -66,15 +67,17 @@ struct DecodeArgs {
   int32_t part_stride;    // partial rows per query head (>= splits / segments of a pair)
   int32_t n_splits;       // head_dim 64: CTAs per (b, kv-head)
   int32_t blocks_per_split;
-  int32_t slots_per_cta;  // head_dim 128: block-list slots per CTA (<= 30)
-  int32_t n_ctas;         // head_dim 128: grid size
+  int32_t chunk_slots;    // head_dim 128: block-list slots per work chunk
+  int32_t chunks_per_pair;  // head_dim 128: chunks of one (b, kv-head) list
+  int32_t n_chunks;       // head_dim 128: chunks in the launch (pairs x chunks_per_pair)
+  int32_t n_ctas;         // head_dim 128: grid size (persistent CTAs)
   float scale_log2;       // softmax_scale * log2(e)
 };
 
 // Work split of one decode launch and the partial rows per query head it needs.
 struct DecodePlan {
   int32_t n_splits, blocks_per_split;   // head_dim 64 kernel
-  int32_t slots_per_cta, n_ctas;        // head_dim 128 kernel
+  int32_t chunk_slots, chunks_per_pair, n_chunks, n_ctas;  // head_dim 128 kernel
   int32_t part_rows;
 };
 
@@ -98,7 +101,6 @@ cudaError_t launch_decode_d64(const DecodeArgs& a, cudaStream_t stream);
 int decode_d64_ctas_per_sm(int g);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 int decode_tc_ctas_per_sm(int g);
-int decode_tc_max_slots();
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);
 
 int device_sm_count();

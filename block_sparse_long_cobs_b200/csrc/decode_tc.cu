@@ -8,27 +8,32 @@
 // attention is reconstructed from the selected blocks only).
 //
 // Work split.  The block lists of all (batch, kv-head) pairs are laid end to
-// end, idx_stride slots per pair, and each CTA of a persistent grid takes one
-// contiguous range of at most 30 slots, so every SM streams about the same
-// number of bytes whatever the pair count.  Pair boundaries cut a range into
+// end, idx_stride slots per pair, and cut into chunks of C slots.  A
+// persistent grid (two CTAs per SM) pulls chunks off a counter, so CTAs that
+// stream faster simply take more chunks.  Pair boundaries cut a chunk into
 // segments; a segment yields one partial (o, m, l) per query head of the
-// group, and the last segment of a pair to finish (atomic ticket, no
-// spinning) merges the partials:  M = max m_i,  out = sum 2^(m_i-M) o_i /
-// sum 2^(m_i-M) l_i,  lse = (M + log2 sum 2^(m_i-M) l_i) ln 2.
+// group (row = chunk index - first chunk of the pair), and the last segment
+// of a pair to finish (atomic ticket, no spinning) merges the partials:
+// M = max m_i, out = sum 2^(m_i-M) o_i / sum 2^(m_i-M) l_i,
+// lse = (M + log2 sum 2^(m_i-M) l_i) ln 2.  The last CTA to run out of work
+// puts the counters back to zero.
 //
-// One segment of nb blocks, T = ceil(nb / 2) tiles of two blocks (128 keys):
-//  * producer warp: TMA of the segment's K tiles, then its V tiles, through a
-//    3-stage ring (two CTAs per SM keep six 32 KB tiles in flight); a tile is 128 keys x 128 dims bf16 as two 64-column slabs
-//    in the 128-byte swizzle.  The query group rides with the first K tile.
-//  * MMA warp: S_t = K_t q^T into TMEM columns [16t, 16t + 16) (M = 128 keys,
-//    N = 16; query rows past the group only fill columns nobody reads); then,
-//    per tile as its probabilities arrive, O^T += V_t^T P_t^T with the V tile
-//    read MN-major (M = 128 dims) and the result in TMEM columns [240, 256).
-//  * softmax warps, one TMEM lane (key) per thread: pass 1 takes the maximum
-//    of each head over the segment, pass 2 writes p = 2^(s - m) into a 2-slot
-//    ring as bf16 hi + lo parts (B rows h and 8 + h), so O_h = D[:, h] +
-//    D[:, 8 + h] keeps fp32-level accuracy, and sums l = sum p in fp32.  Then
-//    each thread reads back the output row of one dimension.
+// One segment of nb blocks, T = ceil(nb / 2) tiles of two blocks (128 keys),
+// in a single pass:
+//  * producer warp: TMA of K_0, V_0, K_1, V_1, ... through a 3-stage ring; a
+//    tile is 128 keys x 128 dims bf16 as two 64-column slabs in the 128-byte
+//    swizzle.  The query group rides with K_0.
+//  * MMA warp: S_t = K_t q^T (M = 128 keys, N = 16; query rows past the group
+//    only fill columns nobody reads) into one of two TMEM score buffers, one
+//    tile ahead of the softmax; O^T += V_t^T P_t^T (V read MN-major, M = 128
+//    dims) into the TMEM output columns once P_t is ready.
+//  * softmax warps, one TMEM lane (key) per thread: p = 2^(s - m) with a
+//    running per-head maximum m that is only raised when a tile's logits
+//    exceed it by more than 2^8 (then O and l are rescaled in place, after the
+//    MMAs that wrote O have completed); P_t goes to a 2-slot ring as bf16 hi +
+//    lo parts (B rows h and 8 + h), so O_h = D[:, h] + D[:, 8 + h] keeps
+//    fp32-level accuracy, and l = sum p in fp32.  At the segment's end each
+//    thread reads back the output row of one dimension.
 // Keys at or past seq_len read as zero through the tensor maps' row bound and
 // are masked; block indices outside [0, ceil(seq_len / B)) are reported and
 // read as empty.  Every wait is bounded; a CTA that gives up records
@@ -47,12 +52,12 @@ constexpr int kStages = 3;
 constexpr int kSlabBytes = 128 * 128;    // 128 keys x 64 dims bf16
 constexpr int kStageBytes = 2 * kSlabBytes;
 constexpr int kHalfBytes = 64 * 128;     // one block's 64 rows of a slab
-constexpr int kMaxTiles = 15;
-constexpr int kMaxSegBlocks = 2 * kMaxTiles;
 constexpr int kPSlots = 2;
 constexpr int kPSlotBytes = 4096;        // 2 halves x (hi atom, lo atom) of 1 KB
-constexpr uint32_t kOCol = 16 * kMaxTiles;
-constexpr uint32_t kTmemCols = 256;
+constexpr int kChunkQ = 4;               // chunk indices handed from producer to consumers
+constexpr uint32_t kOCol = 32;           // two 16-column output buffers after the two score buffers
+constexpr uint32_t kTmemCols = 64;
+constexpr float kRescaleLog2 = 8.f;      // raise m only when exceeded by > 2^8
 // dynamic shared memory, offsets from a 1024-aligned base
 constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;   // 2 buffers x 2 slabs x 1 KB
@@ -62,7 +67,7 @@ constexpr int kOffQ = kOffRing + kStages * kStageBytes;   // 2 buffers x 2 slabs
 constexpr int kOffP = kOffQ + 2 * 2048;
 constexpr int kDynSmem = kOffP + kPSlots * kPSlotBytes + 1024;
 
-static_assert(kOCol + 16 <= kTmemCols, "TMEM columns");
+static_assert(kOCol + 32 <= kTmemCols, "TMEM columns");
 // The query buffer of segment n is reloaded for segment n + 2 once ring item
 // (issue count - kStages) is free; every segment has >= 2 items (a K and a V
 // tile), so with kStages <= 4 that item is at or after segment n's last one,
@@ -90,32 +95,42 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, in
 
 struct Segment {
   int64_t pair;
-  int seg;        // index among the pair's segments
-  int n_seg;      // segments of the pair
+  int seg;        // index among the pair's chunks (= partial row)
+  int n_seg;      // chunks of the pair
   int s0;         // first slot
   int nb;         // blocks (slots below n_sel)
   bool bad_nsel;  // n_sel outside [1, idx_stride]
 };
 
-// Next segment of this CTA's slot range [u, u_end); advances u.
-__device__ __forceinline__ bool next_segment(int64_t& u, int64_t u_end, const DecodeArgs& a,
-                                             Segment& g) {
-  if (u >= u_end) return false;
-  const int64_t S = a.idx_stride, R = a.slots_per_cta;
-  g.pair = u / S;
-  const int64_t p0 = g.pair * S;
-  const int64_t end = u_end < p0 + S ? u_end : p0 + S;
-  const int64_t first = p0 / R;
-  g.seg = int(int64_t(blockIdx.x) - first);
-  g.n_seg = int((p0 + S - 1) / R - first + 1);
+// Chunk c = an even share of one pair's block list.
+__device__ __forceinline__ Segment chunk_segment(int64_t c, const DecodeArgs& a) {
+  Segment g;
+  g.pair = c / a.chunks_per_pair;
+  g.seg = int(c % a.chunks_per_pair);
+  g.n_seg = a.chunks_per_pair;
   int nsel = a.n_sel[g.pair];
   g.bad_nsel = nsel < 1 || nsel > a.idx_stride;
   nsel = nsel < 0 ? 0 : (nsel > a.idx_stride ? a.idx_stride : nsel);
-  g.s0 = int(u - p0);
-  const int s1 = int(end - p0) < nsel ? int(end - p0) : nsel;
+  g.s0 = g.seg * a.chunk_slots;
+  int s1 = g.s0 + a.chunk_slots;
+  s1 = s1 < a.idx_stride ? s1 : a.idx_stride;
+  s1 = s1 < nsel ? s1 : nsel;
   g.nb = s1 > g.s0 ? s1 - g.s0 : 0;
-  u = end;
-  return true;
+  return g;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 template <int G>
@@ -129,11 +144,16 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ __align__(8) uint64_t empty[kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t s_free[2];
   __shared__ __align__(8) uint64_t p_full[kPSlots];
   __shared__ __align__(8) uint64_t p_free[kPSlots];
-  __shared__ __align__(8) uint64_t s_full;
-  __shared__ __align__(8) uint64_t o_full;
+  __shared__ __align__(8) uint64_t o_full[2];
   __shared__ __align__(8) uint64_t drain;
+  __shared__ __align__(8) uint64_t cq_full[kChunkQ];
+  __shared__ __align__(8) uint64_t cq_empty[kChunkQ];
+  __shared__ volatile long long cq_val[kChunkQ];
+  __shared__ long long chunk_s;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_s;
   __shared__ int last_s;
@@ -142,14 +162,10 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  if (a.slots_per_cta < 1 || a.slots_per_cta > kMaxSegBlocks) {  // host contract
+  if (a.chunk_slots < 2 || a.n_chunks < 1) {  // host contract
     if (tid == 0) report(a.status, COBS_ERR_DEVICE);
     return;
   }
-  const int64_t n_slots = int64_t(a.batch) * a.hkv * a.idx_stride;
-  const int64_t u_begin = int64_t(blockIdx.x) * a.slots_per_cta;
-  const int64_t u_end =
-      u_begin + a.slots_per_cta < n_slots ? u_begin + a.slots_per_cta : n_slots;
   const int64_t seq_blocks = (a.seq_len + kBlock - 1) / kBlock;
 
   if (tid == 0) {
@@ -160,12 +176,20 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 1);
+    }
     for (int s = 0; s < kPSlots; ++s) {
       mbar_init(&p_full[s], kSoftThreads);
       mbar_init(&p_free[s], 1);
     }
-    mbar_init(&s_full, 1);
-    mbar_init(&o_full, 1);
+    for (int s = 0; s < kChunkQ; ++s) {
+      mbar_init(&cq_full[s], 1);
+      mbar_init(&cq_empty[s], 2);
+    }
+    mbar_init(&o_full[0], 1);
+    mbar_init(&o_full[1], 1);
     mbar_init(&drain, 1);
     fence_barrier_init();
     abort_s = 0;
@@ -179,46 +203,68 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == 4) {
     // ============================ TMA producer ============================
     if (lane == 0) {
-      uint32_t it = 0;
-      int nonempty = 0;
+      uint32_t it = 0;       // ring items issued
+      int nonempty = 0;      // non-empty segments
       bool ok = true;
-      int64_t u = u_begin;
-      Segment g;
-      while (ok && next_segment(u, u_end, a, g)) {
-        if (g.nb == 0) continue;
-        const int T = (g.nb + 1) >> 1;
-        const int32_t* row = a.idx + g.pair * a.idx_stride + g.s0;
-        const int z = int(g.pair);
-        const int qrow = int((g.pair / a.hkv) * a.hq + (g.pair % a.hkv) * G);
-        uint8_t* qbuf = base + kOffQ + (nonempty & 1) * 2048;
-        for (int pass = 0; pass < 2 && ok; ++pass) {
-          const CUtensorMap* map = pass ? &vmap : &kmap;
-          for (int t = 0; t < T; ++t, ++it) {
-            const int st = it % kStages;
-            if (it >= kStages &&
-                !wait_or_abort(&empty[st], ((it / kStages) - 1) & 1, a.status, &abort_s)) {
-              ok = false;
-              break;
-            }
+      for (uint32_t ci = 0; ok; ++ci) {
+        // ---- next chunk: the first one is the CTA's own index ----
+        const int qs = ci % kChunkQ;
+        if (ci >= kChunkQ &&
+            !wait_or_abort(&cq_empty[qs], ((ci / kChunkQ) - 1) & 1, a.status, &abort_s))
+          break;
+        const int64_t c = ci == 0 ? int64_t(blockIdx.x)
+                                  : int64_t(gridDim.x) + int64_t(atomicAdd(&a.work[0], 1u));
+        cq_val[qs] = c;
+        mbar_arrive(&cq_full[qs]);
+        if (c >= a.n_chunks) {
+          // out of work: the last CTA to get here puts the counters back
+          __threadfence();
+          if (atomicAdd(&a.work[1], 1u) == gridDim.x - 1) {
+            a.work[0] = 0u;
+            a.work[1] = 0u;
+            __threadfence();
+          }
+          break;
+        }
+        const Segment g = chunk_segment(c, a);
+        if (g.nb > 0) {
+          const int T = (g.nb + 1) >> 1;
+          const int32_t* row = a.idx + g.pair * a.idx_stride + g.s0;
+          const int z = int(g.pair);
+          const int qrow = int((g.pair / a.hkv) * a.hq + (g.pair % a.hkv) * G);
+          uint8_t* qbuf = base + kOffQ + (nonempty & 1) * 2048;
+          for (int t = 0; t < T && ok; ++t) {
             const int nh = (2 * t + 1 < g.nb) ? 2 : 1;
-            const bool with_q = pass == 0 && t == 0;
-            mbar_arrive_expect_tx(&full[st],
-                                  uint32_t(nh) * 2u * kHalfBytes + (with_q ? 2048u : 0u));
-            if (with_q) {
-              tma_load_2d(qbuf, &qmap, 0, qrow, &full[st]);
-              tma_load_2d(qbuf + 1024, &qmap, 64, qrow, &full[st]);
-            }
-            uint8_t* dst = base + kOffRing + st * kStageBytes;
+            int y[2] = {0, 0};
             for (int h2 = 0; h2 < nh; ++h2) {
               const int j = row[2 * t + h2];
               // an index outside the sequence reads an all-zero box past seq_len
-              const int y = (j >= 0 && j < seq_blocks) ? j * kBlock : int(seq_blocks * kBlock);
-              tma_load_3d(dst + h2 * kHalfBytes, map, 0, y, z, &full[st]);
-              tma_load_3d(dst + kSlabBytes + h2 * kHalfBytes, map, 64, y, z, &full[st]);
+              y[h2] = (j >= 0 && j < seq_blocks) ? j * kBlock : int(seq_blocks * kBlock);
+            }
+            for (int kv = 0; kv < 2; ++kv, ++it) {   // K_t then V_t
+              const int st = it % kStages;
+              if (it >= kStages &&
+                  !wait_or_abort(&empty[st], ((it / kStages) - 1) & 1, a.status, &abort_s)) {
+                ok = false;
+                break;
+              }
+              const bool with_q = kv == 0 && t == 0;
+              mbar_arrive_expect_tx(&full[st],
+                                    uint32_t(nh) * 2u * kHalfBytes + (with_q ? 2048u : 0u));
+              if (with_q) {
+                tma_load_2d(qbuf, &qmap, 0, qrow, &full[st]);
+                tma_load_2d(qbuf + 1024, &qmap, 64, qrow, &full[st]);
+              }
+              const CUtensorMap* map = kv ? &vmap : &kmap;
+              uint8_t* dst = base + kOffRing + st * kStageBytes;
+              for (int h2 = 0; h2 < nh; ++h2) {
+                tma_load_3d(dst + h2 * kHalfBytes, map, 0, y[h2], z, &full[st]);
+                tma_load_3d(dst + kSlabBytes + h2 * kHalfBytes, map, 64, y[h2], z, &full[st]);
+              }
             }
           }
+          ++nonempty;
         }
-        ++nonempty;
       }
       // the copies of the last kStages items may still be landing
       for (uint32_t x = it > uint32_t(kStages) ? it - kStages : 0u; x < it; ++x)
@@ -230,62 +276,83 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 16);
       constexpr uint32_t idesc_pv = umma_idesc_bf16_amn(128, 16);
-      uint32_t it = 0, pt = 0;
+      uint32_t it = 0;       // ring items consumed (issue order)
+      uint32_t gt = 0;       // score tiles computed (all segments)
+      uint32_t pt = 0;       // P tiles consumed
       int nonempty = 0;
       bool ok = true, issued = false;
-      int64_t u = u_begin;
-      Segment g;
-      while (ok && next_segment(u, u_end, a, g)) {
-        if (g.nb == 0) continue;
-        const int T = (g.nb + 1) >> 1;
-        const uint32_t qaddr = smem_addr(base + kOffQ + (nonempty & 1) * 2048);
-        // ---- S_t = K_t q^T ----
-        for (int t = 0; t < T; ++t, ++it) {
-          const int st = it % kStages;
-          if (!wait_or_abort(&full[st], (it / kStages) & 1, a.status, &abort_s)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_addr(base + kOffRing + st * kStageBytes);
+      // S = K q^T for the tile whose K tile is ring item `kit`
+      auto qk = [&](uint32_t kit, uint32_t qaddr) -> bool {
+        const int sb = gt & 1;
+        if (gt >= 2 && !wait_or_abort(&s_free[sb], ((gt >> 1) - 1) & 1, a.status, &abort_s))
+          return false;
+        const int st = kit % kStages;
+        if (!wait_or_abort(&full[st], (kit / kStages) & 1, a.status, &abort_s)) return false;
+        tc_fence_after();
+        const uint32_t a0 = smem_addr(base + kOffRing + st * kStageBytes);
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint64_t ad = umma_desc_sw128(a0 + (ks >> 2) * kSlabBytes + (ks & 3) * 32);
-            const uint64_t bd = umma_desc_sw128(qaddr + (ks >> 2) * 1024 + (ks & 3) * 32);
-            umma_bf16(tmem + 16u * t, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[st]);
-          issued = true;
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t ad = umma_desc_sw128(a0 + (ks >> 2) * kSlabBytes + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_sw128(qaddr + (ks >> 2) * 1024 + (ks & 3) * 32);
+          umma_bf16(tmem + 16u * sb, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
         }
-        if (!ok) break;
-        umma_commit(&s_full);
-        // ---- O^T += V_t^T P_t^T ----
-        for (int t = 0; t < T; ++t, ++it, ++pt) {
-          const int slot = pt % kPSlots;
-          const int st = it % kStages;
-          if (!wait_or_abort(&p_full[slot], (pt / kPSlots) & 1, a.status, &abort_s) ||
-              !wait_or_abort(&full[st], (it / kStages) & 1, a.status, &abort_s)) {
+        umma_commit(&empty[st]);
+        umma_commit(&s_full[sb]);
+        issued = true;
+        ++gt;
+        return true;
+      };
+      for (uint32_t ci = 0; ok; ++ci) {
+        const int qs = ci % kChunkQ;
+        if (!wait_or_abort(&cq_full[qs], (ci / kChunkQ) & 1, a.status, &abort_s)) break;
+        const int64_t c = cq_val[qs];
+        mbar_arrive(&cq_empty[qs]);
+        if (c >= a.n_chunks) break;
+        const Segment g = chunk_segment(c, a);
+        if (g.nb > 0) {
+          const int T = (g.nb + 1) >> 1;
+          const uint32_t qaddr = smem_addr(base + kOffQ + (nonempty & 1) * 2048);
+          const uint32_t ocol = kOCol + 16u * uint32_t(nonempty & 1);
+          const uint32_t it0 = it;   // K_t is item it0 + 2t, V_t is item it0 + 2t + 1
+          if (!qk(it0, qaddr)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a0 = smem_addr(base + kOffRing + st * kStageBytes);
-          const uint32_t pb = smem_addr(base + kOffP + slot * kPSlotBytes);
-          const int nks = (2 * t + 1 < g.nb) ? 8 : 4;   // a lone block: its 64 keys only
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            if (ks < nks) {
-              const uint64_t ad = umma_desc_sw128_mn(a0 + ks * 2048, kSlabBytes);
-              const uint64_t bd = umma_desc_sw128(pb + (ks >> 2) * 2048 + (ks & 3) * 32);
-              umma_bf16(tmem + kOCol, ad, bd, idesc_pv, (t > 0 || ks > 0) ? 1u : 0u);
+          for (int t = 0; t < T; ++t) {
+            // keep the score of the next tile one step ahead of the softmax
+            if (t + 1 < T && !qk(it0 + 2 * (t + 1), qaddr)) {
+              ok = false;
+              break;
             }
+            const int slot = pt % kPSlots;
+            const uint32_t vit = it0 + 2 * t + 1;
+            const int st = vit % kStages;
+            if (!wait_or_abort(&p_full[slot], (pt / kPSlots) & 1, a.status, &abort_s) ||
+                !wait_or_abort(&full[st], (vit / kStages) & 1, a.status, &abort_s)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_addr(base + kOffRing + st * kStageBytes);
+            const uint32_t pb = smem_addr(base + kOffP + slot * kPSlotBytes);
+            const int nks = (2 * t + 1 < g.nb) ? 8 : 4;   // a lone block: its 64 keys only
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              if (ks < nks) {
+                const uint64_t ad = umma_desc_sw128_mn(a0 + ks * 2048, kSlabBytes);
+                const uint64_t bd = umma_desc_sw128(pb + (ks >> 2) * 2048 + (ks & 3) * 32);
+                umma_bf16(tmem + ocol, ad, bd, idesc_pv, (t > 0 || ks > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit(&empty[st]);
+            umma_commit(&p_free[slot]);
+            ++pt;
           }
-          umma_commit(&empty[st]);
-          umma_commit(&p_free[slot]);
+          if (!ok) break;
+          it = it0 + 2u * uint32_t(T);
+          umma_commit(&o_full[nonempty & 1]);
+          ++nonempty;
         }
-        if (!ok) break;
-        umma_commit(&o_full);
-        ++nonempty;
       }
       if (issued) {  // every MMA issued must be complete before TMEM is freed
         umma_commit(&drain);
@@ -299,32 +366,137 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const int half = r >> 6, kk = r & 63;
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const int64_t hstride = int64_t(a.part_stride) * (kD + 2);
-    uint32_t pt = 0;
+    uint32_t gt = 0;   // score tiles consumed (all segments)
+    uint32_t pt = 0;   // P tiles produced
     int nonempty = 0;
     bool ok = true;
-    int64_t u = u_begin;
-    Segment g;
-    while (ok && next_segment(u, u_end, a, g)) {
+
+    // Output rows of a finished segment, read back from TMEM output buffer
+    // `ob` (phase `use`) one segment later, when its products have long been
+    // complete.  A pair that is a single chunk is normalised here; otherwise
+    // the rows go to the partials and the pair's last chunk to arrive merges.
+    auto epilogue = [&](const Segment& sg, bool has_o, int ob, uint32_t use, const float (&m)[G],
+                        const float (&lpart)[G]) -> bool {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float sum = warp_sum(lpart[h]);
+        if (lane == 0) red[warp][h] = sum;
+      }
+      bool fail = abort_s != 0;
+      if (has_o && r == 0) fail = !wait_or_abort(&o_full[ob], use & 1, a.status, &abort_s);
+      if (named_bar_or(1, kSoftThreads, fail)) return false;
+      float l[G], o[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        l[h] = (red[0][h] + red[1][h]) + (red[2][h] + red[3][h]);
+        o[h] = 0.f;
+      }
+      if (has_o) {
+        tc_fence_after();
+        float ov[16];
+        tmem_ld16(tmem + lane_base + kOCol + 16u * uint32_t(ob), ov);
+        tc_fence_before();
+#pragma unroll
+        for (int h = 0; h < G; ++h) o[h] = ov[h] + ov[8 + h];
+      }
+      const int64_t hq0 = (sg.pair / a.hkv) * a.hq + (sg.pair % a.hkv) * G;
+      constexpr float kLn2 = 0.69314718055994530942f;
+      if (sg.n_seg == 1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          a.out[(hq0 + h) * kD + r] = (l[h] > 0.f) ? o[h] / l[h] : 0.f;
+          if (r == h) a.lse[hq0 + h] = (l[h] > 0.f) ? (m[h] + hw_log2(l[h])) * kLn2 : -INFINITY;
+        }
+        named_bar(1, kSoftThreads);   // red is read before it is rewritten
+        return true;
+      }
+      float* part = a.partials + hq0 * hstride + int64_t(sg.seg) * (kD + 2);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        if (has_o) part[h * hstride + r] = o[h];
+        if (r == h) {
+          part[h * hstride + kD] = m[h];
+          part[h * hstride + kD + 1] = l[h];
+        }
+      }
+      // publish: every thread's rows are written (barrier), then one fence and
+      // the pair's ticket
+      named_bar(1, kSoftThreads);
+      if (r == 0) {
+        __threadfence();
+        const uint32_t prev = atomicAdd(&a.tickets[sg.pair], 1u);
+        last_s = (prev == uint32_t(sg.n_seg - 1));
+      }
+      named_bar(1, kSoftThreads);
+      if (last_s) {
+        __threadfence();
+        for (int e = r; e < G * kD; e += kSoftThreads) {
+          const int h = e / kD, dd = e % kD;
+          const int64_t hq = hq0 + h;
+          const float* pbase = a.partials + hq * hstride;
+          float M = -INFINITY;
+          for (int s = 0; s < sg.n_seg; ++s)
+            M = fmaxf(M, __ldcg(pbase + int64_t(s) * (kD + 2) + kD));
+          float L = 0.f, O = 0.f;
+          if (M != -INFINITY) {
+            for (int s = 0; s < sg.n_seg; ++s) {
+              const float* prow = pbase + int64_t(s) * (kD + 2);
+              const float ms = __ldcg(prow + kD);
+              if (ms == -INFINITY) continue;
+              const float w = hw_exp2(ms - M);
+              L += w * __ldcg(prow + kD + 1);
+              O += w * __ldcg(prow + dd);
+            }
+          }
+          a.out[hq * kD + dd] = (L > 0.f) ? O / L : 0.f;
+          if (dd == 0) a.lse[hq] = (L > 0.f) ? (M + hw_log2(L)) * kLn2 : -INFINITY;
+        }
+        if (r == 0) a.tickets[sg.pair] = 0u;
+      }
+      named_bar(1, kSoftThreads);   // last_s is rewritten by the next segment
+      return true;
+    };
+
+    bool pend = false;                 // a segment whose output is still in TMEM
+    Segment pg{};
+    bool pend_o = false;
+    int pend_ob = 0;
+    uint32_t pend_use = 0;
+    float pm[G], pl[G];
+    for (uint32_t ci = 0; ok; ++ci) {
+      const int qs = ci % kChunkQ;
+      bool fail = abort_s != 0;
+      if (r == 0) {
+        fail = !wait_or_abort(&cq_full[qs], (ci / kChunkQ) & 1, a.status, &abort_s);
+        if (!fail) {
+          chunk_s = cq_val[qs];
+          mbar_arrive(&cq_empty[qs]);
+        }
+      }
+      if (named_bar_or(1, kSoftThreads, fail)) {
+        ok = false;
+        break;
+      }
+      const int64_t c = chunk_s;
+      if (c >= a.n_chunks) break;
+      const Segment g = chunk_segment(c, a);
       if (g.bad_nsel && g.seg == 0 && r == 0) report(a.status, COBS_ERR_DEVICE);
-      const int64_t hq0 = (g.pair / a.hkv) * a.hq + (g.pair % a.hkv) * G;
-      float* part = a.partials + hq0 * hstride + int64_t(g.seg) * (kD + 2);
       float mh[G], lh[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         mh[h] = -INFINITY;
         lh[h] = 0.f;
       }
+      const int ob = nonempty & 1;
+      const uint32_t use = uint32_t(nonempty) >> 1;
       if (g.nb > 0) {
+        const uint32_t ocol = kOCol + 16u * uint32_t(ob);
         const int T = (g.nb + 1) >> 1;
         const int32_t* row = a.idx + g.pair * a.idx_stride + g.s0;
-        bool fail = abort_s != 0;
-        if (r == 0) fail = !wait_or_abort(&s_full, nonempty & 1, a.status, &abort_s);
-        if (named_bar_or(1, kSoftThreads, fail)) break;
-        tc_fence_after();
-
-        // ---- pass 1: per-head maximum of the scaled logits ----
-        uint32_t vmask = 0;
-        for (int t = 0; t < T; ++t) {
+        for (int t = 0; t < T; ++t, ++gt, ++pt) {
+          const int sb = gt & 1;
+          const int slot = pt % kPSlots;
+          // this thread's key: validity from the block index
           const int blk = 2 * t + half;
           bool valid = false;
           if (blk < g.nb) {
@@ -334,51 +506,82 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             else if (kk == 0)
               report(a.status, COBS_ERR_DEVICE);
           }
-          vmask |= uint32_t(valid) << t;
-          __syncwarp();   // the TMEM load is warp-collective
+          fail = abort_s != 0;
+          if (r == 0) {
+            fail = !wait_or_abort(&s_full[sb], (gt >> 1) & 1, a.status, &abort_s);
+            if (!fail && pt >= kPSlots)   // P slot free again
+              fail = !wait_or_abort(&p_free[slot], ((pt / kPSlots) - 1) & 1, a.status,
+                                    &abort_s);
+          }
+          if (named_bar_or(1, kSoftThreads, fail)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
           uint32_t sv[NC];
-          if constexpr (NC == 4) tmem_ld4_nowait(tmem + lane_base + 16u * t, sv);
-          else tmem_ld8_nowait(tmem + lane_base + 16u * t, sv);
+          if constexpr (NC == 4) tmem_ld4_nowait(tmem + lane_base + 16u * sb, sv);
+          else tmem_ld8_nowait(tmem + lane_base + 16u * sb, sv);
           tmem_wait_ld();
+          float s2[G];
+          bool raise = false;
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-            mh[h] = fmaxf(mh[h], valid ? __uint_as_float(sv[h]) * a.scale_log2 : -INFINITY);
-        }
+          for (int h = 0; h < G; ++h) {
+            s2[h] = valid ? __uint_as_float(sv[h]) * a.scale_log2 : -INFINITY;
+            raise |= s2[h] > mh[h] + kRescaleLog2;
+          }
+          tc_fence_before();
+          // every thread has read the score buffer; is a raise of m needed?
+          raise = named_bar_or(1, kSoftThreads, raise);
+          if (r == 0) mbar_arrive(&s_free[sb]);
+          if (raise) {
+            // exact per-head maximum of this tile, then rescale O and l
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float m = warp_max(mh[h]);
-          if (lane == 0) red[warp][h] = m;
-        }
-        named_bar(1, kSoftThreads);
+            for (int h = 0; h < G; ++h) {
+              const float mx = warp_max(s2[h]);
+              if (lane == 0) red[warp][h] = mx;
+            }
+            named_bar(1, kSoftThreads);
+            float alpha[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          mh[h] = fmaxf(fmaxf(red[0][h], red[1][h]), fmaxf(red[2][h], red[3][h]));
-        named_bar(1, kSoftThreads);  // red is reused for the sums
-
-        // ---- pass 2: probabilities into the P ring ----
-        for (int t = 0; t < T; ++t, ++pt) {
-          const int slot = pt % kPSlots;
-          if (pt >= kPSlots) {
-            bool fail = abort_s != 0;
-            if (r == 0)
-              fail = !wait_or_abort(&p_free[slot], ((pt / kPSlots) - 1) & 1, a.status, &abort_s);
-            if (named_bar_or(1, kSoftThreads, fail)) {
-              ok = false;
-              break;
+            for (int h = 0; h < G; ++h) {
+              const float tm = fmaxf(fmaxf(red[0][h], red[1][h]), fmaxf(red[2][h], red[3][h]));
+              const float mn = fmaxf(mh[h], tm);
+              alpha[h] = (mh[h] == -INFINITY) ? 0.f : hw_exp2(mh[h] - mn);
+              mh[h] = mn;
+              lh[h] *= alpha[h];
+            }
+            if (t > 0) {
+              // the products of tiles < t must be complete before O is read
+              fail = abort_s != 0;
+              if (r == 0) {
+                const uint32_t pp = pt - 1;
+                fail = !wait_or_abort(&p_free[pp % kPSlots], (pp / kPSlots) & 1, a.status,
+                                      &abort_s);
+              }
+              if (named_bar_or(1, kSoftThreads, fail)) {   // also: red has been read
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              float ov[16];
+              tmem_ld16(tmem + lane_base + ocol, ov);
+#pragma unroll
+              for (int h = 0; h < G; ++h) {
+                ov[h] *= alpha[h];
+                ov[8 + h] *= alpha[h];
+              }
+              tmem_st16(tmem + lane_base + ocol, ov);
+              tc_fence_before();
+            } else {
+              named_bar(1, kSoftThreads);   // red is read before it is rewritten
             }
           }
-          uint32_t sv[NC];
-          if constexpr (NC == 4) tmem_ld4_nowait(tmem + lane_base + 16u * t, sv);
-          else tmem_ld8_nowait(tmem + lane_base + 16u * t, sv);
-          tmem_wait_ld();
-          const bool valid = (vmask >> t) & 1u;
-          if (2 * t + half < g.nb) {   // rows of a missing second block are never read
+          // ---- probabilities into the P ring ----
+          if (blk < g.nb) {   // rows of a missing second block are never read
             uint8_t* atom = base + kOffP + slot * kPSlotBytes + half * 2048;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-              const float p = (valid && mh[h] != -INFINITY)
-                                  ? hw_exp2(__uint_as_float(sv[h]) * a.scale_log2 - mh[h])
-                                  : 0.f;
+              const float p = valid ? hw_exp2(s2[h] - mh[h]) : 0.f;
               lh[h] += p;
               const uint32_t hi = __float_as_uint(p) & 0xffff0000u;
               const uint16_t lo = float_to_bf16_bits(p - __uint_as_float(hi));
@@ -392,68 +595,25 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           mbar_arrive(&p_full[slot]);
         }
         if (!ok) break;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float s = warp_sum(lh[h]);
-          if (lane == 0) red[warp][h] = s;
-        }
-        fail = abort_s != 0;
-        if (r == 0) fail = !wait_or_abort(&o_full, nonempty & 1, a.status, &abort_s);
-        if (named_bar_or(1, kSoftThreads, fail)) break;
-#pragma unroll
-        for (int h = 0; h < G; ++h) lh[h] = (red[0][h] + red[1][h]) + (red[2][h] + red[3][h]);
-        tc_fence_after();
-
-        // ---- epilogue: unnormalised output row of dim r ----
-        float ov[16];
-        tmem_ld16(tmem + lane_base + kOCol, ov);
-        tc_fence_before();
-#pragma unroll
-        for (int h = 0; h < G; ++h) part[h * hstride + r] = ov[h] + ov[8 + h];
         ++nonempty;
       }
+      // the previous segment's products are complete by now: write its output
+      if (pend && !epilogue(pg, pend_o, pend_ob, pend_use, pm, pl)) {
+        ok = false;
+        break;
+      }
+      pend = true;
+      pg = g;
+      pend_o = g.nb > 0;
+      pend_ob = ob;
+      pend_use = use;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        if (r == h) {
-          part[h * hstride + kD] = mh[h];
-          part[h * hstride + kD + 1] = lh[h];
-        }
-      }
-      // ---- arrival; the last segment of the pair merges ----
-      __threadfence();
-      named_bar(1, kSoftThreads);
-      if (r == 0) {
-        const uint32_t prev = atomicAdd(&a.tickets[g.pair], 1u);
-        last_s = (prev == uint32_t(g.n_seg - 1));
-      }
-      named_bar(1, kSoftThreads);
-      if (last_s) {
-        __threadfence();
-        constexpr float kLn2 = 0.69314718055994530942f;
-        for (int e = r; e < G * kD; e += kSoftThreads) {
-          const int h = e / kD, dd = e % kD;
-          const int64_t hq = hq0 + h;
-          const float* pbase = a.partials + hq * hstride;
-          float M = -INFINITY;
-          for (int s = 0; s < g.n_seg; ++s)
-            M = fmaxf(M, __ldcg(pbase + int64_t(s) * (kD + 2) + kD));
-          float L = 0.f, O = 0.f;
-          if (M != -INFINITY) {
-            for (int s = 0; s < g.n_seg; ++s) {
-              const float* prow = pbase + int64_t(s) * (kD + 2);
-              const float ms = __ldcg(prow + kD);
-              if (ms == -INFINITY) continue;
-              const float w = hw_exp2(ms - M);
-              L += w * __ldcg(prow + kD + 1);
-              O += w * __ldcg(prow + dd);
-            }
-          }
-          a.out[hq * kD + dd] = (L > 0.f) ? O / L : 0.f;
-          if (dd == 0) a.lse[hq] = (L > 0.f) ? (M + hw_log2(L)) * kLn2 : -INFINITY;
-        }
-        if (r == 0) a.tickets[g.pair] = 0u;
+        pm[h] = mh[h];
+        pl[h] = lh[h];
       }
     }
+    if (ok && pend) (void)epilogue(pg, pend_o, pend_ob, pend_use, pm, pl);
   }
   tc_fence_before();
   __syncthreads();
@@ -498,8 +658,6 @@ int decode_tc_ctas_per_sm(int g) {
     default: return occupancy_g<8>();
   }
 }
-
-int decode_tc_max_slots() { return kMaxSegBlocks; }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.hq / a.hkv) {

@@ -108,8 +108,10 @@ COBS_API int32_t cobs_selected_capacity(const cobs_dims* dims, int32_t top_k,
 COBS_API size_t cobs_workspace_bytes(const cobs_dims* dims, int32_t top_k,
                             int32_t sink_blocks, int32_t local_tokens);
 
-/* Zero-fill a workspace.  Required once before its first use; afterwards the
- * kernels leave their counters at zero themselves. */
+/* Zero-fill a workspace.  Required once before its first use, and again after
+ * a call that reported COBS_ERR_TIMEOUT (an interrupted kernel can leave its
+ * counters set); otherwise the kernels leave their counters at zero
+ * themselves.  Calls that share a workspace must not overlap on the GPU. */
 COBS_API cobs_status cobs_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Block statistics for the complete blocks [block_begin, block_end) of every

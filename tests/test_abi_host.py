@@ -61,7 +61,9 @@ def test_selected_capacity_and_workspace_size(name):
     assert nsm == min(w.cap // 64, w.top_k + w.sink_blocks + ceil_div(w.local_tokens, 64) + 1)
     ws = cb.cobs_workspace_bytes(d, w.top_k, w.sink_blocks, w.local_tokens)
     pairs = w.batch * w.kv_heads
-    want = 256 + 2 * align(pairs * 4) + align(pairs * (w.cap // 64) * 4) + \
+    # status, selection tickets, decode tickets + the decode work counters (2),
+    # scores, split partials
+    want = 256 + align(pairs * 4) + align((pairs + 2) * 4) + align(pairs * (w.cap // 64) * 4) + \
         align(w.batch * w.q_heads * nsm * (w.head_dim + 2) * 4)
     assert ws == want
 
