@@ -66,6 +66,8 @@ cobs_status check_dims(const cobs_dims* d) {
 cobs_status check_select_params(int32_t top_k, int32_t sink_blocks, int32_t local_tokens) {
   if (top_k < 0 || sink_blocks < 0 || local_tokens < 0)
     return fail(COBS_ERR_INVALID_ARG, "top_k, sink_blocks and local_tokens must be >= 0");
+  if (top_k > kMaxTopK)
+    return fail(COBS_ERR_UNSUPPORTED, "top_k %d above the supported %d", top_k, kMaxTopK);
   return COBS_OK;
 }
 

@@ -12,6 +12,7 @@ namespace cobs {
 constexpr int kBlock = 64;     // tokens per KV block
 constexpr int kMaxRank = 16;   // columns of the covariance factor
 constexpr int kMaxGroup = 8;   // query heads per kv-head
+constexpr int kMaxTopK = 4096; // candidates a selection may keep
 
 // Byte layout of the caller's workspace.  Every region starts 256-aligned.
 struct WorkspaceLayout {

@@ -15,18 +15,21 @@
 // [rows x d] . [d x G], done on the 5th-generation tensor cores.  A chunk's
 // records are contiguous rows of the stats array seen as a 2-d [rows][d] bf16
 // tensor; a 3-stage ring of TMA tile loads (128-byte swizzle, 128 rows per
-// stage = the largest whole number of records that fit) feeds one
-// tcgen05.mma chain per stage (M = 128 rows, N = 16 = G queries padded with
-// zero rows, K = d, fp32 accumulate in tensor memory).  The epilogue reads
+// stage = the largest whole number of records that fit; the group's query
+// rows ride with the first stage) feeds one tcgen05.mma chain per stage
+// (M = 128 rows, N = 16: operand rows past the G queries only fill
+// accumulator columns nobody reads; K = d, fp32 accumulate in tensor memory).  The epilogue reads
 // the 128 x G products back (tcgen05.ld), scales by 1/sqrt d, keeps row 0 of
 // a record (linear term) and squares-and-halves rows 1..r (quadratic term),
 // sums them per block and per head, adds ln 64 and takes the log-sum-exp over
 // the heads.  Scores go to the workspace (and to the optional output).
 //
-// Phase 2, the last CTA of a (batch, kv-head) (atomic ticket, no spinning)
-// finds the k-th largest score with a 4 x 8-bit radix select over
-// order-preserving integer keys, breaks ties at the threshold by index with a
-// block-wide prefix count, and compacts forced + chosen blocks in index order.
+// Phase 2, the last CTA of a (batch, kv-head) (atomic ticket, no spinning):
+// exact top k over distinct 64-bit keys (order-preserving score key, then the
+// lower block index): the k-th largest of the 128 per-thread maxima bounds
+// the k-th largest key from below, so only the few keys at or above it are
+// ranked; the chosen blocks are written in ascending order (warp ballot scan)
+// between the sink blocks and the local blocks.
 #include <cfloat>
 
 #include "device_common.cuh"
@@ -46,60 +49,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Reduce-scatter over `kLanes` lanes (see decode.cu for the same pattern).
-template <int G, int kLanes>
-__device__ __forceinline__ float reduce_scatter_sel(float (&v)[G], int lane, int& head) {
-  int live = G;
-  head = 0;
-#pragma unroll
-  for (int m = kLanes / 2; m >= 1; m >>= 1) {
-    if (live > 1) {
-      const int half = live / 2;
-      const bool upper = (lane & m) != 0;
-#pragma unroll
-      for (int i = 0; i < G / 2; ++i) {
-        if (i < half) {
-          const float send = upper ? v[i] : v[i + half];
-          const float keep = upper ? v[i + half] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-      }
-      if (upper) head += half;
-      live = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
-    }
-  }
-  return v[0];
-}
 
-// Exclusive prefix sum of one value per thread over the CTA (kSelThreads).
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,
-                                                         uint32_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
-#pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, m);
-    if (lane >= m) x += y;
-  }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  uint32_t base = 0, all = 0;
-#pragma unroll
-  for (int w = 0; w < kSelThreads / 32; ++w) {
-    const uint32_t t = warp_tot[w];
-    if (w < warp) base += t;
-    all += t;
-  }
-  __syncthreads();
-  total = all;
-  return base + x - v;
-}
 
 template <int D, int G>
 __global__ void __launch_bounds__(kSelThreads)
-select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs a) {
+select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
+                     const __grid_constant__ CUtensorMap qmap, const SelectArgs a) {
   constexpr int kRegions = D / 64;                  // 64-column slabs of a row
   constexpr int kStageBytes = kRegions * 128 * 128; // 128 rows x 128 B per slab
   constexpr int kQBytes = kRegions * 16 * 128;      // 16 query rows x 128 B per slab
@@ -113,9 +68,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
   const int rows = 1 + a.rank;
   const int per_stage = kStageRows / rows;          // whole records per stage
 
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t warp_tot[kSelThreads / 32];
-  __shared__ uint32_t sh_u32[4];
   __shared__ int last_s;
   __shared__ uint32_t tmem_slot;
   __shared__ __align__(8) uint64_t full[kSelStages];
@@ -138,6 +90,8 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
     const int64_t row0 = (int64_t(bh) * a.nb_cap) * rows;   // first row of this pair
 
     if (tid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
       for (int s2 = 0; s2 < kSelStages; ++s2) {
         mbar_init(&full[s2], 1);
         mbar_init(&mma_done[s2], 1);
@@ -157,27 +111,21 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
       const int j0 = c_lo + p * per_stage;
       const int y = int(row0 + int64_t(j0) * rows);
       uint8_t* dst = stage + (p % kSelStages) * kStageBytes;
-      // the box is always kStageRows rows; rows past the chunk are ignored
-      mbar_arrive_expect_tx(&full[p % kSelStages], uint32_t(kRegions) * kStageRows * 128);
+      // the box is always kStageRows rows; rows past the chunk are ignored.
+      // Pass 0 also brings the group's 8 query rows (rows past the group and
+      // rows 8..15 of the operand only feed accumulator columns nobody reads)
+      mbar_arrive_expect_tx(&full[p % kSelStages],
+                            uint32_t(kRegions) * (kStageRows + (p == 0 ? 8 : 0)) * 128);
+      if (p == 0)
+        for (int reg = 0; reg < kRegions; ++reg)
+          tma_load_2d(qtile + reg * 16 * 128, &qmap, reg * 64, b * a.hq + kvh * G, &full[0]);
       for (int reg = 0; reg < kRegions; ++reg)
         tma_load_2d(dst + reg * 128 * 128, &smap, reg * 64, y, &full[p % kSelStages]);
     };
-    // start the record stream first, build the query operand while it flies
+    // start the record stream (the query operand rides with the first tile)
     if (tid == 0) {
       for (int p = 0; p < kSelStages && p < npass; ++p) issue(p);
     }
-    // queries as the B operand: row n < G is query head kvh*G + n, rows G..15
-    // zero; 16-byte chunks written straight to their swizzled positions
-    for (int e = tid; e < kRegions * 16 * 8; e += kSelThreads) {
-      const int reg = e / (16 * 8), n = (e / 8) % 16, c = e % 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (n < G)
-        v = *reinterpret_cast<const uint4*>(a.q + (int64_t(b) * a.hq + kvh * G + n) * D +
-                                            reg * 64 + c * 8);
-      *reinterpret_cast<uint4*>(qtile + reg * 16 * 128 + n * 128 + ((c ^ (n & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
 
     const float inv_sqrt_d = rsqrtf(float(D));
     const float ln_n = logf(float(kBlock));
@@ -275,122 +223,132 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap, const SelectArgs 
   }
 
   // ===================== arrival: last CTA of (b, kv-head) selects =========
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const uint32_t prev = atomicAdd(&a.tickets[bh], 1u);
-    last_s = (prev == uint32_t(a.n_chunks - 1));
+  // (a pair scored by one CTA needs no ticket: its scores are this CTA's own)
+  if (a.n_chunks > 1) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const uint32_t prev = atomicAdd(&a.tickets[bh], 1u);
+      last_s = (prev == uint32_t(a.n_chunks - 1));
+    }
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+  } else {
+    __syncthreads();   // every score of the pair is written
   }
-  __syncthreads();
-  if (!last_s) return;
-  __threadfence();
 
   const int c0 = a.cand_begin, c1 = a.cand_end;
   const int n_cand = c1 - c0;
   const int nbs = a.seq_len_blocks;
-  int k = a.top_k < n_cand ? a.top_k : n_cand;
-
-  // order keys of the candidates, staged in shared memory when they fit
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(stage);
-  const bool keys_in_smem = n_cand <= kSelStages * kStageBytes / 4;
-  if (keys_in_smem)
-    for (int j = tid; j < n_cand; j += kSelThreads) skeys[j] = order_key(__ldcg(scores + c0 + j));
-  __syncthreads();
-  auto key_of = [&](int j) -> uint32_t {   // j in [c0, c1)
-    return keys_in_smem ? skeys[j - c0] : order_key(__ldcg(scores + j));
-  };
-
+  const int k = a.top_k < n_cand ? a.top_k : n_cand;
   const bool partial = (k > 0 && k < n_cand);
 
-  // ---- radix select of the k-th largest key among the candidates ----------
-  uint32_t prefix = 0, mask = 0, krem = uint32_t(k);
-  if (partial) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-      __syncthreads();
-      for (int j = c0 + tid; j < c1; j += kSelThreads) {
-        const uint32_t key = key_of(j);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // lane l covers digits [255 - 8l - 7, 255 - 8l], scanned from the top
-        uint32_t c8[8], tot = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          c8[i] = hist[255 - 8 * tid - i];
-          tot += c8[i];
-        }
-        uint32_t incl = tot;
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, m);
-          if (tid >= m) incl += y;
-        }
-        const uint32_t excl = incl - tot;
-        const bool here = excl < krem && incl >= krem;
-        if (here) {
-          uint32_t run = excl;
-          for (int i = 0; i < 8; ++i) {
-            if (run + c8[i] >= krem) {
-              sh_u32[0] = uint32_t(255 - 8 * tid - i);  // digit
-              sh_u32[1] = krem - run;                    // remaining rank in bin
-              break;
-            }
-            run += c8[i];
-          }
-        }
-      }
-      __syncthreads();
-      prefix |= sh_u32[0] << shift;
-      mask |= 0xffu << shift;
-      krem = sh_u32[1];
-      __syncthreads();
-    }
-  }
-  // prefix = threshold key tau; krem = how many keys equal to tau to keep
-
-  // ---- ordered compaction of forced + chosen blocks -------------------------
-  const int per = (nbs + kSelThreads - 1) / kSelThreads;
-  const int j0 = min(nbs, tid * per), j1 = min(nbs, j0 + per);
-  auto is_forced = [&](int j) { return j < a.sink_end || j >= a.first_local; };
-  uint32_t n_eq = 0;
-  if (partial) {
-    for (int j = j0; j < j1; ++j)
-      if (j >= c0 && j < c1 && key_of(j) == prefix) ++n_eq;
-  }
-  uint32_t tot_unused;
-  uint32_t eq_before = block_exclusive_scan(n_eq, warp_tot, tot_unused);
-  auto chosen = [&](int j, uint32_t& eq_seen) -> bool {
-    if (is_forced(j)) return true;
-    if (j < c0 || j >= c1) return false;
-    if (!partial) return k > 0;  // k == n_cand: everything; k == 0: nothing
-    const uint32_t key = key_of(j);
-    if (key > prefix) return true;
-    if (key == prefix) return (eq_seen++) < krem;
-    return false;
+  // ---- exact top-k (score, then lower block index) -------------------------
+  // 64-bit keys (order-preserving score key << 32 | ~candidate) are distinct.
+  // Each thread takes the maximum key of its candidates jj = tid, tid + 128,
+  // ...; tau = the k-th largest of those maxima is a lower bound of the true
+  // k-th largest key (k distinct candidates reach it), and only the keys >= tau
+  // -- at most k * ceil(n / 128) of them -- need ranking.  For k >= 128 every
+  // candidate is ranked.  The record ring (free now) holds the work arrays.
+  uint8_t* chosen_s = stage;                                              // [n_cand]
+  uint64_t* tmax = reinterpret_cast<uint64_t*>(stage + ((n_cand + 15) & ~15));   // [128]
+  uint64_t* surv = tmax + kSelThreads;                                    // survivors
+  constexpr int kRingBytes = kSelStages * kStageBytes;
+  const int surv_cap =
+      int((kRingBytes - ((n_cand + 15) & ~15) - kSelThreads * 8) / 8);
+  auto key64 = [&](int jj) -> uint64_t {
+    return (uint64_t(order_key(__ldcg(scores + c0 + jj))) << 32) |
+           uint64_t(0xFFFFFFFFu - uint32_t(jj));
   };
-  uint32_t cnt = 0;
-  {
-    uint32_t eq_seen = eq_before;
-    for (int j = j0; j < j1; ++j) cnt += chosen(j, eq_seen) ? 1u : 0u;
-  }
-  uint32_t total;
-  uint32_t pos = block_exclusive_scan(cnt, warp_tot, total);
-  int32_t* out = a.idx + int64_t(bh) * a.idx_stride;
-  {
-    uint32_t eq_seen = eq_before;
-    for (int j = j0; j < j1; ++j) {
-      if (chosen(j, eq_seen)) {
-        if (pos < uint32_t(a.idx_stride)) out[pos] = j;
-        ++pos;
+  const bool fits = n_cand + 16 + kSelThreads * 8 <= kRingBytes;
+  if (partial && fits) {
+    for (int jj = tid; jj < n_cand; jj += kSelThreads) chosen_s[jj] = 0;
+    // a thread's first kCached keys stay in registers for the survivor pass
+    constexpr int kCached = 8;
+    uint64_t kc[kCached];
+#pragma unroll
+    for (int i = 0; i < kCached; ++i) {
+      const int jj = tid + i * kSelThreads;
+      kc[i] = jj < n_cand ? key64(jj) : 0ull;
+    }
+    uint64_t mine = 0;
+    if (k < kSelThreads) {
+#pragma unroll
+      for (int i = 0; i < kCached; ++i) mine = kc[i] > mine ? kc[i] : mine;
+      for (int jj = tid + kCached * kSelThreads; jj < n_cand; jj += kSelThreads) {
+        const uint64_t c = key64(jj);
+        mine = c > mine ? c : mine;
       }
     }
+    tmax[tid] = mine;
+    if (tid == 0) last_s = 0;   // reused below as the survivor count
+    __syncthreads();
+    uint64_t tau = 0;
+    if (k < kSelThreads) {
+      // the thread maxima are distinct or 0; rank this thread's among them
+      int rank = 0;
+      for (int u = 0; u < kSelThreads; ++u) rank += tmax[u] > mine;
+      __syncthreads();
+      if (mine != 0 && rank == k - 1) tmax[0] = mine;   // exactly one thread
+      __syncthreads();
+      tau = tmax[0];
+    }
+    // survivors: every candidate key >= tau
+    auto keep = [&](uint64_t c) {
+      if (c >= tau) {
+        const int slot = atomicAdd(&last_s, 1);
+        if (slot < surv_cap) surv[slot] = c;
+      }
+    };
+#pragma unroll
+    for (int i = 0; i < kCached; ++i)
+      if (tid + i * kSelThreads < n_cand) keep(kc[i]);
+    for (int jj = tid + kCached * kSelThreads; jj < n_cand; jj += kSelThreads) keep(key64(jj));
+    __syncthreads();
+    const int ns = last_s < surv_cap ? last_s : surv_cap;
+    if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
+    for (int i = tid; i < ns; i += kSelThreads) {
+      const uint64_t c = surv[i];
+      int rank = 0;
+      for (int u = 0; u < ns; ++u) rank += surv[u] > c;
+      if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
+    }
+    __syncthreads();
+  } else if (partial && tid == 0) {
+    report(a.status, COBS_ERR_DEVICE);   // candidate flags do not fit (host limits prevent it)
   }
-  if (tid == 0) {
-    if (total > uint32_t(a.idx_stride)) report(a.status, COBS_ERR_DEVICE);
-    a.n_sel[bh] = int32_t(min(total, uint32_t(a.idx_stride)));
-    a.tickets[bh] = 0u;
+
+  // ---- sink blocks, chosen candidates ascending, local blocks -------------
+  int32_t* out = a.idx + int64_t(bh) * a.idx_stride;
+  const int n_local = nbs - a.first_local;
+  const int total = a.sink_end + k + n_local;
+  if (warp == 0) {
+    for (int i = lane; i < a.sink_end && i < a.idx_stride; i += 32) out[i] = i;
+    int pos = a.sink_end;
+    if (partial && fits) {
+      for (int j0 = 0; j0 < n_cand; j0 += 32) {
+        const int jj = j0 + lane;
+        const bool take = jj < n_cand && chosen_s[jj] != 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, take);
+        if (take) {
+          const int at = pos + __popc(bal & ((1u << lane) - 1u));
+          if (at < a.idx_stride) out[at] = c0 + jj;
+        }
+        pos += __popc(bal);
+      }
+    } else if (!partial) {   // k == n_cand: every candidate; k == 0: none
+      for (int r = lane; r < k; r += 32)
+        if (pos + r < a.idx_stride) out[pos + r] = c0 + r;
+      pos += k;
+    }
+    for (int i = lane; i < n_local; i += 32)
+      if (pos + i < a.idx_stride) out[pos + i] = a.first_local + i;
+    if (lane == 0) {
+      if (total > a.idx_stride) report(a.status, COBS_ERR_DEVICE);
+      a.n_sel[bh] = total < a.idx_stride ? total : a.idx_stride;
+      a.tickets[bh] = 0u;
+    }
   }
 }
 
@@ -408,9 +366,12 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
   CUtensorMap map;
   const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
   e = make_bf16_tensor_map_sw128(&map, a.stats, D, total_rows, kStageRows);
+  CUtensorMap qmap;
+  if (e == cudaSuccess)
+    e = make_bf16_tensor_map_sw128(&qmap, a.q, D, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.hkv, a.batch);
-  kern<<<grid, kSelThreads, smem, s>>>(map, a);
+  kern<<<grid, kSelThreads, smem, s>>>(map, qmap, a);
   return cudaGetLastError();
 }
 

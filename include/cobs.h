@@ -146,7 +146,7 @@ COBS_API cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k
  *   n_sel       device [batch][Hkv] int32, number of selected blocks.
  *   scores_opt  device [batch][Hkv][capacity/B] fp32 or NULL: S_b of the
  *               scored candidates (other entries untouched).
- * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+ * Errors: INVALID_ARG, UNSUPPORTED (also top_k above 4096), WORKSPACE, CUDA. */
 COBS_API cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q,
                                const void* stats, int64_t seq_len,
                                int32_t top_k, int32_t sink_blocks,
