@@ -254,10 +254,12 @@ def run_reference(args, w, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+        "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_heads": w.q_heads,
                    "kv_heads": w.kv_heads, "head_dim": w.head_dim, "seq_len": w.seq_len,
                    "block": w.block, "rank": w.rank, "top_k": w.top_k,
-                   "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens},
+                   "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
+                   "parallelism": f"replicas x{args.gpus}",
+                   "step": "stats of the completed block + select + sparse decode"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"per step one (batch, kv-head) pair of {pairs}: stats of "
                                    "the completed block + selection + attention, fp64 numpy, "
@@ -346,12 +348,17 @@ def run_cobs(args, w, rank, world, local_rank):
     side = torch.cuda.Stream(dev) if args.stats_stream == "side" else None
     fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
 
-    def step(ev=None, st=None):
-        # ev: [step start, selection start, decode start, step end, stats start, stats end]
+    def step(ev=None, st=None, inner=True, one_stream=False):
+        # ev: [step start, selection start, decode start, step end, stats start, stats end];
+        # with inner=False only the step's start and end are recorded (an event
+        # between two kernels stops the second from starting its prologue early)
         st = stream if st is None else st
-        if ev is not None:
-            ev[0].record(st)
-        if side is not None:
+        evo = ev
+        ev = ev if inner else None
+        if evo is not None:
+            evo[0].record(st)
+        use_side = side is not None and not one_stream
+        if use_side:
             # the block completed at this step lies in the local window, so the
             # selection below never reads the record being written
             fork_ev.record(st)
@@ -376,10 +383,10 @@ def run_cobs(args, w, rank, world, local_rank):
             ev[2].record(st)
         cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
                               ws, ws_bytes, st)
-        if side is not None:
+        if use_side:
             st.wait_event(join_ev)
-        if ev is not None:
-            ev[3].record(st)
+        if evo is not None:
+            evo[3].record(st)
 
     for _ in range(args.warmup):
         flush()
@@ -399,27 +406,47 @@ def run_cobs(args, w, rank, world, local_rank):
     if args.no_graph:
         g_steps = 1
     # external: recorded inside a graph capture as event-record nodes
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
-           for _ in range(g_steps)]
-    graph = None
-    if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+    def make_events():
+        return [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+                for _ in range(g_steps)]
+
+    def capture(evs, inner):
+        if args.no_graph:
+            return None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
             cs = torch.cuda.current_stream(dev)
             for i in range(g_steps):
                 flush()
-                step(evs[i], cs)
+                step(evs[i], cs, inner, one_stream=inner)
         for _ in range(2):
-            graph.replay()
+            g.replay()
         torch.cuda.synchronize(dev)
-    sums = [0.0, 0.0, 0.0, 0.0]   # stats, select, decode, step (ms)
+        return g
 
-    def harvest():
-        for e in evs:
-            sums[0] += e[4].elapsed_time(e[5])
-            sums[1] += e[1].elapsed_time(e[2])
-            sums[2] += e[2].elapsed_time(e[3])
-            sums[3] += e[0].elapsed_time(e[3])
+    def run_timed(evs, graph, n_steps, inner, sums):
+        for _ in range(n_steps // g_steps):
+            if graph is not None:
+                graph.replay()
+            else:
+                flush()
+                step(evs[0], None, inner, one_stream=inner)
+            torch.cuda.synchronize(dev)
+            for e in evs:
+                sums[3] += e[0].elapsed_time(e[3])
+                if inner:
+                    sums[0] += e[4].elapsed_time(e[5])
+                    sums[1] += e[1].elapsed_time(e[2])
+                    sums[2] += e[2].elapsed_time(e[3])
+
+    # (1) the step time: events at step boundaries only; (2) the per-kernel
+    # breakdown: the same steps with all three kernels on one stream and events
+    # between them (each kernel timed alone), a fifth as many (at least 250)
+    evs_step, evs_kern = make_events(), make_events()
+    graph_step = capture(evs_step, False)
+    n_kern = max(min(250, args.steps), args.steps // 5) // g_steps * g_steps or g_steps
+    graph_kern = capture(evs_kern, True)
+    sums_step, sums_kern = [0.0] * 4, [0.0] * 4
 
     clocks = ClockSampler(local_rank)
     if world > 1:
@@ -435,20 +462,16 @@ def run_cobs(args, w, rank, world, local_rank):
             step()
         torch.cuda.synchronize(dev)
     t_host0 = time.perf_counter()
-    for i in range(args.steps // g_steps):
-        if graph is not None:
-            graph.replay()
-        else:
-            flush()
-            step(evs[0])
-        torch.cuda.synchronize(dev)
-        harvest()
+    run_timed(evs_step, graph_step, args.steps, False, sums_step)
     t_host = (time.perf_counter() - t_host0) * 1e3 / args.steps   # wall time per step
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    run_timed(evs_kern, graph_kern, n_kern, True, sums_kern)
+    torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
-    t_stats, t_sel, t_dec, t_step = (x / args.steps for x in sums)
+    t_step = sums_step[3] / args.steps
+    t_stats, t_sel, t_dec, t_step_kern = (x / n_kern for x in sums_kern)
     status = cb.cobs_read_device_status(ws, ws_bytes, stream)
     if status != 0:
         raise RuntimeError(f"device status {cb.cobs_status_string(status)} after timing")
@@ -458,46 +481,86 @@ def run_cobs(args, w, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         q_host = torch.from_numpy(q_bits.view(np.int16)).pin_memory()
-        kn_host = torch.from_numpy(k_bits[:, :, w.seq_len - 1].view(np.int16)).pin_memory()
-        vn_host = torch.from_numpy(v_bits[:, :, w.seq_len - 1].view(np.int16)).pin_memory()
+        kn_host = torch.from_numpy(
+            np.ascontiguousarray(k_bits[:, :, w.seq_len - 1]).view(np.int16)).pin_memory()
+        vn_host = torch.from_numpy(
+            np.ascontiguousarray(v_bits[:, :, w.seq_len - 1]).view(np.int16)).pin_memory()
         out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         kn_dev = torch.empty_like(kn_host, device=dev)
         vn_dev = torch.empty_like(vn_host, device=dev)
         h2d = q_host.numel() * 2 + kn_host.numel() * 2 + vn_host.numel() * 2
         d2h = out_host.numel() * 4 + lse_host.numel() * 4
-        n_e2e = max(1, args.steps // 4)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_e2e)]
+        n_e2e = max(g_steps, args.steps // 4 // g_steps * g_steps)
 
-        def e2e_step(pair):
-            pair[0].record(stream)
+        def e2e_step(pair, st=None):
+            # torch copies go to the current stream: the capture stream inside
+            # a graph capture, `stream` otherwise
+            st = stream if st is None else st
+            pair[0].record(st)
             q.copy_(q_host, non_blocking=True)
             kn_dev.copy_(kn_host, non_blocking=True)
             vn_dev.copy_(vn_host, non_blocking=True)
             k[:, :, w.seq_len - 1].copy_(kn_dev)
             v[:, :, w.seq_len - 1].copy_(vn_dev)
-            step()
+            step(None, st)
             out_host.copy_(out, non_blocking=True)
             lse_host.copy_(lse, non_blocking=True)
-            pair[1].record(stream)
+            pair[1].record(st)
 
-        for _ in range(3):
-            flush()
-            e2e_step(ev[0])
-        torch.cuda.synchronize(dev)
-        for i in range(n_e2e):
-            flush()
-            e2e_step(ev[i])
-        torch.cuda.synchronize(dev)
-        t_e2e = sum(a.elapsed_time(b) for a, b in ev) / n_e2e
+        def time_e2e(use_graph):
+            ev = [(torch.cuda.Event(enable_timing=True, external=use_graph),
+                   torch.cuda.Event(enable_timing=True, external=use_graph))
+                  for _ in range(g_steps)]
+            g = None
+            if use_graph:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    cs = torch.cuda.current_stream(dev)
+                    for i in range(g_steps):
+                        flush()
+                        e2e_step(ev[i], cs)
+            for _ in range(3):
+                if g is not None:
+                    g.replay()
+                else:
+                    flush()
+                    e2e_step(ev[0])
+            torch.cuda.synchronize(dev)
+            total = 0.0
+            for _ in range(n_e2e // g_steps):
+                if g is not None:
+                    g.replay()
+                    torch.cuda.synchronize(dev)
+                    total += sum(a.elapsed_time(b) for a, b in ev)
+                else:
+                    for _ in range(g_steps):
+                        flush()
+                        e2e_step(ev[0])
+                        torch.cuda.synchronize(dev)
+                        total += ev[0][0].elapsed_time(ev[0][1])
+            return total / n_e2e
+
+        # the public-API calls and the per-step copies, replayed as CUDA
+        # graphs (as a decode server drives them); and the same calls made one
+        # by one from Python, which adds the host's call overhead
+        t_e2e = time_e2e(not args.no_graph)
+        t_eager = time_e2e(False)
         if world > 1:
             tt = torch.tensor([t_e2e], device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             t_e2e = float(tt.item())
+            tt = torch.tensor([t_eager], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            t_eager = float(tt.item())
         e2e = {"value": world * w.batch * w.q_heads / (t_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": t_e2e}
+               "ms_per_step": t_e2e,
+               "launch": "CUDA graphs of the API calls and copies" if not args.no_graph
+                         else "one call at a time",
+               "eager": {"value": world * w.batch * w.q_heads / (t_eager * 1e-3),
+                         "ms_per_step": t_eager,
+                         "launch": "one call at a time from Python"}}
 
     if world > 1:
         tt = torch.tensor([t_step, t_stats, t_sel, t_dec], device=dev)
@@ -538,7 +601,7 @@ def run_cobs(args, w, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "step": "stats of the completed block + select + sparse decode",
                    "stats_stream": args.stats_stream,
-                   "launch": (f"CUDA graphs of {g_steps} steps" if graph is not None
+                   "launch": (f"CUDA graphs of {g_steps} steps" if graph_step is not None
                               else "one call at a time")},
         "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
         "hbm_frac_step": step_bytes / (t_step * 1e-3) / 1e9 / hbm,
@@ -551,6 +614,10 @@ def run_cobs(args, w, rank, world, local_rank):
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,
         "wall_ms_per_step": t_host,
+        "kernel_breakdown": {"steps": n_kern, "ms_per_step": t_step_kern,
+                             "note": "per-kernel times from a second graph-replayed run, "
+                                     "the three kernels on one stream with events between "
+                                     "them"},
     }
     if e2e is not None:
         line["e2e"] = e2e

@@ -114,6 +114,25 @@ cudaError_t prepare_kernel(const void* kern, int smem_bytes);
 // Resident CTAs per SM of a prepared kernel (>= 1), cached per (kernel, device).
 int kernel_occupancy(const void* kern, int threads, int smem_bytes);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes; it calls pdl_wait() before
+// reading anything an earlier launch wrote (device_common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 template <typename Kernel>
 cudaError_t set_smem_attrs(Kernel kern, int bytes) {
   return prepare_kernel(reinterpret_cast<const void*>(kern), bytes);

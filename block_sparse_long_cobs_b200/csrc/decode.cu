@@ -118,6 +118,9 @@ sparse_decode_kernel(const DecodeArgs a) {
   const int b = blockIdx.z;
   const int bh = b * a.hkv + kvh;
 
+  pdl_wait();                // block lists and counts come from the launch before
+  pdl_launch_dependents();
+
   // ---- this split's slice of the block list --------------------------------
   int nsel = a.n_sel[bh];
   if (nsel < 1 || nsel > a.idx_stride) {
@@ -358,8 +361,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   cudaError_t e = set_smem_attrs(kern, int(S::kBytes));
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.hkv, a.batch);
-  kern<<<grid, kDecThreads, S::kBytes, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kDecThreads), S::kBytes, stream, a);
 }
 
 template <int D, int G>

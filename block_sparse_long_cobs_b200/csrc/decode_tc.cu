@@ -195,9 +195,11 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     abort_s = 0;
   }
   if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
+  pdl_wait();                // block lists and counts come from the launch before
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_launch_dependents();
   const uint32_t tmem = tmem_slot;
 
   if (warp == 4) {
@@ -644,8 +646,7 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
   auto kern = sparse_decode_tc_kernel<G>;
   e = set_smem_attrs(kern, kDynSmem);
   if (e != cudaSuccess) return e;
-  kern<<<a.n_ctas, kThreads, kDynSmem, stream>>>(kmap, vmap, qmap, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(a.n_ctas), dim3(kThreads), kDynSmem, stream, kmap, vmap, qmap, a);
 }
 
 }  // namespace

@@ -50,6 +50,18 @@ __device__ __forceinline__ void report(int32_t* status, int32_t code) {
   if (status != nullptr) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel of
+// the stream start (its CTAs run their prologue on SMs this grid frees); it
+// takes effect once every CTA of this grid has issued it or exited.  wait
+// blocks until the previous kernel of the stream has completed and its writes
+// are visible; every read of data an earlier launch wrote must come after it.
+// Both are no-ops for a kernel launched without the programmatic
+// serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

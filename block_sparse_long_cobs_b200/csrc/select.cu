@@ -99,9 +99,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       fence_barrier_init();
     }
     if (warp == 0) tmem_alloc(&tmem_slot, 32);
+    pdl_wait();              // queries and records may come from the launch before
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_launch_dependents();
     const uint32_t tmem = tmem_slot;
 
     int n_issued = 0;          // thread 0: passes whose TMA copies were issued
@@ -371,8 +373,7 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
     e = make_bf16_tensor_map_sw128(&qmap, a.q, D, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_chunks, a.hkv, a.batch);
-  kern<<<grid, kSelThreads, smem, s>>>(map, qmap, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kSelThreads), smem, s, map, qmap, a);
 }
 
 template <int D, int G>

@@ -178,9 +178,11 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     *abort_s = 0;
   }
   if (warp == 0) tmem_alloc(tmem_slot, 64);
+  pdl_wait();                // keys may come from the launch before
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
   // ---- 1. TMA load of the block, then the Gram on the tensor cores -----------
@@ -661,8 +663,7 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int64_t n_items = int64_t(a.batch) * a.hkv * (a.block_end - a.block_begin);
   dim3 grid(unsigned(n_items), 1, 1);
-  kern<<<grid, kStatThreads, S::kBytes, stream>>>(map, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kStatThreads), S::kBytes, stream, map, a);
 }
 
 }  // namespace

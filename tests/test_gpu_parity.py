@@ -311,3 +311,33 @@ def test_planted_spectrum_blocks():
         mu_ok, rel, energy = stats_errors(st[0, 0, j], orc, want[j], w.rank)
         assert mu_ok and energy >= 1 - ENERGY_RTOL
         assert rel is None or rel <= PROJ_RTOL
+
+
+@pytest.mark.parametrize("top_k", [127, 128, 200])
+def test_select_large_top_k(top_k):
+    """top_k at and above 128 candidates' worth of threads, with more candidates
+    than top_k: every candidate key is ranked; planted exact ties must still
+    be broken by the lower block index."""
+    w = W["single_32k"].scaled(seq_len=16384 + 5, batch=1, q_heads=8, kv_heads=2,
+                               top_k=top_k)
+    p = Problem(w)
+    recs = {}
+    for h in range(w.kv_heads):
+        r = p.oracle_records(0, h)
+        if h == 1:
+            r[[50, 60, 70, 200]] = r[40]
+        recs[(0, h)] = r
+        p.upload_records(0, h, r)
+    p.select()
+    idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+    for (b, h), r in recs.items():
+        sel, s = O.select_from_records(p.q_group(b, h), r, w.seq_len, w.block, w.top_k,
+                                       w.sink_blocks, w.local_tokens)
+        got = idx[b, h, :n[b, h]]
+        assert np.all(np.diff(got) > 0)
+        assert len(got) == len(sel)
+        if h == 1:
+            assert list(got) == list(sel)
+        else:
+            assert selection_mismatch(got, sel, s, w) == []
+    assert p.device_status() == 0
