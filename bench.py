@@ -91,6 +91,23 @@ def partition(T, B, sink, local):
     return n_blocks, n_full, sink_end, first_local
 
 
+def rank_shard(w, rank):
+    """The workload one rank decodes: the same shapes, its own seeded batch
+    (replicas shard the batch dimension; no data crosses ranks)."""
+    return w if rank == 0 else w.scaled(seed=w.seed + 1000003 * rank)
+
+
+def max_over_ranks(values, dist, device, world):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the
+    job's time); identity on one rank."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def byte_model(w, n_sel):
     """Algorithmic bytes per launch of each kernel for one step."""
     B, d, r = w.block, w.head_dim, w.rank
@@ -546,13 +563,7 @@ def run_cobs(args, w, rank, world, local_rank):
         # by one from Python, which adds the host's call overhead
         t_e2e = time_e2e(not args.no_graph)
         t_eager = time_e2e(False)
-        if world > 1:
-            tt = torch.tensor([t_e2e], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_e2e = float(tt.item())
-            tt = torch.tensor([t_eager], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            t_eager = float(tt.item())
+        t_e2e, t_eager = max_over_ranks([t_e2e, t_eager], dist, dev, world)
         e2e = {"value": world * w.batch * w.q_heads / (t_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e,
@@ -562,10 +573,8 @@ def run_cobs(args, w, rank, world, local_rank):
                          "ms_per_step": t_eager,
                          "launch": "one call at a time from Python"}}
 
-    if world > 1:
-        tt = torch.tensor([t_step, t_stats, t_sel, t_dec], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step, t_stats, t_sel, t_dec = (float(x) for x in tt.tolist())
+    t_step, t_stats, t_sel, t_dec = max_over_ranks([t_step, t_stats, t_sel, t_dec], dist, dev,
+                                                   world)
     if rank != 0:
         return
 
@@ -638,6 +647,9 @@ def main():
     if args.impl == "reference":
         run_reference(args, w, rank)
         return
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    w = rank_shard(w, rank)
     if world > 1:
         import datetime
 
