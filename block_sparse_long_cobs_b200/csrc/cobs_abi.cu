@@ -211,11 +211,13 @@ DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride) {
     // even share of one pair's list, never two pairs.  A pair that is one
     // chunk writes its output directly; splitting a pair costs partials, a
     // ticket, a merge and a pipeline restart (measured: 26-slot pairs of the
-    // 32k workload took 45 us whole, 61 us as halves), so pairs are split
-    // only as far as it takes to give every resident CTA a chunk, with at
-    // least 8 slots per chunk.
+    // 32k workload took 45 us whole, 61 us as halves), so pairs are split only
+    // as far as the resident CTAs can still take every chunk in one wave (a
+    // second, partial wave doubles the time of the CTAs that run it), with at
+    // least 8 slots per chunk (smaller chunks lost on the latency-bound
+    // small problems: more partials to merge).
     const int64_t resident = int64_t(sms) * decode_tc_ctas_per_sm(g);
-    int64_t per_pair = pairs * 4 >= resident * 3 ? 1 : ceil_div(resident, pairs);
+    int64_t per_pair = resident / pairs;
     const int64_t max_per_pair = ceil_div(idx_stride, 8);
     if (per_pair > max_per_pair) per_pair = max_per_pair;
     if (per_pair < 1) per_pair = 1;
@@ -350,6 +352,11 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   int64_t first_local = (seq_len - local_tokens > 0 ? seq_len - local_tokens : 0) / kBlock;
   if (first_local > n_full) first_local = n_full;
   const int64_t sink_end = sink_blocks < first_local ? sink_blocks : first_local;
+  if (!select_topk_fits(dims->head_dim, first_local - sink_end, top_k))
+    return fail(COBS_ERR_UNSUPPORTED,
+                "top_k %d over %lld candidate blocks exceeds the selection kernel's "
+                "shared memory (top_k x candidates / 1024 too large)",
+                top_k, (long long)(first_local - sink_end));
 
   SelectArgs a{};
   char* w = static_cast<char*>(ws);

@@ -96,6 +96,9 @@ struct StatsArgs {
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 int select_ctas_per_sm(int d, int g, int rank);  // resident selection CTAs per SM
 int select_blocks_per_stage(int rank);           // whole records per selection stage
+// Whether the exact top-k of `n_cand` candidates fits the selection kernel's
+// shared memory (its survivors can grow with top_k x n_cand / 1024).
+bool select_topk_fits(int d, int64_t n_cand, int top_k);
 DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);  // either kernel
 cudaError_t launch_decode_d64(const DecodeArgs& a, cudaStream_t stream);

@@ -41,6 +41,27 @@ namespace {
 constexpr int kSelThreads = 128;
 constexpr int kSelStages = 3;
 constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
+constexpr int kTopkGroups = 1024; // candidate groups of the top-k bound
+
+// Candidates per group of the top-k bound (groups never empty: at most 1024).
+__host__ __device__ constexpr int topk_group_size(int n_cand) {
+  return n_cand > kTopkGroups ? (n_cand + kTopkGroups - 1) / kTopkGroups : 1;
+}
+// 64-bit survivor slots left in the record ring after the group maxima, the
+// per-thread maxima and the candidate flags.
+__host__ __device__ constexpr int topk_survivor_capacity(int ring_bytes, int n_cand) {
+  return (ring_bytes -
+          ((n_cand + topk_group_size(n_cand) - 1) / topk_group_size(n_cand) + kSelThreads) * 8 -
+          ((n_cand + 15) & ~15)) / 8;
+}
+// Survivors the exact top-k can hold at most (both levels).
+__host__ __device__ constexpr int topk_survivors_needed(int n_cand, int k) {
+  const int gs = topk_group_size(n_cand);
+  const int ng = (n_cand + gs - 1) / gs;
+  const int lvl1 = k < kSelThreads ? k * ((ng + kSelThreads - 1) / kSelThreads) : ng;
+  const int lvl2 = k <= ng ? k * gs : n_cand;
+  return lvl1 > lvl2 ? lvl1 : lvl2;
+}
 
 // Order-preserving map float -> uint32 (larger float -> larger key); NaN lowest.
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -247,78 +268,111 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   const bool partial = (k > 0 && k < n_cand);
 
   // ---- exact top-k (score, then lower block index) -------------------------
-  // 64-bit keys (order-preserving score key << 32 | ~candidate) are distinct.
-  // Each thread takes the maximum key of its candidates jj = tid, tid + 128,
-  // ...; tau = the k-th largest of those maxima is a lower bound of the true
-  // k-th largest key (k distinct candidates reach it), and only the keys >= tau
-  // -- at most k * ceil(n / 128) of them -- need ranking.  For k >= 128 every
-  // candidate is ranked.  The record ring (free now) holds the work arrays.
-  uint8_t* chosen_s = stage;                                              // [n_cand]
-  uint64_t* tmax = reinterpret_cast<uint64_t*>(stage + ((n_cand + 15) & ~15));   // [128]
-  uint64_t* surv = tmax + kSelThreads;                                    // survivors
-  constexpr int kRingBytes = kSelStages * kStageBytes;
-  const int surv_cap =
-      int((kRingBytes - ((n_cand + 15) & ~15) - kSelThreads * 8) / 8);
+  // Keys: 64-bit, order-preserving score key << 32 | ~candidate, so distinct.
+  // The candidates are cut into ng <= 1024 groups of gs.  Each group maximum
+  // is a real key, so the k-th largest group maximum tau2 bounds the k-th
+  // largest key from below and at most k * gs keys reach it.  To find tau2,
+  // the k-th largest of the 128 per-thread maxima of the group maxima (tau1)
+  // bounds it likewise, so only the group maxima >= tau1 -- at most
+  // k * ceil(ng / 128) -- are ranked (all ng of them for k >= 128).  The
+  // record ring (free now) holds the work arrays; the host rejects settings
+  // whose survivors could overflow it (select_topk_fits).
+  const int gs = topk_group_size(n_cand);
+  const int ng = (n_cand + gs - 1) / gs;                               // no empty group
+  uint64_t* gmax = reinterpret_cast<uint64_t*>(stage);                 // [ng]
+  uint64_t* tmax = gmax + ng;                                          // [128]
+  uint64_t* surv = tmax + kSelThreads;                                 // survivors
+  const int surv_cap = topk_survivor_capacity(kSelStages * kStageBytes, n_cand);
+  uint8_t* chosen_s = reinterpret_cast<uint8_t*>(surv + (surv_cap > 0 ? surv_cap : 0));
   auto key64 = [&](int jj) -> uint64_t {
     return (uint64_t(order_key(__ldcg(scores + c0 + jj))) << 32) |
            uint64_t(0xFFFFFFFFu - uint32_t(jj));
   };
-  const bool fits = n_cand + 16 + kSelThreads * 8 <= kRingBytes;
+  __shared__ unsigned long long tau_s;
+  const bool fits = surv_cap >= topk_survivors_needed(n_cand, k);
   if (partial && fits) {
     for (int jj = tid; jj < n_cand; jj += kSelThreads) chosen_s[jj] = 0;
-    // a thread's first kCached keys stay in registers for the survivor pass
-    constexpr int kCached = 8;
-    uint64_t kc[kCached];
-#pragma unroll
-    for (int i = 0; i < kCached; ++i) {
-      const int jj = tid + i * kSelThreads;
-      kc[i] = jj < n_cand ? key64(jj) : 0ull;
-    }
     uint64_t mine = 0;
-    if (k < kSelThreads) {
-#pragma unroll
-      for (int i = 0; i < kCached; ++i) mine = kc[i] > mine ? kc[i] : mine;
-      for (int jj = tid + kCached * kSelThreads; jj < n_cand; jj += kSelThreads) {
+    for (int g = tid; g < ng; g += kSelThreads) {
+      const int j0 = g * gs, j1 = min(n_cand, j0 + gs);
+      uint64_t m = 0;
+      for (int jj = j0; jj < j1; ++jj) {
         const uint64_t c = key64(jj);
-        mine = c > mine ? c : mine;
+        m = c > m ? c : m;
       }
+      gmax[g] = m;
+      mine = m > mine ? m : mine;
     }
     tmax[tid] = mine;
-    if (tid == 0) last_s = 0;   // reused below as the survivor count
+    if (tid == 0) {
+      last_s = 0;   // survivor count
+      tau_s = 0ull;
+    }
     __syncthreads();
-    uint64_t tau = 0;
+    // tau1: the k-th largest thread maximum (thread maxima are distinct or 0;
+    // at least min(ng, 128) > k of them are non-zero when k < 128)
     if (k < kSelThreads) {
-      // the thread maxima are distinct or 0; rank this thread's among them
       int rank = 0;
       for (int u = 0; u < kSelThreads; ++u) rank += tmax[u] > mine;
-      __syncthreads();
-      if (mine != 0 && rank == k - 1) tmax[0] = mine;   // exactly one thread
-      __syncthreads();
-      tau = tmax[0];
+      if (mine != 0 && rank == k - 1) tau_s = mine;
     }
-    // survivors: every candidate key >= tau
-    auto keep = [&](uint64_t c) {
-      if (c >= tau) {
+    __syncthreads();
+    const uint64_t tau1 = tau_s;
+    for (int g = tid; g < ng; g += kSelThreads) {
+      if (gmax[g] >= tau1) {
         const int slot = atomicAdd(&last_s, 1);
-        if (slot < surv_cap) surv[slot] = c;
+        if (slot < surv_cap) surv[slot] = gmax[g];
       }
-    };
-#pragma unroll
-    for (int i = 0; i < kCached; ++i)
-      if (tid + i * kSelThreads < n_cand) keep(kc[i]);
-    for (int jj = tid + kCached * kSelThreads; jj < n_cand; jj += kSelThreads) keep(key64(jj));
-    __syncthreads();
-    const int ns = last_s < surv_cap ? last_s : surv_cap;
-    if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
-    for (int i = tid; i < ns; i += kSelThreads) {
-      const uint64_t c = surv[i];
-      int rank = 0;
-      for (int u = 0; u < ns; ++u) rank += surv[u] > c;
-      if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
     }
     __syncthreads();
+    const int ns1 = last_s < surv_cap ? last_s : surv_cap;
+    if (gs == 1) {
+      // groups are single candidates: the survivors are the candidate keys
+      // >= tau1, which hold the top k; rank them directly
+      if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
+      for (int i = tid; i < ns1; i += kSelThreads) {
+        const uint64_t c = surv[i];
+        int rank = 0;
+        for (int u = 0; u < ns1; ++u) rank += surv[u] > c;
+        if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
+      }
+      __syncthreads();
+    } else {
+      // tau2: the k-th largest group maximum (0 when there are fewer than k groups)
+      if (k <= ng) {
+        for (int i = tid; i < ns1; i += kSelThreads) {
+          const uint64_t c = surv[i];
+          int rank = 0;
+          for (int u = 0; u < ns1; ++u) rank += surv[u] > c;
+          if (rank == k - 1) tau_s = c;
+        }
+      } else if (tid == 0) {
+        tau_s = 0ull;
+      }
+      __syncthreads();
+      const uint64_t tau2 = tau_s;
+      if (tid == 0) last_s = 0;
+      __syncthreads();
+      for (int jj = tid; jj < n_cand; jj += kSelThreads) {
+        const uint64_t c = key64(jj);
+        if (c >= tau2) {
+          const int slot = atomicAdd(&last_s, 1);
+          if (slot < surv_cap) surv[slot] = c;
+        }
+      }
+      __syncthreads();
+      const int ns = last_s < surv_cap ? last_s : surv_cap;
+      if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
+      for (int i = tid; i < ns; i += kSelThreads) {
+        const uint64_t c = surv[i];
+        int rank = 0;
+        for (int u = 0; u < ns; ++u) rank += surv[u] > c;
+        if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
+      }
+      __syncthreads();
+    }
   } else if (partial && tid == 0) {
-    report(a.status, COBS_ERR_DEVICE);   // candidate flags do not fit (host limits prevent it)
+    report(a.status, COBS_ERR_DEVICE);   // host limits prevent this
   }
 
   // ---- sink blocks, chosen candidates ascending, local blocks -------------
@@ -413,6 +467,13 @@ int select_blocks_per_stage(int rank) { return kStageRows / (1 + rank); }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);
+}
+
+bool select_topk_fits(int d, int64_t n_cand, int top_k) {
+  if (top_k <= 0 || top_k >= n_cand) return true;   // no ranking needed
+  if (n_cand > (int64_t(1) << 24)) return false;
+  const int ring = kSelStages * (d / 64) * 128 * 128;
+  return topk_survivor_capacity(ring, int(n_cand)) >= topk_survivors_needed(int(n_cand), top_k);
 }
 
 }  // namespace cobs

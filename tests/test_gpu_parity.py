@@ -313,12 +313,15 @@ def test_planted_spectrum_blocks():
         assert rel is None or rel <= PROJ_RTOL
 
 
-@pytest.mark.parametrize("top_k", [127, 128, 200])
-def test_select_large_top_k(top_k):
-    """top_k at and above 128 candidates' worth of threads, with more candidates
-    than top_k: every candidate key is ranked; planted exact ties must still
-    be broken by the lower block index."""
-    w = W["single_32k"].scaled(seq_len=16384 + 5, batch=1, q_heads=8, kv_heads=2,
+@pytest.mark.parametrize("seq_len,top_k", [
+    (16384 + 5, 127), (16384 + 5, 128), (16384 + 5, 200),   # <= 1024 candidates
+    (80000 + 5, 100), (80000 + 5, 300),                       # grouped candidates
+])
+def test_select_large_top_k(seq_len, top_k):
+    """top_k below, at and above the 128 threads' worth of maxima, over fewer
+    and more than 1024 candidates (the grouped bound): the selection must be
+    exact; planted exact ties must still be broken by the lower block index."""
+    w = W["single_32k"].scaled(seq_len=seq_len, batch=1, q_heads=8, kv_heads=2,
                                top_k=top_k)
     p = Problem(w)
     recs = {}
