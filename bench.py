@@ -414,6 +414,21 @@ def run_cobs(args, w, rank, world, local_rank):
         raise RuntimeError(f"device status {cb.cobs_status_string(status)} after warm-up")
     sel_counts = n_sel.cpu().numpy()
     n_sel_mean = float(sel_counts.mean())
+    quality = None
+    if w.needles:
+        # needle-block recall of the GPU selection (a quality side-metric):
+        # planted needle blocks that made it into each (batch, kv-head) list
+        from workloads import needle_block_list
+        idx_h = idx.cpu().numpy()
+        hits = total = 0
+        for b in range(w.batch):
+            for h in range(w.kv_heads):
+                nb = needle_block_list(w, b, h)
+                chosen = set(idx_h[b, h, :sel_counts[b, h]].tolist())
+                hits += sum(int(j) in chosen for j in nb)
+                total += len(nb)
+        quality = {"needle_recall": hits / total if total else None,
+                   "needle_blocks": total}
 
     # timed region: the steps are replayed from CUDA graphs of g_steps steps
     # (L2 flush, stats, selection, decode and the per-step events captured),
@@ -623,6 +638,7 @@ def run_cobs(args, w, rank, world, local_rank):
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,
         "wall_ms_per_step": t_host,
+        "quality": quality,
         "kernel_breakdown": {"steps": n_kern, "ms_per_step": t_step_kern,
                              "note": "per-kernel times from a second graph-replayed run, "
                                      "the three kernels on one stream with events between "

@@ -157,3 +157,23 @@ def test_pointer_and_range_checks():
 def test_status_read_rejects_null_output():
     st = cb.lib.cobs_read_device_status(ctypes.c_void_p(1 << 20), 4096, None, None)
     assert st == cb.COBS_ERR_INVALID_ARG
+
+
+def test_selection_limits_are_checked_on_the_host():
+    """top_k above 4096, and settings whose exact top-k survivors could
+    overflow the selection kernel's shared memory, are refused before launch."""
+    A = 1 << 20
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w)
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_select_blocks(d, A, A, 100, 4097, 1, 64, A, 8192, A, None, A, 1 << 30)
+    assert e.value.status == cb.COBS_ERR_UNSUPPORTED
+    # head_dim 64 (a 48 KB record ring), a million-token cache, top_k 4000:
+    # the candidates above the grouped bound would need ~512 KB
+    d64 = dims_of(WORKLOADS["tiny_4k"], capacity_tokens=1 << 20)
+    nsm = cb.cobs_selected_capacity(d64, 4000, 1, 0)
+    ws = cb.cobs_workspace_bytes(d64, 4000, 1, 0)
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_select_blocks(d64, A, A, 1 << 20, 4000, 1, 0, A, nsm, A, None, A, ws)
+    assert e.value.status == cb.COBS_ERR_UNSUPPORTED
+    assert "shared memory" in cb.cobs_last_error()

@@ -147,6 +147,20 @@ def needle_blocks(w: Workload, b: int, h: int, spread: np.ndarray) -> np.ndarray
     return np.sort(g.choice(np.asarray(pool), size=w.needles, replace=False))
 
 
+def needle_block_list(w: Workload, b: int, h: int) -> np.ndarray:
+    """The blocks that make_kv_slice plants needles in for slice (b, h),
+    without drawing the keys: the same generator replays only the draws that
+    decide them (the block means, then the spread flags of the tight/spread
+    recipe), which must stay in step with _per_block."""
+    if not w.needles or w.keys != "tight_spread":
+        return np.zeros(0, np.int64)
+    n_blocks = -(-w.seq_len // w.block)
+    gk = _rng(w, _TAG_K, b, h)
+    gk.standard_normal((n_blocks, 1, w.head_dim), dtype=np.float32)   # block means
+    spread = gk.random(n_blocks) < 0.5
+    return needle_blocks(w, b, h, spread)
+
+
 def _per_block(g, n_blocks, B, d, recipe):
     """Draw [n_blocks * B, d] fp32 values for one recipe (plus spread flags)."""
     if recipe == "offset_scale":
