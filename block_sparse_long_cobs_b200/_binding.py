@@ -19,7 +19,8 @@ __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
     "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
-    "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_read_device_status",
+    "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
+    "cobs_sparse_decode_varlen", "cobs_read_device_status",
     "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
@@ -75,6 +76,9 @@ def _load() -> ctypes.CDLL:
         "cobs_select_blocks": (I32, [D, P, P, I64, I32, I32, I32, P, I32, P, P, P, SZ, P]),
         "cobs_sparse_decode": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P, SZ, P]),
         "cobs_sparse_decode_no_alloc": (I32, [D, P, P, P, P, P, I32, I64, F32, P, P, P]),
+        "cobs_select_blocks_varlen": (I32, [D, P, P, P, I64, I32, I32, I32, P, I32, P, P, P,
+                                            SZ, P]),
+        "cobs_sparse_decode_varlen": (I32, [D, P, P, P, P, P, I32, P, I64, F32, P, P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_last_error": (ctypes.c_char_p, []),
         "cobs_status_string": (ctypes.c_char_p, [I32]),
@@ -190,6 +194,28 @@ def cobs_sparse_decode_no_alloc(dims, q, k, v, idx, n_sel, idx_stride, seq_len,
                                          ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
                                          _stream(stream))
     return _check("cobs_sparse_decode_no_alloc", st, check)
+
+
+def cobs_select_blocks_varlen(dims, q, stats, seq_lens, max_seq_len, top_k, sink_blocks,
+                              local_tokens, idx, idx_stride, n_sel, scores_opt, ws, ws_bytes,
+                              stream=None, check=True) -> int:
+    """cobs_select_blocks with per-sequence lengths (seq_lens: device int64 [batch])."""
+    st = lib.cobs_select_blocks_varlen(ctypes.byref(_dims(dims)), _ptr(q), _ptr(stats),
+                                       _ptr(seq_lens), max_seq_len, top_k, sink_blocks,
+                                       local_tokens, _ptr(idx), idx_stride, _ptr(n_sel),
+                                       _ptr(scores_opt), _ptr(ws), ws_bytes, _stream(stream))
+    return _check("cobs_select_blocks_varlen", st, check)
+
+
+def cobs_sparse_decode_varlen(dims, q, k, v, idx, n_sel, idx_stride, seq_lens, max_seq_len,
+                              softmax_scale, out, lse, ws, ws_bytes, stream=None,
+                              check=True) -> int:
+    """cobs_sparse_decode with per-sequence lengths (seq_lens: device int64 [batch])."""
+    st = lib.cobs_sparse_decode_varlen(ctypes.byref(_dims(dims)), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(idx), _ptr(n_sel), idx_stride, _ptr(seq_lens),
+                                       max_seq_len, ctypes.c_float(softmax_scale), _ptr(out),
+                                       _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
+    return _check("cobs_sparse_decode_varlen", st, check)
 
 
 def cobs_read_device_status(ws, ws_bytes, stream=None) -> int:

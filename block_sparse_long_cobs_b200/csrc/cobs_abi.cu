@@ -323,11 +323,12 @@ cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k, int64_t
   return ok();
 }
 
-cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void* stats,
-                               int64_t seq_len, int32_t top_k, int32_t sink_blocks,
-                               int32_t local_tokens, int32_t* idx, int32_t idx_stride,
-                               int32_t* n_sel, float* scores_opt, void* ws, size_t ws_bytes,
-                               void* stream) {
+// seq_lens null: every sequence is seq_len long; else seq_len bounds them all.
+static cobs_status select_impl(const cobs_dims* dims, const void* q, const void* stats,
+                               const int64_t* seq_lens, int64_t seq_len, int32_t top_k,
+                               int32_t sink_blocks, int32_t local_tokens, int32_t* idx,
+                               int32_t idx_stride, int32_t* n_sel, float* scores_opt, void* ws,
+                               size_t ws_bytes, void* stream) {
   cobs_status st = check_dims(dims);
   if (st != COBS_OK) return st;
   if ((st = check_select_params(top_k, sink_blocks, local_tokens)) != COBS_OK) return st;
@@ -346,12 +347,12 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   const WorkspaceLayout L = layout(dims, nsm);
   if ((st = check_ws(ws, ws_bytes, L.partials)) != COBS_OK) return st;
 
-  // block partition: forced sink [0, sink_end), forced local [first_local, nbs)
-  const int64_t nbs = ceil_div(seq_len, kBlock);
-  const int64_t n_full = seq_len / kBlock;
-  int64_t first_local = (seq_len - local_tokens > 0 ? seq_len - local_tokens : 0) / kBlock;
-  if (first_local > n_full) first_local = n_full;
-  const int64_t sink_end = sink_blocks < first_local ? sink_blocks : first_local;
+  if (seq_lens && !aligned16(seq_lens))
+    return fail(COBS_ERR_INVALID_ARG, "seq_lens must be 16-byte aligned");
+  // block partition of a seq_len sequence (each sequence's own is derived on
+  // the device): forced sink [0, sink_end), forced local [first_local, nbs)
+  const BlockPartition BPm = block_partition(seq_len, sink_blocks, local_tokens);
+  const int64_t nbs = BPm.nbs, first_local = BPm.first_local, sink_end = BPm.sink_end;
   if (!select_topk_fits(dims->head_dim, first_local - sink_end, top_k))
     return fail(COBS_ERR_UNSUPPORTED,
                 "top_k %d over %lld candidate blocks exceeds the selection kernel's "
@@ -381,6 +382,10 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   a.sink_end = int32_t(sink_end);
   a.first_local = int32_t(first_local);
   a.top_k = top_k;
+  a.seq_lens = seq_lens;
+  a.max_seq_len = seq_len;
+  a.sink_blocks = sink_blocks;
+  a.local_tokens = local_tokens;
 
   // chunking: one wave of resident CTAs shared out over the (batch, kv-head)
   // pairs; every chunk is a whole number of stages (128 record rows each)
@@ -406,11 +411,32 @@ cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void*
   return ok();
 }
 
-cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void* k,
-                               const void* v, const int32_t* idx, const int32_t* n_sel,
-                               int32_t idx_stride, int64_t seq_len, float softmax_scale,
-                               float* out, float* lse, void* ws, size_t ws_bytes,
+cobs_status cobs_select_blocks(const cobs_dims* dims, const void* q, const void* stats,
+                               int64_t seq_len, int32_t top_k, int32_t sink_blocks,
+                               int32_t local_tokens, int32_t* idx, int32_t idx_stride,
+                               int32_t* n_sel, float* scores_opt, void* ws, size_t ws_bytes,
                                void* stream) {
+  return select_impl(dims, q, stats, nullptr, seq_len, top_k, sink_blocks, local_tokens, idx,
+                     idx_stride, n_sel, scores_opt, ws, ws_bytes, stream);
+}
+
+cobs_status cobs_select_blocks_varlen(const cobs_dims* dims, const void* q, const void* stats,
+                                      const int64_t* seq_lens, int64_t max_seq_len,
+                                      int32_t top_k, int32_t sink_blocks, int32_t local_tokens,
+                                      int32_t* idx, int32_t idx_stride, int32_t* n_sel,
+                                      float* scores_opt, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  if (!seq_lens) return fail(COBS_ERR_INVALID_ARG, "seq_lens must not be NULL");
+  return select_impl(dims, q, stats, seq_lens, max_seq_len, top_k, sink_blocks, local_tokens,
+                     idx, idx_stride, n_sel, scores_opt, ws, ws_bytes, stream);
+}
+
+// seq_lens null: every sequence is seq_len long; else seq_len bounds them all.
+static cobs_status decode_impl(const cobs_dims* dims, const void* q, const void* k,
+                               const void* v, const int32_t* idx, const int32_t* n_sel,
+                               int32_t idx_stride, const int64_t* seq_lens, int64_t seq_len,
+                               float softmax_scale, float* out, float* lse, void* ws,
+                               size_t ws_bytes, void* stream) {
   cobs_status st = check_dims(dims);
   if (st != COBS_OK) return st;
   if (!q || !k || !v || !idx || !n_sel || !out || !lse)
@@ -421,6 +447,8 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   if (seq_len < 1 || seq_len > dims->capacity_tokens)
     return fail(COBS_ERR_INVALID_ARG, "seq_len %lld outside [1, capacity_tokens]",
                 (long long)seq_len);
+  if (seq_lens && !aligned16(seq_lens))
+    return fail(COBS_ERR_INVALID_ARG, "seq_lens must be 16-byte aligned");
   if (idx_stride < 1) return fail(COBS_ERR_INVALID_ARG, "idx_stride must be >= 1");
   if (int64_t(dims->batch) * dims->num_kv_heads * idx_stride >= (int64_t(1) << 31))
     return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * idx_stride must be < 2^31");
@@ -443,6 +471,7 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   a.status = reinterpret_cast<int32_t*>(w + L.status);
   a.cap = dims->capacity_tokens;
   a.seq_len = seq_len;
+  a.seq_lens = seq_lens;
   a.batch = dims->batch;
   a.hq = dims->num_q_heads;
   a.hkv = dims->num_kv_heads;
@@ -463,6 +492,25 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
   cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
   return ok();
+}
+
+cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void* k,
+                               const void* v, const int32_t* idx, const int32_t* n_sel,
+                               int32_t idx_stride, int64_t seq_len, float softmax_scale,
+                               float* out, float* lse, void* ws, size_t ws_bytes,
+                               void* stream) {
+  return decode_impl(dims, q, k, v, idx, n_sel, idx_stride, nullptr, seq_len, softmax_scale,
+                     out, lse, ws, ws_bytes, stream);
+}
+
+cobs_status cobs_sparse_decode_varlen(const cobs_dims* dims, const void* q, const void* k,
+                                      const void* v, const int32_t* idx, const int32_t* n_sel,
+                                      int32_t idx_stride, const int64_t* seq_lens,
+                                      int64_t max_seq_len, float softmax_scale, float* out,
+                                      float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!seq_lens) return fail(COBS_ERR_INVALID_ARG, "seq_lens must not be NULL");
+  return decode_impl(dims, q, k, v, idx, n_sel, idx_stride, seq_lens, max_seq_len,
+                     softmax_scale, out, lse, ws, ws_bytes, stream);
 }
 
 cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_status,

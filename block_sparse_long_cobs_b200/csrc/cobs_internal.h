@@ -46,7 +46,31 @@ struct SelectArgs {
   int32_t top_k;
   int32_t chunk_blocks;     // candidates per CTA
   int32_t n_chunks;         // CTAs per (b, kv-head)
+  // per-sequence lengths (null: every sequence is max_seq_len tokens long);
+  // the fields above describe the partition of a max_seq_len sequence, each
+  // sequence's own partition is derived on the device (block_partition)
+  const int64_t* seq_lens;  // [b] or null
+  int64_t max_seq_len;
+  int32_t sink_blocks, local_tokens;
 };
+
+// Block partition of one sequence of `len` tokens (COBS explainer §2.1 and
+// the sliding-window glossary: sink blocks, local window, candidates between):
+// blocks [0, nbs); forced sink [0, sink_end); forced local [first_local, nbs);
+// candidates [sink_end, first_local).  Host and device use the same rule.
+struct BlockPartition {
+  int64_t nbs, sink_end, first_local;
+};
+__host__ __device__ inline BlockPartition block_partition(int64_t len, int32_t sink_blocks,
+                                                          int32_t local_tokens) {
+  BlockPartition P;
+  P.nbs = (len + kBlock - 1) / kBlock;
+  const int64_t n_full = len / kBlock;
+  int64_t fl = (len - local_tokens > 0 ? len - local_tokens : 0) / kBlock;
+  P.first_local = fl < n_full ? fl : n_full;
+  P.sink_end = sink_blocks < P.first_local ? sink_blocks : P.first_local;
+  return P;
+}
 
 // Arguments of the split-K decode kernel.
 struct DecodeArgs {
@@ -61,8 +85,9 @@ struct DecodeArgs {
   uint32_t* tickets;      // [b][Hkv]
   uint32_t* work;         // head_dim 128: [2] chunk counter, finished-CTA counter (start at 0)
   int32_t* status;
+  const int64_t* seq_lens;  // [b] per-sequence lengths or null (all seq_len)
   int64_t cap;
-  int64_t seq_len;
+  int64_t seq_len;        // the length, or with seq_lens the upper bound of every length
   int32_t batch, hq, hkv, d;
   int32_t idx_stride;
   int32_t part_stride;    // partial rows per query head (>= splits / segments of a pair)

@@ -131,7 +131,9 @@ sparse_decode_kernel(const DecodeArgs a) {
   const int p1 = min(p0 + a.blocks_per_split, nsel);
   const int nblk = max(0, p1 - p0);
   const int32_t* idx_row = a.idx + int64_t(bh) * a.idx_stride + p0;
-  const int64_t seq_blocks = (a.seq_len + kBlock - 1) / kBlock;
+  const int64_t len_b = sequence_length(a.seq_lens, a.seq_len, b, a.status,
+                                        split == 0 && tid == 0 && kvh == 0);
+  const int64_t seq_blocks = (len_b + kBlock - 1) / kBlock;
   const uint16_t* kbase = a.k + int64_t(bh) * a.cap * D;
   const uint16_t* vbase = a.v + int64_t(bh) * a.cap * D;
 
@@ -146,7 +148,7 @@ sparse_decode_kernel(const DecodeArgs a) {
     const int j = idx_row[i];
     int nv = 0;
     if (j >= 0 && int64_t(j) < seq_blocks) {
-      const int64_t rem = a.seq_len - int64_t(j) * kBlock;
+      const int64_t rem = len_b - int64_t(j) * kBlock;
       nv = int(rem < kBlock ? rem : kBlock);
     } else {
       report(a.status, COBS_ERR_DEVICE);

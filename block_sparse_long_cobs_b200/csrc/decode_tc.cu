@@ -36,7 +36,9 @@
 //    thread reads back the output row of one dimension.
 // Keys at or past seq_len read as zero through the tensor maps' row bound and
 // are masked; block indices outside [0, ceil(seq_len / B)) are reported and
-// read as empty.  Every wait is bounded; a CTA that gives up records
+// read as empty.  With per-sequence lengths the bound is the longest
+// sequence: the tail block of a shorter one brings rows past its end, which
+// the softmax warps zero in the V tile (after it lands, before P.V).  Every wait is bounded; a CTA that gives up records
 // COBS_ERR_TIMEOUT, lets its copies and MMAs finish, frees TMEM and returns.
 #include <cfloat>
 
@@ -166,6 +168,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     if (tid == 0) report(a.status, COBS_ERR_DEVICE);
     return;
   }
+  // blocks of the longest sequence (the tensor maps' row bound is seq_len)
   const int64_t seq_blocks = (a.seq_len + kBlock - 1) / kBlock;
 
   if (tid == 0) {
@@ -234,14 +237,18 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           const int32_t* row = a.idx + g.pair * a.idx_stride + g.s0;
           const int z = int(g.pair);
           const int qrow = int((g.pair / a.hkv) * a.hq + (g.pair % a.hkv) * G);
+          const int64_t len_b =
+              sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status, false);
+          const int64_t blocks_b = (len_b + kBlock - 1) / kBlock;
           uint8_t* qbuf = base + kOffQ + (nonempty & 1) * 2048;
           for (int t = 0; t < T && ok; ++t) {
             const int nh = (2 * t + 1 < g.nb) ? 2 : 1;
             int y[2] = {0, 0};
             for (int h2 = 0; h2 < nh; ++h2) {
               const int j = row[2 * t + h2];
-              // an index outside the sequence reads an all-zero box past seq_len
-              y[h2] = (j >= 0 && j < seq_blocks) ? j * kBlock : int(seq_blocks * kBlock);
+              // an index outside the sequence reads an all-zero box past the
+              // tensor maps' row bound
+              y[h2] = (j >= 0 && j < blocks_b) ? j * kBlock : int(seq_blocks * kBlock);
             }
             for (int kv = 0; kv < 2; ++kv, ++it) {   // K_t then V_t
               const int st = it % kStages;
@@ -370,6 +377,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const int64_t hstride = int64_t(a.part_stride) * (kD + 2);
     uint32_t gt = 0;   // score tiles consumed (all segments)
     uint32_t pt = 0;   // P tiles produced
+    uint32_t items = 0;   // ring items of the segments done (2 per tile)
     int nonempty = 0;
     bool ok = true;
 
@@ -491,22 +499,30 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       const int ob = nonempty & 1;
       const uint32_t use = uint32_t(nonempty) >> 1;
+      const int64_t len_b = sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status,
+                                            g.seg == 0 && r == 0);
+      const int64_t blocks_b = (len_b + kBlock - 1) / kBlock;
       if (g.nb > 0) {
         const uint32_t ocol = kOCol + 16u * uint32_t(ob);
         const int T = (g.nb + 1) >> 1;
         const int32_t* row = a.idx + g.pair * a.idx_stride + g.s0;
+        const uint32_t it0 = items;   // ring item of K_0 (V_t is it0 + 2t + 1)
         for (int t = 0; t < T; ++t, ++gt, ++pt) {
           const int sb = gt & 1;
           const int slot = pt % kPSlots;
           // this thread's key: validity from the block index
           const int blk = 2 * t + half;
-          bool valid = false;
+          bool valid = false, zero_row = false;
           if (blk < g.nb) {
             const int j = row[blk];
-            if (j >= 0 && j < seq_blocks)
-              valid = int64_t(j) * kBlock + kk < a.seq_len;
-            else if (kk == 0)
+            if (j >= 0 && j < blocks_b) {
+              valid = int64_t(j) * kBlock + kk < len_b;
+              // a key past this sequence but inside the tensor maps' bound
+              // (per-sequence lengths only) arrives as whatever the cache holds
+              zero_row = !valid;
+            } else if (kk == 0) {
               report(a.status, COBS_ERR_DEVICE);
+            }
           }
           fail = abort_s != 0;
           if (r == 0) {
@@ -592,11 +608,33 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
               *reinterpret_cast<uint16_t*>(atom + 1024 + off) = lo;
             }
           }
+          if (a.seq_lens != nullptr && named_bar_or(1, kSoftThreads, zero_row)) {
+            // the tail block of a shorter sequence: its V rows past the
+            // sequence must be zero before P.V (a zero weight times a stale
+            // or NaN value is not zero), so wait for the tile and clear them
+            const uint32_t vit = it0 + 2u * uint32_t(t) + 1u;
+            fail = abort_s != 0;
+            if (r == 0)
+              fail = !wait_or_abort(&full[vit % kStages], (vit / kStages) & 1, a.status, &abort_s);
+            if (named_bar_or(1, kSoftThreads, fail)) {
+              ok = false;
+              break;
+            }
+            if (zero_row) {
+              uint8_t* vt = base + kOffRing + (vit % kStages) * kStageBytes + r * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                *reinterpret_cast<uint4*>(vt + c * 16) = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(vt + kSlabBytes + c * 16) = make_uint4(0, 0, 0, 0);
+              }
+            }
+          }
           fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&p_full[slot]);
         }
         if (!ok) break;
+        items += 2u * uint32_t(T);
         ++nonempty;
       }
       // the previous segment's products are complete by now: write its output

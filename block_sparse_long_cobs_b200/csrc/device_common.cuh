@@ -62,6 +62,19 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Length of sequence b: seq_lens[b] when per-sequence lengths are given
+// (clamped to [1, max_len], an out-of-range value reported), else max_len.
+__device__ __forceinline__ int64_t sequence_length(const int64_t* seq_lens, int64_t max_len,
+                                                   int64_t b, int32_t* status, bool reporter) {
+  if (seq_lens == nullptr) return max_len;
+  int64_t len = seq_lens[b];
+  if (len < 1 || len > max_len) {
+    if (reporter) report(status, COBS_ERR_DEVICE);
+    len = len < 1 ? 1 : max_len;
+  }
+  return len;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -8,7 +8,9 @@
 // Selection (§2.1: rank blocks by attention mass; sliding-window glossary:
 // attention sink + local window):  the top_k complete blocks outside the
 // forced sets, ties to the lower block index, united with the sink blocks and
-// the local/tail blocks, written in ascending order.
+// the local/tail blocks, written in ascending order.  With per-sequence
+// lengths each sequence has its own partition (block_partition); chunks are
+// laid out for the longest and cut to each sequence's own candidates.
 //
 // Phase 1, grid (chunk, kv-head, batch), 128 threads: the dot products of
 // every record row with the G queries form a dense contraction
@@ -102,11 +104,18 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   uint8_t* stage = base + kQBytes;                  // [kSelStages][kRegions][128][128 B]
 
   float* scores = a.scores_ws + int64_t(bh) * a.nb_cap;
+  // this sequence's block partition
+  const int64_t seq_len_b =
+      sequence_length(a.seq_lens, a.max_seq_len, b, a.status, chunk == 0 && tid == 0 && kvh == 0);
+  const BlockPartition BP = block_partition(seq_len_b, a.sink_blocks, a.local_tokens);
 
   // ===================== phase 1: scores of this chunk =====================
   {
-    const int c_lo = a.cand_begin + chunk * a.chunk_blocks;
-    const int c_hi = min(a.cand_end, c_lo + a.chunk_blocks);
+    // this chunk's share of the candidates of a max_seq_len sequence, cut to
+    // this sequence's own candidates [sink_end, first_local)
+    const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
+    const int c_lo = max(int(BP.sink_end), c_nom);
+    const int c_hi = min(int(BP.first_local), min(a.cand_end, c_nom + a.chunk_blocks));
     const int npass = c_hi > c_lo ? (c_hi - c_lo + per_stage - 1) / per_stage : 0;
     const int64_t row0 = (int64_t(bh) * a.nb_cap) * rows;   // first row of this pair
 
@@ -261,9 +270,10 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     __syncthreads();   // every score of the pair is written
   }
 
-  const int c0 = a.cand_begin, c1 = a.cand_end;
+  const int c0 = int(BP.sink_end), c1 = int(BP.first_local);
   const int n_cand = c1 - c0;
-  const int nbs = a.seq_len_blocks;
+  const int nbs = int(BP.nbs);
+  const int sink_end = int(BP.sink_end), first_local = int(BP.first_local);
   const int k = a.top_k < n_cand ? a.top_k : n_cand;
   const bool partial = (k > 0 && k < n_cand);
 
@@ -377,11 +387,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
 
   // ---- sink blocks, chosen candidates ascending, local blocks -------------
   int32_t* out = a.idx + int64_t(bh) * a.idx_stride;
-  const int n_local = nbs - a.first_local;
-  const int total = a.sink_end + k + n_local;
+  const int n_local = nbs - first_local;
+  const int total = sink_end + k + n_local;
   if (warp == 0) {
-    for (int i = lane; i < a.sink_end && i < a.idx_stride; i += 32) out[i] = i;
-    int pos = a.sink_end;
+    for (int i = lane; i < sink_end && i < a.idx_stride; i += 32) out[i] = i;
+    int pos = sink_end;
     if (partial && fits) {
       for (int j0 = 0; j0 < n_cand; j0 += 32) {
         const int jj = j0 + lane;
@@ -399,7 +409,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       pos += k;
     }
     for (int i = lane; i < n_local; i += 32)
-      if (pos + i < a.idx_stride) out[pos + i] = a.first_local + i;
+      if (pos + i < a.idx_stride) out[pos + i] = first_local + i;
     if (lane == 0) {
       if (total > a.idx_stride) report(a.status, COBS_ERR_DEVICE);
       a.n_sel[bh] = total < a.idx_stride ? total : a.idx_stride;

@@ -176,6 +176,35 @@ COBS_API cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q,
                                float softmax_scale, float* out, float* lse,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* Per-sequence lengths (ragged batches; this library's widening of the
+ * method's single-length statement of the problem).  Same as
+ * cobs_select_blocks / cobs_sparse_decode, except that sequence b is
+ * seq_lens[b] tokens long:
+ *   seq_lens     device [batch] int64, 16-byte aligned; each in
+ *                [1, max_seq_len] (a value outside is clamped on the device
+ *                and reported as COBS_ERR_DEVICE through the status word).
+ *   max_seq_len  host bound of every length, 1 <= max_seq_len <=
+ *                capacity_tokens; it sizes the launch (candidate chunks,
+ *                tensor-map extents), so keep it tight.
+ * Each sequence has its own block partition: sink blocks, its local window
+ * (every block intersecting its last local_tokens tokens, including its
+ * partial tail block) and the complete blocks between as candidates.
+ * idx_stride, workspace and outputs are as for the single-length calls. */
+COBS_API cobs_status cobs_select_blocks_varlen(const cobs_dims* dims, const void* q,
+                                      const void* stats, const int64_t* seq_lens,
+                                      int64_t max_seq_len, int32_t top_k,
+                                      int32_t sink_blocks, int32_t local_tokens,
+                                      int32_t* idx, int32_t idx_stride, int32_t* n_sel,
+                                      float* scores_opt, void* ws, size_t ws_bytes,
+                                      void* stream);
+COBS_API cobs_status cobs_sparse_decode_varlen(const cobs_dims* dims, const void* q,
+                                      const void* k, const void* v,
+                                      const int32_t* idx, const int32_t* n_sel,
+                                      int32_t idx_stride, const int64_t* seq_lens,
+                                      int64_t max_seq_len, float softmax_scale,
+                                      float* out, float* lse, void* ws,
+                                      size_t ws_bytes, void* stream);
+
 /* Allocation-free form of cobs_sparse_decode (this library's own addition; the
  * method's description has no counterpart).  Same arguments and results, but
  * there is no workspace argument: the split-K partial results and arrival

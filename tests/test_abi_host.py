@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) == 11, names
+    assert len(names) == 13, names
     raw = ctypes.CDLL(cb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
@@ -177,3 +177,23 @@ def test_selection_limits_are_checked_on_the_host():
         cb.cobs_select_blocks(d64, A, A, 1 << 20, 4000, 1, 0, A, nsm, A, None, A, ws)
     assert e.value.status == cb.COBS_ERR_UNSUPPORTED
     assert "shared memory" in cb.cobs_last_error()
+
+
+def test_varlen_host_checks():
+    A = 1 << 20
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w)
+    ws = cb.cobs_workspace_bytes(d, w.top_k, 1, w.local_tokens)
+    nsm = cb.cobs_selected_capacity(d, w.top_k, 1, w.local_tokens)
+    sel = lambda lens, mx: cb.cobs_select_blocks_varlen(d, A, A, lens, mx, w.top_k, 1,
+                                                        w.local_tokens, A, nsm, A, None, A, ws)
+    dec = lambda lens, mx: cb.cobs_sparse_decode_varlen(d, A, A, A, A, A, nsm, lens, mx, 0.1,
+                                                        A, A, A, ws)
+    for call in (sel, dec):
+        for lens, mx, code in [(None, 100, cb.COBS_ERR_INVALID_ARG),
+                               (A + 8, 100, cb.COBS_ERR_INVALID_ARG),
+                               (A, 0, cb.COBS_ERR_INVALID_ARG),
+                               (A, w.cap + 1, cb.COBS_ERR_INVALID_ARG)]:
+            with pytest.raises(cb.CobsError) as e:
+                call(lens, mx)
+            assert e.value.status == code
