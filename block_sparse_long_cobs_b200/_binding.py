@@ -20,8 +20,8 @@ __all__ = [
     "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
-    "cobs_sparse_decode_varlen", "cobs_read_device_status",
-    "cobs_last_error",
+    "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
+    "cobs_read_device_status", "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",
@@ -79,6 +79,9 @@ def _load() -> ctypes.CDLL:
         "cobs_select_blocks_varlen": (I32, [D, P, P, P, I64, I32, I32, I32, P, I32, P, P, P,
                                             SZ, P]),
         "cobs_sparse_decode_varlen": (I32, [D, P, P, P, P, P, I32, P, I64, F32, P, P, P, SZ, P]),
+        "cobs_build_block_stats_paged": (I32, [D, P, I64, P, I32, I64, I64, P, P, SZ, P]),
+        "cobs_sparse_decode_paged": (I32, [D, P, P, P, I64, P, I32, P, P, I32, P, I64, F32, P,
+                                           P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_last_error": (ctypes.c_char_p, []),
         "cobs_status_string": (ctypes.c_char_p, [I32]),
@@ -216,6 +219,30 @@ def cobs_sparse_decode_varlen(dims, q, k, v, idx, n_sel, idx_stride, seq_lens, m
                                        max_seq_len, ctypes.c_float(softmax_scale), _ptr(out),
                                        _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
     return _check("cobs_sparse_decode_varlen", st, check)
+
+
+def cobs_build_block_stats_paged(dims, k_pool, n_pages, block_table, table_stride,
+                                 block_begin, block_end, stats, ws, ws_bytes, stream=None,
+                                 check=True) -> int:
+    """cobs_build_block_stats over a page pool [n_pages, Hkv, 64, d] addressed through
+    block_table (device int32 [batch, table_stride])."""
+    st = lib.cobs_build_block_stats_paged(ctypes.byref(_dims(dims)), _ptr(k_pool), n_pages,
+                                          _ptr(block_table), table_stride, block_begin,
+                                          block_end, _ptr(stats), _ptr(ws), ws_bytes,
+                                          _stream(stream))
+    return _check("cobs_build_block_stats_paged", st, check)
+
+
+def cobs_sparse_decode_paged(dims, q, k_pool, v_pool, n_pages, block_table, table_stride,
+                             idx, n_sel, idx_stride, seq_lens, max_seq_len, softmax_scale,
+                             out, lse, ws, ws_bytes, stream=None, check=True) -> int:
+    """cobs_sparse_decode over page pools; seq_lens (device int64 [batch]) or None."""
+    st = lib.cobs_sparse_decode_paged(ctypes.byref(_dims(dims)), _ptr(q), _ptr(k_pool),
+                                      _ptr(v_pool), n_pages, _ptr(block_table), table_stride,
+                                      _ptr(idx), _ptr(n_sel), idx_stride, _ptr(seq_lens),
+                                      max_seq_len, ctypes.c_float(softmax_scale), _ptr(out),
+                                      _ptr(lse), _ptr(ws), ws_bytes, _stream(stream))
+    return _check("cobs_sparse_decode_paged", st, check)
 
 
 def cobs_read_device_status(ws, ws_bytes, stream=None) -> int:

@@ -248,6 +248,61 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
 
 using namespace cobs;
 
+// block_table null: the contiguous cache [batch, Hkv, capacity_tokens, d];
+// else a page pool [n_pages, Hkv, 64, d] addressed through the table.
+static cobs_status check_paging(const cobs_dims* dims, const int32_t* block_table,
+                                int32_t table_stride, int64_t n_pages, int64_t blocks_needed) {
+  if (!block_table) return COBS_OK;
+  if (!aligned16(block_table))
+    return fail(COBS_ERR_INVALID_ARG, "block_table must be 16-byte aligned");
+  if (table_stride < 1 || table_stride < blocks_needed)
+    return fail(COBS_ERR_INVALID_ARG, "table_stride %d below the %lld blocks addressed",
+                int(table_stride), (long long)blocks_needed);
+  if (n_pages < 1) return fail(COBS_ERR_INVALID_ARG, "n_pages must be >= 1");
+  if (n_pages * dims->num_kv_heads * kBlock >= (int64_t(1) << 31))
+    return fail(COBS_ERR_UNSUPPORTED, "n_pages * num_kv_heads * 64 must be < 2^31");
+  if (int64_t(dims->batch) * table_stride >= (int64_t(1) << 31))
+    return fail(COBS_ERR_UNSUPPORTED, "batch * table_stride must be < 2^31");
+  return COBS_OK;
+}
+
+static cobs_status stats_impl(const cobs_dims* dims, const void* k, const int32_t* block_table,
+                              int32_t table_stride, int64_t n_pages, int64_t block_begin,
+                              int64_t block_end, void* stats, void* ws, size_t ws_bytes,
+                              void* stream) {
+  cobs_status st = check_dims(dims);
+  if (st != COBS_OK) return st;
+  if (!k || !stats) return fail(COBS_ERR_INVALID_ARG, "k and stats must not be NULL");
+  if (!aligned16(k) || !aligned16(stats))
+    return fail(COBS_ERR_INVALID_ARG, "k and stats must be 16-byte aligned");
+  const int64_t nb_cap = dims->capacity_tokens / kBlock;
+  if (block_begin < 0 || block_end < block_begin || block_end > nb_cap)
+    return fail(COBS_ERR_INVALID_ARG, "block range [%lld, %lld) outside [0, %lld]",
+                (long long)block_begin, (long long)block_end, (long long)nb_cap);
+  if ((st = check_paging(dims, block_table, table_stride, n_pages, block_end)) != COBS_OK)
+    return st;
+  if ((st = check_ws(ws, ws_bytes, kStatusBytes)) != COBS_OK) return st;
+  if (block_end == block_begin) return ok();
+  StatsArgs a{};
+  a.k = static_cast<const uint16_t*>(k);
+  a.stats = static_cast<uint16_t*>(stats);
+  a.status = reinterpret_cast<int32_t*>(static_cast<char*>(ws));
+  a.cap = dims->capacity_tokens;
+  a.nb_cap = nb_cap;
+  a.block_begin = block_begin;
+  a.block_end = block_end;
+  a.batch = dims->batch;
+  a.hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.rank = dims->rank;
+  a.block_table = block_table;
+  a.table_stride = table_stride;
+  a.n_pages = n_pages;
+  cudaError_t e = launch_stats(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "block statistics launch");
+  return ok();
+}
+
 extern "C" {
 
 int32_t cobs_abi_version(void) { return COBS_ABI_VERSION; }
@@ -295,32 +350,18 @@ cobs_status cobs_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 cobs_status cobs_build_block_stats(const cobs_dims* dims, const void* k, int64_t block_begin,
                                    int64_t block_end, void* stats, void* ws, size_t ws_bytes,
                                    void* stream) {
-  cobs_status st = check_dims(dims);
-  if (st != COBS_OK) return st;
-  if (!k || !stats) return fail(COBS_ERR_INVALID_ARG, "k and stats must not be NULL");
-  if (!aligned16(k) || !aligned16(stats))
-    return fail(COBS_ERR_INVALID_ARG, "k and stats must be 16-byte aligned");
-  const int64_t nb_cap = dims->capacity_tokens / kBlock;
-  if (block_begin < 0 || block_end < block_begin || block_end > nb_cap)
-    return fail(COBS_ERR_INVALID_ARG, "block range [%lld, %lld) outside [0, %lld]",
-                (long long)block_begin, (long long)block_end, (long long)nb_cap);
-  if ((st = check_ws(ws, ws_bytes, kStatusBytes)) != COBS_OK) return st;
-  if (block_end == block_begin) return ok();
-  StatsArgs a{};
-  a.k = static_cast<const uint16_t*>(k);
-  a.stats = static_cast<uint16_t*>(stats);
-  a.status = reinterpret_cast<int32_t*>(static_cast<char*>(ws));
-  a.cap = dims->capacity_tokens;
-  a.nb_cap = nb_cap;
-  a.block_begin = block_begin;
-  a.block_end = block_end;
-  a.batch = dims->batch;
-  a.hkv = dims->num_kv_heads;
-  a.d = dims->head_dim;
-  a.rank = dims->rank;
-  cudaError_t e = launch_stats(a, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "block statistics launch");
-  return ok();
+  return stats_impl(dims, k, nullptr, 0, 0, block_begin, block_end, stats, ws, ws_bytes,
+                    stream);
+}
+
+cobs_status cobs_build_block_stats_paged(const cobs_dims* dims, const void* k_pool,
+                                         int64_t n_pages, const int32_t* block_table,
+                                         int32_t table_stride, int64_t block_begin,
+                                         int64_t block_end, void* stats, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  if (!block_table) return fail(COBS_ERR_INVALID_ARG, "block_table must not be NULL");
+  return stats_impl(dims, k_pool, block_table, table_stride, n_pages, block_begin, block_end,
+                    stats, ws, ws_bytes, stream);
 }
 
 // seq_lens null: every sequence is seq_len long; else seq_len bounds them all.
@@ -432,8 +473,10 @@ cobs_status cobs_select_blocks_varlen(const cobs_dims* dims, const void* q, cons
 }
 
 // seq_lens null: every sequence is seq_len long; else seq_len bounds them all.
+// block_table null: k and v are the contiguous cache; else page pools.
 static cobs_status decode_impl(const cobs_dims* dims, const void* q, const void* k,
-                               const void* v, const int32_t* idx, const int32_t* n_sel,
+                               const void* v, const int32_t* block_table, int32_t table_stride,
+                               int64_t n_pages, const int32_t* idx, const int32_t* n_sel,
                                int32_t idx_stride, const int64_t* seq_lens, int64_t seq_len,
                                float softmax_scale, float* out, float* lse, void* ws,
                                size_t ws_bytes, void* stream) {
@@ -454,6 +497,9 @@ static cobs_status decode_impl(const cobs_dims* dims, const void* q, const void*
     return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * idx_stride must be < 2^31");
   if (!(std::isfinite(softmax_scale)) || softmax_scale <= 0.f)
     return fail(COBS_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if ((st = check_paging(dims, block_table, table_stride, n_pages,
+                         (seq_len + kBlock - 1) / kBlock)) != COBS_OK)
+    return st;
   const WorkspaceLayout L = layout(dims, idx_stride);
   if ((st = check_ws(ws, ws_bytes, L.total)) != COBS_OK) return st;
 
@@ -472,6 +518,9 @@ static cobs_status decode_impl(const cobs_dims* dims, const void* q, const void*
   a.cap = dims->capacity_tokens;
   a.seq_len = seq_len;
   a.seq_lens = seq_lens;
+  a.block_table = block_table;
+  a.table_stride = table_stride;
+  a.n_pages = n_pages;
   a.batch = dims->batch;
   a.hq = dims->num_q_heads;
   a.hkv = dims->num_kv_heads;
@@ -499,8 +548,8 @@ cobs_status cobs_sparse_decode(const cobs_dims* dims, const void* q, const void*
                                int32_t idx_stride, int64_t seq_len, float softmax_scale,
                                float* out, float* lse, void* ws, size_t ws_bytes,
                                void* stream) {
-  return decode_impl(dims, q, k, v, idx, n_sel, idx_stride, nullptr, seq_len, softmax_scale,
-                     out, lse, ws, ws_bytes, stream);
+  return decode_impl(dims, q, k, v, nullptr, 0, 0, idx, n_sel, idx_stride, nullptr, seq_len,
+                     softmax_scale, out, lse, ws, ws_bytes, stream);
 }
 
 cobs_status cobs_sparse_decode_varlen(const cobs_dims* dims, const void* q, const void* k,
@@ -509,8 +558,21 @@ cobs_status cobs_sparse_decode_varlen(const cobs_dims* dims, const void* q, cons
                                       int64_t max_seq_len, float softmax_scale, float* out,
                                       float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!seq_lens) return fail(COBS_ERR_INVALID_ARG, "seq_lens must not be NULL");
-  return decode_impl(dims, q, k, v, idx, n_sel, idx_stride, seq_lens, max_seq_len,
-                     softmax_scale, out, lse, ws, ws_bytes, stream);
+  return decode_impl(dims, q, k, v, nullptr, 0, 0, idx, n_sel, idx_stride, seq_lens,
+                     max_seq_len, softmax_scale, out, lse, ws, ws_bytes, stream);
+}
+
+cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void* q, const void* k_pool,
+                                     const void* v_pool, int64_t n_pages,
+                                     const int32_t* block_table, int32_t table_stride,
+                                     const int32_t* idx, const int32_t* n_sel,
+                                     int32_t idx_stride, const int64_t* seq_lens,
+                                     int64_t max_seq_len, float softmax_scale, float* out,
+                                     float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!block_table) return fail(COBS_ERR_INVALID_ARG, "block_table must not be NULL");
+  return decode_impl(dims, q, k_pool, v_pool, block_table, table_stride, n_pages, idx, n_sel,
+                     idx_stride, seq_lens, max_seq_len, softmax_scale, out, lse, ws, ws_bytes,
+                     stream);
 }
 
 cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_status,

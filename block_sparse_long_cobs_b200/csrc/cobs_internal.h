@@ -86,6 +86,11 @@ struct DecodeArgs {
   uint32_t* work;         // head_dim 128: [2] chunk counter, finished-CTA counter (start at 0)
   int32_t* status;
   const int64_t* seq_lens;  // [b] per-sequence lengths or null (all seq_len)
+  // paged cache: k and v are page pools [n_pages][Hkv][B][d]; block j of
+  // sequence b is page block_table[b * table_stride + j] (null: contiguous)
+  const int32_t* block_table;
+  int32_t table_stride;
+  int64_t n_pages;
   int64_t cap;
   int64_t seq_len;        // the length, or with seq_lens the upper bound of every length
   int32_t batch, hq, hkv, d;
@@ -109,13 +114,17 @@ struct DecodePlan {
 
 // Arguments of the block-statistics kernel.
 struct StatsArgs {
-  const uint16_t* k;      // [b][Hkv][cap][d]
+  const uint16_t* k;      // [b][Hkv][cap][d], or the page pool [n_pages][Hkv][B][d]
   uint16_t* stats;        // [b][Hkv][nb_cap][1+r][d]
   int32_t* status;
   int64_t cap;
   int64_t nb_cap;
   int64_t block_begin, block_end;
   int32_t batch, hkv, d, rank;
+  // paged cache: block j of sequence b is page block_table[b * table_stride + j]
+  const int32_t* block_table;   // null: contiguous cache
+  int32_t table_stride;
+  int64_t n_pages;
 };
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);

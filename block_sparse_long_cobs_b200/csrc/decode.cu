@@ -134,8 +134,11 @@ sparse_decode_kernel(const DecodeArgs a) {
   const int64_t len_b = sequence_length(a.seq_lens, a.seq_len, b, a.status,
                                         split == 0 && tid == 0 && kvh == 0);
   const int64_t seq_blocks = (len_b + kBlock - 1) / kBlock;
-  const uint16_t* kbase = a.k + int64_t(bh) * a.cap * D;
-  const uint16_t* vbase = a.v + int64_t(bh) * a.cap * D;
+  // contiguous cache: this pair's rows; page pool: the pool itself, a page
+  // holding the Hkv heads' 64-row blocks one after another
+  const int64_t pair_off = a.block_table != nullptr ? 0 : int64_t(bh) * a.cap * D;
+  const uint16_t* kbase = a.k + pair_off;
+  const uint16_t* vbase = a.v + pair_off;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
@@ -147,9 +150,20 @@ sparse_decode_kernel(const DecodeArgs a) {
   auto issue = [&](int i, int st) {  // called by thread 0 only
     const int j = idx_row[i];
     int nv = 0;
+    int64_t off = 0;   // element offset of the block's first row
     if (j >= 0 && int64_t(j) < seq_blocks) {
       const int64_t rem = len_b - int64_t(j) * kBlock;
       nv = int(rem < kBlock ? rem : kBlock);
+      off = int64_t(j) * kBlock * D;
+      if (a.block_table != nullptr) {
+        const int32_t page = a.block_table[int64_t(b) * a.table_stride + j];
+        if (page >= 0 && page < a.n_pages) {
+          off = (int64_t(page) * a.hkv + kvh) * kBlock * D;
+        } else {
+          report(a.status, COBS_ERR_DEVICE);
+          nv = 0;
+        }
+      }
     } else {
       report(a.status, COBS_ERR_DEVICE);
     }
@@ -157,8 +171,8 @@ sparse_decode_kernel(const DecodeArgs a) {
     const uint32_t bytes = uint32_t(nv) * D * 2;
     mbar_arrive_expect_tx(&full[st], 2 * bytes);
     if (nv > 0) {
-      bulk_g2s(ks + st * S::kTileElems, kbase + int64_t(j) * kBlock * D, bytes, &full[st]);
-      bulk_g2s(vs + st * S::kTileElems, vbase + int64_t(j) * kBlock * D, bytes, &full[st]);
+      bulk_g2s(ks + st * S::kTileElems, kbase + off, bytes, &full[st]);
+      bulk_g2s(vs + st * S::kTileElems, vbase + off, bytes, &full[st]);
     }
   };
 

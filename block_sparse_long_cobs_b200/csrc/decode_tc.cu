@@ -243,12 +243,22 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           uint8_t* qbuf = base + kOffQ + (nonempty & 1) * 2048;
           for (int t = 0; t < T && ok; ++t) {
             const int nh = (2 * t + 1 < g.nb) ? 2 : 1;
-            int y[2] = {0, 0};
+            int y[2] = {0, 0}, zz[2] = {z, z};
             for (int h2 = 0; h2 < nh; ++h2) {
               const int j = row[2 * t + h2];
-              // an index outside the sequence reads an all-zero box past the
-              // tensor maps' row bound
-              y[h2] = (j >= 0 && j < blocks_b) ? j * kBlock : int(seq_blocks * kBlock);
+              // an index outside the sequence (or a page outside the pool)
+              // reads an all-zero box past the tensor maps' row bound
+              const bool in_seq = j >= 0 && j < blocks_b;
+              if (a.block_table == nullptr) {
+                y[h2] = in_seq ? j * kBlock : int(seq_blocks * kBlock);
+              } else {
+                const int32_t page =
+                    in_seq ? a.block_table[(g.pair / a.hkv) * a.table_stride + j] : -1;
+                const bool ok_page = page >= 0 && page < a.n_pages;
+                y[h2] = ok_page ? 0 : kBlock;
+                zz[h2] = ok_page ? int(int64_t(page) * a.hkv + g.pair % a.hkv) : 0;
+                if (in_seq && !ok_page) report(a.status, COBS_ERR_DEVICE);
+              }
             }
             for (int kv = 0; kv < 2; ++kv, ++it) {   // K_t then V_t
               const int st = it % kStages;
@@ -267,8 +277,9 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
               const CUtensorMap* map = kv ? &vmap : &kmap;
               uint8_t* dst = base + kOffRing + st * kStageBytes;
               for (int h2 = 0; h2 < nh; ++h2) {
-                tma_load_3d(dst + h2 * kHalfBytes, map, 0, y[h2], z, &full[st]);
-                tma_load_3d(dst + kSlabBytes + h2 * kHalfBytes, map, 64, y[h2], z, &full[st]);
+                tma_load_3d(dst + h2 * kHalfBytes, map, 0, y[h2], zz[h2], &full[st]);
+                tma_load_3d(dst + kSlabBytes + h2 * kHalfBytes, map, 64, y[h2], zz[h2],
+                            &full[st]);
               }
             }
           }
@@ -518,7 +529,8 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             if (j >= 0 && j < blocks_b) {
               valid = int64_t(j) * kBlock + kk < len_b;
               // a key past this sequence but inside the tensor maps' bound
-              // (per-sequence lengths only) arrives as whatever the cache holds
+              // (per-sequence lengths, or the unused rows of a last page)
+              // arrives as whatever the cache holds
               zero_row = !valid;
             } else if (kk == 0) {
               report(a.status, COBS_ERR_DEVICE);
@@ -608,7 +620,8 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
               *reinterpret_cast<uint16_t*>(atom + 1024 + off) = lo;
             }
           }
-          if (a.seq_lens != nullptr && named_bar_or(1, kSoftThreads, zero_row)) {
+          if ((a.seq_lens != nullptr || a.block_table != nullptr) &&
+              named_bar_or(1, kSoftThreads, zero_row)) {
             // the tail block of a shorter sequence: its V rows past the
             // sequence must be zero before P.V (a zero weight times a stale
             // or NaN value is not zero), so wait for the tile and clear them
@@ -671,13 +684,16 @@ int occupancy_g() {
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
   CUtensorMap kmap, vmap, qmap;
-  const uint64_t pairs = uint64_t(a.batch) * a.hkv;
-  const uint64_t pair_bytes = uint64_t(a.cap) * kD * 2;
-  cudaError_t e = make_bf16_tensor_map_3d_sw128(&kmap, a.k, kD, uint64_t(a.seq_len), pairs,
-                                                pair_bytes, kBlock);
+  // contiguous cache: (dim, token < seq_len, pair); page pool: (dim, row of
+  // the page, page x Hkv + kv-head)
+  const bool paged = a.block_table != nullptr;
+  const uint64_t rows = paged ? uint64_t(kBlock) : uint64_t(a.seq_len);
+  const uint64_t depth = paged ? uint64_t(a.n_pages) * a.hkv : uint64_t(a.batch) * a.hkv;
+  const uint64_t depth_bytes = (paged ? uint64_t(kBlock) : uint64_t(a.cap)) * kD * 2;
+  cudaError_t e =
+      make_bf16_tensor_map_3d_sw128(&kmap, a.k, kD, rows, depth, depth_bytes, kBlock);
   if (e == cudaSuccess)
-    e = make_bf16_tensor_map_3d_sw128(&vmap, a.v, kD, uint64_t(a.seq_len), pairs, pair_bytes,
-                                      kBlock);
+    e = make_bf16_tensor_map_3d_sw128(&vmap, a.v, kD, rows, depth, depth_bytes, kBlock);
   if (e == cudaSuccess)
     e = make_bf16_tensor_map_sw128(&qmap, a.q, kD, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;

@@ -169,7 +169,6 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   float* Ws = reinterpret_cast<float*>(smem + S::kW);
   float* V = reinterpret_cast<float*>(smem + S::kVec);
   float* mus = reinterpret_cast<float*>(smem + S::kMu);
-  const uint16_t* kglob = a.k + (item_bh * a.cap + item_j * kBlock) * D;
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);  // TMA
@@ -185,10 +184,27 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
+  // first key row of the block: in the contiguous cache, or its page (the
+  // table may come from the launch before, so it is read after the wait)
+  int64_t row0 = item_bh * a.cap + item_j * kBlock;
+  if (a.block_table != nullptr) {
+    const int64_t bb = item_bh / a.hkv, hh0 = item_bh % a.hkv;
+    const int32_t page = a.block_table[bb * a.table_stride + item_j];
+    if (page < 0 || page >= a.n_pages) {
+      // a negative entry is a block with no page yet: its record is left as
+      // it was; a page past the pool is reported and skipped the same way
+      if (tid == 0 && page >= 0) report(a.status, COBS_ERR_DEVICE);
+      if (warp == 0) tmem_dealloc(tmem, 64);
+      return;
+    }
+    row0 = (int64_t(page) * a.hkv + hh0) * kBlock;
+  }
+  const uint16_t* kglob = a.k + row0 * D;
+
   // ---- 1. TMA load of the block, then the Gram on the tensor cores -----------
   if (tid == 0) {
     mbar_arrive_expect_tx(&bars[0], uint32_t(kBlock) * D * 2);
-    const int y = int(item_bh * a.cap + item_j * kBlock);
+    const int y = int(row0);
     for (int reg = 0; reg < S::kRegions; ++reg)
       tma_load_2d(ktile + reg * S::kRegionBytes, &kmap, reg * 64, y, &bars[0]);
     bool ok = mbar_wait_bounded(&bars[0], 0, a.status);
@@ -655,7 +671,9 @@ template <int D, int M>
 cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
   using S = StatsShape<D>;
   CUtensorMap map;
-  cudaError_t e0 = make_bf16_tensor_map_sw128(&map, a.k, D, uint64_t(a.batch) * a.hkv * a.cap, 64);
+  const uint64_t rows = a.block_table != nullptr ? uint64_t(a.n_pages) * a.hkv * kBlock
+                                                 : uint64_t(a.batch) * a.hkv * a.cap;
+  cudaError_t e0 = make_bf16_tensor_map_sw128(&map, a.k, D, rows, 64);
   if (e0 != cudaSuccess) return e0;
   auto kern = block_stats_kernel<D, M>;
   cudaError_t e =

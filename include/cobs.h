@@ -50,8 +50,9 @@
  *   lse          [batch][num_q_heads]  ln sum exp(logits)         fp32
  *
  * Supported: d in {64, 128}; B = 64; 0 <= r <= 16; G in {1, 2, 4, 8};
- * capacity_tokens a positive multiple of B; one sequence length for the whole
- * batch.
+ * capacity_tokens a positive multiple of B.  One sequence length for the
+ * whole batch, or per-sequence lengths (the _varlen calls); a contiguous
+ * cache, or page pools with a block table (the _paged calls).
  */
 #ifndef COBS_H_
 #define COBS_H_
@@ -204,6 +205,47 @@ COBS_API cobs_status cobs_sparse_decode_varlen(const cobs_dims* dims, const void
                                       int64_t max_seq_len, float softmax_scale,
                                       float* out, float* lse, void* ws,
                                       size_t ws_bytes, void* stream);
+
+/* Paged KV cache (paged KV memory as the glossary page "LLMアテンション機構"
+ * describes it under the KV cache and attention; the COBS method itself keeps
+ * one contiguous cache).  K and V live in page pools of one 64-token block
+ * per page and kv-head, and a block table maps the blocks of every sequence
+ * to pages:
+ *   k_pool, v_pool  device [n_pages][num_kv_heads][B][d] bf16; page p holds
+ *                   block j of sequence b for all kv-heads when
+ *                   block_table[b * table_stride + j] == p.
+ *   n_pages         pages in each pool, n_pages * num_kv_heads * B < 2^31.
+ *   block_table     device [batch][table_stride] int32, 16-byte aligned.
+ *   table_stride    row length of the table; at least the number of blocks
+ *                   addressed (block_end for the statistics,
+ *                   ceil(max_seq_len / B) for the decode), and
+ *                   batch * table_stride < 2^31.
+ * Statistics: as cobs_build_block_stats for blocks [block_begin, block_end)
+ * of every sequence; a negative table entry is a block without a page and
+ * its record is left untouched; an entry >= n_pages is skipped the same way
+ * and reported as COBS_ERR_DEVICE through the status word.
+ * Decode: as cobs_sparse_decode (seq_lens NULL: every sequence is
+ * max_seq_len long) or cobs_sparse_decode_varlen (seq_lens given); every
+ * block a selection names inside its sequence must have a page in
+ * [0, n_pages), else it contributes nothing and COBS_ERR_DEVICE is reported.
+ * Rows of a last page past its sequence's length are never read as keys or
+ * values, whatever they hold.  Results are bit-identical to the contiguous
+ * calls on the same keys and values.  Selection reads only q and the block
+ * records, so cobs_select_blocks(_varlen) serve paged caches unchanged. */
+COBS_API cobs_status cobs_build_block_stats_paged(const cobs_dims* dims,
+                                         const void* k_pool, int64_t n_pages,
+                                         const int32_t* block_table,
+                                         int32_t table_stride, int64_t block_begin,
+                                         int64_t block_end, void* stats, void* ws,
+                                         size_t ws_bytes, void* stream);
+COBS_API cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void* q,
+                                     const void* k_pool, const void* v_pool,
+                                     int64_t n_pages, const int32_t* block_table,
+                                     int32_t table_stride, const int32_t* idx,
+                                     const int32_t* n_sel, int32_t idx_stride,
+                                     const int64_t* seq_lens, int64_t max_seq_len,
+                                     float softmax_scale, float* out, float* lse,
+                                     void* ws, size_t ws_bytes, void* stream);
 
 /* Allocation-free form of cobs_sparse_decode (this library's own addition; the
  * method's description has no counterpart).  Same arguments and results, but

@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) == 13, names
+    assert len(names) == 15, names
     raw = ctypes.CDLL(cb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
@@ -197,3 +197,39 @@ def test_varlen_host_checks():
             with pytest.raises(cb.CobsError) as e:
                 call(lens, mx)
             assert e.value.status == code
+
+
+def test_paged_host_checks():
+    """Block-table arguments are checked before launch: the table itself, its
+    row length against the blocks addressed, the pool size and the index
+    ranges that must fit 32 bits."""
+    A = 1 << 20
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w)
+    ws = cb.cobs_workspace_bytes(d, w.top_k, 1, w.local_tokens)
+    nsm = cb.cobs_selected_capacity(d, w.top_k, 1, w.local_tokens)
+    nb = w.cap // 64
+    stats = lambda tbl, stride, pages, end: cb.cobs_build_block_stats_paged(
+        d, A, pages, tbl, stride, 0, end, A, A, 4096)
+    dec = lambda tbl, stride, pages, mx: cb.cobs_sparse_decode_paged(
+        d, A, A, A, pages, tbl, stride, A, A, nsm, None, mx, 0.1, A, A, A, ws)
+    cases = [
+        (lambda: stats(None, nb, 100, 4), cb.COBS_ERR_INVALID_ARG),
+        (lambda: stats(A + 4, nb, 100, 4), cb.COBS_ERR_INVALID_ARG),
+        (lambda: stats(A, 3, 100, 4), cb.COBS_ERR_INVALID_ARG),        # row shorter than end
+        (lambda: stats(A, nb, 0, 4), cb.COBS_ERR_INVALID_ARG),
+        (lambda: stats(A, nb, 1 << 30, 4), cb.COBS_ERR_UNSUPPORTED),  # pool rows >= 2^31
+        (lambda: cb.cobs_build_block_stats_paged(dims_of(w, batch=2), A, 100, A, 1 << 30, 0,
+                                                 4, A, A, 4096),
+         cb.COBS_ERR_UNSUPPORTED),                                      # batch x stride
+        (lambda: stats(A, nb, 100, nb + 1), cb.COBS_ERR_INVALID_ARG),  # past the capacity
+        (lambda: dec(None, nb, 100, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: dec(A, 63, 100, 4096), cb.COBS_ERR_INVALID_ARG),      # needs 64 blocks
+        (lambda: dec(A, 64, 0, 4096), cb.COBS_ERR_INVALID_ARG),
+        (lambda: dec(A, 64, 1 << 30, 4096), cb.COBS_ERR_UNSUPPORTED),
+        (lambda: dec(A, 64, 100, w.cap + 1), cb.COBS_ERR_INVALID_ARG),
+    ]
+    for fn, code in cases:
+        with pytest.raises(cb.CobsError) as e:
+            fn()
+        assert e.value.status == code, (e.value, code)
