@@ -51,6 +51,13 @@ design notes of the repository):
   complete blocks; ties go to the lower block index.  Output ascending.
 * Attention over the selected blocks is one exact softmax over the union of
   their valid tokens, with the 1/sqrt(d) logit scale.
+* FP4 storage of U (§2.3, quantisation: eigenvectors stored scaled in FP4
+  E2M1, block means in BF16): every U column is cut into groups of 32
+  consecutive components; each group stores E2M1 codes and one power-of-two
+  scale 2^e (an 8-bit biased exponent, as in the E8M0 scales of the OCP
+  microscaling formats), e being the smallest exponent with
+  max |u| <= 6 * 2^e, so that no component saturates; components are rounded
+  to the nearest E2M1 value, ties to the even code.
 """
 
 from __future__ import annotations
@@ -77,6 +84,16 @@ __all__ = [
     "osa_head_masses",
     "osa_group_masses",
     "decode_step",
+    "E2M1_MAGNITUDES",
+    "FP4_GROUP",
+    "e2m1_value",
+    "round_to_e2m1",
+    "fp4_scale_exponent",
+    "quantize_u_fp4",
+    "dequantize_u_fp4",
+    "block_record_fp4",
+    "build_block_records_fp4",
+    "fp4_record_values",
 ]
 
 
@@ -319,3 +336,106 @@ def decode_step(q_group, keys_seq, values_seq, records, seq_len, block, top_k,
     out, lse = sparse_attention(q_group, keys_seq, values_seq, sel, seq_len,
                                 block, scale)
     return sel, scores, out, lse
+
+
+# ---------------------------------------------------------------------------
+# FP4 (E2M1) scaled storage of U (COBS explainer §2.3, quantisation: the
+# eigenvectors are kept in FP4 E2M1 with a scale, the block means in BF16)
+# ---------------------------------------------------------------------------
+
+# magnitudes of the E2M1 codes 0..7 (bit 3 of a code is the sign)
+E2M1_MAGNITUDES = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+FP4_GROUP = 32          # consecutive components of a U column sharing one scale
+
+
+def e2m1_value(codes) -> np.ndarray:
+    """Values of E2M1 codes (4-bit: sign bit 3, magnitude index bits 0-2)."""
+    codes = np.asarray(codes, dtype=np.int64)
+    mag = np.asarray(E2M1_MAGNITUDES)[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def round_to_e2m1(x) -> np.ndarray:
+    """Codes of the E2M1 values nearest to x (ties to the even code).
+
+    Magnitudes above 6 saturate to 6; a value that rounds to zero gets the
+    positive zero code.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 6.0)
+    grid = np.asarray(E2M1_MAGNITUDES)
+    idx = np.arange(len(grid))
+    dist = np.abs(a[..., None] - grid)
+    nearest = dist == dist.min(axis=-1, keepdims=True)   # one code, or two on a tie
+    even = nearest & (idx % 2 == 0)
+    pick = np.where(even.any(axis=-1), np.argmax(even, axis=-1),
+                    np.argmax(nearest, axis=-1))
+    return np.where((x < 0) & (pick != 0), pick | 8, pick).astype(np.uint8)
+
+
+def fp4_scale_exponent(amax: float):
+    """Smallest integer e with amax <= 6 * 2^e, clamped below at -126.
+
+    None for amax == 0 (a group of zeros: scale byte 0, all codes 0).
+    """
+    if amax == 0.0:
+        return None
+    _, ex = math.frexp(amax)          # amax < 2^ex
+    e = ex - 4                        # amax >= 2^(ex-1) > 6 * 2^(ex-4)
+    while amax > 6.0 * 2.0 ** e:
+        e += 1
+    return max(e, -126)
+
+
+def quantize_u_fp4(u_rows: np.ndarray):
+    """E2M1 codes [r, d] and biased scale exponents [r, d/32] of U's columns.
+
+    ``u_rows``: [r, d], row j = column j of U.  Scale byte = e + 127.
+    """
+    u_rows = np.asarray(u_rows, dtype=np.float64)
+    r, d = u_rows.shape
+    codes = np.zeros((r, d), dtype=np.uint8)
+    scale_bytes = np.zeros((r, d // FP4_GROUP), dtype=np.uint8)
+    for j in range(r):
+        for g in range(d // FP4_GROUP):
+            seg = u_rows[j, g * FP4_GROUP:(g + 1) * FP4_GROUP]
+            e = fp4_scale_exponent(float(np.max(np.abs(seg))))
+            if e is None:
+                continue
+            scale_bytes[j, g] = e + 127
+            codes[j, g * FP4_GROUP:(g + 1) * FP4_GROUP] = round_to_e2m1(seg / 2.0 ** e)
+    return codes, scale_bytes
+
+
+def dequantize_u_fp4(codes, scale_bytes) -> np.ndarray:
+    """Component values 2^(byte - 127) * e2m1(code); a zero scale byte is 0."""
+    sb = np.asarray(scale_bytes, dtype=np.int64)
+    scale = np.where(sb == 0, 0.0, np.exp2((sb - 127).astype(np.float64)))
+    return e2m1_value(codes) * np.repeat(scale, FP4_GROUP, axis=-1)
+
+
+def block_record_fp4(keys: np.ndarray, rank: int):
+    """FP4 record of one complete block: (mu in bf16 [d], codes [r, d], scale bytes [r, d/32])."""
+    mu, sigma = block_moments(keys)
+    u, _ = covariance_factor(sigma, rank)
+    codes, scale_bytes = quantize_u_fp4(u.T)
+    return round_to_bf16(mu), codes, scale_bytes
+
+
+def build_block_records_fp4(keys_seq: np.ndarray, block: int, rank: int,
+                            block_begin: int, block_end: int):
+    """FP4 records of complete blocks [block_begin, block_end): stacked (mu, codes, scales)."""
+    d = keys_seq.shape[1]
+    parts = [block_record_fp4(keys_seq[j * block:(j + 1) * block], rank)
+             for j in range(block_begin, block_end)]
+    if not parts:
+        return (np.zeros((0, d)), np.zeros((0, rank, d), np.uint8),
+                np.zeros((0, rank, d // FP4_GROUP), np.uint8))
+    return tuple(np.stack(x, axis=0) for x in zip(*parts))
+
+
+def fp4_record_values(mu, codes, scale_bytes) -> np.ndarray:
+    """The [nb, 1+r, d] records (mu; dequantised U columns) that the score reads."""
+    mu = np.asarray(mu, dtype=np.float64)
+    u = dequantize_u_fp4(codes, scale_bytes)
+    return np.concatenate([mu[:, None, :], u], axis=1)
