@@ -65,6 +65,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true",
                    help="enqueue the timed steps call by call instead of replaying CUDA graphs")
+    p.add_argument("--stats-format", choices=["bf16", "fp4"], default="bf16",
+                   help="block records: mu and U in bf16, or U in scaled FP4 (E2M1)")
     p.add_argument("--stats-stream", choices=["side", "same"], default="side",
                    help="run the completed block's stats build on a forked side stream "
                         "(joined before the step ends) or in line before the selection")
@@ -108,13 +110,14 @@ def max_over_ranks(values, dist, device, world):
     return [float(v) for v in t.tolist()]
 
 
-def byte_model(w, n_sel):
-    """Algorithmic bytes per launch of each kernel for one step."""
+def byte_model(w, n_sel, rec=None):
+    """Algorithmic bytes per launch of each kernel for one step (``rec``: bytes
+    of one block record; bf16 records by default)."""
     B, d, r = w.block, w.head_dim, w.rank
     pairs = w.batch * w.kv_heads
     nbs, nfull, c0, c1 = partition(w.seq_len, B, w.sink_blocks, w.local_tokens)
     q_bytes = w.batch * w.q_heads * d * 2
-    rec = (1 + r) * d * 2
+    rec = (1 + r) * d * 2 if rec is None else rec
     stats_build = pairs * (B * d * 2 + rec)                 # one block in, one record out
     select = pairs * (c1 - c0) * rec + q_bytes + pairs * (c1 - c0) * 4 + pairs * 4 * (1 + n_sel)
     # valid tokens of the selected blocks (all complete here except a ragged tail)
@@ -327,12 +330,15 @@ def run_cobs(args, w, rank, world, local_rank):
 
     dims = dict(batch=w.batch, num_q_heads=w.q_heads, num_kv_heads=w.kv_heads,
                 head_dim=w.head_dim, block_size=w.block, rank=w.rank,
-                capacity_tokens=w.cap)
+                capacity_tokens=w.cap,
+                stats_format=cb.COBS_STATS_FP4 if args.stats_format == "fp4"
+                else cb.COBS_STATS_BF16)
     q, k, v = up(q_bits), up(k_bits), up(v_bits)
     nb_cap = w.cap // w.block
     nfull = w.seq_len // w.block
-    stats = torch.zeros((w.batch, w.kv_heads, nb_cap, 1 + w.rank, w.head_dim),
-                        dtype=torch.int16, device=dev)
+    rec_bytes = cb.cobs_stats_record_bytes(dims)
+    stats = torch.zeros((w.batch, w.kv_heads, nb_cap, rec_bytes), dtype=torch.uint8,
+                        device=dev)
     nsm = cb.cobs_selected_capacity(dims, w.top_k, w.sink_blocks, w.local_tokens)
     idx = torch.zeros((w.batch, w.kv_heads, nsm), dtype=torch.int32, device=dev)
     n_sel = torch.zeros((w.batch, w.kv_heads), dtype=torch.int32, device=dev)
@@ -594,7 +600,8 @@ def run_cobs(args, w, rank, world, local_rank):
         return
 
     hbm, peak_kind = peaks()
-    bm = byte_model(w, round(n_sel_mean))
+    bm = byte_model(w, round(n_sel_mean), rec_bytes)
+    traffic_key = w.name if args.stats_format == "bf16" else f"{w.name}:fp4"
     per_kernel = {"stats": (t_stats, bm["stats"], "stats.cu"),
                   "select": (t_sel, bm["select"], "select.cu"),
                   "decode": (t_dec, bm["decode"],
@@ -625,6 +632,7 @@ def run_cobs(args, w, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "step": "stats of the completed block + select + sparse decode",
                    "stats_stream": args.stats_stream,
+                   "stats_format": args.stats_format, "record_bytes": rec_bytes,
                    "launch": (f"CUDA graphs of {g_steps} steps" if graph_step is not None
                               else "one call at a time")},
         "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
@@ -633,7 +641,7 @@ def run_cobs(args, w, rank, world, local_rank):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",
-                     "traffic": recorded_traffic(file_dom, w.name)},
+                     "traffic": recorded_traffic(file_dom, traffic_key)},
         "gpu_launches": 3 * args.steps,
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,

@@ -11,7 +11,8 @@ from importlib import import_module as _import_module
 
 __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
-    "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
+    "cobs_abi_version", "cobs_stats_record_bytes", "cobs_selected_capacity",
+    "cobs_workspace_bytes", "COBS_STATS_BF16", "COBS_STATS_FP4",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",

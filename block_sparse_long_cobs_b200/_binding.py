@@ -17,7 +17,8 @@ import os
 
 __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
-    "cobs_abi_version", "cobs_selected_capacity", "cobs_workspace_bytes",
+    "cobs_abi_version", "cobs_stats_record_bytes", "cobs_selected_capacity",
+    "cobs_workspace_bytes", "COBS_STATS_BF16", "COBS_STATS_FP4",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
@@ -37,6 +38,9 @@ COBS_ERR_CUDA = 4
 COBS_ERR_TIMEOUT = 5
 COBS_ERR_DEVICE = 6
 
+COBS_STATS_BF16 = 0     # block records: mu and U in bf16
+COBS_STATS_FP4 = 1      # block records: mu in bf16, U in scaled FP4 (E2M1)
+
 
 class CobsError(RuntimeError):
     """A COBS call returned a non-OK status."""
@@ -55,6 +59,7 @@ class cobs_dims(ctypes.Structure):
         ("block_size", ctypes.c_int32),
         ("rank", ctypes.c_int32),
         ("capacity_tokens", ctypes.c_int64),
+        ("stats_format", ctypes.c_int32),       # COBS_STATS_BF16 / COBS_STATS_FP4
     ]
 
 
@@ -69,6 +74,7 @@ def _load() -> ctypes.CDLL:
     D = ctypes.POINTER(cobs_dims)
     sig = {
         "cobs_abi_version": (I32, []),
+        "cobs_stats_record_bytes": (I64, [D]),
         "cobs_selected_capacity": (I32, [D, I32, I32, I32]),
         "cobs_workspace_bytes": (SZ, [D, I32, I32, I32]),
         "cobs_workspace_init": (I32, [P, SZ, P]),
@@ -130,6 +136,14 @@ def _dims(d) -> cobs_dims:
 
 def cobs_abi_version() -> int:
     return lib.cobs_abi_version()
+
+
+def cobs_stats_record_bytes(dims) -> int:
+    """Bytes of one block record for dims' stats_format."""
+    n = lib.cobs_stats_record_bytes(ctypes.byref(_dims(dims)))
+    if n <= 0:
+        raise CobsError("cobs_stats_record_bytes", COBS_ERR_INVALID_ARG, cobs_last_error())
+    return n
 
 
 def cobs_last_error() -> str:

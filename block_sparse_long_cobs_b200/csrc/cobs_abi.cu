@@ -60,6 +60,11 @@ cobs_status check_dims(const cobs_dims* d) {
   const int64_t rows = int64_t(d->batch) * d->num_kv_heads * d->capacity_tokens;
   if (rows >= (int64_t(1) << 31))
     return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * capacity_tokens must be < 2^31");
+  if (d->stats_format != COBS_STATS_BF16 && d->stats_format != COBS_STATS_FP4)
+    return fail(COBS_ERR_INVALID_ARG, "stats_format must be COBS_STATS_BF16 or COBS_STATS_FP4 (got %d)",
+                d->stats_format);
+  if (d->stats_format == COBS_STATS_FP4 && d->rank < 1)
+    return fail(COBS_ERR_UNSUPPORTED, "FP4 records need rank >= 1");
   return COBS_OK;
 }
 
@@ -295,6 +300,8 @@ static cobs_status stats_impl(const cobs_dims* dims, const void* k, const int32_
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.rank = dims->rank;
+  a.stats_format = dims->stats_format;
+  a.rec_bytes = stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
   a.block_table = block_table;
   a.table_stride = table_stride;
   a.n_pages = n_pages;
@@ -306,6 +313,12 @@ static cobs_status stats_impl(const cobs_dims* dims, const void* k, const int32_
 extern "C" {
 
 int32_t cobs_abi_version(void) { return COBS_ABI_VERSION; }
+
+int64_t cobs_stats_record_bytes(const cobs_dims* dims) {
+  if (check_dims(dims) != COBS_OK) return 0;
+  ok();
+  return stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
+}
 
 const char* cobs_last_error(void) { return g_last_error.c_str(); }
 
@@ -416,6 +429,8 @@ static cobs_status select_impl(const cobs_dims* dims, const void* q, const void*
   a.hkv = dims->num_kv_heads;
   a.d = dims->head_dim;
   a.rank = dims->rank;
+  a.stats_format = dims->stats_format;
+  a.rec_bytes = stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
   a.idx_stride = idx_stride;
   a.seq_len_blocks = int32_t(nbs);
   a.cand_begin = int32_t(sink_end);
@@ -430,14 +445,14 @@ static cobs_status select_impl(const cobs_dims* dims, const void* q, const void*
 
   // chunking: one wave of resident CTAs shared out over the (batch, kv-head)
   // pairs; every chunk is a whole number of stages (128 record rows each)
-  const int per_pass = select_blocks_per_stage(dims->rank);
+  const int per_pass = select_blocks_per_stage(dims->head_dim, dims->rank, dims->stats_format);
   const int64_t n_cand = first_local - sink_end;
   const int64_t pairs = int64_t(dims->batch) * dims->num_kv_heads;
   int sms = device_sm_count();
   if (sms <= 0) sms = 148;
   const int resident =
       sms * select_ctas_per_sm(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
-                               dims->rank);
+                               dims->rank, dims->stats_format);
   int64_t chunks = resident / pairs;
   const int64_t max_chunks = n_cand > 0 ? ceil_div(n_cand, per_pass) : 1;
   if (chunks > max_chunks) chunks = max_chunks;

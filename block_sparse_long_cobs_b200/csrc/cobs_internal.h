@@ -38,6 +38,8 @@ struct SelectArgs {
   int32_t* status;
   int64_t nb_cap;
   int32_t batch, hq, hkv, d, rank;
+  int32_t stats_format;     // 0 bf16 records, 1 FP4 U
+  int64_t rec_bytes;        // bytes per block record
   int32_t idx_stride;
   int32_t seq_len_blocks;   // ceil(seq_len / B)
   int32_t cand_begin, cand_end;  // candidate blocks [begin, end)
@@ -53,6 +55,32 @@ struct SelectArgs {
   int64_t max_seq_len;
   int32_t sink_blocks, local_tokens;
 };
+
+// Bytes of one block record: bf16 [1 + r][d], or the FP4 layout (mu bf16,
+// r x d/2 bytes of E2M1 codes, r x d/32 scale exponents, padded to 16).
+__host__ __device__ inline int64_t stats_record_bytes(int d, int r, int fmt) {
+  if (fmt == 0) return int64_t(1 + r) * d * 2;
+  const int64_t raw = int64_t(2) * d + int64_t(r) * (d / 2) + int64_t(r) * (d / 32);
+  return (raw + 15) & ~int64_t(15);
+}
+
+// Selection kernel over FP4 records: per pass, the mu rows of its blocks fill
+// whole 8-row swizzle atoms at the top of a 128-row operand tile and the
+// r U rows of each block follow; the raw records of a pass fit one staging
+// slot of the record ring.  Host and device use the same rule.
+constexpr int kSelFp4RawStages = 5;
+__host__ __device__ inline int fp4_ring_bytes(int d) { return 3 * (d / 64) * 128 * 128; }
+__host__ __device__ inline int fp4_raw_stage_bytes(int d) {
+  return ((fp4_ring_bytes(d) - (d / 64) * 128 * 128) / kSelFp4RawStages) & ~15;
+}
+__host__ __device__ inline int fp4_blocks_per_pass(int d, int r) {
+  const int64_t rec = stats_record_bytes(d, r, 1);
+  int p = 0;
+  while (p < 128 && ((p + 1 + 7) / 8) * 8 + (p + 1) * r <= 128 &&
+         (p + 1) * rec <= fp4_raw_stage_bytes(d))
+    ++p;
+  return p;
+}
 
 // Block partition of one sequence of `len` tokens (COBS explainer §2.1 and
 // the sliding-window glossary: sink blocks, local window, candidates between):
@@ -115,12 +143,14 @@ struct DecodePlan {
 // Arguments of the block-statistics kernel.
 struct StatsArgs {
   const uint16_t* k;      // [b][Hkv][cap][d], or the page pool [n_pages][Hkv][B][d]
-  uint16_t* stats;        // [b][Hkv][nb_cap][1+r][d]
+  uint16_t* stats;        // [b][Hkv][nb_cap] records of rec_bytes
   int32_t* status;
   int64_t cap;
   int64_t nb_cap;
   int64_t block_begin, block_end;
   int32_t batch, hkv, d, rank;
+  int32_t stats_format;   // 0: bf16 [1+r][d] records; 1: mu bf16 + FP4 U
+  int64_t rec_bytes;      // bytes per block record
   // paged cache: block j of sequence b is page block_table[b * table_stride + j]
   const int32_t* block_table;   // null: contiguous cache
   int32_t table_stride;
@@ -128,8 +158,8 @@ struct StatsArgs {
 };
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
-int select_ctas_per_sm(int d, int g, int rank);  // resident selection CTAs per SM
-int select_blocks_per_stage(int rank);           // whole records per selection stage
+int select_ctas_per_sm(int d, int g, int rank, int fmt);  // resident selection CTAs per SM
+int select_blocks_per_stage(int d, int rank, int fmt);    // whole records per selection pass
 // Whether the exact top-k of `n_cand` candidates fits the selection kernel's
 // shared memory (its survivors can grow with top_k x n_cand / 1024).
 bool select_topk_fits(int d, int64_t n_cand, int top_k);

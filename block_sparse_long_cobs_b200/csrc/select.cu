@@ -34,6 +34,8 @@
 // between the sink blocks and the local blocks.
 #include <cfloat>
 
+#include <cuda_fp16.h>
+
 #include "device_common.cuh"
 #include "tcgen05.cuh"
 
@@ -74,7 +76,37 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 
 
-template <int D, int G>
+// Eight E2M1 codes (two per byte, the even component in the low nibble) as
+// eight fp16 values, lowest component first.  Every E2M1 value is exact in
+// fp16.
+__device__ __forceinline__ uint4 e2m1x8_to_f16x8(uint32_t w) {
+  uint4 h;
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
+      : "=r"(h.x), "=r"(h.y), "=r"(h.z), "=r"(h.w)
+      : "r"(w));
+  return h;
+}
+
+// Lane-wise fp16 product (round to nearest; fp16 subnormals are kept).
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Two bf16 values as two fp16 values (round to nearest).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+  const float2 f = bf16x2_to_float2(w);
+  const __half2 h = __floats2half2_rn(f.x, f.y);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int D, int G, bool kFp4>
 __global__ void __launch_bounds__(kSelThreads)
 select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap qmap, const SelectArgs a) {
@@ -101,7 +133,10 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   uint8_t* qtile = base;                            // [kRegions][16][128 B]
-  uint8_t* stage = base + kQBytes;                  // [kSelStages][kRegions][128][128 B]
+  // bf16 records: [kSelStages][kRegions][128][128 B] record ring; FP4 records:
+  // an fp16 copy of the queries, then the same number of bytes holding one
+  // operand tile and the raw record ring.  Phase 2 reuses the ring either way.
+  uint8_t* stage = base + (kFp4 ? 2 : 1) * kQBytes;
 
   float* scores = a.scores_ws + int64_t(bh) * a.nb_cap;
   // this sequence's block partition
@@ -110,7 +145,256 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   const BlockPartition BP = block_partition(seq_len_b, a.sink_blocks, a.local_tokens);
 
   // ===================== phase 1: scores of this chunk =====================
-  {
+  if constexpr (kFp4) {
+    // FP4 records (COBS explainer §2.3, quantisation): mu bf16 [D] | E2M1
+    // codes [r][D/2] | scale exponents [r][D/32] | padding.  A pass stages the
+    // raw records of per_pass consecutive blocks with one bulk copy, then
+    // every thread widens one row of a 128-row operand tile: the mu rows
+    // (bf16) at rows [0, per_pass), the U rows from row mu_rows =
+    // 8 ceil(per_pass / 8) as fp16 values code x 2^(e_g - E), E the largest
+    // group exponent of that column -- exact in fp16 for e_g - E >= -23 (a
+    // group further below contributes nothing: its components are under
+    // 2^-23 of the column's largest).  Both products read the whole tile from
+    // row 0 -- the bf16 one against the bf16 queries, the fp16 one against an
+    // fp16 copy of them -- and each keeps only its own rows' accumulator
+    // lanes; the epilogue scales a U row's product by 2^E.  Accumulators are
+    // double-buffered: the products of pass p run under the epilogue of
+    // pass p - 1.
+    constexpr int kRaw = kSelFp4RawStages;
+    constexpr int kGroups = D / 32;
+    const int r = a.rank;
+    const int rec = int(a.rec_bytes);
+    const int per_pass = fp4_blocks_per_pass(D, r);
+    const int mu_rows = (per_pass + 7) & ~7;
+    const int raw_bytes = fp4_raw_stage_bytes(D);
+    uint8_t* qtile16 = base + kQBytes;
+    uint8_t* atile = stage;                          // [kRegions][128][128 B]
+    uint8_t* raw = stage + kStageBytes;              // [kRaw][raw_bytes]
+    __shared__ __align__(8) uint64_t raw_full[kRaw];
+    __shared__ uint32_t colexp_s[2][kStageRows];     // E of each U row, per buffer
+    // this thread's row of the tile: U row (block, column) or mu row (block)
+    const int my_blk = tid / r, my_col = tid - (tid / r) * r;
+
+    const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
+    const int c_lo = max(int(BP.sink_end), c_nom);
+    const int c_hi = min(int(BP.first_local), min(a.cand_end, c_nom + a.chunk_blocks));
+    const int npass = c_hi > c_lo ? (c_hi - c_lo + per_pass - 1) / per_pass : 0;
+    const uint8_t* recs =
+        reinterpret_cast<const uint8_t*>(a.stats) + int64_t(bh) * a.nb_cap * a.rec_bytes;
+
+    if (tid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
+      for (int s2 = 0; s2 < kRaw; ++s2) mbar_init(&raw_full[s2], 1);
+      mbar_init(&mma_done[0], 1);
+      mbar_init(&mma_done[1], 1);
+      fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_slot, 64);
+    pdl_wait();              // queries and records may come from the launch before
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();
+    const uint32_t tmem = tmem_slot;   // buffer b: mu products at 32 b, U at 32 b + 16
+
+    int n_issued = 0;          // thread 0: passes whose copies were issued
+    int n_mma = 0;             // thread 0: passes whose products were issued
+    auto issue = [&](int p) {  // thread 0 only: raw records of pass p (+ queries)
+      n_issued = p + 1;
+      const int j0 = c_lo + p * per_pass;
+      const int nb = min(per_pass, c_hi - j0);
+      const uint32_t bytes = uint32_t(nb) * uint32_t(rec);
+      uint64_t* bar = &raw_full[p % kRaw];
+      mbar_arrive_expect_tx(bar, bytes + (p == 0 ? uint32_t(kRegions) * 8 * 128 : 0u));
+      if (p == 0)
+        for (int reg = 0; reg < kRegions; ++reg)
+          tma_load_2d(qtile + reg * 16 * 128, &qmap, reg * 64, b * a.hq + kvh * G, bar);
+      bulk_g2s(raw + (p % kRaw) * raw_bytes, recs + int64_t(j0) * rec, bytes, bar);
+    };
+    if (tid == 0) {
+      for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
+    }
+
+    const float inv_sqrt_d = rsqrtf(float(D));
+    const float ln_n = logf(float(kBlock));
+    constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
+    constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
+
+    // scores of pass pe from accumulator buffer pe & 1 (its products are complete)
+    auto epilogue = [&](int pe) {
+      const int j0 = c_lo + pe * per_pass;
+      const int nb = min(per_pass, c_hi - j0);
+      const int row = warp * 32 + lane;
+      const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 32u * uint32_t(pe & 1);
+      uint32_t vm[8], vu[8];
+      tmem_ld8_nowait(lane_base, vm);
+      tmem_ld8_nowait(lane_base + 16u, vu);
+      tmem_wait_ld();
+      const bool is_mu = row < mu_rows;
+      const uint32_t eb = colexp_s[pe & 1][row];
+      const float col_scale = __uint_as_float(eb << 23);   // 2^(E - 127); 0 for E = 0
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float c;
+        if (is_mu) {
+          c = __uint_as_float(vm[h]) * inv_sqrt_d;
+        } else {
+          const float x = __uint_as_float(vu[h]) * col_scale * inv_sqrt_d;
+          c = 0.5f * x * x;
+        }
+        contrib[row * 8 + h] = c;
+      }
+      tc_fence_before();
+      __syncthreads();
+      // per block and head: mu row + its r U rows, then LSE over the heads
+      for (int t0 = 0; t0 < per_pass * G; t0 += kSelThreads) {
+        const int t = t0 + tid;
+        const int jj = t / G, h = t % G;
+        const bool valid = jj < nb;
+        float sacc = 0.f;
+        if (valid) {
+          sacc = contrib[jj * 8 + h];
+          for (int i = 0; i < r; ++i) sacc += contrib[(mu_rows + jj * r + i) * 8 + h];
+        }
+        const float sh = sacc + ln_n;
+        float mx = sh;
+#pragma unroll
+        for (int m = G / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m, G));
+        float e = __expf(sh - mx);
+#pragma unroll
+        for (int m = G / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m, G);
+        if (valid && h == 0) {
+          const float S = mx + __logf(e);
+          scores[j0 + jj] = S;
+          if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
+        }
+      }
+      __syncthreads();   // contrib reused by the next epilogue
+    };
+
+    bool fail = false;
+    for (int p = 0; p < npass; ++p) {
+      const int st = p % kRaw;
+      const uint32_t parity = (p / kRaw) & 1;
+      // the tile is free once the products of pass p - 1 are complete
+      if (tid == 0 && p >= 1 &&
+          !mbar_wait_bounded(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1, a.status))
+        fail = true;
+      if (tid == 0 && !fail && !mbar_wait_bounded(&raw_full[st], parity, a.status)) fail = true;
+      if (__syncthreads_or(fail)) break;
+      if (tid != 0) {
+        (void)mbar_try_wait(&raw_full[st], parity);
+        if (p >= 1) (void)mbar_try_wait(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1);
+      }
+      tc_fence_after();
+      const int j0 = c_lo + p * per_pass;
+      const int nb = min(per_pass, c_hi - j0);
+      const uint8_t* rs = raw + st * raw_bytes;
+      if (p == 0) {
+        // the group's 8 query rows as fp16, at the same byte positions
+        for (int c = tid; c < kRegions * 64; c += kSelThreads) {
+          const int off = (c >> 6) * 16 * 128 + (c & 63) * 16;
+          const uint4 w = *reinterpret_cast<const uint4*>(qtile + off);
+          uint4 h;
+          h.x = bf16x2_to_f16x2(w.x);
+          h.y = bf16x2_to_f16x2(w.y);
+          h.z = bf16x2_to_f16x2(w.z);
+          h.w = bf16x2_to_f16x2(w.w);
+          *reinterpret_cast<uint4*>(qtile16 + off) = h;
+        }
+      }
+      // widen this thread's row of the pass into the tile (128-byte swizzle)
+      if (tid < nb * r) {
+        const uint8_t* rp = rs + my_blk * rec;
+        const int row = mu_rows + tid;
+        const uint8_t* sp = rp + 2 * D + r * (D / 2) + my_col * kGroups;
+        const uint32_t sw = kGroups == 4 ? *reinterpret_cast<const uint32_t*>(sp)
+                                         : uint32_t(*reinterpret_cast<const uint16_t*>(sp));
+        uint32_t emax = 0;
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) emax = max(emax, (sw >> (8 * g)) & 0xFFu);
+        colexp_s[p & 1][row] = emax;
+#pragma unroll
+        for (int gg = 0; gg < kGroups; ++gg) {
+          const int g = (gg + my_col) & (kGroups - 1);   // staggered: fewer bank conflicts
+          const uint32_t eg = (sw >> (8 * g)) & 0xFFu;
+          // fp16 2^(eg - emax): normal for k >= -14, subnormal below; code x 2^k
+          // (a multiple of 2^(k-1)) is an fp16 value for k >= -23, else 0 is used
+          const int k = eg ? int(eg) - int(emax) : -100;
+          const uint32_t mbits = k >= -14 ? uint32_t(k + 15) << 10
+                                          : (k >= -23 ? (1u << (k + 24)) : 0u);
+          const uint32_t mult = mbits | (mbits << 16);
+          const uint4 c4 = *reinterpret_cast<const uint4*>(rp + 2 * D + my_col * (D / 2) + g * 16);
+          const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            uint4 hv = e2m1x8_to_f16x8(cw[t]);
+            hv.x = f16x2_mul(hv.x, mult);
+            hv.y = f16x2_mul(hv.y, mult);
+            hv.z = f16x2_mul(hv.z, mult);
+            hv.w = f16x2_mul(hv.w, mult);
+            const int u = 4 * g + t;               // 16-byte unit of the fp16 row
+            *reinterpret_cast<uint4*>(atile + (u >> 3) * (128 * 128) + row * 128 +
+                                      (((u & 7) ^ (row & 7)) << 4)) = hv;
+          }
+        }
+      } else if (tid < nb * r + nb) {
+        const int blk = tid - nb * r;
+        const uint8_t* rp = rs + blk * rec;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(rp + c * 16);
+          *reinterpret_cast<uint4*>(atile + (c >> 3) * (128 * 128) + blk * 128 +
+                                    (((c & 7) ^ (blk & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();   // generic-proxy tile writes -> tensor-core reads
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t abase = smem_addr(atile);
+        const uint32_t qb = smem_addr(qtile), qh = smem_addr(qtile16);
+        const uint32_t acc = tmem + 32u * uint32_t(p & 1);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+          umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+          const uint64_t bd = umma_desc_sw128(qh + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+          umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&mma_done[p & 1]);
+        n_mma = p + 1;
+        // the raw slot of pass p is free again (its bytes are in the tile)
+        if (p + kRaw < npass) issue(p + kRaw);
+      }
+      if (p >= 1) epilogue(p - 1);
+    }
+    if (!fail && npass > 0) {
+      const int pl = npass - 1;
+      if (tid == 0 && !mbar_wait_bounded(&mma_done[pl & 1], (pl >> 1) & 1, a.status)) fail = true;
+      if (!__syncthreads_or(fail)) {
+        if (tid != 0) (void)mbar_try_wait(&mma_done[pl & 1], (pl >> 1) & 1);
+        tc_fence_after();
+        epilogue(pl);
+      }
+    }
+    if (tid == 0 && fail) {
+      // let the copies and the products still in flight land before TMEM is
+      // freed and the CTA leaves (each wait bounded)
+      for (int p = n_issued > kRaw ? n_issued - kRaw : 0; p < n_issued; ++p)
+        (void)mbar_wait_bounded(&raw_full[p % kRaw], (p / kRaw) & 1, a.status);
+      for (int p = n_mma > 2 ? n_mma - 2 : 0; p < n_mma; ++p)
+        (void)mbar_wait_bounded(&mma_done[p & 1], (p >> 1) & 1, a.status);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+  } else {
     // this chunk's share of the candidates of a max_seq_len sequence, cut to
     // this sequence's own candidates [sink_end, first_local)
     const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
@@ -418,65 +702,74 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   }
 }
 
-template <int D>
+template <int D, bool kFp4>
 constexpr size_t dyn_smem_bytes() {
-  return 1024 + size_t(D / 64) * 16 * 128 + size_t(kSelStages) * (D / 64) * 128 * 128;
+  return 1024 + size_t(kFp4 ? 2 : 1) * (D / 64) * 16 * 128 +
+         size_t(kSelStages) * (D / 64) * 128 * 128;
 }
 
-template <int D, int G>
+template <int D, int G, bool kFp4>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
-  auto kern = select_blocks_kernel<D, G>;
-  constexpr size_t smem = dyn_smem_bytes<D>();
+  auto kern = select_blocks_kernel<D, G, kFp4>;
+  constexpr size_t smem = dyn_smem_bytes<D, kFp4>();
   cudaError_t e = set_smem_attrs(kern, int(smem));
   if (e != cudaSuccess) return e;
-  CUtensorMap map;
-  const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
-  e = make_bf16_tensor_map_sw128(&map, a.stats, D, total_rows, kStageRows);
-  CUtensorMap qmap;
-  if (e == cudaSuccess)
-    e = make_bf16_tensor_map_sw128(&qmap, a.q, D, uint64_t(a.batch) * a.hq, 8);
+  CUtensorMap map, qmap;
+  e = make_bf16_tensor_map_sw128(&qmap, a.q, D, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;
+  if (kFp4) {
+    map = qmap;   // FP4 records arrive by plain bulk copies; the map is unused
+  } else {
+    const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
+    e = make_bf16_tensor_map_sw128(&map, a.stats, D, total_rows, kStageRows);
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid(a.n_chunks, a.hkv, a.batch);
   return launch_pdl(kern, grid, dim3(kSelThreads), smem, s, map, qmap, a);
 }
 
-template <int D, int G>
+template <int D, int G, bool kFp4>
 int occupancy_t() {
-  return kernel_occupancy(reinterpret_cast<const void*>(select_blocks_kernel<D, G>),
-                          kSelThreads, int(dyn_smem_bytes<D>()));
+  return kernel_occupancy(reinterpret_cast<const void*>(select_blocks_kernel<D, G, kFp4>),
+                          kSelThreads, int(dyn_smem_bytes<D, kFp4>()));
 }
 
-template <int D>
+template <int D, bool kFp4>
 cudaError_t dispatch_group(const SelectArgs& a, cudaStream_t s) {
   switch (a.hq / a.hkv) {
-    case 1: return launch_t<D, 1>(a, s);
-    case 2: return launch_t<D, 2>(a, s);
-    case 4: return launch_t<D, 4>(a, s);
-    case 8: return launch_t<D, 8>(a, s);
+    case 1: return launch_t<D, 1, kFp4>(a, s);
+    case 2: return launch_t<D, 2, kFp4>(a, s);
+    case 4: return launch_t<D, 4, kFp4>(a, s);
+    case 8: return launch_t<D, 8, kFp4>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D>
+template <int D, bool kFp4>
 int occupancy_group(int g) {
   switch (g) {
-    case 1: return occupancy_t<D, 1>();
-    case 2: return occupancy_t<D, 2>();
-    case 4: return occupancy_t<D, 4>();
-    default: return occupancy_t<D, 8>();
+    case 1: return occupancy_t<D, 1, kFp4>();
+    case 2: return occupancy_t<D, 2, kFp4>();
+    case 4: return occupancy_t<D, 4, kFp4>();
+    default: return occupancy_t<D, 8, kFp4>();
   }
 }
 
 }  // namespace
 
-int select_ctas_per_sm(int d, int g, int /*rank*/) {
-  return d == 64 ? occupancy_group<64>(g) : occupancy_group<128>(g);
+int select_ctas_per_sm(int d, int g, int /*rank*/, int fmt) {
+  if (fmt != 0) return d == 64 ? occupancy_group<64, true>(g) : occupancy_group<128, true>(g);
+  return d == 64 ? occupancy_group<64, false>(g) : occupancy_group<128, false>(g);
 }
 
-int select_blocks_per_stage(int rank) { return kStageRows / (1 + rank); }
+int select_blocks_per_stage(int d, int rank, int fmt) {
+  return fmt != 0 ? fp4_blocks_per_pass(d, rank) : kStageRows / (1 + rank);
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
-  return a.d == 64 ? dispatch_group<64>(a, stream) : dispatch_group<128>(a, stream);
+  if (a.stats_format != 0)
+    return a.d == 64 ? dispatch_group<64, true>(a, stream) : dispatch_group<128, true>(a, stream);
+  return a.d == 64 ? dispatch_group<64, false>(a, stream) : dispatch_group<128, false>(a, stream);
 }
 
 bool select_topk_fits(int d, int64_t n_cand, int top_k) {

@@ -136,6 +136,36 @@ __device__ __forceinline__ uint32_t k_offset(int row, int col) {
                   ((((c >> 3) ^ (row & 7))) << 4) + ((c & 7) << 1));
 }
 
+// ---- FP4 (E2M1) scaled storage of U (COBS explainer §2.3, quantisation) ----
+// A group of 32 components shares the scale 2^e with e the smallest exponent
+// such that max |u| <= 6 * 2^e (at least -126), stored as e + 127; 0 marks a
+// group of zeros.  From amax = (1 + f) 2^e0 (normal): amax / 2^(e0-2) =
+// 4 (1 + f) is at most 6 exactly when f <= 1/2, else e0 - 1 is needed.
+__device__ __forceinline__ int fp4_scale_exp(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int ef = int((bits >> 23) & 0xFFu);
+  if (ef == 0) return -126;                       // amax below 2^-126
+  const int e0 = ef - 127;
+  const int e = (bits & 0x7FFFFFu) <= 0x400000u ? e0 - 2 : e0 - 1;
+  return e < -126 ? -126 : e;
+}
+__device__ __forceinline__ uint32_t fp4_scale_byte(float amax) {
+  return amax == 0.f ? 0u : uint32_t(fp4_scale_exp(amax) + 127);
+}
+// E2M1 code of v / 2^e: the nearest of 0, .5, 1, 1.5, 2, 3, 4, 6 (ties to
+// the even code: the thresholds at the midpoints include or exclude the
+// midpoint accordingly), sign in bit 3, zero always positive.
+__device__ __forceinline__ uint32_t fp4_code_scaled(float v, float amax) {
+  if (amax == 0.f) return 0u;
+  const int e = fp4_scale_exp(amax);
+  const float x = v * __uint_as_float(uint32_t(127 - e) << 23);   // v / 2^e, exact
+  const float m = fabsf(x);
+  const uint32_t mag = uint32_t(m > 0.25f) + uint32_t(m >= 0.75f) + uint32_t(m > 1.25f) +
+                       uint32_t(m >= 1.75f) + uint32_t(m > 2.5f) + uint32_t(m >= 3.5f) +
+                       uint32_t(m > 5.0f);
+  return (x < 0.f && mag != 0u) ? (mag | 8u) : mag;
+}
+
 template <int D, int M>
 __global__ void __launch_bounds__(kStatThreads)
 block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) {
@@ -654,16 +684,46 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       }
     }
   }
+  uint8_t* rec8 = reinterpret_cast<uint8_t*>(a.stats) +
+                  ((item_bh * a.nb_cap) + item_j) * a.rec_bytes;
   if (bt < D) {
-    uint16_t* rec = a.stats + ((item_bh * a.nb_cap) + item_j) * int64_t(1 + r) * D;
+    uint16_t* rec = reinterpret_cast<uint16_t*>(rec8);
     rec[bt] = float_to_bf16_bits(mu_d);
+    if (a.stats_format == 0) {
 #pragma unroll
-    for (int k = 0; k < kMaxRank; ++k) {
-      if (k < r) {
-        const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
-        rec[int64_t(1 + k) * D + bt] = float_to_bf16_bits(sg * uacc[k]);
+      for (int k = 0; k < kMaxRank; ++k) {
+        if (k < r) {
+          const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
+          rec[int64_t(1 + k) * D + bt] = float_to_bf16_bits(sg * uacc[k]);
+        }
+      }
+    } else {
+      // FP4: warp w holds components [32w, 32w + 32) of every column, one
+      // scale group (D is a multiple of 32, so whole warps take this branch)
+      uint8_t* codes = rec8 + 2 * D;
+      uint8_t* scales = codes + r * (D / 2);
+#pragma unroll
+      for (int k = 0; k < kMaxRank; ++k) {
+        if (k < r) {
+          const float v = ((neg_mask >> k) & 1u) ? -uacc[k] : uacc[k];
+          const float amax = warp_max(fabsf(v));
+          const uint32_t code = fp4_code_scaled(v, amax);
+          // eight neighbouring lanes OR their nibbles into one 32-bit word
+          uint32_t word = code << (4 * (lane & 7));
+          word |= __shfl_xor_sync(0xffffffffu, word, 1);
+          word |= __shfl_xor_sync(0xffffffffu, word, 2);
+          word |= __shfl_xor_sync(0xffffffffu, word, 4);
+          if ((lane & 7) == 0)
+            *reinterpret_cast<uint32_t*>(codes + k * (D / 2) + bt / 2) = word;
+          if (lane == 0) scales[k * (D / 32) + bwarp] = uint8_t(fp4_scale_byte(amax));
+        }
       }
     }
+  }
+  // FP4 records end in zero padding up to a multiple of 16 bytes
+  if (a.stats_format != 0) {
+    const int used = 2 * D + r * (D / 2) + r * (D / 32);
+    if (used + bt < a.rec_bytes) rec8[used + bt] = 0;
   }
 }
 

@@ -84,6 +84,11 @@ constexpr uint32_t umma_idesc_bf16(int M, int N) {
          (uint32_t(M >> 4) << 24);
 }
 
+// Same for fp16 A and B (format fields 0).
+constexpr uint32_t umma_idesc_f16(int M, int N) {
+  return (1u << 4) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
 // Same with A MN-major (bit 15).
 constexpr uint32_t umma_idesc_bf16_amn(int M, int N) { return umma_idesc_bf16(M, N) | (1u << 15); }
 

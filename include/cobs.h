@@ -42,8 +42,10 @@
  *   K, V cache   [batch][num_kv_heads][capacity_tokens][d]        bf16
  *   q            [batch][num_q_heads][d]                          bf16
  *                (query head hq belongs to kv-head hq / G)
- *   stats        [batch][num_kv_heads][capacity_tokens / B][1 + r][d] bf16
- *                (row 0 = mu, rows 1..r = columns of U, eigenvalues descending)
+ *   stats        [batch][num_kv_heads][capacity_tokens / B] records; a
+ *                COBS_STATS_BF16 record is [1 + r][d] bf16 (row 0 = mu,
+ *                rows 1..r = columns of U, eigenvalues descending); the
+ *                COBS_STATS_FP4 record is described at cobs_dims
  *   idx          [batch][num_kv_heads][idx_stride]                int32
  *   n_sel        [batch][num_kv_heads]                            int32
  *   out          [batch][num_q_heads][d]                          fp32
@@ -64,7 +66,7 @@
 extern "C" {
 #endif
 
-#define COBS_ABI_VERSION 1
+#define COBS_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define COBS_API __attribute__((visibility("default")))
@@ -82,6 +84,10 @@ typedef enum cobs_status {
   COBS_ERR_DEVICE = 6        /* device: a kernel rejected its input        */
 } cobs_status;
 
+/* Storage of a block record (cobs_dims.stats_format). */
+#define COBS_STATS_BF16 0    /* mu and U in bf16: (1 + r) x d x 2 bytes      */
+#define COBS_STATS_FP4 1     /* mu in bf16, U in scaled FP4 E2M1 (below)     */
+
 typedef struct cobs_dims {
   int32_t batch;             /* sequences in the batch                      */
   int32_t num_q_heads;       /* query heads Hq                              */
@@ -90,10 +96,37 @@ typedef struct cobs_dims {
   int32_t block_size;        /* B (64)                                      */
   int32_t rank;              /* r, columns of the covariance factor U       */
   int64_t capacity_tokens;   /* cache length per (batch, kv-head)           */
+  int32_t stats_format;      /* COBS_STATS_BF16 (0) or COBS_STATS_FP4 (1)    */
 } cobs_dims;
+
+/* FP4 block record (COBS explainer §2.3, quantisation: eigenvectors stored
+ * scaled in FP4 E2M1, block means in BF16), cobs_stats_record_bytes() bytes:
+ *   [0, 2d)                 mu, d bf16 values
+ *   [2d, 2d + r d/2)        U codes: column j of U is row j of d/2 bytes;
+ *                           component t sits in byte t/2, the low nibble
+ *                           for even t; a code is E2M1 (bit 3 sign, bits 0-2
+ *                           magnitude index into 0, .5, 1, 1.5, 2, 3, 4, 6)
+ *   [.., + r d/32)          scales: byte g of row j scales components
+ *                           [32g, 32g + 32) of column j by 2^(byte - 127);
+ *                           byte 0 marks a group of zeros
+ *   then zero padding to a multiple of 16 bytes.
+ * A group's exponent is the smallest e with max |u| <= 6 * 2^e (clamped at
+ * -126), so no component saturates; components round to the nearest E2M1
+ * value, ties to the even code.  FP4 records need r >= 1.  Selection over
+ * FP4 records multiplies the codes with the queries in fp16: queries must lie
+ * inside the fp16 range (|q| < 65504), and components below 2^-14 are
+ * rounded to fp16's subnormal grid (an error of at most 2^-25 each); a scale
+ * group whose exponent lies more than 23 below the largest of its column
+ * (components under 2^-23 of the column's largest) counts as zero there. */
 
 /* Version of this ABI (COBS_ABI_VERSION). */
 COBS_API int32_t cobs_abi_version(void);
+
+/* Bytes of one block record in `stats` for dims->stats_format:
+ * (1 + r) d 2 for COBS_STATS_BF16, the FP4 layout above for COBS_STATS_FP4.
+ * The stats array is [batch][num_kv_heads][capacity_tokens / B] records.
+ * Returns 0 (and sets the last error) for invalid dims. */
+COBS_API int64_t cobs_stats_record_bytes(const cobs_dims* dims);
 
 /* Length of one row of `idx`: the largest number of blocks a selection can
  * return, min(ceil(capacity/B), top_k + sink_blocks + ceil(local_tokens/B) + 1).
@@ -118,7 +151,8 @@ COBS_API cobs_status cobs_workspace_init(void* ws, size_t ws_bytes, void* stream
 /* Block statistics for the complete blocks [block_begin, block_end) of every
  * (batch, kv-head): mu = mean key; Sigma = (1/B) sum (k - mu)(k - mu)^T;
  * U = top-r eigenvectors of Sigma scaled by sqrt(eigenvalue), each column's
- * largest-magnitude component made positive.  Written to `stats` in bf16.
+ * largest-magnitude component made positive.  Written to `stats` in the
+ * record format dims->stats_format names (bf16, or FP4 U).
  * COBS explainer §2.2 (kappa1, kappa2) and §2.3 (low-rank factorisation).
  * Call it when blocks become complete (e.g. after appending a chunk).
  *   k      device, K cache (see shapes); only the named blocks are read.

@@ -184,3 +184,71 @@ def stats_errors(gpu_rec, orc_rec, orc_keys_block, rank):
     tr_o = float(np.trace(po))
     energy = float(np.trace(pg) / tr_o) if tr_o > 0 else 1.0
     return mu_ok, rel, energy
+
+
+# ---- FP4 records: the byte layout of include/cobs.h (cobs_dims.stats_format) ----
+
+def fp4_record_bytes(d, r):
+    return (2 * d + r * (d // 2) + r * (d // 32) + 15) // 16 * 16
+
+
+def pack_fp4_records(mu, codes, scale_bytes):
+    """Oracle FP4 records (mu [nb, d] exact bf16 values, codes [nb, r, d],
+    scale bytes [nb, r, d/32]) -> [nb, record bytes] uint8."""
+    nb, r, d = codes.shape
+    out = np.zeros((nb, fp4_record_bytes(d, r)), dtype=np.uint8)
+    out[:, :2 * d] = _f64_to_bf16_bits(mu).reshape(nb, d).view(np.uint8).reshape(nb, 2 * d)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    c0 = 2 * d
+    out[:, c0:c0 + r * d // 2] = packed.reshape(nb, -1)
+    s0 = c0 + r * d // 2
+    out[:, s0:s0 + r * d // 32] = scale_bytes.reshape(nb, -1)
+    return out
+
+
+def unpack_fp4_records(raw, d, r):
+    """[nb, record bytes] uint8 -> (mu as fp64, codes, scale bytes, padding bytes)."""
+    raw = np.ascontiguousarray(raw, dtype=np.uint8)
+    nb = raw.shape[0]
+    mu = bits_to_f64(raw[:, :2 * d].copy().view(np.uint16))
+    c0 = 2 * d
+    packed = raw[:, c0:c0 + r * d // 2].reshape(nb, r, d // 2)
+    codes = np.empty((nb, r, d), dtype=np.uint8)
+    codes[..., 0::2] = packed & 15
+    codes[..., 1::2] = packed >> 4
+    s0 = c0 + r * d // 2
+    sb = raw[:, s0:s0 + r * d // 32].reshape(nb, r, d // 32)
+    return mu, codes, sb, raw[:, s0 + r * d // 32:]
+
+
+class Fp4Problem(Problem):
+    """A Problem whose block records are FP4 (COBS_STATS_FP4)."""
+
+    def __init__(self, w, **kw):
+        super().__init__(w, **kw)
+        self.dims4 = dict(self.dims, stats_format=cb.COBS_STATS_FP4)
+        self.rec = cb.cobs_stats_record_bytes(self.dims4)
+        assert self.rec == fp4_record_bytes(w.head_dim, w.rank)
+        self.stats4 = torch.zeros((w.batch, w.kv_heads, w.cap // w.block, self.rec),
+                                  dtype=torch.uint8, device="cuda")
+
+    def build_stats4(self, begin=0, end=None):
+        end = self.w.seq_len // self.w.block if end is None else end
+        cb.cobs_build_block_stats(self.dims4, self.k, begin, end, self.stats4, self.ws,
+                                  self.ws_bytes)
+
+    def select4(self, seq_len=None):
+        w = self.w
+        cb.cobs_select_blocks(self.dims4, self.q, self.stats4,
+                              w.seq_len if seq_len is None else seq_len, w.top_k,
+                              w.sink_blocks, w.local_tokens, self.idx, self.idx.shape[-1],
+                              self.n_sel, self.scores, self.ws, self.ws_bytes)
+
+    def oracle_records4(self, b, h, n_blocks=None):
+        w = self.w
+        n = w.seq_len // w.block if n_blocks is None else n_blocks
+        return O.build_block_records_fp4(self.keys(b, h), w.block, w.rank, 0, n)
+
+    def upload_records4(self, b, h, parts):
+        raw = pack_fp4_records(*parts)
+        self.stats4[b, h, :raw.shape[0]] = torch.from_numpy(raw).cuda()

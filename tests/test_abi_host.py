@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) == 15, names
+    assert len(names) == 16, names
     raw = ctypes.CDLL(cb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert cb.cobs_abi_version() == 1
+    assert cb.cobs_abi_version() == 2
     assert cb.cobs_status_string(0) == "COBS_OK"
     assert cb.cobs_status_string(5) == "COBS_ERR_TIMEOUT"
     assert cb.cobs_status_string(99) == "COBS_ERR_UNKNOWN"
@@ -233,3 +233,54 @@ def test_paged_host_checks():
         with pytest.raises(cb.CobsError) as e:
             fn()
         assert e.value.status == code, (e.value, code)
+
+
+def test_stats_record_bytes_and_format_checks():
+    from harness import fp4_record_bytes
+    for name in ("tiny_4k", "single_32k", "build_256k"):
+        w = WORKLOADS[name]
+        d = dims_of(w)
+        assert cb.cobs_stats_record_bytes(d) == (1 + w.rank) * w.head_dim * 2
+        d4 = dims_of(w, stats_format=cb.COBS_STATS_FP4)
+        n = cb.cobs_stats_record_bytes(d4)
+        assert n == fp4_record_bytes(w.head_dim, w.rank) and n % 16 == 0
+        assert n >= 2 * w.head_dim + w.rank * w.head_dim // 2 + w.rank * w.head_dim // 32
+    # d 128, r 8: 256 B of mu, 512 B of codes, 32 scale bytes
+    assert cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], rank=8,
+                                              stats_format=1)) == 800
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], stats_format=2))
+    assert e.value.status == cb.COBS_ERR_INVALID_ARG
+    with pytest.raises(cb.CobsError):
+        cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], rank=0, stats_format=1))
+    assert "rank" in cb.cobs_last_error()
+    A = 1 << 20
+    with pytest.raises(cb.CobsError) as e:   # FP4 records need a factor
+        cb.cobs_build_block_stats(dims_of(WORKLOADS["single_32k"], rank=0, stats_format=1),
+                                  A, 0, 1, A, A, 4096)
+    assert e.value.status == cb.COBS_ERR_UNSUPPORTED
+    # every call checks the format before launching anything
+    A = 1 << 20
+    bad = dims_of(WORKLOADS["single_32k"], stats_format=7)
+    with pytest.raises(cb.CobsError) as e:
+        cb.cobs_build_block_stats(bad, A, 0, 1, A, A, 4096)
+    assert e.value.status == cb.COBS_ERR_INVALID_ARG
+
+
+def test_fp4_record_packing_round_trip():
+    """The test-side packing of oracle FP4 records follows the header's layout."""
+    import numpy as np
+    import oracle.cobs_oracle as O
+    from harness import pack_fp4_records, unpack_fp4_records
+    rng = np.random.default_rng(0)
+    for d, r in ((128, 8), (64, 4), (128, 1), (64, 16)):
+        keys = O.round_to_bf16(rng.normal(0, 0.5, size=(3 * 64, d)))
+        mu, codes, sb = O.build_block_records_fp4(keys, 64, r, 0, 3)
+        raw = pack_fp4_records(mu, codes, sb)
+        m2, c2, s2, pad = unpack_fp4_records(raw, d, r)
+        np.testing.assert_array_equal(m2, mu)
+        np.testing.assert_array_equal(c2, codes)
+        np.testing.assert_array_equal(s2, sb)
+        assert raw.shape[1] % 16 == 0 and np.all(pad == 0)
+        # component 1 of column 0 is the high nibble of byte 2d
+        assert raw[0, 2 * d] >> 4 == codes[0, 0, 1] and raw[0, 2 * d] & 15 == codes[0, 0, 0]
