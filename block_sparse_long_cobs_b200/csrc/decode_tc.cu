@@ -135,7 +135,10 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-template <int G>
+// kMode: 0 one length for the batch, contiguous cache; 1 per-sequence
+// lengths; 2 page pools (lengths per sequence or one for the batch).  Each
+// instantiation carries only its own addressing and masking code.
+template <int G, int kMode>
 __global__ void __launch_bounds__(kThreads, 2)
 sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap,
@@ -238,8 +241,9 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           const int z = int(g.pair);
           const int qrow = int((g.pair / a.hkv) * a.hq + (g.pair % a.hkv) * G);
           const int64_t len_b =
-              sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status, false);
-          const int64_t blocks_b = (len_b + kBlock - 1) / kBlock;
+              kMode == 0 ? a.seq_len
+                         : sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status, false);
+          const int64_t blocks_b = kMode == 0 ? seq_blocks : (len_b + kBlock - 1) / kBlock;
           uint8_t* qbuf = base + kOffQ + (nonempty & 1) * 2048;
           for (int t = 0; t < T && ok; ++t) {
             const int nh = (2 * t + 1 < g.nb) ? 2 : 1;
@@ -249,7 +253,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
               // an index outside the sequence (or a page outside the pool)
               // reads an all-zero box past the tensor maps' row bound
               const bool in_seq = j >= 0 && j < blocks_b;
-              if (a.block_table == nullptr) {
+              if constexpr (kMode != 2) {
                 y[h2] = in_seq ? j * kBlock : int(seq_blocks * kBlock);
               } else {
                 const int32_t page =
@@ -510,9 +514,11 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       const int ob = nonempty & 1;
       const uint32_t use = uint32_t(nonempty) >> 1;
-      const int64_t len_b = sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status,
-                                            g.seg == 0 && r == 0);
-      const int64_t blocks_b = (len_b + kBlock - 1) / kBlock;
+      const int64_t len_b =
+          kMode == 0 ? a.seq_len
+                     : sequence_length(a.seq_lens, a.seq_len, g.pair / a.hkv, a.status,
+                                       g.seg == 0 && r == 0);
+      const int64_t blocks_b = kMode == 0 ? seq_blocks : (len_b + kBlock - 1) / kBlock;
       if (g.nb > 0) {
         const uint32_t ocol = kOCol + 16u * uint32_t(ob);
         const int T = (g.nb + 1) >> 1;
@@ -620,8 +626,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
               *reinterpret_cast<uint16_t*>(atom + 1024 + off) = lo;
             }
           }
-          if ((a.seq_lens != nullptr || a.block_table != nullptr) &&
-              named_bar_or(1, kSoftThreads, zero_row)) {
+          if (kMode != 0 && named_bar_or(1, kSoftThreads, zero_row)) {
             // the tail block of a shorter sequence: its V rows past the
             // sequence must be zero before P.V (a zero weight times a stale
             // or NaN value is not zero), so wait for the tile and clear them
@@ -675,7 +680,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
 template <int G>
 int occupancy_g() {
-  const int n = kernel_occupancy(reinterpret_cast<const void*>(sparse_decode_tc_kernel<G>),
+  const int n = kernel_occupancy(reinterpret_cast<const void*>(sparse_decode_tc_kernel<G, 0>),
                                  kThreads, kDynSmem);
   const int by_tmem = 512 / int(kTmemCols);   // TMEM columns of an SM
   return n < by_tmem ? n : by_tmem;
@@ -697,7 +702,9 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
   if (e == cudaSuccess)
     e = make_bf16_tensor_map_sw128(&qmap, a.q, kD, uint64_t(a.batch) * a.hq, 8);
   if (e != cudaSuccess) return e;
-  auto kern = sparse_decode_tc_kernel<G>;
+  auto kern = paged ? sparse_decode_tc_kernel<G, 2>
+                    : (a.seq_lens != nullptr ? sparse_decode_tc_kernel<G, 1>
+                                             : sparse_decode_tc_kernel<G, 0>);
   e = set_smem_attrs(kern, kDynSmem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(a.n_ctas), dim3(kThreads), kDynSmem, stream, kmap, vmap, qmap, a);
