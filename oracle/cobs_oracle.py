@@ -51,6 +51,14 @@ design notes of the repository):
   complete blocks; ties go to the lower block index.  Output ascending.
 * Attention over the selected blocks is one exact softmax over the union of
   their valid tokens, with the 1/sqrt(d) logit scale.
+* The min/max box selector (explainer, plain-language summary of what the
+  paper rules out: the spread of a block estimated from the minimum and
+  maximum of its keys; it helps somewhat, less than COBS; no formula is
+  given): the box is the per-dimension minimum lo and maximum hi of the
+  block's keys, and a block's score is ln n_b plus the largest logit any
+  point of the box can reach, max_{lo <= k <= hi} q.k / sqrt(d) =
+  sum_t max(q_t lo_t, q_t hi_t) / sqrt(d) -- an upper bound of the block's
+  log attention mass.  Groups aggregate as for COBS.
 * FP4 storage of U (§2.3, quantisation: eigenvectors stored scaled in FP4
   E2M1, block means in BF16): every U column is cut into groups of 32
   consecutive components; each group stores E2M1 codes and one power-of-two
@@ -94,6 +102,11 @@ __all__ = [
     "block_record_fp4",
     "build_block_records_fp4",
     "fp4_record_values",
+    "block_box",
+    "build_block_boxes",
+    "box_head_scores",
+    "box_group_scores",
+    "select_from_boxes",
 ]
 
 
@@ -439,3 +452,58 @@ def fp4_record_values(mu, codes, scale_bytes) -> np.ndarray:
     mu = np.asarray(mu, dtype=np.float64)
     u = dequantize_u_fp4(codes, scale_bytes)
     return np.concatenate([mu[:, None, :], u], axis=1)
+
+
+# ---------------------------------------------------------------------------
+# Min/max box selector (a comparison selector the explainer mentions: the
+# spread of a block from the minimum and maximum of its keys)
+# ---------------------------------------------------------------------------
+
+def block_box(keys: np.ndarray):
+    """Per-dimension minimum and maximum of one block's keys: (lo [d], hi [d])."""
+    keys = np.asarray(keys, dtype=np.float64)
+    return keys.min(axis=0), keys.max(axis=0)
+
+
+def build_block_boxes(keys_seq: np.ndarray, block: int, block_begin: int, block_end: int):
+    """Boxes of complete blocks [block_begin, block_end): (lo [nb, d], hi [nb, d])."""
+    d = keys_seq.shape[1]
+    boxes = [block_box(keys_seq[j * block:(j + 1) * block])
+             for j in range(block_begin, block_end)]
+    if not boxes:
+        return np.zeros((0, d)), np.zeros((0, d))
+    lo, hi = zip(*boxes)
+    return np.stack(lo), np.stack(hi)
+
+
+def box_head_scores(q: np.ndarray, lo: np.ndarray, hi: np.ndarray,
+                    n_tokens: np.ndarray) -> np.ndarray:
+    """s_b = ln n_b + max over the box of q.k / sqrt(d), for every block.
+
+    The maximum of a linear function over a box is reached at a corner: in
+    each dimension the end that q_t favours, so it is sum_t max(q_t lo_t,
+    q_t hi_t).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    reach = np.sum(np.maximum(q[None, :] * lo, q[None, :] * hi), axis=1)
+    return np.log(np.asarray(n_tokens, dtype=np.float64)) + reach / math.sqrt(d)
+
+
+def box_group_scores(q_group: np.ndarray, lo: np.ndarray, hi: np.ndarray,
+                     n_tokens: np.ndarray) -> np.ndarray:
+    """S_b = ln sum_h exp(s_{h,b}) over the G query heads of one kv-head."""
+    per_head = np.stack([box_head_scores(q, lo, hi, n_tokens)
+                         for q in np.asarray(q_group, dtype=np.float64)], axis=0)
+    return _logsumexp(per_head, axis=0)
+
+
+def select_from_boxes(q_group, lo, hi, seq_len, block, top_k, sink_blocks, local_tokens):
+    """Score every complete block by its box, then select (top-k + sink + local).
+
+    Returns (selected indices, group scores over complete blocks).
+    """
+    n_full = seq_len // block
+    scores = box_group_scores(q_group, lo[:n_full], hi[:n_full], np.full(n_full, block))
+    return select_blocks(scores, seq_len, block, top_k, sink_blocks,
+                         local_tokens), scores
