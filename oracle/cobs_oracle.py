@@ -51,6 +51,12 @@ design notes of the repository):
   complete blocks; ties go to the lower block index.  Output ascending.
 * Attention over the selected blocks is one exact softmax over the union of
   their valid tokens, with the 1/sqrt(d) logit scale.
+* Subspace projection (§2.3): the covariance is projected onto the span P
+  (d x s, orthonormal columns) of the top s eigenvectors of the queries'
+  second moment M = (1/n) sum q q^T over a set of calibration queries, so a
+  block stores U_s = P^T U (r x s values instead of r x d); the score's
+  quadratic term becomes 1/2 |U_s^T P^T q|^2 / d = 1/2 (P P^T q)^T Sigma_r
+  (P P^T q) / d.  The mean and the linear term keep all d dimensions.
 * The min/max box selector (explainer, plain-language summary of what the
   paper rules out: the spread of a block estimated from the minimum and
   maximum of its keys; it helps somewhat, less than COBS; no formula is
@@ -107,6 +113,13 @@ __all__ = [
     "box_head_scores",
     "box_group_scores",
     "select_from_boxes",
+    "query_subspace",
+    "project_factor",
+    "block_record_subspace",
+    "build_block_records_subspace",
+    "subspace_head_scores",
+    "subspace_group_scores",
+    "select_from_subspace_records",
 ]
 
 
@@ -505,5 +518,83 @@ def select_from_boxes(q_group, lo, hi, seq_len, block, top_k, sink_blocks, local
     """
     n_full = seq_len // block
     scores = box_group_scores(q_group, lo[:n_full], hi[:n_full], np.full(n_full, block))
+    return select_blocks(scores, seq_len, block, top_k, sink_blocks,
+                         local_tokens), scores
+
+
+# ---------------------------------------------------------------------------
+# Subspace projection (COBS explainer §2.3: the covariance projected onto the
+# query subspace spanned by the top eigenvectors of the queries' second
+# moment, storage r x d -> r x s)
+# ---------------------------------------------------------------------------
+
+def query_subspace(q_cal: np.ndarray, s: int) -> np.ndarray:
+    """P [d, s]: the top-s eigenvectors of M = (1/n) sum_i q_i q_i^T, descending
+    eigenvalue, each column's largest-magnitude component made positive."""
+    q_cal = np.asarray(q_cal, dtype=np.float64)
+    m = q_cal.T @ q_cal / q_cal.shape[0]
+    lam, vecs = np.linalg.eigh(m)
+    order = np.argsort(-lam, kind="stable")[:s]
+    p = vecs[:, order].copy()
+    for j in range(p.shape[1]):
+        i = int(np.argmax(np.abs(p[:, j])))
+        if p[i, j] < 0:
+            p[:, j] = -p[:, j]
+    return p
+
+
+def project_factor(u: np.ndarray, p: np.ndarray) -> np.ndarray:
+    """U_s = P^T U: the factor's columns in subspace coordinates, [s, r]."""
+    return np.asarray(p, dtype=np.float64).T @ np.asarray(u, dtype=np.float64)
+
+
+def block_record_subspace(keys: np.ndarray, rank: int, p: np.ndarray,
+                          to_bf16: bool = True) -> np.ndarray:
+    """(mu [d], U_s^T [r, s]) of one complete block, rounded to bf16 by default."""
+    mu, sigma = block_moments(keys)
+    u, _ = covariance_factor(sigma, rank)
+    us = project_factor(u, p).T
+    if to_bf16:
+        return round_to_bf16(mu), round_to_bf16(us)
+    return mu, us
+
+
+def build_block_records_subspace(keys_seq, block, rank, p, block_begin, block_end,
+                                 to_bf16: bool = True):
+    """Subspace records of complete blocks [block_begin, block_end): (mu [nb, d], us [nb, r, s])."""
+    d, s = p.shape
+    parts = [block_record_subspace(keys_seq[j * block:(j + 1) * block], rank, p, to_bf16)
+             for j in range(block_begin, block_end)]
+    if not parts:
+        return np.zeros((0, d)), np.zeros((0, rank, s))
+    mu, us = zip(*parts)
+    return np.stack(mu), np.stack(us)
+
+
+def subspace_head_scores(q: np.ndarray, mu: np.ndarray, us: np.ndarray, p: np.ndarray,
+                         n_tokens: np.ndarray) -> np.ndarray:
+    """s_b = ln n_b + (q.mu_b)/sqrt(d) + 1/2 |U_s,b^T (P^T q)|^2 / d."""
+    q = np.asarray(q, dtype=np.float64)
+    d = q.shape[0]
+    qs = np.asarray(p, dtype=np.float64).T @ q              # query in subspace coordinates
+    linear = mu @ q / math.sqrt(d)
+    proj = us @ qs                                         # [nb, r]
+    quadratic = 0.5 * np.sum(proj * proj, axis=1) / d
+    return np.log(np.asarray(n_tokens, dtype=np.float64)) + linear + quadratic
+
+
+def subspace_group_scores(q_group, mu, us, p, n_tokens) -> np.ndarray:
+    """S_b = ln sum_h exp(s_{h,b}) over the G query heads of one kv-head."""
+    per_head = np.stack([subspace_head_scores(q, mu, us, p, n_tokens)
+                         for q in np.asarray(q_group, dtype=np.float64)], axis=0)
+    return _logsumexp(per_head, axis=0)
+
+
+def select_from_subspace_records(q_group, mu, us, p, seq_len, block, top_k, sink_blocks,
+                                 local_tokens):
+    """Score every complete block from its subspace record, then select."""
+    n_full = seq_len // block
+    scores = subspace_group_scores(q_group, mu[:n_full], us[:n_full], p,
+                                   np.full(n_full, block))
     return select_blocks(scores, seq_len, block, top_k, sink_blocks,
                          local_tokens), scores
