@@ -103,11 +103,19 @@ lib = _load()
 
 
 def _ptr(x):
+    """Device address of a buffer argument (every pointer of the C ABI is a
+    device pointer): an int is taken as is; a torch tensor must be a
+    contiguous CUDA tensor (a host or strided tensor would hand the kernels a
+    wrong address)."""
     if x is None:
         return None
     if isinstance(x, int):
         return ctypes.c_void_p(x)
     if hasattr(x, "data_ptr"):
+        if hasattr(x, "is_cuda") and not x.is_cuda:
+            raise TypeError("tensor arguments must be CUDA tensors (got a host tensor)")
+        if hasattr(x, "is_contiguous") and not x.is_contiguous():
+            raise TypeError("tensor arguments must be contiguous")
         return ctypes.c_void_p(x.data_ptr())
     if hasattr(x, "ctypes"):
         return ctypes.c_void_p(x.ctypes.data)

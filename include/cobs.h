@@ -24,8 +24,11 @@
  *
  * Conventions for every call:
  *   - The caller owns all memory.  The library never allocates device or
- *     pinned memory and keeps no global state except a thread-local copy of
- *     the last error message.
+ *     pinned memory at run time.  Its only state is a thread-local copy of
+ *     the last error message, a process-wide, mutex-guarded cache of kernel
+ *     attributes and occupancy per (kernel, device), and the fixed 16 MiB
+ *     device array of cobs_sparse_decode_no_alloc (static device memory that
+ *     the CUDA runtime sets up with the library's module).
  *   - Device pointers must be 16-byte aligned.  Host-side argument checks
  *     happen before anything is launched; a failed check returns an error
  *     code and launches nothing.

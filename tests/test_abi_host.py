@@ -284,3 +284,18 @@ def test_fp4_record_packing_round_trip():
         assert raw.shape[1] % 16 == 0 and np.all(pad == 0)
         # component 1 of column 0 is the high nibble of byte 2d
         assert raw[0, 2 * d] >> 4 == codes[0, 0, 1] and raw[0, 2 * d] & 15 == codes[0, 0, 0]
+
+
+def test_binding_rejects_host_and_strided_tensors():
+    """Every pointer of the ABI is a device pointer: host or strided torch
+    tensors are refused before the library is called."""
+    import torch
+    w = WORKLOADS["tiny_4k"]
+    d = dims_of(w)
+    host = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        cb.cobs_workspace_init(host, 16)
+    strided = torch.zeros((4, 8))[:, ::2]
+    assert not strided.is_contiguous()
+    with pytest.raises(TypeError):
+        cb.cobs_build_block_stats(d, strided, 0, 1, 1 << 20, 1 << 20, 4096)
