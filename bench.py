@@ -2,6 +2,7 @@
 """Decode-step throughput of the COBS block-sparse attention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cobs|reference]
+                    [--stats-format bf16|fp4] [--stats-stream side|same] [--batch B]
 
 One step is one pass of the whole hot path over a batch of synthetic
 queries: the statistics of the block that just became complete (one block per
@@ -9,8 +10,13 @@ queries: the statistics of the block that just became complete (one block per
 local window) and the split-K sparse flash-decode with its log-sum-exp merge —
 three C-ABI calls, three kernel launches.  The KV cache and the statistics of
 all earlier blocks are resident in HBM before timing starts; L2 is flushed
-(256 MiB write) between timed steps and each step is timed with CUDA events
-on the stream its kernels run on.
+(256 MiB written, then read) between timed steps and each step is timed with
+CUDA events on the stream its kernels run on.  The statistics build runs on a
+forked side stream by default (``--stats-stream same`` keeps it in line);
+``--stats-format fp4`` stores U in scaled FP4 (E2M1) instead of bf16.  The
+line also carries an end-to-end figure through the public calls with host
+buffers (``e2e``), the oracle on the host cores (``cpu_baseline``) and the
+roofline of the kernel that dominates the step.
 
 Workload (default): batch 32, 32 query / 8 KV heads, head_dim 128, 32768
 cached tokens, block 64, rank 8, top-k 16 + sink block + 512-token window,
