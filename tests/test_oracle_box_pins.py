@@ -10,6 +10,7 @@ import itertools
 import math
 
 import numpy as np
+import pytest
 
 import oracle.cobs_oracle as O
 
@@ -89,3 +90,28 @@ def test_box_selection_follows_the_selection_rules():
     cand = [j for j in sel if c0 <= j < c1]
     rest = [j for j in range(c0, c1) if j not in cand]
     assert min(scores[j] for j in cand) >= max(scores[j] for j in rest)
+
+
+# ---------------------------------------------------------------------------
+# plausible mistakes planted in the oracle (on the CPU) must trip a pin
+# ---------------------------------------------------------------------------
+
+def _expect_pin_failure(monkeypatch, name, bad, pin):
+    monkeypatch.setattr(O, name, bad)
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_mutation_box_centre_only(monkeypatch):
+    def bad(q, lo, hi, n):      # the box's centre, not its reach
+        return np.log(np.asarray(n, float)) + ((lo + hi) / 2) @ q / math.sqrt(len(q))
+    _expect_pin_failure(monkeypatch, "box_head_scores", bad,
+                        test_score_is_the_maximum_over_the_corners)
+
+
+def test_mutation_box_min_instead_of_max(monkeypatch):
+    def bad(q, lo, hi, n):
+        reach = np.sum(np.minimum(q[None, :] * lo, q[None, :] * hi), axis=1)
+        return np.log(np.asarray(n, float)) + reach / math.sqrt(len(q))
+    _expect_pin_failure(monkeypatch, "box_head_scores", bad,
+                        test_score_bounds_the_exact_log_mass_from_above)

@@ -137,3 +137,59 @@ def test_fp4_factor_error_bounded_by_the_grid():
     deq = O.dequantize_u_fp4(codes, sb)
     step = np.repeat(np.exp2(sb.astype(float) - 127), 32, axis=1)
     assert np.all(np.abs(deq - u.T) <= step + 1e-15)
+
+
+# ---------------------------------------------------------------------------
+# plausible mistakes planted in the oracle (on the CPU) must trip a pin
+# ---------------------------------------------------------------------------
+
+def _expect_pin_failure(monkeypatch, name, bad, pin):
+    monkeypatch.setattr(O, name, bad)
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_mutation_ties_to_odd(monkeypatch):
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.minimum(np.abs(x), 6.0)
+        grid = np.asarray(O.E2M1_MAGNITUDES)
+        dist = np.abs(a[..., None] - grid)
+        nearest = dist == dist.min(axis=-1, keepdims=True)
+        pick = len(grid) - 1 - np.argmax(nearest[..., ::-1], axis=-1)   # the larger code
+        return np.where((x < 0) & (pick != 0), pick | 8, pick).astype(np.uint8)
+    _expect_pin_failure(monkeypatch, "round_to_e2m1", bad, test_known_ties)
+
+
+def test_mutation_saturating_exponent(monkeypatch):
+    def bad(amax):   # floor(log2 amax) - 2: values in (6, 8) x 2^e would clip
+        if amax == 0.0:
+            return None
+        return max(int(math.floor(math.log2(amax))) - 2, -126)
+    _expect_pin_failure(monkeypatch, "fp4_scale_exponent", bad,
+                        test_scale_exponent_is_the_smallest_that_fits)
+
+
+def test_mutation_wrong_grid(monkeypatch):
+    monkeypatch.setattr(O, "E2M1_MAGNITUDES", (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 5.0))
+    with pytest.raises(AssertionError):
+        test_code_values_match_the_bit_field_definition()
+
+
+def test_mutation_groups_of_16(monkeypatch):
+    def bad(u_rows):
+        u_rows = np.asarray(u_rows, dtype=np.float64)
+        r, d = u_rows.shape
+        codes = np.zeros((r, d), dtype=np.uint8)
+        scale_bytes = np.zeros((r, d // 32), dtype=np.uint8)
+        for j in range(r):
+            for g in range(d // 16):
+                seg = u_rows[j, g * 16:(g + 1) * 16]
+                e = O.fp4_scale_exponent(float(np.max(np.abs(seg))))
+                if e is None:
+                    continue
+                scale_bytes[j, g // 2] = e + 127
+                codes[j, g * 16:(g + 1) * 16] = O.round_to_e2m1(seg / 2.0 ** e)
+        return codes, scale_bytes
+    _expect_pin_failure(monkeypatch, "quantize_u_fp4", bad,
+                        test_quantised_components_within_half_a_grid_step)

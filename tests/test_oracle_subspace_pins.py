@@ -9,6 +9,7 @@ covariance's quadratic form at the projected query, by hand."""
 import math
 
 import numpy as np
+import pytest
 
 import oracle.cobs_oracle as O
 
@@ -114,3 +115,33 @@ def test_second_moment_not_covariance():
     p = O.query_subspace(q_cal + m[None, :], 2)
     assert abs(abs(p[:, 0] @ m) / 3.0 - 1.0) <= 1e-10
     assert abs(abs(p[:, 1] @ v[:, 0]) - 1.0) <= 1e-10
+
+
+# ---------------------------------------------------------------------------
+# plausible mistakes planted in the oracle (on the CPU) must trip a pin
+# ---------------------------------------------------------------------------
+
+def _expect_pin_failure(monkeypatch, name, bad, pin):
+    monkeypatch.setattr(O, name, bad)
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_mutation_centred_covariance(monkeypatch):
+    def bad(q_cal, s):
+        q_cal = np.asarray(q_cal, dtype=np.float64)
+        c = q_cal - q_cal.mean(axis=0)
+        lam, vecs = np.linalg.eigh(c.T @ c / q_cal.shape[0])
+        return vecs[:, np.argsort(-lam, kind="stable")[:s]]
+    _expect_pin_failure(monkeypatch, "query_subspace", bad, test_second_moment_not_covariance)
+
+
+def test_mutation_query_not_projected(monkeypatch):
+    def bad(q, mu, us, p, n):   # the first s query components instead of P^T q
+        q = np.asarray(q, dtype=np.float64)
+        d, s = p.shape
+        proj = us @ q[:s]
+        return (np.log(np.asarray(n, float)) + mu @ q / math.sqrt(d)
+                + 0.5 * np.sum(proj * proj, axis=1) / d)
+    _expect_pin_failure(monkeypatch, "subspace_head_scores", bad,
+                        test_queries_inside_the_subspace_lose_nothing)
