@@ -16,7 +16,7 @@ __all__ = [
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
-    "cobs_read_device_status",
+    "cobs_read_device_status", "cobs_no_alloc_read_status",
     "cobs_last_error", "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",

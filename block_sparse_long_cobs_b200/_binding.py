@@ -22,7 +22,7 @@ __all__ = [
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
-    "cobs_read_device_status", "cobs_last_error",
+    "cobs_read_device_status", "cobs_no_alloc_read_status", "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",
@@ -89,6 +89,7 @@ def _load() -> ctypes.CDLL:
         "cobs_sparse_decode_paged": (I32, [D, P, P, P, I64, P, I32, P, P, I32, P, I64, F32, P,
                                            P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
+        "cobs_no_alloc_read_status": (I32, [ctypes.POINTER(I32), P]),
         "cobs_last_error": (ctypes.c_char_p, []),
         "cobs_status_string": (ctypes.c_char_p, [I32]),
     }
@@ -273,4 +274,13 @@ def cobs_read_device_status(ws, ws_bytes, stream=None) -> int:
     st = lib.cobs_read_device_status(_ptr(ws), ws_bytes, ctypes.byref(out),
                                      _stream(stream))
     _check("cobs_read_device_status", st, True)
+    return out.value
+
+
+def cobs_no_alloc_read_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the status word of the
+    allocation-free decode's fixed array on the current device."""
+    out = ctypes.c_int32(0)
+    st = lib.cobs_no_alloc_read_status(ctypes.byref(out), _stream(stream))
+    _check("cobs_no_alloc_read_status", st, True)
     return out.value

@@ -617,7 +617,11 @@ cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_s
 namespace cobs {
 namespace {
 
+// Layout of the fixed array: a status word in the first 256 bytes (kept
+// across calls until cobs_no_alloc_read_status clears it), then the arrival
+// and work counters (cleared by every call), then the split partials.
 constexpr size_t kFixedScratchBytes = size_t(16) << 20;   // per device, held until exit
+constexpr size_t kFixedStatusBytes = 256;
 __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -676,8 +680,9 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   const DecodePlan P = plan_decode(dims->head_dim, dims->num_q_heads / dims->num_kv_heads,
                                    pairs, idx_stride);
   const size_t tickets_bytes = align256((size_t(pairs) + 2) * 4);
-  const size_t need = tickets_bytes + size_t(dims->batch) * dims->num_q_heads *
-                                          size_t(P.part_rows) * (size_t(dims->head_dim) + 2) * 4;
+  const size_t need = kFixedStatusBytes + tickets_bytes +
+                      size_t(dims->batch) * dims->num_q_heads * size_t(P.part_rows) *
+                          (size_t(dims->head_dim) + 2) * 4;
   if (need > kFixedScratchBytes)
     return fail(COBS_ERR_WORKSPACE,
                 "this decode needs %zu bytes of scratch, above the library's fixed %zu; use "
@@ -687,13 +692,14 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   void* scratch = nullptr;
   if ((st = fixed_scratch_address(&scratch)) != COBS_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(scratch);
   // arrival and work counters must start at zero (the kernel leaves them at
-  // zero, but a previous call may have been cut short)
-  cudaError_t e = cudaMemsetAsync(scratch, 0, tickets_bytes, s);
+  // zero, but a previous call may have been cut short); the status word is
+  // left alone so that it collects every call's device errors until read
+  cudaError_t e = cudaMemsetAsync(w + kFixedStatusBytes, 0, tickets_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the fixed scratch counters");
 
   DecodeArgs a{};
-  char* w = static_cast<char*>(scratch);
   a.q = static_cast<const uint16_t*>(q);
   a.k = static_cast<const uint16_t*>(k);
   a.v = static_cast<const uint16_t*>(v);
@@ -701,9 +707,9 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   a.n_sel = n_sel;
   a.out = out;
   a.lse = lse;
-  a.tickets = reinterpret_cast<uint32_t*>(w);
-  a.partials = reinterpret_cast<float*>(w + tickets_bytes);
-  a.status = nullptr;   // no status word: out-of-range blocks are skipped silently
+  a.tickets = reinterpret_cast<uint32_t*>(w + kFixedStatusBytes);
+  a.partials = reinterpret_cast<float*>(w + kFixedStatusBytes + tickets_bytes);
+  a.status = reinterpret_cast<int32_t*>(w);
   a.cap = dims->capacity_tokens;
   a.seq_len = seq_len;
   a.batch = dims->batch;
@@ -722,6 +728,22 @@ cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q, co
   a.work = a.tickets + pairs;
   e = launch_decode(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "sparse decode launch");
+  return ok();
+}
+
+cobs_status cobs_no_alloc_read_status(int32_t* device_status, void* stream) {
+  if (!device_status) return fail(COBS_ERR_INVALID_ARG, "device_status is NULL");
+  void* scratch = nullptr;
+  cobs_status st = fixed_scratch_address(&scratch);
+  if (st != COBS_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(scratch, 0, sizeof(v), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the fixed scratch status word");
+  *device_status = v;
   return ok();
 }
 

@@ -28,7 +28,8 @@
  *     the last error message, a process-wide, mutex-guarded cache of kernel
  *     attributes and occupancy per (kernel, device), and the fixed 16 MiB
  *     device array of cobs_sparse_decode_no_alloc (static device memory that
- *     the CUDA runtime sets up with the library's module).
+ *     the CUDA runtime places in a device's context when the library's
+ *     kernels are first used there).
  *   - Device pointers must be 16-byte aligned.  Host-side argument checks
  *     happen before anything is launched; a failed check returns an error
  *     code and launches nothing.
@@ -286,9 +287,11 @@ COBS_API cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void*
 
 /* Allocation-free form of cobs_sparse_decode (this library's own addition; the
  * method's description has no counterpart).  Same arguments and results, but
- * there is no workspace argument: the split-K partial results and arrival
- * counters go to a fixed 16 MiB array that the library itself places in every
- * GPU's memory when it is loaded and keeps until the process exits.  It is for
+ * there is no workspace argument: the split-K partial results, arrival
+ * counters and a device status word go to a fixed 16 MiB array owned by the
+ * library.  The CUDA runtime places that array in a device's context the
+ * first time any kernel of this library is used on that device (not only
+ * this call's), and it stays there until the process exits.  The call is for
  * callers that cannot hand the library device memory of its own: code whose
  * host framework owns every device allocation, code running where allocation
  * is forbidden or too slow (a real-time or latency-critical loop, an
@@ -302,16 +305,24 @@ COBS_API cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void*
  *     it and give wrong results: serialise them.
  *   - Nothing is allocated or freed (no cudaMalloc / cudaFree / library
  *     allocator calls).  A problem whose scratch would exceed 16 MiB
- *     (batch * num_q_heads * splits * (head_dim + 2) * 4 bytes plus the
- *     counters) is rejected with COBS_ERR_WORKSPACE.
- *   - There is no status word: an out-of-range block index is skipped
- *     without being reported. */
+ *     (256 bytes + batch * num_q_heads * splits * (head_dim + 2) * 4 bytes
+ *     plus the counters) is rejected with COBS_ERR_WORKSPACE.
+ *   - Device-side problems (a block index outside the sequence, an n_sel
+ *     outside [1, idx_stride], a bounded wait that ran out and left out/lse
+ *     partly written) are recorded in the array's own status word, which no
+ *     call clears: read it with cobs_no_alloc_read_status(). */
 COBS_API cobs_status cobs_sparse_decode_no_alloc(const cobs_dims* dims, const void* q,
                                                  const void* k, const void* v,
                                                  const int32_t* idx, const int32_t* n_sel,
                                                  int32_t idx_stride, int64_t seq_len,
                                                  float softmax_scale, float* out,
                                                  float* lse, void* stream);
+
+/* Synchronise `stream`, copy the status word of cobs_sparse_decode_no_alloc's
+ * fixed array on the current device to *device_status (COBS_OK or the first
+ * device-side error code since the last read) and clear it.  Allocates
+ * nothing.  Returns CUDA on a failed copy, INVALID_ARG on a NULL pointer. */
+COBS_API cobs_status cobs_no_alloc_read_status(int32_t* device_status, void* stream);
 
 /* Synchronise `stream`, copy the workspace status word to *device_status
  * (COBS_OK or the first device-side error code since the last read) and

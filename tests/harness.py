@@ -252,3 +252,71 @@ class Fp4Problem(Problem):
     def upload_records4(self, b, h, parts):
         raw = pack_fp4_records(*parts)
         self.stats4[b, h, :raw.shape[0]] = torch.from_numpy(raw).cuda()
+
+
+def explain_selection(w, q_group, gpu_sel, gpu_recs, orc_recs, seq_len=None):
+    """End-to-end selection check that explains every flip.
+
+    ``gpu_recs`` are the records the GPU built (as fp64 values), ``orc_recs``
+    the oracle's, both [n_full, 1 + r, d].  Two facts are asserted:
+
+    1. The GPU selection is the oracle's selection rule applied to the GPU's
+       own records (up to reported ties): the selection kernel adds nothing.
+    2. Every block in which the GPU and the oracle selections differ has an
+       oracle score within 2 Delta (+ the tie tolerance) of the oracle's top-k
+       boundary, Delta = max over candidates |S(gpu record) - S(oracle record)|.
+       Moving every score by at most Delta moves the k-th largest by at most
+       Delta, so a block can only cross the boundary from within 2 Delta.
+
+    Returns (number of differing blocks, Delta, list of (block, oracle score,
+    boundary, per-block score change) for the differing blocks)."""
+    seq_len = w.seq_len if seq_len is None else seq_len
+    n_full = seq_len // w.block
+    n_tok = np.full(n_full, w.block)
+    s_g = O.group_block_scores(q_group, gpu_recs[:n_full], n_tok)
+    s_o = O.group_block_scores(q_group, orc_recs[:n_full], n_tok)
+    sel_g = O.select_blocks(s_g, seq_len, w.block, w.top_k, w.sink_blocks, w.local_tokens)
+    assert selection_mismatch(gpu_sel, sel_g, s_g, w, seq_len) == [], "selection vs own records"
+    sel_o = O.select_blocks(s_o, seq_len, w.block, w.top_k, w.sink_blocks, w.local_tokens)
+    _, c0, c1 = O.block_partition(seq_len, w.block, w.sink_blocks, w.local_tokens)
+    if c1 <= c0:
+        assert set(int(x) for x in gpu_sel) == set(int(x) for x in sel_o)
+        return 0, 0.0, []
+    delta = float(np.max(np.abs(s_g[c0:c1] - s_o[c0:c1])))
+    cand = np.arange(c0, c1)
+    order = np.lexsort((cand, -s_o[c0:c1]))
+    k = min(w.top_k, c1 - c0)
+    boundary = float(s_o[c0:c1][order[k - 1]]) if k > 0 else -np.inf
+    diff = sorted(set(int(x) for x in gpu_sel) ^ set(int(x) for x in sel_o))
+    rows = []
+    for j in diff:
+        assert c0 <= j < c1, ("forced block differs", j)
+        slack = 2 * delta + TIE_RTOL * max(1.0, abs(boundary))
+        assert abs(s_o[j] - boundary) <= slack, (j, float(s_o[j]), boundary, delta)
+        rows.append((j, float(s_o[j]), boundary, float(abs(s_g[j] - s_o[j]))))
+    return len(diff), delta, rows
+
+
+def score_change_bound(q_group, orc_rec, rank):
+    """A-priori bound of |s_h(GPU record) - s_h(oracle record)| over the heads
+    of one block when the GPU record meets the statistics tolerance: each mean
+    component within one bf16 step (|d mu| <= 2^-7 |mu|) and the projector
+    within PROJ_RTOL (relative Frobenius) of the oracle's:
+        |q.d mu| / sqrt(d) + 1/2 |q|^2 |d Sigma_r|_2 / d
+        <= |q| 2^-7 |mu| / sqrt(d) + 1/2 |q|^2 PROJ_RTOL |Sigma_r|_F / d."""
+    d = orc_rec.shape[1]
+    mu, u = orc_rec[0], orc_rec[1:1 + rank].T
+    proj_f = float(np.linalg.norm(u @ u.T)) if rank else 0.0
+    qn = np.linalg.norm(np.asarray(q_group, dtype=np.float64), axis=1)
+    return float(np.max(qn * 2.0 ** -7 * np.linalg.norm(mu) / math.sqrt(d)
+                        + 0.5 * qn ** 2 * PROJ_RTOL * proj_f / d))
+
+
+def block_is_gapped(keys_block, rank):
+    """Whether the block's covariance spectrum fixes its top-r subspace
+    (lambda_r / lambda_{r+1} >= GAP_MIN, or lambda_{r+1} = 0)."""
+    if rank == 0:
+        return True
+    _, sigma = O.block_moments(keys_block)
+    lam = np.sort(np.linalg.eigvalsh(sigma))[::-1]
+    return bool(lam[rank] <= 0 or lam[rank - 1] / lam[rank] >= GAP_MIN)

@@ -37,3 +37,15 @@ def test_traffic_record_is_dropped_when_the_kernel_changes(monkeypatch):
     monkeypatch.setattr(bench, "source_hash", lambda name: "0" * 16)
     assert bench.recorded_traffic("select.cu", "batched_needles_32k") is None
     assert real is None or real > 0
+
+
+def test_oracle_baseline_runs_on_several_cores_at_once():
+    # two spawn-started processes, each decoding its own (batch, kv-head) pair
+    # of a small workload; the rate sums their queries over the slower one's time
+    w = WORKLOADS["tiny_4k"].scaled(batch=2)
+    value, steps, dt, pairs = bench.oracle_rate(w, 2, steps=3, warmup=1)
+    assert steps == 3 and dt > 0 and value > 0
+    assert pairs == [(0, 0), (1, 0)]
+    one, steps1, _, _ = bench.oracle_rate(w, 1, steps=2, warmup=1)
+    assert steps1 == 2 and one > 0
+    assert bench.oracle_cores() >= 1

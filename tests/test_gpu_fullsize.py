@@ -14,8 +14,9 @@ import pytest
 import torch
 
 import oracle.cobs_oracle as O
-from harness import (ENERGY_RTOL, LSE_ATOL, OUT_ATOL, PROJ_RTOL, Problem, from_dev_bits,
-                     selection_mismatch, stats_errors)
+from harness import (ENERGY_RTOL, LSE_ATOL, OUT_ATOL, PROJ_RTOL, Problem, block_is_gapped,
+                     explain_selection, from_dev_bits, score_change_bound, selection_mismatch,
+                     stats_errors)
 from workloads import WORKLOADS, bits_to_f64, make_queries
 
 pytestmark = pytest.mark.gpu
@@ -107,29 +108,42 @@ def test_full_decode_on_oracle_selection(full):
     assert p.device_status() == 0
 
 
-def test_full_end_to_end_flips_reported(full):
-    """GPU stats -> GPU selection, compared with the oracle end to end.  Flips
-    on near-degenerate spectra are reported, not failed (the eigen step is not
-    bit-reproducible); outputs must match wherever the selections agree."""
+def test_full_end_to_end_flips_explained(full):
+    """GPU stats -> GPU selection -> GPU decode, compared with the oracle end
+    to end.  The eigen step is not bit-reproducible, so the GPU and oracle
+    selections may differ on near-degenerate spectra; every such flip must be
+    explained by the records: the GPU selection equals the oracle's rule on
+    the GPU's own records, and a flipped block's oracle score lies within
+    twice the largest record-induced score change of the top-k boundary (on
+    gapped blocks that change also stays under the bound the statistics
+    tolerance implies).  Outputs are checked on every sampled pair against the
+    oracle's attention over the GPU's selection."""
     p, w = full, full.w
     p.stats.copy_(p.gpu_stats)
     p.select()
     p.decode()
     idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
     out = p.out.cpu().numpy()
+    st = from_dev_bits(p.gpu_stats)
     G = w.group
-    flips = 0
+    nfull = w.seq_len // w.block
+    flips, deltas = 0, []
     for (b, h), recs in p.orc_recs.items():
-        sel, s = O.select_from_records(p.q_group(b, h), recs, w.seq_len, w.block, w.top_k,
-                                       w.sink_blocks, w.local_tokens)
         got = idx[b, h, :n[b, h]]
-        if set(got.tolist()) != set(sel.tolist()):
-            flips += 1
-            continue
-        o, _ = O.sparse_attention(p.q_group(b, h), p.keys(b, h), p.values(b, h), sel,
-                                  w.seq_len, w.block, 1 / math.sqrt(w.head_dim))
-        assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL
-    print(f"{w.name}: end-to-end selection flips on {flips} of {len(p.orc_recs)} sampled pairs")
+        gpu_recs = bits_to_f64(st[b, h, :nfull])
+        nd, delta, rows = explain_selection(w, p.q_group(b, h), got, gpu_recs, recs)
+        flips += nd > 0
+        deltas.append(delta)
+        keys = p.keys(b, h)
+        for (j, _, _, change) in rows:
+            if block_is_gapped(keys[j * 64:(j + 1) * 64], w.rank):
+                assert change <= score_change_bound(p.q_group(b, h), recs[j], w.rank), (b, h, j)
+        o, _ = O.sparse_attention(p.q_group(b, h), keys, p.values(b, h),
+                                  got.astype(np.int64), w.seq_len, w.block,
+                                  1 / math.sqrt(w.head_dim))
+        assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL, (b, h)
+    print(f"{w.name}: selections differ from the oracle's on {flips} of {len(p.orc_recs)} "
+          f"sampled pairs, largest record-induced score change {max(deltas):.2e}")
     assert p.device_status() == 0
 
 

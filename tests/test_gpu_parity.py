@@ -11,7 +11,8 @@ import torch
 
 import oracle.cobs_oracle as O
 from harness import (ENERGY_RTOL, LSE_ATOL, OUT_ATOL, PROJ_RTOL, TIE_RTOL, Problem,
-                     from_dev_bits, selection_mismatch, stats_errors, to_dev)
+                     block_is_gapped, explain_selection, from_dev_bits, score_change_bound,
+                     selection_mismatch, stats_errors, to_dev)
 from workloads import WORKLOADS, bits_to_f64
 
 pytestmark = pytest.mark.gpu
@@ -170,26 +171,36 @@ def test_stats_build(prob):
 
 
 def test_end_to_end_pipeline(prob):
+    """GPU stats, selection and decode against the oracle on every pair: each
+    selection flip explained by the records (explain_selection), outputs equal
+    to the oracle's attention over the GPU's selection."""
     p, w = prob, prob.w
     p.build_stats()
     p.select()
     p.decode()
     idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
     out = p.out.cpu().numpy()
+    st = from_dev_bits(p.stats)
     G = w.group
     scale = 1 / math.sqrt(w.head_dim)
+    nfull = w.seq_len // w.block
     flips = 0
     for b in range(w.batch):
         for h in range(w.kv_heads):
-            sel, s = oracle_selection(p, b, h)
+            recs = p.oracle_records(b, h)
             got = idx[b, h, :n[b, h]]
-            if set(got.tolist()) != set(sel.tolist()):
-                flips += 1
-                continue
-            o, _ = O.sparse_attention(p.q_group(b, h), p.keys(b, h), p.values(b, h), sel,
-                                      w.seq_len, w.block, scale)
+            nd, _, rows = explain_selection(w, p.q_group(b, h), got,
+                                            bits_to_f64(st[b, h, :nfull]), recs)
+            flips += nd > 0
+            keys = p.keys(b, h)
+            for (j, _, _, change) in rows:
+                if block_is_gapped(keys[j * 64:(j + 1) * 64], w.rank):
+                    assert change <= score_change_bound(p.q_group(b, h), recs[j], w.rank)
+            o, _ = O.sparse_attention(p.q_group(b, h), keys, p.values(b, h),
+                                      got.astype(np.int64), w.seq_len, w.block, scale)
             assert np.max(np.abs(out[b, h * G:(h + 1) * G] - o)) <= OUT_ATOL
-    print(f"end-to-end selection flips: {flips} of {w.batch * w.kv_heads} pairs")
+    print(f"end-to-end selections differing from the oracle's: {flips} of "
+          f"{w.batch * w.kv_heads} pairs (each explained by its records)")
     assert p.device_status() == 0
 
 
