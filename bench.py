@@ -71,8 +71,12 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true",
                    help="enqueue the timed steps call by call instead of replaying CUDA graphs")
-    p.add_argument("--stats-format", choices=["bf16", "fp4"], default="bf16",
-                   help="block records: mu and U in bf16, or U in scaled FP4 (E2M1)")
+    p.add_argument("--stats-format", choices=["bf16", "fp4", "box", "subspace"], default="bf16",
+                   help="block records: mu and U in bf16, U in scaled FP4 (E2M1), the "
+                        "per-dimension min/max box (comparison selector), or U projected on "
+                        "a query subspace")
+    p.add_argument("--subspace-dim", type=int, default=85,
+                   help="s of the subspace records (the explainer's adaptive s ~ 85 of 128)")
     p.add_argument("--stats-stream", choices=["side", "same"], default="side",
                    help="run the completed block's stats build on a forked side stream "
                         "(joined before the step ends) or in line before the selection")
@@ -378,6 +382,24 @@ def cpu_baseline(w, seconds):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
+def calibrate_subspace(w, s, steps=8):
+    """Query-subspace basis of the subspace records, [kv_heads, s, d] fp32:
+    per kv-head, the top-s eigenvectors of the uncentred second moment
+    (1/n) sum q q^T of calibration queries -- here seeded draws of the
+    workload's own query distribution for `steps` decode steps (there is no
+    trained model to calibrate on).  An offline set-up step, like loading a
+    calibrated basis; it is not part of the timed path."""
+    from workloads import bits_to_f64, make_queries
+    d, G = w.head_dim, w.group
+    qs = np.stack([bits_to_f64(make_queries(w, 1000 + t)) for t in range(steps)])
+    out = np.zeros((w.kv_heads, s, d), dtype=np.float32)
+    for h in range(w.kv_heads):
+        q = qs[:, :, h * G:(h + 1) * G].reshape(-1, d)
+        lam, vec = np.linalg.eigh(q.T @ q / q.shape[0])
+        out[h] = vec[:, np.argsort(-lam, kind="stable")[:s]].T
+    return out
+
+
 def run_cobs(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -394,11 +416,14 @@ def run_cobs(args, w, rank, world, local_rank):
     def up(x):
         return torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).to(dev)
 
+    fmt = {"bf16": cb.COBS_STATS_BF16, "fp4": cb.COBS_STATS_FP4, "box": cb.COBS_STATS_BOX,
+           "subspace": cb.COBS_STATS_SUBSPACE}[args.stats_format]
     dims = dict(batch=w.batch, num_q_heads=w.q_heads, num_kv_heads=w.kv_heads,
                 head_dim=w.head_dim, block_size=w.block, rank=w.rank,
-                capacity_tokens=w.cap,
-                stats_format=cb.COBS_STATS_FP4 if args.stats_format == "fp4"
-                else cb.COBS_STATS_BF16)
+                capacity_tokens=w.cap, stats_format=fmt)
+    if args.stats_format == "subspace":
+        basis = torch.from_numpy(calibrate_subspace(w, args.subspace_dim)).to(dev)
+        dims.update(subspace_dim=args.subspace_dim, subspace_basis=basis)
     q, k, v = up(q_bits), up(k_bits), up(v_bits)
     nb_cap = w.cap // w.block
     nfull = w.seq_len // w.block
@@ -677,8 +702,9 @@ def run_cobs(args, w, rank, world, local_rank):
 
     hbm, peak_kind = peaks()
     bm = byte_model(w, round(n_sel_mean), rec_bytes)
-    traffic_key = w.name if args.stats_format == "bf16" else f"{w.name}:fp4"
-    per_kernel = {"stats": (t_stats, bm["stats"], "stats.cu"),
+    traffic_key = w.name if args.stats_format == "bf16" else f"{w.name}:{args.stats_format}"
+    per_kernel = {"stats": (t_stats, bm["stats"],
+                            "box.cu" if args.stats_format == "box" else "stats.cu"),
                   "select": (t_sel, bm["select"], "select.cu"),
                   "decode": (t_dec, bm["decode"],
                              "decode_tc.cu" if w.head_dim == 128 else "decode.cu")}
@@ -709,6 +735,8 @@ def run_cobs(args, w, rank, world, local_rank):
                    "step": "stats of the completed block + select + sparse decode",
                    "stats_stream": args.stats_stream,
                    "stats_format": args.stats_format, "record_bytes": rec_bytes,
+                   **({"subspace_dim": args.subspace_dim}
+                      if args.stats_format == "subspace" else {}),
                    "launch": (f"CUDA graphs of {g_steps} steps" if graph_step is not None
                               else "one call at a time")},
         "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,

@@ -18,11 +18,13 @@ import os
 __all__ = [
     "CobsError", "cobs_dims", "LIB_PATH", "lib",
     "cobs_abi_version", "cobs_stats_record_bytes", "cobs_selected_capacity",
-    "cobs_workspace_bytes", "COBS_STATS_BF16", "COBS_STATS_FP4",
+    "cobs_workspace_bytes", "COBS_STATS_BF16", "COBS_STATS_FP4", "COBS_STATS_BOX",
+    "COBS_STATS_SUBSPACE",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
-    "cobs_read_device_status", "cobs_no_alloc_read_status", "cobs_last_error",
+    "cobs_read_device_status", "cobs_no_alloc_read_status", "cobs_set_wait_limit_ns",
+    "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
     "COBS_ERR_WORKSPACE", "COBS_ERR_CUDA", "COBS_ERR_TIMEOUT", "COBS_ERR_DEVICE",
@@ -40,6 +42,8 @@ COBS_ERR_DEVICE = 6
 
 COBS_STATS_BF16 = 0     # block records: mu and U in bf16
 COBS_STATS_FP4 = 1      # block records: mu in bf16, U in scaled FP4 (E2M1)
+COBS_STATS_BOX = 2      # block records: per-dimension min and max of the keys (bf16)
+COBS_STATS_SUBSPACE = 3  # block records: mu in bf16, U projected on a query subspace (bf16)
 
 
 class CobsError(RuntimeError):
@@ -59,7 +63,9 @@ class cobs_dims(ctypes.Structure):
         ("block_size", ctypes.c_int32),
         ("rank", ctypes.c_int32),
         ("capacity_tokens", ctypes.c_int64),
-        ("stats_format", ctypes.c_int32),       # COBS_STATS_BF16 / COBS_STATS_FP4
+        ("stats_format", ctypes.c_int32),       # COBS_STATS_BF16 / _FP4 / _BOX / _SUBSPACE
+        ("subspace_dim", ctypes.c_int32),       # s of COBS_STATS_SUBSPACE records
+        ("subspace_basis", ctypes.c_void_p),    # device [Hkv][s][d] fp32 basis
     ]
 
 
@@ -90,6 +96,7 @@ def _load() -> ctypes.CDLL:
                                            P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_no_alloc_read_status": (I32, [ctypes.POINTER(I32), P]),
+        "cobs_set_wait_limit_ns": (I32, [ctypes.c_uint64]),
         "cobs_last_error": (ctypes.c_char_p, []),
         "cobs_status_string": (ctypes.c_char_p, [I32]),
     }
@@ -140,6 +147,9 @@ def _check(func: str, status: int, check: bool) -> int:
 def _dims(d) -> cobs_dims:
     if isinstance(d, cobs_dims):
         return d
+    d = dict(d)
+    if d.get("subspace_basis") is not None:
+        d["subspace_basis"] = _ptr(d["subspace_basis"]).value
     return cobs_dims(**d)
 
 
@@ -284,3 +294,9 @@ def cobs_no_alloc_read_status(stream=None) -> int:
     st = lib.cobs_no_alloc_read_status(ctypes.byref(out), _stream(stream))
     _check("cobs_no_alloc_read_status", st, True)
     return out.value
+
+
+def cobs_set_wait_limit_ns(limit_ns: int) -> int:
+    """Limit of the statistics kernel's first bounded device wait (0: the
+    default 2 s); a testing and diagnostic knob."""
+    return _check("cobs_set_wait_limit_ns", lib.cobs_set_wait_limit_ns(int(limit_ns)), True)

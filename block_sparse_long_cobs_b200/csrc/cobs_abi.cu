@@ -1,6 +1,7 @@
 // C ABI of the COBS decode library: argument checks, workspace layout, launch
 // configuration.  Everything that can be checked on the host is checked here,
 // before any CUDA call; kernels never see an invalid shape.
+#include <atomic>
 #include <mutex>
 #include <vector>
 #include <cmath>
@@ -60,12 +61,28 @@ cobs_status check_dims(const cobs_dims* d) {
   const int64_t rows = int64_t(d->batch) * d->num_kv_heads * d->capacity_tokens;
   if (rows >= (int64_t(1) << 31))
     return fail(COBS_ERR_UNSUPPORTED, "batch * num_kv_heads * capacity_tokens must be < 2^31");
-  if (d->stats_format != COBS_STATS_BF16 && d->stats_format != COBS_STATS_FP4)
-    return fail(COBS_ERR_INVALID_ARG, "stats_format must be COBS_STATS_BF16 or COBS_STATS_FP4 (got %d)",
+  if (d->stats_format != COBS_STATS_BF16 && d->stats_format != COBS_STATS_FP4 &&
+      d->stats_format != COBS_STATS_BOX && d->stats_format != COBS_STATS_SUBSPACE)
+    return fail(COBS_ERR_INVALID_ARG,
+                "stats_format must be COBS_STATS_BF16, _FP4, _BOX or _SUBSPACE (got %d)",
                 d->stats_format);
   if (d->stats_format == COBS_STATS_FP4 && d->rank < 1)
     return fail(COBS_ERR_UNSUPPORTED, "FP4 records need rank >= 1");
+  if (d->stats_format == COBS_STATS_SUBSPACE) {
+    if (d->rank < 1) return fail(COBS_ERR_UNSUPPORTED, "subspace records need rank >= 1");
+    if (d->subspace_dim < 1 || d->subspace_dim > d->head_dim)
+      return fail(COBS_ERR_INVALID_ARG, "subspace_dim %d outside [1, head_dim]",
+                  d->subspace_dim);
+    if (!d->subspace_basis || !aligned16(d->subspace_basis))
+      return fail(COBS_ERR_INVALID_ARG,
+                  "subspace records need a 16-byte aligned subspace_basis");
+  }
   return COBS_OK;
+}
+
+int64_t record_bytes(const cobs_dims* d) {
+  return stats_record_bytes(d->head_dim, d->rank, d->stats_format,
+                            d->stats_format == COBS_STATS_SUBSPACE ? d->subspace_dim : 0);
 }
 
 cobs_status check_select_params(int32_t top_k, int32_t sink_blocks, int32_t local_tokens) {
@@ -116,6 +133,15 @@ cobs_status check_ws(void* ws, size_t have, size_t need) {
 }
 
 }  // namespace
+
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{0};   // 0: the default limit
+}  // namespace
+
+uint64_t wait_limit_ns() {
+  const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v == 0 ? kDefaultWaitLimitNs : v;
+}
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -301,11 +327,17 @@ static cobs_status stats_impl(const cobs_dims* dims, const void* k, const int32_
   a.d = dims->head_dim;
   a.rank = dims->rank;
   a.stats_format = dims->stats_format;
-  a.rec_bytes = stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
+  a.rec_bytes = record_bytes(dims);
+  a.basis = dims->stats_format == COBS_STATS_SUBSPACE ? dims->subspace_basis : nullptr;
+  a.sub_dim = dims->stats_format == COBS_STATS_SUBSPACE ? dims->subspace_dim : 0;
+  a.sub_pad = subspace_pad(a.sub_dim);
   a.block_table = block_table;
   a.table_stride = table_stride;
   a.n_pages = n_pages;
-  cudaError_t e = launch_stats(a, static_cast<cudaStream_t>(stream));
+  a.wait_limit_ns = wait_limit_ns();
+  cudaError_t e = dims->stats_format == COBS_STATS_BOX
+                      ? launch_box_records(a, static_cast<cudaStream_t>(stream))
+                      : launch_stats(a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "block statistics launch");
   return ok();
 }
@@ -317,7 +349,7 @@ int32_t cobs_abi_version(void) { return COBS_ABI_VERSION; }
 int64_t cobs_stats_record_bytes(const cobs_dims* dims) {
   if (check_dims(dims) != COBS_OK) return 0;
   ok();
-  return stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
+  return record_bytes(dims);
 }
 
 const char* cobs_last_error(void) { return g_last_error.c_str(); }
@@ -407,7 +439,7 @@ static cobs_status select_impl(const cobs_dims* dims, const void* q, const void*
   // the device): forced sink [0, sink_end), forced local [first_local, nbs)
   const BlockPartition BPm = block_partition(seq_len, sink_blocks, local_tokens);
   const int64_t nbs = BPm.nbs, first_local = BPm.first_local, sink_end = BPm.sink_end;
-  if (!select_topk_fits(dims->head_dim, first_local - sink_end, top_k))
+  if (!select_topk_fits(dims->head_dim, dims->stats_format, first_local - sink_end, top_k))
     return fail(COBS_ERR_UNSUPPORTED,
                 "top_k %d over %lld candidate blocks exceeds the selection kernel's "
                 "shared memory (top_k x candidates / 1024 too large)",
@@ -430,7 +462,10 @@ static cobs_status select_impl(const cobs_dims* dims, const void* q, const void*
   a.d = dims->head_dim;
   a.rank = dims->rank;
   a.stats_format = dims->stats_format;
-  a.rec_bytes = stats_record_bytes(dims->head_dim, dims->rank, dims->stats_format);
+  a.rec_bytes = record_bytes(dims);
+  a.basis = dims->stats_format == COBS_STATS_SUBSPACE ? dims->subspace_basis : nullptr;
+  a.sub_dim = dims->stats_format == COBS_STATS_SUBSPACE ? dims->subspace_dim : 0;
+  a.sub_pad = subspace_pad(a.sub_dim);
   a.idx_stride = idx_stride;
   a.seq_len_blocks = int32_t(nbs);
   a.cand_begin = int32_t(sink_end);
@@ -588,6 +623,11 @@ cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void* q, const
   return decode_impl(dims, q, k_pool, v_pool, block_table, table_stride, n_pages, idx, n_sel,
                      idx_stride, seq_lens, max_seq_len, softmax_scale, out, lse, ws, ws_bytes,
                      stream);
+}
+
+cobs_status cobs_set_wait_limit_ns(uint64_t limit_ns) {
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  return ok();
 }
 
 cobs_status cobs_read_device_status(void* ws, size_t ws_bytes, int32_t* device_status,

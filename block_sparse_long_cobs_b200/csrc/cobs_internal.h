@@ -13,6 +13,7 @@ constexpr int kBlock = 64;     // tokens per KV block
 constexpr int kMaxRank = 16;   // columns of the covariance factor
 constexpr int kMaxGroup = 8;   // query heads per kv-head
 constexpr int kMaxTopK = 4096; // candidates a selection may keep
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;   // bounded device waits: 2 s
 
 // Byte layout of the caller's workspace.  Every region starts 256-aligned.
 struct WorkspaceLayout {
@@ -38,8 +39,10 @@ struct SelectArgs {
   int32_t* status;
   int64_t nb_cap;
   int32_t batch, hq, hkv, d, rank;
-  int32_t stats_format;     // 0 bf16 records, 1 FP4 U
+  int32_t stats_format;     // 0 bf16 records, 1 FP4 U, 2 min/max box, 3 subspace
   int64_t rec_bytes;        // bytes per block record
+  const float* basis;       // subspace records: [Hkv][s][d] fp32 query-subspace basis
+  int32_t sub_dim, sub_pad; // s and its padding to 8
   int32_t idx_stride;
   int32_t seq_len_blocks;   // ceil(seq_len / B)
   int32_t cand_begin, cand_end;  // candidate blocks [begin, end)
@@ -56,29 +59,42 @@ struct SelectArgs {
   int32_t sink_blocks, local_tokens;
 };
 
-// Bytes of one block record: bf16 [1 + r][d], or the FP4 layout (mu bf16,
-// r x d/2 bytes of E2M1 codes, r x d/32 scale exponents, padded to 16).
-__host__ __device__ inline int64_t stats_record_bytes(int d, int r, int fmt) {
+// Columns of a stored subspace row: s rounded up to 8 (16-byte rows).
+__host__ __device__ inline int subspace_pad(int s) { return (s + 7) & ~7; }
+
+// Bytes of one block record: bf16 [1 + r][d], the FP4 layout (mu bf16,
+// r x d/2 bytes of E2M1 codes, r x d/32 scale exponents, padded to 16), a
+// min/max box [lo; hi] of 2 x d bf16, or a subspace record (mu bf16 [d], then
+// r rows of s coordinates in the query subspace, bf16, padded to 8 columns).
+__host__ __device__ inline int64_t stats_record_bytes(int d, int r, int fmt, int s = 0) {
   if (fmt == 0) return int64_t(1 + r) * d * 2;
+  if (fmt == 2) return int64_t(2) * d * 2;
+  if (fmt == 3) return int64_t(2) * d + int64_t(2) * r * subspace_pad(s);
   const int64_t raw = int64_t(2) * d + int64_t(r) * (d / 2) + int64_t(r) * (d / 32);
   return (raw + 15) & ~int64_t(15);
 }
 
 // Selection kernel over FP4 records: per pass, the mu rows of its blocks fill
 // whole 8-row swizzle atoms at the top of a 128-row operand tile and the
-// r U rows of each block follow; the raw records of a pass fit one staging
-// slot of the record ring.  Host and device use the same rule.
-constexpr int kSelFp4RawStages = 5;
-__host__ __device__ inline int fp4_ring_bytes(int d) { return 3 * (d / 64) * 128 * 128; }
-__host__ __device__ inline int fp4_raw_stage_bytes(int d) {
-  return ((fp4_ring_bytes(d) - (d / 64) * 128 * 128) / kSelFp4RawStages) & ~15;
-}
+// r U rows of each block follow; the raw records of a pass fit one slot of
+// the 3-slot raw ring.  Host and device use the same rule.
+constexpr int kSelFp4RawStages = 3;
+__host__ __device__ constexpr int fp4_raw_stage_bytes(int d) { return (d / 64) * 6144; }
 __host__ __device__ inline int fp4_blocks_per_pass(int d, int r) {
   const int64_t rec = stats_record_bytes(d, r, 1);
   int p = 0;
   while (p < 128 && ((p + 1 + 7) / 8) * 8 + (p + 1) * r <= 128 &&
          (p + 1) * rec <= fp4_raw_stage_bytes(d))
     ++p;
+  return p;
+}
+
+// Selection over subspace records: a pass stages nbp blocks in one 128-row
+// tile, their mu rows at the top (whole 8-row swizzle atoms) and their r U_s
+// rows after them.  Host and device use the same rule.
+__host__ __device__ inline int subspace_blocks_per_pass(int r) {
+  int p = 0;
+  while (p < 64 && ((p + 1 + 7) / 8) * 8 + (p + 1) * r <= 128) ++p;
   return p;
 }
 
@@ -149,20 +165,27 @@ struct StatsArgs {
   int64_t nb_cap;
   int64_t block_begin, block_end;
   int32_t batch, hkv, d, rank;
-  int32_t stats_format;   // 0: bf16 [1+r][d] records; 1: mu bf16 + FP4 U
+  int32_t stats_format;   // 0: bf16 [1+r][d] records; 1: mu bf16 + FP4 U; 2: box [lo; hi];
+                          // 3: mu bf16 + U projected on the query subspace
   int64_t rec_bytes;      // bytes per block record
+  const float* basis;     // subspace records: [Hkv][s][d] fp32 query-subspace basis
+  int32_t sub_dim, sub_pad;
   // paged cache: block j of sequence b is page block_table[b * table_stride + j]
   const int32_t* block_table;   // null: contiguous cache
   int32_t table_stride;
   int64_t n_pages;
+  uint64_t wait_limit_ns;       // limit of the kernel's first bounded wait
 };
+
+// Limit of the statistics kernel's first bounded wait (cobs_set_wait_limit_ns).
+uint64_t wait_limit_ns();
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 int select_ctas_per_sm(int d, int g, int rank, int fmt);  // resident selection CTAs per SM
 int select_blocks_per_stage(int d, int rank, int fmt);    // whole records per selection pass
 // Whether the exact top-k of `n_cand` candidates fits the selection kernel's
 // shared memory (its survivors can grow with top_k x n_cand / 1024).
-bool select_topk_fits(int d, int64_t n_cand, int top_k);
+bool select_topk_fits(int d, int fmt, int64_t n_cand, int top_k);
 DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);  // either kernel
 cudaError_t launch_decode_d64(const DecodeArgs& a, cudaStream_t stream);
@@ -170,6 +193,7 @@ int decode_d64_ctas_per_sm(int g);
 cudaError_t launch_decode_tc(const DecodeArgs& a, cudaStream_t stream);
 int decode_tc_ctas_per_sm(int g);
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream);
+cudaError_t launch_box_records(const StatsArgs& a, cudaStream_t stream);
 
 int device_sm_count();
 

@@ -76,25 +76,6 @@ static_assert(kOCol + 32 <= kTmemCols, "TMEM columns");
 // whose release implies that segment n's S = K q^T products have completed.
 static_assert(kStages <= 4, "query double-buffering relies on kStages <= 4");
 
-// Bounded mbarrier wait that also gives up as soon as another role of the CTA
-// has given up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int32_t* status,
-                                              volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        report(status, COBS_ERR_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
 struct Segment {
   int64_t pair;
   int seg;        // index among the pair's chunks (= partial row)

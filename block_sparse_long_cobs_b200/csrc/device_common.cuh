@@ -130,17 +130,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for phase `parity` of `bar` to complete, for at most ~kWaitLimitNs.
 // Returns false (and records COBS_ERR_TIMEOUT) if it never does.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kWaitLimitNs = kDefaultWaitLimitNs;  // 2 s
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  int32_t* status) {
+                                                  int32_t* status,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+    // the clock is read on the first retry and then every 256 tries
+    if ((it == 1 || (it & 255u) == 0) && global_timer_ns() - t0 > limit_ns) {
       report(status, COBS_ERR_TIMEOUT);
       return false;
+    }
+  }
+}
+
+// Bounded mbarrier wait that also gives up as soon as another role of the CTA
+// has given up (and tells the others when it gives up itself).
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, int32_t* status,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        report(status, COBS_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }

@@ -46,6 +46,12 @@ constexpr int kSelThreads = 128;
 constexpr int kSelStages = 3;
 constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
 constexpr int kTopkGroups = 1024; // candidate groups of the top-k bound
+constexpr int kSubStages = 2;     // record ring of the subspace kind
+
+// Bytes of the record ring (which the top-k phase reuses) by record kind.
+__host__ __device__ constexpr int ring_bytes(int d, int fmt) {
+  return (fmt == 3 ? kSubStages : kSelStages) * (d / 64) * 128 * 128;
+}
 
 // Candidates per group of the top-k bound (groups never empty: at most 1024).
 __host__ __device__ constexpr int topk_group_size(int n_cand) {
@@ -106,10 +112,15 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int D, int G, bool kFp4>
-__global__ void __launch_bounds__(kSelThreads)
+// kFmt: 0 bf16 COBS records [mu; U^T], 1 FP4 COBS records, 2 min/max box
+// records [lo; hi], 3 subspace records [mu; U_s^T].
+template <int D, int G, int kFmt>
+__global__ void __launch_bounds__(kFmt == 1 ? 256 : 128, kFmt == 1 ? 2 : 1)
 select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap qmap, const SelectArgs a) {
+  constexpr bool kFp4 = kFmt == 1;
+  constexpr bool kBox = kFmt == 2;
+  constexpr bool kSub = kFmt == 3;
   constexpr int kRegions = D / 64;                  // 64-column slabs of a row
   constexpr int kStageBytes = kRegions * 128 * 128; // 128 rows x 128 B per slab
   constexpr int kQBytes = kRegions * 16 * 128;      // 16 query rows x 128 B per slab
@@ -120,7 +131,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
   const int bh = b * a.hkv + kvh;
-  const int rows = 1 + a.rank;
+  const int rows = kBox ? 2 : 1 + a.rank;          // record rows
   const int per_stage = kStageRows / rows;          // whole records per stage
 
   __shared__ int last_s;
@@ -136,7 +147,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // bf16 records: [kSelStages][kRegions][128][128 B] record ring; FP4 records:
   // an fp16 copy of the queries, then the same number of bytes holding one
   // operand tile and the raw record ring.  Phase 2 reuses the ring either way.
-  uint8_t* stage = base + (kFp4 ? 2 : 1) * kQBytes;
+  uint8_t* stage = base + kQBytes;
 
   float* scores = a.scores_ws + int64_t(bh) * a.nb_cap;
   // this sequence's block partition
@@ -147,19 +158,26 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // ===================== phase 1: scores of this chunk =====================
   if constexpr (kFp4) {
     // FP4 records (COBS explainer §2.3, quantisation): mu bf16 [D] | E2M1
-    // codes [r][D/2] | scale exponents [r][D/32] | padding.  A pass stages the
-    // raw records of per_pass consecutive blocks with one bulk copy, then
-    // every thread widens one row of a 128-row operand tile: the mu rows
-    // (bf16) at rows [0, per_pass), the U rows from row mu_rows =
-    // 8 ceil(per_pass / 8) as fp16 values code x 2^(e_g - E), E the largest
-    // group exponent of that column -- exact in fp16 for e_g - E >= -23 (a
-    // group further below contributes nothing: its components are under
-    // 2^-23 of the column's largest).  Both products read the whole tile from
-    // row 0 -- the bf16 one against the bf16 queries, the fp16 one against an
-    // fp16 copy of them -- and each keeps only its own rows' accumulator
-    // lanes; the epilogue scales a U row's product by 2^E.  Accumulators are
-    // double-buffered: the products of pass p run under the epilogue of
-    // pass p - 1.
+    // codes [r][D/2] | scale exponents [r][D/32] | padding.  256 threads in
+    // two roles that work on different passes at once:
+    //  * warps 0-3 widen: a pass stages the raw records of per_pass
+    //    consecutive blocks with one bulk copy into a 3-slot ring; each thread
+    //    widens one row of the pass's 128-row operand tile (two tiles, used
+    //    in turn): the mu rows (bf16) at rows [0, per_pass), the U rows from
+    //    row mu_rows = 8 ceil(per_pass / 8) as fp16 values code x 2^(e_g - E),
+    //    E the largest group exponent of that column -- exact in fp16 for
+    //    e_g - E >= -23 (a group further below contributes nothing: its
+    //    components are under 2^-23 of the column's largest).  Thread 0 then
+    //    refills the ring and issues the pass's products: the bf16 one
+    //    against the bf16 queries (query-tile rows 0-7) and the fp16 one
+    //    against the fp16 copy of them (rows 8-15), both over the whole tile,
+    //    into one of two tensor-memory accumulators;
+    //  * warps 4-7 read an accumulator back (one lane per thread), keep each
+    //    row's own product (mu rows: bf16 product, columns 0-7; U rows: fp16
+    //    product, columns 8-15, scaled by 2^E) and write the pass's scores.
+    // mbarriers: raw_full (copy landed), mma_done (products complete: the
+    // tile may be rewritten and the accumulator read), acc_free (the
+    // epilogue has read the accumulator).
     constexpr int kRaw = kSelFp4RawStages;
     constexpr int kGroups = D / 32;
     const int r = a.rank;
@@ -167,13 +185,12 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     const int per_pass = fp4_blocks_per_pass(D, r);
     const int mu_rows = (per_pass + 7) & ~7;
     const int raw_bytes = fp4_raw_stage_bytes(D);
-    uint8_t* qtile16 = base + kQBytes;
-    uint8_t* atile = stage;                          // [kRegions][128][128 B]
-    uint8_t* raw = stage + kStageBytes;              // [kRaw][raw_bytes]
+    uint8_t* tiles = stage;                          // [2][kRegions][128][128 B]
+    uint8_t* raw = stage + 2 * kStageBytes;          // [kRaw][raw_bytes]
     __shared__ __align__(8) uint64_t raw_full[kRaw];
-    __shared__ uint32_t colexp_s[2][kStageRows];     // E of each U row, per buffer
-    // this thread's row of the tile: U row (block, column) or mu row (block)
-    const int my_blk = tid / r, my_col = tid - (tid / r) * r;
+    __shared__ __align__(8) uint64_t acc_free[2];
+    __shared__ uint8_t colexp_s[4][kStageRows];      // E of each U row, per pass mod 4
+    __shared__ volatile int abort_s;
 
     const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
     const int c_lo = max(int(BP.sink_end), c_nom);
@@ -185,9 +202,12 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     if (tid == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
       for (int s2 = 0; s2 < kRaw; ++s2) mbar_init(&raw_full[s2], 1);
-      mbar_init(&mma_done[0], 1);
-      mbar_init(&mma_done[1], 1);
+      for (int s2 = 0; s2 < 2; ++s2) {
+        mbar_init(&mma_done[s2], 1);
+        mbar_init(&acc_free[s2], 1);
+      }
       fence_barrier_init();
+      abort_s = 0;
     }
     if (warp == 0) tmem_alloc(&tmem_slot, 64);
     pdl_wait();              // queries and records may come from the launch before
@@ -195,7 +215,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     __syncthreads();
     tc_fence_after();
     pdl_launch_dependents();
-    const uint32_t tmem = tmem_slot;   // buffer b: mu products at 32 b, U at 32 b + 16
+    const uint32_t tmem = tmem_slot;   // buffer b: bf16 products at 32 b, fp16 at 32 b + 16
 
     int n_issued = 0;          // thread 0: passes whose copies were issued
     int n_mma = 0;             // thread 0: passes whose products were issued
@@ -211,50 +231,375 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           tma_load_2d(qtile + reg * 16 * 128, &qmap, reg * 64, b * a.hq + kvh * G, bar);
       bulk_g2s(raw + (p % kRaw) * raw_bytes, recs + int64_t(j0) * rec, bytes, bar);
     };
-    if (tid == 0) {
-      for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
+
+    if (warp < 4) {
+      // ============================ widening ============================
+      const int my_blk = tid / r, my_col = tid - (tid / r) * r;
+      if (tid == 0)
+        for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
+      constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
+      constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
+      for (int p = 0; p < npass; ++p) {
+        const int buf = p & 1, st = p % kRaw;
+        uint8_t* atile = tiles + buf * kStageBytes;
+        // the tile of pass p - 2 is free once its products are complete
+        bool fail = abort_s != 0;
+        if (!fail && p >= 2)
+          fail = !wait_or_abort(&mma_done[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
+        if (!fail) fail = !wait_or_abort(&raw_full[st], (p / kRaw) & 1, a.status, &abort_s);
+        if (named_bar_or(1, 128, fail)) break;
+        const int j0 = c_lo + p * per_pass;
+        const int nb = min(per_pass, c_hi - j0);
+        const uint8_t* rs = raw + st * raw_bytes;
+        if (p == 0) {
+          // the group's 8 query rows as fp16, into rows 8-15 of the query tile
+          for (int c = tid; c < kRegions * 64; c += 128) {
+            const int reg = c >> 6, row = (c >> 3) & 7, ch = c & 7;
+            const uint32_t off = reg * 16 * 128 + row * 128 + ((ch ^ row) << 4);
+            const uint4 w = *reinterpret_cast<const uint4*>(qtile + off);
+            uint4 h;
+            h.x = bf16x2_to_f16x2(w.x);
+            h.y = bf16x2_to_f16x2(w.y);
+            h.z = bf16x2_to_f16x2(w.z);
+            h.w = bf16x2_to_f16x2(w.w);
+            // row 8 + row of the tile has the same swizzle phase as row
+            *reinterpret_cast<uint4*>(qtile + off + 8 * 128) = h;
+          }
+        }
+        // widen this thread's row of the pass into the tile (128-byte swizzle)
+        if (tid < nb * r) {
+          const uint8_t* rp = rs + my_blk * rec;
+          const int row = mu_rows + tid;
+          const uint8_t* sp = rp + 2 * D + r * (D / 2) + my_col * kGroups;
+          const uint32_t sw = kGroups == 4 ? *reinterpret_cast<const uint32_t*>(sp)
+                                           : uint32_t(*reinterpret_cast<const uint16_t*>(sp));
+          uint32_t emax = 0;
+#pragma unroll
+          for (int g = 0; g < kGroups; ++g) emax = max(emax, (sw >> (8 * g)) & 0xFFu);
+          colexp_s[p & 3][row] = uint8_t(emax);
+#pragma unroll
+          for (int gg = 0; gg < kGroups; ++gg) {
+            const int g = (gg + my_col) & (kGroups - 1);   // staggered: fewer bank conflicts
+            const uint32_t eg = (sw >> (8 * g)) & 0xFFu;
+            // fp16 2^(eg - emax): normal for k >= -14, subnormal below; code x 2^k
+            // (a multiple of 2^(k-1)) is an fp16 value for k >= -23, else 0 is used
+            const int k = eg ? int(eg) - int(emax) : -100;
+            const uint32_t mbits = k >= -14 ? uint32_t(k + 15) << 10
+                                            : (k >= -23 ? (1u << (k + 24)) : 0u);
+            const uint32_t mult = mbits | (mbits << 16);
+            const uint4 c4 = *reinterpret_cast<const uint4*>(rp + 2 * D + my_col * (D / 2) + g * 16);
+            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              uint4 hv = e2m1x8_to_f16x8(cw[t]);
+              hv.x = f16x2_mul(hv.x, mult);
+              hv.y = f16x2_mul(hv.y, mult);
+              hv.z = f16x2_mul(hv.z, mult);
+              hv.w = f16x2_mul(hv.w, mult);
+              const int u = 4 * g + t;               // 16-byte unit of the fp16 row
+              *reinterpret_cast<uint4*>(atile + (u >> 3) * (128 * 128) + row * 128 +
+                                        (((u & 7) ^ (row & 7)) << 4)) = hv;
+            }
+          }
+        } else if (tid < nb * r + nb) {
+          const int blk = tid - nb * r;
+          const uint8_t* rp = rs + blk * rec;
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(rp + c * 16);
+            *reinterpret_cast<uint4*>(atile + (c >> 3) * (128 * 128) + blk * 128 +
+                                      (((c & 7) ^ (blk & 7)) << 4)) = w;
+          }
+        }
+        fence_proxy_async_smem();   // generic-proxy tile writes -> tensor-core reads
+        named_bar(1, 128);          // the tile is written, the raw slot read
+        if (tid == 0) {
+          // the raw slot of pass p is free again (its bytes are in the tile)
+          if (p + kRaw < npass) issue(p + kRaw);
+          // the epilogue must have read this accumulator's pass p - 2
+          bool ok = p < 2 || wait_or_abort(&acc_free[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t abase = smem_addr(atile);
+            const uint32_t qb = smem_addr(qtile);
+            const uint32_t acc = tmem + 32u * uint32_t(buf);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+              const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+              umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
+            }
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+              const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+              umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
+            }
+            umma_commit(&mma_done[buf]);
+            n_mma = p + 1;
+          }
+        }
+      }
+      if (tid == 0) {
+        // let the copies and the products still in flight land before TMEM is
+        // freed and the CTA leaves (each wait bounded)
+        for (int p = n_issued > kRaw ? n_issued - kRaw : 0; p < n_issued; ++p)
+          (void)mbar_wait_bounded(&raw_full[p % kRaw], (p / kRaw) & 1, a.status);
+        for (int p = n_mma > 2 ? n_mma - 2 : 0; p < n_mma; ++p)
+          (void)mbar_wait_bounded(&mma_done[p & 1], (p >> 1) & 1, a.status);
+      }
+    } else {
+      // ============================ epilogue ============================
+      const int et = tid - 128;                       // TMEM lane, tile row
+      const float inv_sqrt_d = rsqrtf(float(D));
+      const float ln_n = logf(float(kBlock));
+      for (int p = 0; p < npass; ++p) {
+        const int buf = p & 1;
+        bool fail = abort_s != 0;
+        if (!fail && et == 0)
+          fail = !wait_or_abort(&mma_done[buf], (p >> 1) & 1, a.status, &abort_s);
+        if (named_bar_or(2, 128, fail)) break;
+        if (et != 0) (void)mbar_try_wait(&mma_done[buf], (p >> 1) & 1);
+        tc_fence_after();
+        const int j0 = c_lo + p * per_pass;
+        const int nb = min(per_pass, c_hi - j0);
+        const uint32_t lane_base = tmem + (uint32_t((warp - 4) * 32) << 16) + 32u * uint32_t(buf);
+        uint32_t vm[8], vu[8];
+        tmem_ld8_nowait(lane_base, vm);
+        tmem_ld8_nowait(lane_base + 24u, vu);        // fp16 product, query rows 8-15
+        tmem_wait_ld();
+        tc_fence_before();
+        const bool is_mu = et < mu_rows;
+        const uint32_t eb = colexp_s[p & 3][et];
+        const float col_scale = __uint_as_float(eb << 23);   // 2^(E - 127); 0 for E = 0
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float c;
+          if (is_mu) {
+            c = __uint_as_float(vm[h]) * inv_sqrt_d;
+          } else {
+            const float x = __uint_as_float(vu[h]) * col_scale * inv_sqrt_d;
+            c = 0.5f * x * x;
+          }
+          contrib[et * 8 + h] = c;
+        }
+        named_bar(2, 128);
+        // the accumulator has been read: its next products may start
+        if (et == 0) mbar_arrive(&acc_free[buf]);
+        // per block and head: mu row + its r U rows, then LSE over the heads
+        for (int t0 = 0; t0 < per_pass * G; t0 += 128) {
+          const int t = t0 + et;
+          const int jj = t / G, h = t % G;
+          const bool valid = jj < nb;
+          float sacc = 0.f;
+          if (valid) {
+            sacc = contrib[jj * 8 + h];
+            for (int i = 0; i < r; ++i) sacc += contrib[(mu_rows + jj * r + i) * 8 + h];
+          }
+          const float sh = sacc + ln_n;
+          float mx = sh;
+#pragma unroll
+          for (int m = G / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m, G));
+          float e = __expf(sh - mx);
+#pragma unroll
+          for (int m = G / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m, G);
+          if (valid && h == 0) {
+            const float S = mx + __logf(e);
+            scores[j0 + jj] = S;
+            if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
+          }
+        }
+        named_bar(2, 128);   // contrib is rewritten by the next pass
+      }
     }
+    __threadfence();         // this thread's scores, before the pair's ticket
+    tc_fence_before();
+    __syncthreads();         // every score of the chunk is written
+    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (tid >= kSelThreads) return;   // the top-k below runs on warps 0-3 (named barrier 3)
+  } else if constexpr (kSub) {
+    // Subspace records (COBS explainer §2.3, subspace projection): mu [D]
+    // bf16 | U_s [r][s8] bf16, U_s = P^T U in the coordinates of this
+    // kv-head's query-subspace basis P ([s][D] fp32 rows).  A pass stages nbp
+    // whole records in one 128-row tile: the mu rows (every 64-column slab)
+    // at rows [0, nbp) by a 2-d tensor map over the records, the U_s rows at
+    // rows [nbp_pad, nbp_pad + nbp r) of the first ceil(s8 / 64) slabs by a
+    // 3-d map (coordinate, row of U_s, record) whose columns past s8 read as
+    // zero.  Two products per pass: the mu rows against the bf16 queries
+    // (N = 16) and the U_s rows against q_s = P^T q, computed in fp32 in the
+    // prologue and split into three bf16 parts hi + mid + lo (operand rows h,
+    // 8 + h, 16 + h; N = 32), so the sum of the three products keeps q_s to
+    // fp32 precision.  Accumulators are double-buffered in tensor memory.
+    const int r = a.rank;
+    const int nbp = subspace_blocks_per_pass(r);
+    const int nbp_pad = (nbp + 7) & ~7;
+    const int sreg = (a.sub_pad + 63) >> 6;       // 64-column slabs of a U_s row
+    const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
+    const int c_lo = max(int(BP.sink_end), c_nom);
+    const int c_hi = min(int(BP.first_local), min(a.cand_end, c_nom + a.chunk_blocks));
+    const int npass = c_hi > c_lo ? (c_hi - c_lo + nbp - 1) / nbp : 0;
+    const int rec0 = int(int64_t(bh) * a.nb_cap);  // first record (map row) of this pair
+    // [2 slabs][32 rows][128 B]; it also takes the rows that the U_s product
+    // of the last stage reads past the ring (unread accumulator lanes)
+    uint8_t* qstile = stage + kSubStages * kStageBytes;
+    float* qf = contrib;                           // the group's queries as fp32 [G][D]
+
+    if (tid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
+      for (int s2 = 0; s2 < kSubStages; ++s2) {
+        mbar_init(&full[s2], 1);
+        mbar_init(&mma_done[s2], 1);
+      }
+      fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tmem_slot, 128);
+    pdl_wait();              // queries and records may come from the launch before
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();
+    const uint32_t tmem = tmem_slot;   // buffer b: mu products at 48 b, U_s at 48 b + 16
+
+    // ---- prologue: the bf16 query operand, q as fp32, zeroed q_s operand ----
+    for (int it = tid; it < G * (D / 8); it += kSelThreads) {
+      const int h = it / (D / 8), ch = it % (D / 8);
+      const uint4 w = *reinterpret_cast<const uint4*>(
+          a.q + (int64_t(b) * a.hq + kvh * G + h) * D + ch * 8);
+      *reinterpret_cast<uint4*>(qtile + (ch >> 3) * 16 * 128 + h * 128 +
+                                (((ch & 7) ^ h) << 4)) = w;
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = bf16x2_to_float2(wv[i]);
+        qf[h * D + ch * 8 + 2 * i] = f.x;
+        qf[h * D + ch * 8 + 2 * i + 1] = f.y;
+      }
+    }
+    for (int e = tid; e < 2 * 32 * 128 / 16; e += kSelThreads)
+      reinterpret_cast<uint4*>(qstile)[e] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    // q_s[h][i] = P[i] . q_h in fp32, then hi + mid + lo as bf16 (exact split of
+    // the fp32 value up to the last bits)
+    if (tid < a.sub_dim) {
+      const int i = tid;
+      const float* prow = a.basis + (int64_t(kvh) * a.sub_dim + i) * D;
+      float acc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 4
+      for (int t = 0; t < D; t += 4) {
+        const float4 p4 = __ldg(reinterpret_cast<const float4*>(prow + t));
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float4 q4 = *reinterpret_cast<const float4*>(qf + h * D + t);
+          acc[h] = fmaf(p4.x, q4.x, fmaf(p4.y, q4.y, fmaf(p4.z, q4.z, fmaf(p4.w, q4.w, acc[h]))));
+        }
+      }
+      uint8_t* slab = qstile + (i >> 6) * 32 * 128;
+      const int c = i & 63;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint16_t hi = float_to_bf16_bits(acc[h]);
+        const float r1 = acc[h] - __uint_as_float(uint32_t(hi) << 16);
+        const uint16_t mid = float_to_bf16_bits(r1);
+        const uint16_t lo = float_to_bf16_bits(r1 - __uint_as_float(uint32_t(mid) << 16));
+        *reinterpret_cast<uint16_t*>(slab + sw128_offset(h, c)) = hi;
+        *reinterpret_cast<uint16_t*>(slab + sw128_offset(8 + h, c)) = mid;
+        *reinterpret_cast<uint16_t*>(slab + sw128_offset(16 + h, c)) = lo;
+      }
+    }
+    fence_proxy_async_smem();   // generic-proxy operand writes -> tensor-core reads
+    __syncthreads();
+
+    int n_issued = 0, n_mma = 0;   // thread 0 only
+    auto issue = [&](int p) {      // thread 0 only: the records of pass p
+      n_issued = p + 1;
+      const int st = p % kSubStages;
+      const int j0 = c_lo + p * nbp;
+      uint8_t* dst = stage + st * kStageBytes;
+      // the boxes are always nbp records; records past the chunk are ignored
+      mbar_arrive_expect_tx(&full[st], uint32_t(kRegions + sreg * r) * uint32_t(nbp) * 128u);
+      for (int reg = 0; reg < kRegions; ++reg)
+        tma_load_2d(dst + reg * 128 * 128, &smap, reg * 64, rec0 + j0, &full[st]);
+      for (int reg = 0; reg < sreg; ++reg)
+        tma_load_3d(dst + reg * 128 * 128 + nbp_pad * 128, &qmap, reg * 64, 0, rec0 + j0,
+                    &full[st]);
+    };
+    if (tid == 0)
+      for (int p = 0; p < kSubStages && p < npass; ++p) issue(p);
 
     const float inv_sqrt_d = rsqrtf(float(D));
     const float ln_n = logf(float(kBlock));
-    constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
-    constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
-
-    // scores of pass pe from accumulator buffer pe & 1 (its products are complete)
-    auto epilogue = [&](int pe) {
-      const int j0 = c_lo + pe * per_pass;
-      const int nb = min(per_pass, c_hi - j0);
-      const int row = warp * 32 + lane;
-      const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 32u * uint32_t(pe & 1);
-      uint32_t vm[8], vu[8];
-      tmem_ld8_nowait(lane_base, vm);
-      tmem_ld8_nowait(lane_base + 16u, vu);
+    constexpr uint32_t idesc_mu = umma_idesc_bf16(128, 16);
+    constexpr uint32_t idesc_us = umma_idesc_bf16(128, 32);
+    auto issue_mma = [&](int p) -> bool {   // thread 0 only
+      const int st = p % kSubStages;
+      if (!mbar_wait_bounded(&full[st], (p / kSubStages) & 1, a.status)) return false;
+      tc_fence_after();
+      const uint32_t abase = smem_addr(stage + st * kStageBytes);
+      const uint32_t qb = smem_addr(qtile), qsb = smem_addr(qstile);
+      const uint32_t acc = tmem + 48u * uint32_t(p & 1);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+        const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+        umma_bf16(acc, ad, bd, idesc_mu, ks > 0 ? 1u : 0u);
+      }
+      for (int ks = 0; ks < 4 * sreg; ++ks) {
+        const uint64_t ad =
+            umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + nbp_pad * 128 + (ks & 3) * 32);
+        const uint64_t bd = umma_desc_sw128(qsb + (ks >> 2) * 32 * 128 + (ks & 3) * 32);
+        umma_bf16(acc + 16u, ad, bd, idesc_us, ks > 0 ? 1u : 0u);
+      }
+      umma_commit(&mma_done[st]);
+      n_mma = p + 1;
+      return true;
+    };
+    bool fail = false;
+    if (tid == 0 && npass > 0 && !issue_mma(0)) fail = true;
+    const int urows = nbp * r;
+    for (int p = 0; p < npass; ++p) {
+      const int st = p % kSubStages;
+      const uint32_t parity = (p / kSubStages) & 1;
+      if (tid == 0 && !fail && !mbar_wait_bounded(&mma_done[st], parity, a.status)) fail = true;
+      if (__syncthreads_or(fail)) break;
+      if (tid != 0) (void)mbar_try_wait(&mma_done[st], parity);
+      tc_fence_after();
+      if (tid == 0) {
+        if (p + kSubStages < npass) issue(p + kSubStages);
+        if (p + 1 < npass && !issue_mma(p + 1)) fail = true;
+      }
+      // epilogue: lane t of the accumulators = mu row t and U_s row t
+      const int j0 = c_lo + p * nbp;
+      const int nb = min(nbp, c_hi - j0);
+      const uint32_t acc = tmem + (uint32_t(warp * 32) << 16) + 48u * uint32_t(p & 1);
+      uint32_t vm[8], vu[8], vmid[8], vlo[8];
+      tmem_ld8_nowait(acc, vm);
+      tmem_ld8_nowait(acc + 16u, vu);
+      tmem_ld8_nowait(acc + 24u, vmid);
+      tmem_ld8_nowait(acc + 32u, vlo);
       tmem_wait_ld();
-      const bool is_mu = row < mu_rows;
-      const uint32_t eb = colexp_s[pe & 1][row];
-      const float col_scale = __uint_as_float(eb << 23);   // 2^(E - 127); 0 for E = 0
+      const int t = tid;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float c;
-        if (is_mu) {
-          c = __uint_as_float(vm[h]) * inv_sqrt_d;
-        } else {
-          const float x = __uint_as_float(vu[h]) * col_scale * inv_sqrt_d;
-          c = 0.5f * x * x;
+        if (t < nbp) contrib[(urows + t) * 8 + h] = __uint_as_float(vm[h]) * inv_sqrt_d;
+        if (t < urows) {
+          const float x = (__uint_as_float(vu[h]) + __uint_as_float(vmid[h]) +
+                           __uint_as_float(vlo[h])) * inv_sqrt_d;
+          contrib[t * 8 + h] = 0.5f * x * x;
         }
-        contrib[row * 8 + h] = c;
       }
       tc_fence_before();
       __syncthreads();
-      // per block and head: mu row + its r U rows, then LSE over the heads
-      for (int t0 = 0; t0 < per_pass * G; t0 += kSelThreads) {
-        const int t = t0 + tid;
-        const int jj = t / G, h = t % G;
+      for (int t0 = 0; t0 < nbp * G; t0 += kSelThreads) {
+        const int tt = t0 + tid;
+        const int jj = tt / G, h = tt % G;
         const bool valid = jj < nb;
         float sacc = 0.f;
         if (valid) {
-          sacc = contrib[jj * 8 + h];
-          for (int i = 0; i < r; ++i) sacc += contrib[(mu_rows + jj * r + i) * 8 + h];
+          sacc = contrib[(urows + jj) * 8 + h];
+          for (int i = 0; i < r; ++i) sacc += contrib[(jj * r + i) * 8 + h];
         }
         const float sh = sacc + ln_n;
         float mx = sh;
@@ -269,131 +614,18 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
         }
       }
-      __syncthreads();   // contrib reused by the next epilogue
-    };
-
-    bool fail = false;
-    for (int p = 0; p < npass; ++p) {
-      const int st = p % kRaw;
-      const uint32_t parity = (p / kRaw) & 1;
-      // the tile is free once the products of pass p - 1 are complete
-      if (tid == 0 && p >= 1 &&
-          !mbar_wait_bounded(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1, a.status))
-        fail = true;
-      if (tid == 0 && !fail && !mbar_wait_bounded(&raw_full[st], parity, a.status)) fail = true;
-      if (__syncthreads_or(fail)) break;
-      if (tid != 0) {
-        (void)mbar_try_wait(&raw_full[st], parity);
-        if (p >= 1) (void)mbar_try_wait(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1);
-      }
-      tc_fence_after();
-      const int j0 = c_lo + p * per_pass;
-      const int nb = min(per_pass, c_hi - j0);
-      const uint8_t* rs = raw + st * raw_bytes;
-      if (p == 0) {
-        // the group's 8 query rows as fp16, at the same byte positions
-        for (int c = tid; c < kRegions * 64; c += kSelThreads) {
-          const int off = (c >> 6) * 16 * 128 + (c & 63) * 16;
-          const uint4 w = *reinterpret_cast<const uint4*>(qtile + off);
-          uint4 h;
-          h.x = bf16x2_to_f16x2(w.x);
-          h.y = bf16x2_to_f16x2(w.y);
-          h.z = bf16x2_to_f16x2(w.z);
-          h.w = bf16x2_to_f16x2(w.w);
-          *reinterpret_cast<uint4*>(qtile16 + off) = h;
-        }
-      }
-      // widen this thread's row of the pass into the tile (128-byte swizzle)
-      if (tid < nb * r) {
-        const uint8_t* rp = rs + my_blk * rec;
-        const int row = mu_rows + tid;
-        const uint8_t* sp = rp + 2 * D + r * (D / 2) + my_col * kGroups;
-        const uint32_t sw = kGroups == 4 ? *reinterpret_cast<const uint32_t*>(sp)
-                                         : uint32_t(*reinterpret_cast<const uint16_t*>(sp));
-        uint32_t emax = 0;
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g) emax = max(emax, (sw >> (8 * g)) & 0xFFu);
-        colexp_s[p & 1][row] = emax;
-#pragma unroll
-        for (int gg = 0; gg < kGroups; ++gg) {
-          const int g = (gg + my_col) & (kGroups - 1);   // staggered: fewer bank conflicts
-          const uint32_t eg = (sw >> (8 * g)) & 0xFFu;
-          // fp16 2^(eg - emax): normal for k >= -14, subnormal below; code x 2^k
-          // (a multiple of 2^(k-1)) is an fp16 value for k >= -23, else 0 is used
-          const int k = eg ? int(eg) - int(emax) : -100;
-          const uint32_t mbits = k >= -14 ? uint32_t(k + 15) << 10
-                                          : (k >= -23 ? (1u << (k + 24)) : 0u);
-          const uint32_t mult = mbits | (mbits << 16);
-          const uint4 c4 = *reinterpret_cast<const uint4*>(rp + 2 * D + my_col * (D / 2) + g * 16);
-          const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            uint4 hv = e2m1x8_to_f16x8(cw[t]);
-            hv.x = f16x2_mul(hv.x, mult);
-            hv.y = f16x2_mul(hv.y, mult);
-            hv.z = f16x2_mul(hv.z, mult);
-            hv.w = f16x2_mul(hv.w, mult);
-            const int u = 4 * g + t;               // 16-byte unit of the fp16 row
-            *reinterpret_cast<uint4*>(atile + (u >> 3) * (128 * 128) + row * 128 +
-                                      (((u & 7) ^ (row & 7)) << 4)) = hv;
-          }
-        }
-      } else if (tid < nb * r + nb) {
-        const int blk = tid - nb * r;
-        const uint8_t* rp = rs + blk * rec;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(rp + c * 16);
-          *reinterpret_cast<uint4*>(atile + (c >> 3) * (128 * 128) + blk * 128 +
-                                    (((c & 7) ^ (blk & 7)) << 4)) = w;
-        }
-      }
-      fence_proxy_async_smem();   // generic-proxy tile writes -> tensor-core reads
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t abase = smem_addr(atile);
-        const uint32_t qb = smem_addr(qtile), qh = smem_addr(qtile16);
-        const uint32_t acc = tmem + 32u * uint32_t(p & 1);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
-          const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-          umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
-          const uint64_t bd = umma_desc_sw128(qh + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-          umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&mma_done[p & 1]);
-        n_mma = p + 1;
-        // the raw slot of pass p is free again (its bytes are in the tile)
-        if (p + kRaw < npass) issue(p + kRaw);
-      }
-      if (p >= 1) epilogue(p - 1);
-    }
-    if (!fail && npass > 0) {
-      const int pl = npass - 1;
-      if (tid == 0 && !mbar_wait_bounded(&mma_done[pl & 1], (pl >> 1) & 1, a.status)) fail = true;
-      if (!__syncthreads_or(fail)) {
-        if (tid != 0) (void)mbar_try_wait(&mma_done[pl & 1], (pl >> 1) & 1);
-        tc_fence_after();
-        epilogue(pl);
-      }
+      __syncthreads();   // contrib and the accumulator reused next pass
     }
     if (tid == 0 && fail) {
-      // let the copies and the products still in flight land before TMEM is
-      // freed and the CTA leaves (each wait bounded)
-      for (int p = n_issued > kRaw ? n_issued - kRaw : 0; p < n_issued; ++p)
-        (void)mbar_wait_bounded(&raw_full[p % kRaw], (p / kRaw) & 1, a.status);
-      for (int p = n_mma > 2 ? n_mma - 2 : 0; p < n_mma; ++p)
-        (void)mbar_wait_bounded(&mma_done[p & 1], (p >> 1) & 1, a.status);
+      for (int p = n_issued > kSubStages ? n_issued - kSubStages : 0; p < n_issued; ++p)
+        (void)mbar_wait_bounded(&full[p % kSubStages], (p / kSubStages) & 1, a.status);
+      if (n_mma > 0)
+        (void)mbar_wait_bounded(&mma_done[(n_mma - 1) % kSubStages],
+                                ((n_mma - 1) / kSubStages) & 1, a.status);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, 128);
   } else {
     // this chunk's share of the candidates of a max_seq_len sequence, cut to
     // this sequence's own candidates [sink_end, first_local)
@@ -419,6 +651,33 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     tc_fence_after();
     pdl_launch_dependents();
     const uint32_t tmem = tmem_slot;
+    if constexpr (kBox) {
+      // the box score needs the signed parts of the queries: operand rows
+      // 0..G-1 hold q+ = max(q, 0), rows 8..8+G-1 hold q- = min(q, 0), so that
+      // the product of a record [lo; hi] gives hi.q+ and lo.q- (exact products
+      // of bf16 values, fp32 sums); rows past the group feed columns nobody
+      // reads
+      for (int it = tid; it < G * (D / 8); it += kSelThreads) {
+        const int h = it / (D / 8), ch = it % (D / 8);
+        const uint4 w = *reinterpret_cast<const uint4*>(
+            a.q + (int64_t(b) * a.hq + kvh * G + h) * D + ch * 8);
+        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+        uint32_t pos[4], neg[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t m = ((wv[i] >> 15) & 0x00010001u) * 0xFFFFu;   // negative halves
+          neg[i] = wv[i] & m;
+          pos[i] = wv[i] & ~m;
+        }
+        uint8_t* reg = qtile + (ch >> 3) * 16 * 128;
+        const uint32_t cs = uint32_t(((ch & 7) ^ h) << 4);
+        *reinterpret_cast<uint4*>(reg + h * 128 + cs) = make_uint4(pos[0], pos[1], pos[2], pos[3]);
+        *reinterpret_cast<uint4*>(reg + (8 + h) * 128 + cs) =
+            make_uint4(neg[0], neg[1], neg[2], neg[3]);
+      }
+      fence_proxy_async_smem();   // generic-proxy writes -> tensor-core reads
+      __syncthreads();
+    }
 
     int n_issued = 0;          // thread 0: passes whose TMA copies were issued
     int n_mma = 0;             // thread 0: passes whose MMA was issued
@@ -431,8 +690,8 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       // Pass 0 also brings the group's 8 query rows (rows past the group and
       // rows 8..15 of the operand only feed accumulator columns nobody reads)
       mbar_arrive_expect_tx(&full[p % kSelStages],
-                            uint32_t(kRegions) * (kStageRows + (p == 0 ? 8 : 0)) * 128);
-      if (p == 0)
+                            uint32_t(kRegions) * (kStageRows + (p == 0 && !kBox ? 8 : 0)) * 128);
+      if (p == 0 && !kBox)
         for (int reg = 0; reg < kRegions; ++reg)
           tma_load_2d(qtile + reg * 16 * 128, &qmap, reg * 64, b * a.hq + kvh * G, &full[0]);
       for (int reg = 0; reg < kRegions; ++reg)
@@ -495,8 +754,13 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       const int rho = row % rows;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float x = v[h] * inv_sqrt_d;
-        contrib[row * 8 + h] = (rho == 0) ? x : 0.5f * x * x;
+        if constexpr (kBox) {
+          // record row 0 (lo) pairs with q-, row 1 (hi) with q+
+          contrib[row * 8 + h] = (rho == 0 ? v[8 + h] : v[h]) * inv_sqrt_d;
+        } else {
+          const float x = v[h] * inv_sqrt_d;
+          contrib[row * 8 + h] = (rho == 0) ? x : 0.5f * x * x;
+        }
       }
       tc_fence_before();
       __syncthreads();
@@ -542,16 +806,16 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // (a pair scored by one CTA needs no ticket: its scores are this CTA's own)
   if (a.n_chunks > 1) {
     __threadfence();
-    __syncthreads();
+    named_bar(3, kSelThreads);
     if (tid == 0) {
       const uint32_t prev = atomicAdd(&a.tickets[bh], 1u);
       last_s = (prev == uint32_t(a.n_chunks - 1));
     }
-    __syncthreads();
+    named_bar(3, kSelThreads);
     if (!last_s) return;
     __threadfence();
   } else {
-    __syncthreads();   // every score of the pair is written
+    named_bar(3, kSelThreads);   // every score of the pair is written
   }
 
   const int c0 = int(BP.sink_end), c1 = int(BP.first_local);
@@ -576,7 +840,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   uint64_t* gmax = reinterpret_cast<uint64_t*>(stage);                 // [ng]
   uint64_t* tmax = gmax + ng;                                          // [128]
   uint64_t* surv = tmax + kSelThreads;                                 // survivors
-  const int surv_cap = topk_survivor_capacity(kSelStages * kStageBytes, n_cand);
+  const int surv_cap = topk_survivor_capacity(ring_bytes(D, kFmt), n_cand);
   uint8_t* chosen_s = reinterpret_cast<uint8_t*>(surv + (surv_cap > 0 ? surv_cap : 0));
   auto key64 = [&](int jj) -> uint64_t {
     return (uint64_t(order_key(__ldcg(scores + c0 + jj))) << 32) |
@@ -602,7 +866,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       last_s = 0;   // survivor count
       tau_s = 0ull;
     }
-    __syncthreads();
+    named_bar(3, kSelThreads);
     // tau1: the k-th largest thread maximum (thread maxima are distinct or 0;
     // at least min(ng, 128) > k of them are non-zero when k < 128)
     if (k < kSelThreads) {
@@ -610,7 +874,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       for (int u = 0; u < kSelThreads; ++u) rank += tmax[u] > mine;
       if (mine != 0 && rank == k - 1) tau_s = mine;
     }
-    __syncthreads();
+    named_bar(3, kSelThreads);
     const uint64_t tau1 = tau_s;
     for (int g = tid; g < ng; g += kSelThreads) {
       if (gmax[g] >= tau1) {
@@ -618,7 +882,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         if (slot < surv_cap) surv[slot] = gmax[g];
       }
     }
-    __syncthreads();
+    named_bar(3, kSelThreads);
     const int ns1 = last_s < surv_cap ? last_s : surv_cap;
     if (gs == 1) {
       // groups are single candidates: the survivors are the candidate keys
@@ -630,7 +894,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         for (int u = 0; u < ns1; ++u) rank += surv[u] > c;
         if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
       }
-      __syncthreads();
+      named_bar(3, kSelThreads);
     } else {
       // tau2: the k-th largest group maximum (0 when there are fewer than k groups)
       if (k <= ng) {
@@ -643,10 +907,10 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       } else if (tid == 0) {
         tau_s = 0ull;
       }
-      __syncthreads();
+      named_bar(3, kSelThreads);
       const uint64_t tau2 = tau_s;
       if (tid == 0) last_s = 0;
-      __syncthreads();
+      named_bar(3, kSelThreads);
       for (int jj = tid; jj < n_cand; jj += kSelThreads) {
         const uint64_t c = key64(jj);
         if (c >= tau2) {
@@ -654,7 +918,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           if (slot < surv_cap) surv[slot] = c;
         }
       }
-      __syncthreads();
+      named_bar(3, kSelThreads);
       const int ns = last_s < surv_cap ? last_s : surv_cap;
       if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
       for (int i = tid; i < ns; i += kSelThreads) {
@@ -663,7 +927,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         for (int u = 0; u < ns; ++u) rank += surv[u] > c;
         if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
       }
-      __syncthreads();
+      named_bar(3, kSelThreads);
     }
   } else if (partial && tid == 0) {
     report(a.status, COBS_ERR_DEVICE);   // host limits prevent this
@@ -702,16 +966,24 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   }
 }
 
-template <int D, bool kFp4>
+template <int D, int kFmt>
 constexpr size_t dyn_smem_bytes() {
-  return 1024 + size_t(kFp4 ? 2 : 1) * (D / 64) * 16 * 128 +
-         size_t(kSelStages) * (D / 64) * 128 * 128;
+  // query tile + record ring (FP4: two operand tiles and the raw ring) +
+  // the subspace query operand
+  return 1024 + size_t(D / 64) * 16 * 128 +
+         (kFmt == 1 ? size_t(2) * (D / 64) * 128 * 128 + size_t(kSelFp4RawStages) *
+                                                             fp4_raw_stage_bytes(D)
+                    : size_t(ring_bytes(D, kFmt))) +
+         (kFmt == 3 ? size_t(2) * 32 * 128 : 0);
 }
+template <int kFmt>
+constexpr int sel_threads() { return kFmt == 1 ? 2 * kSelThreads : kSelThreads; }
 
-template <int D, int G, bool kFp4>
+template <int D, int G, int kFmt>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
-  auto kern = select_blocks_kernel<D, G, kFp4>;
-  constexpr size_t smem = dyn_smem_bytes<D, kFp4>();
+  constexpr bool kFp4 = kFmt == 1;
+  auto kern = select_blocks_kernel<D, G, kFmt>;
+  constexpr size_t smem = dyn_smem_bytes<D, kFmt>();
   cudaError_t e = set_smem_attrs(kern, int(smem));
   if (e != cudaSuccess) return e;
   CUtensorMap map, qmap;
@@ -719,63 +991,90 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (kFp4) {
     map = qmap;   // FP4 records arrive by plain bulk copies; the map is unused
+  } else if (kFmt == 3) {
+    // mu rows: the first D columns of every record; U_s rows: (coordinate,
+    // row, record) starting 2 D bytes into the records
+    const uint64_t n_rec = uint64_t(a.batch) * a.hkv * a.nb_cap;
+    const int nbp = subspace_blocks_per_pass(a.rank);
+    e = make_bf16_tensor_map_rows_sw128(&map, a.stats, D, n_rec, uint64_t(a.rec_bytes), nbp);
+    if (e != cudaSuccess) return e;
+    e = make_bf16_tensor_map_3d_sw128_box(&qmap, reinterpret_cast<const uint8_t*>(a.stats) + 2 * D,
+                                          a.sub_pad, uint64_t(a.rank), n_rec,
+                                          uint64_t(a.sub_pad) * 2, uint64_t(a.rec_bytes),
+                                          a.rank, nbp);
+    if (e != cudaSuccess) return e;
   } else {
-    const uint64_t total_rows = uint64_t(a.batch) * a.hkv * a.nb_cap * (1 + a.rank);
+    const uint64_t total_rows =
+        uint64_t(a.batch) * a.hkv * a.nb_cap * (kFmt == 2 ? 2 : 1 + a.rank);
     e = make_bf16_tensor_map_sw128(&map, a.stats, D, total_rows, kStageRows);
     if (e != cudaSuccess) return e;
   }
   dim3 grid(a.n_chunks, a.hkv, a.batch);
-  return launch_pdl(kern, grid, dim3(kSelThreads), smem, s, map, qmap, a);
+  return launch_pdl(kern, grid, dim3(sel_threads<kFmt>()), smem, s, map, qmap, a);
 }
 
-template <int D, int G, bool kFp4>
+template <int D, int G, int kFmt>
 int occupancy_t() {
-  return kernel_occupancy(reinterpret_cast<const void*>(select_blocks_kernel<D, G, kFp4>),
-                          kSelThreads, int(dyn_smem_bytes<D, kFp4>()));
+  return kernel_occupancy(reinterpret_cast<const void*>(select_blocks_kernel<D, G, kFmt>),
+                          sel_threads<kFmt>(), int(dyn_smem_bytes<D, kFmt>()));
 }
 
-template <int D, bool kFp4>
+template <int D, int kFmt>
 cudaError_t dispatch_group(const SelectArgs& a, cudaStream_t s) {
   switch (a.hq / a.hkv) {
-    case 1: return launch_t<D, 1, kFp4>(a, s);
-    case 2: return launch_t<D, 2, kFp4>(a, s);
-    case 4: return launch_t<D, 4, kFp4>(a, s);
-    case 8: return launch_t<D, 8, kFp4>(a, s);
+    case 1: return launch_t<D, 1, kFmt>(a, s);
+    case 2: return launch_t<D, 2, kFmt>(a, s);
+    case 4: return launch_t<D, 4, kFmt>(a, s);
+    case 8: return launch_t<D, 8, kFmt>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int D, bool kFp4>
+template <int D, int kFmt>
 int occupancy_group(int g) {
   switch (g) {
-    case 1: return occupancy_t<D, 1, kFp4>();
-    case 2: return occupancy_t<D, 2, kFp4>();
-    case 4: return occupancy_t<D, 4, kFp4>();
-    default: return occupancy_t<D, 8, kFp4>();
+    case 1: return occupancy_t<D, 1, kFmt>();
+    case 2: return occupancy_t<D, 2, kFmt>();
+    case 4: return occupancy_t<D, 4, kFmt>();
+    default: return occupancy_t<D, 8, kFmt>();
   }
+}
+
+template <int kFmt>
+cudaError_t dispatch_dim(const SelectArgs& a, cudaStream_t s) {
+  return a.d == 64 ? dispatch_group<64, kFmt>(a, s) : dispatch_group<128, kFmt>(a, s);
 }
 
 }  // namespace
 
 int select_ctas_per_sm(int d, int g, int /*rank*/, int fmt) {
-  if (fmt != 0) return d == 64 ? occupancy_group<64, true>(g) : occupancy_group<128, true>(g);
-  return d == 64 ? occupancy_group<64, false>(g) : occupancy_group<128, false>(g);
+  switch (fmt) {
+    case 1: return d == 64 ? occupancy_group<64, 1>(g) : occupancy_group<128, 1>(g);
+    case 2: return d == 64 ? occupancy_group<64, 2>(g) : occupancy_group<128, 2>(g);
+    case 3: return d == 64 ? occupancy_group<64, 3>(g) : occupancy_group<128, 3>(g);
+    default: return d == 64 ? occupancy_group<64, 0>(g) : occupancy_group<128, 0>(g);
+  }
 }
 
 int select_blocks_per_stage(int d, int rank, int fmt) {
-  return fmt != 0 ? fp4_blocks_per_pass(d, rank) : kStageRows / (1 + rank);
+  if (fmt == 1) return fp4_blocks_per_pass(d, rank);
+  if (fmt == 3) return subspace_blocks_per_pass(rank);
+  return kStageRows / (fmt == 2 ? 2 : 1 + rank);
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
-  if (a.stats_format != 0)
-    return a.d == 64 ? dispatch_group<64, true>(a, stream) : dispatch_group<128, true>(a, stream);
-  return a.d == 64 ? dispatch_group<64, false>(a, stream) : dispatch_group<128, false>(a, stream);
+  switch (a.stats_format) {
+    case 1: return dispatch_dim<1>(a, stream);
+    case 2: return dispatch_dim<2>(a, stream);
+    case 3: return dispatch_dim<3>(a, stream);
+    default: return dispatch_dim<0>(a, stream);
+  }
 }
 
-bool select_topk_fits(int d, int64_t n_cand, int top_k) {
+bool select_topk_fits(int d, int fmt, int64_t n_cand, int top_k) {
   if (top_k <= 0 || top_k >= n_cand) return true;   // no ranking needed
   if (n_cand > (int64_t(1) << 24)) return false;
-  const int ring = kSelStages * (d / 64) * 128 * 128;
+  const int ring = ring_bytes(d, fmt);
   return topk_survivor_capacity(ring, int(n_cand)) >= topk_survivors_needed(int(n_cand), top_k);
 }
 

@@ -7,36 +7,37 @@
 // block means are stored in BF16.
 //
 // Method used on the GPU (same result as the eigen-decomposition of the d x d
-// covariance, computed through the n x n Gram matrix because n = B = 64 < d):
-//   1. Raw Gram G = K K^T of the block's bf16 keys on the 5th-generation tensor
-//      cores: one tcgen05.mma chain (kind::f16, M = 128, N = 64, bf16 in, fp32
-//      accumulate in tensor memory); rows 0-63 of the A tile hold the block,
-//      rows 64-127 are never read back.  Products of bf16 values are exact, so
-//      no precision is lost before the fp32 accumulation.  The keys arrive by
-//      TMA (2-d tensor map, 128-byte swizzle = the UMMA K-major canonical
-//      layout).  One block per CTA of 128 threads with a small shared-memory
-//      footprint (the key tile's space is reused for the Lanczos basis and U
-//      re-reads the keys through L2), so the kernel can share SMs with the
-//      selection and decode kernels when it runs on a side stream.
-//   2. Centring in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
-//      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T; then
-//      A = Gc^2 (same eigenvectors, squared eigenvalues: the top of the
-//      spectrum separates faster, so fewer Lanczos steps are needed).
-//   3. Lanczos tridiagonalisation of A, m = 28 / 36 / 52 steps for r <= 4 /
-//      <= 8 / <= 16 (at least 2 r + 20), every new vector re-orthogonalised
-//      twice against all earlier ones by classical Gram-Schmidt (basis kept
-//      row- and column-major in shared memory so both Gram-Schmidt phases are
-//      128-bit loads), a fresh pseudo-random vector whenever the Krylov space
-//      closes.  Each thread holds 32 entries of A in registers; five barrier
-//      phases per step, norms reduced through those same barriers.
-//   4. Top-r eigenvalues of the m x m tridiagonal T by multisection bisection
-//      on Sturm counts (8 threads x 3 shifts per eigenvalue, 25-way splits),
-//      eigenvectors z_k by inverse iteration (LDL^T of T - theta I, all in
+// covariance, computed through the n x n Gram matrix because n = B = 64 < d).
+// A CTA of four warps takes four block-heads, one warp per block-head:
+//   1. TMA brings the four blocks' keys (2-d tensor map, 128-byte swizzle =
+//      the UMMA K-major canonical layout) into two 128-row tiles, two blocks
+//      per tile.  One tcgen05.mma chain per tile (kind::f16, M = N = 128,
+//      bf16 in, fp32 accumulate in tensor memory) forms [K_a; K_b][K_a; K_b]^T,
+//      whose diagonal 64 x 64 quadrants are the raw Grams G = K K^T of the two
+//      blocks (products of bf16 values are exact in fp32).  The block means
+//      are summed from the tiles meanwhile.
+//   2. The Gram rows come back from tensor memory (each warp reads its 32
+//      lanes), go through shared memory to the warp that owns the block, and
+//      are centred in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
+//      s = 1^T G 1 / n^2, i.e. Gc = Kc Kc^T with Kc = K - 1 mu^T.  Lane l keeps
+//      rows l and l + 32 of Gc in registers.
+//   3. Lanczos on A = Gc^2 (applied as two products with Gc; same eigenvectors,
+//      squared eigenvalues, so the top of the spectrum separates faster), M =
+//      24 / 32 / 44 steps for r <= 4 / <= 8 / <= 16, every new vector
+//      orthogonalised twice against all earlier ones by classical
+//      Gram-Schmidt, a fresh pseudo-random vector whenever the Krylov space
+//      closes.  The warp works alone: its only synchronisation is __syncwarp,
+//      vectors pass through its own shared-memory rows (basis kept row- and
+//      column-major so both Gram-Schmidt phases are 128-bit loads).
+//   4. Top-r eigenvalues of the M x M tridiagonal T by multisection bisection
+//      on Sturm counts (the lanes split among the r eigenvalues, three shifts
+//      each), eigenvectors z_k by inverse iteration (LDL^T of T - theta I, in
 //      registers), re-orthogonalised inside clusters of close eigenvalues;
 //      Ritz vectors w_k = Q z_k are unit eigenvectors of Gc.
 //   5. U[:, k] = Kc^T w_k / sqrt(n) (its squared norm is the covariance
-//      eigenvalue), sign fixed so that the largest-magnitude component is
-//      positive; written with mu as bf16.
+//      eigenvalue), keys re-read through L2 (lane l owns d/32 consecutive
+//      dimensions), sign fixed so that the largest-magnitude component is
+//      positive; written with mu as a bf16 or an FP4 record.
 #include <cfloat>
 #include <cuda.h>
 
@@ -46,49 +47,56 @@
 namespace cobs {
 namespace {
 
-constexpr int kStatThreads = 128;   // one block per CTA
-constexpr int kQStride = 72;        // floats per basis row: halves of 36
-constexpr int kGStride = 68;        // 16-byte aligned row of the staged Grams
-constexpr int kBisectRounds = 5;    // 25-way splits: 25^5 ~ 1e7
+constexpr int kStatWarps = 4;                 // block-heads per CTA, one per warp
+constexpr int kStatThreads = 32 * kStatWarps;
+constexpr int kQStride = 68;                  // floats per row-major basis row
+constexpr int kGStride = 68;                  // floats per staged Gram row
 constexpr int kInverseIters = 2;
+constexpr int kTmemCols = 256;                // two 128 x 128 Gram tiles
 
-// Lanczos length by rank bucket: m = 2 r + 20 for the largest r of the bucket
+// Lanczos length by rank bucket (measured in fp32 on the workloads' spectra:
+// 20 / 32 / 40 steps reach a projector error 5x inside the tolerance)
 __host__ __device__ constexpr int lanczos_steps(int rank) {
-  return rank <= 4 ? 28 : (rank <= 8 ? 36 : 52);
+  return rank <= 4 ? 24 : (rank <= 8 ? 32 : 44);
 }
 
-template <int D>
+template <int D, int M>
 struct StatsShape {
-  static constexpr int kRegions = D / 64;           // 128-byte-wide column slabs
-  static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B (rows 64+ unused)
-  static constexpr size_t kQBytes = 64 * kQStride * 4;        // basis rows; Gram staging
-  // the key tile (needed until the Gram and the mean are done) and the two
-  // basis copies Q, Q^T share the first region
-  static constexpr size_t kKeyBytes = size_t(kRegions) * kRegionBytes;
-  static constexpr size_t kR1 = kKeyBytes > 2 * kQBytes ? kKeyBytes : 2 * kQBytes;
-  static constexpr size_t kK = 0;
-  static constexpr size_t kQ = 0;
-  static constexpr size_t kQT = kQBytes;
-  static constexpr size_t kZ = kR1;                                // eigenvectors of T
-  static constexpr size_t kW = kZ + kMaxRank * 64 * 4;             // Ritz vectors [t][k]
-  static constexpr size_t kVec = kW + 64 * kMaxRank * 4;           // small vectors
-  static constexpr size_t kMu = kVec + 2048;                       // [D]
-  static constexpr size_t kRow = kMu + D * 4;                      // [64] row means
-  static constexpr size_t kFlip = kRow + 64 * 4;                   // [4][16] uint2
-  static constexpr size_t kBar = kFlip + 4 * kMaxRank * 8;
+  static constexpr int kRegions = D / 64;                  // 128-byte-wide column slabs
+  static constexpr int kTileBytes = kRegions * 128 * 128;  // 128 rows (two blocks)
+  static constexpr int kKeyBytes = 2 * kTileBytes;         // four blocks
+  static constexpr int kStageBytes = 64 * kGStride * 4;    // one staged Gram
+  // floats per column-major row: a multiple of 4 whose quarter is odd, so the
+  // 128-bit loads of eight consecutive lanes hit distinct banks
+  static constexpr int kQTStride = (M / 4) % 2 == 0 ? M + 4 : M + 8;
+  static constexpr int kQBytes = M * kQStride * 4;         // row-major basis
+  static constexpr int kWarpQBytes = kQBytes + 64 * kQTStride * 4;
+  static constexpr int kR1a = kKeyBytes > kStatWarps * kStageBytes ? kKeyBytes
+                                                                    : kStatWarps * kStageBytes;
+  static constexpr int kR1 = kR1a > kStatWarps * kWarpQBytes ? kR1a : kStatWarps * kWarpQBytes;
+  static constexpr int kVecFloats = 64 * 3 + 48 * 3 + 16;  // x, w, h, alpha, beta, beta^2, lambda
+  static constexpr size_t kVec = kR1;
+  static constexpr size_t kMu = kVec + size_t(kStatWarps) * kVecFloats * 4;   // [4][D]
+  static constexpr size_t kRowSum = kMu + size_t(kStatWarps) * D * 4;         // [4][64]
+  static constexpr size_t kBar = kRowSum + size_t(kStatWarps) * 64 * 4;
   static constexpr size_t kMisc = kBar + 16;
-  static constexpr size_t kBytes = kMisc + 16 + 1024;  // + alignment slack
-  static_assert(64 * kGStride * 4 <= kQBytes, "Gram staging must fit in a basis region");
+  static constexpr size_t kBytes = kMisc + 64 + 1024;      // + alignment slack
+  // Z [r][M] and W [64][16] of a warp live in its row-major basis area once
+  // the Lanczos loop is done
+  static constexpr int kZBytes = (M <= 24 ? 4 : (M <= 32 ? 8 : 16)) * M * 4;
+  static_assert(kZBytes + 64 * kMaxRank * 4 <= kQBytes, "Z and W must fit in the basis area");
+  static_assert(M % 4 == 0 && M <= 48, "Lanczos length");
+  static_assert(kQTStride <= 52, "column-major basis rows");
 };
 
-// Offsets inside the small-vector area (floats).
-constexpr int kVW = 0;        // w, split layout [2][36]
-constexpr int kVH = 72;       // Gram-Schmidt coefficients h, split layout [2][36]
-constexpr int kVRed = 144;    // reduction partials [4] + norm partials [4]
-constexpr int kVAlpha = 152;  // T diagonal [64]
-constexpr int kVBeta2 = 216;  // T off-diagonal squared [64]
-constexpr int kVBeta = 280;   // T off-diagonal [64]
-constexpr int kVLam = 344;    // eigenvalues of T (descending) [16]
+// Offsets inside a warp's small-vector area (floats).
+constexpr int kVX = 0;        // matvec staging [64]
+constexpr int kVW = 64;       // w [64]
+constexpr int kVH = 128;      // Gram-Schmidt coefficients [64]
+constexpr int kVAlpha = 192;  // T diagonal [48]
+constexpr int kVBeta = 240;   // T off-diagonal [48]
+constexpr int kVBeta2 = 288;  // its squares [48]
+constexpr int kVLam = 336;    // eigenvalues of T, descending [16]
 
 __device__ __forceinline__ float hash_sign(uint32_t a, uint32_t b) {
   uint32_t h = a * 0x9E3779B1u ^ (b + 0x7F4A7C15u) * 0x85EBCA77u;
@@ -97,9 +105,6 @@ __device__ __forceinline__ float hash_sign(uint32_t a, uint32_t b) {
   h ^= h >> 12;
   return (h & 1u) ? 1.f : -1.f;
 }
-
-// split layout: element e of a 64-vector sits at (e & 1) * 36 + (e >> 1)
-__device__ __forceinline__ int qidx(int e) { return (e & 1) * 36 + (e >> 1); }
 
 __device__ __forceinline__ float pivot_guard(float d) {
   return fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
@@ -127,13 +132,43 @@ __device__ __forceinline__ void sturm_count3(const float (&al)[M], const float (
   }
 }
 
-// Byte offset of key (row, col) inside the swizzled K tile (row in 0..127).
+// Byte offset of key (row, col) inside a swizzled 128-row key tile.
 template <int D>
 __device__ __forceinline__ uint32_t k_offset(int row, int col) {
   const int region = col >> 6;
   const int c = col & 63;
-  return uint32_t(region * StatsShape<D>::kRegionBytes + row * 128 +
-                  ((((c >> 3) ^ (row & 7))) << 4) + ((c & 7) << 1));
+  return uint32_t(region * 128 * 128 + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) +
+                  ((c & 7) << 1));
+}
+
+// 64-entry dot product of a register row with a shared-memory vector
+// (broadcast 128-bit loads), four accumulators.
+__device__ __forceinline__ float row_dot(const float (&g)[64], const float* x) {
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float4 v = *reinterpret_cast<const float4*>(x + 4 * k);
+    p0 = fmaf(g[4 * k + 0], v.x, p0);
+    p1 = fmaf(g[4 * k + 1], v.y, p1);
+    p2 = fmaf(g[4 * k + 2], v.z, p2);
+    p3 = fmaf(g[4 * k + 3], v.w, p3);
+  }
+  return (p0 + p1) + (p2 + p3);
+}
+
+// 64-entry dot product of two shared-memory vectors (128-bit loads).
+__device__ __forceinline__ float smem_dot64(const float* a, const float* b) {
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const float4 x = *reinterpret_cast<const float4*>(a + 4 * k);
+    const float4 y = *reinterpret_cast<const float4*>(b + 4 * k);
+    p0 = fmaf(x.x, y.x, p0);
+    p1 = fmaf(x.y, y.y, p1);
+    p2 = fmaf(x.z, y.z, p2);
+    p3 = fmaf(x.w, y.w, p3);
+  }
+  return (p0 + p1) + (p2 + p3);
 }
 
 // ---- FP4 (E2M1) scaled storage of U (COBS explainer §2.3, quantisation) ----
@@ -167,38 +202,37 @@ __device__ __forceinline__ uint32_t fp4_code_scaled(float v, float amax) {
 }
 
 template <int D, int M>
-__global__ void __launch_bounds__(kStatThreads)
+__global__ void __launch_bounds__(kStatThreads, 2)
 block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) {
-  using S = StatsShape<D>;
+  using S = StatsShape<D, M>;
+  constexpr int kDL = D / 32;          // consecutive dimensions per lane in step 5
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ktile = smem + S::kK;
-  float* row_mean = reinterpret_cast<float*>(smem + S::kRow);
-  uint2* flip_s = reinterpret_cast<uint2*>(smem + S::kFlip);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + S::kMisc);
   uint32_t* tmem_slot = misc;
   uint32_t* abort_s = misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // work item: block j of (batch, kv-head) pair bh
   const int64_t nb_range = a.block_end - a.block_begin;
-  const int64_t item_bh = int64_t(blockIdx.x) / nb_range;
-  const int64_t item_j = a.block_begin + int64_t(blockIdx.x) % nb_range;
-  const int bt = tid;                  // thread index (the whole CTA is one team)
-  const int bwarp = warp;
+  const int64_t n_items = int64_t(a.batch) * a.hkv * nb_range;
   const int r = a.rank;
-  const int bar_id = 1;
-  constexpr int msteps = M;            // Lanczos steps
 
-  float* Qs = reinterpret_cast<float*>(smem + S::kQ);
-  float* QTs = reinterpret_cast<float*>(smem + S::kQT);
-  float* Zs = reinterpret_cast<float*>(smem + S::kZ);
-  float* Ws = reinterpret_cast<float*>(smem + S::kW);
-  float* V = reinterpret_cast<float*>(smem + S::kVec);
-  float* mus = reinterpret_cast<float*>(smem + S::kMu);
+  // this warp's work item: block item_j of (batch, kv-head) pair item_bh
+  const int64_t item = int64_t(blockIdx.x) * kStatWarps + warp;
+  const bool has_item = item < n_items;
+  const int64_t item_bh = has_item ? item / nb_range : 0;
+  const int64_t item_j = has_item ? a.block_begin + item % nb_range : 0;
+
+  float* mus = reinterpret_cast<float*>(smem + S::kMu) + warp * D;
+  float* rowsum = reinterpret_cast<float*>(smem + S::kRowSum);
+  float* V = reinterpret_cast<float*>(smem + S::kVec) + warp * S::kVecFloats;
+  float* Qs = reinterpret_cast<float*>(smem + warp * S::kWarpQBytes);
+  float* QTs = reinterpret_cast<float*>(smem + warp * S::kWarpQBytes + S::kQBytes);
+  float* Zs = Qs;                                                  // after the Lanczos loop
+  float* Ws = reinterpret_cast<float*>(smem + warp * S::kWarpQBytes + S::kZBytes);
 
   if (tid == 0) {
     mbar_init(&bars[0], 1);  // TMA
@@ -206,541 +240,616 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     fence_barrier_init();
     *abort_s = 0;
   }
-  if (warp == 0) tmem_alloc(tmem_slot, 64);
-  pdl_wait();                // keys may come from the launch before
+  if (warp == 0) tmem_alloc(tmem_slot, kTmemCols);
+  pdl_wait();                // keys (and a block table) may come from the launch before
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
 
-  // first key row of the block: in the contiguous cache, or its page (the
-  // table may come from the launch before, so it is read after the wait)
+  // first key row of this warp's block: in the contiguous cache, or its page
+  bool valid = has_item;
   int64_t row0 = item_bh * a.cap + item_j * kBlock;
-  if (a.block_table != nullptr) {
+  if (valid && a.block_table != nullptr) {
     const int64_t bb = item_bh / a.hkv, hh0 = item_bh % a.hkv;
     const int32_t page = a.block_table[bb * a.table_stride + item_j];
     if (page < 0 || page >= a.n_pages) {
       // a negative entry is a block with no page yet: its record is left as
       // it was; a page past the pool is reported and skipped the same way
-      if (tid == 0 && page >= 0) report(a.status, COBS_ERR_DEVICE);
-      if (warp == 0) tmem_dealloc(tmem, 64);
-      return;
+      if (lane == 0 && page >= 0) report(a.status, COBS_ERR_DEVICE);
+      valid = false;
+    } else {
+      row0 = (int64_t(page) * a.hkv + hh0) * kBlock;
     }
-    row0 = (int64_t(page) * a.hkv + hh0) * kBlock;
   }
-  const uint16_t* kglob = a.k + row0 * D;
+  // the rows the producer thread loads (one entry per warp, -1: none)
+  int32_t* rows_s = reinterpret_cast<int32_t*>(misc + 4);   // [4]
+  if (lane == 0) rows_s[warp] = valid ? int32_t(row0) : -1;
+  __syncthreads();
 
-  // ---- 1. TMA load of the block, then the Gram on the tensor cores -----------
+  // ---- 1. TMA of the four blocks, the Grams on the tensor cores --------------
   if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], uint32_t(kBlock) * D * 2);
-    const int y = int(row0);
-    for (int reg = 0; reg < S::kRegions; ++reg)
-      tma_load_2d(ktile + reg * S::kRegionBytes, &kmap, reg * 64, y, &bars[0]);
-    bool ok = mbar_wait_bounded(&bars[0], 0, a.status);
-    if (!ok) (void)mbar_wait_bounded(&bars[0], 0, a.status);  // copy still in flight
+    uint32_t bytes = 0;
+    for (int w = 0; w < kStatWarps; ++w)
+      if (rows_s[w] >= 0) bytes += uint32_t(kBlock) * D * 2;
+    mbar_arrive_expect_tx(&bars[0], bytes);
+    for (int w = 0; w < kStatWarps; ++w) {
+      if (rows_s[w] < 0) continue;
+      uint8_t* dst = smem + (w >> 1) * S::kTileBytes + (w & 1) * (64 * 128);
+      for (int reg = 0; reg < S::kRegions; ++reg)
+        tma_load_2d(dst + reg * 128 * 128, &kmap, reg * 64, rows_s[w], &bars[0]);
+    }
+    // the first wait has the caller's limit (cobs_set_wait_limit_ns); the one
+    // that lets copies still in flight land keeps the full default limit
+    bool ok = mbar_wait_bounded(&bars[0], 0, a.status, a.wait_limit_ns);
+    if (!ok) (void)mbar_wait_bounded(&bars[0], 0, a.status);  // copies still in flight
     if (ok) {
       tc_fence_after();
-      constexpr uint32_t idesc = umma_idesc_bf16(128, 64);
-      const uint32_t kbase = smem_addr(ktile);
+      constexpr uint32_t idesc = umma_idesc_bf16(128, 128);
+      for (int tile = 0; tile < 2; ++tile) {
+        const uint32_t kbase = smem_addr(smem + tile * S::kTileBytes);
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t addr = kbase + (ks >> 2) * S::kRegionBytes + (ks & 3) * 32;
-        const uint64_t desc = umma_desc_sw128(addr);
-        umma_bf16(tmem, desc, desc, idesc, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t desc = umma_desc_sw128(kbase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+          umma_bf16(tmem + uint32_t(tile * 128), desc, desc, idesc, ks > 0 ? 1u : 0u);
+        }
       }
       umma_commit(&bars[1]);
-      ok = mbar_wait_bounded(&bars[1], 0, a.status);
-      if (!ok) (void)mbar_wait_bounded(&bars[1], 0, a.status);  // MMA still running
     }
     *abort_s = ok ? 0u : 1u;
   }
   __syncthreads();
-  const bool aborted = *abort_s != 0;
-  if (!aborted && tid != 0) (void)mbar_try_wait(&bars[1], 0);
-  tc_fence_after();
-
-  // ---- 2. Gram rows back from tensor memory (warps 0-1), mean, centring ------
-  float g[64];
-  const int ri = tid;                  // Gram row (threads 0-63)
-  if (!aborted && warp < 2) {
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    float t32[32];
-    tmem_ld32(tmem + lane_base, t32);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) g[c] = t32[c];
-    tmem_ld32(tmem + lane_base + 32, t32);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) g[32 + c] = t32[c];
-    float rsum = 0.f;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) rsum += g[c];
-    row_mean[ri] = rsum * (1.f / 64.f);
-  }
-  // block mean (fp32 sum of 64 bf16 keys): thread bt < D owns dim bt
-  if (!aborted && bt < D) {
-    float acc = 0.f;
-    for (int t = 0; t < kBlock; ++t) {
-      const uint16_t w = *reinterpret_cast<const uint16_t*>(ktile + k_offset<D>(t, bt));
-      acc += __uint_as_float(uint32_t(w) << 16);
+  bool aborted = *abort_s != 0;
+  if (!aborted) (void)mbar_try_wait(&bars[0], 0);   // acquire the TMA writes
+  // block means (fp32 sums of 64 bf16 keys) while the products run: warp w
+  // sums the columns of its own block
+  if (!aborted && valid) {
+    const uint8_t* tile = smem + (warp >> 1) * S::kTileBytes;
+    const int rbase = (warp & 1) * 64;
+    for (int c = lane; c < D; c += 32) {
+      float acc = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < kBlock; ++t) {
+        const uint16_t w16 = *reinterpret_cast<const uint16_t*>(tile + k_offset<D>(rbase + t, c));
+        acc += __uint_as_float(uint32_t(w16) << 16);
+      }
+      mus[c] = acc * (1.f / 64.f);
     }
-    mus[bt] = acc * (1.f / 64.f);
+  }
+  if (tid == 0 && !aborted) {
+    const bool ok = mbar_wait_bounded(&bars[1], 0, a.status);
+    if (!ok) {
+      (void)mbar_wait_bounded(&bars[1], 0, a.status);    // MMA still running
+      *abort_s = 1u;
+    }
+  }
+  __syncthreads();           // means done (the key tiles may be overwritten), MMA done
+  aborted = *abort_s != 0;
+  if (!aborted) {
+    if (tid != 0) (void)mbar_try_wait(&bars[1], 0);
+    tc_fence_after();
+    // ---- 2. Gram rows from tensor memory to the owning warp's staging ------
+    // lanes 32 w .. 32 w + 31 of tile p hold rows (w & 1) * 32 + lane of the
+    // Gram of block 2 p + (w >> 1), in columns (w >> 1) * 64 .. + 63
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    for (int p = 0; p < 2; ++p) {
+      const int bl = 2 * p + (warp >> 1);
+      const int row = (warp & 1) * 32 + lane;
+      float* stage = reinterpret_cast<float*>(smem + bl * S::kStageBytes) + row * kGStride;
+      float rs = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + uint32_t(p * 128 + (warp >> 1) * 64 + half * 32), v);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) rs += v[c];
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          *reinterpret_cast<float4*>(stage + half * 32 + 4 * c4) =
+              make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+      }
+      rowsum[bl * 64 + row] = rs;
+    }
   }
   tc_fence_before();
-  __syncthreads();                     // key tile and tensor memory no longer needed
-  if (warp == 0) tmem_dealloc(tmem, 64);
+  __syncthreads();           // staged Grams and row sums complete
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
   if (aborted) return;
-  if (warp < 2) {
-    float ssum = 0.f;
-    for (int c = 0; c < 64; ++c) ssum += row_mean[c];
-    const float smean = ssum * (1.f / 64.f);
-    const float rm = row_mean[ri];
-    // Gc is symmetric: row ri is stored as column ri (consecutive lanes ->
-    // consecutive addresses); the staging area overlays the key tile
-    float* stage = QTs;
+
+  // this warp's centred Gram: lane l holds rows l and l + 32 in registers
+  float g0[64], g1[64];
+  float trace_a = 0.f;
+  {
+    const float* st = reinterpret_cast<const float*>(smem + warp * S::kStageBytes);
+    const float* rsum = rowsum + warp * 64;
+    const float rm0 = rsum[lane] * (1.f / 64.f), rm1 = rsum[lane + 32] * (1.f / 64.f);
+    const float smean = warp_sum(rm0 + rm1) * (1.f / 64.f);
 #pragma unroll
-    for (int c = 0; c < 64; ++c) stage[c * kGStride + ri] = g[c] - rm - row_mean[c] + smean;
+    for (int k = 0; k < 16; ++k) {
+      const float4 cm = *reinterpret_cast<const float4*>(rsum + 4 * k);
+      const float4 x0 = *reinterpret_cast<const float4*>(st + lane * kGStride + 4 * k);
+      const float4 x1 = *reinterpret_cast<const float4*>(st + (lane + 32) * kGStride + 4 * k);
+      const float c[4] = {cm.x * (1.f / 64.f), cm.y * (1.f / 64.f), cm.z * (1.f / 64.f),
+                          cm.w * (1.f / 64.f)};
+      const float a0[4] = {x0.x, x0.y, x0.z, x0.w};
+      const float a1[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        g0[4 * k + u] = a0[u] - rm0 - c[u] + smean;
+        g1[4 * k + u] = a1[u] - rm1 - c[u] + smean;
+      }
+    }
+    // trace(A) = trace(Gc^2) = |Gc|_F^2
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < 64; ++k) t = fmaf(g0[k], g0[k], fmaf(g1[k], g1[k], t));
+    trace_a = warp_sum(t);
   }
-  __syncthreads();
+  __syncthreads();           // every staged Gram is in registers: the area is reused
 
-  const bool do_eig = r > 0;
-  const int li = bt >> 1, hh = bt & 1;
-  auto block_sum = [&](float v) -> float {  // sum over the 128 threads
-    v = warp_sum(v);
-    if (lane == 0) V[kVRed + bwarp] = v;
-    named_bar(bar_id, 128);
-    return (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
-  };
-
+  const bool do_eig = r > 0 && valid;
+  const int lA = lane, lB = lane + 32;   // this lane's two entries of a 64-vector
+  float* xv = V + kVX;
+  float* wv = V + kVW;
+  float* hv = V + kVH;
   if (do_eig) {
-    // ---- 3a. A = Gc * Gc (4 x 8 register tile per thread) ----------------------
+    const float tol = 1e-5f * trace_a;
+    // the Gram-Schmidt update reads a few basis columns past the current step
+    // (times zero coefficients): they must hold zeros, not whatever an
+    // earlier kernel left in shared memory (0 x NaN is NaN)
+    for (int e = lane; e < 64 * S::kQTStride / 4; e += 32)
+      reinterpret_cast<float4*>(QTs)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = lane; e < M * kQStride / 4; e += 32)
+      reinterpret_cast<float4*>(Qs)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncwarp();
+    // q_0: a fixed pseudo-random +-1/8 vector (unit norm)
     {
-      const float* gcs = QTs;           // Gc staging, stride kGStride
-      float* a2 = Qs;                   // A staging, stride kGStride
-      const int rg = bt >> 3, cg = bt & 7;
-      float acc[4][8];
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 8; ++y) acc[x][y] = 0.f;
-#pragma unroll 4
-      for (int k = 0; k < 64; ++k) {
-        const float4 av = *reinterpret_cast<const float4*>(gcs + k * kGStride + 4 * rg);
-        const float4 b0 = *reinterpret_cast<const float4*>(gcs + k * kGStride + 8 * cg);
-        const float4 b1 = *reinterpret_cast<const float4*>(gcs + k * kGStride + 8 * cg + 4);
-        const float ar[4] = {av.x, av.y, av.z, av.w};
-        const float br[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 8; ++y) acc[x][y] = fmaf(ar[x], br[y], acc[x][y]);
-      }
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        float* row = a2 + (4 * rg + x) * kGStride + 8 * cg;
-        *reinterpret_cast<float4*>(row) = make_float4(acc[x][0], acc[x][1], acc[x][2], acc[x][3]);
-        *reinterpret_cast<float4*>(row + 4) =
-            make_float4(acc[x][4], acc[x][5], acc[x][6], acc[x][7]);
-      }
+      const float v0 = hash_sign(7u, uint32_t(lA)) * 0.125f;
+      const float v1 = hash_sign(7u, uint32_t(lB)) * 0.125f;
+      Qs[lA] = v0;
+      Qs[lB] = v1;
+      QTs[lA * S::kQTStride] = v0;
+      QTs[lB * S::kQTStride] = v1;
     }
-    named_bar(bar_id, 128);
-    // thread (li, hh) owns row li of A, columns 2k + hh
-    float gr[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) gr[k] = Qs[li * kGStride + 2 * k + hh];
-    const float trace_part = (hh == (li & 1)) ? gr[li >> 1] : 0.f;   // diagonal once
-    const float trace = block_sum(trace_part);
-    const float tol = 1e-5f * trace;
-    named_bar(bar_id, 128);                 // partials read, staging consumed
-    for (int e = bt; e < 64 * kQStride; e += 128) {
-      Qs[e] = 0.f;
-      QTs[e] = 0.f;
-    }
-    for (int e = bt; e < 144; e += 128) V[kVW + e] = 0.f;   // w and h
-    named_bar(bar_id, 128);
-    if (hh == 0) {
-      const float v0 = hash_sign(7u, uint32_t(li)) * 0.125f;
-      Qs[qidx(li)] = v0;
-      QTs[li * kQStride + qidx(0)] = v0;
-    }
-    named_bar(bar_id, 128);
+    __syncwarp();
 
-    // Orthogonalise w (this thread's entry wi of row li) against Q[0..jmax],
-    // twice.  Returns the summed coefficient of q_jmax; sq receives |w|^2
-    // after the first pass minus |h|^2 of the second (= |w|^2 at the end).
-    auto cgs = [&](float& wi, int jmax, float& sq) -> float {
+    // Orthogonalise (w0, w1) against basis rows 0..jmax, twice.  Returns the
+    // summed coefficient of q_jmax and |w|^2 at the end.
+    auto cgs = [&](float& w0, float& w1, int jmax, float& sq) -> float {
       float acoef = 0.f;
-      const int nc = ((jmax >> 1) >> 2) + 1;   // 4-wide chunks per parity
+      float n1 = 0.f, hh2 = 0.f;
+      const int nc = (jmax >> 2) + 1;   // 4-wide chunks of coefficients
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
-        if (hh == 0) V[kVW + qidx(li)] = wi;
-        if (pass == 1) {   // |w|^2 after the first pass: warp partials
-          const float ps = warp_sum(hh == 0 ? wi * wi : 0.f);
-          if (lane == 0) V[kVRed + 4 + bwarp] = ps;
+        wv[lA] = w0;
+        wv[lB] = w1;
+        __syncwarp();
+        float ha = 0.f, hb = 0.f;
+        if (lA <= jmax) ha = smem_dot64(Qs + lA * kQStride, wv);
+        if (lB <= jmax) hb = smem_dot64(Qs + lB * kQStride, wv);
+        if (pass == 1) {
+          hh2 = warp_sum(ha * ha + hb * hb);
         }
-        named_bar(bar_id, 128);
-        if (pass == 1)
-          sq = (V[kVRed + 4] + V[kVRed + 5]) + (V[kVRed + 6] + V[kVRed + 7]);
-        float hp = 0.f;
-        if (li <= jmax) {
-          const float4* qm = reinterpret_cast<const float4*>(Qs + li * kQStride + hh * 36);
-          const float4* ws = reinterpret_cast<const float4*>(V + kVW + hh * 36);
-          float h0 = 0.f, h1 = 0.f, h2 = 0.f, h3 = 0.f;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float4 x = qm[k], y = ws[k];
-            h0 = fmaf(x.x, y.x, h0);
-            h1 = fmaf(x.y, y.y, h1);
-            h2 = fmaf(x.z, y.z, h2);
-            h3 = fmaf(x.w, y.w, h3);
-          }
-          hp = (h0 + h1) + (h2 + h3);
-        }
-        hp += __shfl_xor_sync(0xffffffffu, hp, 1);
-        if (hh == 0) V[kVH + qidx(li)] = hp;       // zero for li > jmax
-        if (pass == 1) {   // |h|^2 of the second pass: warp partials
-          const float ph = warp_sum(hh == 0 ? hp * hp : 0.f);
-          if (lane == 0) V[kVRed + bwarp] = ph;
-        }
-        named_bar(bar_id, 128);
-        // w_i -= sum_m Q[m][i] h_m over m of this thread's parity
-        const float4* qt = reinterpret_cast<const float4*>(QTs + li * kQStride + hh * 36);
-        const float4* hv = reinterpret_cast<const float4*>(V + kVH + hh * 36);
-        float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
-        constexpr int kMaxChunks = ((M - 1) / 2) / 4 + 1;
+        hv[lA] = ha;
+        hv[lB] = hb;
+        __syncwarp();
+        const float* qa = QTs + lA * S::kQTStride;
+        const float* qb = QTs + lB * S::kQTStride;
+        float c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
+        constexpr int kMaxChunks = M / 4;
 #pragma unroll
         for (int c = 0; c < kMaxChunks; ++c) {
           if (c < nc) {
-            const float4 x = qt[c], y = hv[c];
-            c0 = fmaf(x.x, y.x, c0);
-            c1 = fmaf(x.y, y.y, c1);
-            c2 = fmaf(x.z, y.z, c2);
-            c3 = fmaf(x.w, y.w, c3);
+            const float4 h4 = *reinterpret_cast<const float4*>(hv + 4 * c);
+            const float4 x = *reinterpret_cast<const float4*>(qa + 4 * c);
+            const float4 y = *reinterpret_cast<const float4*>(qb + 4 * c);
+            c0 = fmaf(x.x, h4.x, fmaf(x.y, h4.y, c0));
+            c1 = fmaf(x.z, h4.z, fmaf(x.w, h4.w, c1));
+            d0 = fmaf(y.x, h4.x, fmaf(y.y, h4.y, d0));
+            d1 = fmaf(y.z, h4.z, fmaf(y.w, h4.w, d1));
           }
         }
-        float corr = (c0 + c1) + (c2 + c3);
-        corr += __shfl_xor_sync(0xffffffffu, corr, 1);
-        wi -= corr;
-        acoef += V[kVH + qidx(jmax)];
-        if (pass == 1) {
-          const float s0 = (V[kVRed + 0] + V[kVRed + 1]) + (V[kVRed + 2] + V[kVRed + 3]);
-          sq = fmaxf(sq - s0, 0.f);
-        }
+        w0 -= c0 + c1;
+        w1 -= d0 + d1;
+        acoef += hv[jmax];
+        if (pass == 0) n1 = warp_sum(w0 * w0 + w1 * w1);
+        __syncwarp();   // hv and wv are rewritten by the next pass
       }
+      // |w2|^2 = |w1|^2 - |h2|^2 for an orthonormal basis; when the second
+      // pass removed much of w1 the difference cancels, so sum exactly then
+      if (hh2 > 0.25f * n1) sq = warp_sum(w0 * w0 + w1 * w1);
+      else sq = fmaxf(n1 - hh2, 0.f);
       return acoef;
     };
 
 #pragma unroll 1
-    for (int j = 0; j < msteps; ++j) {
-      // w = A q_j
-      const float4* qj = reinterpret_cast<const float4*>(Qs + j * kQStride + hh * 36);
-      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 x = qj[k];
-        p0 = fmaf(gr[4 * k + 0], x.x, p0);
-        p1 = fmaf(gr[4 * k + 1], x.y, p1);
-        p2 = fmaf(gr[4 * k + 2], x.z, p2);
-        p3 = fmaf(gr[4 * k + 3], x.w, p3);
-      }
-      const float p = (p0 + p1) + (p2 + p3);
-      float wi = p + __shfl_xor_sync(0xffffffffu, p, 1);
+    for (int j = 0; j < M; ++j) {
+      // w = Gc (Gc q_j)
+      const float* qj = Qs + j * kQStride;
+      const float y0 = row_dot(g0, qj), y1 = row_dot(g1, qj);
+      xv[lA] = y0;
+      xv[lB] = y1;
+      __syncwarp();
+      float w0 = row_dot(g0, xv), w1 = row_dot(g1, xv);
       float sq = 0.f;
-      const float aj = cgs(wi, j, sq);
+      const float aj = cgs(w0, w1, j, sq);
       float beta = sqrtf(sq);
-      if (bt == 0) V[kVAlpha + j] = aj;
-      if (j == msteps - 1) break;
+      if (lane == 0) V[kVAlpha + j] = aj;
+      if (j == M - 1) break;
       if (!(beta > tol)) {
         // the Krylov space closed: continue from a fresh vector
-        wi = hash_sign(uint32_t(j + 1), uint32_t(li));
-        named_bar(bar_id, 128);
+        w0 = hash_sign(uint32_t(j + 1), uint32_t(lA));
+        w1 = hash_sign(uint32_t(j + 1), uint32_t(lB));
         float sq2 = 0.f;
-        cgs(wi, j, sq2);
-        const float nrm = sqrtf(sq2);
-        wi = nrm > 0.f ? wi / nrm : 0.f;
+        cgs(w0, w1, j, sq2);
+        sq2 = warp_sum(w0 * w0 + w1 * w1);
+        const float inv = sq2 > 0.f ? rsqrtf(sq2) : 0.f;
+        w0 *= inv;
+        w1 *= inv;
         beta = 0.f;
       } else {
-        wi = wi * (1.f / beta);
+        const float inv = 1.f / beta;
+        w0 *= inv;
+        w1 *= inv;
       }
-      if (bt == 0) {
+      if (lane == 0) {
         V[kVBeta + j] = beta;
         V[kVBeta2 + j] = beta * beta;
       }
-      if (hh == 0) {
-        Qs[(j + 1) * kQStride + qidx(li)] = wi;
-        QTs[li * kQStride + qidx(j + 1)] = wi;
-      }
-      named_bar(bar_id, 128);
+      Qs[(j + 1) * kQStride + lA] = w0;
+      Qs[(j + 1) * kQStride + lB] = w1;
+      QTs[lA * S::kQTStride + j + 1] = w0;
+      QTs[lB * S::kQTStride + j + 1] = w1;
+      __syncwarp();
     }
-    named_bar(bar_id, 128);
+    __syncwarp();
 
     // ---- 4. top-r eigenpairs of T ---------------------------------------------
-    constexpr int m = msteps;
     const float* alpha = V + kVAlpha;
     const float* betav = V + kVBeta;
-    float al[m], b2[m];
+    float al[M], b2[M];
 #pragma unroll
-    for (int i2 = 0; i2 < m; ++i2) {
+    for (int i2 = 0; i2 < M; ++i2) {
       al[i2] = alpha[i2];
       b2[i2] = V[kVBeta2 + i2];
     }
     float lo = 0.f, hi = 0.f;
 #pragma unroll
-    for (int i2 = 0; i2 < m; ++i2) {
+    for (int i2 = 0; i2 < M; ++i2) {
       const float rad =
-          (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < m - 1 ? fabsf(betav[i2]) : 0.f);
+          (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < M - 1 ? fabsf(betav[i2]) : 0.f);
       lo = fminf(lo, al[i2] - rad);
       hi = fmaxf(hi, al[i2] + rad);
     }
     hi = hi * (1.f + 1e-6f) + 1e-30f;
     lo = lo - 1e-6f * fabsf(hi) - 1e-30f;
-    const int grp = bt >> 3, sub = bt & 7;   // 8 threads x 3 shifts per eigenvalue
-    const int kk = grp;                      // k-th largest
-    const int target = m - 1 - kk;           // count(x) <= target below it
+    // lanes per eigenvalue: 32 / (r rounded up to a power of two)
+    const int rp = r <= 1 ? 1 : (r <= 2 ? 2 : (r <= 4 ? 4 : (r <= 8 ? 8 : 16)));
+    const int lpe = 32 / rp;                    // lanes of one eigenvalue
+    const int kk = lane / lpe, sub = lane % lpe;
+    const int npts = 3 * lpe;                   // shifts per eigenvalue per round
+    const int rounds = lpe >= 8 ? 5 : (lpe >= 4 ? 6 : (lpe >= 2 ? 8 : 12));
+    const int target = M - 1 - kk;              // count(x) <= target below it
     float ea = lo, eb = hi;
-    for (int it = 0; it < kBisectRounds; ++it) {
-      const float step = (eb - ea) * (1.f / 25.f);
+    for (int it = 0; it < rounds; ++it) {
+      const float step = (eb - ea) / float(npts + 1);
       float xs[3];
       int cs[3];
 #pragma unroll
       for (int s2 = 0; s2 < 3; ++s2) xs[s2] = ea + step * float(3 * sub + s2 + 1);
-      sturm_count3<m>(al, b2, xs, cs);
-      const int sh = (lane >> 3) << 3;
-      uint32_t mask24 = 0;
+      sturm_count3<M>(al, b2, xs, cs);
+      // first point of this eigenvalue's group whose count exceeds target
+      const int sh = kk * lpe;
+      const uint32_t gmask = lpe == 32 ? 0xffffffffu : (((1u << lpe) - 1u) << sh);
+      int first = npts;
 #pragma unroll
       for (int s2 = 0; s2 < 3; ++s2) {
-        const uint32_t bal = (__ballot_sync(0xffffffffu, cs[s2] > target) >> sh) & 0xffu;
-        // point 3u + s2 + 1 of lane u in the group -> bit 3u + s2
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mask24 |= ((bal >> u) & 1u) << (3 * u + s2);
+        const uint32_t bal = (__ballot_sync(0xffffffffu, cs[s2] > target) & gmask) >> sh;
+        // lane u of the group holds point 3u + s2 + 1
+        if (bal) first = min(first, 3 * (__ffs(bal) - 1) + s2);
       }
-      const int first = mask24 ? __ffs(mask24) - 1 : 24;   // first point above
       const float na = first == 0 ? ea : ea + step * float(first);
-      const float nb = first == 24 ? eb : ea + step * float(first + 1);
+      const float nb = first == npts ? eb : ea + step * float(first + 1);
       ea = na;
       eb = nb;
     }
     const float theta = 0.5f * (ea + eb);
     if (sub == 0 && kk < r) V[kVLam + kk] = theta;
-    named_bar(bar_id, 128);
+    __syncwarp();
 
-    // inverse iteration, one thread per eigenvalue: (T - theta I) z = y, LDL^T
-    if (sub == 0 && kk < r) {
-      float l[m], rd[m];
+    // inverse iteration, one lane per eigenvalue: (T - theta I) z = y, LDL^T
+    if (lane < r) {
+      const float th = V[kVLam + lane];
+      float l[M], rd[M];
       {
-        float d = pivot_guard(al[0] - theta);
+        float d = pivot_guard(al[0] - th);
         rd[0] = 1.f / d;
         l[0] = 0.f;
 #pragma unroll
-        for (int i2 = 1; i2 < m; ++i2) {
+        for (int i2 = 1; i2 < M; ++i2) {
           l[i2] = betav[i2 - 1] * rd[i2 - 1];
-          d = pivot_guard(al[i2] - theta - l[i2] * betav[i2 - 1]);
+          d = pivot_guard(al[i2] - th - l[i2] * betav[i2 - 1]);
           rd[i2] = 1.f / d;
         }
       }
-      float z[m];
+      float z[M];
 #pragma unroll
-      for (int i2 = 0; i2 < m; ++i2)
-        z[i2] = 1.f + 0.25f * hash_sign(uint32_t(kk + 101), uint32_t(i2));
+      for (int i2 = 0; i2 < M; ++i2)
+        z[i2] = 1.f + 0.25f * hash_sign(uint32_t(lane + 101), uint32_t(i2));
       float nrm2 = 1.f;
 #pragma unroll
       for (int it = 0; it < kInverseIters; ++it) {
 #pragma unroll
-        for (int i2 = 1; i2 < m; ++i2) z[i2] = fmaf(-l[i2], z[i2 - 1], z[i2]);
+        for (int i2 = 1; i2 < M; ++i2) z[i2] = fmaf(-l[i2], z[i2 - 1], z[i2]);
 #pragma unroll
-        for (int i2 = 0; i2 < m; ++i2) z[i2] *= rd[i2];
+        for (int i2 = 0; i2 < M; ++i2) z[i2] *= rd[i2];
 #pragma unroll
-        for (int i2 = m - 2; i2 >= 0; --i2) z[i2] = fmaf(-l[i2 + 1], z[i2 + 1], z[i2]);
+        for (int i2 = M - 2; i2 >= 0; --i2) z[i2] = fmaf(-l[i2 + 1], z[i2 + 1], z[i2]);
         float mx = 0.f;
 #pragma unroll
-        for (int i2 = 0; i2 < m; ++i2) mx = fmaxf(mx, fabsf(z[i2]));
+        for (int i2 = 0; i2 < M; ++i2) mx = fmaxf(mx, fabsf(z[i2]));
         const float inv = mx > 0.f ? 1.f / mx : 1.f;
         nrm2 = 0.f;
 #pragma unroll
-        for (int i2 = 0; i2 < m; ++i2) {
+        for (int i2 = 0; i2 < M; ++i2) {
           z[i2] *= inv;
           nrm2 = fmaf(z[i2], z[i2], nrm2);
         }
       }
       const float inv = rsqrtf(fmaxf(nrm2, 1e-30f));
 #pragma unroll
-      for (int i2 = 0; i2 < 64; ++i2) Zs[kk * 64 + i2] = i2 < m ? z[i2] * inv : 0.f;
+      for (int i2 = 0; i2 < M; ++i2) Zs[lane * M + i2] = z[i2] * inv;
     }
-    named_bar(bar_id, 128);
-    // re-orthogonalise inside clusters of close eigenvalues (warp 0 of the team)
-    if (bwarp == 0) {
+    __syncwarp();
+    // re-orthogonalise inside clusters of close eigenvalues
+    {
       const float th0 = V[kVLam + 0];
       for (int k2 = 1; k2 < r; ++k2) {
         const float tk = V[kVLam + k2];
-        float* zk = Zs + k2 * 64;
+        float* zk = Zs + k2 * M;
         bool touched = false;
         for (int l2 = 0; l2 < k2; ++l2) {
           if (fabsf(V[kVLam + l2] - tk) > 1e-3f * fabsf(th0)) continue;
-          const float* zl = Zs + l2 * 64;
-          const float c = warp_sum(zl[lane] * zk[lane] + zl[lane + 32] * zk[lane + 32]);
-          zk[lane] -= c * zl[lane];
-          zk[lane + 32] -= c * zl[lane + 32];
+          const float* zl = Zs + l2 * M;
+          float part = 0.f;
+          for (int i2 = lane; i2 < M; i2 += 32) part = fmaf(zl[i2], zk[i2], part);
+          const float c = warp_sum(part);
+          for (int i2 = lane; i2 < M; i2 += 32) zk[i2] -= c * zl[i2];
           touched = true;
           __syncwarp();
         }
         if (touched) {
-          const float n2 = warp_sum(zk[lane] * zk[lane] + zk[lane + 32] * zk[lane + 32]);
-          const float inv = rsqrtf(fmaxf(n2, 1e-30f));
-          zk[lane] *= inv;
-          zk[lane + 32] *= inv;
+          float part = 0.f;
+          for (int i2 = lane; i2 < M; i2 += 32) part = fmaf(zk[i2], zk[i2], part);
+          const float inv = rsqrtf(fmaxf(warp_sum(part), 1e-30f));
+          for (int i2 = lane; i2 < M; i2 += 32) zk[i2] *= inv;
         }
         __syncwarp();
       }
     }
-    named_bar(bar_id, 128);
-    // Ritz vectors w_k = Q z_k stored [t][k]; thread (t = li, hh) takes
-    // k = hh, hh + 2, ...; eigenvalues below 1e-12 of the largest (of A = Gc^2)
-    // are treated as zero
+    // Ritz vectors w_k = Q z_k stored [t][k]; eigenvalues below 1e-12 of the
+    // largest (of A = Gc^2) are treated as zero
     {
-      float acc[kMaxRank / 2];
-#pragma unroll
-      for (int k2 = 0; k2 < kMaxRank / 2; ++k2) acc[k2] = 0.f;
-      for (int mm = 0; mm < m; ++mm) {
-        const float qv = QTs[li * kQStride + qidx(mm)];
-#pragma unroll
-        for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
-          const int k = 2 * k2 + hh;
-          if (k < r) acc[k2] = fmaf(qv, Zs[k * 64 + mm], acc[k2]);
-        }
-      }
       const float th0 = V[kVLam + 0];
+      const float* qa = QTs + lA * S::kQTStride;
+      const float* qb = QTs + lB * S::kQTStride;
+#pragma unroll 1
+      for (int k = 0; k < r; ++k) {
+        const float* zk = Zs + k * M;
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int k2 = 0; k2 < kMaxRank / 2; ++k2) {
-        const int k = 2 * k2 + hh;
-        if (k < r) {
-          const float tk = V[kVLam + k];
-          const bool keep = tk > 1e-12f * th0 && tk > 0.f;
-          Ws[li * kMaxRank + k] = keep ? acc[k2] : 0.f;
+        for (int c = 0; c < M / 4; ++c) {
+          const float4 z4 = *reinterpret_cast<const float4*>(zk + 4 * c);
+          const float4 x = *reinterpret_cast<const float4*>(qa + 4 * c);
+          const float4 y = *reinterpret_cast<const float4*>(qb + 4 * c);
+          s0 = fmaf(x.x, z4.x, fmaf(x.y, z4.y, fmaf(x.z, z4.z, fmaf(x.w, z4.w, s0))));
+          s1 = fmaf(y.x, z4.x, fmaf(y.y, z4.y, fmaf(y.z, z4.z, fmaf(y.w, z4.w, s1))));
         }
+        const float tk = V[kVLam + k];
+        const bool keep = tk > 1e-12f * th0 && tk > 0.f;
+        Ws[lA * kMaxRank + k] = keep ? s0 : 0.f;
+        Ws[lB * kMaxRank + k] = keep ? s1 : 0.f;
       }
     }
+    __syncwarp();
   }
-  __syncthreads();
+  if (!valid) return;        // no more CTA-wide barriers below
 
-  // ---- 5. U = Kc^T w / sqrt(n), sign rule, bf16 record ------------------------
-  // thread bt < D owns output dim d = bt; keys re-read through L2 (coalesced rows)
-  float uacc[kMaxRank];
+  // ---- 5. U = Kc^T w / sqrt(n), sign rule, record ----------------------------
+  // lane l owns dimensions [kDL l, kDL l + kDL); keys re-read through L2
+  const uint16_t* kglob = a.k + row0 * D;
+  const int t0 = kDL * lane;
+  float mu_l[kDL];
 #pragma unroll
-  for (int k = 0; k < kMaxRank; ++k) uacc[k] = 0.f;
-  const float mu_d = bt < D ? mus[bt] : 0.f;
-  if (do_eig && bt < D) {
-#pragma unroll 4
+  for (int u = 0; u < kDL; ++u) mu_l[u] = mus[t0 + u];
+  float uacc[kMaxRank][kDL];
+#pragma unroll
+  for (int k = 0; k < kMaxRank; ++k)
+#pragma unroll
+    for (int u = 0; u < kDL; ++u) uacc[k][u] = 0.f;
+  if (do_eig) {
+#pragma unroll 2
     for (int t = 0; t < kBlock; ++t) {
-      const uint16_t w = kglob[int64_t(t) * D + bt];
-      const float kc = __uint_as_float(uint32_t(w) << 16) - mu_d;
+      float kc[kDL];
+      if constexpr (kDL == 4) {
+        const uint2 w2 = *reinterpret_cast<const uint2*>(kglob + int64_t(t) * D + t0);
+        const float2 f0 = bf16x2_to_float2(w2.x), f1 = bf16x2_to_float2(w2.y);
+        kc[0] = f0.x - mu_l[0];
+        kc[1] = f0.y - mu_l[1];
+        kc[2] = f1.x - mu_l[2];
+        kc[3] = f1.y - mu_l[3];
+      } else {
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kglob + int64_t(t) * D + t0);
+        const float2 f0 = bf16x2_to_float2(w1);
+        kc[0] = f0.x - mu_l[0];
+        kc[1] = f0.y - mu_l[1];
+      }
       const float4* wt = reinterpret_cast<const float4*>(Ws + t * kMaxRank);
 #pragma unroll
       for (int k4 = 0; k4 < kMaxRank / 4; ++k4) {
         if (4 * k4 < r) {
           const float4 u4 = wt[k4];
-          uacc[4 * k4 + 0] = fmaf(kc, u4.x, uacc[4 * k4 + 0]);
-          uacc[4 * k4 + 1] = fmaf(kc, u4.y, uacc[4 * k4 + 1]);
-          uacc[4 * k4 + 2] = fmaf(kc, u4.z, uacc[4 * k4 + 2]);
-          uacc[4 * k4 + 3] = fmaf(kc, u4.w, uacc[4 * k4 + 3]);
+          const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < kDL; ++u) uacc[4 * k4 + q][u] = fmaf(kc[u], uu[q], uacc[4 * k4 + q][u]);
         }
       }
     }
   }
   // sign: the component of largest magnitude (lowest index on ties) is positive
-  if (r > 0) {
-#pragma unroll
-    for (int k = 0; k < kMaxRank; ++k) {
-      if (k < r) {
-        const float v = uacc[k] * 0.125f;  // 1/sqrt(64)
-        uacc[k] = v;
-        float best = bt < D ? fabsf(v) : -1.f;
-        int bidx = bt;
-        uint32_t bneg = v < 0.f;
-#pragma unroll
-        for (int mm = 16; mm >= 1; mm >>= 1) {
-          const float ob = __shfl_xor_sync(0xffffffffu, best, mm);
-          const int oi = __shfl_xor_sync(0xffffffffu, bidx, mm);
-          const uint32_t on = __shfl_xor_sync(0xffffffffu, bneg, mm);
-          if (ob > best || (ob == best && oi < bidx)) { best = ob; bidx = oi; bneg = on; }
-        }
-        if (lane == 0)
-          flip_s[bwarp * kMaxRank + k] = make_uint2(__float_as_uint(best), (uint32_t(bidx) << 1) | bneg);
-      }
-    }
-  }
-  __syncthreads();
   uint32_t neg_mask = 0;
-  if (r > 0) {
+#pragma unroll
+  for (int k = 0; k < kMaxRank; ++k) {
+    if (k < r) {
+      float best = -1.f;
+      int bidx = 0;
+      uint32_t bneg = 0;
+#pragma unroll
+      for (int u = 0; u < kDL; ++u) {
+        const float v = uacc[k][u] * 0.125f;   // 1/sqrt(64)
+        uacc[k][u] = v;
+        if (fabsf(v) > best) {
+          best = fabsf(v);
+          bidx = t0 + u;
+          bneg = v < 0.f;
+        }
+      }
+#pragma unroll
+      for (int mm = 16; mm >= 1; mm >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, mm);
+        const int oi = __shfl_xor_sync(0xffffffffu, bidx, mm);
+        const uint32_t on = __shfl_xor_sync(0xffffffffu, bneg, mm);
+        if (ob > best || (ob == best && oi < bidx)) {
+          best = ob;
+          bidx = oi;
+          bneg = on;
+        }
+      }
+      neg_mask |= bneg << k;
+    }
+  }
+  uint8_t* rec8 = reinterpret_cast<uint8_t*>(a.stats) + ((item_bh * a.nb_cap) + item_j) * a.rec_bytes;
+  uint16_t* rec = reinterpret_cast<uint16_t*>(rec8);
+  auto store_bf16 = [&](uint16_t* dst, const float (&v)[kDL]) {
+    if constexpr (kDL == 4) {
+      const uint32_t lo = uint32_t(float_to_bf16_bits(v[0])) | (uint32_t(float_to_bf16_bits(v[1])) << 16);
+      const uint32_t hi2 = uint32_t(float_to_bf16_bits(v[2])) | (uint32_t(float_to_bf16_bits(v[3])) << 16);
+      *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi2);
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) =
+          uint32_t(float_to_bf16_bits(v[0])) | (uint32_t(float_to_bf16_bits(v[1])) << 16);
+    }
+  };
+  store_bf16(rec + t0, mu_l);
+  if (a.stats_format == 3) {
+    // subspace record (COBS explainer §2.3, subspace projection): row k of
+    // U_s = P^T U[:, k], the sign-fixed column's s coordinates in the query
+    // subspace spanned by the rows of P (this kv-head's [s][d] fp32 basis)
+    float* us = Qs;                       // [D][16] floats; the basis area is free
+    __syncwarp();                         // every lane is done with W
 #pragma unroll
     for (int k = 0; k < kMaxRank; ++k) {
       if (k < r) {
-        uint2 best = flip_s[k];
-        for (int w2 = 1; w2 < 4; ++w2) {
-          const uint2 o = flip_s[w2 * kMaxRank + k];
-          const float bo = __uint_as_float(o.x), bb = __uint_as_float(best.x);
-          if (bo > bb || (bo == bb && (o.y >> 1) < (best.y >> 1))) best = o;
-        }
-        neg_mask |= (best.y & 1u) << k;
+        const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
+#pragma unroll
+        for (int u = 0; u < kDL; ++u) us[(t0 + u) * kMaxRank + k] = sg * uacc[k][u];
       }
     }
-  }
-  uint8_t* rec8 = reinterpret_cast<uint8_t*>(a.stats) +
-                  ((item_bh * a.nb_cap) + item_j) * a.rec_bytes;
-  if (bt < D) {
-    uint16_t* rec = reinterpret_cast<uint16_t*>(rec8);
-    rec[bt] = float_to_bf16_bits(mu_d);
-    if (a.stats_format == 0) {
+    __syncwarp();
+    const int s_dim = a.sub_dim, s8 = a.sub_pad;
+    const float* basis = a.basis + int64_t(item_bh % a.hkv) * s_dim * D;
+    uint16_t* urow = rec + D;             // [r][s8] bf16
+    for (int i = lane; i < s8; i += 32) {
+      float acc[kMaxRank];
 #pragma unroll
-      for (int k = 0; k < kMaxRank; ++k) {
-        if (k < r) {
-          const float sg = ((neg_mask >> k) & 1u) ? -1.f : 1.f;
-          rec[int64_t(1 + k) * D + bt] = float_to_bf16_bits(sg * uacc[k]);
+      for (int k = 0; k < kMaxRank; ++k) acc[k] = 0.f;
+      if (i < s_dim) {
+        const float* prow = basis + int64_t(i) * D;
+#pragma unroll 2
+        for (int t = 0; t < D; t += 4) {
+          const float4 p4 = __ldg(reinterpret_cast<const float4*>(prow + t));
+          const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4* ut = reinterpret_cast<const float4*>(us + (t + q) * kMaxRank);
+#pragma unroll
+            for (int k4 = 0; k4 < kMaxRank / 4; ++k4) {
+              if (4 * k4 < r) {
+                const float4 u4 = ut[k4];
+                acc[4 * k4 + 0] = fmaf(pv[q], u4.x, acc[4 * k4 + 0]);
+                acc[4 * k4 + 1] = fmaf(pv[q], u4.y, acc[4 * k4 + 1]);
+                acc[4 * k4 + 2] = fmaf(pv[q], u4.z, acc[4 * k4 + 2]);
+                acc[4 * k4 + 3] = fmaf(pv[q], u4.w, acc[4 * k4 + 3]);
+              }
+            }
+          }
         }
       }
-    } else {
-      // FP4: warp w holds components [32w, 32w + 32) of every column, one
-      // scale group (D is a multiple of 32, so whole warps take this branch)
-      uint8_t* codes = rec8 + 2 * D;
-      uint8_t* scales = codes + r * (D / 2);
 #pragma unroll
-      for (int k = 0; k < kMaxRank; ++k) {
-        if (k < r) {
-          const float v = ((neg_mask >> k) & 1u) ? -uacc[k] : uacc[k];
-          const float amax = warp_max(fabsf(v));
-          const uint32_t code = fp4_code_scaled(v, amax);
-          // eight neighbouring lanes OR their nibbles into one 32-bit word
-          uint32_t word = code << (4 * (lane & 7));
-          word |= __shfl_xor_sync(0xffffffffu, word, 1);
-          word |= __shfl_xor_sync(0xffffffffu, word, 2);
-          word |= __shfl_xor_sync(0xffffffffu, word, 4);
-          if ((lane & 7) == 0)
-            *reinterpret_cast<uint32_t*>(codes + k * (D / 2) + bt / 2) = word;
-          if (lane == 0) scales[k * (D / 32) + bwarp] = uint8_t(fp4_scale_byte(amax));
-        }
+      for (int k = 0; k < kMaxRank; ++k)
+        if (k < r) urow[k * s8 + i] = float_to_bf16_bits(acc[k]);   // zeros past s
+    }
+  } else if (a.stats_format == 0) {
+#pragma unroll
+    for (int k = 0; k < kMaxRank; ++k) {
+      if (k < r) {
+        float v[kDL];
+#pragma unroll
+        for (int u = 0; u < kDL; ++u) v[u] = ((neg_mask >> k) & 1u) ? -uacc[k][u] : uacc[k][u];
+        store_bf16(rec + int64_t(1 + k) * D + t0, v);
       }
     }
-  }
-  // FP4 records end in zero padding up to a multiple of 16 bytes
-  if (a.stats_format != 0) {
+  } else {
+    // FP4: scale group g = dimensions [32 g, 32 g + 32) = the lanes
+    // [32 g / kDL, 32 (g + 1) / kDL) of the warp
+    constexpr int kGL = 32 / kDL;       // lanes per scale group
+    uint8_t* codes = rec8 + 2 * D;
+    uint8_t* scales = codes + r * (D / 2);
+#pragma unroll
+    for (int k = 0; k < kMaxRank; ++k) {
+      if (k < r) {
+        float v[kDL];
+        float amax = 0.f;
+#pragma unroll
+        for (int u = 0; u < kDL; ++u) {
+          v[u] = ((neg_mask >> k) & 1u) ? -uacc[k][u] : uacc[k][u];
+          amax = fmaxf(amax, fabsf(v[u]));
+        }
+#pragma unroll
+        for (int mm = kGL / 2; mm >= 1; mm >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, mm));
+        uint32_t word = 0;   // kDL codes, the lowest dimension in the low nibble
+#pragma unroll
+        for (int u = 0; u < kDL; ++u) word |= fp4_code_scaled(v[u], amax) << (4 * u);
+        if constexpr (kDL == 4)
+          *reinterpret_cast<uint16_t*>(codes + k * (D / 2) + t0 / 2) = uint16_t(word);
+        else
+          codes[k * (D / 2) + t0 / 2] = uint8_t(word);
+        if (lane % kGL == 0) scales[k * (D / 32) + lane / kGL] = uint8_t(fp4_scale_byte(amax));
+      }
+    }
+    // FP4 records end in zero padding up to a multiple of 16 bytes
     const int used = 2 * D + r * (D / 2) + r * (D / 32);
-    if (used + bt < a.rec_bytes) rec8[used + bt] = 0;
+    for (int e = used + lane; e < a.rec_bytes; e += 32) rec8[e] = 0;
   }
 }
 
 template <int D, int M>
 cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
-  using S = StatsShape<D>;
+  using S = StatsShape<D, M>;
   CUtensorMap map;
   const uint64_t rows = a.block_table != nullptr ? uint64_t(a.n_pages) * a.hkv * kBlock
                                                  : uint64_t(a.batch) * a.hkv * a.cap;
   cudaError_t e0 = make_bf16_tensor_map_sw128(&map, a.k, D, rows, 64);
   if (e0 != cudaSuccess) return e0;
   auto kern = block_stats_kernel<D, M>;
-  cudaError_t e =
-      set_smem_attrs(kern, int(S::kBytes));
+  cudaError_t e = set_smem_attrs(kern, int(S::kBytes));
   if (e != cudaSuccess) return e;
   const int64_t n_items = int64_t(a.batch) * a.hkv * (a.block_end - a.block_begin);
-  dim3 grid(unsigned(n_items), 1, 1);
+  dim3 grid(unsigned((n_items + kStatWarps - 1) / kStatWarps), 1, 1);
   return launch_pdl(kern, grid, dim3(kStatThreads), S::kBytes, stream, map, a);
 }
 
@@ -749,13 +858,13 @@ cudaError_t launch_stats_t(const StatsArgs& a, cudaStream_t stream) {
 cudaError_t launch_stats(const StatsArgs& a, cudaStream_t stream) {
   const int m = lanczos_steps(a.rank);
   if (a.d == 64) {
-    if (m == 28) return launch_stats_t<64, 28>(a, stream);
-    if (m == 36) return launch_stats_t<64, 36>(a, stream);
-    return launch_stats_t<64, 52>(a, stream);
+    if (m == 24) return launch_stats_t<64, 24>(a, stream);
+    if (m == 32) return launch_stats_t<64, 32>(a, stream);
+    return launch_stats_t<64, 44>(a, stream);
   }
-  if (m == 28) return launch_stats_t<128, 28>(a, stream);
-  if (m == 36) return launch_stats_t<128, 36>(a, stream);
-  return launch_stats_t<128, 52>(a, stream);
+  if (m == 24) return launch_stats_t<128, 24>(a, stream);
+  if (m == 32) return launch_stats_t<128, 32>(a, stream);
+  return launch_stats_t<128, 44>(a, stream);
 }
 
 }  // namespace cobs

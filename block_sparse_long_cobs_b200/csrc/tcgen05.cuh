@@ -193,4 +193,19 @@ cudaError_t make_bf16_tensor_map_3d_sw128(CUtensorMap* map, const void* base, in
                                           uint64_t rows, uint64_t depth,
                                           uint64_t depth_stride_bytes, int box_rows);
 
+// Host: 2-d tensor map over `rows` rows of `cols` bf16 values that start
+// `row_stride_bytes` apart (the first columns of wider records), box of 64
+// columns x box_rows rows, 128-byte swizzle.
+cudaError_t make_bf16_tensor_map_rows_sw128(CUtensorMap* map, const void* base, int cols,
+                                            uint64_t rows, uint64_t row_stride_bytes,
+                                            int box_rows);
+
+// Host: 3-d tensor map (cols, dim1, dim2) of bf16 with the given byte strides
+// of dims 1 and 2, box of 64 columns x box1 x box2, 128-byte swizzle; columns
+// at or past `cols` read as zero.
+cudaError_t make_bf16_tensor_map_3d_sw128_box(CUtensorMap* map, const void* base, int cols,
+                                              uint64_t dim1, uint64_t dim2,
+                                              uint64_t stride1_bytes, uint64_t stride2_bytes,
+                                              int box1, int box2);
+
 }  // namespace cobs

@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define COBS_ABI_VERSION 2
+#define COBS_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define COBS_API __attribute__((visibility("default")))
@@ -91,6 +91,8 @@ typedef enum cobs_status {
 /* Storage of a block record (cobs_dims.stats_format). */
 #define COBS_STATS_BF16 0    /* mu and U in bf16: (1 + r) x d x 2 bytes      */
 #define COBS_STATS_FP4 1     /* mu in bf16, U in scaled FP4 E2M1 (below)     */
+#define COBS_STATS_BOX 2     /* min/max box [lo; hi]: 2 x d x 2 bytes (below) */
+#define COBS_STATS_SUBSPACE 3 /* mu in bf16, U projected on a query subspace  */
 
 typedef struct cobs_dims {
   int32_t batch;             /* sequences in the batch                      */
@@ -100,7 +102,11 @@ typedef struct cobs_dims {
   int32_t block_size;        /* B (64)                                      */
   int32_t rank;              /* r, columns of the covariance factor U       */
   int64_t capacity_tokens;   /* cache length per (batch, kv-head)           */
-  int32_t stats_format;      /* COBS_STATS_BF16 (0) or COBS_STATS_FP4 (1)    */
+  int32_t stats_format;      /* COBS_STATS_BF16 (0), _FP4 (1), _BOX (2) or   */
+                             /* _SUBSPACE (3)                                */
+  int32_t subspace_dim;      /* s, for COBS_STATS_SUBSPACE (else unused)     */
+  const float* subspace_basis; /* device [Hkv][s][d] fp32, for                */
+                             /* COBS_STATS_SUBSPACE (else unused)            */
 } cobs_dims;
 
 /* FP4 block record (COBS explainer §2.3, quantisation: eigenvectors stored
@@ -122,6 +128,40 @@ typedef struct cobs_dims {
  * rounded to fp16's subnormal grid (an error of at most 2^-25 each); a scale
  * group whose exponent lies more than 23 below the largest of its column
  * (components under 2^-23 of the column's largest) counts as zero there. */
+
+/* Min/max box record (a comparison selector, not COBS: the explainer's
+ * plain-language summary lists estimating a block's spread from the minimum
+ * and maximum of its keys among the ideas that fall short of COBS; it gives
+ * no formula), cobs_stats_record_bytes() = 4 d bytes:
+ *   [0, 2d)     lo, the per-dimension minimum of the block's keys, bf16
+ *   [2d, 4d)    hi, the per-dimension maximum, bf16
+ * (exact: the minimum and maximum of bf16 values are bf16 values).  The rank
+ * field is not used.  cobs_build_block_stats writes box records when
+ * dims->stats_format is COBS_STATS_BOX, and cobs_select_blocks then scores a
+ * block by the largest logit any point of its box can reach,
+ *     s_b = ln n_b + sum_t max(q_t lo_t, q_t hi_t) / sqrt(d),
+ * an upper bound of the block's log attention mass; the group score, top-k,
+ * sink and local window are as for COBS records. */
+
+/* Subspace record (COBS explainer §2.3, subspace projection: the covariance
+ * is projected onto the subspace of the top eigenvectors of the queries'
+ * second moment, storage r d -> r s; §4.3: an adaptive s of about 85 of 128
+ * matches the full dimension), cobs_stats_record_bytes() = 2 d + 2 r s8
+ * bytes with s8 = s rounded up to a multiple of 8:
+ *   [0, 2d)                 mu, d bf16 values (the linear term keeps every
+ *                           dimension)
+ *   [2d, 2d + 2 r s8)       U_s = P^T U: row j holds the s coordinates of
+ *                           column j of U in the subspace, bf16, then zeros
+ *                           up to s8
+ * The basis P is dims->subspace_basis, device [num_kv_heads][s][d] fp32, row
+ * i of head h the i-th basis vector (unit, orthogonal to the others), 16-byte
+ * aligned, 1 <= s <= d; the caller computes it offline (e.g. the top
+ * eigenvectors of (1/n) sum q q^T over calibration queries) and it must stay
+ * the same between the statistics build and the selection.  The statistics
+ * build then writes U_s for each block; the selection scores
+ *     s_b = ln n_b + (q . mu_b) / sqrt(d) + 1/2 |U_s,b^T (P^T q)|^2 / d,
+ * P^T q computed in fp32 per step, so the quadratic term is the covariance's
+ * form at the projected query P P^T q. */
 
 /* Version of this ABI (COBS_ABI_VERSION). */
 COBS_API int32_t cobs_abi_version(void);
@@ -329,6 +369,16 @@ COBS_API cobs_status cobs_no_alloc_read_status(int32_t* device_status, void* str
  * clear it.  Returns CUDA on a failed copy, INVALID_ARG on bad pointers. */
 COBS_API cobs_status cobs_read_device_status(void* ws, size_t ws_bytes,
                                     int32_t* device_status, void* stream);
+
+/* Limit of the first bounded wait of the statistics kernel, for every later
+ * cobs_build_block_stats call of the process (a testing and diagnostic knob:
+ * it lets a test make a device wait run out without faulting or hanging
+ * anything).  0 restores the default of 2 s.  A wait that runs out records
+ * COBS_ERR_TIMEOUT in the workspace status word; the kernel then waits,
+ * with the full default limit, for the copies it already started, frees its
+ * tensor memory and returns without writing the records of its blocks.
+ * Initialise the workspace again (cobs_workspace_init) after such a call. */
+COBS_API cobs_status cobs_set_wait_limit_ns(uint64_t limit_ns);
 
 /* Message for the last error returned on this thread ("" if none). */
 COBS_API const char* cobs_last_error(void);

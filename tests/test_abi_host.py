@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) == 17, names
+    assert len(names) == 18, names
     raw = ctypes.CDLL(cb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert cb.cobs_abi_version() == 2
+    assert cb.cobs_abi_version() == 3
     assert cb.cobs_status_string(0) == "COBS_OK"
     assert cb.cobs_status_string(5) == "COBS_ERR_TIMEOUT"
     assert cb.cobs_status_string(99) == "COBS_ERR_UNKNOWN"
@@ -248,8 +248,14 @@ def test_stats_record_bytes_and_format_checks():
     # d 128, r 8: 256 B of mu, 512 B of codes, 32 scale bytes
     assert cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], rank=8,
                                               stats_format=1)) == 800
+    # min/max box records: lo and hi, d bf16 each, whatever the rank
+    for r in (0, 8, 16):
+        assert cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], rank=r,
+                                                  stats_format=cb.COBS_STATS_BOX)) == 512
+    assert cb.cobs_stats_record_bytes(dims_of(WORKLOADS["tiny_4k"],
+                                              stats_format=cb.COBS_STATS_BOX)) == 256
     with pytest.raises(cb.CobsError) as e:
-        cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], stats_format=2))
+        cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], stats_format=3))
     assert e.value.status == cb.COBS_ERR_INVALID_ARG
     with pytest.raises(cb.CobsError):
         cb.cobs_stats_record_bytes(dims_of(WORKLOADS["single_32k"], rank=0, stats_format=1))
@@ -299,3 +305,36 @@ def test_binding_rejects_host_and_strided_tensors():
     assert not strided.is_contiguous()
     with pytest.raises(TypeError):
         cb.cobs_build_block_stats(d, strided, 0, 1, 1 << 20, 1 << 20, 4096)
+
+
+def test_subspace_dims_checks():
+    """Subspace records (COBS_STATS_SUBSPACE): record size 2 d + 2 r s8 bytes
+    (s8 = s rounded up to 8); s in [1, d], an aligned basis and rank >= 1 are
+    required, checked before anything is launched."""
+    w = WORKLOADS["single_32k"]
+    A = 1 << 20
+    base = dims_of(w, stats_format=cb.COBS_STATS_SUBSPACE, subspace_basis=A)
+    for s, want in ((85, 256 + 2 * 8 * 88), (64, 256 + 2 * 8 * 64), (1, 256 + 2 * 8 * 8),
+                    (128, 9 * 256)):
+        assert cb.cobs_stats_record_bytes(dict(base, subspace_dim=s)) == want
+    assert cb.cobs_stats_record_bytes(dims_of(WORKLOADS["tiny_4k"], rank=4, subspace_dim=40,
+                                              stats_format=cb.COBS_STATS_SUBSPACE,
+                                              subspace_basis=A)) == 128 + 2 * 4 * 40
+    for bad, code in ((dict(subspace_dim=0), cb.COBS_ERR_INVALID_ARG),
+                      (dict(subspace_dim=129), cb.COBS_ERR_INVALID_ARG),
+                      (dict(subspace_dim=85, subspace_basis=None), cb.COBS_ERR_INVALID_ARG),
+                      (dict(subspace_dim=85, subspace_basis=A + 4), cb.COBS_ERR_INVALID_ARG),
+                      (dict(subspace_dim=85, rank=0), cb.COBS_ERR_UNSUPPORTED)):
+        d = dict(base, **bad)
+        with pytest.raises(cb.CobsError):        # a size query only says "invalid"
+            cb.cobs_stats_record_bytes(d)
+        with pytest.raises(cb.CobsError) as e:
+            cb.cobs_build_block_stats(d, A, 0, 1, A, A, 4096)
+        assert e.value.status == code, bad
+    # the other formats ignore the subspace fields
+    assert cb.cobs_stats_record_bytes(dims_of(w, subspace_dim=999)) == 9 * 256
+
+
+def test_wait_limit_knob():
+    assert cb.cobs_set_wait_limit_ns(5_000_000) == cb.COBS_OK
+    assert cb.cobs_set_wait_limit_ns(0) == cb.COBS_OK     # back to the default
