@@ -242,12 +242,20 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       for (int p = 0; p < npass; ++p) {
         const int buf = p & 1, st = p % kRaw;
         uint8_t* atile = tiles + buf * kStageBytes;
-        // the tile of pass p - 2 is free once its products are complete
+        // the tile of pass p - 2 is free once its products are complete; one
+        // thread waits (spinning threads would take issue slots from the
+        // epilogue warps), the others take the result from the barrier
         bool fail = abort_s != 0;
-        if (!fail && p >= 2)
-          fail = !wait_or_abort(&mma_done[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
-        if (!fail) fail = !wait_or_abort(&raw_full[st], (p / kRaw) & 1, a.status, &abort_s);
+        if (tid == 0) {
+          if (!fail && p >= 2)
+            fail = !wait_or_abort(&mma_done[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
+          if (!fail) fail = !wait_or_abort(&raw_full[st], (p / kRaw) & 1, a.status, &abort_s);
+        }
         if (named_bar_or(1, 128, fail)) break;
+        if (tid != 0) {
+          (void)mbar_try_wait(&raw_full[st], (p / kRaw) & 1);   // acquire the copy
+          if (p >= 2) (void)mbar_try_wait(&mma_done[buf], ((p - 2) >> 1) & 1);
+        }
         const int j0 = c_lo + p * per_pass;
         const int nb = min(per_pass, c_hi - j0);
         const uint8_t* rs = raw + st * raw_bytes;

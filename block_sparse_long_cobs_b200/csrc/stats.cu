@@ -14,8 +14,7 @@
 //      per tile.  One tcgen05.mma chain per tile (kind::f16, M = N = 128,
 //      bf16 in, fp32 accumulate in tensor memory) forms [K_a; K_b][K_a; K_b]^T,
 //      whose diagonal 64 x 64 quadrants are the raw Grams G = K K^T of the two
-//      blocks (products of bf16 values are exact in fp32).  The block means
-//      are summed from the tiles meanwhile.
+//      blocks (products of bf16 values are exact in fp32).
 //   2. The Gram rows come back from tensor memory (each warp reads its 32
 //      lanes), go through shared memory to the warp that owns the block, and
 //      are centred in fp32: Gc = G - r 1^T - 1 r^T + s 1 1^T with r = G 1 / n,
@@ -23,10 +22,10 @@
 //      rows l and l + 32 of Gc in registers.
 //   3. Lanczos on A = Gc^2 (applied as two products with Gc; same eigenvectors,
 //      squared eigenvalues, so the top of the spectrum separates faster), M =
-//      24 / 32 / 44 steps for r <= 4 / <= 8 / <= 16, every new vector
-//      orthogonalised twice against all earlier ones by classical
-//      Gram-Schmidt, a fresh pseudo-random vector whenever the Krylov space
-//      closes.  The warp works alone: its only synchronisation is __syncwarp,
+//      24 / 32 / 44 steps for r <= 4 / <= 8 / <= 16: the three-term step
+//      against q_j and q_{j-1}, then one classical Gram-Schmidt pass against
+//      every earlier vector (full re-orthogonalisation), a fresh
+//      pseudo-random vector whenever the Krylov space closes.  The warp works alone: its only synchronisation is __syncwarp,
 //      vectors pass through its own shared-memory rows (basis kept row- and
 //      column-major so both Gram-Schmidt phases are 128-bit loads).
 //   4. Top-r eigenvalues of the M x M tridiagonal T by multisection bisection
@@ -34,10 +33,12 @@
 //      each), eigenvectors z_k by inverse iteration (LDL^T of T - theta I, in
 //      registers), re-orthogonalised inside clusters of close eigenvalues;
 //      Ritz vectors w_k = Q z_k are unit eigenvectors of Gc.
-//   5. U[:, k] = Kc^T w_k / sqrt(n) (its squared norm is the covariance
-//      eigenvalue), keys re-read through L2 (lane l owns d/32 consecutive
-//      dimensions), sign fixed so that the largest-magnitude component is
-//      positive; written with mu as a bf16 or an FP4 record.
+//   5. One pass over the keys (re-read through L2, lane l owns d/32
+//      consecutive dimensions) gives mu and K^T W; U[:, k] = Kc^T w_k / sqrt(n)
+//      = (K^T w_k - mu (1^T w_k)) / sqrt(n) (its squared norm is the
+//      covariance eigenvalue), sign fixed so that the largest-magnitude
+//      component is positive; written with mu as a bf16, FP4 or subspace
+//      record.
 #include <cfloat>
 #include <cuda.h>
 
@@ -76,8 +77,7 @@ struct StatsShape {
   static constexpr int kR1 = kR1a > kStatWarps * kWarpQBytes ? kR1a : kStatWarps * kWarpQBytes;
   static constexpr int kVecFloats = 64 * 3 + 48 * 3 + 16;  // x, w, h, alpha, beta, beta^2, lambda
   static constexpr size_t kVec = kR1;
-  static constexpr size_t kMu = kVec + size_t(kStatWarps) * kVecFloats * 4;   // [4][D]
-  static constexpr size_t kRowSum = kMu + size_t(kStatWarps) * D * 4;         // [4][64]
+  static constexpr size_t kRowSum = kVec + size_t(kStatWarps) * kVecFloats * 4;   // [4][64]
   static constexpr size_t kBar = kRowSum + size_t(kStatWarps) * 64 * 4;
   static constexpr size_t kMisc = kBar + 16;
   static constexpr size_t kBytes = kMisc + 64 + 1024;      // + alignment slack
@@ -110,23 +110,26 @@ __device__ __forceinline__ float pivot_guard(float d) {
   return fabsf(d) < 1e-30f ? (d < 0.f ? -1e-30f : 1e-30f) : d;
 }
 
-// Numbers of eigenvalues of the M x M tridiagonal T (diag al, off-diag^2 b2,
-// both in registers) below three shifts: negative pivots of LDL^T of T - x I,
-// the three recurrences interleaved so their latencies overlap.
+// Numbers of eigenvalues of the M x M tridiagonal T (diagonal al, squared
+// off-diagonal b2, both in shared memory) below three shifts: negative pivots
+// of LDL^T of T - x I, the three recurrences interleaved so their latencies
+// overlap.  The loop is kept rolled (by 4) so the code stays small.
 template <int M>
-__device__ __forceinline__ void sturm_count3(const float (&al)[M], const float (&b2)[M],
+__device__ __forceinline__ void sturm_count3(const float* al, const float* b2,
                                              const float (&x)[3], int (&c)[3]) {
   float d[3];
+  const float a0 = al[0];
 #pragma unroll
   for (int s = 0; s < 3; ++s) {
-    d[s] = al[0] - x[s];
+    d[s] = a0 - x[s];
     c[s] = d[s] < 0.f;
   }
-#pragma unroll
+#pragma unroll 4
   for (int i = 1; i < M; ++i) {
+    const float ai = al[i], bi = b2[i - 1];
 #pragma unroll
     for (int s = 0; s < 3; ++s) {
-      d[s] = al[i] - x[s] - __fdividef(b2[i - 1], pivot_guard(d[s]));
+      d[s] = ai - x[s] - __fdividef(bi, pivot_guard(d[s]));
       c[s] += d[s] < 0.f;
     }
   }
@@ -226,7 +229,6 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   const int64_t item_bh = has_item ? item / nb_range : 0;
   const int64_t item_j = has_item ? a.block_begin + item % nb_range : 0;
 
-  float* mus = reinterpret_cast<float*>(smem + S::kMu) + warp * D;
   float* rowsum = reinterpret_cast<float*>(smem + S::kRowSum);
   float* V = reinterpret_cast<float*>(smem + S::kVec) + warp * S::kVecFloats;
   float* Qs = reinterpret_cast<float*>(smem + warp * S::kWarpQBytes);
@@ -301,22 +303,6 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   }
   __syncthreads();
   bool aborted = *abort_s != 0;
-  if (!aborted) (void)mbar_try_wait(&bars[0], 0);   // acquire the TMA writes
-  // block means (fp32 sums of 64 bf16 keys) while the products run: warp w
-  // sums the columns of its own block
-  if (!aborted && valid) {
-    const uint8_t* tile = smem + (warp >> 1) * S::kTileBytes;
-    const int rbase = (warp & 1) * 64;
-    for (int c = lane; c < D; c += 32) {
-      float acc = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < kBlock; ++t) {
-        const uint16_t w16 = *reinterpret_cast<const uint16_t*>(tile + k_offset<D>(rbase + t, c));
-        acc += __uint_as_float(uint32_t(w16) << 16);
-      }
-      mus[c] = acc * (1.f / 64.f);
-    }
-  }
   if (tid == 0 && !aborted) {
     const bool ok = mbar_wait_bounded(&bars[1], 0, a.status);
     if (!ok) {
@@ -324,7 +310,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       *abort_s = 1u;
     }
   }
-  __syncthreads();           // means done (the key tiles may be overwritten), MMA done
+  __syncthreads();           // products done: the key tiles may be overwritten
   aborted = *abort_s != 0;
   if (!aborted) {
     if (tid != 0) (void)mbar_try_wait(&bars[1], 0);
@@ -414,55 +400,44 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     }
     __syncwarp();
 
-    // Orthogonalise (w0, w1) against basis rows 0..jmax, twice.  Returns the
-    // summed coefficient of q_jmax and |w|^2 at the end.
-    auto cgs = [&](float& w0, float& w1, int jmax, float& sq) -> float {
-      float acoef = 0.f;
-      float n1 = 0.f, hh2 = 0.f;
+    // One classical Gram-Schmidt pass of (w0, w1) against basis rows
+    // 0..jmax; returns the coefficient of q_jmax.
+    auto cgs_pass = [&](float& w0, float& w1, int jmax) -> float {
       const int nc = (jmax >> 2) + 1;   // 4-wide chunks of coefficients
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        wv[lA] = w0;
-        wv[lB] = w1;
-        __syncwarp();
-        float ha = 0.f, hb = 0.f;
-        if (lA <= jmax) ha = smem_dot64(Qs + lA * kQStride, wv);
-        if (lB <= jmax) hb = smem_dot64(Qs + lB * kQStride, wv);
-        if (pass == 1) {
-          hh2 = warp_sum(ha * ha + hb * hb);
-        }
-        hv[lA] = ha;
-        hv[lB] = hb;
-        __syncwarp();
-        const float* qa = QTs + lA * S::kQTStride;
-        const float* qb = QTs + lB * S::kQTStride;
-        float c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
-        constexpr int kMaxChunks = M / 4;
+      wv[lA] = w0;
+      wv[lB] = w1;
+      __syncwarp();
+      float ha = 0.f, hb = 0.f;
+      if (lA <= jmax) ha = smem_dot64(Qs + lA * kQStride, wv);
+      if (lB <= jmax) hb = smem_dot64(Qs + lB * kQStride, wv);
+      hv[lA] = ha;
+      hv[lB] = hb;
+      __syncwarp();
+      const float* qa = QTs + lA * S::kQTStride;
+      const float* qb = QTs + lB * S::kQTStride;
+      float c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
+      constexpr int kMaxChunks = M / 4;
 #pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-          if (c < nc) {
-            const float4 h4 = *reinterpret_cast<const float4*>(hv + 4 * c);
-            const float4 x = *reinterpret_cast<const float4*>(qa + 4 * c);
-            const float4 y = *reinterpret_cast<const float4*>(qb + 4 * c);
-            c0 = fmaf(x.x, h4.x, fmaf(x.y, h4.y, c0));
-            c1 = fmaf(x.z, h4.z, fmaf(x.w, h4.w, c1));
-            d0 = fmaf(y.x, h4.x, fmaf(y.y, h4.y, d0));
-            d1 = fmaf(y.z, h4.z, fmaf(y.w, h4.w, d1));
-          }
+      for (int c = 0; c < kMaxChunks; ++c) {
+        if (c < nc) {
+          const float4 h4 = *reinterpret_cast<const float4*>(hv + 4 * c);
+          const float4 x = *reinterpret_cast<const float4*>(qa + 4 * c);
+          const float4 y = *reinterpret_cast<const float4*>(qb + 4 * c);
+          c0 = fmaf(x.x, h4.x, fmaf(x.y, h4.y, c0));
+          c1 = fmaf(x.z, h4.z, fmaf(x.w, h4.w, c1));
+          d0 = fmaf(y.x, h4.x, fmaf(y.y, h4.y, d0));
+          d1 = fmaf(y.z, h4.z, fmaf(y.w, h4.w, d1));
         }
-        w0 -= c0 + c1;
-        w1 -= d0 + d1;
-        acoef += hv[jmax];
-        if (pass == 0) n1 = warp_sum(w0 * w0 + w1 * w1);
-        __syncwarp();   // hv and wv are rewritten by the next pass
       }
-      // |w2|^2 = |w1|^2 - |h2|^2 for an orthonormal basis; when the second
-      // pass removed much of w1 the difference cancels, so sum exactly then
-      if (hh2 > 0.25f * n1) sq = warp_sum(w0 * w0 + w1 * w1);
-      else sq = fmaxf(n1 - hh2, 0.f);
-      return acoef;
+      w0 -= c0 + c1;
+      w1 -= d0 + d1;
+      const float coef = hv[jmax];
+      __syncwarp();   // hv and wv are rewritten by the next pass
+      return coef;
     };
 
+    // this lane's entries of q_j and q_{j-1}
+    float qa_j = Qs[lA], qb_j = Qs[lB], qa_p = 0.f, qb_p = 0.f, beta_p = 0.f;
 #pragma unroll 1
     for (int j = 0; j < M; ++j) {
       // w = Gc (Gc q_j)
@@ -470,20 +445,30 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       const float y0 = row_dot(g0, qj), y1 = row_dot(g1, qj);
       xv[lA] = y0;
       xv[lB] = y1;
+      // alpha_j = q_j^T Gc^2 q_j = |Gc q_j|^2: its reduction overlaps the
+      // second product
+      float aj = warp_sum(y0 * y0 + y1 * y1);
       __syncwarp();
       float w0 = row_dot(g0, xv), w1 = row_dot(g1, xv);
-      float sq = 0.f;
-      const float aj = cgs(w0, w1, j, sq);
-      float beta = sqrtf(sq);
+      // the local three-term step removes the large components along q_j and
+      // q_{j-1} exactly; one full Gram-Schmidt pass then removes what
+      // rounding left along every basis vector (as accurate as two full
+      // passes, including on exactly rank-deficient blocks, in fp32
+      // emulation on the workloads' spectra)
+      w0 -= aj * qa_j + beta_p * qa_p;
+      w1 -= aj * qb_j + beta_p * qb_p;
+      aj += cgs_pass(w0, w1, j);
+      float beta = sqrtf(warp_sum(w0 * w0 + w1 * w1));
       if (lane == 0) V[kVAlpha + j] = aj;
       if (j == M - 1) break;
       if (!(beta > tol)) {
-        // the Krylov space closed: continue from a fresh vector
+        // the Krylov space closed: continue from a fresh vector, made
+        // orthogonal to the basis by two passes
         w0 = hash_sign(uint32_t(j + 1), uint32_t(lA));
         w1 = hash_sign(uint32_t(j + 1), uint32_t(lB));
-        float sq2 = 0.f;
-        cgs(w0, w1, j, sq2);
-        sq2 = warp_sum(w0 * w0 + w1 * w1);
+        (void)cgs_pass(w0, w1, j);
+        (void)cgs_pass(w0, w1, j);
+        const float sq2 = warp_sum(w0 * w0 + w1 * w1);
         const float inv = sq2 > 0.f ? rsqrtf(sq2) : 0.f;
         w0 *= inv;
         w1 *= inv;
@@ -501,6 +486,11 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       Qs[(j + 1) * kQStride + lB] = w1;
       QTs[lA * S::kQTStride + j + 1] = w0;
       QTs[lB * S::kQTStride + j + 1] = w1;
+      qa_p = qa_j;
+      qb_p = qb_j;
+      qa_j = w0;
+      qb_j = w1;
+      beta_p = beta;
       __syncwarp();
     }
     __syncwarp();
@@ -508,19 +498,13 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     // ---- 4. top-r eigenpairs of T ---------------------------------------------
     const float* alpha = V + kVAlpha;
     const float* betav = V + kVBeta;
-    float al[M], b2[M];
-#pragma unroll
-    for (int i2 = 0; i2 < M; ++i2) {
-      al[i2] = alpha[i2];
-      b2[i2] = V[kVBeta2 + i2];
-    }
     float lo = 0.f, hi = 0.f;
-#pragma unroll
+#pragma unroll 4
     for (int i2 = 0; i2 < M; ++i2) {
       const float rad =
           (i2 > 0 ? fabsf(betav[i2 - 1]) : 0.f) + (i2 < M - 1 ? fabsf(betav[i2]) : 0.f);
-      lo = fminf(lo, al[i2] - rad);
-      hi = fmaxf(hi, al[i2] + rad);
+      lo = fminf(lo, alpha[i2] - rad);
+      hi = fmaxf(hi, alpha[i2] + rad);
     }
     hi = hi * (1.f + 1e-6f) + 1e-30f;
     lo = lo - 1e-6f * fabsf(hi) - 1e-30f;
@@ -529,7 +513,8 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
     const int lpe = 32 / rp;                    // lanes of one eigenvalue
     const int kk = lane / lpe, sub = lane % lpe;
     const int npts = 3 * lpe;                   // shifts per eigenvalue per round
-    const int rounds = lpe >= 8 ? 5 : (lpe >= 4 ? 6 : (lpe >= 2 ? 8 : 12));
+    // (3 lpe + 1)-way splits: enough rounds for ~4e-6 of the spectral width
+    const int rounds = lpe >= 16 ? 3 : (lpe >= 8 ? 4 : (lpe >= 4 ? 5 : 7));
     const int target = M - 1 - kk;              // count(x) <= target below it
     float ea = lo, eb = hi;
     for (int it = 0; it < rounds; ++it) {
@@ -538,7 +523,7 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       int cs[3];
 #pragma unroll
       for (int s2 = 0; s2 < 3; ++s2) xs[s2] = ea + step * float(3 * sub + s2 + 1);
-      sturm_count3<M>(al, b2, xs, cs);
+      sturm_count3<M>(alpha, V + kVBeta2, xs, cs);
       // first point of this eigenvalue's group whose count exceeds target
       const int sh = kk * lpe;
       const uint32_t gmask = lpe == 32 ? 0xffffffffu : (((1u << lpe) - 1u) << sh);
@@ -563,13 +548,13 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
       const float th = V[kVLam + lane];
       float l[M], rd[M];
       {
-        float d = pivot_guard(al[0] - th);
+        float d = pivot_guard(alpha[0] - th);
         rd[0] = 1.f / d;
         l[0] = 0.f;
 #pragma unroll
         for (int i2 = 1; i2 < M; ++i2) {
           l[i2] = betav[i2 - 1] * rd[i2 - 1];
-          d = pivot_guard(al[i2] - th - l[i2] * betav[i2 - 1]);
+          d = pivot_guard(alpha[i2] - th - l[i2] * betav[i2 - 1]);
           rd[i2] = 1.f / d;
         }
       }
@@ -656,49 +641,77 @@ block_stats_kernel(const __grid_constant__ CUtensorMap kmap, const StatsArgs a) 
   }
   if (!valid) return;        // no more CTA-wide barriers below
 
-  // ---- 5. U = Kc^T w / sqrt(n), sign rule, record ----------------------------
-  // lane l owns dimensions [kDL l, kDL l + kDL); keys re-read through L2
+  // ---- 5. mu, U = Kc^T w / sqrt(n), sign rule, record --------------------------
+  // lane l owns dimensions [kDL l, kDL l + kDL); keys re-read through L2, 16
+  // rows in flight at a time.  One pass gives the key sums (mu) and K^T W;
+  // U = K^T W - mu (1^T W) (the Ritz vectors are orthogonal to 1, so the
+  // correction is tiny and nothing cancels)
   const uint16_t* kglob = a.k + row0 * D;
   const int t0 = kDL * lane;
-  float mu_l[kDL];
+  float ksum[kDL];
 #pragma unroll
-  for (int u = 0; u < kDL; ++u) mu_l[u] = mus[t0 + u];
+  for (int u = 0; u < kDL; ++u) ksum[u] = 0.f;
+  float wsum[kMaxRank];
   float uacc[kMaxRank][kDL];
 #pragma unroll
-  for (int k = 0; k < kMaxRank; ++k)
+  for (int k = 0; k < kMaxRank; ++k) {
+    wsum[k] = 0.f;
 #pragma unroll
     for (int u = 0; u < kDL; ++u) uacc[k][u] = 0.f;
-  if (do_eig) {
-#pragma unroll 2
-    for (int t = 0; t < kBlock; ++t) {
-      float kc[kDL];
-      if constexpr (kDL == 4) {
-        const uint2 w2 = *reinterpret_cast<const uint2*>(kglob + int64_t(t) * D + t0);
-        const float2 f0 = bf16x2_to_float2(w2.x), f1 = bf16x2_to_float2(w2.y);
-        kc[0] = f0.x - mu_l[0];
-        kc[1] = f0.y - mu_l[1];
-        kc[2] = f1.x - mu_l[2];
-        kc[3] = f1.y - mu_l[3];
-      } else {
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kglob + int64_t(t) * D + t0);
-        const float2 f0 = bf16x2_to_float2(w1);
-        kc[0] = f0.x - mu_l[0];
-        kc[1] = f0.y - mu_l[1];
+  }
+  {
+    constexpr int kRows = 16;
+#pragma unroll 1
+    for (int t0r = 0; t0r < kBlock; t0r += kRows) {
+      uint32_t kw[kRows][kDL / 2];
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        if constexpr (kDL == 4) {
+          const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(kglob + int64_t(t0r + i) * D + t0));
+          kw[i][0] = w2.x;
+          kw[i][1] = w2.y;
+        } else {
+          kw[i][0] = __ldg(reinterpret_cast<const uint32_t*>(kglob + int64_t(t0r + i) * D + t0));
+        }
       }
-      const float4* wt = reinterpret_cast<const float4*>(Ws + t * kMaxRank);
 #pragma unroll
-      for (int k4 = 0; k4 < kMaxRank / 4; ++k4) {
-        if (4 * k4 < r) {
-          const float4 u4 = wt[k4];
-          const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+      for (int i = 0; i < kRows; ++i) {
+        float kv[kDL];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+        for (int u = 0; u < kDL; u += 2) {
+          const float2 f = bf16x2_to_float2(kw[i][u >> 1]);
+          kv[u] = f.x;
+          kv[u + 1] = f.y;
+        }
 #pragma unroll
-            for (int u = 0; u < kDL; ++u) uacc[4 * k4 + q][u] = fmaf(kc[u], uu[q], uacc[4 * k4 + q][u]);
+        for (int u = 0; u < kDL; ++u) ksum[u] += kv[u];
+        if (do_eig) {
+          const float4* wt = reinterpret_cast<const float4*>(Ws + (t0r + i) * kMaxRank);
+#pragma unroll
+          for (int k4 = 0; k4 < kMaxRank / 4; ++k4) {
+            if (4 * k4 < r) {
+              const float4 u4 = wt[k4];
+              const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                wsum[4 * k4 + q] += uu[q];
+#pragma unroll
+                for (int u = 0; u < kDL; ++u)
+                  uacc[4 * k4 + q][u] = fmaf(kv[u], uu[q], uacc[4 * k4 + q][u]);
+              }
+            }
+          }
         }
       }
     }
   }
+  float mu_l[kDL];
+#pragma unroll
+  for (int u = 0; u < kDL; ++u) mu_l[u] = ksum[u] * (1.f / 64.f);
+#pragma unroll
+  for (int k = 0; k < kMaxRank; ++k)
+#pragma unroll
+    for (int u = 0; u < kDL; ++u) uacc[k][u] = fmaf(-mu_l[u], wsum[k], uacc[k][u]);
   // sign: the component of largest magnitude (lowest index on ties) is positive
   uint32_t neg_mask = 0;
 #pragma unroll
