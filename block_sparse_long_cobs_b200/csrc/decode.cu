@@ -351,17 +351,22 @@ sparse_decode_kernel(const DecodeArgs a) {
     const int h = e / D, dd = e % D;
     const int64_t hq = int64_t(b) * a.hq + kvh * G + h;
     const float* base = a.partials + hq * part_row;
+    // independent loads: unrolled so that many L2 requests are in flight
     float M = -INFINITY;
+#pragma unroll 8
     for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, __ldcg(base + int64_t(s) * (D + 2) + D));
     float L = 0.f, O = 0.f;
     if (M != -INFINITY) {
+#pragma unroll 8
       for (int s = 0; s < a.n_splits; ++s) {
         const float* prow = base + int64_t(s) * (D + 2);
         const float ms = __ldcg(prow + D);
-        if (ms == -INFINITY) continue;
-        const float w = hw_exp2(ms - M);
-        L += w * __ldcg(prow + D + 1);
-        O += w * __ldcg(prow + dd);
+        const float ls = __ldcg(prow + D + 1);
+        const float os = __ldcg(prow + dd);
+        const bool live = ms != -INFINITY;   // a split with no valid key
+        const float w = live ? hw_exp2(ms - M) : 0.f;
+        L = live ? fmaf(w, ls, L) : L;
+        O = live ? fmaf(w, os, O) : O;
       }
     }
     a.out[hq * D + dd] = (L > 0.f) ? O / L : 0.f;

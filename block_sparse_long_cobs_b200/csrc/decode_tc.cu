@@ -70,6 +70,7 @@ constexpr int kOffP = kOffQ + 2 * 2048;
 constexpr int kDynSmem = kOffP + kPSlots * kPSlotBytes + 1024;
 
 static_assert(kOCol + 32 <= kTmemCols, "TMEM columns");
+static_assert(kSoftThreads == kD, "the merge gives thread r output dimension r");
 // The query buffer of segment n is reloaded for segment n + 2 once ring item
 // (issue count - kStages) is free; every segment has >= 2 items (a K and a V
 // tile), so with kStages <= 4 that item is at or after segment n's last one,
@@ -436,22 +437,32 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       named_bar(1, kSoftThreads);
       if (last_s) {
         __threadfence();
-        for (int e = r; e < G * kD; e += kSoftThreads) {
-          const int h = e / kD, dd = e % kD;
+        // thread r merges output dimension r of every head; the loads of the
+        // segments are independent, so the loops are unrolled to keep many
+        // L2 requests in flight (one at a time cost a round trip each)
+        const int nseg = sg.n_seg;
+        const int dd = r;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
           const int64_t hq = hq0 + h;
           const float* pbase = a.partials + hq * hstride;
           float M = -INFINITY;
-          for (int s = 0; s < sg.n_seg; ++s)
+#pragma unroll 8
+          for (int s = 0; s < nseg; ++s)
             M = fmaxf(M, __ldcg(pbase + int64_t(s) * (kD + 2) + kD));
           float L = 0.f, O = 0.f;
           if (M != -INFINITY) {
-            for (int s = 0; s < sg.n_seg; ++s) {
+#pragma unroll 8
+            for (int s = 0; s < nseg; ++s) {
               const float* prow = pbase + int64_t(s) * (kD + 2);
               const float ms = __ldcg(prow + kD);
-              if (ms == -INFINITY) continue;
-              const float w = hw_exp2(ms - M);
-              L += w * __ldcg(prow + kD + 1);
-              O += w * __ldcg(prow + dd);
+              const float ls = __ldcg(prow + kD + 1);
+              const float os = __ldcg(prow + dd);
+              // a segment with no valid key (m = -inf) has no output row
+              const bool live = ms != -INFINITY;
+              const float w = live ? hw_exp2(ms - M) : 0.f;
+              L = live ? fmaf(w, ls, L) : L;
+              O = live ? fmaf(w, os, O) : O;
             }
           }
           a.out[hq * kD + dd] = (L > 0.f) ? O / L : 0.f;
