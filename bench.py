@@ -459,6 +459,31 @@ def run_cobs(args, w, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     build_ms = e0.elapsed_time(e1)
 
+    # a workload built by appends: the statistics build of one appended chunk
+    # (append_chunk / 64 blocks of every (batch, kv-head)), L2 flushed before
+    # each of 20 timed builds
+    append = None
+    if w.append_chunk:
+        per = w.append_chunk // w.block
+        j0 = max(0, nfull - 1 - per)
+        flush_a = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        times = []
+        for i in range(23):
+            flush_a.zero_()
+            e0.record(stream)
+            cb.cobs_build_block_stats(dims, k, j0, j0 + per, stats, ws, ws_bytes, stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                times.append(e0.elapsed_time(e1))
+        del flush_a
+        t_app = statistics.median(times)
+        heads = w.batch * w.kv_heads * per
+        append = {"tokens": w.append_chunk, "block_heads": heads, "ms": t_app,
+                  "gbs": heads * (w.block * w.head_dim * 2 + rec_bytes) / (t_app * 1e-3) / 1e9,
+                  "note": "statistics build of one appended chunk, median of 20 launches "
+                          "after an L2 flush"}
+
     side = torch.cuda.Stream(dev) if args.stats_stream == "side" else None
     fork_ev, join_ev = torch.cuda.Event(), torch.cuda.Event()
 
@@ -752,6 +777,7 @@ def run_cobs(args, w, rank, world, local_rank):
                       "steps without it)",
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,
+        **({"append_chunk_build": append} if append is not None else {}),
         "wall_ms_per_step": t_host,
         "quality": quality,
         "step_variants": {

@@ -245,12 +245,11 @@ DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride) {
     // 32k workload took 45 us whole, 61 us as halves), so pairs are split only
     // as far as the resident CTAs can still take every chunk in one wave (a
     // second, partial wave doubles the time of the CTAs that run it), with at
-    // least 4 slots (two 128-key tiles) per chunk: on problems with few pairs
-    // the CTAs are otherwise idle, and the merge issues the loads of all
-    // partials together, so more partials cost little.
+    // least 8 slots per chunk (smaller chunks lost on the latency-bound
+    // small problems: more partials to merge).
     const int64_t resident = int64_t(sms) * decode_tc_ctas_per_sm(g);
     int64_t per_pair = resident / pairs;
-    const int64_t max_per_pair = ceil_div(idx_stride, 4);
+    const int64_t max_per_pair = ceil_div(idx_stride, 8);
     if (per_pair > max_per_pair) per_pair = max_per_pair;
     if (per_pair < 1) per_pair = 1;
     P.chunk_slots = int32_t(ceil_div(idx_stride, per_pair));

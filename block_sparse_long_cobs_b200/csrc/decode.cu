@@ -351,22 +351,29 @@ sparse_decode_kernel(const DecodeArgs a) {
     const int h = e / D, dd = e % D;
     const int64_t hq = int64_t(b) * a.hq + kvh * G + h;
     const float* base = a.partials + hq * part_row;
-    // independent loads: unrolled so that many L2 requests are in flight
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, __ldcg(base + int64_t(s) * (D + 2) + D));
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 8
-      for (int s = 0; s < a.n_splits; ++s) {
-        const float* prow = base + int64_t(s) * (D + 2);
-        const float ms = __ldcg(prow + D);
-        const float ls = __ldcg(prow + D + 1);
-        const float os = __ldcg(prow + dd);
-        const bool live = ms != -INFINITY;   // a split with no valid key
-        const float w = live ? hw_exp2(ms - M) : 0.f;
-        L = live ? fmaf(w, ls, L) : L;
-        O = live ? fmaf(w, os, O) : O;
+    // one pass with a running maximum; the loads of 8 splits are issued
+    // together so that many L2 requests are in flight
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    for (int s0 = 0; s0 < a.n_splits; s0 += 8) {
+      float ms[8], ls[8], os[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const bool in = s0 + u < a.n_splits;
+        const float* prow = base + int64_t(s0 + u) * (D + 2);
+        ms[u] = in ? __ldcg(prow + D) : -INFINITY;
+        ls[u] = in ? __ldcg(prow + D + 1) : 0.f;
+        os[u] = in ? __ldcg(prow + dd) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (ms[u] != -INFINITY) {   // a split with no valid key has no output row
+          const float mn = fmaxf(M, ms[u]);
+          const float sc = hw_exp2(M - mn);   // 0 while M is -inf
+          const float wgt = hw_exp2(ms[u] - mn);
+          L = fmaf(L, sc, wgt * ls[u]);
+          O = fmaf(O, sc, wgt * os[u]);
+          M = mn;
+        }
       }
     }
     a.out[hq * D + dd] = (L > 0.f) ? O / L : 0.f;

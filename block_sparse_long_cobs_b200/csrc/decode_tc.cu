@@ -60,6 +60,7 @@ constexpr int kChunkQ = 4;               // chunk indices handed from producer t
 constexpr uint32_t kOCol = 32;           // two 16-column output buffers after the two score buffers
 constexpr uint32_t kTmemCols = 64;
 constexpr float kRescaleLog2 = 8.f;      // raise m only when exceeded by > 2^8
+constexpr int kMergeSegs = 32;           // segments staged at a time by the merge
 // dynamic shared memory, offsets from a 1024-aligned base
 constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;   // 2 buffers x 2 slabs x 1 KB
@@ -145,6 +146,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   __shared__ volatile int abort_s;
   __shared__ int last_s;
   __shared__ float red[4][8];
+  __shared__ float2 ml_s[G][kMergeSegs];   // (m, l) of the segments being merged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -437,36 +439,64 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       named_bar(1, kSoftThreads);
       if (last_s) {
         __threadfence();
-        // thread r merges output dimension r of every head; the loads of the
-        // segments are independent, so the loops are unrolled to keep many
-        // L2 requests in flight (one at a time cost a round trip each)
+        // one pass over the segments, thread r merging output dimension r of
+        // every head with a running maximum (a segment's weight 2^(m_s - M)
+        // is rescaled when M rises); the (m, l) of 32 segments at a time are
+        // staged in shared memory by all threads at once, and the o loads of
+        // all heads of a segment are issued together
         const int nseg = sg.n_seg;
         const int dd = r;
+        constexpr int U = G >= 8 ? 2 : 16 / G;   // segments whose o loads are in flight together
+        float M[G], L[G], O[G];
+        const float* pb[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          M[h] = -INFINITY;
+          L[h] = 0.f;
+          O[h] = 0.f;
+          pb[h] = a.partials + (hq0 + h) * hstride + dd;
+        }
+        for (int s0 = 0; s0 < nseg; s0 += kMergeSegs) {
+          const int ns = nseg - s0 < kMergeSegs ? nseg - s0 : kMergeSegs;
+          for (int i = r; i < G * ns; i += kSoftThreads) {
+            const int h = i / ns, s2 = i - (i / ns) * ns;
+            const float* prow = a.partials + (hq0 + h) * hstride + int64_t(s0 + s2) * (kD + 2);
+            ml_s[h][s2] = make_float2(__ldcg(prow + kD), __ldcg(prow + kD + 1));
+          }
+          named_bar(1, kSoftThreads);
+          for (int s2 = 0; s2 < ns; s2 += U) {
+            float ov[U][G];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int64_t off = int64_t(s0 + s2 + u) * (kD + 2);
+#pragma unroll
+              for (int h = 0; h < G; ++h) ov[u][h] = s2 + u < ns ? __ldcg(pb[h] + off) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              if (s2 + u < ns) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                  const float2 ml = ml_s[h][s2 + u];
+                  if (ml.x != -INFINITY) {   // a segment with no valid key has no output row
+                    const float mn = fmaxf(M[h], ml.x);
+                    const float sc = hw_exp2(M[h] - mn);   // 0 while M is -inf
+                    const float wgt = hw_exp2(ml.x - mn);
+                    L[h] = fmaf(L[h], sc, wgt * ml.y);
+                    O[h] = fmaf(O[h], sc, wgt * ov[u][h]);
+                    M[h] = mn;
+                  }
+                }
+              }
+            }
+          }
+          named_bar(1, kSoftThreads);   // ml_s is rewritten by the next group
+        }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const int64_t hq = hq0 + h;
-          const float* pbase = a.partials + hq * hstride;
-          float M = -INFINITY;
-#pragma unroll 8
-          for (int s = 0; s < nseg; ++s)
-            M = fmaxf(M, __ldcg(pbase + int64_t(s) * (kD + 2) + kD));
-          float L = 0.f, O = 0.f;
-          if (M != -INFINITY) {
-#pragma unroll 8
-            for (int s = 0; s < nseg; ++s) {
-              const float* prow = pbase + int64_t(s) * (kD + 2);
-              const float ms = __ldcg(prow + kD);
-              const float ls = __ldcg(prow + kD + 1);
-              const float os = __ldcg(prow + dd);
-              // a segment with no valid key (m = -inf) has no output row
-              const bool live = ms != -INFINITY;
-              const float w = live ? hw_exp2(ms - M) : 0.f;
-              L = live ? fmaf(w, ls, L) : L;
-              O = live ? fmaf(w, os, O) : O;
-            }
-          }
-          a.out[hq * kD + dd] = (L > 0.f) ? O / L : 0.f;
-          if (dd == 0) a.lse[hq] = (L > 0.f) ? (M + hw_log2(L)) * kLn2 : -INFINITY;
+          a.out[hq * kD + dd] = (L[h] > 0.f) ? O[h] / L[h] : 0.f;
+          if (dd == 0) a.lse[hq] = (L[h] > 0.f) ? (M[h] + hw_log2(L[h])) * kLn2 : -INFINITY;
         }
         if (r == 0) a.tickets[sg.pair] = 0u;
       }

@@ -115,7 +115,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 // kFmt: 0 bf16 COBS records [mu; U^T], 1 FP4 COBS records, 2 min/max box
 // records [lo; hi], 3 subspace records [mu; U_s^T].
 template <int D, int G, int kFmt>
-__global__ void __launch_bounds__(kFmt == 1 ? 256 : 128, kFmt == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kFmt == 1 ? 288 : 128, kFmt == 1 ? 2 : 1)
 select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap qmap, const SelectArgs a) {
   constexpr bool kFp4 = kFmt == 1;
@@ -158,26 +158,28 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // ===================== phase 1: scores of this chunk =====================
   if constexpr (kFp4) {
     // FP4 records (COBS explainer §2.3, quantisation): mu bf16 [D] | E2M1
-    // codes [r][D/2] | scale exponents [r][D/32] | padding.  256 threads in
-    // two roles that work on different passes at once:
-    //  * warps 0-3 widen: a pass stages the raw records of per_pass
-    //    consecutive blocks with one bulk copy into a 3-slot ring; each thread
+    // codes [r][D/2] | scale exponents [r][D/32] | padding.  288 threads in
+    // three roles that work on different passes at once:
+    //  * warp 8 (one thread) issues: the bulk copy of a pass's raw records
+    //    (per_pass consecutive blocks) into a 3-slot ring, and, once the pass's
+    //    tile is widened, its two products -- the bf16 one against the bf16
+    //    queries (query-tile rows 0-7) and the fp16 one against the fp16 copy
+    //    of them (rows 8-15), both over the whole tile, into one of two
+    //    tensor-memory accumulators -- then the copy that refills the slot;
+    //  * warps 0-3 widen, each thread
     //    widens one row of the pass's 128-row operand tile (two tiles, used
     //    in turn): the mu rows (bf16) at rows [0, per_pass), the U rows from
     //    row mu_rows = 8 ceil(per_pass / 8) as fp16 values code x 2^(e_g - E),
     //    E the largest group exponent of that column -- exact in fp16 for
     //    e_g - E >= -23 (a group further below contributes nothing: its
-    //    components are under 2^-23 of the column's largest).  Thread 0 then
-    //    refills the ring and issues the pass's products: the bf16 one
-    //    against the bf16 queries (query-tile rows 0-7) and the fp16 one
-    //    against the fp16 copy of them (rows 8-15), both over the whole tile,
-    //    into one of two tensor-memory accumulators;
+    //    components are under 2^-23 of the column's largest);
     //  * warps 4-7 read an accumulator back (one lane per thread), keep each
     //    row's own product (mu rows: bf16 product, columns 0-7; U rows: fp16
     //    product, columns 8-15, scaled by 2^E) and write the pass's scores.
-    // mbarriers: raw_full (copy landed), mma_done (products complete: the
-    // tile may be rewritten and the accumulator read), acc_free (the
-    // epilogue has read the accumulator).
+    // mbarriers: raw_full (copy landed), tile_full (the 128 widening threads
+    // have written the tile and read the raw slot), mma_done (products
+    // complete: the tile may be rewritten and the accumulator read),
+    // acc_free (the epilogue has read the accumulator).
     constexpr int kRaw = kSelFp4RawStages;
     constexpr int kGroups = D / 32;
     const int r = a.rank;
@@ -189,6 +191,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     uint8_t* raw = stage + 2 * kStageBytes;          // [kRaw][raw_bytes]
     __shared__ __align__(8) uint64_t raw_full[kRaw];
     __shared__ __align__(8) uint64_t acc_free[2];
+    __shared__ __align__(8) uint64_t tile_full[2];
     __shared__ uint8_t colexp_s[4][kStageRows];      // E of each U row, per pass mod 4
     __shared__ volatile int abort_s;
 
@@ -205,6 +208,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       for (int s2 = 0; s2 < 2; ++s2) {
         mbar_init(&mma_done[s2], 1);
         mbar_init(&acc_free[s2], 1);
+        mbar_init(&tile_full[s2], kSelThreads);
       }
       fence_barrier_init();
       abort_s = 0;
@@ -217,9 +221,9 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     pdl_launch_dependents();
     const uint32_t tmem = tmem_slot;   // buffer b: bf16 products at 32 b, fp16 at 32 b + 16
 
-    int n_issued = 0;          // thread 0: passes whose copies were issued
-    int n_mma = 0;             // thread 0: passes whose products were issued
-    auto issue = [&](int p) {  // thread 0 only: raw records of pass p (+ queries)
+    int n_issued = 0;          // issuing thread: passes whose copies were issued
+    int n_mma = 0;             // issuing thread: passes whose products were issued
+    auto issue = [&](int p) {  // issuing thread only: raw records of pass p (+ queries)
       n_issued = p + 1;
       const int j0 = c_lo + p * per_pass;
       const int nb = min(per_pass, c_hi - j0);
@@ -235,10 +239,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     if (warp < 4) {
       // ============================ widening ============================
       const int my_blk = tid / r, my_col = tid - (tid / r) * r;
-      if (tid == 0)
-        for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
-      constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
-      constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
       for (int p = 0; p < npass; ++p) {
         const int buf = p & 1, st = p % kRaw;
         uint8_t* atile = tiles + buf * kStageBytes;
@@ -320,35 +320,44 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           }
         }
         fence_proxy_async_smem();   // generic-proxy tile writes -> tensor-core reads
-        named_bar(1, 128);          // the tile is written, the raw slot read
-        if (tid == 0) {
+        mbar_arrive(&tile_full[buf]);   // the tile is written, the raw slot read
+      }
+    } else if (warp == 8) {
+      // ============================= issue ==============================
+      if (lane == 0) {
+        constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
+        constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
+        for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
+        for (int p = 0; p < npass; ++p) {
+          const int buf = p & 1;
+          // pass p's tile is widened; the epilogue has read this
+          // accumulator's pass p - 2
+          bool ok = abort_s == 0 &&
+                    wait_or_abort(&tile_full[buf], (p >> 1) & 1, a.status, &abort_s);
+          if (ok && p >= 2)
+            ok = wait_or_abort(&acc_free[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t abase = smem_addr(tiles + buf * kStageBytes);
+          const uint32_t qb = smem_addr(qtile);
+          const uint32_t acc = tmem + 32u * uint32_t(buf);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+            const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+            umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
+            const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+            umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&mma_done[buf]);
+          n_mma = p + 1;
           // the raw slot of pass p is free again (its bytes are in the tile)
           if (p + kRaw < npass) issue(p + kRaw);
-          // the epilogue must have read this accumulator's pass p - 2
-          bool ok = p < 2 || wait_or_abort(&acc_free[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
-          if (ok) {
-            tc_fence_after();
-            const uint32_t abase = smem_addr(atile);
-            const uint32_t qb = smem_addr(qtile);
-            const uint32_t acc = tmem + 32u * uint32_t(buf);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
-              const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-              umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
-            }
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-              const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
-              const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-              umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
-            }
-            umma_commit(&mma_done[buf]);
-            n_mma = p + 1;
-          }
         }
-      }
-      if (tid == 0) {
         // let the copies and the products still in flight land before TMEM is
         // freed and the CTA leaves (each wait bounded)
         for (int p = n_issued > kRaw ? n_issued - kRaw : 0; p < n_issued; ++p)
@@ -380,17 +389,19 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         const bool is_mu = et < mu_rows;
         const uint32_t eb = colexp_s[p & 3][et];
         const float col_scale = __uint_as_float(eb << 23);   // 2^(E - 127); 0 for E = 0
+        float c8[8];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float c;
+        for (int h = 0; h < 8; ++h) {
           if (is_mu) {
-            c = __uint_as_float(vm[h]) * inv_sqrt_d;
+            c8[h] = __uint_as_float(vm[h]) * inv_sqrt_d;
           } else {
             const float x = __uint_as_float(vu[h]) * col_scale * inv_sqrt_d;
-            c = 0.5f * x * x;
+            c8[h] = 0.5f * x * x;
           }
-          contrib[et * 8 + h] = c;
         }
+        // two 16-byte stores per row (columns past G are never read)
+        reinterpret_cast<float4*>(contrib + et * 8)[0] = make_float4(c8[0], c8[1], c8[2], c8[3]);
+        reinterpret_cast<float4*>(contrib + et * 8)[1] = make_float4(c8[4], c8[5], c8[6], c8[7]);
         named_bar(2, 128);
         // the accumulator has been read: its next products may start
         if (et == 0) mbar_arrive(&acc_free[buf]);
@@ -985,7 +996,7 @@ constexpr size_t dyn_smem_bytes() {
          (kFmt == 3 ? size_t(2) * 32 * 128 : 0);
 }
 template <int kFmt>
-constexpr int sel_threads() { return kFmt == 1 ? 2 * kSelThreads : kSelThreads; }
+constexpr int sel_threads() { return kFmt == 1 ? 2 * kSelThreads + 32 : kSelThreads; }
 
 template <int D, int G, int kFmt>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
