@@ -582,6 +582,20 @@ def run_cobs(args, w, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         return g
 
+    def graph_kernel_nodes(g):
+        """Kernel nodes of a captured graph (None when they cannot be read)."""
+        try:
+            from cuda.bindings import driver as cu
+            gr = cu.CUgraph(init_value=int(g.raw_cuda_graph()))
+            err, _, n = cu.cuGraphGetNodes(gr, 0)
+            err, nodes, n = cu.cuGraphGetNodes(gr, n)
+            if err != cu.CUresult.CUDA_SUCCESS:
+                return None
+            kinds = [cu.cuGraphNodeGetType(nd)[1] for nd in nodes[:n]]
+            return sum(k == cu.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL for k in kinds)
+        except Exception:
+            return None
+
     def run_timed(evs, graph, n_steps, inner, sums, with_stats=True):
         for _ in range(n_steps // g_steps):
             if graph is not None:
@@ -607,6 +621,21 @@ def run_cobs(args, w, rank, world, local_rank):
     n_kern = max(min(250, args.steps), args.steps // 5) // g_steps * g_steps or g_steps
     graph_kern = capture(evs_kern, True)
     graph_sd = capture(evs_sd, False, with_stats=False)
+    # this library's launches per step: the kernel nodes of a captured step
+    # less those of a captured L2 flush (torch's kernels); graphs kept
+    # uninstantiated for reading, never replayed
+    launches_per_step = None
+    if not args.no_graph:
+        g_one, g_flush = torch.cuda.CUDAGraph(keep_graph=True), torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g_one):
+            flush()
+            step(None, torch.cuda.current_stream(dev), False, one_stream=False)
+        with torch.cuda.graph(g_flush):
+            flush()
+        k_all, k_flush = graph_kernel_nodes(g_one), graph_kernel_nodes(g_flush)
+        if k_all is not None and k_flush is not None:
+            launches_per_step = k_all - k_flush
+        del g_one, g_flush
     sums_step, sums_kern, sums_sd = [0.0] * 4, [0.0] * 4, [0.0] * 4
 
     clocks = ClockSampler(local_rank)
@@ -771,7 +800,11 @@ def run_cobs(args, w, rank, world, local_rank):
                      "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "traffic": recorded_traffic(file_dom, traffic_key)},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": (round(launches_per_step * args.steps) if launches_per_step is not None
+                         else 3 * args.steps),
+        "gpu_launches_counted": ("kernel nodes of the captured step graphs, less the L2 flush's"
+                                 if launches_per_step is not None else
+                                 "3 per step (stats, select, decode), not read from a graph"),
         "value_step": "every timed step builds the statistics of one completed block per "
                       "(batch, kv-head) besides selection and decode (step_variants gives the "
                       "steps without it)",

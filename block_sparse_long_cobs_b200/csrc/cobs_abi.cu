@@ -241,15 +241,15 @@ DecodePlan plan_decode(int d, int g, int64_t pairs, int32_t idx_stride) {
     // one wave of persistent CTAs pulling chunks off a counter.  A chunk is an
     // even share of one pair's list, never two pairs.  A pair that is one
     // chunk writes its output directly; splitting a pair costs partials, a
-    // ticket, a merge and a pipeline restart (measured: 26-slot pairs of the
-    // 32k workload took 45 us whole, 61 us as halves), so pairs are split only
-    // as far as the resident CTAs can still take every chunk in one wave (a
-    // second, partial wave doubles the time of the CTAs that run it), with at
-    // least 8 slots per chunk (smaller chunks lost on the latency-bound
-    // small problems: more partials to merge).
+    // pipeline restart and a merge kernel after the decode (measured: 26-slot
+    // pairs of the 32k workload took 45 us whole, 61 us as halves), so pairs
+    // are split only as far as the resident CTAs can still take every chunk
+    // in one wave (a second, partial wave doubles the time of the CTAs that
+    // run it), with at least 4 slots per chunk (2-slot chunks gained nothing
+    // more on the few-pair problems and double the partials).
     const int64_t resident = int64_t(sms) * decode_tc_ctas_per_sm(g);
     int64_t per_pair = resident / pairs;
-    const int64_t max_per_pair = ceil_div(idx_stride, 8);
+    const int64_t max_per_pair = ceil_div(idx_stride, 4);
     if (per_pair > max_per_pair) per_pair = max_per_pair;
     if (per_pair < 1) per_pair = 1;
     P.chunk_slots = int32_t(ceil_div(idx_stride, per_pair));

@@ -11,12 +11,13 @@
 // end, idx_stride slots per pair, and cut into chunks of C slots.  A
 // persistent grid (two CTAs per SM) pulls chunks off a counter, so CTAs that
 // stream faster simply take more chunks.  Pair boundaries cut a chunk into
-// segments; a segment yields one partial (o, m, l) per query head of the
-// group (row = chunk index - first chunk of the pair), and the last segment
-// of a pair to finish (atomic ticket, no spinning) merges the partials:
+// segments.  A pair that is one chunk is normalised in place; a split pair's
+// segments each write one partial (o, m, l) per query head of the group
+// (row = chunk index - first chunk of the pair), and a second kernel, chained
+// by programmatic dependent launch, merges them with one CTA per query head:
 // M = max m_i, out = sum 2^(m_i-M) o_i / sum 2^(m_i-M) l_i,
 // lse = (M + log2 sum 2^(m_i-M) l_i) ln 2.  The last CTA to run out of work
-// puts the counters back to zero.
+// puts the chunk counters back to zero.
 //
 // One segment of nb blocks, T = ceil(nb / 2) tiles of two blocks (128 keys),
 // in a single pass:
@@ -60,7 +61,6 @@ constexpr int kChunkQ = 4;               // chunk indices handed from producer t
 constexpr uint32_t kOCol = 32;           // two 16-column output buffers after the two score buffers
 constexpr uint32_t kTmemCols = 64;
 constexpr float kRescaleLog2 = 8.f;      // raise m only when exceeded by > 2^8
-constexpr int kMergeSegs = 32;           // segments staged at a time by the merge
 // dynamic shared memory, offsets from a 1024-aligned base
 constexpr int kOffRing = 0;
 constexpr int kOffQ = kOffRing + kStages * kStageBytes;   // 2 buffers x 2 slabs x 1 KB
@@ -144,9 +144,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   __shared__ long long chunk_s;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_s;
-  __shared__ int last_s;
   __shared__ float red[4][8];
-  __shared__ float2 ml_s[G][kMergeSegs];   // (m, l) of the segments being merged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -419,6 +417,8 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         named_bar(1, kSoftThreads);   // red is read before it is rewritten
         return true;
       }
+      // a split pair: this segment's partial rows (a segment with no block
+      // writes m = -inf, l = 0 and no o, which the merge skips)
       float* part = a.partials + hq0 * hstride + int64_t(sg.seg) * (kD + 2);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -428,79 +428,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           part[h * hstride + kD + 1] = l[h];
         }
       }
-      // publish: every thread's rows are written (barrier), then one fence and
-      // the pair's ticket
-      named_bar(1, kSoftThreads);
-      if (r == 0) {
-        __threadfence();
-        const uint32_t prev = atomicAdd(&a.tickets[sg.pair], 1u);
-        last_s = (prev == uint32_t(sg.n_seg - 1));
-      }
-      named_bar(1, kSoftThreads);
-      if (last_s) {
-        __threadfence();
-        // one pass over the segments, thread r merging output dimension r of
-        // every head with a running maximum (a segment's weight 2^(m_s - M)
-        // is rescaled when M rises); the (m, l) of 32 segments at a time are
-        // staged in shared memory by all threads at once, and the o loads of
-        // all heads of a segment are issued together
-        const int nseg = sg.n_seg;
-        const int dd = r;
-        constexpr int U = G >= 8 ? 2 : 16 / G;   // segments whose o loads are in flight together
-        float M[G], L[G], O[G];
-        const float* pb[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          M[h] = -INFINITY;
-          L[h] = 0.f;
-          O[h] = 0.f;
-          pb[h] = a.partials + (hq0 + h) * hstride + dd;
-        }
-        for (int s0 = 0; s0 < nseg; s0 += kMergeSegs) {
-          const int ns = nseg - s0 < kMergeSegs ? nseg - s0 : kMergeSegs;
-          for (int i = r; i < G * ns; i += kSoftThreads) {
-            const int h = i / ns, s2 = i - (i / ns) * ns;
-            const float* prow = a.partials + (hq0 + h) * hstride + int64_t(s0 + s2) * (kD + 2);
-            ml_s[h][s2] = make_float2(__ldcg(prow + kD), __ldcg(prow + kD + 1));
-          }
-          named_bar(1, kSoftThreads);
-          for (int s2 = 0; s2 < ns; s2 += U) {
-            float ov[U][G];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-              const int64_t off = int64_t(s0 + s2 + u) * (kD + 2);
-#pragma unroll
-              for (int h = 0; h < G; ++h) ov[u][h] = s2 + u < ns ? __ldcg(pb[h] + off) : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-              if (s2 + u < ns) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                  const float2 ml = ml_s[h][s2 + u];
-                  if (ml.x != -INFINITY) {   // a segment with no valid key has no output row
-                    const float mn = fmaxf(M[h], ml.x);
-                    const float sc = hw_exp2(M[h] - mn);   // 0 while M is -inf
-                    const float wgt = hw_exp2(ml.x - mn);
-                    L[h] = fmaf(L[h], sc, wgt * ml.y);
-                    O[h] = fmaf(O[h], sc, wgt * ov[u][h]);
-                    M[h] = mn;
-                  }
-                }
-              }
-            }
-          }
-          named_bar(1, kSoftThreads);   // ml_s is rewritten by the next group
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const int64_t hq = hq0 + h;
-          a.out[hq * kD + dd] = (L[h] > 0.f) ? O[h] / L[h] : 0.f;
-          if (dd == 0) a.lse[hq] = (L[h] > 0.f) ? (M[h] + hw_log2(L[h])) * kLn2 : -INFINITY;
-        }
-        if (r == 0) a.tickets[sg.pair] = 0u;
-      }
-      named_bar(1, kSoftThreads);   // last_s is rewritten by the next segment
+      named_bar(1, kSoftThreads);   // red is read before it is rewritten
       return true;
     };
 
@@ -700,6 +628,60 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+// The partial rows of a split pair, merged: one CTA per query head of such a
+// pair, thread r for output dimension r.
+//   M = max_s m_s,  w_s = 2^(m_s - M),  L = sum_s w_s l_s,
+//   out = sum_s w_s o_s / L,  lse = (M + log2 L) ln 2
+// (m in base-2 units; a segment with m = -inf has no output row and weight
+// 0).  It runs after the decode grid (programmatic dependent launch: its CTAs
+// may be resident early and wait for the decode's writes), so the merges of
+// all split pairs spread over the whole GPU instead of queueing in the last
+// CTA of each pair.  Every thread loads (m, l, o[r]) of 16 segments at once
+// and merges them with a running maximum: one round trip to L2 per 16
+// segments, no barrier.
+template <int G>
+__global__ void __launch_bounds__(kD) merge_split_rows_kernel(const DecodeArgs a) {
+  constexpr int kB = 16;
+  pdl_wait();                // the decode grid's partial rows
+  pdl_launch_dependents();
+  const int r = threadIdx.x;
+  const int64_t pair = blockIdx.x / G;
+  const int h = int(blockIdx.x % G);
+  const int64_t hq = (pair / a.hkv) * a.hq + (pair % a.hkv) * G + h;
+  const float* prow = a.partials + hq * (int64_t(a.part_stride) * (kD + 2));
+  const int nseg = a.chunks_per_pair;
+  constexpr float kLn2 = 0.69314718055994530942f;
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (int s0 = 0; s0 < nseg; s0 += kB) {
+    float mv[kB], lv[kB], ov[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const bool in = s0 + u < nseg;
+      const float* pr = prow + int64_t(s0 + u) * (kD + 2);
+      mv[u] = in ? __ldcg(pr + kD) : -INFINITY;
+      lv[u] = in ? __ldcg(pr + kD + 1) : 0.f;
+      ov[u] = in ? __ldcg(pr + r) : 0.f;
+    }
+    float mb = M;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) mb = fmaxf(mb, mv[u]);
+    if (mb == -INFINITY) continue;   // no segment so far has a valid key
+    const float sc = hw_exp2(M - mb);   // 0 while M is -inf
+    L *= sc;
+    O *= sc;
+    M = mb;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      // an unwritten row (m = -inf) is never used
+      const float wgt = mv[u] == -INFINITY ? 0.f : hw_exp2(mv[u] - M);
+      L = fmaf(wgt, lv[u], L);
+      O = wgt != 0.f ? fmaf(wgt, ov[u], O) : O;
+    }
+  }
+  a.out[hq * kD + r] = L > 0.f ? O / L : 0.f;
+  if (r == 0) a.lse[hq] = L > 0.f ? (M + hw_log2(L)) * kLn2 : -INFINITY;
+}
+
 template <int G>
 int occupancy_g() {
   const int n = kernel_occupancy(reinterpret_cast<const void*>(sparse_decode_tc_kernel<G, 0>),
@@ -729,7 +711,10 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
                                              : sparse_decode_tc_kernel<G, 0>);
   e = set_smem_attrs(kern, kDynSmem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(a.n_ctas), dim3(kThreads), kDynSmem, stream, kmap, vmap, qmap, a);
+  e = launch_pdl(kern, dim3(a.n_ctas), dim3(kThreads), kDynSmem, stream, kmap, vmap, qmap, a);
+  if (e != cudaSuccess || a.chunks_per_pair == 1) return e;
+  const int64_t pairs = int64_t(a.batch) * a.hkv;
+  return launch_pdl(merge_split_rows_kernel<G>, dim3(unsigned(pairs * G)), dim3(kD), 0, stream, a);
 }
 
 }  // namespace

@@ -196,6 +196,17 @@ __device__ __forceinline__ float hw_log2(float x) {
 // Warp reductions
 // ---------------------------------------------------------------------------
 
+// 16-byte asynchronous copy global -> shared, cached in L2 only (both
+// addresses 16-byte aligned); complete for this thread after cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));

@@ -162,20 +162,24 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     // three roles that work on different passes at once:
     //  * warp 8 (one thread) issues: the bulk copy of a pass's raw records
     //    (per_pass consecutive blocks) into a 3-slot ring, and, once the pass's
-    //    tile is widened, its two products -- the bf16 one against the bf16
-    //    queries (query-tile rows 0-7) and the fp16 one against the fp16 copy
-    //    of them (rows 8-15), both over the whole tile, into one of two
-    //    tensor-memory accumulators -- then the copy that refills the slot;
-    //  * warps 0-3 widen, each thread
-    //    widens one row of the pass's 128-row operand tile (two tiles, used
-    //    in turn): the mu rows (bf16) at rows [0, per_pass), the U rows from
-    //    row mu_rows = 8 ceil(per_pass / 8) as fp16 values code x 2^(e_g - E),
-    //    E the largest group exponent of that column -- exact in fp16 for
+    //    tile is widened, the copy that refills the slot and the pass's one
+    //    fp16 product against an fp16 copy of the queries (query-tile rows
+    //    8-15), into one of two tensor-memory accumulators;
+    //  * warps 0-3 widen, each thread one row of the pass's 128-row operand
+    //    tile (two tiles, used in turn), all rows as fp16 values times a
+    //    power of two per row: the mu rows at rows [0, per_pass) as
+    //    mu_t x 2^(142 - M), M the largest bf16 exponent field of the row
+    //    (exact: a value at or above 2^-32 of the row's largest keeps its 8
+    //    significant bits on the fp16 grid; smaller ones round), the U rows
+    //    from row mu_rows = 8 ceil(per_pass / 8) as code x 2^(e_g - E), E the
+    //    largest group exponent of that column -- exact in fp16 for
     //    e_g - E >= -23 (a group further below contributes nothing: its
     //    components are under 2^-23 of the column's largest);
-    //  * warps 4-7 read an accumulator back (one lane per thread), keep each
-    //    row's own product (mu rows: bf16 product, columns 0-7; U rows: fp16
-    //    product, columns 8-15, scaled by 2^E) and write the pass's scores.
+    //  * warps 4-7 read an accumulator back (one lane per thread, columns
+    //    8-15), undo each row's power of two and write the pass's scores.
+    // One fp16 product over the tile, rather than a bf16 one for the mu rows
+    // beside it, halves the tensor cores' shared-memory reads, which with the
+    // widening's writes bound a pass.
     // mbarriers: raw_full (copy landed), tile_full (the 128 widening threads
     // have written the tile and read the raw slot), mma_done (products
     // complete: the tile may be rewritten and the accumulator read),
@@ -192,7 +196,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     __shared__ __align__(8) uint64_t raw_full[kRaw];
     __shared__ __align__(8) uint64_t acc_free[2];
     __shared__ __align__(8) uint64_t tile_full[2];
-    __shared__ uint8_t colexp_s[4][kStageRows];      // E of each U row, per pass mod 4
+    __shared__ uint8_t colexp_s[4][kStageRows];      // row scale exponents, per pass mod 4
     __shared__ volatile int abort_s;
 
     const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
@@ -309,14 +313,42 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                                         (((u & 7) ^ (row & 7)) << 4)) = hv;
             }
           }
-        } else if (tid < nb * r + nb) {
-          const int blk = tid - nb * r;
-          const uint8_t* rp = rs + blk * rec;
+        }
+        {
+          // the mu rows, D / 8 threads per row (one 16-byte chunk each): the
+          // row's largest exponent field by shuffles within the row's lanes
+          constexpr int kMuLanes = D / 8;
+          const int c = tid % kMuLanes;
+          for (int b0 = 0; b0 < nb; b0 += 128 / kMuLanes) {   // same trip count for all
+            const int blk = b0 + tid / kMuLanes;
+            const bool act = blk < nb;
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (act) w = *reinterpret_cast<const uint4*>(rs + blk * rec + c * 16);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            uint32_t emax = 0;
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const uint4 w = *reinterpret_cast<const uint4*>(rp + c * 16);
-            *reinterpret_cast<uint4*>(atile + (c >> 3) * (128 * 128) + blk * 128 +
-                                      (((c & 7) ^ (blk & 7)) << 4)) = w;
+            for (int t = 0; t < 4; ++t)
+              emax = max(emax, max((ww[t] >> 7) & 0xFFu, (ww[t] >> 23) & 0xFFu));
+#pragma unroll
+            for (int m = kMuLanes / 2; m >= 1; m >>= 1)
+              emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, m));
+            // 2^(142 - M) puts the largest at fp16 exponent 15; a row whose
+            // largest is below 2^-111 is taken as zero (its epilogue scale is 0)
+            const bool live = emax >= 16u;
+            const float sc = live ? __uint_as_float((269u - emax) << 23) : 0.f;
+            if (act) {
+              if (c == 0) colexp_s[p & 3][blk] = uint8_t(live ? emax - 15u : 0u);
+              uint32_t hh[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float2 f = bf16x2_to_float2(ww[t]);
+                const __half2 h2 = __floats2half2_rn(f.x * sc, f.y * sc);
+                hh[t] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+              *reinterpret_cast<uint4*>(atile + (c >> 3) * (128 * 128) + blk * 128 +
+                                        (((c & 7) ^ (blk & 7)) << 4)) =
+                  make_uint4(hh[0], hh[1], hh[2], hh[3]);
+            }
           }
         }
         fence_proxy_async_smem();   // generic-proxy tile writes -> tensor-core reads
@@ -325,7 +357,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     } else if (warp == 8) {
       // ============================= issue ==============================
       if (lane == 0) {
-        constexpr uint32_t idesc_bf16 = umma_idesc_bf16(128, 16);
         constexpr uint32_t idesc_f16 = umma_idesc_f16(128, 16);
         for (int p = 0; p < kRaw && p < npass; ++p) issue(p);
         for (int p = 0; p < npass; ++p) {
@@ -334,29 +365,25 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           // accumulator's pass p - 2
           bool ok = abort_s == 0 &&
                     wait_or_abort(&tile_full[buf], (p >> 1) & 1, a.status, &abort_s);
-          if (ok && p >= 2)
-            ok = wait_or_abort(&acc_free[buf], ((p - 2) >> 1) & 1, a.status, &abort_s);
           if (!ok) break;
+          // the raw slot of pass p is free again (its bytes are in the tile)
+          if (p + kRaw < npass) issue(p + kRaw);
+          if (p >= 2 && !wait_or_abort(&acc_free[buf], ((p - 2) >> 1) & 1, a.status, &abort_s))
+            break;
           tc_fence_after();
           const uint32_t abase = smem_addr(tiles + buf * kStageBytes);
           const uint32_t qb = smem_addr(qtile);
           const uint32_t acc = tmem + 32u * uint32_t(buf);
+          // columns 8-15 take query-tile rows 8-15 (fp16); columns 0-7 read
+          // the bf16 rows as fp16 and are never read back
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
             const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-            umma_bf16(acc, ad, bd, idesc_bf16, ks > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = umma_desc_sw128(abase + (ks >> 2) * 128 * 128 + (ks & 3) * 32);
-            const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-            umma_bf16(acc + 16u, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
+            umma_bf16(acc, ad, bd, idesc_f16, ks > 0 ? 1u : 0u);
           }
           umma_commit(&mma_done[buf]);
           n_mma = p + 1;
-          // the raw slot of pass p is free again (its bytes are in the tile)
-          if (p + kRaw < npass) issue(p + kRaw);
         }
         // let the copies and the products still in flight land before TMEM is
         // freed and the CTA leaves (each wait bounded)
@@ -381,23 +408,19 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         const int j0 = c_lo + p * per_pass;
         const int nb = min(per_pass, c_hi - j0);
         const uint32_t lane_base = tmem + (uint32_t((warp - 4) * 32) << 16) + 32u * uint32_t(buf);
-        uint32_t vm[8], vu[8];
-        tmem_ld8_nowait(lane_base, vm);
-        tmem_ld8_nowait(lane_base + 24u, vu);        // fp16 product, query rows 8-15
+        uint32_t vu[8];
+        tmem_ld8_nowait(lane_base + 8u, vu);         // fp16 product, query rows 8-15
         tmem_wait_ld();
         tc_fence_before();
         const bool is_mu = et < mu_rows;
         const uint32_t eb = colexp_s[p & 3][et];
-        const float col_scale = __uint_as_float(eb << 23);   // 2^(E - 127); 0 for E = 0
+        // 2^(e - 127): the row's power of two undone (0 for e = 0)
+        const float row_scale = __uint_as_float(eb << 23) * inv_sqrt_d;
         float c8[8];
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
-          if (is_mu) {
-            c8[h] = __uint_as_float(vm[h]) * inv_sqrt_d;
-          } else {
-            const float x = __uint_as_float(vu[h]) * col_scale * inv_sqrt_d;
-            c8[h] = 0.5f * x * x;
-          }
+          const float x = __uint_as_float(vu[h]) * row_scale;
+          c8[h] = is_mu ? x : 0.5f * x * x;
         }
         // two 16-byte stores per row (columns past G are never read)
         reinterpret_cast<float4*>(contrib + et * 8)[0] = make_float4(c8[0], c8[1], c8[2], c8[3]);
