@@ -30,8 +30,8 @@
 // exact top k over distinct 64-bit keys (order-preserving score key, then the
 // lower block index): the k-th largest of the 128 per-thread maxima bounds
 // the k-th largest key from below, so only the few keys at or above it are
-// ranked; the chosen blocks are written in ascending order (warp ballot scan)
-// between the sink blocks and the local blocks.
+// ranked; the chosen blocks are written in ascending order (a block-wide scan
+// of per-thread counts) between the sink blocks and the local blocks.
 #include <cfloat>
 
 #include <cuda_fp16.h>
@@ -868,6 +868,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   const bool partial = (k > 0 && k < n_cand);
 
   // ---- exact top-k (score, then lower block index) -------------------------
+  int32_t* out = a.idx + int64_t(bh) * a.idx_stride;
   // Keys: 64-bit, order-preserving score key << 32 | ~candidate, so distinct.
   // The candidates are cut into ng <= 1024 groups of gs.  Each group maximum
   // is a real key, so the k-th largest group maximum tau2 bounds the k-th
@@ -876,22 +877,59 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // bounds it likewise, so only the group maxima >= tau1 -- at most
   // k * ceil(ng / 128) -- are ranked (all ng of them for k >= 128).  The
   // record ring (free now) holds the work arrays; the host rejects settings
-  // whose survivors could overflow it (select_topk_fits).
+  // whose survivors could overflow it (select_topk_fits).  When there is
+  // room, the pair's scores are first copied into it (16 loads in flight per
+  // thread), so that the passes below read shared memory instead of making a
+  // round trip to L2 per few candidates.
   const int gs = topk_group_size(n_cand);
   const int ng = (n_cand + gs - 1) / gs;                               // no empty group
-  uint64_t* gmax = reinterpret_cast<uint64_t*>(stage);                 // [ng]
+  const int need = topk_survivors_needed(n_cand, k);
+  const int staged_bytes = (n_cand * 4 + 15) & ~15;
+  const bool staged =
+      topk_survivor_capacity(ring_bytes(D, kFmt) - staged_bytes, n_cand) >= need;
+  float* score_s = reinterpret_cast<float*>(stage);                   // [n_cand] if staged
+  uint64_t* gmax = reinterpret_cast<uint64_t*>(stage + (staged ? staged_bytes : 0));   // [ng]
   uint64_t* tmax = gmax + ng;                                          // [128]
   uint64_t* surv = tmax + kSelThreads;                                 // survivors
-  const int surv_cap = topk_survivor_capacity(ring_bytes(D, kFmt), n_cand);
+  const int surv_cap =
+      topk_survivor_capacity(ring_bytes(D, kFmt) - (staged ? staged_bytes : 0), n_cand);
+  // one flag byte per candidate, zero up to a multiple of 16 (read as words)
   uint8_t* chosen_s = reinterpret_cast<uint8_t*>(surv + (surv_cap > 0 ? surv_cap : 0));
   auto key64 = [&](int jj) -> uint64_t {
-    return (uint64_t(order_key(__ldcg(scores + c0 + jj))) << 32) |
-           uint64_t(0xFFFFFFFFu - uint32_t(jj));
+    const float sv = staged ? score_s[jj] : __ldcg(scores + c0 + jj);
+    return (uint64_t(order_key(sv)) << 32) | uint64_t(0xFFFFFFFFu - uint32_t(jj));
   };
   __shared__ unsigned long long tau_s;
-  const bool fits = surv_cap >= topk_survivors_needed(n_cand, k);
+  __shared__ int tk_warp[kSelThreads / 32];
+  // a slot in the survivor list for each lane that asks (-1 for the others):
+  // one atomic per warp on the shared count (one per lane would be replayed
+  // once per lane, all lanes adding to the same word)
+  auto append_slot = [&](bool want) -> int {
+    const uint32_t ask = __ballot_sync(0xffffffffu, want);
+    int base = 0;
+    if (lane == 0 && ask != 0u) base = atomicAdd(&last_s, __popc(ask));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    return want ? base + __popc(ask & ((1u << lane) - 1u)) : -1;
+  };
+  const bool fits = surv_cap >= need;
   if (partial && fits) {
-    for (int jj = tid; jj < n_cand; jj += kSelThreads) chosen_s[jj] = 0;
+    if (staged) {
+      for (int j0 = 0; j0 < n_cand; j0 += kSelThreads * 16) {
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int jj = j0 + u * kSelThreads + tid;
+          v[u] = jj < n_cand ? __ldcg(scores + c0 + jj) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int jj = j0 + u * kSelThreads + tid;
+          if (jj < n_cand) score_s[jj] = v[u];
+        }
+      }
+    }
+    for (int jj = tid; jj < ((n_cand + 15) & ~15); jj += kSelThreads) chosen_s[jj] = 0;
+    named_bar(3, kSelThreads);
     uint64_t mine = 0;
     for (int g = tid; g < ng; g += kSelThreads) {
       const int j0 = g * gs, j1 = min(n_cand, j0 + gs);
@@ -918,11 +956,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     }
     named_bar(3, kSelThreads);
     const uint64_t tau1 = tau_s;
-    for (int g = tid; g < ng; g += kSelThreads) {
-      if (gmax[g] >= tau1) {
-        const int slot = atomicAdd(&last_s, 1);
-        if (slot < surv_cap) surv[slot] = gmax[g];
-      }
+    for (int g0 = 0; g0 < ng; g0 += kSelThreads) {   // same trip count for all
+      const int g = g0 + tid;
+      const uint64_t c = g < ng ? gmax[g] : 0ull;
+      const int slot = append_slot(g < ng && c >= tau1);
+      if (slot >= 0 && slot < surv_cap) surv[slot] = c;
     }
     named_bar(3, kSelThreads);
     const int ns1 = last_s < surv_cap ? last_s : surv_cap;
@@ -953,12 +991,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       const uint64_t tau2 = tau_s;
       if (tid == 0) last_s = 0;
       named_bar(3, kSelThreads);
-      for (int jj = tid; jj < n_cand; jj += kSelThreads) {
-        const uint64_t c = key64(jj);
-        if (c >= tau2) {
-          const int slot = atomicAdd(&last_s, 1);
-          if (slot < surv_cap) surv[slot] = c;
-        }
+      for (int j0 = 0; j0 < n_cand; j0 += kSelThreads) {   // same trip count for all
+        const int jj = j0 + tid;
+        const uint64_t c = jj < n_cand ? key64(jj) : 0ull;
+        const int slot = append_slot(jj < n_cand && c >= tau2);
+        if (slot >= 0 && slot < surv_cap) surv[slot] = c;
       }
       named_bar(3, kSelThreads);
       const int ns = last_s < surv_cap ? last_s : surv_cap;
@@ -971,33 +1008,49 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       }
       named_bar(3, kSelThreads);
     }
+    // the chosen blocks in ascending order: thread t counts the flags of its
+    // contiguous run of candidates (whole 4-byte words), an exclusive scan of
+    // the counts over the 128 threads gives its first output slot
+    const int n_fw = (n_cand + 3) >> 2;                        // flag words
+    const int fpt = (n_fw + kSelThreads - 1) / kSelThreads;    // words per thread
+    const int f0 = min(n_fw, tid * fpt), f1 = min(n_fw, f0 + fpt);
+    const uint32_t* fw = reinterpret_cast<const uint32_t*>(chosen_s);
+    int cnt = 0;
+    for (int i = f0; i < f1; ++i) cnt += __popc(fw[i] & 0x01010101u);
+    int incl = cnt;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, m);
+      if (lane >= m) incl += y;
+    }
+    if (lane == 31) tk_warp[warp] = incl;
+    named_bar(3, kSelThreads);
+    int pos = sink_end + incl - cnt;
+    for (int w2 = 0; w2 < warp; ++w2) pos += tk_warp[w2];
+    for (int i = f0; i < f1; ++i) {
+      uint32_t f = fw[i] & 0x01010101u;
+      while (f) {
+        const int byte = (__ffs(f) - 1) >> 3;
+        f &= f - 1u;
+        if (pos < a.idx_stride) out[pos] = c0 + 4 * i + byte;
+        ++pos;
+      }
+    }
   } else if (partial && tid == 0) {
     report(a.status, COBS_ERR_DEVICE);   // host limits prevent this
   }
 
-  // ---- sink blocks, chosen candidates ascending, local blocks -------------
-  int32_t* out = a.idx + int64_t(bh) * a.idx_stride;
+  // ---- sink blocks, all or no candidates when nothing is ranked, local blocks
   const int n_local = nbs - first_local;
   const int total = sink_end + k + n_local;
   if (warp == 0) {
     for (int i = lane; i < sink_end && i < a.idx_stride; i += 32) out[i] = i;
     int pos = sink_end;
-    if (partial && fits) {
-      for (int j0 = 0; j0 < n_cand; j0 += 32) {
-        const int jj = j0 + lane;
-        const bool take = jj < n_cand && chosen_s[jj] != 0;
-        const uint32_t bal = __ballot_sync(0xffffffffu, take);
-        if (take) {
-          const int at = pos + __popc(bal & ((1u << lane) - 1u));
-          if (at < a.idx_stride) out[at] = c0 + jj;
-        }
-        pos += __popc(bal);
-      }
-    } else if (!partial) {   // k == n_cand: every candidate; k == 0: none
+    if (!partial) {   // k == n_cand: every candidate; k == 0: none
       for (int r = lane; r < k; r += 32)
         if (pos + r < a.idx_stride) out[pos + r] = c0 + r;
-      pos += k;
     }
+    pos += k;
     for (int i = lane; i < n_local; i += 32)
       if (pos + i < a.idx_stride) out[pos + i] = first_local + i;
     if (lane == 0) {
