@@ -225,14 +225,19 @@ class OracleSample:
             vals = bits_to_f64(v_bits[b, h])
             qg = bits_to_f64(q_bits[b, h * w.group:(h + 1) * w.group])
             recs = O.build_block_records(keys, w.block, w.rank, 0, nfull - 1)
-            self.items.append((qg, keys, vals, recs))
+            last = O.build_block_records(keys, w.block, w.rank, nfull - 1, nfull)
+            self.items.append((qg, keys, vals, recs, last))
 
     def step(self, i):
-        """Stats of the just-completed block + selection + attention, one pair."""
+        """One decode step of one pair: selection + attention, and the stats of
+        the just-completed block on the pair's steps where a block completes
+        (every block-th step of the pair), as in the GPU stream."""
         O, w = self.O, self.w
-        qg, keys, vals, recs = self.items[i % len(self.items)]
+        n = len(self.items)
+        qg, keys, vals, recs, last = self.items[i % n]
         nfull = w.seq_len // w.block
-        last = O.build_block_records(keys, w.block, w.rank, nfull - 1, nfull)
+        if (i // n) % w.block == w.block - 1:
+            last = O.build_block_records(keys, w.block, w.rank, nfull - 1, nfull)
         allrec = np.concatenate([recs, last])
         O.decode_step(qg, keys, vals, allrec, w.seq_len, w.block, w.top_k,
                       w.sink_blocks, w.local_tokens)
@@ -342,11 +347,14 @@ def run_reference(args, w, rank):
                    "block": w.block, "rank": w.rank, "top_k": w.top_k,
                    "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
                    "parallelism": f"replicas x{args.gpus}",
-                   "step": "stats of the completed block + select + sparse decode"},
+                   "step": ("one decode token of a pair: select + sparse decode, and the "
+                            "stats of the completed block on the pair's steps where a block "
+                            "completes (every block-th)")},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"each step: every one of {cores} host cores (one process, "
                                    f"one BLAS thread each) decodes one (batch, kv-head) pair "
-                                   f"(stats of the completed block + selection + attention, "
+                                   f"(selection + attention, and the stats of the "
+                                   f"completed block every block-th step of a pair, "
                                    f"fp64 numpy); pairs cycle over {len(pairs)} of "
                                    f"{w.batch * w.kv_heads}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -361,7 +369,8 @@ def cpu_baseline(w, seconds):
     one, n1, dt1, p1 = oracle_rate(w, 1, seconds=seconds / 2)
     out = {"value": one, "unit": UNIT, "cores": 1, "kind": "oracle",
            "sample": f"{n1} oracle decode steps of (batch, kv-head) pair {p1[0]} of {w.name} "
-                     f"(stats of the completed block + selection + attention, fp64 numpy, "
+                     f"(selection + attention, and the stats of the completed block "
+                     f"every block-th step of a pair, fp64 numpy, "
                      f"1 thread), {dt1:.1f} s, scaled to queries/s"}
     if cores > 1:
         try:
@@ -369,8 +378,9 @@ def cpu_baseline(w, seconds):
             out = {"value": allv, "unit": UNIT, "cores": cores, "kind": "oracle",
                    "sample": f"{cores} host cores at once, one process and one BLAS thread "
                              f"each, every core decoding its own (batch, kv-head) pair of "
-                             f"{w.name} ({len(pairs)} distinct pairs; stats of the completed "
-                             f"block + selection + attention, fp64 numpy), >= {n} steps per "
+                             f"{w.name} ({len(pairs)} distinct pairs; selection + attention, "
+                             f"and the stats of the completed block every block-th step of a "
+                             f"pair, fp64 numpy), >= {n} steps per "
                              f"core in {dt:.1f} s, scaled to queries/s",
                    "one_core": {"value": one, "cores": 1, "sample": out["sample"]}}
         except Exception as e:            # the one-core figure still stands
@@ -621,21 +631,63 @@ def run_cobs(args, w, rank, world, local_rank):
     n_kern = max(min(250, args.steps), args.steps // 5) // g_steps * g_steps or g_steps
     graph_kern = capture(evs_kern, True)
     graph_sd = capture(evs_sd, False, with_stats=False)
-    # this library's launches per step: the kernel nodes of a captured step
-    # less those of a captured L2 flush (torch's kernels); graphs kept
-    # uninstantiated for reading, never replayed
-    launches_per_step = None
+    # this library's launches per step (with and without a statistics
+    # build): the kernel nodes of a captured step less those of a captured L2
+    # flush (torch's kernels); graphs kept uninstantiated for reading, never
+    # replayed
+    launches = None
     if not args.no_graph:
-        g_one, g_flush = torch.cuda.CUDAGraph(keep_graph=True), torch.cuda.CUDAGraph(keep_graph=True)
-        with torch.cuda.graph(g_one):
+        counts = []
+        for with_stats in (False, True, None):
+            g_one = torch.cuda.CUDAGraph(keep_graph=True)
+            with torch.cuda.graph(g_one):
+                flush()
+                if with_stats is not None:
+                    step(None, torch.cuda.current_stream(dev), False, with_stats=with_stats)
+            counts.append(graph_kernel_nodes(g_one))
+            del g_one
+        if None not in counts:
+            launches = (counts[0] - counts[2], counts[1] - counts[2])
+
+    # the decode stream: every step decodes one token of every sequence
+    # (selection + sparse decode); a block completes every `block` steps and
+    # on that step its statistics are built as well.  The K timed steps hold
+    # round(K / block) such steps (the phase chosen to give that count); each
+    # step is replayed from a one-step graph and timed by its own events
+    per_block = w.block
+    phase = min(per_block - 1, max(0, per_block * round(args.steps / per_block) - args.steps))
+    is_build = [(i + phase) % per_block == per_block - 1 for i in range(args.steps)]
+    builds = sum(is_build)
+
+    def capture_one(ev, with_stats):
+        if args.no_graph:
+            return None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
             flush()
-            step(None, torch.cuda.current_stream(dev), False, one_stream=False)
-        with torch.cuda.graph(g_flush):
-            flush()
-        k_all, k_flush = graph_kernel_nodes(g_one), graph_kernel_nodes(g_flush)
-        if k_all is not None and k_flush is not None:
-            launches_per_step = k_all - k_flush
-        del g_one, g_flush
+            step(ev, torch.cuda.current_stream(dev), False, with_stats=with_stats)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        return g
+
+    ev_plain = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    ev_build = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    g_plain, g_build = capture_one(ev_plain, False), capture_one(ev_build, True)
+
+    def run_stream():
+        total = 0.0
+        for i in range(args.steps):
+            ev, g = (ev_build, g_build) if is_build[i] else (ev_plain, g_plain)
+            if g is not None:
+                g.replay()
+            else:
+                flush()
+                step(ev, None, False, with_stats=is_build[i])
+            torch.cuda.synchronize(dev)
+            total += ev[0].elapsed_time(ev[3])
+        return total / args.steps
+
     sums_step, sums_kern, sums_sd = [0.0] * 4, [0.0] * 4, [0.0] * 4
 
     clocks = ClockSampler(local_rank)
@@ -652,17 +704,19 @@ def run_cobs(args, w, rank, world, local_rank):
             step()
         torch.cuda.synchronize(dev)
     t_host0 = time.perf_counter()
-    run_timed(evs_step, graph_step, args.steps, False, sums_step)
+    t_stream = run_stream()
     t_host = (time.perf_counter() - t_host0) * 1e3 / args.steps   # wall time per step
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    run_timed(evs_step, graph_step, n_kern, False, sums_step)
+    torch.cuda.synchronize(dev)
     run_timed(evs_kern, graph_kern, n_kern, True, sums_kern)
     torch.cuda.synchronize(dev)
     run_timed(evs_sd, graph_sd, n_kern, False, sums_sd, with_stats=False)
     torch.cuda.synchronize(dev)
     clock_info = clocks.stop()
-    t_step = sums_step[3] / args.steps
+    t_every = sums_step[3] / n_kern
     t_stats, t_sel, t_dec, t_step_kern = (x / n_kern for x in sums_kern)
     t_sd = sums_sd[3] / n_kern
     status = cb.cobs_read_device_status(ws, ws_bytes, stream)
@@ -684,9 +738,7 @@ def run_cobs(args, w, rank, world, local_rank):
         vn_dev = torch.empty_like(vn_host, device=dev)
         h2d = q_host.numel() * 2 + kn_host.numel() * 2 + vn_host.numel() * 2
         d2h = out_host.numel() * 4 + lse_host.numel() * 4
-        n_e2e = max(g_steps, args.steps // 4 // g_steps * g_steps)
-
-        def e2e_step(pair, st=None):
+        def e2e_step(pair, st=None, with_stats=True):
             # torch copies go to the current stream: the capture stream inside
             # a graph capture, `stream` otherwise
             st = stream if st is None else st
@@ -696,43 +748,44 @@ def run_cobs(args, w, rank, world, local_rank):
             vn_dev.copy_(vn_host, non_blocking=True)
             k[:, :, w.seq_len - 1].copy_(kn_dev)
             v[:, :, w.seq_len - 1].copy_(vn_dev)
-            step(None, st)
+            step(None, st, with_stats=with_stats)
             out_host.copy_(out, non_blocking=True)
             lse_host.copy_(lse, non_blocking=True)
             pair[1].record(st)
 
         def time_e2e(use_graph):
-            ev = [(torch.cuda.Event(enable_timing=True, external=use_graph),
+            # the same stream of K steps as the device timing: a statistics
+            # build on the steps where a block completes
+            evp = (torch.cuda.Event(enable_timing=True, external=use_graph),
                    torch.cuda.Event(enable_timing=True, external=use_graph))
-                  for _ in range(g_steps)]
-            g = None
+            evb = (torch.cuda.Event(enable_timing=True, external=use_graph),
+                   torch.cuda.Event(enable_timing=True, external=use_graph))
+            graphs = {}
             if use_graph:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    cs = torch.cuda.current_stream(dev)
-                    for i in range(g_steps):
+                for with_stats, ev in ((False, evp), (True, evb)):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
                         flush()
-                        e2e_step(ev[i], cs)
-            for _ in range(3):
-                if g is not None:
-                    g.replay()
+                        e2e_step(ev, torch.cuda.current_stream(dev), with_stats)
+                    graphs[with_stats] = g
+            for i in range(3):
+                if use_graph:
+                    graphs[i == 2].replay()
                 else:
                     flush()
-                    e2e_step(ev[0])
+                    e2e_step(evb if i == 2 else evp, None, i == 2)
             torch.cuda.synchronize(dev)
             total = 0.0
-            for _ in range(n_e2e // g_steps):
-                if g is not None:
-                    g.replay()
-                    torch.cuda.synchronize(dev)
-                    total += sum(a.elapsed_time(b) for a, b in ev)
+            for i in range(args.steps):
+                ev = evb if is_build[i] else evp
+                if use_graph:
+                    graphs[is_build[i]].replay()
                 else:
-                    for _ in range(g_steps):
-                        flush()
-                        e2e_step(ev[0])
-                        torch.cuda.synchronize(dev)
-                        total += ev[0][0].elapsed_time(ev[0][1])
-            return total / n_e2e
+                    flush()
+                    e2e_step(ev, None, is_build[i])
+                torch.cuda.synchronize(dev)
+                total += ev[0].elapsed_time(ev[1])
+            return total / args.steps
 
         # the public-API calls and the per-step copies, replayed as CUDA
         # graphs (as a decode server drives them); and the same calls made one
@@ -743,14 +796,14 @@ def run_cobs(args, w, rank, world, local_rank):
         e2e = {"value": world * w.batch * w.q_heads / (t_e2e * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": t_e2e,
-               "launch": "CUDA graphs of the API calls and copies" if not args.no_graph
+               "launch": "one-step CUDA graphs of the API calls and copies" if not args.no_graph
                          else "one call at a time",
                "eager": {"value": world * w.batch * w.q_heads / (t_eager * 1e-3),
                          "ms_per_step": t_eager,
                          "launch": "one call at a time from Python"}}
 
-    t_step, t_stats, t_sel, t_dec, t_sd = max_over_ranks([t_step, t_stats, t_sel, t_dec, t_sd],
-                                                         dist, dev, world)
+    t_stream, t_every, t_stats, t_sel, t_dec, t_sd = max_over_ranks(
+        [t_stream, t_every, t_stats, t_sel, t_dec, t_sd], dist, dev, world)
     if rank != 0:
         return
 
@@ -765,19 +818,23 @@ def run_cobs(args, w, rank, world, local_rank):
     kernels = {name: {"ms": t, "bytes": b, "gbs": b / (t * 1e-3) / 1e9,
                       "frac_of_hbm": b / (t * 1e-3) / 1e9 / hbm}
                for name, (t, b, _) in per_kernel.items()}
-    # the kernel with the largest share of the step's critical path; a stats
-    # build that overlaps on the side stream is off that path
+    # the kernel with the largest share of the average stream step: the stats
+    # build runs on `builds` of the K steps (and off the critical path when it
+    # overlaps on the side stream)
+    weight = {"stats": builds / args.steps, "select": 1.0, "decode": 1.0}
     on_path = dict(per_kernel)
     if args.stats_stream == "side" and t_stats < t_sel + t_dec:
         on_path.pop("stats")
-    dom = max(on_path, key=lambda n: on_path[n][0])
+    dom = max(on_path, key=lambda n: on_path[n][0] * weight[n])
     t_dom, b_dom, file_dom = per_kernel[dom]
     achieved = b_dom / (t_dom * 1e-3) / 1e9
-    step_bytes = bm["select"] + bm["decode"] + bm["stats"]
-    value = world * w.batch * w.q_heads / (t_step * 1e-3)
+    # bytes of an average stream step: selection and decode every step, the
+    # statistics build on `builds` of the K steps
+    step_bytes = bm["select"] + bm["decode"] + bm["stats"] * builds / args.steps
+    value = world * w.batch * w.q_heads / (t_stream * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_stream,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "q_heads": w.q_heads,
@@ -786,34 +843,42 @@ def run_cobs(args, w, rank, world, local_rank):
                    "sink_blocks": w.sink_blocks, "local_tokens": w.local_tokens,
                    "selected_blocks_mean": n_sel_mean, "l2": "flushed between steps: 256 MiB written, then 256 MiB read",
                    "parallelism": f"replicas x{world}",
-                   "step": "stats of the completed block + select + sparse decode",
+                   "step": (f"one decode token of every sequence: select + sparse decode, "
+                            f"and the stats of the completed block on the steps where a "
+                            f"block completes (every {per_block}th)"),
+                   "blocks_completed_in_timed_steps": builds,
                    "stats_stream": args.stats_stream,
                    "stats_format": args.stats_format, "record_bytes": rec_bytes,
                    **({"subspace_dim": args.subspace_dim}
                       if args.stats_format == "subspace" else {}),
-                   "launch": (f"CUDA graphs of {g_steps} steps" if graph_step is not None
+                   "launch": ("one-step CUDA graphs, one replay per step" if g_plain is not None
                               else "one call at a time")},
-        "hbm_gbs_step": step_bytes / (t_step * 1e-3) / 1e9,
-        "hbm_frac_step": step_bytes / (t_step * 1e-3) / 1e9 / hbm,
+        "hbm_gbs_step": step_bytes / (t_stream * 1e-3) / 1e9,
+        "hbm_frac_step": step_bytes / (t_stream * 1e-3) / 1e9 / hbm,
         "kernels": kernels,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "traffic": recorded_traffic(file_dom, traffic_key)},
-        "gpu_launches": (round(launches_per_step * args.steps) if launches_per_step is not None
-                         else 3 * args.steps),
-        "gpu_launches_counted": ("kernel nodes of the captured step graphs, less the L2 flush's"
-                                 if launches_per_step is not None else
-                                 "3 per step (stats, select, decode), not read from a graph"),
-        "value_step": "every timed step builds the statistics of one completed block per "
-                      "(batch, kv-head) besides selection and decode (step_variants gives the "
-                      "steps without it)",
+        "gpu_launches": ((args.steps - builds) * launches[0] + builds * launches[1]
+                         if launches is not None else 2 * args.steps + builds),
+        "gpu_launches_counted": ("kernel nodes of the captured one-step graphs (with and "
+                                 "without the statistics build), less the L2 flush's"
+                                 if launches is not None else
+                                 "2 per step (select, decode) and 1 per build, not read "
+                                 "from a graph"),
         "clocks": clock_info,
         "setup_stats_build_ms": build_ms,
         **({"append_chunk_build": append} if append is not None else {}),
         "wall_ms_per_step": t_host,
         "quality": quality,
         "step_variants": {
+            "stats_every_step": {
+                "ms_per_step": t_every, "value": world * w.batch * w.q_heads / (t_every * 1e-3),
+                "hbm_frac": (bm["select"] + bm["decode"] + bm["stats"]) / (t_every * 1e-3) / 1e9
+                            / hbm,
+                "note": "every step also builds the statistics of one block per (batch, "
+                        f"kv-head) ({n_kern} graph-replayed steps, events at step boundaries)"},
             "select_decode": {
                 "ms_per_step": t_sd, "value": world * w.batch * w.q_heads / (t_sd * 1e-3),
                 "hbm_frac": (bm["select"] + bm["decode"]) / (t_sd * 1e-3) / 1e9 / hbm,
