@@ -33,8 +33,10 @@
  *   - Device pointers must be 16-byte aligned.  Host-side argument checks
  *     happen before anything is launched; a failed check returns an error
  *     code and launches nothing.
- *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = the
- *     legacy default stream) and may be captured into a CUDA graph.
+ *   - Calls that take a `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) are asynchronous on it.  The statistics, selection and decode
+ *     calls with a workspace (and their _varlen and _paged forms) may be
+ *     captured into a CUDA graph.
  *   - bf16 tensors are raw IEEE bfloat16 (uint16 bit patterns); all layouts
  *     are row-major with the innermost index last.
  *   - Device-side faults the kernels detect themselves (an out-of-range block
