@@ -13,7 +13,7 @@ import oracle.cobs_oracle as O
 from harness import (ENERGY_RTOL, LSE_ATOL, OUT_ATOL, PROJ_RTOL, TIE_RTOL, Problem,
                      block_is_gapped, explain_selection, from_dev_bits, score_change_bound,
                      selection_mismatch, stats_errors, to_dev)
-from workloads import WORKLOADS, bits_to_f64
+from workloads import WORKLOADS, bits_to_f64, to_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -354,4 +354,35 @@ def test_select_large_top_k(seq_len, top_k):
             assert list(got) == list(sel)
         else:
             assert selection_mismatch(got, sel, s, w) == []
+    assert p.device_status() == 0
+
+
+@pytest.mark.parametrize("top_k", [8, 100])
+def test_select_too_many_candidates_to_stage(top_k):
+    """16383 candidate blocks at head_dim 64 (a 1M-token cache): their scores
+    do not fit beside the top-k's work arrays in the 48 KB record ring, so the
+    top-k reads them from global memory instead of shared memory.  Records
+    are seeded random bf16 values (the statistics build is not under test);
+    the selection must equal the oracle's over the same records, and planted
+    exact ties must go to the lower block index."""
+    w = W["tiny_4k"].scaled(seq_len=1 << 20, top_k=top_k)
+    p = Problem(w)
+    rng = np.random.default_rng(17)
+    nfull = w.seq_len // w.block
+    shape = (nfull, 1 + w.rank, w.head_dim)
+    recs = rng.standard_normal(shape) * np.array([0.5] + [0.3] * w.rank)[None, :, None]
+    recs = bits_to_f64(to_bf16_bits(recs))
+    tied = [700, 900, 5000, 12000]
+    recs[tied[1:]] = recs[tied[0]]                 # exact ties: equal scores
+    p.upload_records(0, 0, recs)
+    p.select()
+    idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+    sel, s = O.select_from_records(p.q_group(0, 0), recs, w.seq_len, w.block, w.top_k,
+                                   w.sink_blocks, w.local_tokens)
+    got = idx[0, 0, :n[0, 0]]
+    assert np.all(np.diff(got) > 0)
+    assert len(got) == len(sel)
+    assert selection_mismatch(got, sel, s, w) == []
+    want, have = set(sel.tolist()), set(got.tolist())
+    assert [t in have for t in tied] == [t in want for t in tied]   # lower index first
     assert p.device_status() == 0
