@@ -528,14 +528,20 @@ def run_cobs(args, w, rank, world, local_rank):
             cb.cobs_build_block_stats(dims, k, nfull - 1, nfull, stats, ws, ws_bytes, st)
             if ev is not None:
                 ev[5].record(st)
-        if ev is not None:
+        if ev is None:
+            # one call: the decode takes each (batch, kv-head) as soon as its
+            # selection is written
+            cb.cobs_select_and_decode(dims, q, stats, k, v, w.seq_len, w.top_k, w.sink_blocks,
+                                      w.local_tokens, scale, idx, nsm, n_sel, None, out, lse,
+                                      ws, ws_bytes, st)
+        else:
+            # the kernels one by one, with events between them
             ev[1].record(st)
-        cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
-                              w.local_tokens, idx, nsm, n_sel, None, ws, ws_bytes, st)
-        if ev is not None:
+            cb.cobs_select_blocks(dims, q, stats, w.seq_len, w.top_k, w.sink_blocks,
+                                  w.local_tokens, idx, nsm, n_sel, None, ws, ws_bytes, st)
             ev[2].record(st)
-        cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
-                              ws, ws_bytes, st)
+            cb.cobs_sparse_decode(dims, q, k, v, idx, n_sel, nsm, w.seq_len, scale, out, lse,
+                                  ws, ws_bytes, st)
         if use_side:
             st.wait_event(join_ev)
         if evo is not None:

@@ -15,7 +15,8 @@ __all__ = [
     "cobs_workspace_bytes", "COBS_STATS_BF16", "COBS_STATS_FP4", "COBS_STATS_BOX",
     "COBS_STATS_SUBSPACE",
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
-    "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
+    "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_and_decode",
+    "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
     "cobs_read_device_status", "cobs_no_alloc_read_status", "cobs_set_wait_limit_ns",
     "cobs_last_error", "cobs_status_string",

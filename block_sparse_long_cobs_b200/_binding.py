@@ -23,7 +23,8 @@ __all__ = [
     "cobs_workspace_init", "cobs_build_block_stats", "cobs_select_blocks",
     "cobs_sparse_decode", "cobs_sparse_decode_no_alloc", "cobs_select_blocks_varlen",
     "cobs_sparse_decode_varlen", "cobs_build_block_stats_paged", "cobs_sparse_decode_paged",
-    "cobs_read_device_status", "cobs_no_alloc_read_status", "cobs_set_wait_limit_ns",
+    "cobs_select_and_decode", "cobs_read_device_status", "cobs_no_alloc_read_status",
+    "cobs_set_wait_limit_ns",
     "cobs_last_error",
     "cobs_status_string",
     "COBS_OK", "COBS_ERR_INVALID_ARG", "COBS_ERR_UNSUPPORTED",
@@ -94,6 +95,8 @@ def _load() -> ctypes.CDLL:
         "cobs_build_block_stats_paged": (I32, [D, P, I64, P, I32, I64, I64, P, P, SZ, P]),
         "cobs_sparse_decode_paged": (I32, [D, P, P, P, I64, P, I32, P, P, I32, P, I64, F32, P,
                                            P, P, SZ, P]),
+        "cobs_select_and_decode": (I32, [D, P, P, P, P, I64, I32, I32, I32, F32, P, I32, P, P,
+                                         P, P, P, SZ, P]),
         "cobs_read_device_status": (I32, [P, SZ, ctypes.POINTER(I32), P]),
         "cobs_no_alloc_read_status": (I32, [ctypes.POINTER(I32), P]),
         "cobs_set_wait_limit_ns": (I32, [ctypes.c_uint64]),
@@ -219,6 +222,17 @@ def cobs_sparse_decode(dims, q, k, v, idx, n_sel, idx_stride, seq_len, softmax_s
                                 ctypes.c_float(softmax_scale), _ptr(out), _ptr(lse),
                                 _ptr(ws), ws_bytes, _stream(stream))
     return _check("cobs_sparse_decode", st, check)
+
+
+def cobs_select_and_decode(dims, q, stats, k, v, seq_len, top_k, sink_blocks, local_tokens,
+                           softmax_scale, idx, idx_stride, n_sel, scores_opt, out, lse, ws,
+                           ws_bytes, stream=None, check=True) -> int:
+    st = lib.cobs_select_and_decode(ctypes.byref(_dims(dims)), _ptr(q), _ptr(stats), _ptr(k),
+                                    _ptr(v), seq_len, top_k, sink_blocks, local_tokens,
+                                    ctypes.c_float(softmax_scale), _ptr(idx), idx_stride,
+                                    _ptr(n_sel), _ptr(scores_opt), _ptr(out), _ptr(lse),
+                                    _ptr(ws), ws_bytes, _stream(stream))
+    return _check("cobs_select_and_decode", st, check)
 
 
 def cobs_sparse_decode_no_alloc(dims, q, k, v, idx, n_sel, idx_stride, seq_len,

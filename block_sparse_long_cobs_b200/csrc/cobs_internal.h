@@ -20,6 +20,7 @@ struct WorkspaceLayout {
   size_t status;       // int32 status word (+ padding)
   size_t sel_tickets;  // uint32 [batch * Hkv], selection arrival counters
   size_t dec_tickets;  // uint32 [batch * Hkv + 2], decode arrival counters + work counters
+  size_t handoff;      // uint32 [4] (epoch, published pairs) + uint64 [batch * Hkv] ready list
   size_t scores;       // float  [batch * Hkv * nb_cap], group scores
   size_t partials;     // float  [batch * Hq * n_sel_max * (d + 2)]
   size_t total;
@@ -57,6 +58,12 @@ struct SelectArgs {
   const int64_t* seq_lens;  // [b] or null
   int64_t max_seq_len;
   int32_t sink_blocks, local_tokens;
+  // selection handed to a decode launched right after it (null: not handed
+  // off): the CTA that finishes a pair appends (epoch + 1) << 32 | pair to
+  // ready_q at slot atomicAdd(&handoff[1], 1), after its writes of the pair's
+  // list and count; handoff[0] is the epoch, which only the decode changes
+  uint64_t* ready_q;
+  uint32_t* handoff;
 };
 
 // Columns of a stored subspace row: s rounded up to 8 (16-byte rows).
@@ -147,6 +154,10 @@ struct DecodeArgs {
   int32_t n_chunks;       // head_dim 128: chunks in the launch (pairs x chunks_per_pair)
   int32_t n_ctas;         // head_dim 128: grid size (persistent CTAs)
   float scale_log2;       // softmax_scale * log2(e)
+  // head_dim 128: the selection launched just before hands its pairs over as
+  // they finish (see SelectArgs); null: the lists are complete at launch
+  const uint64_t* ready_q;
+  uint32_t* handoff;
 };
 
 // Work split of one decode launch and the partial rows per query head it needs.

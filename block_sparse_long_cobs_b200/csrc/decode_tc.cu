@@ -93,7 +93,7 @@ __device__ __forceinline__ Segment chunk_segment(int64_t c, const DecodeArgs& a)
   g.pair = c / a.chunks_per_pair;
   g.seg = int(c % a.chunks_per_pair);
   g.n_seg = a.chunks_per_pair;
-  int nsel = a.n_sel[g.pair];
+  int nsel = __ldcg(a.n_sel + g.pair);   // L2: may come from a selection still running
   g.bad_nsel = nsel < 1 || nsel > a.idx_stride;
   nsel = nsel < 0 ? 0 : (nsel > a.idx_stride ? a.idx_stride : nsel);
   g.s0 = g.seg * a.chunk_slots;
@@ -183,7 +183,10 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     abort_s = 0;
   }
   if (warp == 0) tmem_alloc(&tmem_slot, kTmemCols);
-  pdl_wait();                // block lists and counts come from the launch before
+  // block lists and counts come from the launch before; handed over pair by
+  // pair when that launch is the selection (everything else it reads was
+  // complete before the selection started, which waited for it)
+  if (a.ready_q == nullptr) pdl_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,22 +199,60 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
       uint32_t it = 0;       // ring items issued
       int nonempty = 0;      // non-empty segments
       bool ok = true;
+      const uint32_t epoch = a.ready_q != nullptr ? __ldcg(a.handoff) : 0u;
       for (uint32_t ci = 0; ok; ++ci) {
         // ---- next chunk: the first one is the CTA's own index ----
         const int qs = ci % kChunkQ;
         if (ci >= kChunkQ &&
             !wait_or_abort(&cq_empty[qs], ((ci / kChunkQ) - 1) & 1, a.status, &abort_s))
           break;
-        const int64_t c = ci == 0 ? int64_t(blockIdx.x)
-                                  : int64_t(gridDim.x) + int64_t(atomicAdd(&a.work[0], 1u));
+        int64_t c = ci == 0 ? int64_t(blockIdx.x)
+                            : int64_t(gridDim.x) + int64_t(atomicAdd(&a.work[0], 1u));
+        if (a.ready_q != nullptr && c < a.n_chunks) {
+          // chunk c belongs to the (c / chunks_per_pair)-th pair the
+          // selection finishes: wait for its entry (bounded), then read the
+          // pair (acquire: its list and count are visible after this)
+          const uint64_t want = uint64_t(epoch + 1u);
+          const uint64_t* slot = a.ready_q + c / a.chunks_per_pair;
+          uint64_t e = ld_acquire_u64(slot);
+          if ((e >> 32) != want) {
+            const uint64_t t0 = global_timer_ns();
+            for (uint32_t tries = 1; (e >> 32) != want; ++tries) {
+              // polls spaced out, so that waiting CTAs load L2 no more than
+              // the selection CTAs still running need
+              __nanosleep(256);
+              if ((tries & 15u) == 0) {
+                if (abort_s) break;
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                  report(a.status, COBS_ERR_TIMEOUT);
+                  abort_s = 1;
+                  break;
+                }
+              }
+              e = ld_acquire_u64(slot);
+            }
+          }
+          if ((e >> 32) != want) {
+            ok = false;
+            c = a.n_chunks;   // the others see the end of the work and stop
+          } else {
+            c = int64_t(uint32_t(e)) * a.chunks_per_pair + c % a.chunks_per_pair;
+          }
+        }
         cq_val[qs] = c;
         mbar_arrive(&cq_full[qs]);
         if (c >= a.n_chunks) {
           // out of work: the last CTA to get here puts the counters back
+          // (and, after a handed-over selection, the ready list's count and
+          // a new epoch for the next one)
           __threadfence();
           if (atomicAdd(&a.work[1], 1u) == gridDim.x - 1) {
             a.work[0] = 0u;
             a.work[1] = 0u;
+            if (a.ready_q != nullptr) {
+              a.handoff[1] = 0u;
+              a.handoff[0] = epoch + 1u;
+            }
             __threadfence();
           }
           break;
@@ -231,7 +272,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const int nh = (2 * t + 1 < g.nb) ? 2 : 1;
             int y[2] = {0, 0}, zz[2] = {z, z};
             for (int h2 = 0; h2 < nh; ++h2) {
-              const int j = row[2 * t + h2];
+              const int j = __ldcg(row + 2 * t + h2);
               // an index outside the sequence (or a page outside the pool)
               // reads an all-zero box past the tensor maps' row bound
               const bool in_seq = j >= 0 && j < blocks_b;
@@ -481,7 +522,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
           const int blk = 2 * t + half;
           bool valid = false, zero_row = false;
           if (blk < g.nb) {
-            const int j = row[blk];
+            const int j = __ldcg(row + blk);
             if (j >= 0 && j < blocks_b) {
               valid = int64_t(j) * kBlock + kk < len_b;
               // a key past this sequence but inside the tensor maps' bound

@@ -196,6 +196,17 @@ __device__ __forceinline__ float hw_log2(float x) {
 // Warp reductions
 // ---------------------------------------------------------------------------
 
+// Release store / acquire load of a 64-bit word at GPU scope (a flag that
+// orders the writer's earlier writes before the reader's later reads).
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // 16-byte asynchronous copy global -> shared, cached in L2 only (both
 // addresses 16-byte aligned); complete for this thread after cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {

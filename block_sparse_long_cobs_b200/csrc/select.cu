@@ -1059,6 +1059,17 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       a.tickets[bh] = 0u;
     }
   }
+  if (a.ready_q != nullptr) {
+    // hand the pair to the decode: every write of its list and count is
+    // issued (barrier) and ordered before the ready entry (fence)
+    named_bar(3, kSelThreads);
+    if (tid == 0) {
+      __threadfence();
+      const uint32_t epoch = __ldcg(a.handoff);
+      const uint32_t slot = atomicAdd(&a.handoff[1], 1u);
+      st_release_u64(&a.ready_q[slot], (uint64_t(epoch + 1u) << 32) | uint32_t(bh));
+    }
+  }
 }
 
 template <int D, int kFmt>

@@ -35,8 +35,8 @@
  *     code and launches nothing.
  *   - Calls that take a `stream` (a cudaStream_t; NULL = the legacy default
  *     stream) are asynchronous on it.  The statistics, selection and decode
- *     calls with a workspace (and their _varlen and _paged forms) may be
- *     captured into a CUDA graph.
+ *     calls with a workspace (their _varlen and _paged forms, and
+ *     cobs_select_and_decode) may be captured into a CUDA graph.
  *   - bf16 tensors are raw IEEE bfloat16 (uint16 bit patterns); all layouts
  *     are row-major with the innermost index last.
  *   - Device-side faults the kernels detect themselves (an out-of-range block
@@ -72,7 +72,7 @@
 extern "C" {
 #endif
 
-#define COBS_ABI_VERSION 3
+#define COBS_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define COBS_API __attribute__((visibility("default")))
@@ -326,6 +326,28 @@ COBS_API cobs_status cobs_sparse_decode_paged(const cobs_dims* dims, const void*
                                      const int64_t* seq_lens, int64_t max_seq_len,
                                      float softmax_scale, float* out, float* lse,
                                      void* ws, size_t ws_bytes, void* stream);
+
+/* cobs_select_blocks followed by cobs_sparse_decode on the same stream and
+ * workspace, with the same arguments as the two calls (one seq_len for the
+ * batch, a contiguous cache; the workspace sized for both, i.e. by
+ * cobs_workspace_bytes), and the same results, bit for bit.  At head_dim 128,
+ * when there are enough (batch, kv-head) pairs for every pair to be one
+ * decode chunk, the decode does not wait for the whole selection: the
+ * selection appends each pair to a ready list in the workspace when its list
+ * and count are written, and the decode takes the pairs in that order as they
+ * arrive (each wait bounded; a wait that runs out is COBS_ERR_TIMEOUT in the
+ * status word), so the decode of early pairs overlaps the selection of late
+ * ones.  Otherwise (fewer pairs, or head_dim 64) the two kernels run in turn.
+ * Both calls are checked before either is launched.  If the decode cannot be
+ * launched after the selection was, the call fails and the workspace must be
+ * re-initialised (cobs_workspace_init) before its next use. */
+COBS_API cobs_status cobs_select_and_decode(const cobs_dims* dims, const void* q,
+                                   const void* stats, const void* k, const void* v,
+                                   int64_t seq_len, int32_t top_k, int32_t sink_blocks,
+                                   int32_t local_tokens, float softmax_scale, int32_t* idx,
+                                   int32_t idx_stride, int32_t* n_sel, float* scores_opt,
+                                   float* out, float* lse, void* ws, size_t ws_bytes,
+                                   void* stream);
 
 /* Allocation-free form of cobs_sparse_decode (this library's own addition; the
  * method's description has no counterpart).  Same arguments and results, but

@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_every_declared_symbol_is_exported():
     names = declared_functions()
-    assert len(names) == 18, names
+    assert len(names) == 19, names
     raw = ctypes.CDLL(cb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert cb.cobs_abi_version() == 3
+    assert cb.cobs_abi_version() == 4
     assert cb.cobs_status_string(0) == "COBS_OK"
     assert cb.cobs_status_string(5) == "COBS_ERR_TIMEOUT"
     assert cb.cobs_status_string(99) == "COBS_ERR_UNKNOWN"
@@ -62,9 +62,9 @@ def test_selected_capacity_and_workspace_size(name):
     ws = cb.cobs_workspace_bytes(d, w.top_k, w.sink_blocks, w.local_tokens)
     pairs = w.batch * w.kv_heads
     # status, selection tickets, decode tickets + the decode work counters (2),
-    # scores, split partials
-    want = 256 + align(pairs * 4) + align((pairs + 2) * 4) + align(pairs * (w.cap // 64) * 4) + \
-        align(w.batch * w.q_heads * nsm * (w.head_dim + 2) * 4)
+    # the hand-off (epoch, count, ready list), scores, split partials
+    want = 256 + align(pairs * 4) + align((pairs + 2) * 4) + align(16 + pairs * 8) + \
+        align(pairs * (w.cap // 64) * 4) + align(w.batch * w.q_heads * nsm * (w.head_dim + 2) * 4)
     assert ws == want
 
 
@@ -338,3 +338,26 @@ def test_subspace_dims_checks():
 def test_wait_limit_knob():
     assert cb.cobs_set_wait_limit_ns(5_000_000) == cb.COBS_OK
     assert cb.cobs_set_wait_limit_ns(0) == cb.COBS_OK     # back to the default
+
+
+def test_select_and_decode_checks_both_calls_before_launching():
+    """The fused call refuses anything either call would refuse, before it
+    launches anything: a selection argument (top_k above 4096, idx_stride
+    too short), a decode argument (softmax_scale), the workspace size."""
+    A = 1 << 20
+    w = WORKLOADS["single_32k"]
+    d = dims_of(w)
+    ws = cb.cobs_workspace_bytes(d, w.top_k, 1, w.local_tokens)
+    nsm = cb.cobs_selected_capacity(d, w.top_k, 1, w.local_tokens)
+    call = lambda top_k=w.top_k, stride=nsm, scale=0.1, ws_bytes=ws: cb.cobs_select_and_decode(
+        d, A, A, A, A, w.seq_len, top_k, 1, w.local_tokens, scale, A, stride, A, None, A, A,
+        A, ws_bytes)
+    for kw, code, text in [(dict(top_k=4097), cb.COBS_ERR_UNSUPPORTED, "top_k"),
+                           (dict(stride=nsm - 1), cb.COBS_ERR_INVALID_ARG, "idx_stride"),
+                           (dict(scale=-1.0), cb.COBS_ERR_INVALID_ARG, "softmax_scale"),
+                           (dict(scale=float("nan")), cb.COBS_ERR_INVALID_ARG, "softmax_scale"),
+                           (dict(ws_bytes=ws - 256), cb.COBS_ERR_WORKSPACE, "workspace")]:
+        with pytest.raises(cb.CobsError) as e:
+            call(**kw)
+        assert e.value.status == code, kw
+        assert text in cb.cobs_last_error(), (kw, cb.cobs_last_error())
