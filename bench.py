@@ -434,7 +434,15 @@ def run_cobs(args, w, rank, world, local_rank):
     if args.stats_format == "subspace":
         basis = torch.from_numpy(calibrate_subspace(w, args.subspace_dim)).to(dev)
         dims.update(subspace_dim=args.subspace_dim, subspace_basis=basis)
-    q, k, v = up(q_bits), up(k_bits), up(v_bits)
+    k, v = up(k_bits), up(v_bits)
+    # one device buffer for a step's inputs (the queries, then the appended
+    # token's K and V rows) and one for its results (out, then lse), so that
+    # the end-to-end step moves each with a single copy
+    nq = w.batch * w.q_heads * w.head_dim
+    nkv = w.batch * w.kv_heads * w.head_dim
+    inputs = torch.empty(nq + 2 * nkv, dtype=torch.int16, device=dev)
+    q = inputs[:nq].view(w.batch, w.q_heads, w.head_dim)
+    q.copy_(up(q_bits))
     nb_cap = w.cap // w.block
     nfull = w.seq_len // w.block
     rec_bytes = cb.cobs_stats_record_bytes(dims)
@@ -443,8 +451,9 @@ def run_cobs(args, w, rank, world, local_rank):
     nsm = cb.cobs_selected_capacity(dims, w.top_k, w.sink_blocks, w.local_tokens)
     idx = torch.zeros((w.batch, w.kv_heads, nsm), dtype=torch.int32, device=dev)
     n_sel = torch.zeros((w.batch, w.kv_heads), dtype=torch.int32, device=dev)
-    out = torch.zeros((w.batch, w.q_heads, w.head_dim), dtype=torch.float32, device=dev)
-    lse = torch.zeros((w.batch, w.q_heads), dtype=torch.float32, device=dev)
+    results = torch.zeros(w.batch * w.q_heads * (w.head_dim + 1), dtype=torch.float32, device=dev)
+    out = results[:nq].view(w.batch, w.q_heads, w.head_dim)
+    lse = results[nq:].view(w.batch, w.q_heads)
     ws_bytes = cb.cobs_workspace_bytes(dims, w.top_k, w.sink_blocks, w.local_tokens)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -733,30 +742,28 @@ def run_cobs(args, w, rank, world, local_rank):
     # appended token's K/V go host -> device, outputs come back
     e2e = None
     if not args.no_e2e:
-        q_host = torch.from_numpy(q_bits.view(np.int16)).pin_memory()
-        kn_host = torch.from_numpy(
-            np.ascontiguousarray(k_bits[:, :, w.seq_len - 1]).view(np.int16)).pin_memory()
-        vn_host = torch.from_numpy(
-            np.ascontiguousarray(v_bits[:, :, w.seq_len - 1]).view(np.int16)).pin_memory()
-        out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        kn_dev = torch.empty_like(kn_host, device=dev)
-        vn_dev = torch.empty_like(vn_host, device=dev)
-        h2d = q_host.numel() * 2 + kn_host.numel() * 2 + vn_host.numel() * 2
-        d2h = out_host.numel() * 4 + lse_host.numel() * 4
+        # pinned host images of the input and result buffers: the queries and
+        # the appended token's K and V rows in, out and lse back
+        inputs_host = torch.from_numpy(np.concatenate([
+            q_bits.view(np.int16).reshape(-1),
+            np.ascontiguousarray(k_bits[:, :, w.seq_len - 1]).view(np.int16).reshape(-1),
+            np.ascontiguousarray(v_bits[:, :, w.seq_len - 1]).view(np.int16).reshape(-1)]))
+        inputs_host = inputs_host.pin_memory()
+        results_host = torch.empty(results.shape, dtype=results.dtype).pin_memory()
+        kn_dev = inputs[nq:nq + nkv].view(w.batch, w.kv_heads, w.head_dim)
+        vn_dev = inputs[nq + nkv:].view(w.batch, w.kv_heads, w.head_dim)
+        h2d = inputs_host.numel() * 2
+        d2h = results_host.numel() * 4
         def e2e_step(pair, st=None, with_stats=True):
             # torch copies go to the current stream: the capture stream inside
             # a graph capture, `stream` otherwise
             st = stream if st is None else st
             pair[0].record(st)
-            q.copy_(q_host, non_blocking=True)
-            kn_dev.copy_(kn_host, non_blocking=True)
-            vn_dev.copy_(vn_host, non_blocking=True)
+            inputs.copy_(inputs_host, non_blocking=True)
             k[:, :, w.seq_len - 1].copy_(kn_dev)
             v[:, :, w.seq_len - 1].copy_(vn_dev)
             step(None, st, with_stats=with_stats)
-            out_host.copy_(out, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
+            results_host.copy_(results, non_blocking=True)
             pair[1].record(st)
 
         def time_e2e(use_graph):
