@@ -454,8 +454,9 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         named_bar(2, 128);   // contrib is rewritten by the next pass
       }
     }
+    __threadfence();         // this thread's scores, before the pair's ticket
     tc_fence_before();
-    __syncthreads();         // every score of the chunk is written (fenced before the ticket)
+    __syncthreads();         // every score of the chunk is written
     if (warp == 0) tmem_dealloc(tmem, 64);
     if (tid >= kSelThreads) return;   // the top-k below runs on warps 0-3 (named barrier 3)
   } else if constexpr (kSub) {
@@ -846,18 +847,15 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // ===================== arrival: last CTA of (b, kv-head) selects =========
   // (a pair scored by one CTA needs no ticket: its scores are this CTA's own)
   if (a.n_chunks > 1) {
-    // every thread's scores are written (barrier); one fence orders them
-    // before the ticket, and the last CTA's fence orders the other chunks'
-    // scores before its threads read them (after the second barrier)
+    __threadfence();
     named_bar(3, kSelThreads);
     if (tid == 0) {
-      __threadfence();
       const uint32_t prev = atomicAdd(&a.tickets[bh], 1u);
       last_s = (prev == uint32_t(a.n_chunks - 1));
-      if (last_s) __threadfence();
     }
     named_bar(3, kSelThreads);
     if (!last_s) return;
+    __threadfence();
   } else {
     named_bar(3, kSelThreads);   // every score of the pair is written
   }
