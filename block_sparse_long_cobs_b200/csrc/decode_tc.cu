@@ -71,7 +71,7 @@ constexpr int kOffP = kOffQ + 2 * 2048;
 constexpr int kDynSmem = kOffP + kPSlots * kPSlotBytes + 1024;
 
 static_assert(kOCol + 32 <= kTmemCols, "TMEM columns");
-static_assert(kSoftThreads == kD, "the merge gives thread r output dimension r");
+static_assert(kSoftThreads == kD, "the epilogue gives thread r output dimension r");
 // The query buffer of segment n is reloaded for segment n + 2 once ring item
 // (issue count - kStages) is free; every segment has >= 2 items (a K and a V
 // tile), so with kStages <= 4 that item is at or after segment n's last one,
@@ -422,7 +422,7 @@ sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     // Output rows of a finished segment, read back from TMEM output buffer
     // `ob` (phase `use`) one segment later, when its products have long been
     // complete.  A pair that is a single chunk is normalised here; otherwise
-    // the rows go to the partials and the pair's last chunk to arrive merges.
+    // the rows go to the partials, which merge_split_rows_kernel combines.
     auto epilogue = [&](const Segment& sg, bool has_o, int ob, uint32_t use, const float (&m)[G],
                         const float (&lpart)[G]) -> bool {
 #pragma unroll
