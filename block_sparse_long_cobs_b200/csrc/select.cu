@@ -901,15 +901,61 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   };
   __shared__ unsigned long long tau_s;
   __shared__ int tk_warp[kSelThreads / 32];
-  // a slot in the survivor list for each lane that asks (-1 for the others):
-  // one atomic per warp on the shared count (one per lane would be replayed
-  // once per lane, all lanes adding to the same word)
-  auto append_slot = [&](bool want) -> int {
-    const uint32_t ask = __ballot_sync(0xffffffffu, want);
-    int base = 0;
-    if (lane == 0 && ask != 0u) base = atomicAdd(&last_s, __popc(ask));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    return want ? base + __popc(ask & ((1u << lane) - 1u)) : -1;
+  // the rank (number of larger keys) of every survivor, passed with it to
+  // `use`: each thread takes up to four survivors per sweep and compares them
+  // all with every survivor it loads (one load per comparison of four)
+  auto rank_survivors = [&](int ns, auto use) {
+    for (int b0 = 0; b0 < ns; b0 += 4 * kSelThreads) {
+      uint64_t c[4];
+      int rank[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = b0 + q * kSelThreads + tid;
+        c[q] = i < ns ? surv[i] : ~0ull;
+        rank[q] = 0;
+      }
+#pragma unroll 8
+      for (int u = 0; u < ns; ++u) {
+        const uint64_t v = surv[u];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) rank[q] += v > c[q];
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (b0 + q * kSelThreads + tid < ns) use(c[q], rank[q]);
+    }
+  };
+  // the items i < n with key_at(i) >= tau, written to surv[0, count) (as many
+  // as fit) in any order; returns count.  Two strided passes over the items,
+  // the first counting, the second writing from the thread's offset (an
+  // exclusive scan of the counts): no atomic on a shared counter, whose
+  // latency would sit in every step of a single pass
+  auto compact = [&](int n, auto key_at, uint64_t tau) -> int {
+    int cnt = 0;
+    for (int i = tid; i < n; i += kSelThreads) cnt += key_at(i) >= tau;
+    int incl = cnt;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, m);
+      if (lane >= m) incl += y;
+    }
+    if (lane == 31) tk_warp[warp] = incl;
+    named_bar(3, kSelThreads);
+    int pos = incl - cnt, total = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kSelThreads / 32; ++w2) {
+      pos += w2 < warp ? tk_warp[w2] : 0;
+      total += tk_warp[w2];
+    }
+    for (int i = tid; i < n; i += kSelThreads) {
+      const uint64_t c = key_at(i);
+      if (c >= tau) {
+        if (pos < surv_cap) surv[pos] = c;
+        ++pos;
+      }
+    }
+    named_bar(3, kSelThreads);   // survivors written; tk_warp may be rewritten
+    return total;
   };
   const bool fits = surv_cap >= need;
   if (partial && fits) {
@@ -934,6 +980,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     for (int g = tid; g < ng; g += kSelThreads) {
       const int j0 = g * gs, j1 = min(n_cand, j0 + gs);
       uint64_t m = 0;
+#pragma unroll 4
       for (int jj = j0; jj < j1; ++jj) {
         const uint64_t c = key64(jj);
         m = c > m ? c : m;
@@ -942,70 +989,45 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       mine = m > mine ? m : mine;
     }
     tmax[tid] = mine;
-    if (tid == 0) {
-      last_s = 0;   // survivor count
-      tau_s = 0ull;
-    }
+    if (tid == 0) tau_s = 0ull;
     named_bar(3, kSelThreads);
     // tau1: the k-th largest thread maximum (thread maxima are distinct or 0;
     // at least min(ng, 128) > k of them are non-zero when k < 128)
     if (k < kSelThreads) {
       int rank = 0;
+#pragma unroll 16
       for (int u = 0; u < kSelThreads; ++u) rank += tmax[u] > mine;
       if (mine != 0 && rank == k - 1) tau_s = mine;
     }
     named_bar(3, kSelThreads);
     const uint64_t tau1 = tau_s;
-    for (int g0 = 0; g0 < ng; g0 += kSelThreads) {   // same trip count for all
-      const int g = g0 + tid;
-      const uint64_t c = g < ng ? gmax[g] : 0ull;
-      const int slot = append_slot(g < ng && c >= tau1);
-      if (slot >= 0 && slot < surv_cap) surv[slot] = c;
-    }
-    named_bar(3, kSelThreads);
-    const int ns1 = last_s < surv_cap ? last_s : surv_cap;
+    const int n1 = compact(ng, [&](int g) { return gmax[g]; }, tau1);
+    const int ns1 = n1 < surv_cap ? n1 : surv_cap;
     if (gs == 1) {
       // groups are single candidates: the survivors are the candidate keys
       // >= tau1, which hold the top k; rank them directly
-      if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
-      for (int i = tid; i < ns1; i += kSelThreads) {
-        const uint64_t c = surv[i];
-        int rank = 0;
-        for (int u = 0; u < ns1; ++u) rank += surv[u] > c;
+      if (tid == 0 && n1 > surv_cap) report(a.status, COBS_ERR_DEVICE);
+      rank_survivors(ns1, [&](uint64_t c, int rank) {
         if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
-      }
+      });
       named_bar(3, kSelThreads);
     } else {
       // tau2: the k-th largest group maximum (0 when there are fewer than k groups)
       if (k <= ng) {
-        for (int i = tid; i < ns1; i += kSelThreads) {
-          const uint64_t c = surv[i];
-          int rank = 0;
-          for (int u = 0; u < ns1; ++u) rank += surv[u] > c;
+        rank_survivors(ns1, [&](uint64_t c, int rank) {
           if (rank == k - 1) tau_s = c;
-        }
+        });
       } else if (tid == 0) {
         tau_s = 0ull;
       }
       named_bar(3, kSelThreads);
       const uint64_t tau2 = tau_s;
-      if (tid == 0) last_s = 0;
-      named_bar(3, kSelThreads);
-      for (int j0 = 0; j0 < n_cand; j0 += kSelThreads) {   // same trip count for all
-        const int jj = j0 + tid;
-        const uint64_t c = jj < n_cand ? key64(jj) : 0ull;
-        const int slot = append_slot(jj < n_cand && c >= tau2);
-        if (slot >= 0 && slot < surv_cap) surv[slot] = c;
-      }
-      named_bar(3, kSelThreads);
-      const int ns = last_s < surv_cap ? last_s : surv_cap;
-      if (tid == 0 && last_s > surv_cap) report(a.status, COBS_ERR_DEVICE);
-      for (int i = tid; i < ns; i += kSelThreads) {
-        const uint64_t c = surv[i];
-        int rank = 0;
-        for (int u = 0; u < ns; ++u) rank += surv[u] > c;
+      const int n2 = compact(n_cand, key64, tau2);
+      const int ns = n2 < surv_cap ? n2 : surv_cap;
+      if (tid == 0 && n2 > surv_cap) report(a.status, COBS_ERR_DEVICE);
+      rank_survivors(ns, [&](uint64_t c, int rank) {
         if (rank < k) chosen_s[0xFFFFFFFFu - uint32_t(c)] = 1;
-      }
+      });
       named_bar(3, kSelThreads);
     }
     // the chosen blocks in ascending order: thread t counts the flags of its
