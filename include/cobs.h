@@ -361,8 +361,7 @@ COBS_API cobs_status cobs_select_and_decode(const cobs_dims* dims, const void* q
  * is forbidden or too slow (a real-time or latency-critical loop, an
  * allocator callback), or bindings without a device allocator at all.
  *   - The first call on a device looks the array's device address up
- *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture.
+ *     (cudaGetSymbolAddress) and caches it.
  *   - All calls share the one array, which keeps the last call's contents;
  *     the arrival counters are cleared at the start of every call.  Calls
  *     that overlap on the GPU (for example on two streams at once) race on
