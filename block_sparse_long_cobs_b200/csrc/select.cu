@@ -35,6 +35,7 @@
 #include <cfloat>
 
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "device_common.cuh"
 #include "tcgen05.cuh"
@@ -47,10 +48,17 @@ constexpr int kSelStages = 3;
 constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
 constexpr int kTopkGroups = 1024; // candidate groups of the top-k bound
 constexpr int kSubStages = 2;     // record ring of the subspace kind
+// FP4 records read by kind::f8f6f4 products (d = 128, r = 8 or 16): a stage
+// holds the mu rows of up to 16 records (two 64-column slabs of 2 KB) and
+// their 128 code rows (16 KB)
+constexpr int kFdStages = 4;
+constexpr int kFdStageBytes = 20480;
 
-// Bytes of the record ring (which the top-k phase reuses) by record kind.
+// Bytes of the record ring (which the top-k phase reuses) by record kind
+// (4: FP4 records read by kind::f8f6f4 products).
 __host__ __device__ constexpr int ring_bytes(int d, int fmt) {
-  return (fmt == 3 ? kSubStages : kSelStages) * (d / 64) * 128 * 128;
+  return fmt == 4 ? kFdStages * kFdStageBytes
+                  : (fmt == 3 ? kSubStages : kSelStages) * (d / 64) * 128 * 128;
 }
 
 // Candidates per group of the top-k bound (groups never empty: at most 1024).
@@ -112,13 +120,17 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// kFmt: 0 bf16 COBS records [mu; U^T], 1 FP4 COBS records, 2 min/max box
-// records [lo; hi], 3 subspace records [mu; U_s^T].
+// kFmt: 0 bf16 COBS records [mu; U^T], 1 FP4 COBS records (codes widened by
+// threads), 2 min/max box records [lo; hi], 3 subspace records [mu; U_s^T],
+// 4 FP4 COBS records read by kind::f8f6f4 products (d = 128, r = 8 or 16).
 template <int D, int G, int kFmt>
-__global__ void __launch_bounds__(kFmt == 1 ? 288 : 128, kFmt == 1 ? 2 : 1)
+__global__ void __launch_bounds__(kFmt == 1 ? 288 : (kFmt == 4 ? 160 : 128),
+                                  kFmt == 1 || kFmt == 4 ? 2 : 1)
 select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                      const __grid_constant__ CUtensorMap qmap, const SelectArgs a) {
   constexpr bool kFp4 = kFmt == 1;
+  constexpr bool kFp4d = kFmt == 4;
+  static_assert(!kFp4d || D == 128, "kind::f8f6f4 FP4 selection is for d = 128");
   constexpr bool kBox = kFmt == 2;
   constexpr bool kSub = kFmt == 3;
   constexpr int kRegions = D / 64;                  // 64-column slabs of a row
@@ -156,7 +168,275 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   const BlockPartition BP = block_partition(seq_len_b, a.sink_blocks, a.local_tokens);
 
   // ===================== phase 1: scores of this chunk =====================
-  if constexpr (kFp4) {
+  if constexpr (kFp4d) {
+    // FP4 records (COBS explainer §2.3, quantisation: mu bf16 [D] | E2M1
+    // codes [r][D/2] | scale exponents [r][D/32]) read by the tensor cores as
+    // they are stored: kind::f8f6f4 products take the E2M1 codes from shared
+    // memory, so no thread converts them.  A pass is per_pass = 128 / r whole
+    // records of one ring stage, brought by two tensor maps over the records:
+    // the mu rows (both 64-column slabs, bf16) and the r code rows of every
+    // record (3-d: component, row, record), whose element type lands every 16
+    // codes in the low half of a 16-byte unit, the layout the products read.
+    // Per pass, into one of two accumulator buffers:
+    //  * q . mu: kind::f16, the mu rows against the bf16 queries (N = 16),
+    //    columns [0, 16).  It spans 128 operand rows; those past the pass's
+    //    records read the rest of the stage and are never read back;
+    //  * q . codes per group g of 32 components: kind::f8f6f4, E2M1 codes
+    //    against the queries as E4M3 (N = 16), columns [16 + 16 g, 32 + 16 g).
+    //    Query row h is scaled by 2^(6 - E_h), E_h the exponent of its
+    //    largest component, and split into hi + lo (operand rows h and
+    //    G + h); two E4M3 parts hold a bf16 value exactly (components below
+    //    2^-9 of the row's largest round at 2^-17 of it).
+    // The epilogue forms u . q_h = 2^(E_h - 6) sum_g 2^(e_g - 127)
+    // (hi_g + lo_g) in fp32 from these exact products.
+    // Roles: warps 0-3 read an accumulator back (TMEM lane = operand row =
+    // thread), fetch their row's scale bytes one pass ahead, and write the
+    // scores; warp 4 (one thread) issues the copies into a kFdStages-slot
+    // ring and the products.  mbarriers: fd_full (a stage's copies landed),
+    // mma_done (a pass's products complete: its stage may be refilled and
+    // its accumulator read), fd_acc_free (the epilogue has read it).
+    const int r = a.rank;
+    const int per_pass = kStageRows / r;
+    const int rec = int(a.rec_bytes);
+    const int c_nom = a.cand_begin + chunk * a.chunk_blocks;
+    const int c_lo = max(int(BP.sink_end), c_nom);
+    const int c_hi = min(int(BP.first_local), min(a.cand_end, c_nom + a.chunk_blocks));
+    const int npass = c_hi > c_lo ? (c_hi - c_lo + per_pass - 1) / per_pass : 0;
+    const int rec0 = int(int64_t(bh) * a.nb_cap);   // first record (map row) of this pair
+    const uint8_t* recs =
+        reinterpret_cast<const uint8_t*>(a.stats) + int64_t(bh) * a.nb_cap * a.rec_bytes;
+    uint8_t* q8tile = base + kQBytes;               // [16 rows][128 B] E4M3 query parts
+    uint8_t* ring = q8tile + 2048;                  // [kFdStages][kFdStageBytes]
+    __shared__ __align__(8) uint64_t fd_full[kFdStages];
+    __shared__ __align__(8) uint64_t fd_acc_free[2];
+    __shared__ float qinv_s[8];                     // 2^(E_h - 6)
+    __shared__ __align__(16) float contrib_mu[16 * 8];
+    __shared__ volatile int fd_abort;
+    constexpr int kIssuer = 4 * 32;                 // warp 4, lane 0
+
+    if (tid == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
+      for (int s2 = 0; s2 < kFdStages; ++s2) mbar_init(&fd_full[s2], 1);
+      for (int s2 = 0; s2 < 2; ++s2) {
+        mbar_init(&mma_done[s2], 1);
+        mbar_init(&fd_acc_free[s2], 1);
+      }
+      fence_barrier_init();
+      fd_abort = 0;
+    }
+    if (warp == 0) tmem_alloc(&tmem_slot, 256);
+    pdl_wait();              // queries and records may come from the launch before
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_launch_dependents();
+    const uint32_t tmem = tmem_slot;   // buffer b at column 128 b: mu . q at +0, groups at +16
+
+    int n_issued = 0;          // issuing thread: passes whose copies were issued
+    int n_mma = 0;             // issuing thread: passes whose products were issued
+    auto issue = [&](int p) {  // issuing thread only: the records of pass p
+      n_issued = p + 1;
+      const int st = p % kFdStages;
+      const int j0 = c_lo + p * per_pass;
+      uint8_t* dst = ring + st * kFdStageBytes;
+      // the boxes are always per_pass records; records past the chunk are
+      // ignored (past the array they read as zero).  Code bytes count packed.
+      mbar_arrive_expect_tx(&fd_full[st],
+                            uint32_t(per_pass) * (uint32_t(kRegions) * 128u + uint32_t(r * D / 2)));
+      tma_load_2d(dst, &smap, 0, rec0 + j0, &fd_full[st]);
+      tma_load_2d(dst + 2048, &smap, 64, rec0 + j0, &fd_full[st]);
+      tma_load_3d(dst + 4096, &qmap, 0, 0, rec0 + j0, &fd_full[st]);
+    };
+    if (tid == kIssuer)
+      for (int p = 0; p < kFdStages && p < npass; ++p) issue(p);
+
+    // ---- the query operands: bf16 rows for mu, E4M3 hi / lo rows for codes
+    for (int e2 = tid; e2 < (kQBytes + 2048) / 16; e2 += kSelThreads + 32)
+      reinterpret_cast<uint4*>(qtile)[e2] = make_uint4(0u, 0u, 0u, 0u);   // qtile, q8tile
+    __syncthreads();
+    {
+      // thread h * 16 + ch: components 8 ch .. 8 ch + 7 of query row h
+      const int h = tid >> 4, ch = tid & 15;
+      const bool act = h < G;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (act) w = *reinterpret_cast<const uint4*>(a.q + (int64_t(b) * a.hq + kvh * G + h) * D + ch * 8);
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = bf16x2_to_float2(wv[i]);
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+      }
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      // E = the exponent field of the row maximum less the bias, kept in
+      // [-100, 120] so both powers of two below are normal fp32 values
+      int E = int((__float_as_uint(m) >> 23) & 0xFFu) - 127;
+      E = E < -100 ? -100 : (E > 120 ? 120 : E);
+      const float sc = __uint_as_float(uint32_t(133 - E) << 23);    // 2^(6 - E)
+      if (act) {
+        if (ch == 0) qinv_s[h] = __uint_as_float(uint32_t(121 + E) << 23);   // 2^(E - 6)
+        *reinterpret_cast<uint4*>(qtile + (ch >> 3) * 16 * 128 + h * 128 +
+                                  (((ch & 7) ^ h) << 4)) = w;
+        uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float v = x[i] * sc;
+          const __nv_fp8_storage_t hb = __nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+          const float hv = __half2float(__half(__nv_cvt_fp8_to_halfraw(hb, __NV_E4M3)));
+          const __nv_fp8_storage_t lb = __nv_cvt_float_to_fp8(v - hv, __NV_SATFINITE, __NV_E4M3);
+          hw[i >> 2] |= uint32_t(hb) << (8 * (i & 3));
+          lw[i >> 2] |= uint32_t(lb) << (8 * (i & 3));
+        }
+        // component 8 ch + i: 16-byte unit ch / 2, byte 8 (ch & 1) + i
+        const int u = ch >> 1, o8 = (ch & 1) * 8;
+        *reinterpret_cast<uint2*>(q8tile + h * 128 + ((u ^ (h & 7)) << 4) + o8) =
+            make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2*>(q8tile + (G + h) * 128 + ((u ^ ((G + h) & 7)) << 4) + o8) =
+            make_uint2(lw[0], lw[1]);
+      }
+    }
+    fence_proxy_async_smem();   // generic-proxy operand writes -> tensor-core reads
+    __syncthreads();
+
+    if (warp == 4) {
+      // ============================= issue ==============================
+      if (lane == 0) {
+        constexpr uint32_t idesc_mu = umma_idesc_bf16(128, 16);
+        constexpr uint32_t idesc_u = umma_idesc_e2m1_e4m3(128, 16);
+        const uint32_t qb = smem_addr(qtile), q8b = smem_addr(q8tile);
+        for (int p = 0; p < npass; ++p) {
+          const int st = p % kFdStages, buf = p & 1;
+          bool ok = fd_abort == 0 &&
+                    wait_or_abort(&fd_full[st], (p / kFdStages) & 1, a.status, &fd_abort);
+          // the epilogue has read this accumulator's pass p - 2
+          if (ok && p >= 2)
+            ok = wait_or_abort(&fd_acc_free[buf], ((p - 2) >> 1) & 1, a.status, &fd_abort);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sb = smem_addr(ring + st * kFdStageBytes);
+          const uint32_t acc = tmem + 128u * uint32_t(buf);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint64_t ad = umma_desc_sw128(sb + (ks >> 2) * 2048 + (ks & 3) * 32);
+            const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
+            umma_bf16(acc, ad, bd, idesc_mu, ks > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int g = 0; g < D / 32; ++g)
+            umma_f8f6f4(acc + 16u + 16u * uint32_t(g), umma_desc_sw128(sb + 4096 + 32 * g),
+                        umma_desc_sw128(q8b + 32 * g), idesc_u, 0u);
+          umma_commit(&mma_done[buf]);
+          n_mma = p + 1;
+          // refill the slot of pass p - 1, whose products were issued a pass ago
+          if (p >= 1 && p - 1 + kFdStages < npass) {
+            if (!wait_or_abort(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1, a.status, &fd_abort))
+              break;
+            issue(p - 1 + kFdStages);
+          }
+        }
+        // let the copies and the products still in flight land before TMEM is
+        // freed and the CTA leaves (each wait bounded)
+        for (int p = n_mma; p < n_issued; ++p)
+          (void)mbar_wait_bounded(&fd_full[p % kFdStages], (p / kFdStages) & 1, a.status);
+        for (int p = n_mma > 2 ? n_mma - 2 : 0; p < n_mma; ++p)
+          (void)mbar_wait_bounded(&mma_done[p & 1], (p >> 1) & 1, a.status);
+      }
+    } else {
+      // ============================ epilogue ============================
+      const int et = tid;                            // TMEM lane, operand row
+      const float inv_sqrt_d = rsqrtf(float(D));
+      const float ln_n = logf(float(kBlock));
+      float qinv[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) qinv[h] = qinv_s[h] * inv_sqrt_d;
+      const int sc_off = 2 * D + r * (D / 2);        // scale bytes of row 0 of a record
+      auto scale_word = [&](int p) -> uint32_t {     // this row's 4 group exponents
+        const int j0 = c_lo + p * per_pass;
+        const int nb = min(per_pass, c_hi - j0);
+        if (et >= nb * r) return 0u;
+        const int jj = et / r, k = et - jj * r;
+        return __ldg(reinterpret_cast<const uint32_t*>(recs + int64_t(j0 + jj) * rec + sc_off +
+                                                       k * (D / 32)));
+      };
+      uint32_t sc_next = npass > 0 ? scale_word(0) : 0u;
+      for (int p = 0; p < npass; ++p) {
+        const int buf = p & 1;
+        const uint32_t scw = sc_next;
+        if (p + 1 < npass) sc_next = scale_word(p + 1);
+        bool fail = fd_abort != 0;
+        if (!fail && et == 0)
+          fail = !wait_or_abort(&mma_done[buf], (p >> 1) & 1, a.status, &fd_abort);
+        if (named_bar_or(2, 128, fail)) break;
+        if (et != 0) (void)mbar_try_wait(&mma_done[buf], (p >> 1) & 1);
+        tc_fence_after();
+        const int j0 = c_lo + p * per_pass;
+        const int nb = min(per_pass, c_hi - j0);
+        const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 128u * uint32_t(buf);
+        uint32_t vm[8];
+        float vu0[32], vu1[32];
+        tmem_ld8_nowait(lane_base, vm);
+        tmem_ld32(lane_base + 16u, vu0);             // groups 0, 1
+        tmem_ld32(lane_base + 48u, vu1);             // groups 2, 3 (waits for all three)
+        tc_fence_before();
+        if (et < nb * r) {
+          float s4[4];
+#pragma unroll
+          for (int g = 0; g < 4; ++g) s4[g] = __uint_as_float(((scw >> (8 * g)) & 0xFFu) << 23);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float x = s4[0] * (vu0[h] + vu0[G + h]);
+            x = fmaf(s4[1], vu0[16 + h] + vu0[16 + G + h], x);
+            x = fmaf(s4[2], vu1[h] + vu1[G + h], x);
+            x = fmaf(s4[3], vu1[16 + h] + vu1[16 + G + h], x);
+            x *= qinv[h];
+            contrib[et * 8 + h] = 0.5f * x * x;
+          }
+        }
+        if (et < nb) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) contrib_mu[et * 8 + h] = __uint_as_float(vm[h]) * inv_sqrt_d;
+        }
+        named_bar(2, 128);
+        // the accumulator has been read: its next products may start
+        if (et == 0) mbar_arrive(&fd_acc_free[buf]);
+        // per block and head: mu row + its r code rows, then LSE over the heads
+        for (int t0 = 0; t0 < per_pass * G; t0 += 128) {
+          const int t = t0 + et;
+          const int jj = t / G, h = t % G;
+          const bool valid = jj < nb;
+          float sacc = 0.f;
+          if (valid) {
+            sacc = contrib_mu[jj * 8 + h];
+            for (int i = 0; i < r; ++i) sacc += contrib[(jj * r + i) * 8 + h];
+          }
+          const float sh = sacc + ln_n;
+          float mx = sh;
+#pragma unroll
+          for (int m = G / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m, G));
+          float e = __expf(sh - mx);
+#pragma unroll
+          for (int m = G / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m, G);
+          if (valid && h == 0) {
+            const float S = mx + __logf(e);
+            scores[j0 + jj] = S;
+            if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
+          }
+        }
+        named_bar(2, 128);   // contrib is rewritten by the next pass
+      }
+    }
+    __threadfence();         // this thread's scores, before the pair's ticket
+    tc_fence_before();
+    __syncthreads();         // every score of the chunk is written
+    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (tid >= kSelThreads) return;   // the top-k below runs on warps 0-3 (named barrier 3)
+  } else if constexpr (kFp4) {
     // FP4 records (COBS explainer §2.3, quantisation): mu bf16 [D] | E2M1
     // codes [r][D/2] | scale exponents [r][D/32] | padding.  288 threads in
     // three roles that work on different passes at once:
@@ -1102,10 +1382,12 @@ constexpr size_t dyn_smem_bytes() {
          (kFmt == 1 ? size_t(2) * (D / 64) * 128 * 128 + size_t(kSelFp4RawStages) *
                                                              fp4_raw_stage_bytes(D)
                     : size_t(ring_bytes(D, kFmt))) +
-         (kFmt == 3 ? size_t(2) * 32 * 128 : 0);
+         (kFmt == 3 ? size_t(2) * 32 * 128 : 0) + (kFmt == 4 ? size_t(2048) : 0);
 }
 template <int kFmt>
-constexpr int sel_threads() { return kFmt == 1 ? 2 * kSelThreads + 32 : kSelThreads; }
+constexpr int sel_threads() {
+  return kFmt == 1 ? 2 * kSelThreads + 32 : (kFmt == 4 ? kSelThreads + 32 : kSelThreads);
+}
 
 template <int D, int G, int kFmt>
 cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
@@ -1119,6 +1401,18 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (kFp4) {
     map = qmap;   // FP4 records arrive by plain bulk copies; the map is unused
+  } else if (kFmt == 4) {
+    // mu rows: the first D columns of every record; code rows: (component,
+    // row, record) starting 2 D bytes into the records
+    const uint64_t n_rec = uint64_t(a.batch) * a.hkv * a.nb_cap;
+    const int per_pass = kStageRows / a.rank;
+    e = make_bf16_tensor_map_rows_sw128(&map, a.stats, D, n_rec, uint64_t(a.rec_bytes), per_pass);
+    if (e != cudaSuccess) return e;
+    e = make_e2m1_unpacked_tensor_map_3d_sw128(&qmap,
+                                               reinterpret_cast<const uint8_t*>(a.stats) + 2 * D,
+                                               D, uint64_t(a.rank), n_rec, uint64_t(D / 2),
+                                               uint64_t(a.rec_bytes), a.rank, per_pass);
+    if (e != cudaSuccess) return e;
   } else if (kFmt == 3) {
     // mu rows: the first D columns of every record; U_s rows: (coordinate,
     // row, record) starting 2 D bytes into the records
@@ -1173,11 +1467,22 @@ cudaError_t dispatch_dim(const SelectArgs& a, cudaStream_t s) {
   return a.d == 64 ? dispatch_group<64, kFmt>(a, s) : dispatch_group<128, kFmt>(a, s);
 }
 
+// FP4 records whose codes the tensor cores can read as stored: d = 128, r =
+// 8 or 16 (a pass is 128 / r whole records), records a multiple of 32 bytes
+// apart and the array 32-byte aligned (the code map's requirements).
+bool fp4_direct_shape(int d, int rank) { return d == 128 && (rank == 8 || rank == 16); }
+bool fp4_direct(const SelectArgs& a) {
+  return fp4_direct_shape(a.d, a.rank) && a.rec_bytes % 32 == 0 &&
+         reinterpret_cast<uintptr_t>(a.stats) % 32 == 0;
+}
+
 }  // namespace
 
-int select_ctas_per_sm(int d, int g, int /*rank*/, int fmt) {
+int select_ctas_per_sm(int d, int g, int rank, int fmt) {
   switch (fmt) {
-    case 1: return d == 64 ? occupancy_group<64, 1>(g) : occupancy_group<128, 1>(g);
+    case 1:
+      if (fp4_direct_shape(d, rank)) return occupancy_group<128, 4>(g);
+      return d == 64 ? occupancy_group<64, 1>(g) : occupancy_group<128, 1>(g);
     case 2: return d == 64 ? occupancy_group<64, 2>(g) : occupancy_group<128, 2>(g);
     case 3: return d == 64 ? occupancy_group<64, 3>(g) : occupancy_group<128, 3>(g);
     default: return d == 64 ? occupancy_group<64, 0>(g) : occupancy_group<128, 0>(g);
@@ -1185,14 +1490,14 @@ int select_ctas_per_sm(int d, int g, int /*rank*/, int fmt) {
 }
 
 int select_blocks_per_stage(int d, int rank, int fmt) {
-  if (fmt == 1) return fp4_blocks_per_pass(d, rank);
+  if (fmt == 1) return fp4_direct_shape(d, rank) ? kStageRows / rank : fp4_blocks_per_pass(d, rank);
   if (fmt == 3) return subspace_blocks_per_pass(rank);
   return kStageRows / (fmt == 2 ? 2 : 1 + rank);
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   switch (a.stats_format) {
-    case 1: return dispatch_dim<1>(a, stream);
+    case 1: return fp4_direct(a) ? dispatch_group<128, 4>(a, stream) : dispatch_dim<1>(a, stream);
     case 2: return dispatch_dim<2>(a, stream);
     case 3: return dispatch_dim<3>(a, stream);
     default: return dispatch_dim<0>(a, stream);
@@ -1202,7 +1507,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
 bool select_topk_fits(int d, int fmt, int64_t n_cand, int top_k) {
   if (top_k <= 0 || top_k >= n_cand) return true;   // no ranking needed
   if (n_cand > (int64_t(1) << 24)) return false;
-  const int ring = ring_bytes(d, fmt);
+  // FP4 records may be selected by either kernel: the smaller ring bounds both
+  const int ring = fmt == 1 && d == 128 ? min(ring_bytes(d, 1), ring_bytes(d, 4)) : ring_bytes(d, fmt);
   return topk_survivor_capacity(ring, int(n_cand)) >= topk_survivors_needed(int(n_cand), top_k);
 }
 

@@ -92,12 +92,30 @@ constexpr uint32_t umma_idesc_f16(int M, int N) {
 // Same with A MN-major (bit 15).
 constexpr uint32_t umma_idesc_bf16_amn(int M, int N) { return umma_idesc_bf16(M, N) | (1u << 15); }
 
+// Instruction descriptor, kind::f8f6f4: D fp32, A E2M1 (format 5), B E4M3
+// (format 0), both K-major.  A's E2M1 operand sits in shared memory with
+// every 16 codes (8 bytes) in the low half of a 16-byte unit.
+constexpr uint32_t umma_idesc_e2m1_e4m3(int M, int N) {
+  return (1u << 4) | (5u << 7) | (0u << 10) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// One kind::f8f6f4 product (K = 32 per instruction).
+__device__ __forceinline__ void umma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -207,5 +225,17 @@ cudaError_t make_bf16_tensor_map_3d_sw128_box(CUtensorMap* map, const void* base
                                               uint64_t dim1, uint64_t dim2,
                                               uint64_t stride1_bytes, uint64_t stride2_bytes,
                                               int box1, int box2);
+
+// Host: 3-d tensor map (component, row, record) over packed E2M1 codes (two
+// per byte, `cols` components a row, rows `stride1_bytes` apart, records
+// `stride2_bytes` apart; base 32-byte aligned, strides multiples of 32, cols
+// a multiple of 128), box of 128 components x box1 x box2, 128-byte swizzle.
+// The copy lands every 16 codes in the low half of a 16-byte unit (128 bytes
+// of shared memory per 128-component row): the E2M1 operand layout of
+// kind::f8f6f4 products.  Its transaction bytes are the packed bytes.
+cudaError_t make_e2m1_unpacked_tensor_map_3d_sw128(CUtensorMap* map, const void* base, int cols,
+                                                   uint64_t dim1, uint64_t dim2,
+                                                   uint64_t stride1_bytes,
+                                                   uint64_t stride2_bytes, int box1, int box2);
 
 }  // namespace cobs

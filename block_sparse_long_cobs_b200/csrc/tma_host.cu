@@ -89,4 +89,24 @@ cudaError_t make_bf16_tensor_map_3d_sw128_box(CUtensorMap* map, const void* base
   return cudaSuccess;
 }
 
+cudaError_t make_e2m1_unpacked_tensor_map_3d_sw128(CUtensorMap* map, const void* base, int cols,
+                                                   uint64_t dim1, uint64_t dim2,
+                                                   uint64_t stride1_bytes,
+                                                   uint64_t stride2_bytes, int box1, int box2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  if (cols % 128 != 0 || stride1_bytes % 32 != 0 || stride2_bytes % 32 != 0 ||
+      reinterpret_cast<uintptr_t>(base) % 32 != 0)
+    return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {cuuint64_t(cols), cuuint64_t(dim1), cuuint64_t(dim2)};
+  const cuuint64_t strides[2] = {cuuint64_t(stride1_bytes), cuuint64_t(stride2_bytes)};
+  const cuuint32_t box[3] = {128, cuuint32_t(box1), cuuint32_t(box2)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  if (enc(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(base), dims, strides,
+          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  return cudaSuccess;
+}
+
 }  // namespace cobs
