@@ -36,6 +36,7 @@
 
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
+#include <type_traits>
 
 #include "device_common.cuh"
 #include "tcgen05.cuh"
@@ -49,10 +50,11 @@ constexpr int kStageRows = 128;   // rows of records per TMA stage / MMA tile
 constexpr int kTopkGroups = 1024; // candidate groups of the top-k bound
 constexpr int kSubStages = 2;     // record ring of the subspace kind
 // FP4 records read by kind::f8f6f4 products (d = 128, r = 8 or 16): a stage
-// holds the mu rows of up to 16 records (two 64-column slabs of 2 KB) and
-// their 128 code rows (16 KB)
-constexpr int kFdStages = 4;
-constexpr int kFdStageBytes = 20480;
+// holds the 128 code rows of a pass (16 KB); each epilogue thread's mu chunk
+// and scale bytes are fetched kFdAhead passes before their use
+constexpr int kFdStages = 5;
+constexpr int kFdStageBytes = 16384;
+constexpr int kFdAhead = 3;
 
 // Bytes of the record ring (which the top-k phase reuses) by record kind
 // (4: FP4 records read by kind::f8f6f4 products).
@@ -170,31 +172,32 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
   // ===================== phase 1: scores of this chunk =====================
   if constexpr (kFp4d) {
     // FP4 records (COBS explainer §2.3, quantisation: mu bf16 [D] | E2M1
-    // codes [r][D/2] | scale exponents [r][D/32]) read by the tensor cores as
-    // they are stored: kind::f8f6f4 products take the E2M1 codes from shared
-    // memory, so no thread converts them.  A pass is per_pass = 128 / r whole
-    // records of one ring stage, brought by two tensor maps over the records:
-    // the mu rows (both 64-column slabs, bf16) and the r code rows of every
-    // record (3-d: component, row, record), whose element type lands every 16
-    // codes in the low half of a 16-byte unit, the layout the products read.
-    // Per pass, into one of two accumulator buffers:
-    //  * q . mu: kind::f16, the mu rows against the bf16 queries (N = 16),
-    //    columns [0, 16).  It spans 128 operand rows; those past the pass's
-    //    records read the rest of the stage and are never read back;
-    //  * q . codes per group g of 32 components: kind::f8f6f4, E2M1 codes
-    //    against the queries as E4M3 (N = 16), columns [16 + 16 g, 32 + 16 g).
-    //    Query row h is scaled by 2^(6 - E_h), E_h the exponent of its
-    //    largest component, and split into hi + lo (operand rows h and
-    //    G + h); two E4M3 parts hold a bf16 value exactly (components below
-    //    2^-9 of the row's largest round at 2^-17 of it).
-    // The epilogue forms u . q_h = 2^(E_h - 6) sum_g 2^(e_g - 127)
-    // (hi_g + lo_g) in fp32 from these exact products.
-    // Roles: warps 0-3 read an accumulator back (TMEM lane = operand row =
-    // thread), fetch their row's scale bytes one pass ahead, and write the
-    // scores; warp 4 (one thread) issues the copies into a kFdStages-slot
-    // ring and the products.  mbarriers: fd_full (a stage's copies landed),
-    // mma_done (a pass's products complete: its stage may be refilled and
-    // its accumulator read), fd_acc_free (the epilogue has read it).
+    // codes [r][D/2] | scale exponents [r][D/32]) with the codes read by the
+    // tensor cores as they are stored.  A pass is per_pass = 128 / r whole
+    // records: a 3-d tensor map (component, row, record) brings their 128
+    // code rows into a ring stage, its element type landing every 16 codes
+    // in the low half of a 16-byte unit, the layout kind::f8f6f4 products
+    // read.  Per pass, one product per group g of 32 components: E2M1 codes
+    // against the queries as E4M3 (M = 128 rows, N = 16), into accumulator
+    // columns [16 g, 16 g + 16) of one of two buffers.  Query row h is
+    // scaled by 2^(6 - E_h), E_h the exponent of its largest component, and
+    // split into hi + lo (operand rows h and G + h): two E4M3 parts hold a
+    // bf16 value exactly (components below 2^-9 of the row's largest round at
+    // 2^-17 of it).  So u . q_h = 2^(E_h - 6) sum_g 2^(e_g - 127) (hi_g + lo_g)
+    // is formed in fp32 from exact products.
+    // Roles: warps 0-3 are the epilogue, thread t = TMEM lane = code row t of
+    // the pass, i.e. row t % r of record t / r, and also chunk t % r of that
+    // record's mu (D / r components), whose q . mu it forms on the CUDA cores
+    // (bf16 products are exact in fp32), so the tensor cores see only the
+    // codes.  Each thread fetches its mu chunk and its row's scale bytes
+    // kFdAhead passes ahead (asynchronous copies into a per-thread ring: one
+    // pass of HBM latency is not enough under load); a record's sums over its
+    // r lanes are formed by shuffles and its first lane writes the score, so
+    // the epilogue needs no block barrier.  Warp 4 (one thread) issues the
+    // code copies (a kFdStages-slot ring) and the products.  mbarriers:
+    // fd_full (a stage's codes landed), mma_done (a pass's products
+    // complete: its stage may be refilled and its accumulator read),
+    // fd_acc_free (the four epilogue warps have read it).
     const int r = a.rank;
     const int per_pass = kStageRows / r;
     const int rec = int(a.rec_bytes);
@@ -205,55 +208,52 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     const int rec0 = int(int64_t(bh) * a.nb_cap);   // first record (map row) of this pair
     const uint8_t* recs =
         reinterpret_cast<const uint8_t*>(a.stats) + int64_t(bh) * a.nb_cap * a.rec_bytes;
-    uint8_t* q8tile = base + kQBytes;               // [16 rows][128 B] E4M3 query parts
-    uint8_t* ring = q8tile + 2048;                  // [kFdStages][kFdStageBytes]
+    uint8_t* q8tile = base;                         // [16 rows][128 B] E4M3 query parts
+    uint8_t* ring = base + kQBytes;                 // [kFdStages][128 rows][128 B] codes
+    // per-thread mu chunks, kFdAhead + 1 passes: [slot][half][thread][16 B]
+    uint8_t* mu_ring = ring + kFdStages * kFdStageBytes;
     __shared__ __align__(8) uint64_t fd_full[kFdStages];
     __shared__ __align__(8) uint64_t fd_acc_free[2];
     __shared__ float qinv_s[8];                     // 2^(E_h - 6)
-    __shared__ __align__(16) float contrib_mu[16 * 8];
+    __shared__ uint32_t fd_scale[kFdAhead + 1][kStageRows];   // scale-byte ring
     __shared__ volatile int fd_abort;
     constexpr int kIssuer = 4 * 32;                 // warp 4, lane 0
 
     if (tid == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
       for (int s2 = 0; s2 < kFdStages; ++s2) mbar_init(&fd_full[s2], 1);
       for (int s2 = 0; s2 < 2; ++s2) {
         mbar_init(&mma_done[s2], 1);
-        mbar_init(&fd_acc_free[s2], 1);
+        mbar_init(&fd_acc_free[s2], 4);
       }
       fence_barrier_init();
       fd_abort = 0;
     }
-    if (warp == 0) tmem_alloc(&tmem_slot, 256);
+    if (warp == 0) tmem_alloc(&tmem_slot, 128);
     pdl_wait();              // queries and records may come from the launch before
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     pdl_launch_dependents();
-    const uint32_t tmem = tmem_slot;   // buffer b at column 128 b: mu . q at +0, groups at +16
+    const uint32_t tmem = tmem_slot;   // buffer b at column 64 b, group g at + 16 g
 
     int n_issued = 0;          // issuing thread: passes whose copies were issued
     int n_mma = 0;             // issuing thread: passes whose products were issued
-    auto issue = [&](int p) {  // issuing thread only: the records of pass p
+    auto issue = [&](int p) {  // issuing thread only: the code rows of pass p
       n_issued = p + 1;
       const int st = p % kFdStages;
-      const int j0 = c_lo + p * per_pass;
-      uint8_t* dst = ring + st * kFdStageBytes;
-      // the boxes are always per_pass records; records past the chunk are
-      // ignored (past the array they read as zero).  Code bytes count packed.
-      mbar_arrive_expect_tx(&fd_full[st],
-                            uint32_t(per_pass) * (uint32_t(kRegions) * 128u + uint32_t(r * D / 2)));
-      tma_load_2d(dst, &smap, 0, rec0 + j0, &fd_full[st]);
-      tma_load_2d(dst + 2048, &smap, 64, rec0 + j0, &fd_full[st]);
-      tma_load_3d(dst + 4096, &qmap, 0, 0, rec0 + j0, &fd_full[st]);
+      // the box is always per_pass records; records past the chunk are
+      // ignored (past the array they read as zero).  Its bytes count packed.
+      mbar_arrive_expect_tx(&fd_full[st], uint32_t(per_pass * r * (D / 2)));
+      tma_load_3d(ring + st * kFdStageBytes, &qmap, 0, 0, rec0 + c_lo + p * per_pass,
+                  &fd_full[st]);
     };
     if (tid == kIssuer)
       for (int p = 0; p < kFdStages && p < npass; ++p) issue(p);
 
-    // ---- the query operands: bf16 rows for mu, E4M3 hi / lo rows for codes
-    for (int e2 = tid; e2 < (kQBytes + 2048) / 16; e2 += kSelThreads + 32)
-      reinterpret_cast<uint4*>(qtile)[e2] = make_uint4(0u, 0u, 0u, 0u);   // qtile, q8tile
+    // ---- the E4M3 query operand (hi and lo rows) --------------------------
+    for (int e2 = tid; e2 < 2048 / 16; e2 += kSelThreads + 32)
+      reinterpret_cast<uint4*>(q8tile)[e2] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
     {
       // thread h * 16 + ch: components 8 ch .. 8 ch + 7 of query row h
@@ -281,8 +281,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       const float sc = __uint_as_float(uint32_t(133 - E) << 23);    // 2^(6 - E)
       if (act) {
         if (ch == 0) qinv_s[h] = __uint_as_float(uint32_t(121 + E) << 23);   // 2^(E - 6)
-        *reinterpret_cast<uint4*>(qtile + (ch >> 3) * 16 * 128 + h * 128 +
-                                  (((ch & 7) ^ h) << 4)) = w;
         uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -307,9 +305,8 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     if (warp == 4) {
       // ============================= issue ==============================
       if (lane == 0) {
-        constexpr uint32_t idesc_mu = umma_idesc_bf16(128, 16);
-        constexpr uint32_t idesc_u = umma_idesc_e2m1_e4m3(128, 16);
-        const uint32_t qb = smem_addr(qtile), q8b = smem_addr(q8tile);
+        constexpr uint32_t idesc = umma_idesc_e2m1_e4m3(128, 16);
+        const uint32_t q8b = smem_addr(q8tile);
         for (int p = 0; p < npass; ++p) {
           const int st = p % kFdStages, buf = p & 1;
           bool ok = fd_abort == 0 &&
@@ -320,17 +317,10 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           if (!ok) break;
           tc_fence_after();
           const uint32_t sb = smem_addr(ring + st * kFdStageBytes);
-          const uint32_t acc = tmem + 128u * uint32_t(buf);
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint64_t ad = umma_desc_sw128(sb + (ks >> 2) * 2048 + (ks & 3) * 32);
-            const uint64_t bd = umma_desc_sw128(qb + (ks >> 2) * 16 * 128 + (ks & 3) * 32);
-            umma_bf16(acc, ad, bd, idesc_mu, ks > 0 ? 1u : 0u);
-          }
 #pragma unroll
           for (int g = 0; g < D / 32; ++g)
-            umma_f8f6f4(acc + 16u + 16u * uint32_t(g), umma_desc_sw128(sb + 4096 + 32 * g),
-                        umma_desc_sw128(q8b + 32 * g), idesc_u, 0u);
+            umma_f8f6f4(tmem + 64u * uint32_t(buf) + 16u * uint32_t(g),
+                        umma_desc_sw128(sb + 32 * g), umma_desc_sw128(q8b + 32 * g), idesc, 0u);
           umma_commit(&mma_done[buf]);
           n_mma = p + 1;
           // refill the slot of pass p - 1, whose products were issued a pass ago
@@ -349,92 +339,145 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       }
     } else {
       // ============================ epilogue ============================
-      const int et = tid;                            // TMEM lane, operand row
+      // compiled for each chunk width, so the query chunk stays in registers
+      auto epilogue = [&](auto cpc_tag) {
+      constexpr int cpc = decltype(cpc_tag)::value;   // mu components per chunk: D / r
+      constexpr int kCols = 2 * G <= 8 ? 8 : 16;    // accumulator columns read per group
+      const int et = tid;                           // TMEM lane, code row of the pass
+      const int jr = et / r, c = et - jr * r;       // record of the pass, mu chunk
       const float inv_sqrt_d = rsqrtf(float(D));
       const float ln_n = logf(float(kBlock));
       float qinv[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) qinv[h] = qinv_s[h] * inv_sqrt_d;
+      for (int h = 0; h < G; ++h) qinv[h] = qinv_s[h];
+      // this thread's query components c cpc .. c cpc + cpc - 1 of every head
+      // (bf16 pairs)
+      uint32_t qc[G][cpc / 2];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const uint16_t* qh = a.q + (int64_t(b) * a.hq + kvh * G + h) * D + c * cpc;
+#pragma unroll
+        for (int i = 0; i < cpc / 8; ++i) {
+          const uint4 w = *reinterpret_cast<const uint4*>(qh + 8 * i);
+          qc[h][4 * i] = w.x; qc[h][4 * i + 1] = w.y; qc[h][4 * i + 2] = w.z; qc[h][4 * i + 3] = w.w;
+        }
+      }
       const int sc_off = 2 * D + r * (D / 2);        // scale bytes of row 0 of a record
-      auto scale_word = [&](int p) -> uint32_t {     // this row's 4 group exponents
-        const int j0 = c_lo + p * per_pass;
-        const int nb = min(per_pass, c_hi - j0);
-        if (et >= nb * r) return 0u;
-        const int jj = et / r, k = et - jj * r;
-        return __ldg(reinterpret_cast<const uint32_t*>(recs + int64_t(j0 + jj) * rec + sc_off +
-                                                       k * (D / 32)));
+      // this thread's mu chunk and scale bytes of pass p into ring slot
+      // p % (kFdAhead + 1), one committed group per pass (empty past the
+      // chunk or the pass's records)
+      auto fetch = [&](int p) {
+        if (p < npass) {
+          const int j0 = c_lo + p * per_pass;
+          const int nb = min(per_pass, c_hi - j0);
+          if (jr < nb) {
+            const int slot = p % (kFdAhead + 1);
+            const uint8_t* rp = recs + int64_t(j0 + jr) * rec;
+            uint8_t* ms = mu_ring + slot * (2 * kStageRows * 16) + et * 16;
+#pragma unroll
+            for (int i = 0; i < cpc / 8; ++i)
+              cp_async16(ms + i * (kStageRows * 16), rp + c * cpc * 2 + 16 * i);
+            cp_async4(&fd_scale[slot][et], rp + sc_off + c * (D / 32));
+          }
+        }
+        cp_async_commit();
       };
-      uint32_t sc_next = npass > 0 ? scale_word(0) : 0u;
+      for (int p = 0; p < kFdAhead; ++p) fetch(p);
       for (int p = 0; p < npass; ++p) {
         const int buf = p & 1;
-        const uint32_t scw = sc_next;
-        if (p + 1 < npass) sc_next = scale_word(p + 1);
-        bool fail = fd_abort != 0;
-        if (!fail && et == 0)
-          fail = !wait_or_abort(&mma_done[buf], (p >> 1) & 1, a.status, &fd_abort);
-        if (named_bar_or(2, 128, fail)) break;
-        if (et != 0) (void)mbar_try_wait(&mma_done[buf], (p >> 1) & 1);
+        fetch(p + kFdAhead);
+        // lane 0 of each warp waits (bounded) for the pass's products
+        bool ok = true;
+        if (lane == 0)
+          ok = fd_abort == 0 && wait_or_abort(&mma_done[buf], (p >> 1) & 1, a.status, &fd_abort);
+        if (!__shfl_sync(0xffffffffu, int(ok), 0)) break;
+        if (lane != 0) (void)mbar_try_wait(&mma_done[buf], (p >> 1) & 1);
         tc_fence_after();
         const int j0 = c_lo + p * per_pass;
         const int nb = min(per_pass, c_hi - j0);
-        const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 128u * uint32_t(buf);
-        uint32_t vm[8];
-        float vu0[32], vu1[32];
-        tmem_ld8_nowait(lane_base, vm);
-        tmem_ld32(lane_base + 16u, vu0);             // groups 0, 1
-        tmem_ld32(lane_base + 48u, vu1);             // groups 2, 3 (waits for all three)
-        tc_fence_before();
-        if (et < nb * r) {
-          float s4[4];
+        const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 64u * uint32_t(buf);
+        uint32_t v[4][kCols];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) s4[g] = __uint_as_float(((scw >> (8 * g)) & 0xFFu) << 23);
+        for (int g = 0; g < 4; ++g) {
+          if constexpr (kCols == 8)
+            tmem_ld8_nowait(lane_base + 16u * uint32_t(g), v[g]);
+          else
+            tmem_ld16_nowait(lane_base + 16u * uint32_t(g), v[g]);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        // the accumulator is read: once all four warps are here its next
+        // products may start
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&fd_acc_free[buf]);
+        cp_async_wait_group<kFdAhead>();            // this pass's mu chunk and scales landed
+        const bool live = jr < nb;
+        const int slot = p % (kFdAhead + 1);
+        const uint32_t scw = fd_scale[slot][et];
+        uint32_t mw[cpc / 2];
+#pragma unroll
+        for (int i = 0; i < cpc / 8; ++i) {
+          const uint4 m4 = *reinterpret_cast<const uint4*>(mu_ring + slot * (2 * kStageRows * 16) +
+                                                           i * (kStageRows * 16) + et * 16);
+          mw[4 * i] = m4.x; mw[4 * i + 1] = m4.y; mw[4 * i + 2] = m4.z; mw[4 * i + 3] = m4.w;
+        }
+        float s4[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) s4[g] = __uint_as_float(((scw >> (8 * g)) & 0xFFu) << 23);
+        float sq[G], mq[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float x = 0.f;
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            x = fmaf(s4[g], __uint_as_float(v[g][h]) + __uint_as_float(v[g][G + h]), x);
+          x *= qinv[h] * inv_sqrt_d;
+          sq[h] = live ? 0.5f * x * x : 0.f;
+          float y = 0.f;
+#pragma unroll
+          for (int i = 0; i < cpc / 2; ++i) {
+            const float2 mf = bf16x2_to_float2(mw[i]);
+            const float2 qf = bf16x2_to_float2(qc[h][i]);
+            y = fmaf(mf.x, qf.x, fmaf(mf.y, qf.y, y));
+          }
+          mq[h] = live ? y : 0.f;
+        }
+        // a record's r rows and r mu chunks are r consecutive lanes
+        for (int o = 1; o < r; o <<= 1) {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            float x = s4[0] * (vu0[h] + vu0[G + h]);
-            x = fmaf(s4[1], vu0[16 + h] + vu0[16 + G + h], x);
-            x = fmaf(s4[2], vu1[h] + vu1[G + h], x);
-            x = fmaf(s4[3], vu1[16 + h] + vu1[16 + G + h], x);
-            x *= qinv[h];
-            contrib[et * 8 + h] = 0.5f * x * x;
+            sq[h] += __shfl_xor_sync(0xffffffffu, sq[h], o);
+            mq[h] += __shfl_xor_sync(0xffffffffu, mq[h], o);
           }
         }
-        if (et < nb) {
+        if (live && c == 0) {
+          // s_h = ln n + q_h . mu / sqrt d + 1/2 sum_k (u_k . q_h)^2 / d; S =
+          // the log-sum-exp over the heads
+          float sh[G], mx = -FLT_MAX;
 #pragma unroll
-          for (int h = 0; h < G; ++h) contrib_mu[et * 8 + h] = __uint_as_float(vm[h]) * inv_sqrt_d;
-        }
-        named_bar(2, 128);
-        // the accumulator has been read: its next products may start
-        if (et == 0) mbar_arrive(&fd_acc_free[buf]);
-        // per block and head: mu row + its r code rows, then LSE over the heads
-        for (int t0 = 0; t0 < per_pass * G; t0 += 128) {
-          const int t = t0 + et;
-          const int jj = t / G, h = t % G;
-          const bool valid = jj < nb;
-          float sacc = 0.f;
-          if (valid) {
-            sacc = contrib_mu[jj * 8 + h];
-            for (int i = 0; i < r; ++i) sacc += contrib[(jj * r + i) * 8 + h];
+          for (int h = 0; h < G; ++h) {
+            sh[h] = ln_n + mq[h] * inv_sqrt_d + sq[h];
+            mx = fmaxf(mx, sh[h]);
           }
-          const float sh = sacc + ln_n;
-          float mx = sh;
+          float e = 0.f;
 #pragma unroll
-          for (int m = G / 2; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m, G));
-          float e = __expf(sh - mx);
-#pragma unroll
-          for (int m = G / 2; m >= 1; m >>= 1) e += __shfl_xor_sync(0xffffffffu, e, m, G);
-          if (valid && h == 0) {
-            const float S = mx + __logf(e);
-            scores[j0 + jj] = S;
-            if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jj] = S;
-          }
+          for (int h = 0; h < G; ++h) e += __expf(sh[h] - mx);
+          const float S = mx + __logf(e);
+          scores[j0 + jr] = S;
+          if (a.scores_opt) a.scores_opt[int64_t(bh) * a.nb_cap + j0 + jr] = S;
         }
-        named_bar(2, 128);   // contrib is rewritten by the next pass
       }
+      cp_async_wait_all();   // no copy of this thread outlives the loop
+      };
+      if (r == 8)
+        epilogue(std::integral_constant<int, D / 8>{});
+      else
+        epilogue(std::integral_constant<int, D / 16>{});
     }
     __threadfence();         // this thread's scores, before the pair's ticket
     tc_fence_before();
     __syncthreads();         // every score of the chunk is written
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 128);
     if (tid >= kSelThreads) return;   // the top-k below runs on warps 0-3 (named barrier 3)
   } else if constexpr (kFp4) {
     // FP4 records (COBS explainer §2.3, quantisation): mu bf16 [D] | E2M1
@@ -1382,7 +1425,8 @@ constexpr size_t dyn_smem_bytes() {
          (kFmt == 1 ? size_t(2) * (D / 64) * 128 * 128 + size_t(kSelFp4RawStages) *
                                                              fp4_raw_stage_bytes(D)
                     : size_t(ring_bytes(D, kFmt))) +
-         (kFmt == 3 ? size_t(2) * 32 * 128 : 0) + (kFmt == 4 ? size_t(2048) : 0);
+         (kFmt == 3 ? size_t(2) * 32 * 128 : 0) +
+         (kFmt == 4 ? size_t(kFdAhead + 1) * 2 * kStageRows * 16 : 0);
 }
 template <int kFmt>
 constexpr int sel_threads() {
@@ -1402,12 +1446,11 @@ cudaError_t launch_t(const SelectArgs& a, cudaStream_t s) {
   if (kFp4) {
     map = qmap;   // FP4 records arrive by plain bulk copies; the map is unused
   } else if (kFmt == 4) {
-    // mu rows: the first D columns of every record; code rows: (component,
-    // row, record) starting 2 D bytes into the records
+    // code rows: (component, row, record) starting 2 D bytes into the
+    // records (the mu rows and scale bytes are read by the epilogue threads)
     const uint64_t n_rec = uint64_t(a.batch) * a.hkv * a.nb_cap;
     const int per_pass = kStageRows / a.rank;
-    e = make_bf16_tensor_map_rows_sw128(&map, a.stats, D, n_rec, uint64_t(a.rec_bytes), per_pass);
-    if (e != cudaSuccess) return e;
+    map = qmap;   // unused
     e = make_e2m1_unpacked_tensor_map_3d_sw128(&qmap,
                                                reinterpret_cast<const uint8_t*>(a.stats) + 2 * D,
                                                D, uint64_t(a.rank), n_rec, uint64_t(D / 2),
