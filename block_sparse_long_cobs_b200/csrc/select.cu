@@ -194,10 +194,11 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     // pass of HBM latency is not enough under load); a record's sums over its
     // r lanes are formed by shuffles and its first lane writes the score, so
     // the epilogue needs no block barrier.  Warp 4 (one thread) issues the
-    // code copies (a kFdStages-slot ring) and the products.  mbarriers:
-    // fd_full (a stage's codes landed), mma_done (a pass's products
-    // complete: its stage may be refilled and its accumulator read),
-    // fd_acc_free (the four epilogue warps have read it).
+    // code copies (a kFdStages-slot ring) and the products; it never waits
+    // for products itself.  mbarriers: fd_full (a stage's codes landed),
+    // mma_done (a pass's products complete: its accumulator may be read),
+    // fd_acc_free (the four epilogue warps have read it: the accumulator may
+    // be rewritten and the pass's stage refilled).
     const int r = a.rank;
     const int per_pass = kStageRows / r;
     const int rec = int(a.rec_bytes);
@@ -216,6 +217,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     __shared__ __align__(8) uint64_t fd_acc_free[2];
     __shared__ float qinv_s[8];                     // 2^(E_h - 6)
     __shared__ uint32_t fd_scale[kFdAhead + 1][kStageRows];   // scale-byte ring
+    __shared__ __align__(16) uint32_t fd_q[8 * 64];            // the queries, bf16 pairs
     __shared__ volatile int fd_abort;
     constexpr int kIssuer = 4 * 32;                 // warp 4, lane 0
 
@@ -281,6 +283,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       const float sc = __uint_as_float(uint32_t(133 - E) << 23);    // 2^(6 - E)
       if (act) {
         if (ch == 0) qinv_s[h] = __uint_as_float(uint32_t(121 + E) << 23);   // 2^(E - 6)
+        *reinterpret_cast<uint4*>(&fd_q[h * (D / 2) + ch * 4]) = w;
         uint32_t hw[2] = {0u, 0u}, lw[2] = {0u, 0u};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -311,9 +314,12 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           const int st = p % kFdStages, buf = p & 1;
           bool ok = fd_abort == 0 &&
                     wait_or_abort(&fd_full[st], (p / kFdStages) & 1, a.status, &fd_abort);
-          // the epilogue has read this accumulator's pass p - 2
-          if (ok && p >= 2)
+          // the epilogue has read this accumulator's pass p - 2, so that
+          // pass's products are complete and its ring slot is free: refill it
+          if (ok && p >= 2) {
             ok = wait_or_abort(&fd_acc_free[buf], ((p - 2) >> 1) & 1, a.status, &fd_abort);
+            if (ok && p - 2 + kFdStages < npass) issue(p - 2 + kFdStages);
+          }
           if (!ok) break;
           tc_fence_after();
           const uint32_t sb = smem_addr(ring + st * kFdStageBytes);
@@ -323,12 +329,6 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
                         umma_desc_sw128(sb + 32 * g), umma_desc_sw128(q8b + 32 * g), idesc, 0u);
           umma_commit(&mma_done[buf]);
           n_mma = p + 1;
-          // refill the slot of pass p - 1, whose products were issued a pass ago
-          if (p >= 1 && p - 1 + kFdStages < npass) {
-            if (!wait_or_abort(&mma_done[(p - 1) & 1], ((p - 1) >> 1) & 1, a.status, &fd_abort))
-              break;
-            issue(p - 1 + kFdStages);
-          }
         }
         // let the copies and the products still in flight land before TMEM is
         // freed and the CTA leaves (each wait bounded)
@@ -347,38 +347,35 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
       const int jr = et / r, c = et - jr * r;       // record of the pass, mu chunk
       const float inv_sqrt_d = rsqrtf(float(D));
       const float ln_n = logf(float(kBlock));
-      float qinv[G];
+      float qinv[G];                                 // 2^(E_h - 6) / sqrt d
 #pragma unroll
-      for (int h = 0; h < G; ++h) qinv[h] = qinv_s[h];
+      for (int h = 0; h < G; ++h) qinv[h] = qinv_s[h] * inv_sqrt_d;
       // this thread's query components c cpc .. c cpc + cpc - 1 of every head
-      // (bf16 pairs)
-      uint32_t qc[G][cpc / 2];
+      // (bf16 pairs), in registers unless that takes more than 32 of them
+      constexpr bool kQShared = G * (cpc / 2) > 32;
+      constexpr int kQh = kQShared ? 1 : G, kQi = kQShared ? 1 : cpc / 2;
+      uint32_t qc[kQh][kQi];
+      if constexpr (!kQShared) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const uint16_t* qh = a.q + (int64_t(b) * a.hq + kvh * G + h) * D + c * cpc;
+        for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int i = 0; i < cpc / 8; ++i) {
-          const uint4 w = *reinterpret_cast<const uint4*>(qh + 8 * i);
-          qc[h][4 * i] = w.x; qc[h][4 * i + 1] = w.y; qc[h][4 * i + 2] = w.z; qc[h][4 * i + 3] = w.w;
-        }
+          for (int i = 0; i < cpc / 2; ++i) qc[h][i] = fd_q[h * (D / 2) + c * (cpc / 2) + i];
       }
-      const int sc_off = 2 * D + r * (D / 2);        // scale bytes of row 0 of a record
       // this thread's mu chunk and scale bytes of pass p into ring slot
       // p % (kFdAhead + 1), one committed group per pass (empty past the
       // chunk or the pass's records)
+      static_assert(((kFdAhead + 1) & kFdAhead) == 0, "ring slots: a power of two");
+      const uint8_t* my_mu = recs + int64_t(c_lo + jr) * rec + c * cpc * 2;
+      const uint8_t* my_sc = recs + int64_t(c_lo + jr) * rec + 2 * D + r * (D / 2) + c * (D / 32);
+      const int64_t pass_bytes = int64_t(per_pass) * rec;
       auto fetch = [&](int p) {
-        if (p < npass) {
-          const int j0 = c_lo + p * per_pass;
-          const int nb = min(per_pass, c_hi - j0);
-          if (jr < nb) {
-            const int slot = p % (kFdAhead + 1);
-            const uint8_t* rp = recs + int64_t(j0 + jr) * rec;
-            uint8_t* ms = mu_ring + slot * (2 * kStageRows * 16) + et * 16;
+        if (p < npass && c_lo + p * per_pass + jr < c_hi) {
+          const int slot = p & kFdAhead;
+          uint8_t* ms = mu_ring + slot * (2 * kStageRows * 16) + et * 16;
 #pragma unroll
-            for (int i = 0; i < cpc / 8; ++i)
-              cp_async16(ms + i * (kStageRows * 16), rp + c * cpc * 2 + 16 * i);
-            cp_async4(&fd_scale[slot][et], rp + sc_off + c * (D / 32));
-          }
+          for (int i = 0; i < cpc / 8; ++i)
+            cp_async16(ms + i * (kStageRows * 16), my_mu + p * pass_bytes + 16 * i);
+          cp_async4(&fd_scale[slot][et], my_sc + p * pass_bytes);
         }
         cp_async_commit();
       };
@@ -396,15 +393,28 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         const int j0 = c_lo + p * per_pass;
         const int nb = min(per_pass, c_hi - j0);
         const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16) + 64u * uint32_t(buf);
-        uint32_t v[4][kCols];
+        // u[g][h] = hi + lo product of group g and head h
+        float u[4][G];
+        if constexpr (kCols == 8) {
+          uint32_t v[4][8];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if constexpr (kCols == 8)
-            tmem_ld8_nowait(lane_base + 16u * uint32_t(g), v[g]);
-          else
-            tmem_ld16_nowait(lane_base + 16u * uint32_t(g), v[g]);
+          for (int g = 0; g < 4; ++g) tmem_ld8_nowait(lane_base + 16u * uint32_t(g), v[g]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int h = 0; h < G; ++h) u[g][h] = __uint_as_float(v[g][h]) + __uint_as_float(v[g][G + h]);
+        } else {
+          // G = 8: one group at a time keeps the registers in bounds
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint32_t v[16];
+            tmem_ld16_nowait(lane_base + 16u * uint32_t(g), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < G; ++h) u[g][h] = __uint_as_float(v[h]) + __uint_as_float(v[G + h]);
+          }
         }
-        tmem_wait_ld();
         tc_fence_before();
         // the accumulator is read: once all four warps are here its next
         // products may start
@@ -412,7 +422,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         if (lane == 0) mbar_arrive(&fd_acc_free[buf]);
         cp_async_wait_group<kFdAhead>();            // this pass's mu chunk and scales landed
         const bool live = jr < nb;
-        const int slot = p % (kFdAhead + 1);
+        const int slot = p & kFdAhead;
         const uint32_t scw = fd_scale[slot][et];
         uint32_t mw[cpc / 2];
 #pragma unroll
@@ -424,31 +434,29 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
         float s4[4];
 #pragma unroll
         for (int g = 0; g < 4; ++g) s4[g] = __uint_as_float(((scw >> (8 * g)) & 0xFFu) << 23);
-        float sq[G], mq[G];
+        // this lane's share of s_h - ln n: its chunk of q_h . mu / sqrt d
+        // plus half its row's (u . q_h / sqrt d)^2
+        float t[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float x = 0.f;
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            x = fmaf(s4[g], __uint_as_float(v[g][h]) + __uint_as_float(v[g][G + h]), x);
-          x *= qinv[h] * inv_sqrt_d;
-          sq[h] = live ? 0.5f * x * x : 0.f;
+          for (int g = 0; g < 4; ++g) x = fmaf(s4[g], u[g][h], x);
+          x *= qinv[h];
           float y = 0.f;
 #pragma unroll
           for (int i = 0; i < cpc / 2; ++i) {
             const float2 mf = bf16x2_to_float2(mw[i]);
-            const float2 qf = bf16x2_to_float2(qc[h][i]);
+            const float2 qf = bf16x2_to_float2(kQShared ? fd_q[h * (D / 2) + c * (cpc / 2) + i]
+                                                        : qc[kQShared ? 0 : h][kQShared ? 0 : i]);
             y = fmaf(mf.x, qf.x, fmaf(mf.y, qf.y, y));
           }
-          mq[h] = live ? y : 0.f;
+          t[h] = live ? fmaf(y, inv_sqrt_d, 0.5f * x * x) : 0.f;
         }
         // a record's r rows and r mu chunks are r consecutive lanes
         for (int o = 1; o < r; o <<= 1) {
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            sq[h] += __shfl_xor_sync(0xffffffffu, sq[h], o);
-            mq[h] += __shfl_xor_sync(0xffffffffu, mq[h], o);
-          }
+          for (int h = 0; h < G; ++h) t[h] += __shfl_xor_sync(0xffffffffu, t[h], o);
         }
         if (live && c == 0) {
           // s_h = ln n + q_h . mu / sqrt d + 1/2 sum_k (u_k . q_h)^2 / d; S =
@@ -456,7 +464,7 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
           float sh[G], mx = -FLT_MAX;
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            sh[h] = ln_n + mq[h] * inv_sqrt_d + sq[h];
+            sh[h] = ln_n + t[h];
             mx = fmaxf(mx, sh[h]);
           }
           float e = 0.f;
