@@ -301,3 +301,38 @@ def test_select_fp4_at_full_size(name, pairs):
         np.testing.assert_allclose(sc_h[b, h, c0:c1], s[c0:c1], rtol=0,
                                    atol=TIE_RTOL * max(1, np.max(np.abs(s))))
     assert cb.cobs_read_device_status(ws, ws_bytes) == 0
+
+
+def test_select_fp4_misaligned_stats_uses_widening_kernel():
+    """FP4 records 16-byte but not 32-byte aligned: the tensor-core kernel's
+    code map needs 32-byte alignment, so the selection falls back to the
+    kernel that widens the codes in shared memory, and still equals the
+    oracle's selection from the records (ties reported)."""
+    w = CASES["needles_b2_r8"]
+    p = Fp4Problem(w, poison="nan")
+    orc = {}
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            parts = p.oracle_records4(b, h)
+            p.upload_records4(b, h, parts)
+            orc[(b, h)] = oracle_selection4(p, b, h, parts)
+    # the same records, starting 16 bytes past a 32-byte boundary
+    flat = torch.zeros(p.stats4.numel() + 64, dtype=torch.uint8, device="cuda")
+    off = (16 - flat.data_ptr() % 32) % 32
+    shifted = flat[off:off + p.stats4.numel()].view(p.stats4.shape)
+    shifted.copy_(p.stats4)
+    assert shifted.data_ptr() % 32 == 16
+    cb.cobs_select_blocks(p.dims4, p.q, shifted, w.seq_len, w.top_k, w.sink_blocks,
+                          w.local_tokens, p.idx, p.idx.shape[-1], p.n_sel, p.scores, p.ws,
+                          p.ws_bytes)
+    idx, n = p.idx.cpu().numpy(), p.n_sel.cpu().numpy()
+    scores = p.scores.cpu().numpy()
+    _, c0, c1 = O.block_partition(w.seq_len, w.block, w.sink_blocks, w.local_tokens)
+    for (b, h), (sel, s) in orc.items():
+        got = idx[b, h, :n[b, h]]
+        assert np.all(np.diff(got) > 0)
+        assert n[b, h] == len(sel)
+        assert selection_mismatch(got, sel, s, w) == [], (b, h)
+        np.testing.assert_allclose(scores[b, h, c0:c1], s[c0:c1],
+                                   rtol=0, atol=TIE_RTOL * max(1, np.max(np.abs(s))))
+    assert p.device_status() == 0
