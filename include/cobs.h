@@ -124,12 +124,21 @@ typedef struct cobs_dims {
  *   then zero padding to a multiple of 16 bytes.
  * A group's exponent is the smallest e with max |u| <= 6 * 2^e (clamped at
  * -126), so no component saturates; components round to the nearest E2M1
- * value, ties to the even code.  FP4 records need r >= 1.  Selection over
- * FP4 records multiplies the codes with the queries in fp16: queries must lie
- * inside the fp16 range (|q| < 65504), and components below 2^-14 are
- * rounded to fp16's subnormal grid (an error of at most 2^-25 each); a scale
- * group whose exponent lies more than 23 below the largest of its column
- * (components under 2^-23 of the column's largest) counts as zero there. */
+ * value, ties to the even code.  FP4 records need r >= 1.
+ * Selection over FP4 records takes one of two kernels:
+ *   - d = 128, r = 8 or 16, and the stats array 32-byte aligned (so are all
+ *     records, whose size is then a multiple of 32 bytes): the tensor cores
+ *     read the codes as stored.  Each query row is scaled by a power of two
+ *     and split into two E4M3 parts, which hold a bf16 value exactly; only
+ *     components below 2^-9 of the row's largest are rounded, by at most
+ *     2^-16 of it.  This is the faster kernel: allocate FP4 stats 32-byte
+ *     aligned.
+ *   - otherwise the codes are widened to fp16 in shared memory: queries must
+ *     lie inside the fp16 range (|q| < 65504), and components below 2^-14
+ *     are rounded to fp16's subnormal grid (an error of at most 2^-25 each);
+ *     a scale group whose exponent lies more than 23 below the largest of its
+ *     column (components under 2^-23 of the column's largest) counts as zero
+ *     there. */
 
 /* Min/max box record (a comparison selector, not COBS: the explainer's
  * plain-language summary lists estimating a block's spread from the minimum
