@@ -182,8 +182,8 @@ select_blocks_kernel(const __grid_constant__ CUtensorMap smap,
     // columns [16 g, 16 g + 16) of one of two buffers.  Query row h is
     // scaled by 2^(6 - E_h), E_h the exponent of its largest component, and
     // split into hi + lo (operand rows h and G + h): two E4M3 parts hold a
-    // bf16 value exactly (components below 2^-9 of the row's largest round at
-    // 2^-17 of it).  So u . q_h = 2^(E_h - 6) sum_g 2^(e_g - 127) (hi_g + lo_g)
+    // bf16 value exactly (components below 2^-8 of the row's largest round by
+    // <= 2^-16 of it).  So u . q_h = 2^(E_h - 6) sum_g 2^(e_g - 127) (hi_g + lo_g)
     // is formed in fp32 from exact products.
     // Roles: warps 0-3 are the epilogue, thread t = TMEM lane = code row t of
     // the pass, i.e. row t % r of record t / r, and also chunk t % r of that

@@ -130,7 +130,7 @@ typedef struct cobs_dims {
  *     records, whose size is then a multiple of 32 bytes): the tensor cores
  *     read the codes as stored.  Each query row is scaled by a power of two
  *     and split into two E4M3 parts, which hold a bf16 value exactly; only
- *     components below 2^-9 of the row's largest are rounded, by at most
+ *     components below 2^-8 of the row's largest are rounded, by at most
  *     2^-16 of it.  This is the faster kernel: allocate FP4 stats 32-byte
  *     aligned.
  *   - otherwise the codes are widened to fp16 in shared memory: queries must
